@@ -1,0 +1,460 @@
+#!/usr/bin/env python
+"""Throughput of the MISA token indexer on B200 (one JSON line on rank 0).
+
+Workload (N = 1): DeepSeek-V3.2-shaped indexer decode -- 32 sequences x 1
+query, L = 32768 bf16 keys each, d = 128, H = 64 indexer heads of which h = 8
+are routed per query from B = 128 mean-pooled key blocks, top-k = 2048.  One
+step is the whole per-query path: router, routed token scoring, top-k (the
+block statistics are per-cache state maintained on KV append; they are timed
+separately).  The metric is indexed q.k pairs per second = sum over queries of
+the keys each query's top-k decision covers, divided by the step time.
+
+Multi-GPU (torchrun): every rank runs its own batch of the same shape (weak
+scaling, no collective on the data path); the step time is the max over ranks.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--quick]
+
+`--impl reference` times the fp64 CPU oracle (this repository's reference
+implementation of the same path) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import make_workload  # noqa: E402
+
+WORKLOAD = "dsv32_decode_L32768"
+METRIC = "indexed q.k pairs/s (top-k=2048, L=32K, MISA h=8 of H=64)"
+UNIT = "pairs/s"
+L2_FLUSH_BYTES = 256 << 20
+SCORE_SOURCES = ["sparse_attention_token_misa_b200/csrc/score_tc.cu",
+                 "sparse_attention_token_misa_b200/csrc/misa_device.cuh"]
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def _source_hash(paths) -> str:
+    h = hashlib.sha256()
+    for rel in paths:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic_for(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel)
+    if not e or e.get("workload") != workload or e.get("source_sha256_16") != _source_hash(e.get("sources", [])):
+        return None
+    return e.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        if not self.lines:
+            return None
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            try:
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        under_load = [s for s in sm if s > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(under_load), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def _time_steps(step, steps, flush, stream, marks=None):
+    """Per-step CUDA-event timing with an untimed L2 flush before every step.
+    marks: optional list of names; step(ev) records intermediate events."""
+    tot = 0.0
+    marks = list(marks or [])
+    parts = {m: 0.0 for m in marks}
+    n_ev = max(2, len(marks) + 1)  # start, one event between consecutive parts, end
+    for _ in range(steps):
+        flush()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+        evs[0].record(stream)
+        step(evs[1:-1])
+        evs[-1].record(stream)
+        torch.cuda.synchronize()
+        tot += evs[0].elapsed_time(evs[-1])
+        for i, m in enumerate(marks):
+            parts[m] += evs[i].elapsed_time(evs[i + 1])
+    return tot, parts
+
+
+def run_cuda(args):
+    import sparse_attention_token_misa_b200 as misa
+
+    ws_n, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dist = None
+    if ws_n > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+
+    wl = make_workload(WORKLOAD)
+    if rank:
+        # every rank gets its own batch of the same shape (different seed)
+        from workloads import make_decode
+        wl = make_decode(WORKLOAD, 2 + 1000 * rank, T=32, L=32768, H=64, h=8, B=128, k=2048, n_planted=16)
+    q, w, keys = wl.q.to(dev), wl.w.to(dev), wl.keys.to(dev)
+    seq_of, plen = wl.seq_of.to(dev), wl.prefix_len.to(dev)
+    T, H, h, L, B, k = wl.T, wl.H, wl.h, wl.L, wl.B, wl.k
+    pairs = int(wl.prefix_len.sum())
+
+    means = misa.block_stats(keys, B)
+    ix = misa.MisaIndexer(T, H, h, L, B, k, q_block=1, device=dev)
+    dense = misa.DenseIndexer(T, H, L, k, device=dev)
+    flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def flush():
+        flush_buf.fill_(1.0)
+
+    def misa_step(evs):
+        ix.route(q, w, means, seq_of, plen)
+        if evs:
+            evs[0].record(stream)
+        ix.score(q, w, keys, seq_of, plen)
+        if evs:
+            evs[1].record(stream)
+        ix.select(plen)
+
+    def dense_step(evs):
+        dense.run(q, w, keys, seq_of, plen)
+
+    def stats_step(evs):
+        misa.block_stats(keys, B, out=means)
+
+    for _ in range(args.warmup):
+        misa_step([])
+        dense_step([])
+    torch.cuda.synchronize()
+    misa.error_reset(ix.ws)
+    misa.error_reset(ix.ws_route)
+
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t0 = time.perf_counter()
+        tot_ms, parts = _time_steps(misa_step, args.steps, flush, stream, marks=["route", "score", "topk"])
+        wall = time.perf_counter() - t0
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    dev_err = misa.error_query(ix.ws) | misa.error_query(ix.ws_route)
+    if dev_err:
+        raise RuntimeError(f"device error word {dev_err:#x}")
+    ms_step = tot_ms / args.steps
+    if dist:
+        t = torch.tensor([ms_step], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step = float(t.item())
+
+    # dense 64-head indexer and block statistics on the same batch (same protocol)
+    dense_ms, _ = _time_steps(dense_step, args.steps, flush, stream)
+    stats_ms, _ = _time_steps(stats_step, args.steps, flush, stream)
+    dense_ms /= args.steps
+    stats_ms /= args.steps
+
+    # e2e through the public API: pinned host inputs -> device, indexer, idx -> host
+    q_h = wl.q.pin_memory()
+    w_h = wl.w.pin_memory()
+    so_h = wl.seq_of.pin_memory()
+    pl_h = wl.prefix_len.pin_memory()
+    idx_h = torch.empty((T, k), dtype=torch.int32).pin_memory()
+    q_d, w_d, so_d, pl_d = torch.empty_like(q), torch.empty_like(w), torch.empty_like(seq_of), torch.empty_like(plen)
+
+    def e2e_step(evs):
+        q_d.copy_(q_h, non_blocking=True)
+        w_d.copy_(w_h, non_blocking=True)
+        so_d.copy_(so_h, non_blocking=True)
+        pl_d.copy_(pl_h, non_blocking=True)
+        out = ix.run(q_d, w_d, keys, means, so_d, pl_d)
+        idx_h.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step([])
+    torch.cuda.synchronize()
+    e2e_ms, _ = _time_steps(e2e_step, args.steps, flush, stream)
+    e2e_ms /= args.steps
+    if dist:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = q_h.numel() * 2 + w_h.numel() * 4 + so_h.numel() * 4 + pl_h.numel() * 4
+    d2h = idx_h.numel() * 4
+
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    hbm_gbs, tc_tflops, peak_kind = _peaks()
+    score_ms = parts["score"] / args.steps
+    # algorithmic bytes of one scoring launch: K once, the routed query rows and
+    # weights, the fp32 score rows written
+    score_bytes = T * L * 128 * 2 + T * h * (128 * 2 + 4 + 4) + T * L * 4
+    achieved = score_bytes / (score_ms * 1e-3) / 1e9
+    traffic = _traffic_for("score_kernel", WORKLOAD)
+    value = pairs * ws_n / (ms_step * 1e-3)
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": UNIT,
+        "n_gpus": ws_n,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; shapes of the DeepSeek-V3.2 indexer decode)",
+        "config": {"workload": WORKLOAD, "queries": T, "L": L, "H": H, "h": h, "B": B, "k": k, "d": 128,
+                   "parallelism": f"dp{ws_n} (independent batches)",
+                   "l2": "flushed before every timed step (256 MiB write, untimed); K is 268 MB > L2"},
+        "queries_per_s": T * ws_n / (ms_step * 1e-3),
+        "gpu_launches": 4 * args.steps,
+        "roofline": {"bound": "hbm", "kernel": "score_kernel (misa_index_score)", "achieved": achieved,
+                     "peak": hbm_gbs, "peak_kind": f"{peak_kind} hbm copy GB/s", "unit": "GB/s",
+                     "frac": achieved / hbm_gbs, "traffic": traffic,
+                     "algorithmic_bytes_per_launch": score_bytes, "launch_ms": score_ms},
+        "e2e": {"value": pairs * ws_n / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "detail": {"route_ms": parts["route"] / args.steps, "score_ms": score_ms, "topk_ms": parts["topk"] / args.steps,
+                   "misa8_ms": ms_step, "dense64_ms": dense_ms, "dense64_over_misa8": dense_ms / ms_step,
+                   "block_stats_ms": stats_ms,
+                   "block_stats_GBps": (T * L * 128 * 2 + T * (L // B) * 128 * 4) / (stats_ms * 1e-3) / 1e9,
+                   "wall_s_timed_region": wall},
+    }
+    summ = clk.summary()
+    if summ:
+        line["clocks"] = summ
+    if not args.quick and ws_n == 1:
+        line["other_workloads"] = other_workloads(misa, dev, stream, flush, max(3, min(args.steps, 10)))
+        del flush_buf
+    if ws_n == 1:
+        line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_budget)
+    print(json.dumps(line), flush=True)
+
+
+def other_workloads(misa, dev, stream, flush, steps):
+    """The other four workloads through their indexers (same timing protocol)."""
+    out = {}
+
+    def timed(fn):
+        for _ in range(3):
+            fn([])
+        torch.cuda.synchronize()
+        ms, _ = _time_steps(fn, steps, flush, stream)
+        return ms / steps
+
+    wl = make_workload("prefill_L131072")
+    q, w, keys, so, pl = (x.to(dev) for x in (wl.q, wl.w, wl.keys, wl.seq_of, wl.prefix_len))
+    means = misa.block_stats(keys, wl.B)
+    ix = misa.MisaIndexer(wl.T, wl.H, wl.h, wl.L, wl.B, wl.k, wl.q_block, device=dev)
+    pairs = int(wl.prefix_len.sum())
+    parts = {}
+
+    def pf(evs):
+        ix.route(q, w, means, so, pl)
+        if evs:
+            evs[0].record(stream)
+        ix.score(q, w, keys, so, pl)
+        if evs:
+            evs[1].record(stream)
+        ix.select(pl)
+
+    for _ in range(2):
+        pf([])
+    torch.cuda.synchronize()
+    ms, parts = _time_steps(pf, steps, flush, stream, marks=["route", "score", "topk"])
+    score_ms = parts["score"] / steps
+    flops = 2.0 * 128 * wl.h * pairs
+    _, tc, kind = _peaks()
+    out["prefill_L131072"] = {"ms_per_step": ms / steps, "pairs_per_s": pairs / (ms / steps * 1e-3),
+                              "route_ms": parts["route"] / steps, "score_ms": score_ms,
+                              "topk_ms": parts["topk"] / steps,
+                              "score_tflops": flops / (score_ms * 1e-3) / 1e12,
+                              "score_frac_of_bf16_peak": flops / (score_ms * 1e-3) / 1e12 / tc}
+    del ix, q, w, keys, means
+
+    wl = make_workload("glm5_dagger_decode_L65536")
+    q, w, keys, so, pl = (x.to(dev) for x in (wl.q, wl.w, wl.keys, wl.seq_of, wl.prefix_len))
+    means = misa.block_stats(keys, wl.B)
+    dg = misa.MisaDaggerIndexer(wl.T, wl.H, wl.h, wl.L, wl.B, wl.kp, wl.k, device=dev)
+    ms = timed(lambda evs: dg.run(q, w, keys, means, so, pl))
+    out["glm5_dagger_decode_L65536"] = {"ms_per_step": ms, "pairs_per_s": int(wl.prefix_len.sum()) / (ms * 1e-3)}
+    del dg, q, w, keys, means
+
+    wl = make_workload("hisa_decode_L131072")
+    q, w, keys, so, pl = (x.to(dev) for x in (wl.q, wl.w, wl.keys, wl.seq_of, wl.prefix_len))
+    for B, m in ((128, 64), (64, 128)):
+        means = misa.block_stats(keys, B)
+        hx = misa.HisaIndexer(wl.T, wl.H, wl.L, B, m, wl.k, device=dev)
+        ms = timed(lambda evs: hx.run(q, w, keys, means, so, pl))
+        out[f"hisa_decode_L131072_B{B}_m{m}"] = {"ms_per_step": ms,
+                                                 "pairs_per_s": int(wl.prefix_len.sum()) / (ms * 1e-3)}
+    dx = misa.DenseIndexer(wl.T, wl.H, wl.L, wl.k, device=dev)
+    ms = timed(lambda evs: dx.run(q, w, keys, so, pl))
+    out["hisa_decode_L131072_dense64"] = {"ms_per_step": ms, "pairs_per_s": int(wl.prefix_len.sum()) / (ms * 1e-3)}
+    return out
+
+
+def _blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:  # noqa: BLE001
+        return 1
+
+
+def cpu_baseline(wl, budget_s: float = 15.0, max_queries: int | None = None):
+    """The fp64 oracle on whole queries of the workload until ~budget_s of CPU
+    work; pairs/s over the queries done."""
+    import oracle
+
+    done, pairs, t_used = 0, 0, 0.0
+    limit = max_queries or wl.T
+    for t in range(limit):
+        sub_q = wl.q[t:t + 1].to(torch.float64).numpy()
+        sub_w = wl.w[t:t + 1].numpy().astype(np.float64)
+        keys = wl.keys[int(wl.seq_of[t]):int(wl.seq_of[t]) + 1].to(torch.float64).numpy()
+        plen = wl.prefix_len[t:t + 1].numpy().astype(np.int64)
+        t0 = time.perf_counter()
+        oracle.misa_indexer(sub_q, sub_w, keys, np.zeros(1, np.int64), plen, wl.B, 1, wl.h, wl.k)
+        t_used += time.perf_counter() - t0
+        done += 1
+        pairs += int(plen[0])
+        if t_used >= budget_s:
+            break
+    return {"value": pairs / t_used, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{done} of {wl.T} queries of {wl.name} (full route+score+top-k each), {t_used:.1f} s"}
+
+
+def run_reference(args):
+    ws_n, rank, _ = _dist()
+    if rank != 0:
+        return
+    wl = make_workload(WORKLOAD)
+    # one query per step (its whole path); warm-up steps untimed
+    for i in range(args.warmup):
+        cpu_baseline(wl, budget_s=0.0, max_queries=1)
+    t0 = time.perf_counter()
+    res = [cpu_baseline(wl, budget_s=0.0, max_queries=1) for _ in range(args.steps)]
+    wall = time.perf_counter() - t0
+    value = statistics.median(r["value"] for r in res)
+    line = {
+        "impl": "reference",
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws_n, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": wall / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "queries": wl.T, "L": wl.L, "H": wl.H, "h": wl.h, "B": wl.B, "k": wl.k},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+                         "sample": "1 query of the batch per step (route + score + top-k in fp64 numpy)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
+    ap.add_argument("--quick", action="store_true", help="skip the other four workloads")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_cuda(args)
+
+
+if __name__ == "__main__":
+    main()

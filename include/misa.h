@@ -1,0 +1,260 @@
+/*
+ * misa.h -- C ABI of the B200 (sm_100a) token-indexer library libmisa.so.
+ *
+ * The library implements the indexer that sits in front of sparse attention in
+ * three forms:
+ *   - MISA: a router reads mean-pooled key blocks and keeps h of the H indexer
+ *     heads per query (block); only those heads score every prefix token; a
+ *     per-query top-k follows.
+ *     ["MISA: Mixture of Indexer Sparse Attention for Long-Context LLM
+ *     Inference" (gist.science), technical summary, "Methodology: MISA".]
+ *   - MISA-dagger (hierarchical MISA): the routed pass keeps k' candidates, all
+ *     H heads rescore them, top-k over the candidates.
+ *     [same page, "Hierarchical variant (MISA-dagger)".]
+ *   - HISA: mean-pooled B-token blocks are scored with all heads, the top-m
+ *     blocks are kept, the token indexer runs inside them, top-k.
+ *     ["HISA：为什么长文本理解的关键，藏在图书馆的分类索引里？" (zhichai.net),
+ *     section 三, Stage 1 and Stage 2.]
+ *   - the dense DSA indexer (all H heads score every token) is the same calls
+ *     with heads == NULL.  [MISA page, "Problem statement".]
+ *
+ * Indexer score (the pages print no formula; this is the library's definition):
+ *     S[t, s] = sum over active heads h (ascending id) of w[t, h] * ReLU(q[t, h] . k[s])
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Head dimension d is fixed at MISA_HEAD_DIM (128).
+ *  - bf16 arrays are passed as uint16_t bit patterns.  Layouts are row-major with
+ *    the innermost dimension contiguous:
+ *        q        [T][H][128]            bf16
+ *        w        [T][H]                 fp32
+ *        keys     row s of sequence b at keys + b * key_seq_stride + s * 128 (bf16)
+ *        means    block j of sequence b at means + b * means_seq_stride + j * 128 (fp32)
+ *        seq_of   [T] int32   which sequence (key cache) query t reads
+ *        prefix_len [T] int32 query t may see keys 0 <= s < prefix_len[t]
+ *  - Every pointer argument is a DEVICE pointer owned by the caller (except
+ *    where a comment says "host").  The library allocates no device memory,
+ *    keeps no pointer after a call returns and holds no global state apart from
+ *    constant tables and the cached address of the driver's tensor-map encoder.
+ *  - Every compute call is asynchronous on `stream` and never synchronises.
+ *    Only misa_error_query() synchronises (on the given stream).
+ *  - Arguments are checked on the host before anything is launched; a bad
+ *    argument returns MISA_ERR_INVALID_ARG (or MISA_ERR_UNSUPPORTED for a
+ *    well-formed request outside what the kernels implement, or
+ *    MISA_ERR_WORKSPACE for a workspace smaller than misa_workspace_bytes()).
+ *    Such a call has no effect.  A CUDA launch error returns MISA_ERR_CUDA.
+ *  - Device-side checks: an out-of-range seq_of[t] or head id, and a pipeline
+ *    wait that gives up (a bounded wait of about two seconds), are recorded as
+ *    bits in the error word at the start of the workspace (MISA_DEVERR_*); the
+ *    kernel then skips the affected work and returns.  Read the word with
+ *    misa_error_query(); clear it with misa_error_reset().
+ *  - Top-k order: larger score first, ties to the lower position; -0.0 ranks
+ *    equal to +0.0; entries equal to -inf (masked) are never selected.  The
+ *    selected positions are written in ascending order; when fewer than k
+ *    entries are valid the row is padded with -1.
+ *  - Visibility: key s is visible to query t iff 0 <= s < min(prefix_len[t], L).
+ *    A routing decision (and a HISA block score) sees block j iff the whole
+ *    block lies inside the prefix: min((j + 1) * B, L) <= prefix_len.
+ */
+#ifndef MISA_H
+#define MISA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Exported symbols of libmisa.so (the library is built with hidden default
+ * visibility; only the functions declared here are exported). */
+#if defined(__GNUC__)
+#define MISA_API __attribute__((visibility("default")))
+#else
+#define MISA_API
+#endif
+
+#define MISA_HEAD_DIM 128
+#define MISA_MAX_HEADS 128     /* H limit */
+#define MISA_MAX_TOPK 16384    /* k (and k') limit of misa_topk */
+#define MISA_ABI_VERSION 1
+
+/* Same object as cudaStream_t (a CUDA runtime stream handle); NULL is the
+ * legacy default stream. */
+typedef struct CUstream_st* misa_stream_t;
+
+typedef enum misa_status {
+  MISA_OK = 0,
+  MISA_ERR_INVALID_ARG = 1,  /* bad pointer, size, alignment or combination */
+  MISA_ERR_UNSUPPORTED = 2,  /* valid request the kernels do not implement */
+  MISA_ERR_WORKSPACE = 3,    /* workspace NULL or smaller than required */
+  MISA_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+  MISA_ERR_DEVICE = 5        /* misa_error_query: the device recorded an error */
+} misa_status;
+
+/* Bits of the device error word (first 4 bytes of every workspace). */
+#define MISA_DEVERR_TIMEOUT 1u    /* a bounded pipeline wait gave up */
+#define MISA_DEVERR_BAD_SEQ 2u    /* seq_of[t] outside [0, nseq) */
+#define MISA_DEVERR_BAD_HEAD 4u   /* a head id outside [0, H) */
+
+/* Static description of a status code (never NULL). */
+MISA_API const char* misa_status_string(int status);
+
+/* MISA_ABI_VERSION of the loaded library. */
+MISA_API int misa_abi_version(void);
+
+/* Operation ids for misa_workspace_bytes. */
+#define MISA_OP_ROUTE_HEADS 1
+#define MISA_OP_INDEX_SCORE 2
+#define MISA_OP_TOPK 3
+#define MISA_OP_HIER_RERANK 4
+#define MISA_OP_HISA_BLOCK_FILTER 5
+
+/* Bytes of device workspace the operation needs for these sizes (>= 256: the
+ * first 256 bytes hold the device error word).  Arguments an operation does not
+ * use are ignored:
+ *   ROUTE_HEADS: T, H, L, B;  INDEX_SCORE: none;  TOPK: none;
+ *   HIER_RERANK: T, kp;  HISA_BLOCK_FILTER: T, L, B.
+ * Returns 0 for an unknown op or negative sizes. */
+MISA_API size_t misa_workspace_bytes(int op, int T, int H, int64_t L, int B, int k, int kp);
+
+/* Set the device error word of `workspace` to 0 (asynchronous on stream). */
+MISA_API misa_status misa_error_reset(void* workspace, misa_stream_t stream);
+
+/* Synchronise `stream`, copy the device error word to *host_bits (host
+ * pointer) and return MISA_OK if it is 0, MISA_ERR_DEVICE otherwise. */
+MISA_API misa_status misa_error_query(const void* workspace, misa_stream_t stream, uint32_t* host_bits);
+
+/*
+ * misa_block_stats -- mean-pooled key blocks (the router's block statistics).
+ *   [MISA page, "Methodology: MISA": the prefix is split into M = ceil(L/B)
+ *   blocks summarised by their mean-pooled indexer keys; HISA page, Stage 1:
+ *   one mean-pooled representative per B-token block.]
+ * keys: nseq caches of L keys (row stride 128, sequence stride key_seq_stride
+ * elements; key_seq_stride may be 0 when nseq == 1).  Writes
+ *   means[b * M * 128 + j * 128 + c] = mean over s in block j of keys[b][s][c]
+ * as fp32 (fp32 accumulation of the bf16 inputs), M = ceil(L / B); the last,
+ * partial block averages the L - (M-1)*B keys it holds.
+ * Limits: 1 <= B <= 4096, L >= 1, nseq >= 1.  keys 16-byte aligned,
+ * key_seq_stride % 8 == 0.
+ */
+MISA_API misa_status misa_block_stats(const uint16_t* keys, int64_t nseq, int64_t L, int64_t key_seq_stride,
+                             int B, float* means, misa_stream_t stream);
+
+/*
+ * misa_route_heads -- block-aggregated head router (MISA).
+ *   [MISA page, "Methodology: MISA": per-head affinities against the block
+ *   statistics, aggregated into an importance per head, top-h heads kept; cost
+ *   O(H * M) per query.  MISA forum thread (zingnex.cn), "核心架构：轻量级路由器",
+ *   step 2: 8 of 64 heads kept per query.]
+ * Affinity A[t, h, j] = w[t, h] * ReLU(q[t, h] . means[seq_of[t]][j]).
+ * Queries [g*q_block, min((g+1)*q_block, T)) form routing decision g; block j is
+ * visible to it iff min((j+1)*B, L) <= prefix_len[g*q_block].
+ * importance[g][h] = sum over the decision's queries t and visible blocks j of
+ * A[t, h, j]; heads[g][0..h) = the h heads of largest importance (ties: lower
+ * head id), written in ascending id order.
+ *   means: nseq sequences of [M][128] fp32 at sequence stride means_seq_stride
+ *          elements (as written by misa_block_stats: M * 128); 16-byte aligned,
+ *          means_seq_stride % 4 == 0; seq_of values must lie in [0, nseq).
+ *   heads: [ceil(T/q_block)][h] int32 out.  importance: [ceil(T/q_block)][H]
+ *          fp32 out, may be NULL.
+ * Limits: 1 <= H <= 128, 1 <= h <= H, 1 <= q_block, T >= 1.
+ * workspace: >= misa_workspace_bytes(MISA_OP_ROUTE_HEADS, T, H, L, B, 0, 0).
+ */
+MISA_API misa_status misa_route_heads(const uint16_t* q, const float* w, const float* means,
+                             int64_t nseq, int64_t means_seq_stride, const int32_t* seq_of,
+                             const int32_t* prefix_len, int T, int H, int64_t L, int B,
+                             int q_block, int h, int32_t* heads, float* importance,
+                             void* workspace, size_t workspace_bytes, misa_stream_t stream);
+
+/*
+ * misa_index_score -- indexer scores of the active heads (the hot loop).
+ *   [MISA page, "Methodology: MISA": only the h active heads score every
+ *   prefix token; "Problem statement": the dense DSA indexer scores every prefix
+ *   token with all H_I heads.  HISA page, Stage 2: the token indexer runs only
+ *   inside the selected blocks (candidate mode).]
+ * Active heads of query t: heads[(t / q_block) * h + i], i < h (any order; the
+ * sum runs in ascending i), or all H heads when heads == NULL (dense indexer; h
+ * is then ignored and taken as H).
+ *   cand == NULL: scores[t * scores_row_stride + s] for 0 <= s < L, -inf where
+ *     s >= prefix_len[t].
+ *   cand != NULL: cand is [T][n_cand] int32 token ids (-1 = empty slot);
+ *     scores[t * scores_row_stride + p] for 0 <= p < n_cand is the score of token
+ *     cand[t][p], or -inf if that id is < 0 or >= min(prefix_len[t], L).
+ * keys: nkeyseq caches (seq_of values must lie in [0, nkeyseq)); key_seq_stride
+ *   must be 0 when nkeyseq == 1 and queries share the cache.
+ * Limits: 1 <= H <= 128, 1 <= h <= 128, L >= 1, keys 16-byte aligned,
+ *   key_seq_stride % 128 == 0, scores_row_stride >= (cand ? n_cand : L).
+ * workspace: >= 256 bytes (error word).
+ */
+MISA_API misa_status misa_index_score(const uint16_t* q, const float* w, const uint16_t* keys,
+                             int64_t nkeyseq, int64_t key_seq_stride, const int32_t* seq_of,
+                             const int32_t* prefix_len, int T, int H, int64_t L,
+                             const int32_t* heads, int h, int q_block,
+                             const int32_t* cand, int n_cand,
+                             float* scores, int64_t scores_row_stride,
+                             void* workspace, size_t workspace_bytes, misa_stream_t stream);
+
+/*
+ * misa_topk -- per-row top-k of fp32 scores (fused radix select).
+ *   [MISA forum thread, "DeepSeek稀疏注意力（DSA）的突破": the indexer keeps the
+ *   most relevant token subset; HISA page, section 二: top-k tokens per query;
+ *   section 四: the output is k token indices.]
+ * Row t is scores[t * row_stride + p], 0 <= p < n_t, with n_t = n, or
+ * min(n, row_valid[t]) when row_valid != NULL.  idx[t * k + i] receives the
+ * selected positions in ascending order (translated through
+ * id_map[t * id_map_stride + p] when id_map != NULL), -1 padded.
+ * Limits: 1 <= k <= MISA_MAX_TOPK, n >= 1, row_stride % 4 == 0 and >= n,
+ *   scores 16-byte aligned.
+ * workspace: >= 256 bytes.
+ */
+MISA_API misa_status misa_topk(const float* scores, int T, int64_t n, int64_t row_stride,
+                      const int32_t* row_valid, const int32_t* id_map, int64_t id_map_stride,
+                      int k, int32_t* idx, void* workspace, size_t workspace_bytes,
+                      misa_stream_t stream);
+
+/*
+ * misa_hier_rerank -- fine stage of MISA-dagger: all H heads rescore each
+ * query's k' candidates and the top-k of them are kept.
+ *   [MISA page, "Hierarchical variant (MISA-dagger)": the original DSA indexer
+ *   (all H_I heads) rescores only the candidate set; the final top-k is taken
+ *   among the candidates.]
+ * cand: [T][kp] int32 token ids (typically the coarse misa_topk output, -1 =
+ * empty).  cand_scores: [T][kp] fp32 out, may be NULL.  idx: [T][k] out
+ * (token ids, ascending candidate position order, -1 padded).
+ * Limits: as misa_index_score and misa_topk; 1 <= k <= kp.
+ * workspace: >= misa_workspace_bytes(MISA_OP_HIER_RERANK, T, H, L, B, k, kp).
+ */
+MISA_API misa_status misa_hier_rerank(const uint16_t* q, const float* w, const uint16_t* keys,
+                             int64_t nkeyseq, int64_t key_seq_stride, const int32_t* seq_of,
+                             const int32_t* prefix_len, int T, int H, int64_t L,
+                             const int32_t* cand, int kp, int k, float* cand_scores,
+                             int32_t* idx, void* workspace, size_t workspace_bytes,
+                             misa_stream_t stream);
+
+/*
+ * hisa_block_filter -- HISA Stage 1: block scores with all heads, top-m blocks,
+ * candidate token list.
+ *   [HISA page, section 三, Stage 1: the query is scored against the
+ *   mean-pooled block representatives only and the top-m blocks are kept, cost
+ *   O(L/B); Stage 2 then looks at the at most m*B tokens inside them.]
+ * block score bs[t][j] = sum over all H heads of w[t,h] * ReLU(q[t,h] . means_j)
+ * for visible blocks (min((j+1)*B, L) <= prefix_len[t]), -inf otherwise.
+ * blocks[t][0..m): chosen block ids ascending, -1 padded.
+ * cand[t][i*B + r] = blocks[t][i]*B + r, or -1 if that block slot is empty or the
+ * id is >= min(prefix_len[t], L).  block_scores: [T][M] fp32 out, may be NULL.
+ * means / nseq / means_seq_stride as for misa_route_heads.
+ * Limits: 1 <= H <= 128, 1 <= m <= MISA_MAX_TOPK, 1 <= B.
+ * workspace: >= misa_workspace_bytes(MISA_OP_HISA_BLOCK_FILTER, T, H, L, B, m, 0).
+ */
+MISA_API misa_status hisa_block_filter(const uint16_t* q, const float* w, const float* means,
+                              int64_t nseq, int64_t means_seq_stride, const int32_t* seq_of,
+                              const int32_t* prefix_len, int T, int H, int64_t L, int B, int m,
+                              int32_t* blocks, int32_t* cand, float* block_scores,
+                              void* workspace, size_t workspace_bytes, misa_stream_t stream);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif /* MISA_H */

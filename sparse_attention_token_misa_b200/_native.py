@@ -1,0 +1,254 @@
+"""ctypes binding of libmisa.so (argument marshalling only).
+
+Every function here forwards device pointers, sizes and the current CUDA
+stream of torch to the C ABI declared in include/misa.h; all arithmetic runs
+in the library's CUDA kernels.  If the library is missing or cannot be
+loaded, the first call raises: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmisa.so")
+
+OP_ROUTE_HEADS = 1
+OP_INDEX_SCORE = 2
+OP_TOPK = 3
+OP_HIER_RERANK = 4
+OP_HISA_BLOCK_FILTER = 5
+
+DEVERR_TIMEOUT = 1
+DEVERR_BAD_SEQ = 2
+DEVERR_BAD_HEAD = 4
+
+HEAD_DIM = 128
+
+_lib = None
+
+c_i64 = ctypes.c_int64
+c_int = ctypes.c_int
+c_size = ctypes.c_size_t
+c_vp = ctypes.c_void_p
+
+# name -> (restype, argtypes), in the order of include/misa.h
+SIGNATURES = {
+    "misa_status_string": (ctypes.c_char_p, [c_int]),
+    "misa_abi_version": (c_int, []),
+    "misa_workspace_bytes": (c_size, [c_int, c_int, c_int, c_i64, c_int, c_int, c_int]),
+    "misa_error_reset": (c_int, [c_vp, c_vp]),
+    "misa_error_query": (c_int, [c_vp, c_vp, ctypes.POINTER(ctypes.c_uint32)]),
+    "misa_block_stats": (c_int, [c_vp, c_i64, c_i64, c_i64, c_int, c_vp, c_vp]),
+    "misa_route_heads": (c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_i64, c_int,
+                                 c_int, c_int, c_vp, c_vp, c_vp, c_size, c_vp]),
+    "misa_index_score": (c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_i64, c_vp, c_int,
+                                 c_int, c_vp, c_int, c_vp, c_i64, c_vp, c_size, c_vp]),
+    "misa_topk": (c_int, [c_vp, c_int, c_i64, c_i64, c_vp, c_vp, c_i64, c_int, c_vp, c_vp, c_size, c_vp]),
+    "misa_hier_rerank": (c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_i64, c_vp, c_int,
+                                 c_int, c_vp, c_vp, c_vp, c_size, c_vp]),
+    "hisa_block_filter": (c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_i64, c_int, c_int,
+                                  c_vp, c_vp, c_vp, c_vp, c_size, c_vp]),
+}
+
+
+class MisaError(RuntimeError):
+    """A libmisa call returned a non-OK status."""
+
+    def __init__(self, name: str, status: int):
+        self.status = status
+        super().__init__(f"{name}: status {status} ({status_string(status)})")
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmisa.so (once).  Raises if it is missing: nothing runs without it."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"libmisa.so not found at {LIB_PATH}; build it with "
+                "`python -m sparse_attention_token_misa_b200.build`")
+        l = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(l, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = l
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().misa_status_string(int(status)).decode()
+
+
+def _call(name: str, *args) -> None:
+    st = getattr(lib(), name)(*args)
+    if st != 0:
+        raise MisaError(name, st)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _p(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libmisa takes device tensors")
+    return t.data_ptr()
+
+
+def _req(t: torch.Tensor, dtype, name: str, contiguous: bool = True):
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if contiguous and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def workspace_bytes(op: int, T: int, H: int, L: int, B: int, k: int = 0, kp: int = 0) -> int:
+    return int(lib().misa_workspace_bytes(op, T, H, L, B, k, kp))
+
+
+def alloc_workspace(nbytes: int, device=None) -> torch.Tensor:
+    """Zeroed uint8 device buffer of at least nbytes (16-byte aligned by torch)."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device or "cuda")
+
+
+def error_reset(workspace: torch.Tensor, stream=None) -> None:
+    _call("misa_error_reset", _p(workspace), _stream(stream))
+
+
+def error_query(workspace: torch.Tensor, stream=None) -> int:
+    bits = ctypes.c_uint32(0)
+    st = lib().misa_error_query(_p(workspace), _stream(stream), ctypes.byref(bits))
+    if st not in (0, 5):
+        raise MisaError("misa_error_query", st)
+    return int(bits.value)
+
+
+def _key_stride(keys: torch.Tensor) -> int:
+    # one cache for every query -> stride 0 lets the kernel batch queries per MMA
+    return 0 if keys.shape[0] == 1 else int(keys.stride(0))
+
+
+def block_stats(keys: torch.Tensor, B: int, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """misa_block_stats: keys [nseq, L, 128] bf16 -> means [nseq, M, 128] fp32."""
+    _req(keys, torch.bfloat16, "keys", contiguous=False)
+    if keys.stride(2) != 1 or keys.stride(1) != HEAD_DIM:
+        raise ValueError("keys rows must be contiguous 128-element rows")
+    nseq, L, _ = keys.shape
+    M = (L + B - 1) // B
+    if out is None:
+        out = torch.empty((nseq, M, HEAD_DIM), dtype=torch.float32, device=keys.device)
+    _call("misa_block_stats", _p(keys), nseq, L, _key_stride(keys) if nseq > 1 else 0, B, _p(out), _stream(stream))
+    return out
+
+
+def route_heads(q, w, means, seq_of, prefix_len, L: int, B: int, q_block: int, h: int,
+                heads=None, importance=None, workspace=None, want_importance: bool = True, stream=None):
+    """misa_route_heads -> (heads [G, h] int32, importance [G, H] fp32 or None)."""
+    _req(q, torch.bfloat16, "q"); _req(w, torch.float32, "w"); _req(means, torch.float32, "means")
+    _req(seq_of, torch.int32, "seq_of"); _req(prefix_len, torch.int32, "prefix_len")
+    T, H, _ = q.shape
+    G = (T + q_block - 1) // q_block
+    dev = q.device
+    if heads is None:
+        heads = torch.empty((G, h), dtype=torch.int32, device=dev)
+    if importance is None and want_importance:
+        importance = torch.empty((G, H), dtype=torch.float32, device=dev)
+    need = workspace_bytes(OP_ROUTE_HEADS, T, H, L, B)
+    if workspace is None:
+        workspace = alloc_workspace(need, dev)
+    _call("misa_route_heads", _p(q), _p(w), _p(means), means.shape[0], int(means.stride(0)), _p(seq_of),
+          _p(prefix_len), T, H, L, B, q_block, h, _p(heads), _p(importance), _p(workspace),
+          workspace.numel(), _stream(stream))
+    return heads, importance
+
+
+def index_score(q, w, keys, seq_of, prefix_len, heads=None, h: int | None = None, q_block: int = 1,
+                cand=None, scores=None, workspace=None, stream=None) -> torch.Tensor:
+    """misa_index_score -> scores [T, L] (or [T, n_cand]) fp32."""
+    _req(q, torch.bfloat16, "q"); _req(w, torch.float32, "w"); _req(keys, torch.bfloat16, "keys")
+    _req(seq_of, torch.int32, "seq_of"); _req(prefix_len, torch.int32, "prefix_len")
+    T, H, _ = q.shape
+    L = keys.shape[1]
+    if heads is not None:
+        _req(heads, torch.int32, "heads")
+        h = heads.shape[1] if h is None else h
+    n_cand = 0
+    if cand is not None:
+        _req(cand, torch.int32, "cand")
+        n_cand = cand.shape[1]
+    ncol = n_cand if cand is not None else L
+    if scores is None:
+        scores = torch.empty((T, ncol), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(256, q.device)
+    _call("misa_index_score", _p(q), _p(w), _p(keys), keys.shape[0], _key_stride(keys), _p(seq_of),
+          _p(prefix_len), T, H, L, _p(heads), int(h or H), q_block, _p(cand), n_cand, _p(scores),
+          int(scores.stride(0)), _p(workspace), workspace.numel(), _stream(stream))
+    return scores
+
+
+def topk(scores, k: int, n: int | None = None, row_valid=None, id_map=None, idx=None, workspace=None,
+         stream=None) -> torch.Tensor:
+    """misa_topk -> idx [T, k] int32 (ascending positions / ids, -1 padded)."""
+    _req(scores, torch.float32, "scores", contiguous=False)
+    T = scores.shape[0]
+    n = scores.shape[1] if n is None else n
+    if idx is None:
+        idx = torch.empty((T, k), dtype=torch.int32, device=scores.device)
+    if workspace is None:
+        workspace = alloc_workspace(256, scores.device)
+    idm_stride = 0
+    if id_map is not None:
+        _req(id_map, torch.int32, "id_map", contiguous=False)
+        idm_stride = int(id_map.stride(0))
+    _call("misa_topk", _p(scores), T, n, int(scores.stride(0)), _p(row_valid), _p(id_map), idm_stride, k, _p(idx),
+          _p(workspace), workspace.numel(), _stream(stream))
+    return idx
+
+
+def hier_rerank(q, w, keys, seq_of, prefix_len, cand, k: int, idx=None, cand_scores=None, want_scores=False,
+                workspace=None, stream=None):
+    """misa_hier_rerank -> (idx [T, k], cand_scores [T, kp] or None)."""
+    T, H, _ = q.shape
+    L = keys.shape[1]
+    kp = cand.shape[1]
+    _req(cand, torch.int32, "cand")
+    if idx is None:
+        idx = torch.empty((T, k), dtype=torch.int32, device=q.device)
+    if cand_scores is None and want_scores:
+        cand_scores = torch.empty((T, kp), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(workspace_bytes(OP_HIER_RERANK, T, H, L, 1, k, kp), q.device)
+    _call("misa_hier_rerank", _p(q), _p(w), _p(keys), keys.shape[0], _key_stride(keys), _p(seq_of),
+          _p(prefix_len), T, H, L, _p(cand), kp, k, _p(cand_scores), _p(idx), _p(workspace), workspace.numel(),
+          _stream(stream))
+    return idx, cand_scores
+
+
+def hisa_block_filter(q, w, means, seq_of, prefix_len, L: int, B: int, m: int, blocks=None, cand=None,
+                      block_scores=None, want_scores=False, workspace=None, stream=None):
+    """hisa_block_filter -> (blocks [T, m], cand [T, m*B], block_scores [T, M] or None)."""
+    T, H, _ = q.shape
+    M = (L + B - 1) // B
+    dev = q.device
+    if blocks is None:
+        blocks = torch.empty((T, m), dtype=torch.int32, device=dev)
+    if cand is None:
+        cand = torch.empty((T, m * B), dtype=torch.int32, device=dev)
+    if block_scores is None and want_scores:
+        block_scores = torch.empty((T, M), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = alloc_workspace(workspace_bytes(OP_HISA_BLOCK_FILTER, T, H, L, B, m), dev)
+    _call("hisa_block_filter", _p(q), _p(w), _p(means), means.shape[0], int(means.stride(0)), _p(seq_of),
+          _p(prefix_len), T, H, L, B, m, _p(blocks), _p(cand), _p(block_scores), _p(workspace), workspace.numel(),
+          _stream(stream))
+    return blocks, cand, block_scores

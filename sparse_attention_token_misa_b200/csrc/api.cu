@@ -1,0 +1,328 @@
+// C ABI of libmisa: host-side argument checks, workspace sizing, TMA tensor
+// maps and kernel launches.  See include/misa.h for the contract of each call.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstring>
+#include <mutex>
+
+#include "../../include/misa.h"
+#include "launch.h"
+
+namespace {
+
+constexpr size_t kErrBytes = 256;
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline int64_t round_up4(int64_t x) { return (x + 3) / 4 * 4; }
+
+inline misa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MISA_OK : MISA_ERR_CUDA; }
+
+uint32_t* err_word(void* ws) { return reinterpret_cast<uint32_t*>(ws); }
+
+// cuTensorMapEncodeTiled, fetched once from the driver through the runtime so
+// that the library needs no link-time dependency on libcuda.
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D map over all key rows: dim0 = 128 bf16 (256 B), dim1 = rows; box = 64 x 128
+// with 128-byte swizzle, the layout the UMMA descriptors expect.
+misa_status make_key_map(const uint16_t* keys, int64_t rows, CUtensorMap* map) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return MISA_ERR_CUDA;
+  std::memset(map, 0, sizeof(*map));
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(MISA_HEAD_DIM), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(MISA_HEAD_DIM) * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(keys), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MISA_OK : MISA_ERR_CUDA;
+}
+
+misa_status check_ws(const void* ws, size_t have, size_t need) {
+  if (!ws || have < need) return MISA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return MISA_ERR_INVALID_ARG;
+  return MISA_OK;
+}
+
+// Shared argument checks of the scoring call.
+misa_status check_score_args(const uint16_t* q, const float* w, const uint16_t* keys, int64_t nkeyseq,
+                             int64_t key_seq_stride, const int32_t* seq_of, const int32_t* prefix_len, int T, int H,
+                             int64_t L, const int32_t* heads, int h, int q_block, const int32_t* cand, int n_cand,
+                             const float* scores, int64_t row_stride) {
+  if (!q || !w || !keys || !seq_of || !prefix_len || !scores) return MISA_ERR_INVALID_ARG;
+  if (T < 1 || H < 1 || L < 1 || nkeyseq < 1) return MISA_ERR_INVALID_ARG;
+  if (H > MISA_MAX_HEADS) return MISA_ERR_UNSUPPORTED;
+  if (heads) {
+    if (h < 1 || h > H || q_block < 1) return MISA_ERR_INVALID_ARG;
+  }
+  if (!aligned16(q) || !aligned16(keys)) return MISA_ERR_INVALID_ARG;
+  if (key_seq_stride < 0 || key_seq_stride % MISA_HEAD_DIM != 0) return MISA_ERR_INVALID_ARG;
+  if (key_seq_stride != 0 && key_seq_stride < L * MISA_HEAD_DIM) return MISA_ERR_INVALID_ARG;
+  if (cand) {
+    if (n_cand < 1 || row_stride < n_cand) return MISA_ERR_INVALID_ARG;
+  } else {
+    if (row_stride < L) return MISA_ERR_INVALID_ARG;
+  }
+  const int64_t rows = (nkeyseq - 1) * (key_seq_stride / MISA_HEAD_DIM) + L;
+  if (rows + 128 >= (static_cast<int64_t>(1) << 31)) return MISA_ERR_UNSUPPORTED;  // TMA coordinates are int32
+  if (L >= (static_cast<int64_t>(1) << 31) - 128) return MISA_ERR_UNSUPPORTED;
+  return MISA_OK;
+}
+
+misa_status check_topk_args(const float* scores, int T, int64_t n, int64_t row_stride, const int32_t* id_map,
+                            int64_t id_map_stride, int k, const int32_t* idx) {
+  if (!scores || !idx) return MISA_ERR_INVALID_ARG;
+  if (T < 1 || n < 1 || k < 1) return MISA_ERR_INVALID_ARG;
+  if (k > MISA_MAX_TOPK) return MISA_ERR_UNSUPPORTED;
+  if (n >= (static_cast<int64_t>(1) << 31)) return MISA_ERR_UNSUPPORTED;
+  if (row_stride < n || row_stride % 4 != 0 || !aligned16(scores)) return MISA_ERR_INVALID_ARG;
+  if (id_map && id_map_stride < n) return MISA_ERR_INVALID_ARG;
+  return MISA_OK;
+}
+
+misa_status check_block_args(const uint16_t* q, const float* w, const float* means, int64_t nseq,
+                             int64_t means_seq_stride, const int32_t* seq_of, const int32_t* prefix_len, int T,
+                             int H, int64_t L, int B) {
+  if (!q || !w || !means || !seq_of || !prefix_len) return MISA_ERR_INVALID_ARG;
+  if (T < 1 || H < 1 || L < 1 || B < 1 || nseq < 1) return MISA_ERR_INVALID_ARG;
+  if (H > MISA_MAX_HEADS) return MISA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(means) || means_seq_stride < 0 || means_seq_stride % 4 != 0)
+    return MISA_ERR_INVALID_ARG;
+  const int64_t M = ceil_div(L, B);
+  if (nseq > 1 && means_seq_stride < M * MISA_HEAD_DIM) return MISA_ERR_INVALID_ARG;
+  if (M >= (static_cast<int64_t>(1) << 24) || nseq >= (static_cast<int64_t>(1) << 31)) return MISA_ERR_UNSUPPORTED;
+  return MISA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* misa_status_string(int status) {
+  switch (status) {
+    case MISA_OK: return "ok";
+    case MISA_ERR_INVALID_ARG: return "invalid argument";
+    case MISA_ERR_UNSUPPORTED: return "unsupported size or mode";
+    case MISA_ERR_WORKSPACE: return "workspace missing or too small";
+    case MISA_ERR_CUDA: return "CUDA runtime error";
+    case MISA_ERR_DEVICE: return "device recorded an error";
+    default: return "unknown status";
+  }
+}
+
+int misa_abi_version(void) { return MISA_ABI_VERSION; }
+
+size_t misa_workspace_bytes(int op, int T, int H, int64_t L, int B, int k, int kp) {
+  (void)k;
+  if (T < 0 || H < 0 || L < 0 || B < 0 || kp < 0) return 0;
+  switch (op) {
+    case MISA_OP_ROUTE_HEADS: {
+      if (B < 1) return 0;
+      const int64_t M = ceil_div(L, B);
+      const int64_t nch = misa::router_chunks(static_cast<int>(M));
+      return kErrBytes + static_cast<size_t>(T) * nch * H * sizeof(float);
+    }
+    case MISA_OP_INDEX_SCORE:
+    case MISA_OP_TOPK:
+      return kErrBytes;
+    case MISA_OP_HIER_RERANK:
+      return kErrBytes + static_cast<size_t>(T) * round_up4(kp) * sizeof(float);
+    case MISA_OP_HISA_BLOCK_FILTER: {
+      if (B < 1) return 0;
+      const int64_t M = ceil_div(L, B);
+      return kErrBytes + static_cast<size_t>(T) * round_up4(M) * sizeof(float);
+    }
+    default:
+      return 0;
+  }
+}
+
+misa_status misa_error_reset(void* workspace, misa_stream_t stream) {
+  if (!workspace) return MISA_ERR_INVALID_ARG;
+  return cuda_status(cudaMemsetAsync(workspace, 0, sizeof(uint32_t), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+misa_status misa_error_query(const void* workspace, misa_stream_t stream, uint32_t* host_bits) {
+  if (!workspace || !host_bits) return MISA_ERR_INVALID_ARG;
+  uint32_t v = 0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return MISA_ERR_CUDA;
+  *host_bits = v;
+  return v == 0 ? MISA_OK : MISA_ERR_DEVICE;
+}
+
+misa_status misa_block_stats(const uint16_t* keys, int64_t nseq, int64_t L, int64_t key_seq_stride, int B,
+                             float* means, misa_stream_t stream) {
+  if (!keys || !means || nseq < 1 || L < 1 || B < 1) return MISA_ERR_INVALID_ARG;
+  if (B > 4096) return MISA_ERR_UNSUPPORTED;
+  if (!aligned16(keys) || !aligned16(means) || key_seq_stride < 0 || key_seq_stride % 8 != 0)
+    return MISA_ERR_INVALID_ARG;
+  if (nseq > 1 && key_seq_stride < L * MISA_HEAD_DIM) return MISA_ERR_INVALID_ARG;
+  return cuda_status(misa::launch_block_stats(keys, nseq, L, key_seq_stride, B, means,
+                                              reinterpret_cast<cudaStream_t>(stream)));
+}
+
+misa_status misa_route_heads(const uint16_t* q, const float* w, const float* means, int64_t nseq,
+                             int64_t means_seq_stride, const int32_t* seq_of, const int32_t* prefix_len, int T, int H,
+                             int64_t L, int B, int q_block, int h, int32_t* heads, float* importance, void* workspace,
+                             size_t workspace_bytes, misa_stream_t stream) {
+  misa_status st = check_block_args(q, w, means, nseq, means_seq_stride, seq_of, prefix_len, T, H, L, B);
+  if (st != MISA_OK) return st;
+  if (!heads || q_block < 1 || h < 1 || h > H) return MISA_ERR_INVALID_ARG;
+  st = check_ws(workspace, workspace_bytes, misa_workspace_bytes(MISA_OP_ROUTE_HEADS, T, H, L, B, 0, 0));
+  if (st != MISA_OK) return st;
+  float* partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kErrBytes);
+  return cuda_status(misa::launch_route_heads(q, w, means, means_seq_stride, seq_of, prefix_len, T, H, L, B, q_block,
+                                              h, static_cast<int>(nseq), heads, importance, partial,
+                                              err_word(workspace), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+misa_status misa_index_score(const uint16_t* q, const float* w, const uint16_t* keys, int64_t nkeyseq,
+                             int64_t key_seq_stride, const int32_t* seq_of, const int32_t* prefix_len, int T, int H,
+                             int64_t L, const int32_t* heads, int h, int q_block, const int32_t* cand, int n_cand,
+                             float* scores, int64_t scores_row_stride, void* workspace, size_t workspace_bytes,
+                             misa_stream_t stream) {
+  misa_status st = check_score_args(q, w, keys, nkeyseq, key_seq_stride, seq_of, prefix_len, T, H, L, heads, h,
+                                    q_block, cand, n_cand, scores, scores_row_stride);
+  if (st != MISA_OK) return st;
+  st = check_ws(workspace, workspace_bytes, kErrBytes);
+  if (st != MISA_OK) return st;
+  CUtensorMap map;
+  const CUtensorMap* mp = nullptr;
+  if (!cand) {
+    const int64_t rows = (nkeyseq - 1) * (key_seq_stride / MISA_HEAD_DIM) + L;
+    st = make_key_map(keys, rows, &map);
+    if (st != MISA_OK) return st;
+    mp = &map;
+  }
+  misa::ScoreArgs a;
+  a.q = q;
+  a.w = w;
+  a.keys = keys;
+  a.nkeyseq = nkeyseq;
+  a.key_seq_stride = key_seq_stride;
+  a.seq_of = seq_of;
+  a.prefix_len = prefix_len;
+  a.T = T;
+  a.H = H;
+  a.L = L;
+  a.heads = heads;
+  a.h = heads ? h : H;
+  a.q_block = heads ? q_block : 1;
+  a.cand = cand;
+  a.n_cand = cand ? n_cand : 0;
+  a.scores = scores;
+  a.row_stride = scores_row_stride;
+  a.err = err_word(workspace);
+  return cuda_status(misa::launch_index_score(mp, a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+misa_status misa_topk(const float* scores, int T, int64_t n, int64_t row_stride, const int32_t* row_valid,
+                      const int32_t* id_map, int64_t id_map_stride, int k, int32_t* idx, void* workspace,
+                      size_t workspace_bytes, misa_stream_t stream) {
+  misa_status st = check_topk_args(scores, T, n, row_stride, id_map, id_map_stride, k, idx);
+  if (st != MISA_OK) return st;
+  st = check_ws(workspace, workspace_bytes, kErrBytes);
+  if (st != MISA_OK) return st;
+  return cuda_status(misa::launch_topk(scores, T, n, row_stride, row_valid, id_map, id_map_stride, k, idx,
+                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
+misa_status misa_hier_rerank(const uint16_t* q, const float* w, const uint16_t* keys, int64_t nkeyseq,
+                             int64_t key_seq_stride, const int32_t* seq_of, const int32_t* prefix_len, int T, int H,
+                             int64_t L, const int32_t* cand, int kp, int k, float* cand_scores, int32_t* idx,
+                             void* workspace, size_t workspace_bytes, misa_stream_t stream) {
+  if (!cand || !idx || kp < 1 || k < 1 || k > kp || T < 1) return MISA_ERR_INVALID_ARG;
+  if (k > MISA_MAX_TOPK) return MISA_ERR_UNSUPPORTED;
+  misa_status st = check_ws(workspace, workspace_bytes, misa_workspace_bytes(MISA_OP_HIER_RERANK, T, H, L, 1, k, kp));
+  if (st != MISA_OK) return st;
+  const int64_t kp_pad = round_up4(kp);
+  float* ws_scores = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kErrBytes);
+  st = check_score_args(q, w, keys, nkeyseq, key_seq_stride, seq_of, prefix_len, T, H, L, nullptr, H, 1, cand, kp,
+                        ws_scores, kp_pad);
+  if (st != MISA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  misa::ScoreArgs a;
+  a.q = q;
+  a.w = w;
+  a.keys = keys;
+  a.nkeyseq = nkeyseq;
+  a.key_seq_stride = key_seq_stride;
+  a.seq_of = seq_of;
+  a.prefix_len = prefix_len;
+  a.T = T;
+  a.H = H;
+  a.L = L;
+  a.heads = nullptr;
+  a.h = H;
+  a.q_block = 1;
+  a.cand = cand;
+  a.n_cand = kp;
+  a.scores = ws_scores;
+  a.row_stride = kp_pad;
+  a.err = err_word(workspace);
+  cudaError_t e = misa::launch_index_score(nullptr, a, s);
+  if (e != cudaSuccess) return MISA_ERR_CUDA;
+  e = misa::launch_topk(ws_scores, T, kp, kp_pad, nullptr, cand, kp, k, idx, s);
+  if (e != cudaSuccess) return MISA_ERR_CUDA;
+  if (cand_scores) {
+    e = cudaMemcpy2DAsync(cand_scores, static_cast<size_t>(kp) * sizeof(float), ws_scores,
+                          static_cast<size_t>(kp_pad) * sizeof(float), static_cast<size_t>(kp) * sizeof(float), T,
+                          cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return MISA_ERR_CUDA;
+  }
+  return MISA_OK;
+}
+
+misa_status hisa_block_filter(const uint16_t* q, const float* w, const float* means, int64_t nseq,
+                              int64_t means_seq_stride, const int32_t* seq_of, const int32_t* prefix_len, int T, int H,
+                              int64_t L, int B, int m, int32_t* blocks, int32_t* cand, float* block_scores,
+                              void* workspace, size_t workspace_bytes, misa_stream_t stream) {
+  misa_status st = check_block_args(q, w, means, nseq, means_seq_stride, seq_of, prefix_len, T, H, L, B);
+  if (st != MISA_OK) return st;
+  if (!blocks || !cand || m < 1) return MISA_ERR_INVALID_ARG;
+  if (m > MISA_MAX_TOPK) return MISA_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(m) * B >= (static_cast<int64_t>(1) << 31)) return MISA_ERR_UNSUPPORTED;
+  st = check_ws(workspace, workspace_bytes, misa_workspace_bytes(MISA_OP_HISA_BLOCK_FILTER, T, H, L, B, m, 0));
+  if (st != MISA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t M = ceil_div(L, B);
+  const int64_t M_pad = round_up4(M);
+  float* bs = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kErrBytes);
+  cudaError_t e = misa::launch_hisa_block_scores(q, w, means, means_seq_stride, seq_of, prefix_len, T, H, L, B,
+                                                 static_cast<int>(nseq), bs, M_pad, err_word(workspace), s);
+  if (e != cudaSuccess) return MISA_ERR_CUDA;
+  e = misa::launch_topk(bs, T, M, M_pad, nullptr, nullptr, 0, m, blocks, s);
+  if (e != cudaSuccess) return MISA_ERR_CUDA;
+  e = misa::launch_hisa_expand(blocks, prefix_len, T, m, B, L, cand, s);
+  if (e != cudaSuccess) return MISA_ERR_CUDA;
+  if (block_scores) {
+    e = cudaMemcpy2DAsync(block_scores, static_cast<size_t>(M) * sizeof(float), bs,
+                          static_cast<size_t>(M_pad) * sizeof(float), static_cast<size_t>(M) * sizeof(float), T,
+                          cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return MISA_ERR_CUDA;
+  }
+  return MISA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,107 @@
+"""The four indexers as sequences of libmisa calls with preallocated buffers.
+
+Each class owns its device buffers (outputs and workspaces) for one batch shape
+and issues the C-ABI calls on the current CUDA stream in `run`, so a step
+allocates nothing and can be captured in a CUDA graph.  All arithmetic runs in
+the library's kernels.
+
+* MisaIndexer   -- router (h of H heads per query block), routed token scoring,
+                   top-k.  MISA page (gist.science), "Methodology: MISA".
+* DenseIndexer  -- all H heads score every token, top-k (the DSA indexer).
+* MisaDaggerIndexer -- routed coarse top-k', all-head rerank, top-k.  MISA page,
+                   "Hierarchical variant (MISA-dagger)".
+* HisaIndexer   -- block filter (top-m blocks), all-head scoring of their
+                   tokens, top-k.  HISA explainer (zhichai.net), 三, Stage 1/2.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import _native as nat
+
+
+def _pad4(n: int) -> int:
+    return (n + 3) // 4 * 4
+
+
+class MisaIndexer:
+    def __init__(self, T: int, H: int, h: int, L: int, B: int, k: int, q_block: int = 1, device="cuda"):
+        self.T, self.H, self.h, self.L, self.B, self.k, self.q_block = T, H, h, L, B, k, q_block
+        G = (T + q_block - 1) // q_block
+        self.heads = torch.empty((G, h), dtype=torch.int32, device=device)
+        self.importance = torch.empty((G, H), dtype=torch.float32, device=device)
+        self.scores_buf = torch.empty((T, _pad4(L)), dtype=torch.float32, device=device)
+        self.scores = self.scores_buf[:, :L]
+        self.idx = torch.empty((T, k), dtype=torch.int32, device=device)
+        self.ws_route = nat.alloc_workspace(nat.workspace_bytes(nat.OP_ROUTE_HEADS, T, H, L, B), device)
+        self.ws = nat.alloc_workspace(256, device)
+
+    def route(self, q, w, means, seq_of, prefix_len, stream=None):
+        nat.route_heads(q, w, means, seq_of, prefix_len, self.L, self.B, self.q_block, self.h,
+                        heads=self.heads, importance=self.importance, workspace=self.ws_route, stream=stream)
+
+    def score(self, q, w, keys, seq_of, prefix_len, stream=None):
+        nat.index_score(q, w, keys, seq_of, prefix_len, heads=self.heads, h=self.h, q_block=self.q_block,
+                        scores=self.scores_buf, workspace=self.ws, stream=stream)
+
+    def select(self, prefix_len, stream=None):
+        nat.topk(self.scores_buf, self.k, n=self.L, row_valid=prefix_len, idx=self.idx, workspace=self.ws,
+                 stream=stream)
+
+    def run(self, q, w, keys, means, seq_of, prefix_len, stream=None) -> torch.Tensor:
+        self.route(q, w, means, seq_of, prefix_len, stream)
+        self.score(q, w, keys, seq_of, prefix_len, stream)
+        self.select(prefix_len, stream)
+        return self.idx
+
+
+class DenseIndexer:
+    def __init__(self, T: int, H: int, L: int, k: int, device="cuda"):
+        self.T, self.H, self.L, self.k = T, H, L, k
+        self.scores_buf = torch.empty((T, _pad4(L)), dtype=torch.float32, device=device)
+        self.scores = self.scores_buf[:, :L]
+        self.idx = torch.empty((T, k), dtype=torch.int32, device=device)
+        self.ws = nat.alloc_workspace(256, device)
+
+    def run(self, q, w, keys, seq_of, prefix_len, stream=None) -> torch.Tensor:
+        nat.index_score(q, w, keys, seq_of, prefix_len, scores=self.scores_buf, workspace=self.ws, stream=stream)
+        nat.topk(self.scores_buf, self.k, n=self.L, row_valid=prefix_len, idx=self.idx, workspace=self.ws,
+                 stream=stream)
+        return self.idx
+
+
+class MisaDaggerIndexer:
+    def __init__(self, T: int, H: int, h: int, L: int, B: int, kp: int, k: int, q_block: int = 1, device="cuda"):
+        self.coarse = MisaIndexer(T, H, h, L, B, kp, q_block, device)
+        self.T, self.H, self.L, self.kp, self.k = T, H, L, kp, k
+        self.idx = torch.empty((T, k), dtype=torch.int32, device=device)
+        self.cand_scores = torch.empty((T, kp), dtype=torch.float32, device=device)
+        self.ws_rerank = nat.alloc_workspace(nat.workspace_bytes(nat.OP_HIER_RERANK, T, H, L, 1, k, kp), device)
+
+    def run(self, q, w, keys, means, seq_of, prefix_len, stream=None, want_scores=False) -> torch.Tensor:
+        cand = self.coarse.run(q, w, keys, means, seq_of, prefix_len, stream)
+        nat.hier_rerank(q, w, keys, seq_of, prefix_len, cand, self.k, idx=self.idx,
+                        cand_scores=self.cand_scores if want_scores else None, workspace=self.ws_rerank,
+                        stream=stream)
+        return self.idx
+
+
+class HisaIndexer:
+    def __init__(self, T: int, H: int, L: int, B: int, m: int, k: int, device="cuda"):
+        self.T, self.H, self.L, self.B, self.m, self.k = T, H, L, B, m, k
+        self.blocks = torch.empty((T, m), dtype=torch.int32, device=device)
+        self.cand = torch.empty((T, m * B), dtype=torch.int32, device=device)
+        self.scores_buf = torch.empty((T, _pad4(m * B)), dtype=torch.float32, device=device)
+        self.scores = self.scores_buf[:, : m * B]
+        self.idx = torch.empty((T, k), dtype=torch.int32, device=device)
+        self.ws_filter = nat.alloc_workspace(nat.workspace_bytes(nat.OP_HISA_BLOCK_FILTER, T, H, L, B, m), device)
+        self.ws = nat.alloc_workspace(256, device)
+
+    def run(self, q, w, keys, means, seq_of, prefix_len, stream=None) -> torch.Tensor:
+        nat.hisa_block_filter(q, w, means, seq_of, prefix_len, self.L, self.B, self.m, blocks=self.blocks,
+                              cand=self.cand, workspace=self.ws_filter, stream=stream)
+        nat.index_score(q, w, keys, seq_of, prefix_len, cand=self.cand, scores=self.scores_buf, workspace=self.ws,
+                        stream=stream)
+        nat.topk(self.scores_buf, self.k, n=self.m * self.B, id_map=self.cand, idx=self.idx, workspace=self.ws,
+                 stream=stream)
+        return self.idx

@@ -1,0 +1,173 @@
+"""Host-side checks of the C ABI (no GPU needed).
+
+* the library loads without a GPU and exports every function include/misa.h
+  declares (and the binding knows each of them);
+* argument validation rejects bad calls with the documented status before
+  anything reaches the CUDA runtime (the pointers below are never touched);
+* workspace sizing follows its documented formula.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_attention_token_misa_b200 as pkg
+from sparse_attention_token_misa_b200 import _native as nat
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "misa.h")
+
+OK, INVALID, UNSUPPORTED, WORKSPACE, CUDA, DEVICE = 0, 1, 2, 3, 4, 5
+
+# fake, 16-byte aligned "device" addresses: validation must fail before use
+P = 1 << 20
+P2 = (1 << 20) + 4096
+MIS = (1 << 20) + 4  # misaligned
+
+
+def declared_functions():
+    text = open(HEADER, encoding="utf-8").read()
+    return re.findall(r"MISA_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    l = pkg.lib()
+    names = declared_functions()
+    assert len(names) == 11, names
+    for n in names:
+        assert hasattr(l, n), n
+        assert n in nat.SIGNATURES, n
+    assert set(nat.SIGNATURES) == set(names)
+    assert l.misa_abi_version() == 1
+
+
+def test_status_strings():
+    for code in range(6):
+        assert nat.status_string(code) != "unknown status"
+    assert nat.status_string(99) == "unknown status"
+
+
+def test_workspace_formula():
+    ws = nat.workspace_bytes
+    # router: 256 + T * ceil(M/32) * H * 4
+    assert ws(nat.OP_ROUTE_HEADS, 32, 64, 32768, 128) == 256 + 32 * 8 * 64 * 4
+    assert ws(nat.OP_ROUTE_HEADS, 3, 5, 100, 7) == 256 + 3 * 1 * 5 * 4
+    assert ws(nat.OP_INDEX_SCORE, 5, 5, 5, 5) == 256
+    assert ws(nat.OP_TOPK, 5, 5, 5, 5) == 256
+    assert ws(nat.OP_HIER_RERANK, 64, 32, 65536, 128, 2048, 8192) == 256 + 64 * 8192 * 4
+    assert ws(nat.OP_HIER_RERANK, 2, 32, 100, 1, 3, 5) == 256 + 2 * 8 * 4
+    assert ws(nat.OP_HISA_BLOCK_FILTER, 16, 64, 131072, 128, 64) == 256 + 16 * 1024 * 4
+    assert ws(nat.OP_HISA_BLOCK_FILTER, 1, 2, 8, 3, 2) == 256 + 1 * 4 * 4
+    assert ws(99, 1, 1, 1, 1) == 0
+    assert ws(nat.OP_ROUTE_HEADS, -1, 1, 1, 1) == 0
+
+
+def topk(scores=P, T=2, n=64, row_stride=64, row_valid=None, id_map=None, id_map_stride=0, k=8, idx=P2,
+         ws=P2 + 4096, ws_bytes=256):
+    return pkg.lib().misa_topk(scores, T, n, row_stride, row_valid, id_map, id_map_stride, k, idx, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(k=0), INVALID),
+    (dict(k=16385), UNSUPPORTED),
+    (dict(T=0), INVALID),
+    (dict(n=0), INVALID),
+    (dict(scores=MIS), INVALID),
+    (dict(row_stride=66), INVALID),
+    (dict(row_stride=60), INVALID),
+    (dict(scores=None), INVALID),
+    (dict(idx=None), INVALID),
+    (dict(id_map=P, id_map_stride=10), INVALID),
+    (dict(ws=None), WORKSPACE),
+    (dict(ws_bytes=255), WORKSPACE),
+])
+def test_topk_rejects(kw, status):
+    assert topk(**kw) == status
+
+
+def score(q=P, w=P, keys=P, nkeyseq=1, stride=0, seq_of=P, plen=P, T=4, H=64, L=1000, heads=P2, h=8, q_block=1,
+          cand=None, n_cand=0, scores=P, row_stride=1000, ws=P2, ws_bytes=256):
+    return pkg.lib().misa_index_score(q, w, keys, nkeyseq, stride, seq_of, plen, T, H, L, heads, h, q_block, cand,
+                                      n_cand, scores, row_stride, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(T=0), INVALID),
+    (dict(H=0), INVALID),
+    (dict(H=129), UNSUPPORTED),
+    (dict(h=0), INVALID),
+    (dict(h=65), INVALID),
+    (dict(q_block=0), INVALID),
+    (dict(L=0), INVALID),
+    (dict(q=MIS), INVALID),
+    (dict(keys=MIS), INVALID),
+    (dict(stride=100, nkeyseq=2), INVALID),
+    (dict(stride=128, nkeyseq=2), INVALID),          # sequences would overlap (stride < L*128)
+    (dict(row_stride=999), INVALID),
+    (dict(cand=P, n_cand=0), INVALID),
+    (dict(cand=P, n_cand=300, row_stride=200), INVALID),
+    (dict(nkeyseq=0), INVALID),
+    (dict(q=None), INVALID),
+    (dict(scores=None), INVALID),
+    (dict(ws=None), WORKSPACE),
+    (dict(ws_bytes=100), WORKSPACE),
+    (dict(nkeyseq=70000, stride=1 << 22, L=32768, row_stride=32768), UNSUPPORTED),  # rows beyond int32 TMA coords
+])
+def test_index_score_rejects(kw, status):
+    assert score(**kw) == status
+
+
+def route(q=P, w=P, means=P, nseq=1, mstride=0, seq_of=P, plen=P, T=4, H=64, L=1024, B=128, q_block=1, h=8,
+          heads=P2, imp=None, ws=P2, ws_bytes=1 << 20):
+    return pkg.lib().misa_route_heads(q, w, means, nseq, mstride, seq_of, plen, T, H, L, B, q_block, h, heads, imp, ws,
+                                      ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(h=0), INVALID),
+    (dict(h=65), INVALID),
+    (dict(q_block=0), INVALID),
+    (dict(B=0), INVALID),
+    (dict(H=200), UNSUPPORTED),
+    (dict(means=MIS), INVALID),
+    (dict(mstride=6, nseq=2), INVALID),
+    (dict(mstride=8 * 128 - 4, nseq=2), INVALID),   # M * 128 = 1024 required
+    (dict(heads=None), INVALID),
+    (dict(ws_bytes=256), WORKSPACE),
+    (dict(ws=None), WORKSPACE),
+])
+def test_route_rejects(kw, status):
+    assert route(**kw) == status
+
+
+def test_block_stats_rejects():
+    f = pkg.lib().misa_block_stats
+    assert f(P, 1, 100, 0, 0, P2, None) == INVALID
+    assert f(P, 1, 100, 0, 5000, P2, None) == UNSUPPORTED
+    assert f(MIS, 1, 100, 0, 4, P2, None) == INVALID
+    assert f(P, 1, 100, 0, 4, MIS, None) == INVALID
+    assert f(P, 2, 100, 4, 4, P2, None) == INVALID        # stride % 8
+    assert f(P, 2, 100, 128, 4, P2, None) == INVALID      # overlapping sequences
+    assert f(None, 1, 100, 0, 4, P2, None) == INVALID
+    assert f(P, 0, 100, 0, 4, P2, None) == INVALID
+
+
+def test_hier_rerank_and_hisa_reject():
+    l = pkg.lib()
+    r = l.misa_hier_rerank
+    # k > kp
+    assert r(P, P, P, 1, 0, P, P, 2, 32, 100, P, 4, 5, None, P2, P2, 1 << 20, None) == INVALID
+    assert r(P, P, P, 1, 0, P, P, 2, 32, 100, None, 4, 2, None, P2, P2, 1 << 20, None) == INVALID
+    assert r(P, P, P, 1, 0, P, P, 2, 32, 100, P, 4, 2, None, P2, P2, 64, None) == WORKSPACE
+    hf = l.hisa_block_filter
+    assert hf(P, P, P, 1, 0, P, P, 2, 64, 1000, 128, 0, P2, P2, None, P2, 1 << 20, None) == INVALID
+    assert hf(P, P, P, 1, 0, P, P, 2, 64, 1000, 128, 20000, P2, P2, None, P2, 1 << 20, None) == UNSUPPORTED
+    assert hf(P, P, P, 1, 0, P, P, 2, 64, 1000, 128, 4, None, P2, None, P2, 1 << 20, None) == INVALID
+    assert hf(P, P, P, 1, 0, P, P, 2, 64, 1000, 128, 4, P2, P2, None, P2, 256, None) == WORKSPACE
+
+
+def test_error_query_rejects_null():
+    bits = ctypes.c_uint32(0)
+    assert pkg.lib().misa_error_query(None, None, ctypes.byref(bits)) == INVALID
+    assert pkg.lib().misa_error_reset(None, None) == INVALID
