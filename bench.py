@@ -137,6 +137,25 @@ def _dist():
     return ws, rank, local
 
 
+def rank_batch(rank: int):
+    """The batch rank `rank` indexes: the bench workload's shape on every rank
+    (weak scaling, no data shared between ranks); rank 0 is the named workload,
+    rank r > 0 the same shape drawn with seed 2 + 1000 r."""
+    if rank == 0:
+        return make_workload(WORKLOAD)
+    from workloads import make_decode
+    return make_decode(WORKLOAD, 2 + 1000 * rank, T=32, L=32768, H=64, h=8, B=128, k=2048, n_planted=16)
+
+
+def reduce_max(x: float, dist, device) -> float:
+    """Max of a per-rank time over all ranks (identity without a process group)."""
+    if not dist:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def _time_steps(step, steps, flush, stream, marks=None):
     """Per-step CUDA-event timing with an untimed L2 flush before every step.
     marks: optional list of names; step(ev) records intermediate events."""
@@ -171,11 +190,7 @@ def run_cuda(args):
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
 
-    wl = make_workload(WORKLOAD)
-    if rank:
-        # every rank gets its own batch of the same shape (different seed)
-        from workloads import make_decode
-        wl = make_decode(WORKLOAD, 2 + 1000 * rank, T=32, L=32768, H=64, h=8, B=128, k=2048, n_planted=16)
+    wl = rank_batch(rank)
     q, w, keys = wl.q.to(dev), wl.w.to(dev), wl.keys.to(dev)
     seq_of, plen = wl.seq_of.to(dev), wl.prefix_len.to(dev)
     T, H, h, L, B, k = wl.T, wl.H, wl.h, wl.L, wl.B, wl.k
@@ -224,11 +239,7 @@ def run_cuda(args):
     dev_err = misa.error_query(ix.ws) | misa.error_query(ix.ws_route)
     if dev_err:
         raise RuntimeError(f"device error word {dev_err:#x}")
-    ms_step = tot_ms / args.steps
-    if dist:
-        t = torch.tensor([ms_step], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step = float(t.item())
+    ms_step = reduce_max(tot_ms / args.steps, dist, dev)
 
     # dense 64-head indexer and block statistics on the same batch (same protocol)
     dense_ms, _ = _time_steps(dense_step, args.steps, flush, stream)
@@ -256,11 +267,7 @@ def run_cuda(args):
         e2e_step([])
     torch.cuda.synchronize()
     e2e_ms, _ = _time_steps(e2e_step, args.steps, flush, stream)
-    e2e_ms /= args.steps
-    if dist:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = reduce_max(e2e_ms / args.steps, dist, dev)
     h2d = q_h.numel() * 2 + w_h.numel() * 4 + so_h.numel() * 4 + pl_h.numel() * 4
     d2h = idx_h.numel() * 4
 
