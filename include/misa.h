@@ -168,6 +168,37 @@ MISA_API misa_status misa_route_heads(const uint16_t* q, const float* w, const f
                              void* workspace, size_t workspace_bytes, misa_stream_t stream);
 
 /*
+ * misa_route_heads_noalloc -- misa_route_heads without a caller workspace.
+ *   The papers have no counterpart to this call; it is a library convenience.
+ * For callers that cannot allocate device memory at the point where they route:
+ * an inference engine that reserved all device memory up front and gives its
+ * plug-ins no allocator, or a serving loop that must not call cudaMalloc /
+ * cudaFree because they can synchronise the whole device.  Inputs, outputs and
+ * results are exactly those of misa_route_heads (same kernels); only the
+ * router's per-chunk partial importances move from the workspace into a fixed
+ * array of MISA_ROUTE_NOALLOC_SCRATCH_BYTES bytes compiled into the library,
+ * which every device that loads the library holds until the process exits.
+ *  - Calls with T * ceil(ceil(L/B) / 32) * H * 4 > MISA_ROUTE_NOALLOC_SCRATCH_BYTES
+ *    are rejected with MISA_ERR_UNSUPPORTED before anything is launched.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - All calls on one device share the array and it keeps the last call's
+ *    contents (nothing in it needs to start at zero).  Calls whose kernels can
+ *    overlap on the GPU (unordered streams) race on it and give wrong results:
+ *    order them on one stream or with events.
+ *  - There is no device error word: an out-of-range seq_of is clamped to 0
+ *    without being reported.
+ *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ */
+#define MISA_ROUTE_NOALLOC_SCRATCH_BYTES (2u << 20)
+MISA_API misa_status misa_route_heads_noalloc(const uint16_t* q, const float* w, const float* means,
+                                              int64_t nseq, int64_t means_seq_stride, const int32_t* seq_of,
+                                              const int32_t* prefix_len, int T, int H, int64_t L, int B,
+                                              int q_block, int h, int32_t* heads, float* importance,
+                                              misa_stream_t stream);
+
+/*
  * misa_index_score -- indexer scores of the active heads (the hot loop).
  *   [MISA page, "Methodology: MISA": only the h active heads score every
  *   prefix token; "Problem statement": the dense DSA indexer scores every prefix

@@ -44,6 +44,8 @@ SIGNATURES = {
     "misa_block_stats": (c_int, [c_vp, c_i64, c_i64, c_i64, c_int, c_vp, c_vp]),
     "misa_route_heads": (c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_i64, c_int,
                                  c_int, c_int, c_vp, c_vp, c_vp, c_size, c_vp]),
+    "misa_route_heads_noalloc": (c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_i64, c_int,
+                                         c_int, c_int, c_vp, c_vp, c_vp]),
     "misa_index_score": (c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_i64, c_vp, c_int,
                                  c_int, c_vp, c_int, c_vp, c_i64, c_vp, c_size, c_vp]),
     "misa_topk": (c_int, [c_vp, c_int, c_i64, c_i64, c_vp, c_vp, c_i64, c_int, c_vp, c_vp, c_size, c_vp]),
@@ -168,6 +170,22 @@ def route_heads(q, w, means, seq_of, prefix_len, L: int, B: int, q_block: int, h
     _call("misa_route_heads", _p(q), _p(w), _p(means), means.shape[0], int(means.stride(0)), _p(seq_of),
           _p(prefix_len), T, H, L, B, q_block, h, _p(heads), _p(importance), _p(workspace),
           workspace.numel(), _stream(stream))
+    return heads, importance
+
+
+def route_heads_noalloc(q, w, means, seq_of, prefix_len, L: int, B: int, q_block: int, h: int,
+                        heads=None, importance=None, want_importance: bool = True, stream=None):
+    """misa_route_heads_noalloc (no workspace; library-owned fixed scratch)."""
+    _req(q, torch.bfloat16, "q"); _req(w, torch.float32, "w"); _req(means, torch.float32, "means")
+    _req(seq_of, torch.int32, "seq_of"); _req(prefix_len, torch.int32, "prefix_len")
+    T, H, _ = q.shape
+    G = (T + q_block - 1) // q_block
+    if heads is None:
+        heads = torch.empty((G, h), dtype=torch.int32, device=q.device)
+    if importance is None and want_importance:
+        importance = torch.empty((G, H), dtype=torch.float32, device=q.device)
+    _call("misa_route_heads_noalloc", _p(q), _p(w), _p(means), means.shape[0], int(means.stride(0)), _p(seq_of),
+          _p(prefix_len), T, H, L, B, q_block, h, _p(heads), _p(importance), _stream(stream))
     return heads, importance
 
 

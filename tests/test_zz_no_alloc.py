@@ -1,0 +1,59 @@
+"""misa_route_heads_noalloc against misa_route_heads, on the GPU.
+
+The no-workspace router exists for callers that cannot allocate device memory
+where they route (an engine that reserved all device memory and gives plug-ins
+no allocator; a serving loop where cudaMalloc / cudaFree, which can
+synchronise the device, are not allowed).  It runs the same kernels with the
+partial importances in a fixed array inside the library, so its heads and
+importances must equal those of the workspace version, call after call: the
+second call below reuses the array the first call left filled, with a
+different shape.  This file is collected last so that a failure here cannot
+stop the rest of the suite from running first.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_attention_token_misa_b200 as misa
+from sparse_attention_token_misa_b200 import _native as nat
+from workloads import make_decode, make_prefill
+
+pytestmark = pytest.mark.gpu
+
+
+def _inputs(wl):
+    dev = torch.device("cuda", 0)
+    q, w, keys = wl.q.to(dev), wl.w.to(dev), wl.keys.to(dev)
+    so, pl = wl.seq_of.to(dev), wl.prefix_len.to(dev)
+    means = misa.block_stats(keys, wl.B)
+    return q, w, means, so, pl
+
+
+@pytest.mark.parametrize("order", ["large_then_small", "small_then_large"])
+def test_noalloc_router_matches_workspace_router(order):
+    a = make_decode("na_a", 41, T=32, L=32768, H=64, h=8, B=128, k=16, n_planted=4)
+    b = make_prefill("na_b", 42, T=70, L=3000, H=32, h=5, B=64, k=16, q_block=16, n_regions=1, region_len=256)
+    cases = [a, b] if order == "large_then_small" else [b, a]
+    for wl in cases:  # two calls in a row through the C ABI; the scratch keeps the previous call's data
+        q, w, means, so, pl = _inputs(wl)
+        ref_heads, ref_imp = misa.route_heads(q, w, means, so, pl, wl.L, wl.B, wl.q_block, wl.h)
+        heads, imp = nat.route_heads_noalloc(q, w, means, so, pl, wl.L, wl.B, wl.q_block, wl.h)
+        torch.cuda.synchronize()
+        assert torch.equal(heads, ref_heads)
+        assert torch.allclose(imp, ref_imp, rtol=1e-6, atol=0.0)
+        # and the routed heads are a valid top-h of the importances (selection rule sanity)
+        imp_np = imp.cpu().numpy()
+        for g in range(heads.shape[0]):
+            exp = np.sort(np.lexsort((np.arange(wl.H), -imp_np[g].astype(np.float64)))[: wl.h])
+            assert np.array_equal(heads[g].cpu().numpy(), exp)
+
+
+def test_noalloc_router_rejects_sizes_beyond_its_scratch():
+    # 4096 queries x 32 chunks x 64 heads x 4 B = 32 MiB > the fixed scratch
+    f = nat.lib().misa_route_heads_noalloc
+    P, P2 = 1 << 20, (1 << 20) + 4096
+    st = f(P, P, P, 1, 0, P, P, 4096, 64, 131072, 128, 64, 8, P2, None, None)
+    assert st == 2  # MISA_ERR_UNSUPPORTED, before any launch
