@@ -204,27 +204,25 @@ def run_cuda(args):
     def flush():
         flush_buf.fill_(1.0)
 
-    def misa_step(evs):
-        ix.route(q, w, means, seq_of, plen)
-        if evs:
-            evs[0].record(stream)
-        ix.score(q, w, keys, seq_of, plen)
-        if evs:
-            evs[1].record(stream)
-        ix.select(plen)
-
-    def dense_step(evs):
-        dense.run(q, w, keys, seq_of, plen)
-
-    def stats_step(evs):
-        misa.block_stats(keys, B, out=means)
-
+    # warm-up (eager), then one CUDA graph per stage of the step
     for _ in range(args.warmup):
-        misa_step([])
-        dense_step([])
+        ix.run(q, w, keys, means, seq_of, plen)
+        dense.run(q, w, keys, seq_of, plen)
+    torch.cuda.synchronize()
+    ix.capture(q, w, keys, means, seq_of, plen)
+    dense.capture(q, w, keys, seq_of, plen)
+    for _ in range(args.warmup):
+        ix.g_route.replay(); ix.g_score.replay(); ix.g_select.replay()
     torch.cuda.synchronize()
     misa.error_reset(ix.ws)
     misa.error_reset(ix.ws_route)
+
+    def misa_step(evs):
+        ix.g_route.replay()
+        evs[0].record(stream)
+        ix.g_score.replay()
+        evs[1].record(stream)
+        ix.g_select.replay()
 
     if dist:
         dist.barrier()
@@ -241,33 +239,46 @@ def run_cuda(args):
         raise RuntimeError(f"device error word {dev_err:#x}")
     ms_step = reduce_max(tot_ms / args.steps, dist, dev)
 
-    # dense 64-head indexer and block statistics on the same batch (same protocol)
-    dense_ms, _ = _time_steps(dense_step, args.steps, flush, stream)
-    stats_ms, _ = _time_steps(stats_step, args.steps, flush, stream)
+    # the same step as one graph, the dense 64-head indexer and the block
+    # statistics on the same batch (same protocol)
+    one_ms, _ = _time_steps(lambda evs: ix.g_step.replay(), args.steps, flush, stream)
+    dense_ms, dparts = _time_steps(lambda evs: (dense.g_score.replay(), evs[0].record(stream),
+                                                dense.g_select.replay()), args.steps, flush, stream,
+                                   marks=["score", "topk"])
+    stats_ms, _ = _time_steps(lambda evs: misa.block_stats(keys, B, out=means), args.steps, flush, stream)
+    one_ms /= args.steps
     dense_ms /= args.steps
     stats_ms /= args.steps
 
-    # e2e through the public API: pinned host inputs -> device, indexer, idx -> host
+    # e2e through the public API: the step's inputs copied from pinned host
+    # memory, the indexer, the indices copied back -- captured as one graph
     q_h = wl.q.pin_memory()
     w_h = wl.w.pin_memory()
     so_h = wl.seq_of.pin_memory()
     pl_h = wl.prefix_len.pin_memory()
     idx_h = torch.empty((T, k), dtype=torch.int32).pin_memory()
     q_d, w_d, so_d, pl_d = torch.empty_like(q), torch.empty_like(w), torch.empty_like(seq_of), torch.empty_like(plen)
+    ix_e = misa.MisaIndexer(T, H, h, L, B, k, q_block=1, device=dev)
 
-    def e2e_step(evs):
+    def e2e_eager():
         q_d.copy_(q_h, non_blocking=True)
         w_d.copy_(w_h, non_blocking=True)
         so_d.copy_(so_h, non_blocking=True)
         pl_d.copy_(pl_h, non_blocking=True)
-        out = ix.run(q_d, w_d, keys, means, so_d, pl_d)
+        out = ix_e.run(q_d, w_d, keys, means, so_d, pl_d)
         idx_h.copy_(out, non_blocking=True)
 
-    for _ in range(2):
-        e2e_step([])
+    from sparse_attention_token_misa_b200.indexer import capture_graph
+    g_e2e = capture_graph(e2e_eager)
+    for _ in range(3):
+        g_e2e.replay()
     torch.cuda.synchronize()
-    e2e_ms, _ = _time_steps(e2e_step, args.steps, flush, stream)
+    e2e_ms, _ = _time_steps(lambda evs: g_e2e.replay(), args.steps, flush, stream)
     e2e_ms = reduce_max(e2e_ms / args.steps, dist, dev)
+    e2e_eager_ms, _ = _time_steps(lambda evs: e2e_eager(), args.steps, flush, stream)
+    e2e_eager_ms /= args.steps
+    if not torch.equal(idx_h.cuda(dev), ix.idx):
+        raise RuntimeError("e2e indices differ from the device-timed step")
     h2d = q_h.numel() * 2 + w_h.numel() * 4 + so_h.numel() * 4 + pl_h.numel() * 4
     d2h = idx_h.numel() * 4
 
@@ -303,14 +314,21 @@ def run_cuda(args):
                    "l2": "flushed before every timed step (256 MiB write, untimed); K is 268 MB > L2"},
         "queries_per_s": T * ws_n / (ms_step * 1e-3),
         "gpu_launches": 4 * args.steps,
+        "timing": "CUDA events on the launching stream around graph replays of the route, score and top-k "
+                  "stages of each step",
         "roofline": {"bound": "hbm", "kernel": "score_kernel (misa_index_score)", "achieved": achieved,
                      "peak": hbm_gbs, "peak_kind": f"{peak_kind} hbm copy GB/s", "unit": "GB/s",
                      "frac": achieved / hbm_gbs, "traffic": traffic,
                      "algorithmic_bytes_per_launch": score_bytes, "launch_ms": score_ms},
         "e2e": {"value": pairs * ws_n / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "how": "pinned host q/w/seq_of/prefix_len -> device, MisaIndexer step, idx -> pinned host; one "
+                       "CUDA graph replay per step",
+                "eager_ms_per_step": e2e_eager_ms},
         "detail": {"route_ms": parts["route"] / args.steps, "score_ms": score_ms, "topk_ms": parts["topk"] / args.steps,
-                   "misa8_ms": ms_step, "dense64_ms": dense_ms, "dense64_over_misa8": dense_ms / ms_step,
+                   "misa8_ms": ms_step, "misa8_one_graph_ms": one_ms,
+                   "dense64_ms": dense_ms, "dense64_score_ms": dparts["score"] / args.steps,
+                   "dense64_topk_ms": dparts["topk"] / args.steps, "dense64_over_misa8": dense_ms / ms_step,
                    "block_stats_ms": stats_ms,
                    "block_stats_GBps": (T * L * 128 * 2 + T * (L // B) * 128 * 4) / (stats_ms * 1e-3) / 1e9,
                    "wall_s_timed_region": wall},
@@ -330,11 +348,14 @@ def other_workloads(misa, dev, stream, flush, steps):
     """The other four workloads through their indexers (same timing protocol)."""
     out = {}
 
+    from sparse_attention_token_misa_b200.indexer import capture_graph
+
     def timed(fn):
+        g = capture_graph(lambda: fn([]))
         for _ in range(3):
-            fn([])
+            g.replay()
         torch.cuda.synchronize()
-        ms, _ = _time_steps(fn, steps, flush, stream)
+        ms, _ = _time_steps(lambda evs: g.replay(), steps, flush, stream)
         return ms / steps
 
     wl = make_workload("prefill_L131072")
@@ -344,17 +365,17 @@ def other_workloads(misa, dev, stream, flush, steps):
     pairs = int(wl.prefix_len.sum())
     parts = {}
 
+    ix.capture(q, w, keys, means, so, pl)
+
     def pf(evs):
-        ix.route(q, w, means, so, pl)
-        if evs:
-            evs[0].record(stream)
-        ix.score(q, w, keys, so, pl)
-        if evs:
-            evs[1].record(stream)
-        ix.select(pl)
+        ix.g_route.replay()
+        evs[0].record(stream)
+        ix.g_score.replay()
+        evs[1].record(stream)
+        ix.g_select.replay()
 
     for _ in range(2):
-        pf([])
+        ix.g_step.replay()
     torch.cuda.synchronize()
     ms, parts = _time_steps(pf, steps, flush, stream, marks=["route", "score", "topk"])
     score_ms = parts["score"] / steps

@@ -40,7 +40,7 @@ EncodeTiledFn encode_tiled() {
   return fn;
 }
 
-// 2-D map over all key rows: dim0 = 128 bf16 (256 B), dim1 = rows; box = 64 x 128
+// 2-D map over all key rows: dim0 = 128 bf16 (256 B), dim1 = rows; box = 64 x kTmaBoxRows
 // with 128-byte swizzle, the layout the UMMA descriptors expect.
 misa_status make_key_map(const uint16_t* keys, int64_t rows, CUtensorMap* map) {
   EncodeTiledFn fn = encode_tiled();
@@ -48,7 +48,7 @@ misa_status make_key_map(const uint16_t* keys, int64_t rows, CUtensorMap* map) {
   std::memset(map, 0, sizeof(*map));
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(MISA_HEAD_DIM), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(MISA_HEAD_DIM) * 2};
-  cuuint32_t box[2] = {64, 128};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(misa::kTmaBoxRows)};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(keys), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,

@@ -9,6 +9,12 @@
 
 namespace misa {
 
+// SM count of the current device (cached; 0 on error).
+int device_sm_count();
+// Raise `func`'s dynamic shared-memory limit to at least `bytes` on the current
+// device; cudaFuncSetAttribute runs only the first time a size is needed.
+cudaError_t ensure_dynamic_smem(const void* func, int bytes);
+
 cudaError_t launch_block_stats(const uint16_t* keys, int64_t nseq, int64_t L, int64_t key_seq_stride, int B,
                                float* means, cudaStream_t stream);
 
@@ -26,6 +32,13 @@ cudaError_t launch_hisa_block_scores(const uint16_t* q, const float* w, const fl
 
 cudaError_t launch_hisa_expand(const int32_t* blocks, const int32_t* prefix_len, int T, int m, int B, int64_t L,
                                int32_t* cand, cudaStream_t stream);
+
+// Rows per TMA box of the key map (a 128-key tile is loaded as 128 / kTmaBoxRows
+// boxes per 64-element K half; the host encodes the map with this box height).
+#ifndef MISA_TMA_BOX_ROWS
+#define MISA_TMA_BOX_ROWS 64
+#endif
+constexpr int kTmaBoxRows = MISA_TMA_BOX_ROWS;
 
 struct ScoreArgs {
   const uint16_t* q;

@@ -260,8 +260,7 @@ cudaError_t launch_route_heads(const uint16_t* q, const float* w, const float* m
   const int M = static_cast<int>((L + B - 1) / B);
   const int nch = router_chunks(M);
   const size_t smem = affinity_smem_bytes(H);
-  cudaError_t e = cudaFuncSetAttribute(affinity_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(affinity_kernel<false>), static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   affinity_kernel<false><<<dim3(T, nch), kThreads, smem, stream>>>(q, w, means, means_seq_stride, seq_of, prefix_len,
                                                                    T, H, L, B, M, q_block, nseq_means, partial,
@@ -282,8 +281,7 @@ cudaError_t launch_hisa_block_scores(const uint16_t* q, const float* w, const fl
   const int M = static_cast<int>((L + B - 1) / B);
   const int nch = router_chunks(M);
   const size_t smem = affinity_smem_bytes(H);
-  cudaError_t e = cudaFuncSetAttribute(affinity_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(affinity_kernel<true>), static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   affinity_kernel<true><<<dim3(T, nch), kThreads, smem, stream>>>(q, w, means, means_seq_stride, seq_of, prefix_len, T,
                                                                   H, L, B, M, 1, nseq_means, nullptr, bscore, bs_stride,

@@ -21,9 +21,10 @@
 // Warp roles (288 threads):
 //   warps 0-3  epilogue (TMEM lane quarter = warp id)
 //   warp  4    TMEM allocation + single-thread MMA issue
-//   warps 5-8  producer: the group's query rows (all 128 threads) and the key
-//              tiles, either by TMA (contiguous keys, one thread) or by a
-//              16-byte cp.async gather of candidate rows (all 128 threads).
+//   warps 5-8  producers.  Contiguous keys: warp 5 (one thread) streams the key
+//              tiles by TMA from the first cycle while warps 6-8 stage the
+//              group's query rows.  Candidate keys: all 128 threads stage the
+//              query rows, then gather candidate rows with 16-byte cp.async.
 // Every mbarrier wait is bounded; a wait that gives up records
 // MISA_DEVERR_TIMEOUT, the role stops, in-flight copies and MMAs are waited for
 // (bounded), TMEM is freed and the kernel returns.
@@ -102,6 +103,33 @@ __device__ __forceinline__ void item_range(int64_t n_items, int64_t& i0, int64_t
   i1 = n_items * (c + 1) / g;
 }
 
+// Stage the query rows of column group g into the B operand (K-major, 128-byte
+// swizzled): column c = ql * HP + i holds q[t][head_i] of query t = g*QPG + ql,
+// or zeros for padding columns.  Threads [0, nthreads) of the caller share it.
+template <int HP, int QPG>
+__device__ __forceinline__ void stage_query_rows(const ScoreParams& p, int g, uint8_t* sQ, int tid, int nthreads) {
+  constexpr int N = HP * QPG;
+  for (int x = tid; x < N * 16; x += nthreads) {
+    const int c = x >> 4, ch = x & 15;
+    const int ql = c / HP, i = c % HP;
+    const int t = g * QPG + ql;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (t < p.T && i < p.h) {
+      int head = i;
+      if (p.heads) {
+        head = p.heads[static_cast<int64_t>(t / p.q_block) * p.h + i];
+        if (head < 0 || head >= p.H) {
+          record_error(p.err, MISA_DEVERR_BAD_HEAD);
+          head = -1;
+        }
+      }
+      if (head >= 0)
+        v = __ldg(reinterpret_cast<const uint4*>(p.q + (static_cast<int64_t>(t) * p.H + head) * kD + ch * 8));
+    }
+    *reinterpret_cast<uint4*>(sQ + sw128_tile_offset(N, c, ch)) = v;
+  }
+}
+
 template <int HP, int QPG, bool kGather>
 __global__ void __launch_bounds__(kThreads, 1)
 score_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreParams p) {
@@ -139,7 +167,7 @@ score_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreParams p) {
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], kEpiThreads);
     }
-    mbar_init(qfull, kProdThreads);
+    mbar_init(qfull, kGather ? kProdThreads : kProdThreads - 32);
     mbar_init(qempty, 1);
     mbar_init(done, 1);
     fence_mbar_init();
@@ -159,61 +187,84 @@ score_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreParams p) {
   const int tpg = p.tiles_per_group;
 
   if (warp >= kProdWarp0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ producers
     const int pt = tid - kProdWarp0 * 32;
-    int64_t it = 0;
-    int groups = 0;
-    int cur_g = -1;
-    bool ok = true;
-    int64_t seq_row0 = 0;
-    int32_t t_gather = 0;
-    int64_t pending_from = 0;  // gather mode: first iteration not yet signalled
-    for (int64_t item = i0; item < i1 && ok; ++item) {
-      const int g = static_cast<int>(item / tpg);
-      const int j = static_cast<int>(item - static_cast<int64_t>(g) * tpg);
-      if (g != cur_g) {
-        if (kGather) {
+    if (!kGather) {
+      if (warp == kProdWarp0) {
+        // one thread streams the key tiles by TMA; it starts at once and never
+        // waits for the query rows
+        if (lane == 0) {
+          const uint64_t policy = l2_evict_first_policy();
+          int64_t it = 0;
+          int cur_g = -1;
+          int64_t seq_row0 = 0;
+          for (int64_t item = i0; item < i1; ++item) {
+            const int g = static_cast<int>(item / tpg);
+            const int j = static_cast<int>(item - static_cast<int64_t>(g) * tpg);
+            if (g != cur_g) {
+              int64_t seq = 0;
+              if (QPG == 1) {
+                seq = p.seq_of[g];
+                if (seq < 0 || seq >= p.nkeyseq) {
+                  record_error(p.err, MISA_DEVERR_BAD_SEQ);
+                  seq = 0;
+                }
+              }
+              seq_row0 = seq * (p.key_seq_stride / kD);
+              cur_g = g;
+            }
+            const int s = static_cast<int>(it % S);
+            const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
+            if (!mbar_wait(&empty[s], ph ^ 1u, p.err)) break;
+            uint8_t* dst = sA + s * kATileBytes;
+            mbar_arrive_expect_tx(&full[s], kATileBytes);
+            const int y = static_cast<int>(seq_row0 + static_cast<int64_t>(j) * kTileM);
+#pragma unroll
+            for (int r0 = 0; r0 < kTileM; r0 += kTmaBoxRows) {
+              tma_load_2d_hint(dst + r0 * 128, &tmap, &full[s], 0, y + r0, policy);
+              tma_load_2d_hint(dst + kATileBytes / 2 + r0 * 128, &tmap, &full[s], 64, y + r0, policy);
+            }
+            ++it;
+          }
+          // make sure no TMA write into shared memory is still in flight
+          const int64_t first = it > S ? it - S : 0;
+          for (int64_t k = first; k < it; ++k) mbar_wait(&full[k % S], static_cast<uint32_t>((k / S) & 1), p.err);
+        }
+      } else {
+        // the other three warps stage each group's query rows
+        const int g0 = static_cast<int>(i0 / tpg);
+        const int g1 = static_cast<int>((i1 - 1) / tpg);
+        for (int g = g0, groups = 0; g <= g1; ++g, ++groups) {
+          if (groups > 0 && !mbar_wait(qempty, (groups - 1) & 1, p.err)) break;
+          stage_query_rows<HP, QPG>(p, g, sQ, pt - 32, kProdThreads - 32);
+          fence_proxy_async_smem();
+          mbar_arrive(qfull);
+        }
+      }
+    } else {
+      // gather mode: all 128 producer threads stage the query rows, then
+      // gather the candidate key rows with 16-byte cp.async
+      int64_t it = 0;
+      int groups = 0;
+      int cur_g = -1;
+      bool ok = true;
+      int64_t seq_row0 = 0;
+      int32_t t_gather = 0;
+      int64_t pending_from = 0;  // first iteration not yet signalled
+      for (int64_t item = i0; item < i1 && ok; ++item) {
+        const int g = static_cast<int>(item / tpg);
+        const int j = static_cast<int>(item - static_cast<int64_t>(g) * tpg);
+        if (g != cur_g) {
           // signal every outstanding stage before waiting on the MMA
           cp_async_wait_group<0>();
           fence_proxy_async_smem();
           for (; pending_from < it; ++pending_from) mbar_arrive(&full[pending_from % S]);
-        }
-        if (groups > 0 && !mbar_wait(qempty, (groups - 1) & 1, p.err)) { ok = false; break; }
-        // stage the group's query rows: column c = ql * HP + i
-        for (int x = pt; x < N * 16; x += kProdThreads) {
-          const int c = x >> 4, ch = x & 15;
-          const int ql = c / HP, i = c % HP;
-          const int t = g * QPG + ql;
-          uint4 v = make_uint4(0u, 0u, 0u, 0u);
-          if (t < p.T && i < p.h) {
-            int head = i;
-            if (p.heads) {
-              head = p.heads[static_cast<int64_t>(t / p.q_block) * p.h + i];
-              if (head < 0 || head >= p.H) {
-                record_error(p.err, MISA_DEVERR_BAD_HEAD);
-                head = -1;
-              }
-            }
-            if (head >= 0)
-              v = __ldg(reinterpret_cast<const uint4*>(p.q + (static_cast<int64_t>(t) * p.H + head) * kD + ch * 8));
-          }
-          *reinterpret_cast<uint4*>(sQ + sw128_tile_offset(N, c, ch)) = v;
-        }
-        fence_proxy_async_smem();
-        mbar_arrive(qfull);
-        ++groups;
-        cur_g = g;
-        if (!kGather) {
-          int64_t seq = 0;
-          if (QPG == 1) {
-            seq = p.seq_of[g];
-            if (seq < 0 || seq >= p.nkeyseq) {
-              if (pt == 0) record_error(p.err, MISA_DEVERR_BAD_SEQ);
-              seq = 0;
-            }
-          }
-          seq_row0 = seq * (p.key_seq_stride / kD);
-        } else {
+          if (groups > 0 && !mbar_wait(qempty, (groups - 1) & 1, p.err)) { ok = false; break; }
+          stage_query_rows<HP, QPG>(p, g, sQ, pt, kProdThreads);
+          fence_proxy_async_smem();
+          mbar_arrive(qfull);
+          ++groups;
+          cur_g = g;
           t_gather = g;
           int64_t seq = p.seq_of[g];
           if (seq < 0 || seq >= p.nkeyseq) {
@@ -222,27 +273,17 @@ score_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreParams p) {
           }
           seq_row0 = seq * (p.key_seq_stride / kD);
         }
-      }
-      const int s = static_cast<int>(it % S);
-      const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
-      if (!mbar_wait(&empty[s], ph ^ 1u, p.err)) { ok = false; break; }
-      uint8_t* dst = sA + s * kATileBytes;
-      if (!kGather) {
-        if (pt == 0) {
-          mbar_arrive_expect_tx(&full[s], kATileBytes);
-          const int y = static_cast<int>(seq_row0 + static_cast<int64_t>(j) * kTileM);
-          tma_load_2d(dst, &tmap, &full[s], 0, y);
-          tma_load_2d(dst + kATileBytes / 2, &tmap, &full[s], 64, y);
-        }
-      } else {
+        const int s = static_cast<int>(it % S);
+        const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
+        if (!mbar_wait(&empty[s], ph ^ 1u, p.err)) { ok = false; break; }
+        uint8_t* dst = sA + s * kATileBytes;
         const int32_t* crow = p.cand + static_cast<int64_t>(t_gather) * p.n_cand;
-        const int64_t limit = p.L;
         for (int x = pt; x < kTileM * 16; x += kProdThreads) {
           const int r = x >> 4, ch = x & 15;
           const int64_t pos = static_cast<int64_t>(j) * kTileM + r;
           int64_t id = -1;
           if (pos < p.n_cand) id = crow[pos];
-          const bool valid = (id >= 0) && (id < limit);
+          const bool valid = (id >= 0) && (id < p.L);
           const uint16_t* src = p.keys + (seq_row0 + (valid ? id : 0)) * kD + ch * 8;
           cp_async_16(dst + sw128_tile_offset(kTileM, r, ch), src, valid);
         }
@@ -254,17 +295,11 @@ score_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreParams p) {
           mbar_arrive(&full[pending_from % S]);
           ++pending_from;
         }
+        ++it;
       }
-      ++it;
-    }
-    if (kGather) {
       cp_async_wait_group<0>();
       fence_proxy_async_smem();
       for (; pending_from < it; ++pending_from) mbar_arrive(&full[pending_from % S]);
-    } else if (pt == 0) {
-      // make sure no TMA write into shared memory is still in flight
-      const int64_t first = it > S ? it - S : 0;
-      for (int64_t k = first; k < it; ++k) mbar_wait(&full[k % S], static_cast<uint32_t>((k / S) & 1), p.err);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issue
@@ -403,7 +438,7 @@ template <int HP, int QPG, bool kGather>
 cudaError_t launch_cfg(const CUtensorMap& tmap, const ScoreParams& p, int num_sms, cudaStream_t stream) {
   using C = Cfg<HP, QPG, kGather>;
   auto kern = score_kernel<HP, QPG, kGather>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), C::kSmemBytes);
   if (e != cudaSuccess) return e;
   int64_t grid = std::min<int64_t>(p.n_items, num_sms);
   if (grid < 1) grid = 1;
@@ -419,12 +454,8 @@ int score_mode_hp(int h_eff, bool shared_groups) {
 }
 
 cudaError_t launch_index_score(const CUtensorMap* tmap, const ScoreArgs& a, cudaStream_t stream) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  int num_sms = 0;
-  e = cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev);
-  if (e != cudaSuccess) return e;
+  const int num_sms = device_sm_count();
+  if (num_sms <= 0) return cudaErrorInvalidDevice;
 
   const int h_eff = a.heads ? a.h : a.H;
   const bool gather = a.cand != nullptr;

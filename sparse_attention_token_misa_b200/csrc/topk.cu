@@ -395,8 +395,7 @@ size_t topk_smem_bytes() { return kSmemFast; }
 
 cudaError_t launch_topk(const float* scores, int T, int64_t n, int64_t row_stride, const int32_t* row_valid,
                         const int32_t* id_map, int64_t id_map_stride, int k, int32_t* idx, cudaStream_t stream) {
-  cudaError_t e =
-      cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kSmemFast));
+  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(topk_kernel), static_cast<int>(kSmemFast));
   if (e != cudaSuccess) return e;
   topk_kernel<<<T, kThreads, kSmemFast, stream>>>(scores, n, row_stride, row_valid, id_map, id_map_stride, k, idx);
   return cudaGetLastError();

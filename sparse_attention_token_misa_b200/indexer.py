@@ -24,7 +24,30 @@ def _pad4(n: int) -> int:
     return (n + 3) // 4 * 4
 
 
+def capture_graph(fn) -> torch.cuda.CUDAGraph:
+    """Capture the library calls `fn` issues into a CUDA graph.
+
+    `fn` runs once eagerly on a side stream first (kernel attributes, TMA maps
+    and modules are set up outside the capture), then once under capture.  The
+    graph replays the same kernels on the same buffers with one launch.
+    """
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fn()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
 class MisaIndexer:
+    """Router + routed token scoring + top-k for one batch shape."""
+
     def __init__(self, T: int, H: int, h: int, L: int, B: int, k: int, q_block: int = 1, device="cuda"):
         self.T, self.H, self.h, self.L, self.B, self.k, self.q_block = T, H, h, L, B, k, q_block
         G = (T + q_block - 1) // q_block
@@ -54,6 +77,14 @@ class MisaIndexer:
         self.select(prefix_len, stream)
         return self.idx
 
+    def capture(self, q, w, keys, means, seq_of, prefix_len):
+        """Graphs of the whole step and of its three stages, on these buffers."""
+        self.g_step = capture_graph(lambda: self.run(q, w, keys, means, seq_of, prefix_len))
+        self.g_route = capture_graph(lambda: self.route(q, w, means, seq_of, prefix_len))
+        self.g_score = capture_graph(lambda: self.score(q, w, keys, seq_of, prefix_len))
+        self.g_select = capture_graph(lambda: self.select(prefix_len))
+        return self
+
 
 class DenseIndexer:
     def __init__(self, T: int, H: int, L: int, k: int, device="cuda"):
@@ -63,11 +94,23 @@ class DenseIndexer:
         self.idx = torch.empty((T, k), dtype=torch.int32, device=device)
         self.ws = nat.alloc_workspace(256, device)
 
-    def run(self, q, w, keys, seq_of, prefix_len, stream=None) -> torch.Tensor:
+    def score(self, q, w, keys, seq_of, prefix_len, stream=None):
         nat.index_score(q, w, keys, seq_of, prefix_len, scores=self.scores_buf, workspace=self.ws, stream=stream)
+
+    def select(self, prefix_len, stream=None):
         nat.topk(self.scores_buf, self.k, n=self.L, row_valid=prefix_len, idx=self.idx, workspace=self.ws,
                  stream=stream)
+
+    def run(self, q, w, keys, seq_of, prefix_len, stream=None) -> torch.Tensor:
+        self.score(q, w, keys, seq_of, prefix_len, stream)
+        self.select(prefix_len, stream)
         return self.idx
+
+    def capture(self, q, w, keys, seq_of, prefix_len):
+        self.g_step = capture_graph(lambda: self.run(q, w, keys, seq_of, prefix_len))
+        self.g_score = capture_graph(lambda: self.score(q, w, keys, seq_of, prefix_len))
+        self.g_select = capture_graph(lambda: self.select(prefix_len))
+        return self
 
 
 class MisaDaggerIndexer:
@@ -84,6 +127,10 @@ class MisaDaggerIndexer:
                         cand_scores=self.cand_scores if want_scores else None, workspace=self.ws_rerank,
                         stream=stream)
         return self.idx
+
+    def capture(self, q, w, keys, means, seq_of, prefix_len):
+        self.g_step = capture_graph(lambda: self.run(q, w, keys, means, seq_of, prefix_len))
+        return self
 
 
 class HisaIndexer:
@@ -105,3 +152,7 @@ class HisaIndexer:
         nat.topk(self.scores_buf, self.k, n=self.m * self.B, id_map=self.cand, idx=self.idx, workspace=self.ws,
                  stream=stream)
         return self.idx
+
+    def capture(self, q, w, keys, means, seq_of, prefix_len):
+        self.g_step = capture_graph(lambda: self.run(q, w, keys, means, seq_of, prefix_len))
+        return self
