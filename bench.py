@@ -344,7 +344,7 @@ def run_cuda(args):
     print(json.dumps(line), flush=True)
 
 
-def other_workloads(misa, dev, stream, flush, steps):
+def other_workloads(misa, dev, stream, flush, steps, only=None):
     """The other four workloads through their indexers (same timing protocol)."""
     out = {}
 
@@ -358,6 +358,17 @@ def other_workloads(misa, dev, stream, flush, steps):
         ms, _ = _time_steps(lambda evs: g.replay(), steps, flush, stream)
         return ms / steps
 
+    if only in (None, "prefill"):
+        out.update(_prefill(misa, dev, stream, flush, steps))
+    if only in (None, "dagger"):
+        out.update(_dagger(misa, dev, stream, flush, steps, timed))
+    if only in (None, "hisa"):
+        out.update(_hisa(misa, dev, stream, flush, steps, timed))
+    return out
+
+
+def _prefill(misa, dev, stream, flush, steps):
+    out = {}
     wl = make_workload("prefill_L131072")
     q, w, keys, so, pl = (x.to(dev) for x in (wl.q, wl.w, wl.keys, wl.seq_of, wl.prefix_len))
     means = misa.block_stats(keys, wl.B)
@@ -386,16 +397,22 @@ def other_workloads(misa, dev, stream, flush, steps):
                               "topk_ms": parts["topk"] / steps,
                               "score_tflops": flops / (score_ms * 1e-3) / 1e12,
                               "score_frac_of_bf16_peak": flops / (score_ms * 1e-3) / 1e12 / tc}
-    del ix, q, w, keys, means
+    return out
 
+
+def _dagger(misa, dev, stream, flush, steps, timed):
+    out = {}
     wl = make_workload("glm5_dagger_decode_L65536")
     q, w, keys, so, pl = (x.to(dev) for x in (wl.q, wl.w, wl.keys, wl.seq_of, wl.prefix_len))
     means = misa.block_stats(keys, wl.B)
     dg = misa.MisaDaggerIndexer(wl.T, wl.H, wl.h, wl.L, wl.B, wl.kp, wl.k, device=dev)
     ms = timed(lambda evs: dg.run(q, w, keys, means, so, pl))
     out["glm5_dagger_decode_L65536"] = {"ms_per_step": ms, "pairs_per_s": int(wl.prefix_len.sum()) / (ms * 1e-3)}
-    del dg, q, w, keys, means
+    return out
 
+
+def _hisa(misa, dev, stream, flush, steps, timed):
+    out = {}
     wl = make_workload("hisa_decode_L131072")
     q, w, keys, so, pl = (x.to(dev) for x in (wl.q, wl.w, wl.keys, wl.seq_of, wl.prefix_len))
     for B, m in ((128, 64), (64, 128)):
@@ -475,11 +492,20 @@ def main():
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     ap.add_argument("--quick", action="store_true", help="skip the other four workloads")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--only", choices=["prefill", "dagger", "hisa"], default=None,
+                    help="time one of the other workloads alone (for profiler captures); prints its own JSON")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.only:
+        import sparse_attention_token_misa_b200 as misa
+        dev = torch.device("cuda", 0)
+        flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+        res = other_workloads(misa, dev, torch.cuda.current_stream(), lambda: flush_buf.fill_(1.0),
+                              max(3, args.steps), only=args.only)
+        print(json.dumps({"only": args.only, "results": res}), flush=True)
     else:
         run_cuda(args)
 

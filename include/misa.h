@@ -77,6 +77,7 @@ extern "C" {
 #define MISA_HEAD_DIM 128
 #define MISA_MAX_HEADS 128     /* H limit */
 #define MISA_MAX_TOPK 16384    /* k (and k') limit of misa_topk */
+#define MISA_MAX_TOPK_ROWS 65535 /* rows (T) limit of the calls that run a top-k */
 #define MISA_ABI_VERSION 1
 
 /* Same object as cudaStream_t (a CUDA runtime stream handle); NULL is the
@@ -178,13 +179,15 @@ MISA_API misa_status misa_route_heads(const uint16_t* q, const float* w, const f
  * router's per-chunk partial importances move from the workspace into a fixed
  * array of MISA_ROUTE_NOALLOC_SCRATCH_BYTES bytes compiled into the library,
  * which every device that loads the library holds until the process exits.
- *  - Calls with T * ceil(ceil(L/B) / 32) * H * 4 > MISA_ROUTE_NOALLOC_SCRATCH_BYTES
- *    are rejected with MISA_ERR_UNSUPPORTED before anything is launched.
+ *  - Calls with T * ceil(ceil(L/B) / 32) * H * 4 (rounded up to 256) +
+ *    4 * ceil(T / q_block) > MISA_ROUTE_NOALLOC_SCRATCH_BYTES are rejected with
+ *    MISA_ERR_UNSUPPORTED before anything is launched.
  *  - The first call on a device looks up the array's device address
  *    (cudaGetSymbolAddress) with that device current; make that first call
  *    before any stream capture.
  *  - All calls on one device share the array and it keeps the last call's
- *    contents (nothing in it needs to start at zero).  Calls whose kernels can
+ *    contents; each call clears the per-decision counters it uses (an
+ *    asynchronous memset on `stream`, no allocation).  Calls whose kernels can
  *    overlap on the GPU (unordered streams) race on it and give wrong results:
  *    order them on one stream or with events.
  *  - There is no device error word: an out-of-range seq_of is clamped to 0
@@ -235,8 +238,8 @@ MISA_API misa_status misa_index_score(const uint16_t* q, const float* w, const u
  * min(n, row_valid[t]) when row_valid != NULL.  idx[t * k + i] receives the
  * selected positions in ascending order (translated through
  * id_map[t * id_map_stride + p] when id_map != NULL), -1 padded.
- * Limits: 1 <= k <= MISA_MAX_TOPK, n >= 1, row_stride % 4 == 0 and >= n,
- *   scores 16-byte aligned.
+ * Limits: 1 <= k <= MISA_MAX_TOPK, 1 <= T <= MISA_MAX_TOPK_ROWS, 1 <= n < 2^31,
+ *   row_stride % 4 == 0 and >= n, scores 16-byte aligned.
  * workspace: >= 256 bytes.
  */
 MISA_API misa_status misa_topk(const float* scores, int T, int64_t n, int64_t row_stride,

@@ -91,7 +91,7 @@ misa_status check_topk_args(const float* scores, int T, int64_t n, int64_t row_s
                             int64_t id_map_stride, int k, const int32_t* idx) {
   if (!scores || !idx) return MISA_ERR_INVALID_ARG;
   if (T < 1 || n < 1 || k < 1) return MISA_ERR_INVALID_ARG;
-  if (k > MISA_MAX_TOPK) return MISA_ERR_UNSUPPORTED;
+  if (k > MISA_MAX_TOPK || T > MISA_MAX_TOPK_ROWS) return MISA_ERR_UNSUPPORTED;
   if (n >= (static_cast<int64_t>(1) << 31)) return MISA_ERR_UNSUPPORTED;
   if (row_stride < n || row_stride % 4 != 0 || !aligned16(scores)) return MISA_ERR_INVALID_ARG;
   if (id_map && id_map_stride < n) return MISA_ERR_INVALID_ARG;
@@ -134,12 +134,10 @@ size_t misa_workspace_bytes(int op, int T, int H, int64_t L, int B, int k, int k
   (void)k;
   if (T < 0 || H < 0 || L < 0 || B < 0 || kp < 0) return 0;
   switch (op) {
-    case MISA_OP_ROUTE_HEADS: {
+    case MISA_OP_ROUTE_HEADS:
+      // sized for q_block = 1 (the most routing decisions a call can have)
       if (B < 1) return 0;
-      const int64_t M = ceil_div(L, B);
-      const int64_t nch = misa::router_chunks(static_cast<int>(M));
-      return kErrBytes + static_cast<size_t>(T) * nch * H * sizeof(float);
-    }
+      return kErrBytes + misa::router_scratch_bytes(T, H, L, B, 1);
     case MISA_OP_INDEX_SCORE:
     case MISA_OP_TOPK:
       return kErrBytes;
@@ -191,9 +189,11 @@ misa_status misa_route_heads(const uint16_t* q, const float* w, const float* mea
   if (!heads || q_block < 1 || h < 1 || h > H) return MISA_ERR_INVALID_ARG;
   st = check_ws(workspace, workspace_bytes, misa_workspace_bytes(MISA_OP_ROUTE_HEADS, T, H, L, B, 0, 0));
   if (st != MISA_OK) return st;
-  float* partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kErrBytes);
+  uint8_t* scratch = static_cast<uint8_t*>(workspace) + kErrBytes;
+  float* partial = reinterpret_cast<float*>(scratch);
+  unsigned* counters = reinterpret_cast<unsigned*>(scratch + misa::router_counters_offset(T, H, L, B));
   return cuda_status(misa::launch_route_heads(q, w, means, means_seq_stride, seq_of, prefix_len, T, H, L, B, q_block,
-                                              h, static_cast<int>(nseq), heads, importance, partial,
+                                              h, static_cast<int>(nseq), heads, importance, partial, counters,
                                               err_word(workspace), reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -253,7 +253,7 @@ misa_status misa_hier_rerank(const uint16_t* q, const float* w, const uint16_t* 
                              int64_t L, const int32_t* cand, int kp, int k, float* cand_scores, int32_t* idx,
                              void* workspace, size_t workspace_bytes, misa_stream_t stream) {
   if (!cand || !idx || kp < 1 || k < 1 || k > kp || T < 1) return MISA_ERR_INVALID_ARG;
-  if (k > MISA_MAX_TOPK) return MISA_ERR_UNSUPPORTED;
+  if (k > MISA_MAX_TOPK || T > MISA_MAX_TOPK_ROWS) return MISA_ERR_UNSUPPORTED;
   misa_status st = check_ws(workspace, workspace_bytes, misa_workspace_bytes(MISA_OP_HIER_RERANK, T, H, L, 1, k, kp));
   if (st != MISA_OK) return st;
   const int64_t kp_pad = round_up4(kp);
@@ -301,7 +301,7 @@ misa_status hisa_block_filter(const uint16_t* q, const float* w, const float* me
   misa_status st = check_block_args(q, w, means, nseq, means_seq_stride, seq_of, prefix_len, T, H, L, B);
   if (st != MISA_OK) return st;
   if (!blocks || !cand || m < 1) return MISA_ERR_INVALID_ARG;
-  if (m > MISA_MAX_TOPK) return MISA_ERR_UNSUPPORTED;
+  if (m > MISA_MAX_TOPK || T > MISA_MAX_TOPK_ROWS) return MISA_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(m) * B >= (static_cast<int64_t>(1) << 31)) return MISA_ERR_UNSUPPORTED;
   st = check_ws(workspace, workspace_bytes, misa_workspace_bytes(MISA_OP_HISA_BLOCK_FILTER, T, H, L, B, m, 0));
   if (st != MISA_OK) return st;

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <map>
+#include <tuple>
 #include <mutex>
 #include <utility>
 
@@ -41,6 +42,20 @@ cudaError_t ensure_dynamic_smem(const void* func, int bytes) {
   e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e == cudaSuccess) g_smem[key] = bytes;
   return e;
+}
+
+int occupancy_blocks(const void* func, int threads, size_t smem) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+  static std::map<std::tuple<int, const void*, int, size_t>, int> cache;
+  std::lock_guard<std::mutex> lock(g_mu);
+  auto key = std::make_tuple(dev, func, threads, smem);
+  auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, func, threads, smem) != cudaSuccess || n < 1) n = 1;
+  cache[key] = n;
+  return n;
 }
 
 }  // namespace misa

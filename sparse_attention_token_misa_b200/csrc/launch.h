@@ -14,6 +14,9 @@ int device_sm_count();
 // Raise `func`'s dynamic shared-memory limit to at least `bytes` on the current
 // device; cudaFuncSetAttribute runs only the first time a size is needed.
 cudaError_t ensure_dynamic_smem(const void* func, int bytes);
+// Resident CTAs per SM of `func` at this block size and dynamic shared memory
+// (cached; 1 if the query fails).
+int occupancy_blocks(const void* func, int threads, size_t smem);
 
 cudaError_t launch_block_stats(const uint16_t* keys, int64_t nseq, int64_t L, int64_t key_seq_stride, int B,
                                float* means, cudaStream_t stream);
@@ -23,7 +26,12 @@ int router_chunks(int M);
 cudaError_t launch_route_heads(const uint16_t* q, const float* w, const float* means, int64_t means_seq_stride,
                                const int32_t* seq_of, const int32_t* prefix_len, int T, int H, int64_t L, int B,
                                int q_block, int h, int nseq_means, int32_t* heads, float* importance, float* partial,
-                               uint32_t* err, cudaStream_t stream);
+                               unsigned* counters, uint32_t* err, cudaStream_t stream);
+
+// Bytes of router scratch: partial importances [T][ceil(M/32)][H] fp32 followed
+// (at a 256-byte boundary) by one counter per routing decision.
+size_t router_scratch_bytes(int T, int H, int64_t L, int B, int q_block);
+size_t router_counters_offset(int T, int H, int64_t L, int B);
 
 cudaError_t launch_hisa_block_scores(const uint16_t* q, const float* w, const float* means, int64_t means_seq_stride,
                                      const int32_t* seq_of, const int32_t* prefix_len, int T, int H, int64_t L, int B,

@@ -17,8 +17,9 @@
 
 namespace {
 
-// Scratch for the partial head importances, [T][ceil(M/32)][H] fp32.  Every
-// device that loads the library holds these bytes until the process exits.
+// Scratch for the partial head importances, [T][ceil(M/32)][H] fp32, and one
+// counter per routing decision.  Every device that loads the library holds
+// these bytes until the process exits.
 constexpr size_t kScratchBytes = MISA_ROUTE_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_route_scratch[kScratchBytes];
 
@@ -63,18 +64,21 @@ misa_status misa_route_heads_noalloc(const uint16_t* q, const float* w, const fl
   const int64_t M = (L + B - 1) / B;
   if (nseq > 1 && means_seq_stride < M * MISA_HEAD_DIM) return MISA_ERR_INVALID_ARG;
   if (M >= (static_cast<int64_t>(1) << 24) || nseq >= (static_cast<int64_t>(1) << 31)) return MISA_ERR_UNSUPPORTED;
-  // The partial importances must fit in the fixed scratch array.
-  const int64_t need = static_cast<int64_t>(T) * misa::router_chunks(static_cast<int>(M)) * H * 4;
-  if (need > static_cast<int64_t>(kScratchBytes)) return MISA_ERR_UNSUPPORTED;
+  // The partial importances and the per-decision counters must fit in the
+  // fixed scratch array.
+  if (misa::router_scratch_bytes(T, H, L, B, q_block) > kScratchBytes) return MISA_ERR_UNSUPPORTED;
 
   float* partial = nullptr;
   misa_status st = scratch_on_current_device(&partial);
   if (st != MISA_OK) return st;
-  // Every entry of the scratch that the select step reads is written first by
-  // the affinity step of this call, so nothing needs clearing; device-side
-  // index checks clamp a bad seq_of without reporting it (no error word).
+  unsigned* counters = reinterpret_cast<unsigned*>(reinterpret_cast<uint8_t*>(partial) +
+                                                   misa::router_counters_offset(T, H, L, B));
+  // The launcher clears the counters (the only part that must start at zero)
+  // on the stream before the kernel; the partials are written before they are
+  // read.  Device-side index checks clamp a bad seq_of without reporting it
+  // (there is no error word).
   cudaError_t e = misa::launch_route_heads(q, w, means, means_seq_stride, seq_of, prefix_len, T, H, L, B, q_block, h,
-                                           static_cast<int>(nseq), heads, importance, partial, nullptr,
+                                           static_cast<int>(nseq), heads, importance, partial, counters, nullptr,
                                            reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MISA_OK : MISA_ERR_CUDA;
 }

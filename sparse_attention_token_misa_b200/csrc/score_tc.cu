@@ -18,10 +18,12 @@
 // multiplies by the head weight and sums the heads of each query in ascending
 // head order, and writes fp32 scores (coalesced, -inf past the prefix).
 //
-// Warp roles (288 threads):
-//   warps 0-3  epilogue (TMEM lane quarter = warp id)
-//   warp  4    TMEM allocation + single-thread MMA issue
-//   warps 5-8  producers.  Contiguous keys: warp 5 (one thread) streams the key
+// Warp roles (EW epilogue warps per TMEM lane quarter: 1 when a group is one
+// query, 4 when 32 queries share a tile of N = 256 columns):
+//   warps 0 .. 4EW-1   epilogue (warp w reads TMEM lane quarter w % 4 and
+//                      owns columns [(w / 4) N / EW, (w / 4 + 1) N / EW))
+//   warp  4EW          TMEM allocation + single-thread MMA issue
+//   warps 4EW+1 .. +4  producers.  Contiguous keys: warp 5 (one thread) streams the key
 //              tiles by TMA from the first cycle while warps 6-8 stage the
 //              group's query rows.  Candidate keys: all 128 threads stage the
 //              query rows, then gather candidate rows with 16-byte cp.async.
@@ -40,12 +42,20 @@ namespace {
 
 constexpr int kTileM = 128;                      // keys per tile (MMA M)
 constexpr int kATileBytes = kTileM * kD * 2;     // 32 KB
-constexpr int kThreads = 288;
-constexpr int kEpiThreads = 128;
 constexpr int kProdThreads = 128;
-constexpr int kProdWarp0 = 5;
-constexpr int kMmaWarp = 4;
-constexpr int kGatherLag = 2;                    // cp.async groups left in flight per producer thread
+constexpr int kGatherLag = 2;
+#ifndef MISA_SHARED_EPI_WARPS
+#define MISA_SHARED_EPI_WARPS 4
+#endif
+constexpr int kSharedEW = MISA_SHARED_EPI_WARPS;  // epilogue warps per lane quarter, shared-cache groups
+#ifndef MISA_DECODE_CTAS
+#define MISA_DECODE_CTAS 2
+#endif
+#ifndef MISA_DECODE_STAGES
+#define MISA_DECODE_STAGES 3
+#endif
+constexpr int kDecodeCtas = MISA_DECODE_CTAS;
+constexpr int kDecodeStages = MISA_DECODE_STAGES;                    // cp.async groups left in flight per producer thread
 
 struct ScoreParams {
   const uint16_t* q;
@@ -77,11 +87,23 @@ __host__ __device__ constexpr int pow2_at_least(int x, int lo) {
   return p;
 }
 
-template <int HP, int QPG, bool kGather>
+template <int HP, int QPG, int EW, bool kGather>
 struct Cfg {
   static constexpr int N = HP * QPG;
   static_assert(N % 16 == 0 && N >= 16 && N <= 256, "MMA N must be a multiple of 16 in [16, 256]");
-  static constexpr int kStages = N >= 256 ? 4 : (N >= 128 ? 5 : 6);
+  // EW epilogue warps per TMEM lane quarter, each owning N / EW columns (whole queries)
+  static_assert((N / EW) % HP == 0, "an epilogue warp must own whole queries");
+  static constexpr int kEpiWarps = 4 * EW;
+  static constexpr int kEpiThreads = 32 * kEpiWarps;
+  static constexpr int kMmaWarp = kEpiWarps;
+  static constexpr int kProdWarp0 = kEpiWarps + 1;
+  static constexpr int kThreads = 32 * (kEpiWarps + 1 + kProdThreads / 32);
+  static constexpr int kColsPerWarp = N / EW;
+  // a CTA per query group streams its own key cache: kDecodeCtas CTAs per SM
+  // with kDecodeStages 32 KB stages each; shared-cache groups: one CTA per SM
+  static constexpr bool kPerQuery = (QPG == 1) && !kGather;
+  static constexpr int kCtasPerSm = kPerQuery ? kDecodeCtas : 1;
+  static constexpr int kStages = kPerQuery ? kDecodeStages : (N >= 256 ? 4 : (N >= 128 ? 5 : 6));
   static constexpr int kQBytes = N * kD * 2;
   static constexpr int kTmemCols = pow2_at_least(2 * N, 32);
   static constexpr uint32_t kIdesc = idesc_bf16_f32(kTileM, N);
@@ -93,7 +115,7 @@ struct Cfg {
   static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
   static constexpr int kOffW = (kOffTmemSlot + 4 + 15) / 16 * 16;
   static constexpr int kOffPlen = kOffW + N * 4;
-  static constexpr int kOffRow = kOffPlen + QPG * 8;
+  static constexpr int kOffRow = kOffPlen + (QPG * 4 + 7) / 8 * 8;
   static constexpr int kSmemBytes = kOffRow + QPG * 8 + 1024;  // + alignment slack
 };
 
@@ -130,10 +152,13 @@ __device__ __forceinline__ void stage_query_rows(const ScoreParams& p, int g, ui
   }
 }
 
-template <int HP, int QPG, bool kGather>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int HP, int QPG, int EW, bool kGather>
+__global__ void __launch_bounds__(Cfg<HP, QPG, EW, kGather>::kThreads, Cfg<HP, QPG, EW, kGather>::kCtasPerSm)
 score_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreParams p) {
-  using C = Cfg<HP, QPG, kGather>;
+  using C = Cfg<HP, QPG, EW, kGather>;
+  constexpr int kEpiThreads = C::kEpiThreads;
+  constexpr int kMmaWarp = C::kMmaWarp;
+  constexpr int kProdWarp0 = C::kProdWarp0;
   constexpr int N = C::N;
   constexpr int S = C::kStages;
 
@@ -151,8 +176,8 @@ score_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreParams p) {
   uint64_t* done = bars + 2 * S + 6;    // all MMAs of this CTA finished
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffTmemSlot);
   float* w_s = reinterpret_cast<float*>(smem + C::kOffW);
-  int64_t* plen_s = reinterpret_cast<int64_t*>(smem + C::kOffPlen);
-  int64_t* row_s = reinterpret_cast<int64_t*>(smem + C::kOffRow);
+  int32_t* plen_s = reinterpret_cast<int32_t*>(smem + C::kOffPlen);   // visible keys of each group query
+  float** rowp_s = reinterpret_cast<float**>(smem + C::kOffRow);       // its score row (NULL past T)
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -194,7 +219,9 @@ score_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreParams p) {
         // one thread streams the key tiles by TMA; it starts at once and never
         // waits for the query rows
         if (lane == 0) {
-          const uint64_t policy = l2_evict_first_policy();
+          // a per-query cache is streamed once (evict first); a shared cache is
+          // read by every column group (keep it in L2)
+          const uint64_t policy = QPG == 1 ? l2_evict_first_policy() : l2_evict_last_policy();
           int64_t it = 0;
           int cur_g = -1;
           int64_t seq_row0 = 0;
@@ -342,8 +369,13 @@ score_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreParams p) {
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    const int r = warp * 32 + lane;  // TMEM lane = key row of the tile
-    const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+    const int quarter = warp & 3;          // TMEM lane quarter this warp may read
+    const int cslice = warp >> 2;          // which N / EW columns it owns
+    constexpr int NW = C::kColsPerWarp;
+    const int col0 = cslice * NW;
+    const int ql0 = col0 / HP;
+    const int r = quarter * 32 + lane;     // TMEM lane = key row of the tile
+    const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
     int64_t it = 0;
     int cur_g = -1;
     for (int64_t item = i0; item < i1; ++item) {
@@ -370,8 +402,8 @@ score_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreParams p) {
             if (pl > p.L) pl = p.L;
             if (pl < 0) pl = 0;
           }
-          plen_s[ql] = pl;
-          row_s[ql] = (t < p.T) ? static_cast<int64_t>(t) * p.row_stride : -1;
+          plen_s[ql] = static_cast<int32_t>(pl);
+          rowp_s[ql] = (t < p.T) ? p.scores + static_cast<int64_t>(t) * p.row_stride : nullptr;
         }
         named_bar_sync(1, kEpiThreads);
         cur_g = g;
@@ -382,9 +414,9 @@ score_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreParams p) {
       tc_fence_after();
 
       // which output slot this lane's key row maps to, and whether it is visible
-      int64_t pos = static_cast<int64_t>(j) * kTileM + r;  // column of the score row
+      const int pos = j * kTileM + r;  // column of the score row (< 2^31)
       bool in_row;
-      int64_t key_id;
+      int key_id;
       if (kGather) {
         in_row = pos < p.n_cand;
         key_id = in_row ? p.cand[static_cast<int64_t>(g) * p.n_cand + pos] : -1;
@@ -393,33 +425,38 @@ score_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreParams p) {
         key_id = pos;
       }
 
-      constexpr int kBatch = N < 64 ? N : 64;
-      const uint32_t t_acc = t_lane + static_cast<uint32_t>(a * N);
+      constexpr int kBatch = EW == 1 ? (NW < 64 ? NW : 64) : (NW < 32 ? NW : 32);
+      const uint32_t t_acc = t_lane + static_cast<uint32_t>(a * N + col0);
+      const float* wcol = w_s + col0;
       float sacc = 0.f;
 #pragma unroll
-      for (int c0 = 0; c0 < N; c0 += kBatch) {
+      for (int c0 = 0; c0 < NW; c0 += kBatch) {
         uint32_t v[kBatch];
 #pragma unroll
         for (int u = 0; u < kBatch / 16; ++u)
           tmem_ld16(t_acc + static_cast<uint32_t>(c0 + 16 * u), v + 16 * u);
         tmem_wait_ld();
-        if (c0 + kBatch == N) {
-          // accumulator fully read: hand it back to the MMA warp
+        if (c0 + kBatch == NW) {
+          // this warp's part of the accumulator is read: hand it back
           tc_fence_before();
           mbar_arrive(&tempty[a]);
         }
 #pragma unroll
         for (int jj = 0; jj < kBatch; ++jj) {
-          const int col = c0 + jj;
-          const int ql = col / HP;
+          const int col = c0 + jj;  // within this warp's columns
           const int i = col % HP;
           if (i == 0) sacc = 0.f;
-          sacc = fmaf(w_s[col], fmaxf(__uint_as_float(v[jj]), 0.f), sacc);
+          sacc = fmaf(wcol[col], fmaxf(__uint_as_float(v[jj]), 0.f), sacc);
           if (i == HP - 1) {
-            const int64_t rb = row_s[ql];
-            if (rb >= 0 && in_row) {
-              const bool vis = (key_id >= 0) && (key_id < plen_s[ql]);
-              p.scores[rb + pos] = vis ? sacc : -__int_as_float(0x7f800000);
+            const int ql = ql0 + col / HP;
+            float* rp = rowp_s[ql];
+            if (rp != nullptr && in_row) {
+              // visible iff 0 <= key_id < prefix (one unsigned compare)
+              const float val = static_cast<uint32_t>(key_id) < static_cast<uint32_t>(plen_s[ql])
+                                    ? sacc
+                                    : -__int_as_float(0x7f800000);
+              if (QPG == 1) rp[pos] = val;     // re-read soon by the top-k: keep in L2
+              else __stcs(rp + pos, val);      // large score matrix: stream past L2
             }
           }
         }
@@ -434,15 +471,16 @@ score_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreParams p) {
   if (warp == kMmaWarp) tmem_dealloc(tmem_base, C::kTmemCols);
 }
 
-template <int HP, int QPG, bool kGather>
+template <int HP, int QPG, int EW, bool kGather>
 cudaError_t launch_cfg(const CUtensorMap& tmap, const ScoreParams& p, int num_sms, cudaStream_t stream) {
-  using C = Cfg<HP, QPG, kGather>;
-  auto kern = score_kernel<HP, QPG, kGather>;
+  using C = Cfg<HP, QPG, EW, kGather>;
+  auto kern = score_kernel<HP, QPG, EW, kGather>;
   cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), C::kSmemBytes);
   if (e != cudaSuccess) return e;
-  int64_t grid = std::min<int64_t>(p.n_items, num_sms);
+  const int per_sm = occupancy_blocks(reinterpret_cast<const void*>(kern), C::kThreads, C::kSmemBytes);
+  int64_t grid = std::min<int64_t>(p.n_items, static_cast<int64_t>(num_sms) * std::max(1, std::min(per_sm, C::kCtasPerSm)));
   if (grid < 1) grid = 1;
-  kern<<<static_cast<unsigned>(grid), kThreads, C::kSmemBytes, stream>>>(tmap, p);
+  kern<<<static_cast<unsigned>(grid), C::kThreads, C::kSmemBytes, stream>>>(tmap, p);
   return cudaGetLastError();
 }
 
@@ -498,31 +536,31 @@ cudaError_t launch_index_score(const CUtensorMap* tmap, const ScoreArgs& a, cuda
 
   if (gather) {
     switch (hp) {
-      case 16: return launch_cfg<16, 1, true>(tm, p, num_sms, stream);
-      case 32: return launch_cfg<32, 1, true>(tm, p, num_sms, stream);
-      case 64: return launch_cfg<64, 1, true>(tm, p, num_sms, stream);
-      case 128: return launch_cfg<128, 1, true>(tm, p, num_sms, stream);
+      case 16: return launch_cfg<16, 1, 1, true>(tm, p, num_sms, stream);
+      case 32: return launch_cfg<32, 1, 1, true>(tm, p, num_sms, stream);
+      case 64: return launch_cfg<64, 1, 1, true>(tm, p, num_sms, stream);
+      case 128: return launch_cfg<128, 1, 1, true>(tm, p, num_sms, stream);
       default: return cudaErrorInvalidValue;
     }
   }
   if (!shared_groups) {
     switch (hp) {
-      case 16: return launch_cfg<16, 1, false>(tm, p, num_sms, stream);
-      case 32: return launch_cfg<32, 1, false>(tm, p, num_sms, stream);
-      case 64: return launch_cfg<64, 1, false>(tm, p, num_sms, stream);
-      case 128: return launch_cfg<128, 1, false>(tm, p, num_sms, stream);
+      case 16: return launch_cfg<16, 1, 1, false>(tm, p, num_sms, stream);
+      case 32: return launch_cfg<32, 1, 1, false>(tm, p, num_sms, stream);
+      case 64: return launch_cfg<64, 1, 1, false>(tm, p, num_sms, stream);
+      case 128: return launch_cfg<128, 1, 1, false>(tm, p, num_sms, stream);
       default: return cudaErrorInvalidValue;
     }
   }
   switch (hp) {
-    case 1: return launch_cfg<1, 256, false>(tm, p, num_sms, stream);
-    case 2: return launch_cfg<2, 128, false>(tm, p, num_sms, stream);
-    case 4: return launch_cfg<4, 64, false>(tm, p, num_sms, stream);
-    case 8: return launch_cfg<8, 32, false>(tm, p, num_sms, stream);
-    case 16: return launch_cfg<16, 16, false>(tm, p, num_sms, stream);
-    case 32: return launch_cfg<32, 8, false>(tm, p, num_sms, stream);
-    case 64: return launch_cfg<64, 4, false>(tm, p, num_sms, stream);
-    case 128: return launch_cfg<128, 2, false>(tm, p, num_sms, stream);
+    case 1: return launch_cfg<1, 256, kSharedEW, false>(tm, p, num_sms, stream);
+    case 2: return launch_cfg<2, 128, kSharedEW, false>(tm, p, num_sms, stream);
+    case 4: return launch_cfg<4, 64, kSharedEW, false>(tm, p, num_sms, stream);
+    case 8: return launch_cfg<8, 32, kSharedEW, false>(tm, p, num_sms, stream);
+    case 16: return launch_cfg<16, 16, kSharedEW, false>(tm, p, num_sms, stream);
+    case 32: return launch_cfg<32, 8, kSharedEW, false>(tm, p, num_sms, stream);
+    case 64: return launch_cfg<64, 4, kSharedEW, false>(tm, p, num_sms, stream);
+    case 128: return launch_cfg<128, 2, 2, false>(tm, p, num_sms, stream);
     default: return cudaErrorInvalidValue;
   }
 }

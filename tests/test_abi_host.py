@@ -50,9 +50,9 @@ def test_status_strings():
 
 def test_workspace_formula():
     ws = nat.workspace_bytes
-    # router: 256 + T * ceil(M/32) * H * 4
-    assert ws(nat.OP_ROUTE_HEADS, 32, 64, 32768, 128) == 256 + 32 * 8 * 64 * 4
-    assert ws(nat.OP_ROUTE_HEADS, 3, 5, 100, 7) == 256 + 3 * 1 * 5 * 4
+    # router: 256 + (T * ceil(M/32) * H * 4 rounded up to 256) + 4 * T
+    assert ws(nat.OP_ROUTE_HEADS, 32, 64, 32768, 128) == 256 + 32 * 8 * 64 * 4 + 4 * 32
+    assert ws(nat.OP_ROUTE_HEADS, 3, 5, 100, 7) == 256 + 256 + 4 * 3
     assert ws(nat.OP_INDEX_SCORE, 5, 5, 5, 5) == 256
     assert ws(nat.OP_TOPK, 5, 5, 5, 5) == 256
     assert ws(nat.OP_HIER_RERANK, 64, 32, 65536, 128, 2048, 8192) == 256 + 64 * 8192 * 4

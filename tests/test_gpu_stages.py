@@ -46,6 +46,10 @@ def test_block_stats(nseq, L, B):
     (2, 9000, 16384, 0.0, 0.2, 0.0),      # fewer valid entries than k (padding)
     (3, 7, 3, 0.5, 0.3, 0.3),             # tiny row
     (2, 20000, 1, 0.5, 0.0, 0.5),
+    (2, 300000, 2048, 0.0, 0.0, 0.0),     # slices too long for shared memory (keys re-read from global)
+    (3, 16385, 100, 0.2, 0.1, 0.1),       # 8-CTA cluster, last slice nearly empty
+    (4, 4097, 50, 0.3, 0.0, 0.2),         # 2-CTA cluster
+    (65, 1024, 64, 0.1, 0.0, 0.0),        # single-CTA clusters, many rows
 ])
 def test_topk_exact(T, n, k, ties, neg_inf, zeros):
     s = random_scores(1000 + n + k, T, n, tie_frac=ties, neg_inf_frac=neg_inf, zero_frac=zeros)
