@@ -49,10 +49,34 @@ def test_block_stats(nseq, L, B):
     (2, 300000, 2048, 0.0, 0.0, 0.0),     # slices too long for shared memory (keys re-read from global)
     (3, 16385, 100, 0.2, 0.1, 0.1),       # 8-CTA cluster, last slice nearly empty
     (4, 4097, 50, 0.3, 0.0, 0.2),         # 2-CTA cluster
-    (65, 1024, 64, 0.1, 0.0, 0.0),        # single-CTA clusters, many rows
+    (65, 1024, 64, 0.1, 0.0, 0.0),        # many short rows
+    (3, 30000, 100, 0.9, 0.0, 0.0),       # one-CTA rows: threshold bin beyond the candidate capacity
+    (2, 12000, 700, 0.35, 0.0, 0.0),      # heavy ties inside the threshold bin
+    (2, 5000, 100, 0.0, 0.0, 1.0),        # every entry +-0: one value range, select by position
+    (2, 3000, 10, 0.0, 0.0, 1.0),         # same, candidates fit (radix over the candidates)
+    (2, 40960, 2048, 0.0, 0.0, 0.0),      # largest one-CTA row
+    (2, 40961, 2048, 0.0, 0.0, 0.0),      # smallest cluster row
 ])
 def test_topk_exact(T, n, k, ties, neg_inf, zeros):
-    s = random_scores(1000 + n + k, T, n, tie_frac=ties, neg_inf_frac=neg_inf, zero_frac=zeros)
+    _check_topk(random_scores(1000 + n + k, T, n, tie_frac=ties, neg_inf_frac=neg_inf, zero_frac=zeros), n, k)
+
+
+def test_topk_unusual_rows():
+    """Rows whose first entries are all masked, +-inf entries, a single huge
+    outlier that squeezes every other value into one bin."""
+    n = 20000
+    s = random_scores(5, 4, n)
+    s[0, :8000] = float("-inf")
+    s[1, 100] = float("inf")
+    s[1, 5000] = float("-inf")
+    s[2, 7] = 1e30
+    s[3, :] = torch.linspace(-1.0, 1.0, n)
+    for k in (1, 50, 2048, 15000):
+        _check_topk(s, n, k)
+
+
+def _check_topk(s, n, k):
+    T = s.shape[0]
     stride = (n + 3) // 4 * 4
     buf = torch.full((T, stride), float("nan"), dtype=torch.float32)
     buf[:, :n] = s
