@@ -192,9 +192,10 @@ misa_status misa_route_heads(const uint16_t* q, const float* w, const float* mea
   uint8_t* scratch = static_cast<uint8_t*>(workspace) + kErrBytes;
   float* partial = reinterpret_cast<float*>(scratch);
   unsigned* counters = reinterpret_cast<unsigned*>(scratch + misa::router_counters_offset(T, H, L, B));
-  return cuda_status(misa::launch_route_heads(q, w, means, means_seq_stride, seq_of, prefix_len, T, H, L, B, q_block,
-                                              h, static_cast<int>(nseq), heads, importance, partial, counters,
-                                              err_word(workspace), reinterpret_cast<cudaStream_t>(stream)));
+  const int qpm = misa::route_tc_queries_per_group(H, q_block, nseq == 1 || means_seq_stride == 0);
+  return cuda_status(misa::launch_route_heads_tc(q, w, means, means_seq_stride, static_cast<int>(nseq), seq_of,
+                                                 prefix_len, T, H, L, B, q_block, h, qpm, heads, importance, partial,
+                                                 counters, err_word(workspace), reinterpret_cast<cudaStream_t>(stream)));
 }
 
 misa_status misa_index_score(const uint16_t* q, const float* w, const uint16_t* keys, int64_t nkeyseq,

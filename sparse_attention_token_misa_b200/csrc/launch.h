@@ -28,6 +28,14 @@ cudaError_t launch_route_heads(const uint16_t* q, const float* w, const float* m
                                int q_block, int h, int nseq_means, int32_t* heads, float* importance, float* partial,
                                unsigned* counters, uint32_t* err, cudaStream_t stream);
 
+// Tensor-core router (route_tc.cu).  qpm = queries per MMA row group (>1 only
+// when the queries share one sequence's block means).
+int route_tc_queries_per_group(int H, int q_block, bool shared_sequence);
+cudaError_t launch_route_heads_tc(const uint16_t* q, const float* w, const float* means, int64_t means_seq_stride,
+                                  int nseq, const int32_t* seq_of, const int32_t* prefix_len, int T, int H, int64_t L,
+                                  int B, int q_block, int h, int qpm, int32_t* heads, float* importance,
+                                  float* partial, unsigned* counters, uint32_t* err, cudaStream_t stream);
+
 // Bytes of router scratch: partial importances [T][ceil(M/32)][H] fp32 followed
 // (at a 256-byte boundary) by one counter per routing decision.
 size_t router_scratch_bytes(int T, int H, int64_t L, int B, int q_block);

@@ -70,14 +70,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 // Bounded wait for the phase of `parity` to complete.  Returns false (after
 // recording MISA_DEVERR_TIMEOUT) if it has not completed within ~2 s.
+// With `abort` (a CTA-wide flag in shared memory) the wait also gives up as
+// soon as another thread of the CTA has given up, and a wait that times out
+// raises the flag, so every role of the CTA stops within one spin.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err,
+                                          volatile uint32_t* abort = nullptr) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
+    if (abort && *abort) return false;
     if (globaltimer_ns() - t0 > kWaitLimitNs) {
       record_error(err, MISA_DEVERR_TIMEOUT);
+      if (abort) *abort = 1u;
       return false;
     }
   }

@@ -113,7 +113,8 @@ struct Cfg {
   static constexpr int kOffBar = kOffQ + kQBytes;
   static constexpr int kNumBars = 2 * kStages + 2 + 2 + 3;
   static constexpr int kOffTmemSlot = kOffBar + kNumBars * 8;
-  static constexpr int kOffW = (kOffTmemSlot + 4 + 15) / 16 * 16;
+  static constexpr int kOffAbort = kOffTmemSlot + 4;
+  static constexpr int kOffW = (kOffAbort + 4 + 15) / 16 * 16;
   static constexpr int kOffPlen = kOffW + N * 4;
   static constexpr int kOffRow = kOffPlen + (QPG * 4 + 7) / 8 * 8;
   static constexpr int kSmemBytes = kOffRow + QPG * 8 + 1024;  // + alignment slack
@@ -175,6 +176,7 @@ score_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreParams p) {
   uint64_t* qempty = bars + 2 * S + 5;  // MMAs of the group finished
   uint64_t* done = bars + 2 * S + 6;    // all MMAs of this CTA finished
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffTmemSlot);
+  volatile uint32_t* abort = reinterpret_cast<volatile uint32_t*>(smem + C::kOffAbort);
   float* w_s = reinterpret_cast<float*>(smem + C::kOffW);
   int32_t* plen_s = reinterpret_cast<int32_t*>(smem + C::kOffPlen);   // visible keys of each group query
   float** rowp_s = reinterpret_cast<float**>(smem + C::kOffRow);       // its score row (NULL past T)
@@ -195,6 +197,7 @@ score_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreParams p) {
     mbar_init(qfull, kGather ? kProdThreads : kProdThreads - 32);
     mbar_init(qempty, 1);
     mbar_init(done, 1);
+    *abort = 0u;
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -242,7 +245,7 @@ score_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreParams p) {
             }
             const int s = static_cast<int>(it % S);
             const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
-            if (!mbar_wait(&empty[s], ph ^ 1u, p.err)) break;
+            if (!mbar_wait(&empty[s], ph ^ 1u, p.err, abort)) break;
             uint8_t* dst = sA + s * kATileBytes;
             mbar_arrive_expect_tx(&full[s], kATileBytes);
             const int y = static_cast<int>(seq_row0 + static_cast<int64_t>(j) * kTileM);
@@ -262,7 +265,7 @@ score_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreParams p) {
         const int g0 = static_cast<int>(i0 / tpg);
         const int g1 = static_cast<int>((i1 - 1) / tpg);
         for (int g = g0, groups = 0; g <= g1; ++g, ++groups) {
-          if (groups > 0 && !mbar_wait(qempty, (groups - 1) & 1, p.err)) break;
+          if (groups > 0 && !mbar_wait(qempty, (groups - 1) & 1, p.err, abort)) break;
           stage_query_rows<HP, QPG>(p, g, sQ, pt - 32, kProdThreads - 32);
           fence_proxy_async_smem();
           mbar_arrive(qfull);
@@ -286,7 +289,7 @@ score_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreParams p) {
           cp_async_wait_group<0>();
           fence_proxy_async_smem();
           for (; pending_from < it; ++pending_from) mbar_arrive(&full[pending_from % S]);
-          if (groups > 0 && !mbar_wait(qempty, (groups - 1) & 1, p.err)) { ok = false; break; }
+          if (groups > 0 && !mbar_wait(qempty, (groups - 1) & 1, p.err, abort)) { ok = false; break; }
           stage_query_rows<HP, QPG>(p, g, sQ, pt, kProdThreads);
           fence_proxy_async_smem();
           mbar_arrive(qfull);
@@ -302,7 +305,7 @@ score_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreParams p) {
         }
         const int s = static_cast<int>(it % S);
         const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
-        if (!mbar_wait(&empty[s], ph ^ 1u, p.err)) { ok = false; break; }
+        if (!mbar_wait(&empty[s], ph ^ 1u, p.err, abort)) { ok = false; break; }
         uint8_t* dst = sA + s * kATileBytes;
         const int32_t* crow = p.cand + static_cast<int64_t>(t_gather) * p.n_cand;
         for (int x = pt; x < kTileM * 16; x += kProdThreads) {
@@ -338,16 +341,16 @@ score_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreParams p) {
       for (int64_t item = i0; item < i1; ++item) {
         const int g = static_cast<int>(item / tpg);
         if (g != cur_g) {
-          if (!mbar_wait(qfull, groups & 1, p.err)) break;
+          if (!mbar_wait(qfull, groups & 1, p.err, abort)) break;
           ++groups;
           cur_g = g;
         }
         const int a = static_cast<int>(it & 1);
         const uint32_t aph = static_cast<uint32_t>((it >> 1) & 1);
-        if (!mbar_wait(&tempty[a], aph ^ 1u, p.err)) break;
+        if (!mbar_wait(&tempty[a], aph ^ 1u, p.err, abort)) break;
         const int s = static_cast<int>(it % S);
         const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
-        if (!mbar_wait(&full[s], ph, p.err)) break;
+        if (!mbar_wait(&full[s], ph, p.err, abort)) break;
         tc_fence_after();
         const uint32_t a_addr = smem_u32(sA + s * kATileBytes);
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * N);
@@ -376,8 +379,11 @@ score_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreParams p) {
     const int ql0 = col0 / HP;
     const int r = quarter * 32 + lane;     // TMEM lane = key row of the tile
     const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
+    // After a wait gives up the loop keeps running without work ("skip"), so
+    // every epilogue thread still reaches every named barrier.
     int64_t it = 0;
     int cur_g = -1;
+    bool skip = false;
     for (int64_t item = i0; item < i1; ++item) {
       const int g = static_cast<int>(item / tpg);
       const int j = static_cast<int>(item - static_cast<int64_t>(g) * tpg);
@@ -410,7 +416,11 @@ score_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreParams p) {
       }
       const int a = static_cast<int>(it & 1);
       const uint32_t aph = static_cast<uint32_t>((it >> 1) & 1);
-      if (!mbar_wait(&tfull[a], aph, p.err)) break;
+      if (skip || !mbar_wait(&tfull[a], aph, p.err, abort)) {
+        skip = true;
+        ++it;
+        continue;
+      }
       tc_fence_after();
 
       // which output slot this lane's key row maps to, and whether it is visible
