@@ -156,9 +156,10 @@ def reduce_max(x: float, dist, device) -> float:
     return float(t.item())
 
 
-def _time_steps(step, steps, flush, stream, marks=None):
+def _time_steps(step, steps, flush, stream, marks=None, after=None):
     """Per-step CUDA-event timing with an untimed L2 flush before every step.
-    marks: optional list of names; step(ev) records intermediate events."""
+    marks: optional list of names; step(ev) records intermediate events.
+    after: called after every step (its events have completed)."""
     tot = 0.0
     marks = list(marks or [])
     parts = {m: 0.0 for m in marks}
@@ -173,6 +174,8 @@ def _time_steps(step, steps, flush, stream, marks=None):
         tot += evs[0].elapsed_time(evs[-1])
         for i, m in enumerate(marks):
             parts[m] += evs[i].elapsed_time(evs[i + 1])
+        if after:
+            after()
     return tot, parts
 
 
@@ -204,32 +207,48 @@ def run_cuda(args):
     def flush():
         flush_buf.fill_(1.0)
 
-    # warm-up (eager), then one CUDA graph per stage of the step
+    # warm-up (eager), then the step as one CUDA graph with timing events
+    # recorded inside it between the stages
+    from sparse_attention_token_misa_b200.indexer import capture_graph
     for _ in range(args.warmup):
         ix.run(q, w, keys, means, seq_of, plen)
         dense.run(q, w, keys, seq_of, plen)
     torch.cuda.synchronize()
-    ix.capture(q, w, keys, means, seq_of, plen)
+    inner = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+
+    def misa_graph_body():
+        inner[0].record()
+        ix.route(q, w, means, seq_of, plen)
+        inner[1].record()
+        ix.score(q, w, keys, seq_of, plen)
+        inner[2].record()
+        ix.select(plen)
+        inner[3].record()
+
+    g_step = capture_graph(misa_graph_body)
     dense.capture(q, w, keys, seq_of, plen)
     for _ in range(args.warmup):
-        ix.g_route.replay(); ix.g_score.replay(); ix.g_select.replay()
+        g_step.replay()
     torch.cuda.synchronize()
     misa.error_reset(ix.ws)
     misa.error_reset(ix.ws_route)
 
+    parts = {"route": 0.0, "score": 0.0, "topk": 0.0}
+
     def misa_step(evs):
-        ix.g_route.replay()
-        evs[0].record(stream)
-        ix.g_score.replay()
-        evs[1].record(stream)
-        ix.g_select.replay()
+        g_step.replay()
+
+    def after_step():
+        parts["route"] += inner[0].elapsed_time(inner[1])
+        parts["score"] += inner[1].elapsed_time(inner[2])
+        parts["topk"] += inner[2].elapsed_time(inner[3])
 
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         t0 = time.perf_counter()
-        tot_ms, parts = _time_steps(misa_step, args.steps, flush, stream, marks=["route", "score", "topk"])
+        tot_ms, _ = _time_steps(misa_step, args.steps, flush, stream, after=after_step)
         wall = time.perf_counter() - t0
     torch.cuda.synchronize()
     if dist:
@@ -239,15 +258,15 @@ def run_cuda(args):
         raise RuntimeError(f"device error word {dev_err:#x}")
     ms_step = reduce_max(tot_ms / args.steps, dist, dev)
 
-    # the same step as one graph, the dense 64-head indexer and the block
-    # statistics on the same batch (same protocol)
-    one_ms, _ = _time_steps(lambda evs: ix.g_step.replay(), args.steps, flush, stream)
+    # the dense 64-head indexer and the block statistics on the same batch
+    # (same protocol)
     dense_ms, dparts = _time_steps(lambda evs: (dense.g_score.replay(), evs[0].record(stream),
                                                 dense.g_select.replay()), args.steps, flush, stream,
                                    marks=["score", "topk"])
+    dense_one_ms, _ = _time_steps(lambda evs: dense.g_step.replay(), args.steps, flush, stream)
     stats_ms, _ = _time_steps(lambda evs: misa.block_stats(keys, B, out=means), args.steps, flush, stream)
-    one_ms /= args.steps
     dense_ms /= args.steps
+    dense_one_ms /= args.steps
     stats_ms /= args.steps
 
     # e2e through the public API: the step's inputs copied from pinned host
@@ -268,7 +287,6 @@ def run_cuda(args):
         out = ix_e.run(q_d, w_d, keys, means, so_d, pl_d)
         idx_h.copy_(out, non_blocking=True)
 
-    from sparse_attention_token_misa_b200.indexer import capture_graph
     g_e2e = capture_graph(e2e_eager)
     for _ in range(3):
         g_e2e.replay()
@@ -314,8 +332,8 @@ def run_cuda(args):
                    "l2": "flushed before every timed step (256 MiB write, untimed); K is 268 MB > L2"},
         "queries_per_s": T * ws_n / (ms_step * 1e-3),
         "gpu_launches": 4 * args.steps,
-        "timing": "CUDA events on the launching stream around graph replays of the route, score and top-k "
-                  "stages of each step",
+        "timing": "CUDA events on the launching stream around one graph replay per step (route, score, top-k); "
+                  "the per-kernel split from timing events recorded inside the graph",
         "roofline": {"bound": "hbm", "kernel": "score_kernel (misa_index_score)", "achieved": achieved,
                      "peak": hbm_gbs, "peak_kind": f"{peak_kind} hbm copy GB/s", "unit": "GB/s",
                      "frac": achieved / hbm_gbs, "traffic": traffic,
@@ -326,9 +344,9 @@ def run_cuda(args):
                        "CUDA graph replay per step",
                 "eager_ms_per_step": e2e_eager_ms},
         "detail": {"route_ms": parts["route"] / args.steps, "score_ms": score_ms, "topk_ms": parts["topk"] / args.steps,
-                   "misa8_ms": ms_step, "misa8_one_graph_ms": one_ms,
-                   "dense64_ms": dense_ms, "dense64_score_ms": dparts["score"] / args.steps,
-                   "dense64_topk_ms": dparts["topk"] / args.steps, "dense64_over_misa8": dense_ms / ms_step,
+                   "misa8_ms": ms_step,
+                   "dense64_ms": dense_one_ms, "dense64_score_ms": dparts["score"] / args.steps,
+                   "dense64_topk_ms": dparts["topk"] / args.steps, "dense64_over_misa8": dense_one_ms / ms_step,
                    "block_stats_ms": stats_ms,
                    "block_stats_GBps": (T * L * 128 * 2 + T * (L // B) * 128 * 4) / (stats_ms * 1e-3) / 1e9,
                    "wall_s_timed_region": wall},
@@ -374,21 +392,31 @@ def _prefill(misa, dev, stream, flush, steps):
     means = misa.block_stats(keys, wl.B)
     ix = misa.MisaIndexer(wl.T, wl.H, wl.h, wl.L, wl.B, wl.k, wl.q_block, device=dev)
     pairs = int(wl.prefix_len.sum())
-    parts = {}
 
-    ix.capture(q, w, keys, means, so, pl)
+    from sparse_attention_token_misa_b200.indexer import capture_graph
+    inner = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
 
-    def pf(evs):
-        ix.g_route.replay()
-        evs[0].record(stream)
-        ix.g_score.replay()
-        evs[1].record(stream)
-        ix.g_select.replay()
+    def body():
+        inner[0].record()
+        ix.route(q, w, means, so, pl)
+        inner[1].record()
+        ix.score(q, w, keys, so, pl)
+        inner[2].record()
+        ix.select(pl)
+        inner[3].record()
 
+    g = capture_graph(body)
     for _ in range(2):
-        ix.g_step.replay()
+        g.replay()
     torch.cuda.synchronize()
-    ms, parts = _time_steps(pf, steps, flush, stream, marks=["route", "score", "topk"])
+    parts = {"route": 0.0, "score": 0.0, "topk": 0.0}
+
+    def after():
+        parts["route"] += inner[0].elapsed_time(inner[1])
+        parts["score"] += inner[1].elapsed_time(inner[2])
+        parts["topk"] += inner[2].elapsed_time(inner[3])
+
+    ms, _ = _time_steps(lambda evs: g.replay(), steps, flush, stream, after=after)
     score_ms = parts["score"] / steps
     flops = 2.0 * 128 * wl.h * pairs
     _, tc, kind = _peaks()

@@ -156,7 +156,7 @@ MISA_API misa_status misa_block_stats(const uint16_t* keys, int64_t nseq, int64_
  * head id), written in ascending id order.
  *   means: nseq sequences of [M][128] fp32 at sequence stride means_seq_stride
  *          elements (as written by misa_block_stats: M * 128); 16-byte aligned,
- *          means_seq_stride % 4 == 0; seq_of values must lie in [0, nseq).
+ *          means_seq_stride % 128 == 0; seq_of values must lie in [0, nseq).
  *   heads: [ceil(T/q_block)][h] int32 out.  importance: [ceil(T/q_block)][H]
  *          fp32 out, may be NULL.
  * Limits: 1 <= H <= 128, 1 <= h <= H, 1 <= q_block, T >= 1.
@@ -277,7 +277,7 @@ MISA_API misa_status misa_hier_rerank(const uint16_t* q, const float* w, const u
  * blocks[t][0..m): chosen block ids ascending, -1 padded.
  * cand[t][i*B + r] = blocks[t][i]*B + r, or -1 if that block slot is empty or the
  * id is >= min(prefix_len[t], L).  block_scores: [T][M] fp32 out, may be NULL.
- * means / nseq / means_seq_stride as for misa_route_heads.
+ * means / nseq / seq_of as for misa_route_heads (means_seq_stride % 4 == 0 suffices).
  * Limits: 1 <= H <= 128, 1 <= m <= MISA_MAX_TOPK, 1 <= B.
  * workspace: >= misa_workspace_bytes(MISA_OP_HISA_BLOCK_FILTER, T, H, L, B, m, 0).
  */

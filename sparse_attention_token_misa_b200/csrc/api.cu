@@ -4,7 +4,6 @@
 #include <cuda_runtime.h>
 
 #include <cstring>
-#include <mutex>
 
 #include "../../include/misa.h"
 #include "launch.h"
@@ -21,39 +20,13 @@ inline misa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MISA_O
 
 uint32_t* err_word(void* ws) { return reinterpret_cast<uint32_t*>(ws); }
 
-// cuTensorMapEncodeTiled, fetched once from the driver through the runtime so
-// that the library needs no link-time dependency on libcuda.
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_tiled() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  });
-  return fn;
-}
-
 // 2-D map over all key rows: dim0 = 128 bf16 (256 B), dim1 = rows; box = 64 x kTmaBoxRows
 // with 128-byte swizzle, the layout the UMMA descriptors expect.
 misa_status make_key_map(const uint16_t* keys, int64_t rows, CUtensorMap* map) {
-  EncodeTiledFn fn = encode_tiled();
-  if (!fn) return MISA_ERR_CUDA;
-  std::memset(map, 0, sizeof(*map));
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(MISA_HEAD_DIM), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(MISA_HEAD_DIM) * 2};
-  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(misa::kTmaBoxRows)};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(keys), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? MISA_OK : MISA_ERR_CUDA;
+  return misa::encode_2d_map(map, true, keys, MISA_HEAD_DIM, static_cast<uint64_t>(rows), MISA_HEAD_DIM * 2, 64,
+                             static_cast<uint32_t>(misa::kTmaBoxRows), true)
+             ? MISA_OK
+             : MISA_ERR_CUDA;
 }
 
 misa_status check_ws(const void* ws, size_t have, size_t need) {
@@ -187,6 +160,7 @@ misa_status misa_route_heads(const uint16_t* q, const float* w, const float* mea
   misa_status st = check_block_args(q, w, means, nseq, means_seq_stride, seq_of, prefix_len, T, H, L, B);
   if (st != MISA_OK) return st;
   if (!heads || q_block < 1 || h < 1 || h > H) return MISA_ERR_INVALID_ARG;
+  if (means_seq_stride % MISA_HEAD_DIM != 0) return MISA_ERR_INVALID_ARG;  // rows of 128 means for the TMA map
   st = check_ws(workspace, workspace_bytes, misa_workspace_bytes(MISA_OP_ROUTE_HEADS, T, H, L, B, 0, 0));
   if (st != MISA_OK) return st;
   uint8_t* scratch = static_cast<uint8_t*>(workspace) + kErrBytes;
@@ -195,7 +169,8 @@ misa_status misa_route_heads(const uint16_t* q, const float* w, const float* mea
   const int qpm = misa::route_tc_queries_per_group(H, q_block, nseq == 1 || means_seq_stride == 0);
   return cuda_status(misa::launch_route_heads_tc(q, w, means, means_seq_stride, static_cast<int>(nseq), seq_of,
                                                  prefix_len, T, H, L, B, q_block, h, qpm, heads, importance, partial,
-                                                 counters, err_word(workspace), reinterpret_cast<cudaStream_t>(stream)));
+                                                 counters, false, err_word(workspace),
+                                                 reinterpret_cast<cudaStream_t>(stream)));
 }
 
 misa_status misa_index_score(const uint16_t* q, const float* w, const uint16_t* keys, int64_t nkeyseq,

@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace misa {
 
 // SM count of the current device (cached; 0 on error).
@@ -14,19 +16,48 @@ int device_sm_count();
 // Raise `func`'s dynamic shared-memory limit to at least `bytes` on the current
 // device; cudaFuncSetAttribute runs only the first time a size is needed.
 cudaError_t ensure_dynamic_smem(const void* func, int bytes);
+// 2-D TMA map over `rows` rows of `inner` elements (bf16 or fp32), rows
+// `row_bytes` apart; box = box_inner x box_rows; optional 128-byte swizzle.
+bool encode_2d_map(CUtensorMap* map, bool bf16, const void* base, uint64_t inner, uint64_t rows, uint64_t row_bytes,
+                   uint32_t box_inner, uint32_t box_rows, bool swizzle128);
 // Resident CTAs per SM of `func` at this block size and dynamic shared memory
 // (cached; 1 if the query fails).
 int occupancy_blocks(const void* func, int threads, size_t smem);
+
+// Launch with programmatic stream serialization (the kernel may start while the
+// previous kernel of the stream is still running; it calls pdl_wait_inputs()
+// before reading anything) and an optional cluster size.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       int cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster_x > 0) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
 
 cudaError_t launch_block_stats(const uint16_t* keys, int64_t nseq, int64_t L, int64_t key_seq_stride, int B,
                                float* means, cudaStream_t stream);
 
 int router_chunks(int M);
-
-cudaError_t launch_route_heads(const uint16_t* q, const float* w, const float* means, int64_t means_seq_stride,
-                               const int32_t* seq_of, const int32_t* prefix_len, int T, int H, int64_t L, int B,
-                               int q_block, int h, int nseq_means, int32_t* heads, float* importance, float* partial,
-                               unsigned* counters, uint32_t* err, cudaStream_t stream);
 
 // Tensor-core router (route_tc.cu).  qpm = queries per MMA row group (>1 only
 // when the queries share one sequence's block means).
@@ -34,10 +65,11 @@ int route_tc_queries_per_group(int H, int q_block, bool shared_sequence);
 cudaError_t launch_route_heads_tc(const uint16_t* q, const float* w, const float* means, int64_t means_seq_stride,
                                   int nseq, const int32_t* seq_of, const int32_t* prefix_len, int T, int H, int64_t L,
                                   int B, int q_block, int h, int qpm, int32_t* heads, float* importance,
-                                  float* partial, unsigned* counters, uint32_t* err, cudaStream_t stream);
+                                  float* partial, unsigned* counters, bool clear_counters, uint32_t* err,
+                                  cudaStream_t stream);
 
-// Bytes of router scratch: partial importances [T][ceil(M/32)][H] fp32 followed
-// (at a 256-byte boundary) by one counter per routing decision.
+// Bytes of router scratch: partial importances (at most [T][ceil(M/32)][H]
+// fp32) followed, at a 256-byte boundary, by one counter per routing decision.
 size_t router_scratch_bytes(int T, int H, int64_t L, int B, int q_block);
 size_t router_counters_offset(int T, int H, int64_t L, int B);
 

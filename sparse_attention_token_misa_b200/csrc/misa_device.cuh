@@ -42,6 +42,14 @@ __device__ __forceinline__ uint32_t float_key(float f) {
 // Key of -inf; valid (selectable) entries have key > kNegInfKey.
 constexpr uint32_t kNegInfKey = 0x007FFFFFu;
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// Kernels are launched so that they may start while the previous kernel on the
+// stream finishes; every kernel waits here (all threads) before it reads any
+// input, so whatever ran before has completed and its writes are visible.
+__device__ __forceinline__ void pdl_wait_inputs() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the next kernel on the stream start its prologue.
+__device__ __forceinline__ void pdl_allow_next() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");

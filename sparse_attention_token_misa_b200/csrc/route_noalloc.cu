@@ -59,7 +59,7 @@ misa_status misa_route_heads_noalloc(const uint16_t* q, const float* w, const fl
   if (!q || !w || !means || !seq_of || !prefix_len || !heads) return MISA_ERR_INVALID_ARG;
   if (T < 1 || H < 1 || L < 1 || B < 1 || nseq < 1 || q_block < 1 || h < 1 || h > H) return MISA_ERR_INVALID_ARG;
   if (H > MISA_MAX_HEADS) return MISA_ERR_UNSUPPORTED;
-  if (!aligned16(q) || !aligned16(means) || means_seq_stride < 0 || means_seq_stride % 4 != 0)
+  if (!aligned16(q) || !aligned16(means) || means_seq_stride < 0 || means_seq_stride % MISA_HEAD_DIM != 0)
     return MISA_ERR_INVALID_ARG;
   const int64_t M = (L + B - 1) / B;
   if (nseq > 1 && means_seq_stride < M * MISA_HEAD_DIM) return MISA_ERR_INVALID_ARG;
@@ -80,7 +80,7 @@ misa_status misa_route_heads_noalloc(const uint16_t* q, const float* w, const fl
   const int qpm = misa::route_tc_queries_per_group(H, q_block, nseq == 1 || means_seq_stride == 0);
   cudaError_t e = misa::launch_route_heads_tc(q, w, means, means_seq_stride, static_cast<int>(nseq), seq_of,
                                               prefix_len, T, H, L, B, q_block, h, qpm, heads, importance, partial,
-                                              counters, nullptr, reinterpret_cast<cudaStream_t>(stream));
+                                              counters, true, nullptr, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MISA_OK : MISA_ERR_CUDA;
 }
 

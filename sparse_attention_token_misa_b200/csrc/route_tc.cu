@@ -8,23 +8,24 @@
 //   importance[g][h] = sum over the queries t of decision g, and over the blocks
 //                      j visible to g, of w[t][h] * ReLU(q[t][h] . mean_j)
 //
-// The contraction q . mean_j for all (query, head) rows and all blocks is an MMA:
-// M = 128 (query, head) rows of one sequence (qpm queries x H heads, zero rows
-// past them), N = 128 blocks per tile, K = 128.  The fp32 block means are split
-// on the fly into bf16 hi = bf16(m) and lo = bf16(m - hi) (together about 16
-// significant bits), and D = q . hi + q . lo accumulates in fp32 in TMEM.  The
-// epilogue thread of row (t, h) sums ReLU(D) over the visible blocks of the tile
-// in registers and over the tiles of its row group, then multiplies by w[t][h]:
-// no cross-thread reduction.  A decision's rows are combined in shared memory;
-// when a decision spans several row groups (prefill), the last CTA to finish
-// one of them (atomic counter) sums the groups' partials in a fixed order.
-// The top-h selection (ties to the lower head id, ids ascending) is one warp.
+// The contraction q . mean_j is an MMA: M = 128 (query, head) rows of one
+// sequence (qpm queries x H heads, zero rows past them), N = 64 blocks per
+// tile, K = 128.  The fp32 block means of a tile arrive by one TMA copy; the
+// producers split them into bf16 hi = bf16(m) and lo = bf16(m - hi) (together
+// about 16 significant bits) and D = q . hi + q . lo accumulates in fp32 in
+// TMEM.  The epilogue thread of row (t, h) sums ReLU(D) over the tile's
+// visible blocks and multiplies by w[t][h] (no cross-thread reduction); the
+// rows of one head are added in shared memory and each work item (row group,
+// block tile) stores its H partial importances.  When a CTA finishes its items
+// of a decision it adds their count to the decision's counter (one atomic per
+// run of items); the CTA that completes the count sums the decision's partials
+// in item order (deterministic) and selects the top-h (ties to the lower head
+// id, ids ascending).
 //
 // Roles (288 threads): warps 0-3 epilogue (TMEM lane quarter = warp), warp 4
-// TMEM allocation + MMA issue, warps 5-8 producers (query rows once per row
-// group; block-mean tiles converted to hi/lo each tile).  Waits are bounded.
-#include <algorithm>
-
+// TMEM allocation + MMA issue, warp 5 lane 0 TMA of the query rows (once per
+// row group) and of the fp32 mean tiles, warps 6-8 the hi/lo conversion.
+// Waits are bounded and share a CTA-wide abort flag.
 #include "launch.h"
 #include "misa_device.cuh"
 
@@ -33,33 +34,33 @@ namespace misa {
 namespace {
 
 constexpr int kRM = 128;                       // MMA M: (query, head) rows
-constexpr int kRN = 128;                       // MMA N: blocks per tile
+constexpr int kRN = 64;                        // MMA N: blocks per tile
 constexpr int kRStages = 2;
 constexpr int kREpiThreads = 128;
-constexpr int kRProdThreads = 128;
+constexpr int kRConvThreads = 96;              // warps 6-8
 constexpr int kRMmaWarp = 4;
-constexpr int kRProdWarp0 = 5;
+constexpr int kRTmaWarp = 5;
 constexpr int kRThreads = 288;
-constexpr int kRATileBytes = kRM * kD * 2;     // 32 KB of query rows
-constexpr int kRBTileBytes = kRN * kD * 2;     // 32 KB per hi or lo tile
-constexpr int kRStageBytes = 2 * kRBTileBytes;
+constexpr int kRATileBytes = kRM * kD * 2;     // 32 KB of query rows (bf16)
+constexpr int kRFTileBytes = kRN * kD * 4;     // 32 KB of fp32 means
+constexpr int kRBTileBytes = kRN * kD * 2;     // 16 KB per hi or lo tile
+constexpr int kRStageBytes = kRFTileBytes + 2 * kRBTileBytes;
 constexpr int kRTmemCols = 2 * kRN;            // two accumulators
 constexpr uint32_t kRIdesc = idesc_bf16_f32(kRM, kRN);
 constexpr int kROffA = 0;
-constexpr int kROffB = kRATileBytes;
-constexpr int kROffBar = kROffB + kRStages * kRStageBytes;
-constexpr int kRNumBars = 2 * kRStages + 2 + 2 + 3;
+constexpr int kROffS = kRATileBytes;
+constexpr int kROffBar = kROffS + kRStages * kRStageBytes;
+constexpr int kRNumBars = 3 * kRStages + 2 + 2 + 3;
 constexpr int kROffTmem = kROffBar + kRNumBars * 8;
-constexpr int kROffRed = (kROffTmem + 4 + 15) / 16 * 16;       // [128] row sums
+constexpr int kROffRed = (kROffTmem + 4 + 15) / 16 * 16;       // [128] row contributions
 constexpr int kROffImp = kROffRed + kRM * 4;                     // [MISA_MAX_HEADS] decision importances
-constexpr int kROffFlag = kROffImp + MISA_MAX_HEADS * 4;
+constexpr int kROffFlag = kROffImp + MISA_MAX_HEADS * 4;         // flag, abort
 constexpr int kRSmemBytes = kROffFlag + 16 + 1024;
 
 struct RouteParams {
   const uint16_t* q;
   const float* w;
-  const float* means;
-  int64_t means_seq_stride;
+  int64_t means_seq_rows;    // rows of 128 means between sequences in the TMA map
   int nseq;
   const int32_t* seq_of;
   const int32_t* prefix_len;
@@ -69,8 +70,9 @@ struct RouteParams {
   int qpm;        // queries per row group (share one sequence and one decision)
   int n_pg;       // row groups
   int n_bt;       // block tiles
-  float* partial;            // [n_pg][H] row-group importances (decisions spanning several groups)
-  unsigned* counters;        // [G] groups finished per decision (zero on entry)
+  int64_t n_items;
+  float* partial;            // [n_items][H] partial importances per work item
+  unsigned* counters;        // [G] items finished per decision (zero on entry)
   int32_t* heads;            // [G][h]
   float* importance;         // [G][H] or NULL
   uint32_t* err;
@@ -139,19 +141,22 @@ __device__ void select_top_h(const float* imp, int H, int h, int g, int32_t* hea
   }
 }
 
-__global__ void __launch_bounds__(kRThreads, 1) route_tc_kernel(const RouteParams p) {
+__global__ void __launch_bounds__(kRThreads, 1)
+route_tc_kernel(const __grid_constant__ CUtensorMap means_map, const __grid_constant__ CUtensorMap q_map,
+                const RouteParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem + kROffA;
-  uint8_t* sB = smem + kROffB;
+  uint8_t* sS = smem + kROffS;  // stage s: [fp32 means | hi | lo]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kROffBar);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + kRStages;
-  uint64_t* tfull = bars + 2 * kRStages;
-  uint64_t* tempty = bars + 2 * kRStages + 2;
-  uint64_t* afull = bars + 2 * kRStages + 4;
-  uint64_t* aempty = bars + 2 * kRStages + 5;
-  uint64_t* done = bars + 2 * kRStages + 6;
+  uint64_t* ffull = bars;                    // [S] fp32 tile landed (TMA)
+  uint64_t* bfull = bars + kRStages;         // [S] hi/lo tile written
+  uint64_t* empty = bars + 2 * kRStages;     // [S] MMAs of the stage done
+  uint64_t* tfull = bars + 3 * kRStages;     // [2]
+  uint64_t* tempty = bars + 3 * kRStages + 2;
+  uint64_t* afull = bars + 3 * kRStages + 4;
+  uint64_t* aempty = bars + 3 * kRStages + 5;
+  uint64_t* done = bars + 3 * kRStages + 6;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kROffTmem);
   float* red = reinterpret_cast<float*>(smem + kROffRed);
   float* imp = reinterpret_cast<float*>(smem + kROffImp);
@@ -161,14 +166,15 @@ __global__ void __launch_bounds__(kRThreads, 1) route_tc_kernel(const RouteParam
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
     for (int s = 0; s < kRStages; ++s) {
-      mbar_init(&full[s], kRProdThreads);
+      mbar_init(&ffull[s], 1);
+      mbar_init(&bfull[s], kRConvThreads);
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], kREpiThreads);
     }
-    mbar_init(afull, kRProdThreads);
+    mbar_init(afull, 1);
     mbar_init(aempty, 1);
     mbar_init(done, 1);
     *abort = 0u;
@@ -178,116 +184,123 @@ __global__ void __launch_bounds__(kRThreads, 1) route_tc_kernel(const RouteParam
     tmem_alloc(tmem_slot, kRTmemCols);
     tmem_relinquish();
   }
+  if (tid == kRTmaWarp * 32) {
+    tma_prefetch_desc(&means_map);
+    tma_prefetch_desc(&q_map);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait_inputs();
+  pdl_allow_next();
 
-  // this CTA's row groups (whole groups, so the block sums stay in registers)
-  const int pg0 = static_cast<int>(static_cast<int64_t>(p.n_pg) * blockIdx.x / gridDim.x);
-  const int pg1 = static_cast<int>(static_cast<int64_t>(p.n_pg) * (blockIdx.x + 1) / gridDim.x);
+  const int64_t i0 = p.n_items * blockIdx.x / gridDim.x;
+  const int64_t i1 = p.n_items * (blockIdx.x + 1) / gridDim.x;
+  const int nbt = p.n_bt;
 
-  if (warp >= kRProdWarp0) {
-    // ------------------------------------------------------------ producers
-    const int pt = tid - kRProdWarp0 * 32;
-    int64_t it = 0;
-    bool ok = true;
-    for (int pg = pg0, ng = 0; pg < pg1 && ok; ++pg, ++ng) {
-      // query rows of the group: row r = ql * H + hh
-      if (ng > 0 && !mbar_wait(aempty, (ng - 1) & 1, p.err, abort)) break;
-      for (int x = pt; x < kRM * 16; x += kRProdThreads) {
-        const int r = x >> 4, ch = x & 15;
-        const int ql = r / p.H, hh = r - ql * p.H;
-        const int t = pg * p.qpm + ql;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (ql < p.qpm && t < p.T)
-          v = __ldg(reinterpret_cast<const uint4*>(p.q + (static_cast<int64_t>(t) * p.H + hh) * kD + ch * 8));
-        *reinterpret_cast<uint4*>(sA + sw128_tile_offset(kRM, r, ch)) = v;
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(afull);
-      const float* mb = p.means + static_cast<int64_t>(group_seq(p, pg)) * p.means_seq_stride;
-      for (int bt = 0; bt < p.n_bt; ++bt, ++it) {
+  if (warp == kRTmaWarp) {
+    // ------------------------------------------------------------ query rows and fp32 mean tiles by TMA
+    if (lane == 0) {
+      int64_t it = 0;
+      int cur_pg = -1, ng = 0;
+      bool a_pending = false;
+      for (int64_t item = i0; item < i1; ++item, ++it) {
+        const int pg = static_cast<int>(item / nbt);
+        const int bt = static_cast<int>(item - static_cast<int64_t>(pg) * nbt);
+        if (pg != cur_pg) {
+          // the group's 128 query rows (rows past its queries belong to later
+          // queries or lie past the tensor: their results are weighted by 0)
+          if (ng > 0 && !mbar_wait(aempty, (ng - 1) & 1, p.err, abort)) break;
+          mbar_arrive_expect_tx(afull, kRATileBytes);
+          const int ya = pg * p.qpm * p.H;
+          tma_load_2d(sA, &q_map, afull, 0, ya);
+          tma_load_2d(sA + kRATileBytes / 2, &q_map, afull, 64, ya);
+          a_pending = true;
+          cur_pg = pg;
+          ++ng;
+        }
         const int s = static_cast<int>(it % kRStages);
         const uint32_t ph = static_cast<uint32_t>((it / kRStages) & 1);
-        if (!mbar_wait(&empty[s], ph ^ 1u, p.err, abort)) { ok = false; break; }
-        uint8_t* hi_t = sB + s * kRStageBytes;
-        uint8_t* lo_t = hi_t + kRBTileBytes;
-        // 128 blocks x 16 chunks of 8 means; 4 chunks in flight per thread
-        for (int x0 = pt; x0 < kRN * 16; x0 += 4 * kRProdThreads) {
-          float4 f[4][2];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int x = x0 + u * kRProdThreads;
-            const int r = x >> 4, ch = x & 15;
-            const int j = bt * kRN + r;
-            if (x < kRN * 16 && j < p.M) {
-              const float4* src = reinterpret_cast<const float4*>(mb + static_cast<int64_t>(j) * kD + ch * 8);
-              f[u][0] = __ldg(src);
-              f[u][1] = __ldg(src + 1);
-            } else {
-              f[u][0] = f[u][1] = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-          }
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int x = x0 + u * kRProdThreads;
-            if (x >= kRN * 16) continue;
-            const int r = x >> 4, ch = x & 15;
-            const float e[8] = {f[u][0].x, f[u][0].y, f[u][0].z, f[u][0].w,
-                                f[u][1].x, f[u][1].y, f[u][1].z, f[u][1].w};
-            uint32_t hw[4], lw[4];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const __nv_bfloat16 h0 = __float2bfloat16_rn(e[2 * c]);
-              const __nv_bfloat16 h1 = __float2bfloat16_rn(e[2 * c + 1]);
-              const __nv_bfloat16 l0 = __float2bfloat16_rn(e[2 * c] - __bfloat162float(h0));
-              const __nv_bfloat16 l1 = __float2bfloat16_rn(e[2 * c + 1] - __bfloat162float(h1));
-              hw[c] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
-                      (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
-              lw[c] = static_cast<uint32_t>(__bfloat16_as_ushort(l0)) |
-                      (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
-            }
-            const uint32_t off = sw128_tile_offset(kRN, r, ch);
-            *reinterpret_cast<uint4*>(hi_t + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-            *reinterpret_cast<uint4*>(lo_t + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-          }
-        }
-        fence_proxy_async_smem();
-        mbar_arrive(&full[s]);
+        if (!mbar_wait(&empty[s], ph ^ 1u, p.err, abort)) break;
+        mbar_arrive_expect_tx(&ffull[s], kRFTileBytes);
+        const int y = static_cast<int>(group_seq(p, pg) * p.means_seq_rows + static_cast<int64_t>(bt) * kRN);
+        tma_load_2d(sS + s * kRStageBytes, &means_map, &ffull[s], 0, y);
       }
+      // no TMA write may still be in flight when the CTA exits
+      const int64_t first = it > kRStages ? it - kRStages : 0;
+      for (int64_t k2 = first; k2 < it; ++k2)
+        mbar_wait(&ffull[k2 % kRStages], static_cast<uint32_t>((k2 / kRStages) & 1), p.err);
+      if (a_pending && ng > 0) mbar_wait(afull, (ng - 1) & 1, p.err);
+    }
+  } else if (warp > kRTmaWarp) {
+    // ------------------------------------------------------------ hi/lo conversion
+    const int ct = tid - (kRTmaWarp + 1) * 32;
+    int64_t it = 0;
+    for (int64_t item = i0; item < i1; ++item, ++it) {
+      const int s = static_cast<int>(it % kRStages);
+      const uint32_t ph = static_cast<uint32_t>((it / kRStages) & 1);
+      if (!mbar_wait(&ffull[s], ph, p.err, abort)) break;
+      const float* ft = reinterpret_cast<const float*>(sS + s * kRStageBytes);
+      uint8_t* hi_t = sS + s * kRStageBytes + kRFTileBytes;
+      uint8_t* lo_t = hi_t + kRBTileBytes;
+      for (int x = ct; x < kRN * 16; x += kRConvThreads) {
+        const int r = x >> 4, ch = x & 15;
+        const float4 a0 = *reinterpret_cast<const float4*>(ft + r * kD + ch * 8);
+        const float4 a1 = *reinterpret_cast<const float4*>(ft + r * kD + ch * 8 + 4);
+        const float e[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const __nv_bfloat16 h0 = __float2bfloat16_rn(e[2 * c]);
+          const __nv_bfloat16 h1 = __float2bfloat16_rn(e[2 * c + 1]);
+          const __nv_bfloat16 l0 = __float2bfloat16_rn(e[2 * c] - __bfloat162float(h0));
+          const __nv_bfloat16 l1 = __float2bfloat16_rn(e[2 * c + 1] - __bfloat162float(h1));
+          hw[c] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
+          lw[c] = static_cast<uint32_t>(__bfloat16_as_ushort(l0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
+        }
+        const uint32_t off = sw128_tile_offset(kRN, r, ch);
+        *reinterpret_cast<uint4*>(hi_t + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4*>(lo_t + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&bfull[s]);
     }
   } else if (warp == kRMmaWarp) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
       int64_t it = 0;
+      int cur_pg = -1, ng = 0;
       const uint32_t a_addr = smem_u32(sA);
-      bool ok = true;
-      for (int pg = pg0, ng = 0; pg < pg1 && ok; ++pg, ++ng) {
-        if (!mbar_wait(afull, ng & 1, p.err, abort)) break;
-        for (int bt = 0; bt < p.n_bt; ++bt, ++it) {
-          const int a = static_cast<int>(it & 1);
-          const uint32_t aph = static_cast<uint32_t>((it >> 1) & 1);
-          if (!mbar_wait(&tempty[a], aph ^ 1u, p.err, abort)) { ok = false; break; }
-          const int s = static_cast<int>(it % kRStages);
-          const uint32_t ph = static_cast<uint32_t>((it / kRStages) & 1);
-          if (!mbar_wait(&full[s], ph, p.err, abort)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t hi_addr = smem_u32(sB + s * kRStageBytes);
-          const uint32_t lo_addr = hi_addr + kRBTileBytes;
-          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * kRN);
-#pragma unroll
-          for (int kk = 0; kk < kD / 16; ++kk) {
-            const uint32_t koff = (kk >> 2) * (kRM * 128) + (kk & 3) * 32;
-            const uint32_t boff = (kk >> 2) * (kRN * 128) + (kk & 3) * 32;
-            const uint64_t adesc = sw128_kmajor_desc(a_addr + koff);
-            umma_bf16(d_tmem, adesc, sw128_kmajor_desc(hi_addr + boff), kRIdesc, kk > 0 ? 1u : 0u);
-            umma_bf16(d_tmem, adesc, sw128_kmajor_desc(lo_addr + boff), kRIdesc, 1u);
-          }
-          umma_commit(&empty[s]);
-          if (bt + 1 == p.n_bt) umma_commit(aempty);
-          umma_commit(&tfull[a]);
+      for (int64_t item = i0; item < i1; ++item, ++it) {
+        const int pg = static_cast<int>(item / nbt);
+        if (pg != cur_pg) {
+          if (!mbar_wait(afull, ng & 1, p.err, abort)) break;
+          cur_pg = pg;
+          ++ng;
         }
+        const int a = static_cast<int>(it & 1);
+        const uint32_t aph = static_cast<uint32_t>((it >> 1) & 1);
+        if (!mbar_wait(&tempty[a], aph ^ 1u, p.err, abort)) break;
+        const int s = static_cast<int>(it % kRStages);
+        const uint32_t ph = static_cast<uint32_t>((it / kRStages) & 1);
+        if (!mbar_wait(&bfull[s], ph, p.err, abort)) break;
+        tc_fence_after();
+        const uint32_t hi_addr = smem_u32(sS + s * kRStageBytes + kRFTileBytes);
+        const uint32_t lo_addr = hi_addr + kRBTileBytes;
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(a * kRN);
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t aoff = (kk >> 2) * (kRM * 128) + (kk & 3) * 32;
+          const uint32_t boff = (kk >> 2) * (kRN * 128) + (kk & 3) * 32;
+          const uint64_t adesc = sw128_kmajor_desc(a_addr + aoff);
+          umma_bf16(d_tmem, adesc, sw128_kmajor_desc(hi_addr + boff), kRIdesc, kk > 0 ? 1u : 0u);
+          umma_bf16(d_tmem, adesc, sw128_kmajor_desc(lo_addr + boff), kRIdesc, 1u);
+        }
+        umma_commit(&empty[s]);
+        const bool group_ends = (item + 1 == i1) || (static_cast<int>((item + 1) / nbt) != pg);
+        if (group_ends) umma_commit(aempty);
+        umma_commit(&tfull[a]);
       }
       umma_commit(done);
       mbar_wait(done, 0, p.err);
@@ -295,93 +308,93 @@ __global__ void __launch_bounds__(kRThreads, 1) route_tc_kernel(const RouteParam
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
+    // After a wait gives up the loop keeps running without work ("skip"), so
+    // every epilogue thread still reaches every named barrier.
     const int r = warp * 32 + lane;  // row (ql, hh) of the group
     const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
-    // After a wait gives up the loops keep running without work ("skip"), so
-    // every epilogue thread still reaches every named barrier.
+    const int pgs_per_dec = p.q_block / p.qpm;
     int64_t it = 0;
+    int cur_pg = -1;
+    float wrow = 0.f;
+    int nvis = 0, g = 0;
+    int64_t run_items = 0;  // items of decision g done by this CTA since the last counter update
     bool skip = false;
-    for (int pg = pg0; pg < pg1; ++pg) {
-      const int g = (pg * p.qpm) / p.q_block;
-      const int nvis = visible_blocks(p, g);
-      float rowsum = 0.f;
-      for (int bt = 0; bt < p.n_bt; ++bt, ++it) {
-        const int a = static_cast<int>(it & 1);
-        const uint32_t aph = static_cast<uint32_t>((it >> 1) & 1);
-        if (skip || !mbar_wait(&tfull[a], aph, p.err, abort)) {
-          skip = true;
-          continue;
-        }
+    for (int64_t item = i0; item < i1; ++item, ++it) {
+      const int pg = static_cast<int>(item / nbt);
+      const int bt = static_cast<int>(item - static_cast<int64_t>(pg) * nbt);
+      if (pg != cur_pg) {
+        cur_pg = pg;
+        g = (pg * p.qpm) / p.q_block;
+        nvis = visible_blocks(p, g);
+        const int ql = r / p.H, hh = r - ql * p.H;
+        const int t = pg * p.qpm + ql;
+        wrow = (ql < p.qpm && t < p.T) ? p.w[static_cast<int64_t>(t) * p.H + hh] : 0.f;
+      }
+      const int a = static_cast<int>(it & 1);
+      const uint32_t aph = static_cast<uint32_t>((it >> 1) & 1);
+      float contrib = 0.f;
+      if (!skip && mbar_wait(&tfull[a], aph, p.err, abort)) {
         tc_fence_after();
         int nc = nvis - bt * kRN;  // visible columns of this tile
         nc = nc < 0 ? 0 : (nc > kRN ? kRN : nc);
-        const uint32_t t_acc = t_lane + static_cast<uint32_t>(a * kRN);
-        float s = 0.f;
+        uint32_t v[kRN];
 #pragma unroll
-        for (int c0 = 0; c0 < kRN; c0 += 64) {
-          uint32_t v[64];
+        for (int u = 0; u < kRN / 16; ++u) tmem_ld16(t_lane + static_cast<uint32_t>(a * kRN + 16 * u), v + 16 * u);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&tempty[a]);
+        float sum = 0.f;
+        if (nc == kRN) {
 #pragma unroll
-          for (int u = 0; u < 4; ++u) tmem_ld16(t_acc + static_cast<uint32_t>(c0 + 16 * u), v + 16 * u);
-          tmem_wait_ld();
-          if (c0 + 64 == kRN) {
-            tc_fence_before();
-            mbar_arrive(&tempty[a]);
-          }
-          if (c0 + 64 <= nc) {
+          for (int jj = 0; jj < kRN; ++jj) sum += fmaxf(__uint_as_float(v[jj]), 0.f);
+        } else {
 #pragma unroll
-            for (int jj = 0; jj < 64; ++jj) s += fmaxf(__uint_as_float(v[jj]), 0.f);
-          } else {
-#pragma unroll
-            for (int jj = 0; jj < 64; ++jj) s += (c0 + jj < nc) ? fmaxf(__uint_as_float(v[jj]), 0.f) : 0.f;
-          }
+          for (int jj = 0; jj < kRN; ++jj) sum += jj < nc ? fmaxf(__uint_as_float(v[jj]), 0.f) : 0.f;
         }
-        rowsum += s;
+        contrib = wrow * sum;
+      } else {
+        skip = true;
       }
-      // row (t, hh) importance contribution, combined over the group's queries
-      const int ql = r / p.H, hh = r - ql * p.H;
-      const int t = pg * p.qpm + ql;
-      float contrib = 0.f;
-      if (ql < p.qpm && t < p.T) contrib = p.w[static_cast<int64_t>(t) * p.H + hh] * rowsum;
+      // this item's partial importance of each head: the rows of one head added
       red[r] = contrib;
       named_bar_sync(1, kREpiThreads);
-      const int pgs_per_dec = p.q_block / p.qpm;  // row groups of a full decision
-      const int first_pg = g * pgs_per_dec;
-      const int last_pg = (first_pg + pgs_per_dec < p.n_pg ? first_pg + pgs_per_dec : p.n_pg) - 1;
-      if (first_pg == last_pg) {
-        // the whole decision is this group: select here
-        if (tid < p.H) {
-          float sum = 0.f;
-          for (int k2 = 0; k2 < p.qpm; ++k2) sum += red[k2 * p.H + tid];
-          imp[tid] = sum;
-        }
-        named_bar_sync(1, kREpiThreads);
-        if (warp == 0 && !*abort) select_top_h(imp, p.H, p.h, g, p.heads, p.importance);
-      } else {
-        if (tid < p.H) {
-          float sum = 0.f;
-          for (int k2 = 0; k2 < p.qpm; ++k2) sum += red[k2 * p.H + tid];
-          p.partial[static_cast<int64_t>(pg) * p.H + tid] = sum;
-        }
+      if (tid < p.H && !skip) {
+        float sum = 0.f;
+        for (int k2 = 0; k2 < p.qpm; ++k2) sum += red[k2 * p.H + tid];
+        p.partial[item * p.H + tid] = sum;
+      }
+      ++run_items;
+      // last item of decision g in this CTA's range: count them in
+      const bool run_ends = (item + 1 == i1) || (static_cast<int>((((item + 1) / nbt) * p.qpm) / p.q_block) != g);
+      if (run_ends) {
+        const int first_pg = g * pgs_per_dec;
+        const int last_pg = (first_pg + pgs_per_dec < p.n_pg ? first_pg + pgs_per_dec : p.n_pg) - 1;
+        const int64_t first_item = static_cast<int64_t>(first_pg) * nbt;
+        const int64_t end_item = static_cast<int64_t>(last_pg + 1) * nbt;
         __threadfence();
         named_bar_sync(1, kREpiThreads);
         if (tid == 0) {
-          const unsigned expected = static_cast<unsigned>(last_pg - first_pg + 1);
-          flag[0] = (!*abort && atomicAdd(&p.counters[g], 1u) + 1u == expected) ? 1u : 0u;
+          const unsigned expected = static_cast<unsigned>(end_item - first_item);
+          flag[0] = (!*abort && atomicAdd(&p.counters[g], static_cast<unsigned>(run_items)) +
+                                        static_cast<unsigned>(run_items) == expected)
+                        ? 1u
+                        : 0u;
         }
         named_bar_sync(1, kREpiThreads);
         if (flag[0]) {
           __threadfence();
           if (tid < p.H) {
             float sum = 0.f;
-            for (int x = first_pg; x <= last_pg; ++x) sum += __ldcg(&p.partial[static_cast<int64_t>(x) * p.H + tid]);
+            for (int64_t x = first_item; x < end_item; ++x) sum += __ldcg(&p.partial[x * p.H + tid]);
             imp[tid] = sum;
           }
           named_bar_sync(1, kREpiThreads);
           if (warp == 0) select_top_h(imp, p.H, p.h, g, p.heads, p.importance);
           if (tid == 0) p.counters[g] = 0u;  // ready for the next call
         }
+        run_items = 0;
       }
-      named_bar_sync(1, kREpiThreads);  // red / imp / flag are reused by the next group
+      named_bar_sync(1, kREpiThreads);  // red / imp / flag are reused by the next item
     }
   }
 
@@ -400,19 +413,15 @@ int route_tc_queries_per_group(int H, int q_block, bool shared_sequence) {
   return qpm;
 }
 
-size_t route_tc_partial_floats(int T, int H, int qpm) {
-  return static_cast<size_t>((T + qpm - 1) / qpm) * H;
-}
-
 cudaError_t launch_route_heads_tc(const uint16_t* q, const float* w, const float* means, int64_t means_seq_stride,
                                   int nseq, const int32_t* seq_of, const int32_t* prefix_len, int T, int H, int64_t L,
                                   int B, int q_block, int h, int qpm, int32_t* heads, float* importance,
-                                  float* partial, unsigned* counters, uint32_t* err, cudaStream_t stream) {
+                                  float* partial, unsigned* counters, bool clear_counters, uint32_t* err,
+                                  cudaStream_t stream) {
   RouteParams p;
   p.q = q;
   p.w = w;
-  p.means = means;
-  p.means_seq_stride = means_seq_stride;
+  p.means_seq_rows = means_seq_stride / kD;
   p.nseq = nseq;
   p.seq_of = seq_of;
   p.prefix_len = prefix_len;
@@ -426,21 +435,33 @@ cudaError_t launch_route_heads_tc(const uint16_t* q, const float* w, const float
   p.qpm = qpm;
   p.n_pg = (T + qpm - 1) / qpm;
   p.n_bt = (p.M + kRN - 1) / kRN;
+  p.n_items = static_cast<int64_t>(p.n_pg) * p.n_bt;
   p.partial = partial;
   p.counters = counters;
   p.heads = heads;
   p.importance = importance;
   p.err = err;
-  const int G = (T + q_block - 1) / q_block;
-  cudaError_t e = cudaMemsetAsync(counters, 0, static_cast<size_t>(G) * sizeof(unsigned), stream);
-  if (e != cudaSuccess) return e;
+  // fp32 means as rows of 128: sequence b's block j is row b * means_seq_rows + j
+  CUtensorMap map;
+  const uint64_t rows = static_cast<uint64_t>(nseq - 1) * static_cast<uint64_t>(p.means_seq_rows) + p.M;
+  if (!encode_2d_map(&map, false, means, kD, rows, kD * 4, kD, kRN, false)) return cudaErrorInvalidValue;
+  // query rows, bf16, 128-byte swizzled K-major like the keys
+  CUtensorMap qmap;
+  if (!encode_2d_map(&qmap, true, q, kD, static_cast<uint64_t>(T) * H, kD * 2, 64, kRM, true))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaSuccess;
+  if (clear_counters) {
+    const int G = (T + q_block - 1) / q_block;
+    e = cudaMemsetAsync(counters, 0, static_cast<size_t>(G) * sizeof(unsigned), stream);
+    if (e != cudaSuccess) return e;
+  }
   e = ensure_dynamic_smem(reinterpret_cast<const void*>(route_tc_kernel), kRSmemBytes);
   if (e != cudaSuccess) return e;
   const int sms = device_sm_count();
   if (sms <= 0) return cudaErrorInvalidDevice;
-  const int grid = std::max(1, std::min(p.n_pg, sms));
-  route_tc_kernel<<<grid, kRThreads, kRSmemBytes, stream>>>(p);
-  return cudaGetLastError();
+  const int64_t grid = p.n_items < sms ? p.n_items : sms;
+  return launch_pdl(route_tc_kernel, dim3(static_cast<unsigned>(grid)), dim3(kRThreads), kRSmemBytes, stream, 0, map,
+                    qmap, p);
 }
 
 }  // namespace misa

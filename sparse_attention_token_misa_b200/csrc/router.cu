@@ -1,20 +1,14 @@
-// Block-level affinity shared by the MISA router and the HISA block filter,
-// the router's per-query-block head selection, and HISA's candidate expansion.
+// HISA block filter (block scores and candidate expansion) and the router's
+// scratch layout.
 //
-// Affinity of head h of query t with key block j:
-//     A[t, h, j] = w[t, h] * ReLU(q[t, h] . mean_j)
-// "MISA: Mixture of Indexer Sparse Attention for Long-Context LLM Inference"
-// (gist.science), Methodology: per-head affinities against block-aggregated
-// keys, aggregated into a head importance, top-h heads kept (cost O(H_I * M)).
+// Block score of query t for key block j (all heads):
+//     bs[t, j] = sum over h of w[t, h] * ReLU(q[t, h] . mean_j)
 // HISA explainer (zhichai.net), section 三, Stage 1: the query is scored against
-// the block representatives only, top-m blocks kept.
-//
-// The router reduces A over blocks (and over the queries of a routing
-// decision; the last CTA of a decision to finish, found with an atomic
-// counter, sums the partials in a fixed order and selects the heads); HISA
-// reduces A over heads.  Both are O(H * M * d) per query, a few
-// percent of the token scoring, and run here on the fp32 CUDA cores with the
-// query heads and a chunk of block means staged in shared memory.
+// the block representatives only and the top-m blocks are kept.  O(H * M * d)
+// per query, a few percent of the token scoring; it runs on the fp32 CUDA cores
+// with the query's heads and a chunk of block means staged in shared memory.
+// (The MISA router, which reduces the same affinity over blocks instead of
+// heads, runs on the tensor cores: route_tc.cu.)
 #include "launch.h"
 #include "misa_device.cuh"
 
@@ -26,105 +20,22 @@ constexpr int kThreads = 256;
 constexpr int kChunk = 32;        // blocks per CTA (8 warps x 4 blocks)
 constexpr int kPad = kD + 4;      // fp32 row pitch in shared memory (keeps float4 alignment, spreads banks)
 
-// Selection of routing decision g by one CTA (kThreads threads): importance =
-// sum of the partials of its queries and chunks in a fixed order (thread
-// (part, head) sums every P-th partial, then warp 0 adds the P parts in order),
-// then h rounds of warp arg-max (value desc, id asc), then the chosen ids in
-// ascending order.
-__device__ void select_heads(const float* __restrict__ partial, float* sred, int T, int H, int n_chunks, int q_block,
-                             int g, int h, int32_t* __restrict__ heads, float* __restrict__ importance) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int t0 = g * q_block;
-  const int t1 = (t0 + q_block < T) ? t0 + q_block : T;
-  const int n_pairs = (t1 - t0) * n_chunks;
-  const int P = kThreads / H;  // >= 2 since H <= 128
-  if (tid < P * H) {
-    const int hh = tid % H, part = tid / H;
-    float s = 0.f;
-    for (int x = part; x < n_pairs; x += P) {
-      const int t = t0 + x / n_chunks, c = x % n_chunks;
-      s += __ldcg(&partial[(static_cast<int64_t>(t) * n_chunks + c) * H + hh]);
-    }
-    sred[part * H + hh] = s;
-  }
-  __syncthreads();
-  if (warp != 0) return;
-  constexpr int kMaxHB = MISA_MAX_HEADS / 32;
-  float imp[kMaxHB];
-  bool taken[kMaxHB];
-#pragma unroll
-  for (int a = 0; a < kMaxHB; ++a) {
-    const int hh = lane + 32 * a;
-    float s = 0.f;
-    if (hh < H) {
-      for (int part = 0; part < P; ++part) s += sred[part * H + hh];
-      if (importance) importance[static_cast<int64_t>(g) * H + hh] = s;
-    }
-    imp[a] = s;
-    taken[a] = false;
-  }
-  for (int r = 0; r < h; ++r) {
-    float best = 0.f;
-    int bid = 0x7fffffff;
-#pragma unroll
-    for (int a = 0; a < kMaxHB; ++a) {
-      const int hh = lane + 32 * a;
-      if (hh < H && !taken[a]) {
-        if (bid == 0x7fffffff || imp[a] > best || (imp[a] == best && hh < bid)) {
-          best = imp[a];
-          bid = hh;
-        }
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ob = __shfl_xor_sync(0xffffffffu, best, o);
-      const int oid = __shfl_xor_sync(0xffffffffu, bid, o);
-      const bool better = (oid != 0x7fffffff) && (bid == 0x7fffffff || ob > best || (ob == best && oid < bid));
-      if (better) {
-        best = ob;
-        bid = oid;
-      }
-    }
-#pragma unroll
-    for (int a = 0; a < kMaxHB; ++a)
-      if (lane + 32 * a == bid) taken[a] = true;
-  }
-  // Ascending output: rank of a chosen head = chosen heads with a smaller id.
-  int before = 0;
-#pragma unroll
-  for (int a = 0; a < kMaxHB; ++a) {
-    const unsigned mask = __ballot_sync(0xffffffffu, taken[a]);
-    if (taken[a]) {
-      const int pos = before + __popc(mask & ((1u << lane) - 1u));
-      heads[static_cast<int64_t>(g) * h + pos] = lane + 32 * a;
-    }
-    before += __popc(mask);
-  }
-}
-
 // grid: (T, n_chunks).  Thread (warp jq, lane hp) owns heads hp + 32*a and
-// blocks chunk*32 + 4*jq + u (u < 4).
-template <bool kHisa>
+// blocks chunk*32 + 4*jq + u (u < 4); a warp reduces its heads per block.
 __global__ void __launch_bounds__(kThreads)
-affinity_kernel(const uint16_t* __restrict__ q, const float* __restrict__ w, const float* __restrict__ means,
+block_score_kernel(const uint16_t* __restrict__ q, const float* __restrict__ w, const float* __restrict__ means,
                 int64_t means_seq_stride, const int32_t* __restrict__ seq_of, const int32_t* __restrict__ prefix_len,
-                int T, int H, int64_t L, int B, int M, int q_block, int nseq_means,
-                float* __restrict__ partial,  // router: [T][n_chunks][H]
-                unsigned* __restrict__ counters,  // router: [G] CTAs finished per decision (zero on entry)
-                int h, int32_t* __restrict__ heads, float* __restrict__ importance,
-                float* __restrict__ bscore,   // HISA:   [T][bs_stride]
+                int T, int H, int64_t L, int B, int M, int nseq_means,
+                float* __restrict__ bscore,   // [T][bs_stride]
                 int64_t bs_stride,
                 uint32_t* __restrict__ err) {
   extern __shared__ float4 smem_f4[];
   float* sq = reinterpret_cast<float*>(smem_f4);   // [H][kPad]
   float* sm = sq + H * kPad;                        // [kChunk][kPad]
-  float* sred = sm + kChunk * kPad;                 // [8][H] (router) or unused
   __shared__ float sw[MISA_MAX_HEADS];
 
   const int t = blockIdx.x;
   const int chunk = blockIdx.y;
-  const int n_chunks = gridDim.y;
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int jq = tid >> 5;
@@ -134,10 +45,8 @@ affinity_kernel(const uint16_t* __restrict__ q, const float* __restrict__ w, con
     if (tid == 0) record_error(err, MISA_DEVERR_BAD_SEQ);
     seq = 0;
   }
-  // Visibility: a block is seen iff it lies wholly inside the prefix of the
-  // query that owns the decision (the first query of its query block).
-  const int t_dec = kHisa ? t : (t / q_block) * q_block;
-  const int64_t plen = prefix_len[t_dec];
+  // Visibility: a block is seen iff it lies wholly inside the query's prefix.
+  const int64_t plen = prefix_len[t];
 
   // Stage q[t] (bf16 -> fp32), w[t] and the chunk's block means (zeros past
   // M).  Every global load of a thread is issued before any of them is used,
@@ -229,39 +138,6 @@ affinity_kernel(const uint16_t* __restrict__ q, const float* __restrict__ w, con
     for (int u = 0; u < 4; ++u) acc[a][u] = vis[u] ? wh * fmaxf(acc[a][u], 0.f) : 0.f;
   }
 
-  if constexpr (!kHisa) {
-    // Router: sum over this thread's 4 blocks, then over the 8 warps.
-#pragma unroll
-    for (int a = 0; a < kMaxHB; ++a) {
-      const int h = lane + 32 * a;
-      if (a < HB && h < H) sred[jq * H + h] = ((acc[a][0] + acc[a][1]) + acc[a][2]) + acc[a][3];
-    }
-    __syncthreads();
-    for (int hh = tid; hh < H; hh += kThreads) {
-      float s = 0.f;
-#pragma unroll
-      for (int k = 0; k < kThreads / 32; ++k) s += sred[k * H + hh];
-      partial[(static_cast<int64_t>(t) * n_chunks + chunk) * H + hh] = s;
-    }
-    // The last CTA of this routing decision to finish selects its heads.
-    __shared__ unsigned s_last;
-    const int g = t / q_block;
-    const int tq0 = g * q_block;
-    const int tq1 = (tq0 + q_block < T) ? tq0 + q_block : T;
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) {
-      const unsigned expected = static_cast<unsigned>((tq1 - tq0) * n_chunks);
-      const unsigned old = atomicAdd(&counters[g], 1u);
-      s_last = (old + 1u == expected) ? 1u : 0u;
-    }
-    __syncthreads();
-    if (s_last) {
-      __threadfence();
-      select_heads(partial, sred, T, H, n_chunks, q_block, g, h, heads, importance);
-      if (tid == 0) counters[g] = 0u;  // leave the counter ready for the next call
-    }
-  } else {
     // HISA: block score = sum over heads (this thread's heads, then the warp).
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -272,7 +148,6 @@ affinity_kernel(const uint16_t* __restrict__ q, const float* __restrict__ w, con
       for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
       const int j = chunk * kChunk + jq * 4 + u;
       if (lane == 0 && j < M) bscore[static_cast<int64_t>(t) * bs_stride + j] = vis[u] ? s : -__int_as_float(0x7f800000);
-    }
   }
 }
 
@@ -297,10 +172,7 @@ __global__ void hisa_expand_kernel(const int32_t* __restrict__ blocks, const int
   }
 }
 
-size_t affinity_smem_bytes(int H) {
-  const int red = 8 * H > kThreads ? 8 * H : kThreads;  // per-warp sums, then the selection's partial sums
-  return static_cast<size_t>(H * kPad + kChunk * kPad + red) * sizeof(float);
-}
+size_t affinity_smem_bytes(int H) { return static_cast<size_t>(H * kPad + kChunk * kPad) * sizeof(float); }
 
 }  // namespace
 
@@ -317,24 +189,6 @@ size_t router_scratch_bytes(int T, int H, int64_t L, int B, int q_block) {
   return router_counters_offset(T, H, L, B) + static_cast<size_t>(G) * sizeof(unsigned);
 }
 
-cudaError_t launch_route_heads(const uint16_t* q, const float* w, const float* means, int64_t means_seq_stride,
-                               const int32_t* seq_of, const int32_t* prefix_len, int T, int H, int64_t L, int B,
-                               int q_block, int h, int nseq_means, int32_t* heads, float* importance, float* partial,
-                               unsigned* counters, uint32_t* err, cudaStream_t stream) {
-  const int M = static_cast<int>((L + B - 1) / B);
-  const int nch = router_chunks(M);
-  const int G = (T + q_block - 1) / q_block;
-  cudaError_t e = cudaMemsetAsync(counters, 0, static_cast<size_t>(G) * sizeof(unsigned), stream);
-  if (e != cudaSuccess) return e;
-  const size_t smem = affinity_smem_bytes(H);
-  e = ensure_dynamic_smem(reinterpret_cast<const void*>(affinity_kernel<false>), static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  affinity_kernel<false><<<dim3(T, nch), kThreads, smem, stream>>>(q, w, means, means_seq_stride, seq_of, prefix_len,
-                                                                   T, H, L, B, M, q_block, nseq_means, partial,
-                                                                   counters, h, heads, importance, nullptr, 0, err);
-  return cudaGetLastError();
-}
-
 cudaError_t launch_hisa_block_scores(const uint16_t* q, const float* w, const float* means, int64_t means_seq_stride,
                                      const int32_t* seq_of, const int32_t* prefix_len, int T, int H, int64_t L, int B,
                                      int nseq_means, float* bscore, int64_t bs_stride, uint32_t* err,
@@ -342,11 +196,10 @@ cudaError_t launch_hisa_block_scores(const uint16_t* q, const float* w, const fl
   const int M = static_cast<int>((L + B - 1) / B);
   const int nch = router_chunks(M);
   const size_t smem = affinity_smem_bytes(H);
-  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(affinity_kernel<true>), static_cast<int>(smem));
+  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(block_score_kernel), static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  affinity_kernel<true><<<dim3(T, nch), kThreads, smem, stream>>>(q, w, means, means_seq_stride, seq_of, prefix_len, T,
-                                                                  H, L, B, M, 1, nseq_means, nullptr, nullptr, 0,
-                                                                  nullptr, nullptr, bscore, bs_stride, err);
+  block_score_kernel<<<dim3(T, nch), kThreads, smem, stream>>>(q, w, means, means_seq_stride, seq_of, prefix_len, T, H,
+                                                               L, B, M, nseq_means, bscore, bs_stride, err);
   return cudaGetLastError();
 }
 

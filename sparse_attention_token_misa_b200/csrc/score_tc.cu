@@ -209,6 +209,8 @@ score_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreParams p) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait_inputs();
+  pdl_allow_next();
 
   int64_t i0, i1;
   item_range(p.n_items, i0, i1);
@@ -490,8 +492,7 @@ cudaError_t launch_cfg(const CUtensorMap& tmap, const ScoreParams& p, int num_sm
   const int per_sm = occupancy_blocks(reinterpret_cast<const void*>(kern), C::kThreads, C::kSmemBytes);
   int64_t grid = std::min<int64_t>(p.n_items, static_cast<int64_t>(num_sms) * std::max(1, std::min(per_sm, C::kCtasPerSm)));
   if (grid < 1) grid = 1;
-  kern<<<static_cast<unsigned>(grid), C::kThreads, C::kSmemBytes, stream>>>(tmap, p);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3(C::kThreads), C::kSmemBytes, stream, 0, tmap, p);
 }
 
 }  // namespace

@@ -168,6 +168,8 @@ topk_cluster_kernel(const float* __restrict__ scores, int64_t n, int64_t row_str
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
   uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + kKeysOff);
 
+  pdl_wait_inputs();
+  pdl_allow_next();
   cg::cluster_group cl = cg::this_cluster();
   const int CL = static_cast<int>(cl.num_blocks());
   const int rank = static_cast<int>(cl.block_rank());
@@ -465,6 +467,8 @@ topk_row_kernel(const float* __restrict__ scores, int64_t n, int64_t row_stride,
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const float kNegInf = -__int_as_float(0x7f800000);
   const int64_t t = blockIdx.x;
+  pdl_wait_inputs();
+  pdl_allow_next();
   const float* row = scores + t * row_stride;
   const int32_t* idrow = id_map ? id_map + t * id_map_stride : nullptr;
   int32_t* out = idx + t * k;
@@ -733,8 +737,8 @@ cudaError_t launch_topk(const float* scores, int T, int64_t n, int64_t row_strid
     const size_t smem = row_smem(n);
     cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(topk_row_kernel), static_cast<int>(row_smem(kRowMaxN)));
     if (e != cudaSuccess) return e;
-    topk_row_kernel<<<T, kRowThreads, smem, stream>>>(scores, n, row_stride, row_valid, id_map, id_map_stride, k, idx);
-    return cudaGetLastError();
+    return launch_pdl(topk_row_kernel, dim3(T), dim3(kRowThreads), smem, stream, 0, scores, n, row_stride, row_valid,
+                      id_map, id_map_stride, k, idx);
   }
   const int CL = pick_cluster(n);
   int64_t slice = (n + CL - 1) / CL;
@@ -746,26 +750,11 @@ cudaError_t launch_topk(const float* scores, int T, int64_t n, int64_t row_strid
   cudaError_t e = ensure_dynamic_smem(fn, static_cast<int>(topk_smem_bytes()));
   if (e != cudaSuccess) return e;
 
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(CL, T, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = CL;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
   if (in_smem)
-    e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel<true>, scores, n, row_stride, row_valid, id_map, id_map_stride, k,
-                           idx, slice);
-  else
-    e = cudaLaunchKernelEx(&cfg, topk_cluster_kernel<false>, scores, n, row_stride, row_valid, id_map, id_map_stride,
-                           k, idx, slice);
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
+    return launch_pdl(topk_cluster_kernel<true>, dim3(CL, T, 1), dim3(kThreads), smem, stream, CL, scores, n,
+                      row_stride, row_valid, id_map, id_map_stride, k, idx, slice);
+  return launch_pdl(topk_cluster_kernel<false>, dim3(CL, T, 1), dim3(kThreads), smem, stream, CL, scores, n,
+                    row_stride, row_valid, id_map, id_map_stride, k, idx, slice);
 }
 
 }  // namespace misa

@@ -133,6 +133,7 @@ def route(q=P, w=P, means=P, nseq=1, mstride=0, seq_of=P, plen=P, T=4, H=64, L=1
     (dict(means=MIS), INVALID),
     (dict(mstride=6, nseq=2), INVALID),
     (dict(mstride=8 * 128 - 4, nseq=2), INVALID),   # M * 128 = 1024 required
+    (dict(mstride=8 * 128 + 4, nseq=2), INVALID),   # rows of 128 means
     (dict(heads=None), INVALID),
     (dict(ws_bytes=256), WORKSPACE),
     (dict(ws=None), WORKSPACE),
