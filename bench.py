@@ -225,20 +225,23 @@ def run_cuda(args):
         ix.select(plen)
         inner[3].record()
 
-    g_step = capture_graph(misa_graph_body)
+    # the timed step: one graph of route, score, top-k with nothing between
+    # the kernels (so each one's prologue overlaps the previous one's tail);
+    # the per-kernel split comes from a second graph with timing events
+    # recorded between the stages
+    ix.capture(q, w, keys, means, seq_of, plen)
+    g_split = capture_graph(misa_graph_body)
     dense.capture(q, w, keys, seq_of, plen)
     for _ in range(args.warmup):
-        g_step.replay()
+        ix.g_step.replay()
+        g_split.replay()
     torch.cuda.synchronize()
     misa.error_reset(ix.ws)
     misa.error_reset(ix.ws_route)
 
     parts = {"route": 0.0, "score": 0.0, "topk": 0.0}
 
-    def misa_step(evs):
-        g_step.replay()
-
-    def after_step():
+    def after_split():
         parts["route"] += inner[0].elapsed_time(inner[1])
         parts["score"] += inner[1].elapsed_time(inner[2])
         parts["topk"] += inner[2].elapsed_time(inner[3])
@@ -248,11 +251,12 @@ def run_cuda(args):
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         t0 = time.perf_counter()
-        tot_ms, _ = _time_steps(misa_step, args.steps, flush, stream, after=after_step)
+        tot_ms, _ = _time_steps(lambda evs: ix.g_step.replay(), args.steps, flush, stream)
         wall = time.perf_counter() - t0
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
+    split_ms, _ = _time_steps(lambda evs: g_split.replay(), args.steps, flush, stream, after=after_split)
     dev_err = misa.error_query(ix.ws) | misa.error_query(ix.ws_route)
     if dev_err:
         raise RuntimeError(f"device error word {dev_err:#x}")
@@ -331,9 +335,10 @@ def run_cuda(args):
                    "parallelism": f"dp{ws_n} (independent batches)",
                    "l2": "flushed before every timed step (256 MiB write, untimed); K is 268 MB > L2"},
         "queries_per_s": T * ws_n / (ms_step * 1e-3),
-        "gpu_launches": 4 * args.steps,
-        "timing": "CUDA events on the launching stream around one graph replay per step (route, score, top-k); "
-                  "the per-kernel split from timing events recorded inside the graph",
+        "gpu_launches": 3 * args.steps,  # route, score, top-k kernels per step
+        "timing": "CUDA events on the launching stream around one graph replay per step (route, score, top-k "
+                  "with nothing between them); the per-kernel split from a second graph with timing events "
+                  "recorded between the stages (its total is detail.misa8_split_ms)",
         "roofline": {"bound": "hbm", "kernel": "score_kernel (misa_index_score)", "achieved": achieved,
                      "peak": hbm_gbs, "peak_kind": f"{peak_kind} hbm copy GB/s", "unit": "GB/s",
                      "frac": achieved / hbm_gbs, "traffic": traffic,
@@ -344,7 +349,7 @@ def run_cuda(args):
                        "CUDA graph replay per step",
                 "eager_ms_per_step": e2e_eager_ms},
         "detail": {"route_ms": parts["route"] / args.steps, "score_ms": score_ms, "topk_ms": parts["topk"] / args.steps,
-                   "misa8_ms": ms_step,
+                   "misa8_ms": ms_step, "misa8_split_ms": split_ms / args.steps,
                    "dense64_ms": dense_one_ms, "dense64_score_ms": dparts["score"] / args.steps,
                    "dense64_topk_ms": dparts["topk"] / args.steps, "dense64_over_misa8": dense_one_ms / ms_step,
                    "block_stats_ms": stats_ms,
@@ -470,8 +475,9 @@ def cpu_baseline(wl, budget_s: float = 15.0, max_queries: int | None = None):
     import oracle
 
     done, pairs, t_used = 0, 0, 0.0
-    limit = max_queries or wl.T
-    for t in range(limit):
+    limit = max_queries or 64 * wl.T  # passes over the batch until the budget is spent
+    for i in range(limit):
+        t = i % wl.T
         sub_q = wl.q[t:t + 1].to(torch.float64).numpy()
         sub_w = wl.w[t:t + 1].numpy().astype(np.float64)
         keys = wl.keys[int(wl.seq_of[t]):int(wl.seq_of[t]) + 1].to(torch.float64).numpy()
@@ -484,7 +490,8 @@ def cpu_baseline(wl, budget_s: float = 15.0, max_queries: int | None = None):
         if t_used >= budget_s:
             break
     return {"value": pairs / t_used, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
-            "sample": f"{done} of {wl.T} queries of {wl.name} (full route+score+top-k each), {t_used:.1f} s"}
+            "sample": f"{done} queries (cycling over the {wl.T} of {wl.name}; full route+score+top-k each), "
+                      f"{t_used:.1f} s"}
 
 
 def run_reference(args):

@@ -15,21 +15,31 @@
 // about 16 significant bits) and D = q . hi + q . lo accumulates in fp32 in
 // TMEM.  The epilogue thread of row (t, h) sums ReLU(D) over the tile's
 // visible blocks and multiplies by w[t][h] (no cross-thread reduction); the
-// rows of one head are added in shared memory and each work item (row group,
-// block tile) stores its H partial importances.  When a CTA finishes its items
-// of a decision it adds their count to the decision's counter (one atomic per
-// run of items); the CTA that completes the count sums the decision's partials
-// in item order (deterministic) and selects the top-h (ties to the lower head
-// id, ids ascending).
+// rows of one head are added in shared memory.  Two ways to combine the work
+// items (row group, block tile) of one decision:
+//  * a cluster of D <= 8 CTAs per decision (small batches: one wave of
+//    clusters): each CTA adds its items' contributions in registers, then CTA
+//    0 of the cluster sums the D per-CTA importances in rank order through
+//    distributed shared memory and selects;
+//  * persistent CTAs over all items (large batches): each item stores its H
+//    partial importances; when a CTA finishes its items of a decision it adds
+//    their count to the decision's counter (one atomic per run of items); the
+//    CTA that completes the count sums the decision's partials in item order.
+// Both orders are fixed, so the result is deterministic.  The top-h are taken
+// by rank (value desc, ties to the lower head id), ids ascending.
 //
-// Roles (288 threads): warps 0-3 epilogue (TMEM lane quarter = warp), warp 4
+// Roles (416 threads): warps 0-3 epilogue (TMEM lane quarter = warp), warp 4
 // TMEM allocation + MMA issue, warp 5 lane 0 TMA of the query rows (once per
-// row group) and of the fp32 mean tiles, warps 6-8 the hi/lo conversion.
+// row group) and of the fp32 mean tiles, warps 6-12 the hi/lo conversion.
 // Waits are bounded and share a CTA-wide abort flag.
+#include <cooperative_groups.h>
+
 #include "launch.h"
 #include "misa_device.cuh"
 
 namespace misa {
+
+namespace cg = cooperative_groups;
 
 namespace {
 
@@ -37,10 +47,11 @@ constexpr int kRM = 128;                       // MMA M: (query, head) rows
 constexpr int kRN = 64;                        // MMA N: blocks per tile
 constexpr int kRStages = 2;
 constexpr int kREpiThreads = 128;
-constexpr int kRConvThreads = 96;              // warps 6-8
+constexpr int kRConvThreads = 224;             // warps 6-12
 constexpr int kRMmaWarp = 4;
 constexpr int kRTmaWarp = 5;
-constexpr int kRThreads = 288;
+constexpr int kRThreads = 416;
+constexpr int kRMaxCluster = 8;
 constexpr int kRATileBytes = kRM * kD * 2;     // 32 KB of query rows (bf16)
 constexpr int kRFTileBytes = kRN * kD * 4;     // 32 KB of fp32 means
 constexpr int kRBTileBytes = kRN * kD * 2;     // 16 KB per hi or lo tile
@@ -54,8 +65,9 @@ constexpr int kRNumBars = 3 * kRStages + 2 + 2 + 3;
 constexpr int kROffTmem = kROffBar + kRNumBars * 8;
 constexpr int kROffRed = (kROffTmem + 4 + 15) / 16 * 16;       // [128] row contributions
 constexpr int kROffImp = kROffRed + kRM * 4;                     // [MISA_MAX_HEADS] decision importances
-constexpr int kROffFlag = kROffImp + MISA_MAX_HEADS * 4;         // flag, abort
-constexpr int kRSmemBytes = kROffFlag + 16 + 1024;
+constexpr int kROffImp2 = kROffImp + MISA_MAX_HEADS * 4;         // [MISA_MAX_HEADS] cluster sums
+constexpr int kROffFlag = kROffImp2 + MISA_MAX_HEADS * 4;        // flag, abort, 4 warp counts
+constexpr int kRSmemBytes = kROffFlag + 32 + 1024;
 
 struct RouteParams {
   const uint16_t* q;
@@ -95,52 +107,36 @@ __device__ __forceinline__ int visible_blocks(const RouteParams& p, int g) {
   return static_cast<int>(pl / p.B);
 }
 
-// Top-h of imp[0, H) (value desc, id asc), ids ascending into heads[g]; one warp.
-__device__ void select_top_h(const float* imp, int H, int h, int g, int32_t* heads, float* importance) {
-  const int lane = threadIdx.x & 31;
-  constexpr int kMaxHB = MISA_MAX_HEADS / 32;
-  float v[kMaxHB];
-  bool taken[kMaxHB];
-#pragma unroll
-  for (int a = 0; a < kMaxHB; ++a) {
-    const int hh = lane + 32 * a;
-    v[a] = hh < H ? imp[hh] : 0.f;
-    taken[a] = false;
-    if (importance && hh < H) importance[static_cast<int64_t>(g) * H + hh] = v[a];
-  }
-  for (int r = 0; r < h; ++r) {
-    float best = 0.f;
-    int bid = 0x7fffffff;
-#pragma unroll
-    for (int a = 0; a < kMaxHB; ++a) {
-      const int hh = lane + 32 * a;
-      if (hh < H && !taken[a] && (bid == 0x7fffffff || v[a] > best || (v[a] == best && hh < bid))) {
-        best = v[a];
-        bid = hh;
-      }
+// Top-h of imp[0, H) (value desc, ties to the lower id; NaN ranks as -inf),
+// ids ascending into heads[g].  The 128 epilogue threads call it; thread i
+// ranks head i by counting.  wcnt: 4 words of shared memory.
+__device__ void select_top_h(const float* imp, int H, int h, int g, int32_t* heads, float* importance,
+                             uint32_t* wcnt) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const float kNegInf = -__int_as_float(0x7f800000);
+  bool sel = false;
+  if (tid < H) {
+    float x = imp[tid];
+    if (importance) importance[static_cast<int64_t>(g) * H + tid] = x;
+    x = x == x ? x : kNegInf;
+    int rk = 0;
+    for (int j = 0; j < H; ++j) {
+      float y = imp[j];
+      y = y == y ? y : kNegInf;
+      rk += (y > x || (y == x && j < tid)) ? 1 : 0;
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ob = __shfl_xor_sync(0xffffffffu, best, o);
-      const int oid = __shfl_xor_sync(0xffffffffu, bid, o);
-      if (oid != 0x7fffffff && (bid == 0x7fffffff || ob > best || (ob == best && oid < bid))) {
-        best = ob;
-        bid = oid;
-      }
-    }
-#pragma unroll
-    for (int a = 0; a < kMaxHB; ++a)
-      if (lane + 32 * a == bid) taken[a] = true;
+    sel = rk < h;
   }
+  const unsigned m = __ballot_sync(0xffffffffu, sel);
+  if (lane == 0) wcnt[warp] = static_cast<uint32_t>(__popc(m));
+  named_bar_sync(2, kREpiThreads);
   int before = 0;
-#pragma unroll
-  for (int a = 0; a < kMaxHB; ++a) {
-    const unsigned mask = __ballot_sync(0xffffffffu, taken[a]);
-    if (taken[a]) heads[static_cast<int64_t>(g) * h + before + __popc(mask & ((1u << lane) - 1u))] = lane + 32 * a;
-    before += __popc(mask);
-  }
+  for (int w2 = 0; w2 < warp; ++w2) before += static_cast<int>(wcnt[w2]);
+  const int pos = before + __popc(m & ((1u << lane) - 1u));
+  if (sel && pos < h) heads[static_cast<int64_t>(g) * h + pos] = tid;
 }
 
+template <bool kCluster>
 __global__ void __launch_bounds__(kRThreads, 1)
 route_tc_kernel(const __grid_constant__ CUtensorMap means_map, const __grid_constant__ CUtensorMap q_map,
                 const RouteParams p) {
@@ -160,8 +156,10 @@ route_tc_kernel(const __grid_constant__ CUtensorMap means_map, const __grid_cons
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kROffTmem);
   float* red = reinterpret_cast<float*>(smem + kROffRed);
   float* imp = reinterpret_cast<float*>(smem + kROffImp);
+  float* imp2 = reinterpret_cast<float*>(smem + kROffImp2);
   unsigned* flag = reinterpret_cast<unsigned*>(smem + kROffFlag);
   volatile uint32_t* abort = reinterpret_cast<volatile uint32_t*>(smem + kROffFlag + 4);
+  uint32_t* wcnt = reinterpret_cast<uint32_t*>(smem + kROffFlag + 16);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
@@ -195,9 +193,26 @@ route_tc_kernel(const __grid_constant__ CUtensorMap means_map, const __grid_cons
   pdl_wait_inputs();
   pdl_allow_next();
 
-  const int64_t i0 = p.n_items * blockIdx.x / gridDim.x;
-  const int64_t i1 = p.n_items * (blockIdx.x + 1) / gridDim.x;
   const int nbt = p.n_bt;
+  const int pgs_per_dec = p.q_block / p.qpm;
+  int64_t i0, i1;
+  int crank = 0, csize = 1, cdec = 0;
+  if constexpr (kCluster) {
+    // the items of decision cdec, split over the D CTAs of its cluster
+    cg::cluster_group cl = cg::this_cluster();
+    csize = static_cast<int>(cl.num_blocks());
+    crank = static_cast<int>(cl.block_rank());
+    cdec = static_cast<int>(blockIdx.x) / csize;
+    const int first_pg = cdec * pgs_per_dec;
+    const int end_pg = first_pg + pgs_per_dec < p.n_pg ? first_pg + pgs_per_dec : p.n_pg;
+    const int64_t first_item = static_cast<int64_t>(first_pg) * nbt;
+    const int64_t cnt = (end_pg > first_pg ? static_cast<int64_t>(end_pg - first_pg) * nbt : 0);
+    i0 = first_item + cnt * crank / csize;
+    i1 = first_item + cnt * (crank + 1) / csize;
+  } else {
+    i0 = p.n_items * blockIdx.x / gridDim.x;
+    i1 = p.n_items * (blockIdx.x + 1) / gridDim.x;
+  }
 
   if (warp == kRTmaWarp) {
     // ------------------------------------------------------------ query rows and fp32 mean tiles by TMA
@@ -312,8 +327,8 @@ route_tc_kernel(const __grid_constant__ CUtensorMap means_map, const __grid_cons
     // every epilogue thread still reaches every named barrier.
     const int r = warp * 32 + lane;  // row (ql, hh) of the group
     const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
-    const int pgs_per_dec = p.q_block / p.qpm;
     int64_t it = 0;
+    float acc = 0.f;  // cluster mode: this CTA's importance of head tid
     int cur_pg = -1;
     float wrow = 0.f;
     int nvis = 0, g = 0;
@@ -361,7 +376,12 @@ route_tc_kernel(const __grid_constant__ CUtensorMap means_map, const __grid_cons
       if (tid < p.H && !skip) {
         float sum = 0.f;
         for (int k2 = 0; k2 < p.qpm; ++k2) sum += red[k2 * p.H + tid];
-        p.partial[item * p.H + tid] = sum;
+        if constexpr (kCluster) acc += sum;
+        else p.partial[item * p.H + tid] = sum;
+      }
+      if constexpr (kCluster) {
+        named_bar_sync(1, kREpiThreads);  // red is reused by the next item
+        continue;
       }
       ++run_items;
       // last item of decision g in this CTA's range: count them in
@@ -389,12 +409,15 @@ route_tc_kernel(const __grid_constant__ CUtensorMap means_map, const __grid_cons
             imp[tid] = sum;
           }
           named_bar_sync(1, kREpiThreads);
-          if (warp == 0) select_top_h(imp, p.H, p.h, g, p.heads, p.importance);
+          select_top_h(imp, p.H, p.h, g, p.heads, p.importance, wcnt);
           if (tid == 0) p.counters[g] = 0u;  // ready for the next call
         }
         run_items = 0;
       }
       named_bar_sync(1, kREpiThreads);  // red / imp / flag are reused by the next item
+    }
+    if constexpr (kCluster) {
+      if (tid < p.H) imp[tid] = acc;
     }
   }
 
@@ -402,6 +425,21 @@ route_tc_kernel(const __grid_constant__ CUtensorMap means_map, const __grid_cons
   __syncthreads();
   tc_fence_after();
   if (warp == kRMmaWarp) tmem_dealloc(tmem_base, kRTmemCols);
+  if constexpr (kCluster) {
+    cg::cluster_group cl = cg::this_cluster();
+    cl.sync();  // every CTA's importances are complete
+    if (crank == 0 && warp < kREpiThreads / 32) {
+      if (tid < p.H) {
+        float sum = 0.f;
+        for (int c = 0; c < csize; ++c) sum += cl.map_shared_rank(imp, c)[tid];
+        imp2[tid] = sum;
+      }
+      named_bar_sync(1, kREpiThreads);
+      if (cdec < p.n_pg / pgs_per_dec + (p.n_pg % pgs_per_dec ? 1 : 0))
+        select_top_h(imp2, p.H, p.h, cdec, p.heads, p.importance, wcnt);
+    }
+    cl.sync();  // CTA 0 has read every CTA's importances
+  }
 }
 
 }  // namespace
@@ -449,19 +487,30 @@ cudaError_t launch_route_heads_tc(const uint16_t* q, const float* w, const float
   CUtensorMap qmap;
   if (!encode_2d_map(&qmap, true, q, kD, static_cast<uint64_t>(T) * H, kD * 2, 64, kRM, true))
     return cudaErrorInvalidValue;
+  const int sms = device_sm_count();
+  if (sms <= 0) return cudaErrorInvalidDevice;
+  // cluster mode when one wave of clusters covers the batch: D CTAs per
+  // decision, each with at most 8 items
+  const int G = (T + q_block - 1) / q_block;
+  const int64_t items_per_dec = static_cast<int64_t>(q_block / qpm) * p.n_bt;
+  const int D = static_cast<int>(items_per_dec < kRMaxCluster ? items_per_dec : kRMaxCluster);
+  const bool cluster = items_per_dec <= 8 * kRMaxCluster && static_cast<int64_t>(G) * D <= sms;
   cudaError_t e = cudaSuccess;
+  if (cluster) {
+    e = ensure_dynamic_smem(reinterpret_cast<const void*>(route_tc_kernel<true>), kRSmemBytes);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(route_tc_kernel<true>, dim3(static_cast<unsigned>(G * D)), dim3(kRThreads), kRSmemBytes, stream,
+                      D, map, qmap, p);
+  }
   if (clear_counters) {
-    const int G = (T + q_block - 1) / q_block;
     e = cudaMemsetAsync(counters, 0, static_cast<size_t>(G) * sizeof(unsigned), stream);
     if (e != cudaSuccess) return e;
   }
-  e = ensure_dynamic_smem(reinterpret_cast<const void*>(route_tc_kernel), kRSmemBytes);
+  e = ensure_dynamic_smem(reinterpret_cast<const void*>(route_tc_kernel<false>), kRSmemBytes);
   if (e != cudaSuccess) return e;
-  const int sms = device_sm_count();
-  if (sms <= 0) return cudaErrorInvalidDevice;
   const int64_t grid = p.n_items < sms ? p.n_items : sms;
-  return launch_pdl(route_tc_kernel, dim3(static_cast<unsigned>(grid)), dim3(kRThreads), kRSmemBytes, stream, 0, map,
-                    qmap, p);
+  return launch_pdl(route_tc_kernel<false>, dim3(static_cast<unsigned>(grid)), dim3(kRThreads), kRSmemBytes, stream, 0,
+                    map, qmap, p);
 }
 
 }  // namespace misa

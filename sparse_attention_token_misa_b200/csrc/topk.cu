@@ -9,22 +9,25 @@
 // (and NaN) never selected; the selected positions come out in ascending order,
 // -1 padded when the row holds fewer than k selectable entries.
 //
-// Rows of up to 40960 entries: one 1024-thread CTA per row keeps the whole
-// row in shared memory (topk_row_kernel; value-range histogram, a position
-// bitmap of the chosen entries, ascending output from its population counts).  Longer rows are split into CL
-// contiguous slices, one per CTA of a cluster of CL CTAs (CL = 2..8, by row
-// length; topk_cluster_kernel).  Scores become order-preserving uint32 keys,
-// kept in shared memory for the whole selection, so the row is read from
-// global memory exactly once.  The k-th largest key tau is found digit by
-// digit (12 + 10 + 10 bits): every CTA histograms the digit over its slice
-// (keys whose higher digits match the prefix found so far), the CL histograms
-// are summed through distributed shared memory (each CTA owns 1/CL of the
-// bins), every CTA pulls the summed histogram and finds the bin holding the
-// k-th key.  A final pass writes the selected positions: each warp owns a
-// contiguous chunk of its slice, warp ballots, a scan over the warps and the
-// per-CTA counts exchanged across the cluster give every selected entry its
-// output slot, so the output is in position order without a sort.  Keys equal to tau are taken lowest
-// position first, exactly as many as needed.
+// Rows of up to 131072 entries (topk_range_kernel): a cluster of up to 8 CTAs
+// per row, the row's entries held in registers, a value-range histogram whose
+// threshold bin is gathered across the cluster; described above the kernel.
+//
+// Longer rows (topk_cluster_kernel) are split into CL = 8 contiguous slices,
+// one per CTA of a cluster.  Scores become order-preserving uint32 keys
+// (re-read from global memory when a slice does not fit in shared memory).
+// The k-th largest key tau is found digit by digit (12 + 10 + 10 bits): every
+// CTA histograms the digit over its slice (keys whose higher digits match the
+// prefix found so far), the CL histograms are summed through distributed
+// shared memory (each CTA owns 1/CL of the bins), every CTA pulls the summed
+// histogram and finds the bin holding the k-th key.  A final pass writes the
+// selected positions: each warp owns a contiguous chunk of its slice, warp
+// ballots, a scan over the warps and the per-CTA counts exchanged across the
+// cluster give every selected entry its output slot, so the output is in
+// position order without a sort.
+//
+// In both kernels keys equal to tau are taken lowest position first, exactly
+// as many as needed.
 #include <cooperative_groups.h>
 
 #include "launch.h"
@@ -58,6 +61,8 @@ __device__ __forceinline__ bool selectable(float v) { return v == v && v > -__in
 
 // key of a score, 0 for entries that can never be selected
 __device__ __forceinline__ uint32_t sel_key(float v) { return selectable(v) ? float_key(v) : 0u; }
+
+__device__ __forceinline__ float valid_or_neg_inf(float v) { return selectable(v) ? v : -__int_as_float(0x7f800000); }
 
 __device__ __forceinline__ uint32_t block_sum(Smem& sm, uint32_t x) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -336,139 +341,165 @@ topk_cluster_kernel(const float* __restrict__ scores, int64_t n, int64_t row_str
 }
 
 // ---------------------------------------------------------------------------
-// One CTA per row, for rows that fit in shared memory (decode rows, candidate
-// lists, block scores): no cluster barriers.  Instead of bit digits (whose top
-// bits put most scores of a row into a handful of exponent bins, serialising the
-// shared-memory atomics) the first pass histograms the scores into 4096 equal
-// value ranges between the row's min and max, a monotone map, so the threshold
-// bin holds few entries.  Those candidates are collected with one atomic per
-// warp and the exact threshold among them is found by counting (few) or by a
-// bit-digit radix select over them (many).
-constexpr int kRowThreads = 1024;
-constexpr int kRowWarps = kRowThreads / 32;
-constexpr int kRowBins = 4096;
-constexpr int kRowMaxN = 40960;    // scores held in shared memory
-constexpr int kRowCandCap = 4096;  // entries of the threshold bin kept
-constexpr int kRowQuadCap = 1024;  // up to this many candidates: exact rank by counting
+// Rows of up to 8 x 512 x 32 entries: a cluster of CL <= 8 CTAs of 512
+// threads per row, each thread holding V contiguous entries of the row in
+// registers (V = 8, 16 or 32 by row length).  Instead of bit digits (whose top
+// bits put most scores of a row into a few exponent bins) the first histogram
+// splits the value range of a fixed sample of the row (the same 512 entries in
+// every CTA, so every CTA derives the same bins) into 2048 equal ranges; the
+// map is monotone, values outside the sample's range go to the end bins.
+// The threshold bin is located from the CL histograms in two rounds of
+// distributed shared memory reads (64 super-bin totals, then the 32 bins of
+// the chosen super-bin), its entries (few) are gathered from every CTA and the
+// exact threshold among them is found by counting.  Every CTA then knows how
+// many entries above and equal to the threshold each slice holds, so the
+// output slots follow from a scan: two cluster barriers on this path.  A
+// threshold bin too full to gather (massive ties, a sample range spoilt by
+// outliers) falls back to a cluster-wide bit-digit radix select inside it.
+constexpr int kXThreads = 512;
+constexpr int kXWarps = kXThreads / 32;
+constexpr int kXBins = 2048;          // value-range bins = 64 super-bins x 32
+constexpr int kXSup = kXBins / 32;
+constexpr int kXCandCap = 512;        // threshold-bin entries kept per CTA
+constexpr int kXMergeCap = 2048;      // and over the cluster
+constexpr int kXMaxV = 32;
 
-struct RowSmem {
-  uint32_t hist[kRowBins];
-  float cval[kRowCandCap];
-  int32_t cpos[kRowCandCap];
-  uint32_t warp_u[kRowWarps];
-  float warp_f[2][kRowWarps];
-  uint32_t bcast[8];
-  float fcast[4];
-  uint32_t ccount;
+struct XSmem {
+  uint32_t hist[kXBins];     // this CTA's histogram (read by the cluster)
+  uint32_t sup[kXSup];       // its super-bin totals (read by the cluster)
+  uint32_t meta[4];          // valid entries, entries above the threshold bin, threshold-bin entries (read by the cluster)
+  uint32_t cnt2[2];          // fallback: entries above / equal to tau (read by the cluster)
+  uint32_t gsup[kXSup];      // super-bin totals summed over the cluster
+  uint32_t gbin[32];
+  uint32_t bc[4];
+  float fbc;
+  uint32_t rv[kMaxCluster], ra[kMaxCluster], rc[kMaxCluster];
+  uint32_t at[kMaxCluster], et[kMaxCluster];
+  float wmin[kXWarps], wmax[kXWarps];
+  uint64_t wscan[kXWarps];
+  union {
+    struct {
+      float cval[kXCandCap];     // this CTA's threshold-bin entries (read by the cluster)
+      float mval[kXMergeCap];    // all of the cluster's, by rank
+      uint8_t mrank[kXMergeCap];
+    } c;
+    struct {
+      uint32_t h[kXBins];        // fallback digit histogram, second buffer (read by the cluster)
+      uint32_t s[kXSup];
+    } r;
+  } u;
 };
-constexpr size_t kRowValsOff = (sizeof(RowSmem) + 15) / 16 * 16;
 
-__device__ __forceinline__ float valid_or_neg_inf(float v) { return selectable(v) ? v : -__int_as_float(0x7f800000); }
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 
-__device__ __forceinline__ uint32_t row_sum_u32(RowSmem& sm, uint32_t x) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-  if (lane == 0) sm.warp_u[warp] = x;
-  __syncthreads();
-  uint32_t s = 0;
-  for (int i = 0; i < kRowWarps; ++i) s += sm.warp_u[i];
-  __syncthreads();
-  return s;
-}
-
-// bin b of hist[0, nbins) with sum(hist[b+1..]) < need <= sum(hist[b..])
-__device__ __forceinline__ int row_find_bin(RowSmem& sm, int nbins, uint32_t need, uint32_t* above) {
-  const int per = nbins / kRowThreads;
-  const int b0 = threadIdx.x * per;
+// One warp: among tot[0, cnt) (cnt <= 128) the index i with
+// above(i) < need <= above(i) + tot[i], above(i) = sum of tot[i+1 .. cnt);
+// out[0] = i, out[1] = above(i).
+__device__ __forceinline__ void warp_suffix_find(const uint32_t* tot, int cnt, uint32_t need, uint32_t* out) {
+  const int lane = threadIdx.x & 31;
+  const int per = (cnt + 31) / 32;
+  const int b0 = lane * per;
   uint32_t local = 0;
-  for (int i = 0; i < per; ++i) local += sm.hist[b0 + i];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint32_t inc = local;
+  for (int i = 0; i < per; ++i)
+    if (b0 + i < cnt) local += tot[b0 + i];
+  uint32_t inc = local;  // sum over lanes >= this one
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const uint32_t y = __shfl_down_sync(0xffffffffu, inc, o);
     if (lane + o < 32) inc += y;
   }
-  if (lane == 0) sm.warp_u[warp] = inc;
-  __syncthreads();
-  if (warp == 0) {
-    const uint32_t tw = sm.warp_u[lane];
-    uint32_t ti = tw;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_down_sync(0xffffffffu, ti, o);
-      if (lane + o < 32) ti += y;
-    }
-    sm.warp_u[lane] = ti - tw;
-  }
-  __syncthreads();
-  const uint32_t after = sm.warp_u[warp] + inc - local;
-  if (after < need && after + local >= need) {
+  const uint32_t after = inc - local;
+  if (after < need && need <= inc) {
     uint32_t acc = after;
     for (int i = per - 1; i >= 0; --i) {
-      const uint32_t c = sm.hist[b0 + i];
+      if (b0 + i >= cnt) continue;
+      const uint32_t c = tot[b0 + i];
       if (acc + c >= need) {
-        sm.bcast[0] = static_cast<uint32_t>(b0 + i);
-        sm.bcast[1] = acc;
+        out[0] = static_cast<uint32_t>(b0 + i);
+        out[1] = acc;
         break;
       }
       acc += c;
     }
   }
-  __syncthreads();
-  const int bin = static_cast<int>(sm.bcast[0]);
-  *above = sm.bcast[1];
-  __syncthreads();
-  return bin;
 }
 
-// Radix select (12 + 10 + 10 key bits) of the need-th largest key among the
-// entries i < cnt of `src` for which in_set(v) holds; returns its key and sets
-// *gt = number of those entries with a larger key.
-template <class Src, class InSet>
-__device__ uint32_t row_radix_select(RowSmem& sm, Src src, int cnt, InSet in_set, uint32_t need, uint32_t* gt) {
-  uint32_t prefix = 0, above = 0;
-  const int shift[3] = {20, 10, 0};
-  const uint32_t mask[3] = {0xfffu, 0x3ffu, 0x3ffu};
-  for (int round = 0; round < 3; ++round) {
-    const int nb = round == 0 ? kRowBins : 1024;
-    for (int i = threadIdx.x; i < nb; i += kRowThreads) sm.hist[i] = 0;
-    __syncthreads();
-    for (int i = threadIdx.x; i < cnt; i += kRowThreads) {
-      const float v = src(i);
-      if (!in_set(v)) continue;
-      const uint32_t kk = float_key(v);
-      const bool match = round == 0 || (kk >> (shift[round - 1])) == prefix;
-      if (match) atomicAdd(&sm.hist[(kk >> shift[round]) & mask[round]], 1u);
-    }
-    __syncthreads();
-    uint32_t a;
-    const int b = row_find_bin(sm, nb, need, &a);
-    above += a;
-    need -= a;
-    prefix = round == 0 ? static_cast<uint32_t>(b) : ((prefix << 10) | static_cast<uint32_t>(b));
+// Super-bin totals of a histogram of nbins (a multiple of 128, <= 2048): each
+// thread adds 4 bins, 8 lanes make one super-bin of 32.
+__device__ __forceinline__ void make_supers(const uint32_t* h, uint32_t* sup, int nbins) {
+  const int base = threadIdx.x * 4;
+  if (base < nbins) {  // whole warps
+    const uint4 x = *reinterpret_cast<const uint4*>(h + base);
+    uint32_t s = x.x + x.y + x.z + x.w;
+    s += __shfl_xor_sync(0xffffffffu, s, 1);
+    s += __shfl_xor_sync(0xffffffffu, s, 2);
+    s += __shfl_xor_sync(0xffffffffu, s, 4);
+    if ((threadIdx.x & 7) == 0) sup[base / 32] = s;
   }
-  *gt = above;
-  return prefix;
 }
+
+// The bin holding the need-th largest entry of the histogram summed over nsrc
+// sources (hist_of(r), sup_of(r): source r's bins and super-bin totals, all
+// complete); *above = entries in higher bins.  Every thread of the CTA calls.
+template <class HistOf, class SupOf>
+__device__ int two_level_find(XSmem& sm, int nsrc, HistOf hist_of, SupOf sup_of, int nsup, uint32_t need,
+                              uint32_t* above) {
+  const int tid = threadIdx.x;
+  for (int i = tid; i < nsup; i += kXThreads) sm.gsup[i] = 0;
+  if (tid < 32) sm.gbin[tid] = 0;
+  __syncthreads();
+  for (int i = tid; i < nsup * nsrc; i += kXThreads) {
+    const int s = i % nsup, r = i / nsup;
+    atomicAdd(&sm.gsup[s], sup_of(r)[s]);
+  }
+  __syncthreads();
+  if (tid < 32) warp_suffix_find(sm.gsup, nsup, need, sm.bc);
+  __syncthreads();
+  // (the index is in range by construction; the clamps only keep a wrong
+  // count from addressing outside the arrays)
+  const int S = sm.bc[0] < static_cast<uint32_t>(nsup) ? static_cast<int>(sm.bc[0]) : nsup - 1;
+  const uint32_t above_s = sm.bc[1];
+  for (int i = tid; i < 32 * nsrc; i += kXThreads) {
+    const int j = i & 31, r = i >> 5;
+    atomicAdd(&sm.gbin[j], hist_of(r)[S * 32 + j]);
+  }
+  __syncthreads();
+  if (tid < 32) warp_suffix_find(sm.gbin, 32, need - above_s, sm.bc + 2);
+  __syncthreads();
+  *above = above_s + sm.bc[3];
+  return S * 32 + static_cast<int>(sm.bc[2] & 31u);
+}
+
+// Bit digits of a key for the radix rounds: 11, 11, 10 bits from the top.
+__device__ __forceinline__ int digit_shift(int round) { return round == 0 ? 21 : (round == 1 ? 10 : 0); }
+__device__ __forceinline__ int digit_bins(int round) { return round == 2 ? 1024 : 2048; }
 
 __device__ __forceinline__ float key_to_float(uint32_t kk) {
   const uint32_t u = (kk & 0x80000000u) ? (kk ^ 0x80000000u) : ~kk;
   return __uint_as_float(u);
 }
 
-__global__ void __launch_bounds__(kRowThreads, 1)
-topk_row_kernel(const float* __restrict__ scores, int64_t n, int64_t row_stride, const int32_t* __restrict__ row_valid,
-                const int32_t* __restrict__ id_map, int64_t id_map_stride, int k, int32_t* __restrict__ idx) {
+template <int V>
+__global__ void __launch_bounds__(kXThreads, V >= 32 ? 1 : 2)
+topk_range_kernel(const float* __restrict__ scores, int64_t n, int64_t row_stride, const int32_t* __restrict__ row_valid,
+                  const int32_t* __restrict__ id_map, int64_t id_map_stride, int k, int32_t* __restrict__ idx) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  RowSmem& sm = *reinterpret_cast<RowSmem*>(smem_raw);
-  float* vals = reinterpret_cast<float*>(smem_raw + kRowValsOff);
+  XSmem& sm = *reinterpret_cast<XSmem*>(smem_raw);
+  cg::cluster_group cl = cg::this_cluster();
+  const int CL = static_cast<int>(cl.num_blocks());
+  const int rank = static_cast<int>(cl.block_rank());
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t t = blockIdx.y;
+  constexpr int kSlice = kXThreads * V;
   const float kNegInf = -__int_as_float(0x7f800000);
-  const int64_t t = blockIdx.x;
+  const float kPosInf = __int_as_float(0x7f800000);
+
+  for (int i = tid; i < kXBins; i += kXThreads) sm.hist[i] = 0;
+  if (tid < 4) sm.meta[tid] = 0;
   pdl_wait_inputs();
   pdl_allow_next();
+
   const float* row = scores + t * row_stride;
   const int32_t* idrow = id_map ? id_map + t * id_map_stride : nullptr;
   int32_t* out = idx + t * k;
@@ -478,245 +509,295 @@ topk_row_kernel(const float* __restrict__ scores, int64_t n, int64_t row_stride,
     nt64 = rv < 0 ? 0 : (rv < n ? rv : n);
   }
   const int nt = static_cast<int>(nt64);
-  const int nwords = (nt + 31) / 32;
-  uint32_t* bitmap = reinterpret_cast<uint32_t*>(vals + (nt + 3) / 4 * 4);  // 1 bit per position
+  const int s0 = rank * kSlice < nt ? rank * kSlice : nt;
+  const int s1 = s0 + kSlice < nt ? s0 + kSlice : nt;
+  const int p0 = s0 + tid * V;  // this thread's entries: positions [p0, p0 + V) of the row
 
-  for (int i = tid; i < kRowBins; i += kRowThreads) sm.hist[i] = 0;
-  if (tid == 0) sm.ccount = 0;
-
-  // ---------------- pass A: load the row once; the value range of a sample
-  // (each thread's first 16 bytes) sets the histogram's bins (values outside
-  // it go to the end bins, which keeps the map monotone)
-  const int nv = nt / 4;
-  const float4* r4 = reinterpret_cast<const float4*>(row);
-  constexpr int kPer = kRowMaxN / 4 / kRowThreads;  // float4 per thread at most (10)
-  float4 f[kPer];
+  // ---------------- load (the slice start and p0 are multiples of 4 entries)
+  float v[V];
 #pragma unroll
-  for (int u = 0; u < kPer; ++u) {
-    const int i = tid + u * kRowThreads;
-    f[u] = i < nv ? __ldg(r4 + i) : make_float4(kNegInf, kNegInf, kNegInf, kNegInf);
-  }
-  float smax = kNegInf, smin = __int_as_float(0x7f800000);
-  {
-    const float e[4] = {valid_or_neg_inf(f[0].x), valid_or_neg_inf(f[0].y), valid_or_neg_inf(f[0].z),
-                        valid_or_neg_inf(f[0].w)};
+  for (int j = 0; j < V; j += 4) {
+    const int p = p0 + j;
+    if (p + 3 < s1) {
+      const float4 f = __ldg(reinterpret_cast<const float4*>(row + p));
+      v[j] = f.x;
+      v[j + 1] = f.y;
+      v[j + 2] = f.z;
+      v[j + 3] = f.w;
+    } else {
 #pragma unroll
-    for (int c = 0; c < 4; ++c)
-      if (e[c] > kNegInf) {
-        smax = fmaxf(smax, e[c]);
-        smin = fminf(smin, e[c]);
-      }
-  }
-  if (tid == 0)  // short rows: the scalar tail is part of the sample
-    for (int i = 4 * nv; i < nt; ++i) {
-      const float v = valid_or_neg_inf(__ldg(row + i));
-      if (v > kNegInf) {
-        smax = fmaxf(smax, v);
-        smin = fminf(smin, v);
-      }
+      for (int c = 0; c < 4; ++c) v[j + c] = p + c < s1 ? __ldg(row + p + c) : kNegInf;
     }
+  }
+  float smp = nt > 0 ? __ldg(row + static_cast<int64_t>(tid) * nt / kXThreads) : kNegInf;
+  smp = valid_or_neg_inf(smp);
+  float mx = smp, mn = smp > kNegInf ? smp : kPosInf;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
-    smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, o));
-    smin = fminf(smin, __shfl_xor_sync(0xffffffffu, smin, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
   }
   if (lane == 0) {
-    sm.warp_f[0][warp] = smax;
-    sm.warp_f[1][warp] = smin;
+    sm.wmax[warp] = mx;
+    sm.wmin[warp] = mn;
   }
   __syncthreads();
-  smax = sm.warp_f[0][0];
-  smin = sm.warp_f[1][0];
-  for (int i = 1; i < kRowWarps; ++i) {
-    smax = fmaxf(smax, sm.warp_f[0][i]);
-    smin = fminf(smin, sm.warp_f[1][i]);
+  mx = sm.wmax[0];
+  mn = sm.wmin[0];
+#pragma unroll
+  for (int i = 1; i < kXWarps; ++i) {
+    mx = fmaxf(mx, sm.wmax[i]);
+    mn = fminf(mn, sm.wmin[i]);
   }
-  const float range = smax - smin;
-  const float scale = (range > 0.f && range < __int_as_float(0x7f800000)) ? static_cast<float>(kRowBins) / range : 0.f;
-  // monotone in v; any NaN intermediate (no valid sample, infinite values) maps to bin 0
-  auto bin_of = [&](float v) -> int {
-    const float x = (v - smin) * scale;
-    return x > 0.f ? (x >= static_cast<float>(kRowBins - 1) ? kRowBins - 1 : static_cast<int>(x)) : 0;
+  const float range = mx - mn;
+  const float scale = (range > 0.f && range < kPosInf) ? static_cast<float>(kXBins) / range : 0.f;
+  // monotone in x; a NaN intermediate (no valid sample, infinite entries) maps to bin 0
+  auto bin_of = [&](float x) -> int {
+    const float y = __fmul_rn(__fsub_rn(x, mn), scale);
+    return y > 0.f ? (y >= static_cast<float>(kXBins - 1) ? kXBins - 1 : static_cast<int>(y)) : 0;
   };
-  uint32_t nvalid = 0;
-#pragma unroll
-  for (int u = 0; u < kPer; ++u) {
-    const int i = tid + u * kRowThreads;
-    if (i < nv) {
-      const float4 g = make_float4(valid_or_neg_inf(f[u].x), valid_or_neg_inf(f[u].y), valid_or_neg_inf(f[u].z),
-                                   valid_or_neg_inf(f[u].w));
-      *reinterpret_cast<float4*>(&vals[4 * i]) = g;
-      const float e[4] = {g.x, g.y, g.z, g.w};
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-        if (e[c] > kNegInf) {
-          atomicAdd(&sm.hist[bin_of(e[c])], 1u);
-          ++nvalid;
-        }
-    }
-  }
-  for (int i = 4 * nv + tid; i < nt; i += kRowThreads) {
-    const float v = valid_or_neg_inf(__ldg(row + i));
-    vals[i] = v;
-    if (v > kNegInf) {
-      atomicAdd(&sm.hist[bin_of(v)], 1u);
-      ++nvalid;
-    }
-  }
-  const uint32_t total = row_sum_u32(sm, nvalid);  // (synchronises)
 
-  // ---------------- threshold bin, then pass B: one sweep sets the bitmap of
-  // every entry above the threshold bin (warp ballots, one word per step) and
-  // collects the threshold bin's entries as candidates
-  int b1 = -1;
-  uint32_t need = 0;
-  if (total > static_cast<uint32_t>(k)) {
-    uint32_t gt1;
-    b1 = row_find_bin(sm, kRowBins, static_cast<uint32_t>(k), &gt1);
-    need = static_cast<uint32_t>(k) - gt1;
-  }
-  const uint32_t nb1 = b1 >= 0 ? sm.hist[b1] : 0u;
-  const bool keep_cand = nb1 <= static_cast<uint32_t>(kRowCandCap);
-  for (int w = warp; w < nwords; w += kRowWarps) {
-    const int i = w * 32 + lane;
-    const float v = i < nt ? vals[i] : kNegInf;
-    const bool valid = v > kNegInf;
-    const int b = valid ? bin_of(v) : -1;
-    const uint32_t above = __ballot_sync(0xffffffffu, valid && b > b1);
-    const uint32_t inbin = __ballot_sync(0xffffffffu, valid && b == b1);
-    if (lane == 0) bitmap[w] = above;
-    if (keep_cand && inbin) {
-      uint32_t base = 0;
-      if (lane == 0) base = atomicAdd(&sm.ccount, static_cast<uint32_t>(__popc(inbin)));
-      base = __shfl_sync(0xffffffffu, base, 0);
-      if ((inbin >> lane) & 1u) {
-        const uint32_t slot = base + __popc(inbin & ((1u << lane) - 1u));
-        sm.cval[slot] = v;
-        sm.cpos[slot] = i;
-      }
+  // ---------------- value-range histogram of the slice
+  uint32_t nval = 0;
+#pragma unroll
+  for (int j = 0; j < V; ++j) {
+    v[j] = valid_or_neg_inf(v[j]);
+    if (v[j] > kNegInf) {
+      atomicAdd(&sm.hist[bin_of(v[j])], 1u);
+      ++nval;
     }
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) nval += __shfl_xor_sync(0xffffffffu, nval, o);
+  if (lane == 0 && nval) atomicAdd(&sm.meta[0], nval);
   __syncthreads();
+  make_supers(sm.hist, sm.sup, kXBins);
+  __syncthreads();
+  cl.sync();  // (1) every CTA's histogram, super-bins and valid count are complete
 
-  if (b1 >= 0) {
-    // ---------------- exact threshold tau inside bin b1, and how many entries
-    // equal to tau are taken (the lowest positions)
-    float tau;
-    uint32_t need_eq;
-    if (nb1 <= static_cast<uint32_t>(kRowQuadCap)) {
-      const int c = static_cast<int>(nb1);
-      if (tid < c) {
-        const float v = sm.cval[tid];
-        uint32_t g = 0, ge = 0;
-        for (int j = 0; j < c; ++j) {
-          const float u = sm.cval[j];
-          g += u > v ? 1u : 0u;
-          ge += u >= v ? 1u : 0u;
-        }
-        if (g < need && need <= ge) {
-          sm.fcast[0] = v;
-          sm.bcast[2] = need - g;
-        }
-      }
-      __syncthreads();
-      tau = sm.fcast[0];
-      need_eq = sm.bcast[2];
-    } else {
-      uint32_t gt, kk;
-      if (keep_cand)
-        kk = row_radix_select(sm, [&](int i) { return sm.cval[i]; }, static_cast<int>(nb1), [](float) { return true; },
-                              need, &gt);
-      else
-        kk = row_radix_select(sm, [&](int i) { return vals[i]; }, nt,
-                              [&](float v) { return v > kNegInf && bin_of(v) == b1; }, need, &gt);
-      tau = key_to_float(kk);
-      need_eq = need - gt;
-    }
-    // ---------------- mark the chosen entries of bin b1 in the bitmap
-    if (keep_cand) {
-      const int c = static_cast<int>(nb1);
-      for (int x = tid; x < c; x += kRowThreads) {
-        const float v = sm.cval[x];
-        bool take = v > tau;
-        if (!take && v == tau) {  // rank among the equal entries by position
-          const int p = sm.cpos[x];
-          uint32_t r = 0;
-          for (int j = 0; j < c; ++j) r += (sm.cval[j] == tau && sm.cpos[j] < p) ? 1u : 0u;
-          take = r < need_eq;
-        }
-        if (take) atomicOr(&bitmap[sm.cpos[x] >> 5], 1u << (sm.cpos[x] & 31));
-      }
-    } else {
-      // the bin is too large to keep: sweep it in position order
-      uint32_t eq_before = 0;
-      for (int w0 = 0; w0 < nwords; w0 += kRowWarps) {
-        const int w = w0 + warp;
-        const int i = w * 32 + lane;
-        const float v = (w < nwords && i < nt) ? vals[i] : kNegInf;
-        const bool inb = v > kNegInf && bin_of(v) == b1;
-        const bool gtt = inb && v > tau;
-        const bool eqt = inb && v == tau;
-        const uint32_t beq = __ballot_sync(0xffffffffu, eqt);
-        if (lane == 0) sm.warp_u[warp] = __popc(beq);
-        __syncthreads();
-        uint32_t before_w = eq_before, tot_w = 0;
-        for (int j = 0; j < kRowWarps; ++j) {
-          if (j < warp) before_w += sm.warp_u[j];
-          tot_w += sm.warp_u[j];
-        }
-        const uint32_t my_rank = before_w + __popc(beq & ((1u << lane) - 1u));
-        const bool take = gtt || (eqt && my_rank < need_eq);
-        const uint32_t bt = __ballot_sync(0xffffffffu, take);
-        if (lane == 0 && w < nwords && bt) bitmap[w] |= bt;
-        eq_before += tot_w;
-        __syncthreads();
-      }
+  if (tid < CL) sm.rv[tid] = cl.map_shared_rank(&sm.meta[0], tid)[0];
+  __syncthreads();
+  uint32_t total = 0;
+  for (int r = 0; r < CL; ++r) total += sm.rv[r];
+
+  float tau = kNegInf;  // selected: entries above tau, and the first need_eq entries equal to it
+  uint32_t need_eq = 0;
+  if (total <= static_cast<uint32_t>(k)) {
+    if (tid < CL) {
+      sm.at[tid] = sm.rv[tid];
+      sm.et[tid] = 0;
     }
   } else {
-    // every valid entry is chosen: the whole bitmap is "above" already (b1 = -1)
+    uint32_t above_b;
+    const int bstar = two_level_find(
+        sm, CL, [&](int r) { return cl.map_shared_rank(&sm.hist[0], r); },
+        [&](int r) { return cl.map_shared_rank(&sm.sup[0], r); }, kXSup, static_cast<uint32_t>(k), &above_b);
+    const uint32_t need = static_cast<uint32_t>(k) - above_b;
+    // entries above the threshold bin, and the threshold bin's entries
+    uint32_t a = 0;
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+      if (v[j] > kNegInf) {
+        const int b = bin_of(v[j]);
+        a += b > bstar ? 1u : 0u;
+        if (b == bstar) {
+          const uint32_t slot = atomicAdd(&sm.meta[2], 1u);
+          if (slot < static_cast<uint32_t>(kXCandCap)) sm.u.c.cval[slot] = v[j];
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+    if (lane == 0 && a) atomicAdd(&sm.meta[1], a);
+    __syncthreads();
+    cl.sync();  // (2) every CTA's counts and threshold-bin entries are complete
+    if (tid < CL) {
+      const uint32_t* m = cl.map_shared_rank(&sm.meta[0], tid);
+      sm.ra[tid] = m[1];
+      sm.rc[tid] = m[2];
+    }
+    __syncthreads();
+    uint32_t ctot = 0;
+    bool overflow = false;
+    for (int r = 0; r < CL; ++r) {
+      ctot += sm.rc[r];
+      overflow |= sm.rc[r] > static_cast<uint32_t>(kXCandCap);
+    }
+    overflow |= ctot > static_cast<uint32_t>(kXMergeCap);
+    if (!overflow) {
+      // ---------------- gather the threshold bin from the cluster
+      for (int i = tid; i < static_cast<int>(ctot); i += kXThreads) {
+        int r = 0;
+        uint32_t off = 0;
+        while (off + sm.rc[r] <= static_cast<uint32_t>(i)) off += sm.rc[r++];
+        sm.u.c.mval[i] = cl.map_shared_rank(&sm.u.c.cval[0], r)[i - off];
+        sm.u.c.mrank[i] = static_cast<uint8_t>(r);
+      }
+      __syncthreads();
+      if (ctot <= static_cast<uint32_t>(kXThreads)) {
+        // exact rank by counting
+        if (tid < static_cast<int>(ctot)) {
+          const float x = sm.u.c.mval[tid];
+          uint32_t g = 0, ge = 0;
+          for (int j = 0; j < static_cast<int>(ctot); ++j) {
+            const float y = sm.u.c.mval[j];
+            g += y > x ? 1u : 0u;
+            ge += y >= x ? 1u : 0u;
+          }
+          if (g < need && need <= ge) {
+            sm.fbc = x;
+            sm.bc[0] = need - g;
+          }
+        }
+        __syncthreads();
+        tau = sm.fbc;
+        need_eq = sm.bc[0];
+      } else {
+        // bit-digit radix select over the gathered entries (local; the
+        // histogram arrays are no longer read by the cluster after (2))
+        uint32_t prefix = 0, gt = 0, nd = need;
+        for (int round = 0; round < 3; ++round) {
+          const int sh = digit_shift(round), nb = digit_bins(round);
+          for (int i = tid; i < nb; i += kXThreads) sm.hist[i] = 0;
+          __syncthreads();
+          for (int i = tid; i < static_cast<int>(ctot); i += kXThreads) {
+            const uint32_t kk = float_key(sm.u.c.mval[i]);
+            if (round == 0 || (kk >> digit_shift(round - 1)) == prefix) atomicAdd(&sm.hist[(kk >> sh) & (nb - 1)], 1u);
+          }
+          __syncthreads();
+          make_supers(sm.hist, sm.sup, nb);
+          __syncthreads();
+          uint32_t ab;
+          const int b = two_level_find(
+              sm, 1, [&](int) { return &sm.hist[0]; }, [&](int) { return &sm.sup[0]; }, nb / 32, nd, &ab);
+          gt += ab;
+          nd -= ab;
+          prefix = round == 0 ? static_cast<uint32_t>(b) : ((prefix << (round == 1 ? 11 : 10)) | static_cast<uint32_t>(b));
+        }
+        tau = key_to_float(prefix);
+        need_eq = nd;
+      }
+      // entries above / equal to tau in every slice
+      if (tid < CL) {
+        sm.at[tid] = sm.ra[tid];
+        sm.et[tid] = 0;
+      }
+      __syncthreads();
+      for (int i = tid; i < static_cast<int>(ctot); i += kXThreads) {
+        const float x = sm.u.c.mval[i];
+        if (x > tau) atomicAdd(&sm.at[sm.u.c.mrank[i]], 1u);
+        else if (x == tau) atomicAdd(&sm.et[sm.u.c.mrank[i]], 1u);
+      }
+    } else {
+      // ---------------- fallback: cluster-wide radix select inside bin bstar.
+      // Digit histograms alternate between two buffers, so a CTA never
+      // overwrites one that another CTA may still be reading.
+      uint32_t prefix = 0, gt = 0, nd = need;
+      for (int round = 0; round < 3; ++round) {
+        uint32_t* H = (round & 1) ? sm.u.r.h : sm.hist;
+        uint32_t* S = (round & 1) ? sm.u.r.s : sm.sup;
+        const int sh = digit_shift(round), nb = digit_bins(round);
+        for (int i = tid; i < nb; i += kXThreads) H[i] = 0;
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+          if (v[j] > kNegInf && bin_of(v[j]) == bstar) {
+            const uint32_t kk = float_key(v[j]);
+            if (round == 0 || (kk >> digit_shift(round - 1)) == prefix) atomicAdd(&H[(kk >> sh) & (nb - 1)], 1u);
+          }
+        }
+        __syncthreads();
+        make_supers(H, S, nb);
+        __syncthreads();
+        cl.sync();
+        uint32_t ab;
+        const int b = two_level_find(
+            sm, CL, [&](int r) { return cl.map_shared_rank(H, r); }, [&](int r) { return cl.map_shared_rank(S, r); },
+            nb / 32, nd, &ab);
+        gt += ab;
+        nd -= ab;
+        prefix = round == 0 ? static_cast<uint32_t>(b) : ((prefix << (round == 1 ? 11 : 10)) | static_cast<uint32_t>(b));
+      }
+      tau = key_to_float(prefix);
+      need_eq = nd;
+      uint32_t ac = 0, ec = 0;
+#pragma unroll
+      for (int j = 0; j < V; ++j) {
+        ac += v[j] > tau ? 1u : 0u;
+        ec += (v[j] > kNegInf && v[j] == tau) ? 1u : 0u;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        ac += __shfl_xor_sync(0xffffffffu, ac, o);
+        ec += __shfl_xor_sync(0xffffffffu, ec, o);
+      }
+      if (tid < 2) sm.cnt2[tid] = 0;
+      __syncthreads();
+      if (lane == 0) {
+        atomicAdd(&sm.cnt2[0], ac);
+        atomicAdd(&sm.cnt2[1], ec);
+      }
+      __syncthreads();
+      cl.sync();
+      if (tid < CL) {
+        const uint32_t* c2 = cl.map_shared_rank(&sm.cnt2[0], tid);
+        sm.at[tid] = c2[0];
+        sm.et[tid] = c2[1];
+      }
+    }
   }
   __syncthreads();
+  // this CTA reads no other CTA's shared memory after this point
+  cluster_arrive();
 
-  // ---------------- output: positions of the set bits, ascending (one word
-  // per thread step, block-wide prefix over the words' population counts)
-  uint32_t base = 0;
-  for (int w0 = 0; w0 < nwords; w0 += kRowThreads) {
-    const int w = w0 + tid;
-    const uint32_t bits = w < nwords ? bitmap[w] : 0u;
-    const uint32_t cnt = __popc(bits);
-    uint32_t inc = cnt;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
-      if (lane >= o) inc += y;
+  // ---------------- output slots: entries above tau before this one, plus the
+  // equal entries before it (at most need_eq of them)
+  uint32_t a_before = 0, e_before = 0, a_all = 0, e_all = 0;
+  for (int r = 0; r < CL; ++r) {
+    if (r < rank) {
+      a_before += sm.at[r];
+      e_before += sm.et[r];
     }
-    if (lane == 31) sm.warp_u[warp] = inc;
-    __syncthreads();
-    if (warp == 0) {
-      const uint32_t tw = sm.warp_u[lane];
-      uint32_t ti = tw;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, ti, o);
-        if (lane >= o) ti += y;
-      }
-      sm.warp_u[lane] = ti - tw;
-      if (lane == 31) sm.bcast[3] = ti;
-    }
-    __syncthreads();
-    uint32_t slot = base + sm.warp_u[warp] + inc - cnt;
-    uint32_t b = bits;
-    while (b) {
-      const int bit = __ffs(b) - 1;
-      b &= b - 1;
-      const int pos = w * 32 + bit;
-      if (slot < static_cast<uint32_t>(k)) out[slot] = idrow ? idrow[pos] : pos;
-      ++slot;
-    }
-    base += sm.bcast[3];
-    __syncthreads();
+    a_all += sm.at[r];
+    e_all += sm.et[r];
   }
-  for (uint32_t i = base + tid; i < static_cast<uint32_t>(k); i += kRowThreads) out[i] = -1;
+  uint32_t a_t = 0, e_t = 0;
+#pragma unroll
+  for (int j = 0; j < V; ++j) {
+    a_t += v[j] > tau ? 1u : 0u;
+    e_t += (v[j] > kNegInf && v[j] == tau) ? 1u : 0u;
+  }
+  uint64_t x = static_cast<uint64_t>(a_t) | (static_cast<uint64_t>(e_t) << 32);
+  uint64_t inc = x;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint64_t y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  if (lane == 31) sm.wscan[warp] = inc;
+  __syncthreads();
+  uint64_t wbase = 0;
+  for (int i = 0; i < warp; ++i) wbase += sm.wscan[i];
+  const uint64_t excl = wbase + inc - x;
+  uint32_t A = a_before + static_cast<uint32_t>(excl & 0xffffffffull);
+  uint32_t E = e_before + static_cast<uint32_t>(excl >> 32);
+#pragma unroll
+  for (int j = 0; j < V; ++j) {
+    const float y = v[j];
+    if (y > tau) {
+      const uint32_t slot = A + (E < need_eq ? E : need_eq);
+      if (slot < static_cast<uint32_t>(k)) out[slot] = idrow ? idrow[p0 + j] : p0 + j;
+      ++A;
+    } else if (y > kNegInf && y == tau) {
+      if (E < need_eq && A + E < static_cast<uint32_t>(k)) out[A + E] = idrow ? idrow[p0 + j] : p0 + j;
+      ++E;
+    }
+  }
+  if (rank == CL - 1) {
+    const uint32_t chosen = a_all + (e_all < need_eq ? e_all : need_eq);
+    for (uint32_t i = chosen + tid; i < static_cast<uint32_t>(k); i += kXThreads) out[i] = -1;
+  }
+  cluster_wait();  // no CTA exits while another may still read its shared memory
 }
 
 int pick_cluster(int64_t n) {
@@ -731,14 +812,22 @@ size_t topk_smem_bytes() { return kKeysOff + static_cast<size_t>(kSliceCap) * 4;
 
 cudaError_t launch_topk(const float* scores, int T, int64_t n, int64_t row_stride, const int32_t* row_valid,
                         const int32_t* id_map, int64_t id_map_stride, int k, int32_t* idx, cudaStream_t stream) {
-  if (n <= kRowMaxN) {
-    // the row's values, then a bitmap of n bits
-    auto row_smem = [](int64_t m) { return kRowValsOff + static_cast<size_t>((m + 3) / 4 * 4) * 4 + ((m + 31) / 32) * 4; };
-    const size_t smem = row_smem(n);
-    cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(topk_row_kernel), static_cast<int>(row_smem(kRowMaxN)));
-    if (e != cudaSuccess) return e;
-    return launch_pdl(topk_row_kernel, dim3(T), dim3(kRowThreads), smem, stream, 0, scores, n, row_stride, row_valid,
-                      id_map, id_map_stride, k, idx);
+  if (n <= static_cast<int64_t>(kMaxCluster) * kXThreads * kXMaxV) {
+    // smallest V with ceil(n / (512 V)) <= 8 CTAs per row
+    const int V = n <= static_cast<int64_t>(kMaxCluster) * kXThreads * 8 ? 8
+                  : (n <= static_cast<int64_t>(kMaxCluster) * kXThreads * 16 ? 16 : 32);
+    const int64_t slice = static_cast<int64_t>(kXThreads) * V;
+    const int CL = static_cast<int>((n + slice - 1) / slice);
+    const size_t smem = sizeof(XSmem);
+    auto go = [&](auto kern) -> cudaError_t {
+      cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
+      if (e != cudaSuccess) return e;
+      return launch_pdl(kern, dim3(CL, T, 1), dim3(kXThreads), smem, stream, CL, scores, n, row_stride, row_valid,
+                        id_map, id_map_stride, k, idx);
+    };
+    if (V == 8) return go(topk_range_kernel<8>);
+    if (V == 16) return go(topk_range_kernel<16>);
+    return go(topk_range_kernel<32>);
   }
   const int CL = pick_cluster(n);
   int64_t slice = (n + CL - 1) / CL;

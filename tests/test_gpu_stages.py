@@ -50,12 +50,16 @@ def test_block_stats(nseq, L, B):
     (3, 16385, 100, 0.2, 0.1, 0.1),       # 8-CTA cluster, last slice nearly empty
     (4, 4097, 50, 0.3, 0.0, 0.2),         # 2-CTA cluster
     (65, 1024, 64, 0.1, 0.0, 0.0),        # many short rows
-    (3, 30000, 100, 0.9, 0.0, 0.0),       # one-CTA rows: threshold bin beyond the candidate capacity
-    (2, 12000, 700, 0.35, 0.0, 0.0),      # heavy ties inside the threshold bin
+    (3, 30000, 100, 0.9, 0.0, 0.0),       # threshold bin beyond the gather capacity: cluster radix inside it
+    (2, 12000, 700, 0.35, 0.0, 0.0),      # heavy ties: threshold bin gathered (> 512 entries, radix over them)
     (2, 5000, 100, 0.0, 0.0, 1.0),        # every entry +-0: one value range, select by position
-    (2, 3000, 10, 0.0, 0.0, 1.0),         # same, candidates fit (radix over the candidates)
-    (2, 40960, 2048, 0.0, 0.0, 0.0),      # largest one-CTA row
-    (2, 40961, 2048, 0.0, 0.0, 0.0),      # smallest cluster row
+    (2, 3000, 10, 0.0, 0.0, 1.0),         # same, one CTA
+    (2, 40960, 2048, 0.0, 0.0, 0.0),
+    (2, 32768, 2048, 0.1, 0.0, 0.0),      # largest row of 8 entries per thread
+    (2, 32769, 2048, 0.0, 0.0, 0.0),      # smallest row of 16 per thread
+    (2, 65537, 2048, 0.0, 0.1, 0.0),      # smallest row of 32 per thread
+    (2, 131072, 5000, 0.2, 0.0, 0.0),     # largest row held in registers
+    (2, 131073, 2048, 0.0, 0.0, 0.0),     # smallest row of the digit-radix cluster kernel
 ])
 def test_topk_exact(T, n, k, ties, neg_inf, zeros):
     _check_topk(random_scores(1000 + n + k, T, n, tie_frac=ties, neg_inf_frac=neg_inf, zero_frac=zeros), n, k)
