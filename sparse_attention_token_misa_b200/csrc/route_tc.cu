@@ -430,8 +430,14 @@ route_tc_kernel(const __grid_constant__ CUtensorMap means_map, const __grid_cons
     cl.sync();  // every CTA's importances are complete
     if (crank == 0 && warp < kREpiThreads / 32) {
       if (tid < p.H) {
+        // all reads issued first, then added in rank order
+        float part[kRMaxCluster];
+#pragma unroll
+        for (int c = 0; c < kRMaxCluster; ++c) part[c] = c < csize ? cl.map_shared_rank(imp, c)[tid] : 0.f;
         float sum = 0.f;
-        for (int c = 0; c < csize; ++c) sum += cl.map_shared_rank(imp, c)[tid];
+#pragma unroll
+        for (int c = 0; c < kRMaxCluster; ++c)
+          if (c < csize) sum += part[c];
         imp2[tid] = sum;
       }
       named_bar_sync(1, kREpiThreads);

@@ -9,7 +9,7 @@
 // (and NaN) never selected; the selected positions come out in ascending order,
 // -1 padded when the row holds fewer than k selectable entries.
 //
-// Rows of up to 131072 entries (topk_range_kernel): a cluster of up to 8 CTAs
+// Rows of up to 65536 entries (topk_range_kernel): a cluster of up to 8 CTAs
 // per row, the row's entries held in registers, a value-range histogram whose
 // threshold bin is gathered across the cluster; described above the kernel.
 //
@@ -51,7 +51,7 @@ struct Smem {
   uint32_t own[kBins1];    // this CTA's share of the summed histogram
   uint32_t warp_tot[kWarps];
   uint32_t bcast[4];
-  uint32_t counts[2];      // (above tau, equal to tau) in this CTA's slice
+  alignas(8) uint32_t counts[2];  // (above tau, equal to tau) in this CTA's slice
   uint64_t warp_tot64[kWarps];
   uint64_t block_tot64;
 };
@@ -152,8 +152,12 @@ __device__ __forceinline__ void cluster_hist_sum(cg::cluster_group& cl, Smem& sm
   const int share = nbins / CL;
   const int base = rank * share;
   for (int i = threadIdx.x; i < share; i += kThreads) {
+    uint32_t x[kMaxCluster];  // all reads issued before the first is used
+#pragma unroll
+    for (int c = 0; c < kMaxCluster; ++c) x[c] = c < CL ? cl.map_shared_rank(&sm.hist[0], c)[base + i] : 0u;
     uint32_t s = 0;
-    for (int c = 0; c < CL; ++c) s += cl.map_shared_rank(&sm.hist[0], c)[base + i];
+#pragma unroll
+    for (int c = 0; c < kMaxCluster; ++c) s += x[c];
     sm.own[i] = s;
   }
   cl.sync();  // every share is summed; local histograms are no longer read remotely
@@ -300,15 +304,18 @@ topk_cluster_kernel(const float* __restrict__ scores, int64_t n, int64_t row_str
   }
   cl.sync();  // per-CTA counts visible cluster-wide
   uint32_t a_before = 0, e_before = 0, a_all = 0, e_all = 0;
-  for (int c = 0; c < CL; ++c) {
-    const uint32_t* rc = cl.map_shared_rank(&sm.counts[0], c);
-    const uint32_t ca = rc[0], ce = rc[1];
+  uint2 cc[kMaxCluster];  // all reads issued before the first is used
+#pragma unroll
+  for (int c = 0; c < kMaxCluster; ++c)
+    cc[c] = c < CL ? *reinterpret_cast<const uint2*>(cl.map_shared_rank(&sm.counts[0], c)) : make_uint2(0u, 0u);
+#pragma unroll
+  for (int c = 0; c < kMaxCluster; ++c) {
     if (c < rank) {
-      a_before += ca;
-      e_before += ce;
+      a_before += cc[c].x;
+      e_before += cc[c].y;
     }
-    a_all += ca;
-    e_all += ce;
+    a_all += cc[c].x;
+    e_all += cc[c].y;
   }
   cl.sync();  // no CTA reads another's shared memory after this point
   uint32_t a_pos = a_before + static_cast<uint32_t>(wpre & 0xffffffffull);
@@ -341,37 +348,48 @@ topk_cluster_kernel(const float* __restrict__ scores, int64_t n, int64_t row_str
 }
 
 // ---------------------------------------------------------------------------
-// Rows of up to 8 x 512 x 32 entries: a cluster of CL <= 8 CTAs of 512
+// Rows of up to 8 x 512 x 16 entries: a cluster of CL <= 8 CTAs of 512
 // threads per row, each thread holding V contiguous entries of the row in
-// registers (V = 8, 16 or 32 by row length).  Instead of bit digits (whose top
-// bits put most scores of a row into a few exponent bins) the first histogram
-// splits the value range of a fixed sample of the row (the same 512 entries in
-// every CTA, so every CTA derives the same bins) into 2048 equal ranges; the
-// map is monotone, values outside the sample's range go to the end bins.
-// The threshold bin is located from the CL histograms in two rounds of
-// distributed shared memory reads (64 super-bin totals, then the 32 bins of
-// the chosen super-bin), its entries (few) are gathered from every CTA and the
-// exact threshold among them is found by counting.  Every CTA then knows how
-// many entries above and equal to the threshold each slice holds, so the
-// output slots follow from a scan: two cluster barriers on this path.  A
-// threshold bin too full to gather (massive ties, a sample range spoilt by
-// outliers) falls back to a cluster-wide bit-digit radix select inside it.
+// registers (V = 8 or 16 by row length).  Instead of bit digits (whose top
+// bits put most scores of a row into a few exponent bins) the histogram splits
+// the value range of a fixed sample of the row (the same 512 entries in every
+// CTA, so every CTA derives the same bins) into 1024 equal ranges; the map is
+// monotone, values outside the sample's range go to the end bins.  The path
+// is a short chain of dependent steps, each a cluster barrier followed by
+// small rounds of distributed shared memory reads (they are slow; bytes are
+// kept few):
+//   (1) every CTA sums the CL histograms' 32 super-bin totals, finds the
+//       super-bin holding the k-th entry, then sums its 32 bins (a second
+//       read round) and finds the threshold bin;
+//   (2) every CTA reads the counts above the threshold bin and the threshold
+//       bin's entries (few) of every slice, finds the exact threshold among
+//       them by counting, and so knows how many entries above and equal to it
+//       each slice holds: the output slots follow from a scan.
+// A threshold bin with more entries than one read round takes is gathered in
+// a second round (radix select over the gathered entries when they are many);
+// one too full to gather (massive ties, a sample range spoilt by outliers)
+// falls back to a cluster-wide bit-digit radix select inside it.
 constexpr int kXThreads = 512;
 constexpr int kXWarps = kXThreads / 32;
-constexpr int kXBins = 2048;          // value-range bins = 64 super-bins x 32
+constexpr int kXBins = 2048;          // histogram array (fallback digits use all of it)
+constexpr int kXFastBins = 1024;      // value-range bins: 2 per thread
 constexpr int kXSup = kXBins / 32;
+constexpr int kXFastCand = kXThreads / kMaxCluster;  // threshold-bin entries per slice read in one round
 constexpr int kXCandCap = 512;        // threshold-bin entries kept per CTA
 constexpr int kXMergeCap = 2048;      // and over the cluster
-constexpr int kXMaxV = 32;
+#ifndef MISA_TOPK_RANGE_CLUSTER
+#define MISA_TOPK_RANGE_CLUSTER 8
+#endif
+constexpr int kXRangeCluster = MISA_TOPK_RANGE_CLUSTER;  // CTAs per row at most
 
 struct XSmem {
   uint32_t hist[kXBins];     // this CTA's histogram (read by the cluster)
-  uint32_t sup[kXSup];       // its super-bin totals (read by the cluster)
+  uint32_t sup[kXSup];       // fallback: its super-bin totals (read by the cluster)
   uint32_t meta[4];          // valid entries, entries above the threshold bin, threshold-bin entries (read by the cluster)
   uint32_t cnt2[2];          // fallback: entries above / equal to tau (read by the cluster)
   uint32_t gsup[kXSup];      // super-bin totals summed over the cluster
   uint32_t gbin[32];
-  uint32_t bc[4];
+  uint32_t bc[8];
   float fbc;
   uint32_t rv[kMaxCluster], ra[kMaxCluster], rc[kMaxCluster];
   uint32_t at[kMaxCluster], et[kMaxCluster];
@@ -380,7 +398,8 @@ struct XSmem {
   union {
     struct {
       float cval[kXCandCap];     // this CTA's threshold-bin entries (read by the cluster)
-      float mval[kXMergeCap];    // all of the cluster's, by rank
+      float fval[kXThreads];     // first kXFastCand entries of every slice, [rank][i]
+      float mval[kXMergeCap];    // the cluster's threshold-bin entries, by rank
       uint8_t mrank[kXMergeCap];
     } c;
     struct {
@@ -390,8 +409,10 @@ struct XSmem {
   } u;
 };
 
-__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
-__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
 
 // One warp: among tot[0, cnt) (cnt <= 128) the index i with
 // above(i) < need <= above(i) + tot[i], above(i) = sum of tot[i+1 .. cnt);
@@ -481,7 +502,7 @@ __device__ __forceinline__ float key_to_float(uint32_t kk) {
 }
 
 template <int V>
-__global__ void __launch_bounds__(kXThreads, V >= 32 ? 1 : 2)
+__global__ void __launch_bounds__(kXThreads, 2)
 topk_range_kernel(const float* __restrict__ scores, int64_t n, int64_t row_stride, const int32_t* __restrict__ row_valid,
                   const int32_t* __restrict__ id_map, int64_t id_map_stride, int k, int32_t* __restrict__ idx) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -494,8 +515,9 @@ topk_range_kernel(const float* __restrict__ scores, int64_t n, int64_t row_strid
   constexpr int kSlice = kXThreads * V;
   const float kNegInf = -__int_as_float(0x7f800000);
   const float kPosInf = __int_as_float(0x7f800000);
+  const uint32_t ku = static_cast<uint32_t>(k);
 
-  for (int i = tid; i < kXBins; i += kXThreads) sm.hist[i] = 0;
+  for (int i = tid; i < kXFastBins; i += kXThreads) sm.hist[i] = 0;
   if (tid < 4) sm.meta[tid] = 0;
   pdl_wait_inputs();
   pdl_allow_next();
@@ -550,11 +572,11 @@ topk_range_kernel(const float* __restrict__ scores, int64_t n, int64_t row_strid
     mn = fminf(mn, sm.wmin[i]);
   }
   const float range = mx - mn;
-  const float scale = (range > 0.f && range < kPosInf) ? static_cast<float>(kXBins) / range : 0.f;
+  const float scale = (range > 0.f && range < kPosInf) ? static_cast<float>(kXFastBins) / range : 0.f;
   // monotone in x; a NaN intermediate (no valid sample, infinite entries) maps to bin 0
   auto bin_of = [&](float x) -> int {
     const float y = __fmul_rn(__fsub_rn(x, mn), scale);
-    return y > 0.f ? (y >= static_cast<float>(kXBins - 1) ? kXBins - 1 : static_cast<int>(y)) : 0;
+    return y > 0.f ? (y >= static_cast<float>(kXFastBins - 1) ? kXFastBins - 1 : static_cast<int>(y)) : 0;
   };
 
   // ---------------- value-range histogram of the slice
@@ -571,28 +593,60 @@ topk_range_kernel(const float* __restrict__ scores, int64_t n, int64_t row_strid
   for (int o = 16; o > 0; o >>= 1) nval += __shfl_xor_sync(0xffffffffu, nval, o);
   if (lane == 0 && nval) atomicAdd(&sm.meta[0], nval);
   __syncthreads();
-  make_supers(sm.hist, sm.sup, kXBins);
+  make_supers(sm.hist, sm.sup, kXFastBins);
   __syncthreads();
-  cl.sync();  // (1) every CTA's histogram, super-bins and valid count are complete
+  cl.sync();  // (1) every CTA's histogram, super-bin totals and valid count are complete
 
-  if (tid < CL) sm.rv[tid] = cl.map_shared_rank(&sm.meta[0], tid)[0];
+  // ---------------- the threshold bin, from the CL histograms in two read
+  // rounds of 32 x CL words each: super-bin totals, then the 32 bins of the
+  // super-bin holding the k-th entry.  Thread (s, r) = (tid / 8, tid % 8)
+  // reads item s of source (r + rank) mod CL (the CTAs start on different
+  // SMs); 8 lanes add their sources.
+  const int fs = tid >> 3, fr = tid & 7;
+  const int fsrc = fr + rank < CL ? fr + rank : fr + rank - CL;
+  if (tid >= 32 * kMaxCluster && tid < 32 * kMaxCluster + CL)
+    sm.rv[tid - 32 * kMaxCluster] = cl.map_shared_rank(&sm.meta[0], tid - 32 * kMaxCluster)[0];
+  if (tid < 32 * kMaxCluster) {
+    uint32_t x = fr < CL ? cl.map_shared_rank(&sm.sup[0], fsrc)[fs] : 0u;
+    x += __shfl_xor_sync(0xffffffffu, x, 1);
+    x += __shfl_xor_sync(0xffffffffu, x, 2);
+    x += __shfl_xor_sync(0xffffffffu, x, 4);
+    if (fr == 0) sm.gsup[fs] = x;
+  }
   __syncthreads();
-  uint32_t total = 0;
-  for (int r = 0; r < CL; ++r) total += sm.rv[r];
+  if (warp == 0) {
+    uint32_t x = sm.gsup[lane];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    if (lane == 0) sm.bc[3] = x;  // valid entries of the row
+    if (x > ku) warp_suffix_find(sm.gsup, 32, ku, sm.bc);
+  }
+  __syncthreads();
+  const uint32_t total = sm.bc[3];
 
   float tau = kNegInf;  // selected: entries above tau, and the first need_eq entries equal to it
   uint32_t need_eq = 0;
-  if (total <= static_cast<uint32_t>(k)) {
+  if (total <= ku) {
     if (tid < CL) {
       sm.at[tid] = sm.rv[tid];
       sm.et[tid] = 0;
     }
   } else {
-    uint32_t above_b;
-    const int bstar = two_level_find(
-        sm, CL, [&](int r) { return cl.map_shared_rank(&sm.hist[0], r); },
-        [&](int r) { return cl.map_shared_rank(&sm.sup[0], r); }, kXSup, static_cast<uint32_t>(k), &above_b);
-    const uint32_t need = static_cast<uint32_t>(k) - above_b;
+    const int S = static_cast<int>(sm.bc[0] & 31u);
+    const uint32_t above_s = sm.bc[1];
+    if (tid < 32 * kMaxCluster) {
+      uint32_t x = fr < CL ? cl.map_shared_rank(&sm.hist[0], fsrc)[S * 32 + fs] : 0u;
+      x += __shfl_xor_sync(0xffffffffu, x, 1);
+      x += __shfl_xor_sync(0xffffffffu, x, 2);
+      x += __shfl_xor_sync(0xffffffffu, x, 4);
+      if (fr == 0) sm.gbin[fs] = x;
+    }
+    __syncthreads();
+    if (warp == 0) warp_suffix_find(sm.gbin, 32, ku - above_s, sm.bc + 4);
+    __syncthreads();
+    const int bstar = S * 32 + static_cast<int>(sm.bc[4] & 31u);
+    const uint32_t above_b = above_s + sm.bc[5];
+    const uint32_t need = ku - above_b;
     // entries above the threshold bin, and the threshold bin's entries
     uint32_t a = 0;
 #pragma unroll
@@ -611,21 +665,43 @@ topk_range_kernel(const float* __restrict__ scores, int64_t n, int64_t row_strid
     if (lane == 0 && a) atomicAdd(&sm.meta[1], a);
     __syncthreads();
     cl.sync();  // (2) every CTA's counts and threshold-bin entries are complete
-    if (tid < CL) {
-      const uint32_t* m = cl.map_shared_rank(&sm.meta[0], tid);
-      sm.ra[tid] = m[1];
-      sm.rc[tid] = m[2];
+    {
+      // one read round: slice r's counts and its first kXFastCand entries
+      // (thread group j of CTA c reads slice (j + c) mod CL: the CTAs start on
+      // different slices)
+      const int j = tid / kXFastCand, i = tid - j * kXFastCand;
+      if (j < CL) {
+        const int r = j + rank < CL ? j + rank : j + rank - CL;
+        const uint32_t* m = cl.map_shared_rank(&sm.meta[0], r);
+        const float x = cl.map_shared_rank(&sm.u.c.cval[0], r)[i];
+        if (i == 0) {
+          sm.ra[r] = m[1];
+          sm.rc[r] = m[2];
+        }
+        sm.u.c.fval[r * kXFastCand + i] = x;
+      }
     }
     __syncthreads();
-    uint32_t ctot = 0;
-    bool overflow = false;
-    for (int r = 0; r < CL; ++r) {
-      ctot += sm.rc[r];
-      overflow |= sm.rc[r] > static_cast<uint32_t>(kXCandCap);
+    uint32_t ctot = 0, cmax = 0;
+#pragma unroll
+    for (int r = 0; r < kMaxCluster; ++r) {
+      const uint32_t c = r < CL ? sm.rc[r] : 0u;
+      ctot += c;
+      cmax = c > cmax ? c : cmax;
     }
-    overflow |= ctot > static_cast<uint32_t>(kXMergeCap);
-    if (!overflow) {
-      // ---------------- gather the threshold bin from the cluster
+    const bool overflow = cmax > static_cast<uint32_t>(kXCandCap) || ctot > static_cast<uint32_t>(kXMergeCap);
+    if (cmax <= static_cast<uint32_t>(kXFastCand)) {
+      // compact the entries read in the round above
+      const int r = tid / kXFastCand, i = tid - r * kXFastCand;
+      if (r < CL && static_cast<uint32_t>(i) < sm.rc[r]) {
+        uint32_t off = 0;
+        for (int r2 = 0; r2 < r; ++r2) off += sm.rc[r2];
+        sm.u.c.mval[off + i] = sm.u.c.fval[tid];
+        sm.u.c.mrank[off + i] = static_cast<uint8_t>(r);
+      }
+      __syncthreads();
+    } else if (!overflow) {
+      // a second read round for the rest of the threshold bin
       for (int i = tid; i < static_cast<int>(ctot); i += kXThreads) {
         int r = 0;
         uint32_t off = 0;
@@ -634,11 +710,14 @@ topk_range_kernel(const float* __restrict__ scores, int64_t n, int64_t row_strid
         sm.u.c.mrank[i] = static_cast<uint8_t>(r);
       }
       __syncthreads();
+    }
+    if (!overflow) {
       if (ctot <= static_cast<uint32_t>(kXThreads)) {
         // exact rank by counting
         if (tid < static_cast<int>(ctot)) {
           const float x = sm.u.c.mval[tid];
           uint32_t g = 0, ge = 0;
+#pragma unroll 4
           for (int j = 0; j < static_cast<int>(ctot); ++j) {
             const float y = sm.u.c.mval[j];
             g += y > x ? 1u : 0u;
@@ -646,16 +725,16 @@ topk_range_kernel(const float* __restrict__ scores, int64_t n, int64_t row_strid
           }
           if (g < need && need <= ge) {
             sm.fbc = x;
-            sm.bc[0] = need - g;
+            sm.bc[2] = need - g;
           }
         }
         __syncthreads();
         tau = sm.fbc;
-        need_eq = sm.bc[0];
+        need_eq = sm.bc[2];
       } else {
         // bit-digit radix select over the gathered entries (local; the
         // histogram arrays are no longer read by the cluster after (2))
-        uint32_t prefix = 0, gt = 0, nd = need;
+        uint32_t prefix = 0, nd = need;
         for (int round = 0; round < 3; ++round) {
           const int sh = digit_shift(round), nb = digit_bins(round);
           for (int i = tid; i < nb; i += kXThreads) sm.hist[i] = 0;
@@ -670,7 +749,6 @@ topk_range_kernel(const float* __restrict__ scores, int64_t n, int64_t row_strid
           uint32_t ab;
           const int b = two_level_find(
               sm, 1, [&](int) { return &sm.hist[0]; }, [&](int) { return &sm.sup[0]; }, nb / 32, nd, &ab);
-          gt += ab;
           nd -= ab;
           prefix = round == 0 ? static_cast<uint32_t>(b) : ((prefix << (round == 1 ? 11 : 10)) | static_cast<uint32_t>(b));
         }
@@ -692,7 +770,7 @@ topk_range_kernel(const float* __restrict__ scores, int64_t n, int64_t row_strid
       // ---------------- fallback: cluster-wide radix select inside bin bstar.
       // Digit histograms alternate between two buffers, so a CTA never
       // overwrites one that another CTA may still be reading.
-      uint32_t prefix = 0, gt = 0, nd = need;
+      uint32_t prefix = 0, nd = need;
       for (int round = 0; round < 3; ++round) {
         uint32_t* H = (round & 1) ? sm.u.r.h : sm.hist;
         uint32_t* S = (round & 1) ? sm.u.r.s : sm.sup;
@@ -714,7 +792,6 @@ topk_range_kernel(const float* __restrict__ scores, int64_t n, int64_t row_strid
         const int b = two_level_find(
             sm, CL, [&](int r) { return cl.map_shared_rank(H, r); }, [&](int r) { return cl.map_shared_rank(S, r); },
             nb / 32, nd, &ab);
-        gt += ab;
         nd -= ab;
         prefix = round == 0 ? static_cast<uint32_t>(b) : ((prefix << (round == 1 ? 11 : 10)) | static_cast<uint32_t>(b));
       }
@@ -747,19 +824,20 @@ topk_range_kernel(const float* __restrict__ scores, int64_t n, int64_t row_strid
     }
   }
   __syncthreads();
-  // this CTA reads no other CTA's shared memory after this point
-  cluster_arrive();
+  // every value read from another CTA's shared memory has arrived: it may exit
+  // once all CTAs are here
+  cluster_arrive_relaxed();
 
   // ---------------- output slots: entries above tau before this one, plus the
   // equal entries before it (at most need_eq of them)
   uint32_t a_before = 0, e_before = 0, a_all = 0, e_all = 0;
-  for (int r = 0; r < CL; ++r) {
-    if (r < rank) {
-      a_before += sm.at[r];
-      e_before += sm.et[r];
-    }
-    a_all += sm.at[r];
-    e_all += sm.et[r];
+#pragma unroll
+  for (int r = 0; r < kMaxCluster; ++r) {
+    const uint32_t ar = r < CL ? sm.at[r] : 0u, er = r < CL ? sm.et[r] : 0u;
+    a_before += r < rank ? ar : 0u;
+    e_before += r < rank ? er : 0u;
+    a_all += ar;
+    e_all += er;
   }
   uint32_t a_t = 0, e_t = 0;
 #pragma unroll
@@ -768,17 +846,17 @@ topk_range_kernel(const float* __restrict__ scores, int64_t n, int64_t row_strid
     e_t += (v[j] > kNegInf && v[j] == tau) ? 1u : 0u;
   }
   uint64_t x = static_cast<uint64_t>(a_t) | (static_cast<uint64_t>(e_t) << 32);
-  uint64_t inc = x;
+  uint64_t incl = x;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const uint64_t y = __shfl_up_sync(0xffffffffu, inc, o);
-    if (lane >= o) inc += y;
+    const uint64_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
   }
-  if (lane == 31) sm.wscan[warp] = inc;
+  if (lane == 31) sm.wscan[warp] = incl;
   __syncthreads();
   uint64_t wbase = 0;
   for (int i = 0; i < warp; ++i) wbase += sm.wscan[i];
-  const uint64_t excl = wbase + inc - x;
+  const uint64_t excl = wbase + incl - x;
   uint32_t A = a_before + static_cast<uint32_t>(excl & 0xffffffffull);
   uint32_t E = e_before + static_cast<uint32_t>(excl >> 32);
 #pragma unroll
@@ -786,16 +864,16 @@ topk_range_kernel(const float* __restrict__ scores, int64_t n, int64_t row_strid
     const float y = v[j];
     if (y > tau) {
       const uint32_t slot = A + (E < need_eq ? E : need_eq);
-      if (slot < static_cast<uint32_t>(k)) out[slot] = idrow ? idrow[p0 + j] : p0 + j;
+      if (slot < ku) out[slot] = idrow ? idrow[p0 + j] : p0 + j;
       ++A;
     } else if (y > kNegInf && y == tau) {
-      if (E < need_eq && A + E < static_cast<uint32_t>(k)) out[A + E] = idrow ? idrow[p0 + j] : p0 + j;
+      if (E < need_eq && A + E < ku) out[A + E] = idrow ? idrow[p0 + j] : p0 + j;
       ++E;
     }
   }
   if (rank == CL - 1) {
     const uint32_t chosen = a_all + (e_all < need_eq ? e_all : need_eq);
-    for (uint32_t i = chosen + tid; i < static_cast<uint32_t>(k); i += kXThreads) out[i] = -1;
+    for (uint32_t i = chosen + tid; i < ku; i += kXThreads) out[i] = -1;
   }
   cluster_wait();  // no CTA exits while another may still read its shared memory
 }
@@ -812,10 +890,9 @@ size_t topk_smem_bytes() { return kKeysOff + static_cast<size_t>(kSliceCap) * 4;
 
 cudaError_t launch_topk(const float* scores, int T, int64_t n, int64_t row_stride, const int32_t* row_valid,
                         const int32_t* id_map, int64_t id_map_stride, int k, int32_t* idx, cudaStream_t stream) {
-  if (n <= static_cast<int64_t>(kMaxCluster) * kXThreads * kXMaxV) {
-    // smallest V with ceil(n / (512 V)) <= 8 CTAs per row
-    const int V = n <= static_cast<int64_t>(kMaxCluster) * kXThreads * 8 ? 8
-                  : (n <= static_cast<int64_t>(kMaxCluster) * kXThreads * 16 ? 16 : 32);
+  if (n <= static_cast<int64_t>(kXRangeCluster) * kXThreads * 16) {
+    // smallest V with ceil(n / (512 V)) <= kXRangeCluster CTAs per row
+    const int V = n <= static_cast<int64_t>(kXRangeCluster) * kXThreads * 8 ? 8 : 16;
     const int64_t slice = static_cast<int64_t>(kXThreads) * V;
     const int CL = static_cast<int>((n + slice - 1) / slice);
     const size_t smem = sizeof(XSmem);
@@ -826,8 +903,7 @@ cudaError_t launch_topk(const float* scores, int T, int64_t n, int64_t row_strid
                         id_map, id_map_stride, k, idx);
     };
     if (V == 8) return go(topk_range_kernel<8>);
-    if (V == 16) return go(topk_range_kernel<16>);
-    return go(topk_range_kernel<32>);
+    return go(topk_range_kernel<16>);
   }
   const int CL = pick_cluster(n);
   int64_t slice = (n + CL - 1) / CL;

@@ -57,9 +57,9 @@ def test_block_stats(nseq, L, B):
     (2, 40960, 2048, 0.0, 0.0, 0.0),
     (2, 32768, 2048, 0.1, 0.0, 0.0),      # largest row of 8 entries per thread
     (2, 32769, 2048, 0.0, 0.0, 0.0),      # smallest row of 16 per thread
-    (2, 65537, 2048, 0.0, 0.1, 0.0),      # smallest row of 32 per thread
-    (2, 131072, 5000, 0.2, 0.0, 0.0),     # largest row held in registers
-    (2, 131073, 2048, 0.0, 0.0, 0.0),     # smallest row of the digit-radix cluster kernel
+    (2, 65536, 2048, 0.0, 0.1, 0.0),      # largest row held in registers
+    (2, 131072, 5000, 0.2, 0.0, 0.0),     # digit-radix cluster kernel, keys in shared memory
+    (2, 65537, 2048, 0.0, 0.0, 0.0),      # smallest row of the digit-radix cluster kernel
 ])
 def test_topk_exact(T, n, k, ties, neg_inf, zeros):
     _check_topk(random_scores(1000 + n + k, T, n, tie_frac=ties, neg_inf_frac=neg_inf, zero_frac=zeros), n, k)
