@@ -878,6 +878,407 @@ topk_range_kernel(const float* __restrict__ scores, int64_t n, int64_t row_strid
   cluster_wait();  // no CTA exits while another may still read its shared memory
 }
 
+// ---------------------------------------------------------------------------
+// One CTA of 512 threads per row, no cluster (topk_band_kernel).  A sample of
+// the row (up to 4096 evenly spaced entries) gives a value band that holds the
+// k-th largest entry with a wide margin: the sample is binned over its value
+// range (4096 equal ranges, a monotone map), and the bins holding sample ranks
+// r - d and r + d (r the rank the k-th entry has in the sample on average, d =
+// 3 sqrt(r) + 8) bound the band.  One pass over the row counts, per warp, the
+// entries in bins above the band and gathers the band's entries (few: about
+// 2 d / 4096 of the row).  When the band holds the k-th entry, a radix select
+// over the gathered entries gives the exact threshold tau; otherwise (the
+// sample misled, or too many ties to gather) a radix select over the whole row
+// does.  A second pass writes the selected positions in order: each warp owns
+// a contiguous segment, and the per-warp counts of entries above and equal to
+// tau, scanned over the warps, give every selected entry its output slot.
+// The row is read twice (the second time mostly from L2); shared-memory
+// atomics only for the sample histogram and the radix rounds over the band.
+constexpr int kBThreads = 512;
+constexpr int kBWarps = kBThreads / 32;
+constexpr int kBSample = 4096;
+constexpr int kBBins = 4096;
+constexpr int kBCandCap = 4096;  // band entries kept
+#ifndef MISA_BAND_UNROLL
+#define MISA_BAND_UNROLL 1
+#endif
+constexpr int kBUnroll = MISA_BAND_UNROLL;  // 128-entry steps loaded together per warp
+
+struct BSmem {
+  uint32_t hist[kBBins];
+  float sval[kBSample];
+  float cval[kBCandCap];    // band entries and their warps
+  uint8_t cwarp[kBCandCap];
+  uint32_t wa[kBWarps], wv[kBWarps];  // per warp: entries above the band, valid entries
+  uint32_t at[kBWarps], et[kBWarps];  // per warp: entries above / equal to tau
+  uint32_t wtmp[kBWarps];
+  float wmin[kBWarps], wmax[kBWarps];
+  uint32_t bc[8];
+  uint32_t ccount;
+};
+
+// Over hist[0, nbins) (nbins a multiple of 512, <= 4096): for each of the two
+// targets the bin b with above(b) < need <= above(b) + hist[b], above(b) = sum
+// of the higher bins: out[0] = b, out[1] = above(b) for need1, out[2], out[3]
+// for need2 (left unchanged when a target exceeds the total).  All threads.
+__device__ __forceinline__ void band_find(BSmem& sm, const uint32_t* hist, int nbins, uint32_t need1,
+                                          uint32_t need2, uint32_t* out) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int per = nbins / kBThreads;
+  const int b0 = tid * per;
+  uint32_t local = 0;
+  for (int i = 0; i < per; ++i) local += hist[b0 + i];
+  uint32_t inc = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_down_sync(0xffffffffu, inc, o);
+    if (lane + o < 32) inc += y;
+  }
+  if (lane == 0) sm.wtmp[warp] = inc;
+  __syncthreads();
+  uint32_t higher = 0;
+#pragma unroll
+  for (int w2 = 0; w2 < kBWarps; ++w2) higher += w2 > warp ? sm.wtmp[w2] : 0u;
+  const uint32_t after = higher + inc - local;
+  const uint32_t needs[2] = {need1, need2};
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const uint32_t need = needs[q];
+    if (after < need && need <= after + local) {
+      uint32_t acc = after;
+      for (int i = per - 1; i >= 0; --i) {
+        const uint32_t c = hist[b0 + i];
+        if (acc + c >= need) {
+          out[2 * q] = static_cast<uint32_t>(b0 + i);
+          out[2 * q + 1] = acc;
+          break;
+        }
+        acc += c;
+      }
+    }
+  }
+  __syncthreads();
+}
+
+// Exact radix select (12 + 10 + 10 key bits) of the need-th largest key among
+// n_keys keys produced by key_at(i) (0 = not a candidate); returns its key and
+// sets *gt to the number of larger keys.  All threads.
+template <class KeyAt>
+__device__ uint32_t band_radix(BSmem& sm, int n_keys, KeyAt key_at, uint32_t need, uint32_t* gt) {
+  const int tid = threadIdx.x;
+  uint32_t prefix = 0, above = 0;
+  for (int round = 0; round < 3; ++round) {
+    const int sh = round == 0 ? 20 : (round == 1 ? 10 : 0);
+    const int nb = round == 0 ? 4096 : 1024;
+    for (int i = tid; i < nb; i += kBThreads) sm.hist[i] = 0;
+    __syncthreads();
+    for (int i = tid; i < n_keys; i += kBThreads) {
+      const uint32_t kk = key_at(i);
+      if (kk == 0u) continue;
+      const bool match = round == 0 || (kk >> (round == 1 ? 20 : 10)) == prefix;
+      if (match) atomicAdd(&sm.hist[(kk >> sh) & static_cast<uint32_t>(nb - 1)], 1u);
+    }
+    __syncthreads();
+    band_find(sm, sm.hist, nb, need, 0xffffffffu, sm.bc);
+    const uint32_t b = sm.bc[0] & static_cast<uint32_t>(nb - 1);
+    const uint32_t ab = sm.bc[1];
+    __syncthreads();
+    above += ab;
+    need -= ab;
+    prefix = round == 0 ? b : ((prefix << 10) | b);
+  }
+  *gt = above;
+  return prefix;
+}
+
+__global__ void __launch_bounds__(kBThreads, 2)
+topk_band_kernel(const float* __restrict__ scores, int64_t n, int64_t row_stride, const int32_t* __restrict__ row_valid,
+                 const int32_t* __restrict__ id_map, int64_t id_map_stride, int k, int32_t* __restrict__ idx) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  BSmem& sm = *reinterpret_cast<BSmem*>(smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t t = blockIdx.x;
+  const float kNegInf = -__int_as_float(0x7f800000);
+  const float kPosInf = __int_as_float(0x7f800000);
+  const uint32_t ku = static_cast<uint32_t>(k);
+  const uint32_t lt = (1u << lane) - 1u;
+
+  if (tid == 0) sm.ccount = 0;
+  pdl_wait_inputs();
+  pdl_allow_next();
+  const float* row = scores + t * row_stride;
+  const int32_t* idrow = id_map ? id_map + t * id_map_stride : nullptr;
+  int32_t* out = idx + t * k;
+  int64_t nt64 = n;
+  if (row_valid) {
+    const int64_t rv = row_valid[t];
+    nt64 = rv < 0 ? 0 : (rv < n ? rv : n);
+  }
+  const int nt = static_cast<int>(nt64);
+  // warp segments: multiples of 128 entries (32 lanes x 4)
+  const int seg = ((nt + kBWarps - 1) / kBWarps + 127) / 128 * 128;
+  const int w0 = warp * seg < nt ? warp * seg : nt;
+  const int w1 = w0 + seg < nt ? w0 + seg : nt;
+  auto load4 = [&](int p, float x[4]) {
+    if (p + 3 < w1) {
+      const float4 f = __ldg(reinterpret_cast<const float4*>(row + p));
+      x[0] = f.x;
+      x[1] = f.y;
+      x[2] = f.z;
+      x[3] = f.w;
+    } else {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) x[c] = p + c < w1 ? __ldg(row + p + c) : kNegInf;
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) x[c] = valid_or_neg_inf(x[c]);
+  };
+
+  // ---------------- sample: value range, then its histogram
+  const int ns = nt < kBSample ? nt : kBSample;
+  float mx = kNegInf, mn = kPosInf;
+  {
+    float sv[kBSample / kBThreads];  // all sample loads in flight together
+#pragma unroll
+    for (int u = 0; u < kBSample / kBThreads; ++u) {
+      const int i = tid + u * kBThreads;
+      sv[u] = i < ns ? __ldg(row + static_cast<int64_t>(i) * nt / ns) : kNegInf;
+    }
+#pragma unroll
+    for (int u = 0; u < kBSample / kBThreads; ++u) {
+      const int i = tid + u * kBThreads;
+      const float v = valid_or_neg_inf(sv[u]);
+      if (i < ns) sm.sval[i] = v;
+      if (v > kNegInf) {
+        mx = fmaxf(mx, v);
+        mn = fminf(mn, v);
+      }
+    }
+  }
+  for (int i = tid; i < kBBins; i += kBThreads) sm.hist[i] = 0;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+  }
+  if (lane == 0) {
+    sm.wmax[warp] = mx;
+    sm.wmin[warp] = mn;
+  }
+  __syncthreads();
+  mx = sm.wmax[0];
+  mn = sm.wmin[0];
+#pragma unroll
+  for (int i = 1; i < kBWarps; ++i) {
+    mx = fmaxf(mx, sm.wmax[i]);
+    mn = fminf(mn, sm.wmin[i]);
+  }
+  const float range = mx - mn;
+  const float scale = (range > 0.f && range < kPosInf) ? static_cast<float>(kBBins) / range : 0.f;
+  // monotone in x; a NaN intermediate (no valid sample, infinite entries) maps to bin 0
+  auto bin_of = [&](float x) -> int {
+    const float y = __fmul_rn(__fsub_rn(x, mn), scale);
+    return y > 0.f ? (y >= static_cast<float>(kBBins - 1) ? kBBins - 1 : static_cast<int>(y)) : 0;
+  };
+  uint32_t nsv = 0;
+  for (int i = tid; i < ns; i += kBThreads) {
+    const float v = sm.sval[i];
+    if (v > kNegInf) {
+      atomicAdd(&sm.hist[bin_of(v)], 1u);
+      ++nsv;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) nsv += __shfl_xor_sync(0xffffffffu, nsv, o);
+  if (lane == 0) sm.wtmp[warp] = nsv;
+  __syncthreads();
+  nsv = 0;
+#pragma unroll
+  for (int i = 0; i < kBWarps; ++i) nsv += sm.wtmp[i];
+  __syncthreads();
+  // the band: bins [b_lo, b_hi] around sample rank r = k * ns / nt (from the top)
+  const int64_t r = static_cast<int64_t>(k) * ns / (nt > 0 ? nt : 1);
+  const int64_t d = static_cast<int64_t>(3.f * sqrtf(static_cast<float>(r))) + 8;
+  const int64_t r_hi = r - d, r_lo = r + d;  // 0-based ranks
+  if (tid == 0) {
+    sm.bc[0] = kBBins;  // b_hi when r_hi < 0: no bin lies above the band
+    sm.bc[2] = 0;       // b_lo when r_lo is past the valid sample: the band reaches down to bin 0
+  }
+  __syncthreads();
+  band_find(sm, sm.hist, kBBins, r_hi >= 0 ? static_cast<uint32_t>(r_hi + 1) : 0xffffffffu,
+            r_lo < static_cast<int64_t>(nsv) ? static_cast<uint32_t>(r_lo + 1) : 0xffffffffu, sm.bc);
+  const int b_hi = static_cast<int>(sm.bc[0]);
+  const int b_lo = static_cast<int>(sm.bc[2]);
+
+  // ---------------- pass 1: per warp, entries above the band and valid
+  // entries; the band's entries are gathered
+  uint32_t a_l = 0, v_l = 0;
+
+  // kBUnroll steps' loads are issued before the first is used (memory-level
+  // parallelism: one warp keeps kBUnroll x 512 bytes in flight)
+  for (int base0 = w0; base0 < w1; base0 += 128 * kBUnroll) {
+    float xs[kBUnroll][4];
+#pragma unroll
+    for (int u = 0; u < kBUnroll; ++u) load4(base0 + 128 * u + 4 * lane, xs[u]);
+#pragma unroll
+    for (int u = 0; u < kBUnroll; ++u) {
+    const int p = base0 + 128 * u + 4 * lane;
+    const float* x = xs[u];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const bool valid = x[c] > kNegInf;
+      const int b = bin_of(x[c]);
+      a_l += (valid && b > b_hi) ? 1u : 0u;
+      v_l += valid ? 1u : 0u;
+      const bool band = valid && b >= b_lo && b <= b_hi;
+      const uint32_t bm = __ballot_sync(0xffffffffu, band);
+      if (bm) {
+        uint32_t slot0 = 0;
+        if (lane == 0) slot0 = atomicAdd(&sm.ccount, static_cast<uint32_t>(__popc(bm)));
+        slot0 = __shfl_sync(0xffffffffu, slot0, 0);
+        if (band) {
+          const uint32_t sl = slot0 + __popc(bm & lt);
+          if (sl < static_cast<uint32_t>(kBCandCap)) {
+            sm.cval[sl] = x[c];
+            sm.cwarp[sl] = static_cast<uint8_t>(warp);
+          }
+        }
+      }
+    }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    a_l += __shfl_xor_sync(0xffffffffu, a_l, o);
+    v_l += __shfl_xor_sync(0xffffffffu, v_l, o);
+  }
+  if (lane == 0) {
+    sm.wa[warp] = a_l;
+    sm.wv[warp] = v_l;
+  }
+  __syncthreads();
+  uint32_t A = 0, V = 0;
+#pragma unroll
+  for (int i = 0; i < kBWarps; ++i) {
+    A += sm.wa[i];
+    V += sm.wv[i];
+  }
+  const uint32_t C = sm.ccount;
+
+  float tau;
+  uint32_t need_eq;
+  if (V <= ku) {
+    // every valid entry is selected
+    tau = kNegInf;
+    need_eq = 0;
+    if (tid < kBWarps) {
+      sm.at[tid] = sm.wv[tid];
+      sm.et[tid] = 0;
+    }
+  } else if (A < ku && ku <= A + C && C <= static_cast<uint32_t>(kBCandCap)) {
+    // the k-th entry is in the band: exact tau among the gathered entries
+    uint32_t gt;
+    const uint32_t kk = band_radix(sm, static_cast<int>(C), [&](int i) { return float_key(sm.cval[i]); }, ku - A, &gt);
+    tau = key_to_float(kk);
+    need_eq = ku - A - gt;
+    if (tid < kBWarps) {
+      sm.at[tid] = sm.wa[tid];
+      sm.et[tid] = 0;
+    }
+    __syncthreads();
+    for (int i = tid; i < static_cast<int>(C); i += kBThreads) {
+      const int w = sm.cwarp[i];
+      const float x = sm.cval[i];
+      if (x > tau) atomicAdd(&sm.at[w], 1u);
+      else if (x == tau) atomicAdd(&sm.et[w], 1u);
+    }
+  } else {
+    // the sample misled (or the band is too full): radix select over the row,
+    // then count per warp
+    uint32_t gt;
+    const uint32_t kk = band_radix(sm, nt, [&](int i) { return sel_key(__ldg(row + i)); }, ku, &gt);
+    tau = key_to_float(kk);
+    need_eq = ku - gt;
+    uint32_t ac = 0, ec = 0;
+    for (int base0 = w0; base0 < w1; base0 += 128 * kBUnroll) {
+      float xs[kBUnroll][4];
+#pragma unroll
+      for (int u = 0; u < kBUnroll; ++u) load4(base0 + 128 * u + 4 * lane, xs[u]);
+#pragma unroll
+      for (int u = 0; u < kBUnroll; ++u)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          ac += xs[u][c] > tau ? 1u : 0u;
+          ec += (xs[u][c] > kNegInf && xs[u][c] == tau) ? 1u : 0u;
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      ac += __shfl_xor_sync(0xffffffffu, ac, o);
+      ec += __shfl_xor_sync(0xffffffffu, ec, o);
+    }
+    if (lane == 0) {
+      sm.at[warp] = ac;
+      sm.et[warp] = ec;
+    }
+  }
+  __syncthreads();
+
+  // ---------------- pass 2: output slots (entries above tau before this one,
+  // plus the equal entries before it, at most need_eq of them)
+  uint32_t Aw = 0, Ew = 0, a_all = 0, e_all = 0;
+#pragma unroll
+  for (int i = 0; i < kBWarps; ++i) {
+    const uint32_t ai = sm.at[i], ei = sm.et[i];
+    Aw += i < warp ? ai : 0u;
+    Ew += i < warp ? ei : 0u;
+    a_all += ai;
+    e_all += ei;
+  }
+  const uint32_t chosen = a_all + (e_all < need_eq ? e_all : need_eq);
+  for (int base0 = w0; base0 < w1 && (Aw < ku); base0 += 128 * kBUnroll) {
+    float xs[kBUnroll][4];
+#pragma unroll
+    for (int u = 0; u < kBUnroll; ++u) load4(base0 + 128 * u + 4 * lane, xs[u]);
+#pragma unroll
+    for (int u = 0; u < kBUnroll; ++u) {
+    const int p = base0 + 128 * u + 4 * lane;
+    const float* x = xs[u];
+    uint32_t na = 0, ne = 0;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      na += x[c] > tau ? 1u : 0u;
+      ne += (x[c] > kNegInf && x[c] == tau) ? 1u : 0u;
+    }
+    const uint32_t packed = na | (ne << 16);
+    if (!__any_sync(0xffffffffu, packed != 0u)) continue;  // (next u)
+    uint32_t incl = packed;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const uint32_t tot = __shfl_sync(0xffffffffu, incl, 31);
+    uint32_t a_pos = Aw + ((incl - packed) & 0xffffu);
+    uint32_t e_pos = Ew + ((incl - packed) >> 16);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      if (x[c] > tau) {
+        const uint32_t slot = a_pos + (e_pos < need_eq ? e_pos : need_eq);
+        if (slot < ku) out[slot] = idrow ? idrow[p + c] : p + c;
+        ++a_pos;
+      } else if (x[c] > kNegInf && x[c] == tau) {
+        if (e_pos < need_eq && a_pos + e_pos < ku) out[a_pos + e_pos] = idrow ? idrow[p + c] : p + c;
+        ++e_pos;
+      }
+    }
+    Aw += tot & 0xffffu;
+    Ew += tot >> 16;
+    }
+  }
+  for (uint32_t i = chosen + tid; i < ku; i += kBThreads) out[i] = -1;
+}
+
 int pick_cluster(int64_t n) {
   int cl = 1;
   while (cl < kMaxCluster && static_cast<int64_t>(cl) * kSliceCap < n) cl <<= 1;
@@ -890,6 +1291,17 @@ size_t topk_smem_bytes() { return kKeysOff + static_cast<size_t>(kSliceCap) * 4;
 
 cudaError_t launch_topk(const float* scores, int T, int64_t n, int64_t row_stride, const int32_t* row_valid,
                         const int32_t* id_map, int64_t id_map_stride, int k, int32_t* idx, cudaStream_t stream) {
+  // Many rows (at least two per SM): one CTA per row, no cluster traffic.
+  // Few rows: a cluster per row, so that a small batch still spreads over the
+  // GPU.
+  const int sms = device_sm_count();
+  if (sms > 0 && static_cast<int64_t>(T) >= 2 * static_cast<int64_t>(sms)) {
+    const size_t smem = sizeof(BSmem);
+    cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(topk_band_kernel), static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    return launch_pdl(topk_band_kernel, dim3(T), dim3(kBThreads), smem, stream, 0, scores, n, row_stride, row_valid,
+                      id_map, id_map_stride, k, idx);
+  }
   if (n <= static_cast<int64_t>(kXRangeCluster) * kXThreads * 16) {
     // smallest V with ceil(n / (512 V)) <= kXRangeCluster CTAs per row
     const int V = n <= static_cast<int64_t>(kXRangeCluster) * kXThreads * 8 ? 8 : 16;

@@ -65,6 +65,33 @@ def test_topk_exact(T, n, k, ties, neg_inf, zeros):
     _check_topk(random_scores(1000 + n + k, T, n, tie_frac=ties, neg_inf_frac=neg_inf, zero_frac=zeros), n, k)
 
 
+@pytest.mark.parametrize("T,n,k,ties,neg_inf,zeros", [
+    (300, 20000, 2048, 0.0, 0.0, 0.0),     # one CTA per row (at least two rows per SM)
+    (300, 5001, 300, 0.3, 0.1, 0.1),       # ties, masked, +-0, ragged length
+    (300, 3000, 100, 0.9, 0.0, 0.0),       # threshold among massive ties: radix over the row
+    (300, 2000, 50, 0.0, 0.0, 1.0),        # all +-0
+    (300, 700, 1000, 0.0, 0.3, 0.0),       # fewer valid entries than k
+    (300, 131072, 2048, 0.1, 0.0, 0.0),    # prefill-length rows
+])
+def test_topk_many_rows(T, n, k, ties, neg_inf, zeros):
+    _check_topk(random_scores(3000 + n + k, T, n, tie_frac=ties, neg_inf_frac=neg_inf, zero_frac=zeros), n, k)
+
+
+def test_topk_many_rows_valid_and_id_map():
+    T, n, k = 320, 6000, 128
+    s = random_scores(78, T, n, tie_frac=0.2)
+    valid = torch.from_numpy(np.random.default_rng(6).integers(0, n + 1, size=T).astype(np.int32))
+    ids = torch.from_numpy(np.random.default_rng(7).integers(0, 10**6, size=(T, n)).astype(np.int32))
+    idx = misa.topk(s.cuda(), k, row_valid=valid.cuda(), id_map=ids.cuda())
+    torch.cuda.synchronize()
+    got = np_i(idx)
+    for t in range(T):
+        row = s[t].numpy().astype(np.float64).copy()
+        row[int(valid[t]):] = -np.inf
+        exp = oracle.topk_ascending(row, k, ids[t].numpy())
+        assert np.array_equal(got[t], exp), t
+
+
 def test_topk_unusual_rows():
     """Rows whose first entries are all masked, +-inf entries, a single huge
     outlier that squeezes every other value into one bin."""
