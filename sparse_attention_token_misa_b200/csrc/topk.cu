@@ -30,6 +30,8 @@
 // as many as needed.
 #include <cooperative_groups.h>
 
+#include <cstddef>
+
 #include "launch.h"
 #include "misa_device.cuh"
 
@@ -879,42 +881,47 @@ topk_range_kernel(const float* __restrict__ scores, int64_t n, int64_t row_strid
 }
 
 // ---------------------------------------------------------------------------
-// One CTA of 512 threads per row, no cluster (topk_band_kernel).  A sample of
-// the row (up to 4096 evenly spaced entries) gives a value band that holds the
-// k-th largest entry with a wide margin: the sample is binned over its value
-// range (4096 equal ranges, a monotone map), and the bins holding sample ranks
-// r - d and r + d (r the rank the k-th entry has in the sample on average, d =
-// 3 sqrt(r) + 8) bound the band.  One pass over the row counts, per warp, the
-// entries in bins above the band and gathers the band's entries (few: about
-// 2 d / 4096 of the row).  When the band holds the k-th entry, a radix select
-// over the gathered entries gives the exact threshold tau; otherwise (the
-// sample misled, or too many ties to gather) a radix select over the whole row
-// does.  A second pass writes the selected positions in order: each warp owns
-// a contiguous segment, and the per-warp counts of entries above and equal to
-// tau, scanned over the warps, give every selected entry its output slot.
-// The row is read twice (the second time mostly from L2); shared-memory
-// atomics only for the sample histogram and the radix rounds over the band.
+// One CTA of 512 threads per row, no cluster (topk_band_kernel), rows of up
+// to 131072 entries.  A sample of the row (up to 4096 evenly spaced entries)
+// gives two thresholds lo <= hi that bracket the k-th largest entry with a
+// wide margin: the sample is binned over its value range (4096 equal ranges,
+// a monotone map); the bins holding sample ranks r - d and r + d (r the rank
+// the k-th entry has in the sample on average, d = 3 sqrt(r) + 8) give hi (the
+// largest sample value not above the upper bin) and lo (the smallest sample
+// value not below the lower bin).  One pass over the row (128-entry steps
+// dealt round-robin to the warps, lane l reading entries 32 c + l so that one
+// ballot is one bitmap word) writes a bitmap of the entries above hi, counts
+// them, and gathers the band [lo, hi] with positions into per-warp buffers.
+// When the band holds the k-th entry, a radix select over the gathered
+// entries gives the exact threshold tau and the band entries above / equal to
+// it join the bitmaps; otherwise (the sample misled, too many ties to gather,
+// or fewer valid entries than k) a radix select over the whole row gives tau
+// and one more pass rebuilds the bitmaps.  The output comes from the bitmaps:
+// per-warp counts, a scan over the warps and over each warp's words give every
+// selected position its slot, so the row is read once on the common path.
 constexpr int kBThreads = 512;
 constexpr int kBWarps = kBThreads / 32;
 constexpr int kBSample = 4096;
 constexpr int kBBins = 4096;
-constexpr int kBCandCap = 4096;  // band entries kept
-#ifndef MISA_BAND_UNROLL
-#define MISA_BAND_UNROLL 1
-#endif
-constexpr int kBUnroll = MISA_BAND_UNROLL;  // 128-entry steps loaded together per warp
+constexpr int kBWarpCap = 256;                  // band entries kept per warp
+constexpr int kBCandCap = kBWarpCap * kBWarps;  // 4096
+constexpr int kBMaxN = 131072;                  // longest row (bitmaps in shared memory)
+constexpr int kBWords = kBMaxN / 32 + kBWarps * 4;  // + segment rounding
+constexpr int kBUnroll = 2;                     // steps whose loads are in flight together per warp
 
 struct BSmem {
   uint32_t hist[kBBins];
   float sval[kBSample];
-  float cval[kBCandCap];    // band entries and their warps
-  uint8_t cwarp[kBCandCap];
-  uint32_t wa[kBWarps], wv[kBWarps];  // per warp: entries above the band, valid entries
-  uint32_t at[kBWarps], et[kBWarps];  // per warp: entries above / equal to tau
+  float cval[kBCandCap];    // band entries, kBWarpCap per warp, and their positions
+  int32_t cpos[kBCandCap];
+  uint32_t gt[kBWords];     // bitmap: selected, above tau
+  uint32_t eq[kBWords];     // bitmap: equal to tau
+  uint32_t wa[kBWarps], wc[kBWarps];  // per warp: entries above hi, entries gathered
+  uint32_t at[kBWarps], et[kBWarps];  // per warp: bits set in gt / eq
   uint32_t wtmp[kBWarps];
   float wmin[kBWarps], wmax[kBWarps];
   uint32_t bc[8];
-  uint32_t ccount;
+  float fbc[2];
 };
 
 // Over hist[0, nbins) (nbins a multiple of 512, <= 4096): for each of the two
@@ -993,17 +1000,19 @@ __device__ uint32_t band_radix(BSmem& sm, int n_keys, KeyAt key_at, uint32_t nee
 
 __global__ void __launch_bounds__(kBThreads, 2)
 topk_band_kernel(const float* __restrict__ scores, int64_t n, int64_t row_stride, const int32_t* __restrict__ row_valid,
-                 const int32_t* __restrict__ id_map, int64_t id_map_stride, int k, int32_t* __restrict__ idx) {
+                 const int32_t* __restrict__ id_map, int64_t id_map_stride, int k, int32_t* __restrict__ idx,
+                 uint32_t* __restrict__ err) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   BSmem& sm = *reinterpret_cast<BSmem*>(smem_raw);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t t = blockIdx.x;
   const float kNegInf = -__int_as_float(0x7f800000);
   const float kPosInf = __int_as_float(0x7f800000);
+  const float kLowest = -__int_as_float(0x7f7fffff);  // -FLT_MAX: v >= it iff v is selectable
   const uint32_t ku = static_cast<uint32_t>(k);
   const uint32_t lt = (1u << lane) - 1u;
+  (void)err;
 
-  if (tid == 0) sm.ccount = 0;
   pdl_wait_inputs();
   pdl_allow_next();
   const float* row = scores + t * row_stride;
@@ -1015,23 +1024,13 @@ topk_band_kernel(const float* __restrict__ scores, int64_t n, int64_t row_stride
     nt64 = rv < 0 ? 0 : (rv < n ? rv : n);
   }
   const int nt = static_cast<int>(nt64);
-  // warp segments: multiples of 128 entries (32 lanes x 4)
-  const int seg = ((nt + kBWarps - 1) / kBWarps + 127) / 128 * 128;
-  const int w0 = warp * seg < nt ? warp * seg : nt;
-  const int w1 = w0 + seg < nt ? w0 + seg : nt;
-  auto load4 = [&](int p, float x[4]) {
-    if (p + 3 < w1) {
-      const float4 f = __ldg(reinterpret_cast<const float4*>(row + p));
-      x[0] = f.x;
-      x[1] = f.y;
-      x[2] = f.z;
-      x[3] = f.w;
-    } else {
+  const int nsteps = (nt + 127) / 128;  // 128-entry steps; warp w takes steps w, w + 16, ...
+  auto load_step = [&](int base, float x[4]) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) x[c] = p + c < w1 ? __ldg(row + p + c) : kNegInf;
+    for (int c = 0; c < 4; ++c) {
+      const int p = base + 32 * c + lane;
+      x[c] = p < nt ? __ldg(row + p) : kNegInf;
     }
-#pragma unroll
-    for (int c = 0; c < 4; ++c) x[c] = valid_or_neg_inf(x[c]);
   };
 
   // ---------------- sample: value range, then its histogram
@@ -1096,136 +1095,188 @@ topk_band_kernel(const float* __restrict__ scores, int64_t n, int64_t row_stride
 #pragma unroll
   for (int i = 0; i < kBWarps; ++i) nsv += sm.wtmp[i];
   __syncthreads();
-  // the band: bins [b_lo, b_hi] around sample rank r = k * ns / nt (from the top)
+  // bins holding sample ranks r -/+ d (0-based, from the top)
   const int64_t r = static_cast<int64_t>(k) * ns / (nt > 0 ? nt : 1);
   const int64_t d = static_cast<int64_t>(3.f * sqrtf(static_cast<float>(r))) + 8;
-  const int64_t r_hi = r - d, r_lo = r + d;  // 0-based ranks
+  const int64_t r_hi = r - d, r_lo = r + d;
   if (tid == 0) {
-    sm.bc[0] = kBBins;  // b_hi when r_hi < 0: no bin lies above the band
-    sm.bc[2] = 0;       // b_lo when r_lo is past the valid sample: the band reaches down to bin 0
+    sm.bc[0] = kBBins;  // r_hi < 0: nothing lies above the band
+    sm.bc[2] = 0;
   }
   __syncthreads();
   band_find(sm, sm.hist, kBBins, r_hi >= 0 ? static_cast<uint32_t>(r_hi + 1) : 0xffffffffu,
             r_lo < static_cast<int64_t>(nsv) ? static_cast<uint32_t>(r_lo + 1) : 0xffffffffu, sm.bc);
   const int b_hi = static_cast<int>(sm.bc[0]);
   const int b_lo = static_cast<int>(sm.bc[2]);
-
-  // ---------------- pass 1: per warp, entries above the band and valid
-  // entries; the band's entries are gathered
-  uint32_t a_l = 0, v_l = 0;
-
-  // kBUnroll steps' loads are issued before the first is used (memory-level
-  // parallelism: one warp keeps kBUnroll x 512 bytes in flight)
-  for (int base0 = w0; base0 < w1; base0 += 128 * kBUnroll) {
-    float xs[kBUnroll][4];
-#pragma unroll
-    for (int u = 0; u < kBUnroll; ++u) load4(base0 + 128 * u + 4 * lane, xs[u]);
-#pragma unroll
-    for (int u = 0; u < kBUnroll; ++u) {
-    const int p = base0 + 128 * u + 4 * lane;
-    const float* x = xs[u];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const bool valid = x[c] > kNegInf;
-      const int b = bin_of(x[c]);
-      a_l += (valid && b > b_hi) ? 1u : 0u;
-      v_l += valid ? 1u : 0u;
-      const bool band = valid && b >= b_lo && b <= b_hi;
-      const uint32_t bm = __ballot_sync(0xffffffffu, band);
-      if (bm) {
-        uint32_t slot0 = 0;
-        if (lane == 0) slot0 = atomicAdd(&sm.ccount, static_cast<uint32_t>(__popc(bm)));
-        slot0 = __shfl_sync(0xffffffffu, slot0, 0);
-        if (band) {
-          const uint32_t sl = slot0 + __popc(bm & lt);
-          if (sl < static_cast<uint32_t>(kBCandCap)) {
-            sm.cval[sl] = x[c];
-            sm.cwarp[sl] = static_cast<uint8_t>(warp);
-          }
-        }
-      }
-    }
+  // thresholds in value space: hi = the largest sample not above bin b_hi
+  // (+inf when nothing lies above), lo = the smallest sample not below bin b_lo
+  // (-FLT_MAX, every selectable entry, when r + d is past the valid sample)
+  float hv = kNegInf, lv = kPosInf;
+  for (int i = tid; i < ns; i += kBThreads) {
+    const float v = sm.sval[i];
+    if (v > kNegInf) {
+      const int b = bin_of(v);
+      if (b <= b_hi) hv = fmaxf(hv, v);
+      if (b >= b_lo) lv = fminf(lv, v);
     }
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
-    a_l += __shfl_xor_sync(0xffffffffu, a_l, o);
-    v_l += __shfl_xor_sync(0xffffffffu, v_l, o);
+    hv = fmaxf(hv, __shfl_xor_sync(0xffffffffu, hv, o));
+    lv = fminf(lv, __shfl_xor_sync(0xffffffffu, lv, o));
   }
   if (lane == 0) {
-    sm.wa[warp] = a_l;
-    sm.wv[warp] = v_l;
+    sm.wmax[warp] = hv;
+    sm.wmin[warp] = lv;
   }
   __syncthreads();
-  uint32_t A = 0, V = 0;
+  hv = sm.wmax[0];
+  lv = sm.wmin[0];
+#pragma unroll
+  for (int i = 1; i < kBWarps; ++i) {
+    hv = fmaxf(hv, sm.wmax[i]);
+    lv = fminf(lv, sm.wmin[i]);
+  }
+  const float hi_v = b_hi >= kBBins ? kPosInf : hv;
+  const float lo_v = (r_lo >= static_cast<int64_t>(nsv) || !(lv <= hi_v)) ? kLowest : lv;
+
+  // ---------------- pass 1 (the only read of the row on the common path)
+  uint32_t a_w = 0, c_w = 0;  // (warp-uniform) entries above hi, band entries seen
+  float* wcval = sm.cval + warp * kBWarpCap;
+  int32_t* wcpos = sm.cpos + warp * kBWarpCap;
+  for (int s0 = warp; s0 < nsteps; s0 += kBWarps * kBUnroll) {
+    float xs[kBUnroll][4];
+#pragma unroll
+    for (int u = 0; u < kBUnroll; ++u) load_step(128 * (s0 + kBWarps * u), xs[u]);
+#pragma unroll
+    for (int u = 0; u < kBUnroll; ++u) {
+      const int st = s0 + kBWarps * u;
+      if (st >= nsteps) break;
+      const int base = 128 * st;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const float x = xs[u][c];
+        const bool above = x > hi_v;                  // false for NaN
+        const bool band = !above && x >= lo_v;        // false for NaN and -inf
+        const uint32_t am = __ballot_sync(0xffffffffu, above);
+        const uint32_t bm = __ballot_sync(0xffffffffu, band);
+        if (lane == 0) sm.gt[(base >> 5) + c] = am;
+        a_w += __popc(am);
+        if (band) {
+          const uint32_t sl = c_w + __popc(bm & lt);
+          if (sl < static_cast<uint32_t>(kBWarpCap)) {
+            wcval[sl] = x;
+            wcpos[sl] = base + 32 * c + lane;
+          }
+        }
+        c_w += __popc(bm);
+      }
+    }
+  }
+  if (lane == 0) {
+    sm.wa[warp] = a_w;
+    sm.wc[warp] = c_w;
+  }
+  // the equal-to-tau bitmap starts empty
+  const int nwords = nsteps * 4;
+  for (int i = tid; i < nwords; i += kBThreads) sm.eq[i] = 0u;
+  __syncthreads();
+  uint32_t A = 0, C = 0;
+  bool full = false;
 #pragma unroll
   for (int i = 0; i < kBWarps; ++i) {
     A += sm.wa[i];
-    V += sm.wv[i];
+    C += sm.wc[i];
+    full |= sm.wc[i] > static_cast<uint32_t>(kBWarpCap);
   }
-  const uint32_t C = sm.ccount;
 
   float tau;
   uint32_t need_eq;
-  if (V <= ku) {
-    // every valid entry is selected
-    tau = kNegInf;
-    need_eq = 0;
-    if (tid < kBWarps) {
-      sm.at[tid] = sm.wv[tid];
-      sm.et[tid] = 0;
-    }
-  } else if (A < ku && ku <= A + C && C <= static_cast<uint32_t>(kBCandCap)) {
-    // the k-th entry is in the band: exact tau among the gathered entries
+  if (A < ku && ku <= A + C && !full) {
+    // the k-th entry is in the band (so at least k entries are selectable):
+    // exact tau among the gathered entries, which then join the bitmaps
     uint32_t gt;
-    const uint32_t kk = band_radix(sm, static_cast<int>(C), [&](int i) { return float_key(sm.cval[i]); }, ku - A, &gt);
+    const uint32_t kk = band_radix(
+        sm, kBCandCap,
+        [&](int i) {
+          return (i % kBWarpCap) < static_cast<int>(sm.wc[i / kBWarpCap]) ? float_key(sm.cval[i]) : 0u;
+        },
+        ku - A, &gt);
     tau = key_to_float(kk);
     need_eq = ku - A - gt;
-    if (tid < kBWarps) {
-      sm.at[tid] = sm.wa[tid];
-      sm.et[tid] = 0;
-    }
-    __syncthreads();
-    for (int i = tid; i < static_cast<int>(C); i += kBThreads) {
-      const int w = sm.cwarp[i];
+    for (int i = tid; i < kBCandCap; i += kBThreads) {
+      if ((i % kBWarpCap) >= static_cast<int>(sm.wc[i / kBWarpCap])) continue;
       const float x = sm.cval[i];
-      if (x > tau) atomicAdd(&sm.at[w], 1u);
-      else if (x == tau) atomicAdd(&sm.et[w], 1u);
+      const int p = sm.cpos[i];
+      if (x > tau) atomicOr(&sm.gt[p >> 5], 1u << (p & 31));
+      else if (x == tau) atomicOr(&sm.eq[p >> 5], 1u << (p & 31));
     }
   } else {
-    // the sample misled (or the band is too full): radix select over the row,
-    // then count per warp
-    uint32_t gt;
-    const uint32_t kk = band_radix(sm, nt, [&](int i) { return sel_key(__ldg(row + i)); }, ku, &gt);
-    tau = key_to_float(kk);
-    need_eq = ku - gt;
-    uint32_t ac = 0, ec = 0;
-    for (int base0 = w0; base0 < w1; base0 += 128 * kBUnroll) {
-      float xs[kBUnroll][4];
+    // the sample misled, too many ties to gather, or fewer selectable entries
+    // than k: count the selectable entries; exact tau by a radix select over
+    // the row when there are more than k; one more pass rebuilds the bitmaps
+    uint32_t nv = 0;
+    for (int st = warp; st < nsteps; st += kBWarps) {
+      float x[4];
+      load_step(128 * st, x);
 #pragma unroll
-      for (int u = 0; u < kBUnroll; ++u) load4(base0 + 128 * u + 4 * lane, xs[u]);
+      for (int c = 0; c < 4; ++c) nv += __popc(__ballot_sync(0xffffffffu, x[c] >= kLowest));
+    }
+    if (lane == 0) sm.wtmp[warp] = nv;
+    __syncthreads();
+    nv = 0;
 #pragma unroll
-      for (int u = 0; u < kBUnroll; ++u)
+    for (int i = 0; i < kBWarps; ++i) nv += sm.wtmp[i];
+    __syncthreads();
+    if (nv <= ku) {
+      tau = kNegInf;  // every selectable entry
+      need_eq = 0;
+    } else {
+      uint32_t gt;
+      const uint32_t kk = band_radix(sm, nt, [&](int i) { return sel_key(__ldg(row + i)); }, ku, &gt);
+      tau = key_to_float(kk);
+      need_eq = ku - gt;
+    }
+    for (int st = warp; st < nsteps; st += kBWarps) {
+      float x[4];
+      load_step(128 * st, x);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          ac += xs[u][c] > tau ? 1u : 0u;
-          ec += (xs[u][c] > kNegInf && xs[u][c] == tau) ? 1u : 0u;
+      for (int c = 0; c < 4; ++c) {
+        const float v = valid_or_neg_inf(x[c]);
+        const uint32_t gm = __ballot_sync(0xffffffffu, v > tau);
+        const uint32_t em = __ballot_sync(0xffffffffu, v > kNegInf && v == tau);
+        if (lane == 0) {
+          sm.gt[4 * st + c] = gm;
+          sm.eq[4 * st + c] = em;
         }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      ac += __shfl_xor_sync(0xffffffffu, ac, o);
-      ec += __shfl_xor_sync(0xffffffffu, ec, o);
-    }
-    if (lane == 0) {
-      sm.at[warp] = ac;
-      sm.et[warp] = ec;
+      }
     }
   }
   __syncthreads();
 
-  // ---------------- pass 2: output slots (entries above tau before this one,
-  // plus the equal entries before it, at most need_eq of them)
+  // ---------------- per-warp counts from the bitmaps, then the output: warp w
+  // owns a contiguous range of bitmap words and walks it 32 words at a time
+  // (one per lane); a scan over the lanes gives each word's first slot
+  const int wpw = (nsteps * 4 + kBWarps - 1) / kBWarps;
+  const int wd0 = warp * wpw < nsteps * 4 ? warp * wpw : nsteps * 4;
+  const int wd1 = wd0 + wpw < nsteps * 4 ? wd0 + wpw : nsteps * 4;
+  {
+    uint32_t g = 0, e = 0;
+    for (int i = wd0 + lane; i < wd1; i += 32) {
+      g += __popc(sm.gt[i]);
+      e += __popc(sm.eq[i]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      g += __shfl_xor_sync(0xffffffffu, g, o);
+      e += __shfl_xor_sync(0xffffffffu, e, o);
+    }
+    if (lane == 0) {
+      sm.at[warp] = g;
+      sm.et[warp] = e;
+    }
+  }
+  __syncthreads();
   uint32_t Aw = 0, Ew = 0, a_all = 0, e_all = 0;
 #pragma unroll
   for (int i = 0; i < kBWarps; ++i) {
@@ -1236,22 +1287,11 @@ topk_band_kernel(const float* __restrict__ scores, int64_t n, int64_t row_stride
     e_all += ei;
   }
   const uint32_t chosen = a_all + (e_all < need_eq ? e_all : need_eq);
-  for (int base0 = w0; base0 < w1 && (Aw < ku); base0 += 128 * kBUnroll) {
-    float xs[kBUnroll][4];
-#pragma unroll
-    for (int u = 0; u < kBUnroll; ++u) load4(base0 + 128 * u + 4 * lane, xs[u]);
-#pragma unroll
-    for (int u = 0; u < kBUnroll; ++u) {
-    const int p = base0 + 128 * u + 4 * lane;
-    const float* x = xs[u];
-    uint32_t na = 0, ne = 0;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      na += x[c] > tau ? 1u : 0u;
-      ne += (x[c] > kNegInf && x[c] == tau) ? 1u : 0u;
-    }
-    const uint32_t packed = na | (ne << 16);
-    if (!__any_sync(0xffffffffu, packed != 0u)) continue;  // (next u)
+  for (int i0 = wd0; i0 < wd1 && Aw < ku; i0 += 32) {
+    const int i = i0 + lane;
+    const uint32_t gw = i < wd1 ? sm.gt[i] : 0u;
+    const uint32_t ew = i < wd1 ? sm.eq[i] : 0u;
+    const uint32_t packed = static_cast<uint32_t>(__popc(gw)) | (static_cast<uint32_t>(__popc(ew)) << 16);
     uint32_t incl = packed;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -1261,20 +1301,22 @@ topk_band_kernel(const float* __restrict__ scores, int64_t n, int64_t row_stride
     const uint32_t tot = __shfl_sync(0xffffffffu, incl, 31);
     uint32_t a_pos = Aw + ((incl - packed) & 0xffffu);
     uint32_t e_pos = Ew + ((incl - packed) >> 16);
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      if (x[c] > tau) {
+    uint32_t bits = gw | ew;
+    while (bits) {
+      const int bit = __ffs(bits) - 1;
+      bits &= bits - 1;
+      const int p = i * 32 + bit;
+      if ((gw >> bit) & 1u) {
         const uint32_t slot = a_pos + (e_pos < need_eq ? e_pos : need_eq);
-        if (slot < ku) out[slot] = idrow ? idrow[p + c] : p + c;
+        if (slot < ku) out[slot] = idrow ? idrow[p] : p;
         ++a_pos;
-      } else if (x[c] > kNegInf && x[c] == tau) {
-        if (e_pos < need_eq && a_pos + e_pos < ku) out[a_pos + e_pos] = idrow ? idrow[p + c] : p + c;
+      } else {
+        if (e_pos < need_eq && a_pos + e_pos < ku) out[a_pos + e_pos] = idrow ? idrow[p] : p;
         ++e_pos;
       }
     }
     Aw += tot & 0xffffu;
     Ew += tot >> 16;
-    }
   }
   for (uint32_t i = chosen + tid; i < ku; i += kBThreads) out[i] = -1;
 }
@@ -1290,17 +1332,18 @@ int pick_cluster(int64_t n) {
 size_t topk_smem_bytes() { return kKeysOff + static_cast<size_t>(kSliceCap) * 4; }
 
 cudaError_t launch_topk(const float* scores, int T, int64_t n, int64_t row_stride, const int32_t* row_valid,
-                        const int32_t* id_map, int64_t id_map_stride, int k, int32_t* idx, cudaStream_t stream) {
+                        const int32_t* id_map, int64_t id_map_stride, int k, int32_t* idx, uint32_t* err,
+                        cudaStream_t stream) {
   // Many rows (at least two per SM): one CTA per row, no cluster traffic.
   // Few rows: a cluster per row, so that a small batch still spreads over the
   // GPU.
   const int sms = device_sm_count();
-  if (sms > 0 && static_cast<int64_t>(T) >= 2 * static_cast<int64_t>(sms)) {
+  if (sms > 0 && static_cast<int64_t>(T) >= 2 * static_cast<int64_t>(sms) && n <= kBMaxN) {
     const size_t smem = sizeof(BSmem);
     cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(topk_band_kernel), static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     return launch_pdl(topk_band_kernel, dim3(T), dim3(kBThreads), smem, stream, 0, scores, n, row_stride, row_valid,
-                      id_map, id_map_stride, k, idx);
+                      id_map, id_map_stride, k, idx, err);
   }
   if (n <= static_cast<int64_t>(kXRangeCluster) * kXThreads * 16) {
     // smallest V with ceil(n / (512 V)) <= kXRangeCluster CTAs per row
