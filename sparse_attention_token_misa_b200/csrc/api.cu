@@ -221,7 +221,7 @@ misa_status misa_topk(const float* scores, int T, int64_t n, int64_t row_stride,
   st = check_ws(workspace, workspace_bytes, kErrBytes);
   if (st != MISA_OK) return st;
   return cuda_status(misa::launch_topk(scores, T, n, row_stride, row_valid, id_map, id_map_stride, k, idx,
-                                       err_word(workspace), reinterpret_cast<cudaStream_t>(stream)));
+                                       reinterpret_cast<cudaStream_t>(stream)));
 }
 
 misa_status misa_hier_rerank(const uint16_t* q, const float* w, const uint16_t* keys, int64_t nkeyseq,
@@ -259,7 +259,7 @@ misa_status misa_hier_rerank(const uint16_t* q, const float* w, const uint16_t* 
   a.err = err_word(workspace);
   cudaError_t e = misa::launch_index_score(nullptr, a, s);
   if (e != cudaSuccess) return MISA_ERR_CUDA;
-  e = misa::launch_topk(ws_scores, T, kp, kp_pad, nullptr, cand, kp, k, idx, err_word(workspace), s);
+  e = misa::launch_topk(ws_scores, T, kp, kp_pad, nullptr, cand, kp, k, idx, s);
   if (e != cudaSuccess) return MISA_ERR_CUDA;
   if (cand_scores) {
     e = cudaMemcpy2DAsync(cand_scores, static_cast<size_t>(kp) * sizeof(float), ws_scores,
@@ -288,7 +288,7 @@ misa_status hisa_block_filter(const uint16_t* q, const float* w, const float* me
   cudaError_t e = misa::launch_hisa_block_scores(q, w, means, means_seq_stride, seq_of, prefix_len, T, H, L, B,
                                                  static_cast<int>(nseq), bs, M_pad, err_word(workspace), s);
   if (e != cudaSuccess) return MISA_ERR_CUDA;
-  e = misa::launch_topk(bs, T, M, M_pad, nullptr, nullptr, 0, m, blocks, err_word(workspace), s);
+  e = misa::launch_topk(bs, T, M, M_pad, nullptr, nullptr, 0, m, blocks, s);
   if (e != cudaSuccess) return MISA_ERR_CUDA;
   e = misa::launch_hisa_expand(blocks, prefix_len, T, m, B, L, cand, s);
   if (e != cudaSuccess) return MISA_ERR_CUDA;

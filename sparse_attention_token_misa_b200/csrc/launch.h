@@ -118,7 +118,6 @@ cudaError_t launch_index_score(const CUtensorMap* tmap, const ScoreArgs& a, cuda
 size_t topk_smem_bytes();
 
 cudaError_t launch_topk(const float* scores, int T, int64_t n, int64_t row_stride, const int32_t* row_valid,
-                        const int32_t* id_map, int64_t id_map_stride, int k, int32_t* idx, uint32_t* err,
-                        cudaStream_t stream);
+                        const int32_t* id_map, int64_t id_map_stride, int k, int32_t* idx, cudaStream_t stream);
 
 }  // namespace misa

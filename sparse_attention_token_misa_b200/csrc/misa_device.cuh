@@ -140,15 +140,6 @@ __device__ __forceinline__ void tma_load_2d_hint(void* dst, const void* map, uin
       : "memory");
 }
 
-// Bulk copy global -> shared (no tensor map): both addresses 16-byte aligned,
-// bytes a multiple of 16; completion counted in bytes on `bar`.
-__device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                   smem_u32(dst)),
-               "l"(src), "r"(bytes), "r"(smem_u32(bar))
-               : "memory");
-}
-
 // ---------------------------------------------------------------- cp.async (16-byte, zero fill)
 __device__ __forceinline__ void cp_async_16(void* dst, const void* src, bool valid) {
   const uint32_t n = valid ? 16u : 0u;

@@ -30,8 +30,6 @@
 // as many as needed.
 #include <cooperative_groups.h>
 
-#include <cstddef>
-
 #include "launch.h"
 #include "misa_device.cuh"
 
@@ -907,7 +905,10 @@ constexpr int kBWarpCap = 256;                  // band entries kept per warp
 constexpr int kBCandCap = kBWarpCap * kBWarps;  // 4096
 constexpr int kBMaxN = 131072;                  // longest row (bitmaps in shared memory)
 constexpr int kBWords = kBMaxN / 32 + kBWarps * 4;  // + segment rounding
-constexpr int kBUnroll = 2;                     // steps whose loads are in flight together per warp
+#ifndef MISA_BAND_UNROLL
+#define MISA_BAND_UNROLL 2
+#endif
+constexpr int kBUnroll = MISA_BAND_UNROLL;  // steps whose loads are in flight together per warp
 
 struct BSmem {
   uint32_t hist[kBBins];
@@ -1000,8 +1001,7 @@ __device__ uint32_t band_radix(BSmem& sm, int n_keys, KeyAt key_at, uint32_t nee
 
 __global__ void __launch_bounds__(kBThreads, 2)
 topk_band_kernel(const float* __restrict__ scores, int64_t n, int64_t row_stride, const int32_t* __restrict__ row_valid,
-                 const int32_t* __restrict__ id_map, int64_t id_map_stride, int k, int32_t* __restrict__ idx,
-                 uint32_t* __restrict__ err) {
+                 const int32_t* __restrict__ id_map, int64_t id_map_stride, int k, int32_t* __restrict__ idx) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   BSmem& sm = *reinterpret_cast<BSmem*>(smem_raw);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -1011,7 +1011,6 @@ topk_band_kernel(const float* __restrict__ scores, int64_t n, int64_t row_stride
   const float kLowest = -__int_as_float(0x7f7fffff);  // -FLT_MAX: v >= it iff v is selectable
   const uint32_t ku = static_cast<uint32_t>(k);
   const uint32_t lt = (1u << lane) - 1u;
-  (void)err;
 
   pdl_wait_inputs();
   pdl_allow_next();
@@ -1332,8 +1331,7 @@ int pick_cluster(int64_t n) {
 size_t topk_smem_bytes() { return kKeysOff + static_cast<size_t>(kSliceCap) * 4; }
 
 cudaError_t launch_topk(const float* scores, int T, int64_t n, int64_t row_stride, const int32_t* row_valid,
-                        const int32_t* id_map, int64_t id_map_stride, int k, int32_t* idx, uint32_t* err,
-                        cudaStream_t stream) {
+                        const int32_t* id_map, int64_t id_map_stride, int k, int32_t* idx, cudaStream_t stream) {
   // Many rows (at least two per SM): one CTA per row, no cluster traffic.
   // Few rows: a cluster per row, so that a small batch still spreads over the
   // GPU.
@@ -1343,7 +1341,7 @@ cudaError_t launch_topk(const float* scores, int T, int64_t n, int64_t row_strid
     cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(topk_band_kernel), static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     return launch_pdl(topk_band_kernel, dim3(T), dim3(kBThreads), smem, stream, 0, scores, n, row_stride, row_valid,
-                      id_map, id_map_stride, k, idx, err);
+                      id_map, id_map_stride, k, idx);
   }
   if (n <= static_cast<int64_t>(kXRangeCluster) * kXThreads * 16) {
     // smallest V with ceil(n / (512 V)) <= kXRangeCluster CTAs per row
