@@ -880,8 +880,8 @@ topk_range_kernel(const float* __restrict__ scores, int64_t n, int64_t row_strid
 
 // ---------------------------------------------------------------------------
 // One CTA of 512 threads per row, no cluster (topk_band_kernel), rows of up
-// to 131072 entries.  A sample of the row (up to 4096 evenly spaced entries)
-// gives two thresholds lo <= hi that bracket the k-th largest entry with a
+// to 131072 entries.  A sample of the row (4096 entries: 1024 evenly spaced
+// groups of 4 adjacent ones) gives two thresholds lo <= hi that bracket the k-th largest entry with a
 // wide margin: the sample is binned over its value range (4096 equal ranges,
 // a monotone map); the bins holding sample ranks r - d and r + d (r the rank
 // the k-th entry has in the sample on average, d = 3 sqrt(r) + 8) give hi (the
@@ -1032,24 +1032,42 @@ topk_band_kernel(const float* __restrict__ scores, int64_t n, int64_t row_stride
     }
   };
 
-  // ---------------- sample: value range, then its histogram
+  // ---------------- sample: value range, then its histogram.  Rows longer
+  // than the sample give 1024 evenly spaced groups of 4 adjacent entries (one
+  // 16-byte load each: a quarter of the DRAM bursts of 4096 scattered
+  // entries); shorter rows are sampled whole.
   const int ns = nt < kBSample ? nt : kBSample;
   float mx = kNegInf, mn = kPosInf;
   {
-    float sv[kBSample / kBThreads];  // all sample loads in flight together
+    constexpr int kG = kBSample / 4 / kBThreads;  // groups per thread (2)
+    float4 sv[kG];
 #pragma unroll
-    for (int u = 0; u < kBSample / kBThreads; ++u) {
-      const int i = tid + u * kBThreads;
-      sv[u] = i < ns ? __ldg(row + static_cast<int64_t>(i) * nt / ns) : kNegInf;
+    for (int u = 0; u < kG; ++u) {
+      const int g = tid + u * kBThreads;  // group: sample entries 4 g .. 4 g + 3
+      if (nt <= kBSample) {
+        float e[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) e[j] = 4 * g + j < nt ? __ldg(row + 4 * g + j) : kNegInf;
+        sv[u] = make_float4(e[0], e[1], e[2], e[3]);
+      } else {
+        const int p = static_cast<int>(static_cast<int64_t>(g) * nt / (kBSample / 4)) & ~3;
+        sv[u] = p + 3 < nt ? __ldg(reinterpret_cast<const float4*>(row + p))
+                           : make_float4(__ldg(row + p), p + 1 < nt ? __ldg(row + p + 1) : kNegInf,
+                                         p + 2 < nt ? __ldg(row + p + 2) : kNegInf, kNegInf);
+      }
     }
 #pragma unroll
-    for (int u = 0; u < kBSample / kBThreads; ++u) {
-      const int i = tid + u * kBThreads;
-      const float v = valid_or_neg_inf(sv[u]);
-      if (i < ns) sm.sval[i] = v;
-      if (v > kNegInf) {
-        mx = fmaxf(mx, v);
-        mn = fminf(mn, v);
+    for (int u = 0; u < kG; ++u) {
+      const int g = tid + u * kBThreads;
+      const float e[4] = {sv[u].x, sv[u].y, sv[u].z, sv[u].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float v = valid_or_neg_inf(e[j]);
+        if (4 * g + j < ns) sm.sval[4 * g + j] = v;
+        if (v > kNegInf) {
+          mx = fmaxf(mx, v);
+          mn = fminf(mn, v);
+        }
       }
     }
   }
