@@ -335,6 +335,10 @@ def run_cuda(args):
                    "parallelism": f"dp{ws_n} (independent batches)",
                    "l2": "flushed before every timed step (256 MiB write, untimed); K is 268 MB > L2"},
         "queries_per_s": T * ws_n / (ms_step * 1e-3),
+        # the work actually done: q.k products over the routed heads (MISA-8),
+        # and over all heads for the dense indexer on the same batch
+        "scored_head_pairs_per_s": pairs * h * ws_n / (ms_step * 1e-3),
+        "dense64_scored_head_pairs_per_s": pairs * H * ws_n / (dense_one_ms * 1e-3),
         "gpu_launches": 3 * args.steps,  # route, score, top-k kernels per step
         "timing": "CUDA events on the launching stream around one graph replay per step (route, score, top-k "
                   "with nothing between them); the per-kernel split from a second graph with timing events "
@@ -385,6 +389,7 @@ def other_workloads(misa, dev, stream, flush, steps, only=None):
         out.update(_prefill(misa, dev, stream, flush, steps))
     if only in (None, "dagger"):
         out.update(_dagger(misa, dev, stream, flush, steps, timed))
+        out.update(_dagger_prefill(misa, dev, stream, flush, steps, timed))
     if only in (None, "hisa"):
         out.update(_hisa(misa, dev, stream, flush, steps, timed))
     return out
@@ -430,6 +435,19 @@ def _prefill(misa, dev, stream, flush, steps):
                               "topk_ms": parts["topk"] / steps,
                               "score_tflops": flops / (score_ms * 1e-3) / 1e12,
                               "score_frac_of_bf16_peak": flops / (score_ms * 1e-3) / 1e12 / tc}
+    return out
+
+
+def _dagger_prefill(misa, dev, stream, flush, steps, timed):
+    """MISA-dagger on the causal 128K prefill: coarse top-8192 of the routed
+    scores, all-head rerank of the candidates, top-2048."""
+    out = {}
+    wl = make_workload("prefill_L131072")
+    q, w, keys, so, pl = (x.to(dev) for x in (wl.q, wl.w, wl.keys, wl.seq_of, wl.prefix_len))
+    means = misa.block_stats(keys, wl.B)
+    dg = misa.MisaDaggerIndexer(wl.T, wl.H, wl.h, wl.L, wl.B, 8192, wl.k, wl.q_block, device=dev)
+    ms = timed(lambda evs: dg.run(q, w, keys, means, so, pl))
+    out["prefill_L131072_dagger_kp8192"] = {"ms_per_step": ms, "pairs_per_s": int(wl.prefix_len.sum()) / (ms * 1e-3)}
     return out
 
 

@@ -97,6 +97,7 @@ typedef enum misa_status {
 #define MISA_DEVERR_TIMEOUT 1u    /* a bounded pipeline wait gave up */
 #define MISA_DEVERR_BAD_SEQ 2u    /* seq_of[t] outside [0, nseq) */
 #define MISA_DEVERR_BAD_HEAD 4u   /* a head id outside [0, H) */
+#define MISA_DEVERR_BAD_LEN 8u    /* misa_append_keys: len[b] < 0 or len[b] + n_new > L_cap */
 
 /* Static description of a status code (never NULL). */
 MISA_API const char* misa_status_string(int status);
@@ -110,12 +111,13 @@ MISA_API int misa_abi_version(void);
 #define MISA_OP_TOPK 3
 #define MISA_OP_HIER_RERANK 4
 #define MISA_OP_HISA_BLOCK_FILTER 5
+#define MISA_OP_APPEND_KEYS 6
 
 /* Bytes of device workspace the operation needs for these sizes (>= 256: the
  * first 256 bytes hold the device error word).  Arguments an operation does not
  * use are ignored:
  *   ROUTE_HEADS: T, H, L, B;  INDEX_SCORE: none;  TOPK: none;
- *   HIER_RERANK: T, kp;  HISA_BLOCK_FILTER: T, L, B.
+ *   HIER_RERANK: T, kp;  HISA_BLOCK_FILTER: T, L, B;  APPEND_KEYS: none.
  * Returns 0 for an unknown op or negative sizes. */
 MISA_API size_t misa_workspace_bytes(int op, int T, int H, int64_t L, int B, int k, int kp);
 
@@ -141,6 +143,35 @@ MISA_API misa_status misa_error_query(const void* workspace, misa_stream_t strea
  */
 MISA_API misa_status misa_block_stats(const uint16_t* keys, int64_t nseq, int64_t L, int64_t key_seq_stride,
                              int B, float* means, misa_stream_t stream);
+
+/*
+ * misa_append_keys -- append indexer keys to nseq caches and keep their block
+ * statistics current (the step before the indexer on every decode step).
+ *   [MISA page, "Methodology: MISA": the router reads mean-pooled blocks of the
+ *   indexer keys; HISA page, Stage 1: one mean-pooled representative per block.
+ *   How the statistics are maintained as the cache grows is not described; this
+ *   call recomputes the blocks the new keys touch.]
+ * keys: nseq caches of capacity L_cap rows (row stride 128, sequence stride
+ *   key_seq_stride >= L_cap * 128 elements when nseq > 1), device, in/out.
+ * len: [nseq] int32, device: keys already in each cache (not modified; the
+ *   caller advances it by n_new).
+ * new_keys: [nseq][n_new][128] bf16, device: copied to rows
+ *   [len[b], len[b] + n_new) of cache b.
+ * means: [nseq] x means_seq_stride fp32, device, in/out; means_seq_stride >=
+ *   ceil(L_cap / B) * 128, a multiple of 128.  Every block j that the new rows
+ *   touch is rewritten as the mean of rows [j*B, min((j+1)*B, len[b] + n_new)),
+ *   bit for bit what misa_block_stats computes on the longer cache; other
+ *   blocks are untouched.
+ * A sequence with len[b] < 0 or len[b] + n_new > L_cap is skipped and sets
+ * MISA_DEVERR_BAD_LEN in the workspace error word.
+ * Limits: 1 <= B <= 4096, 1 <= n_new, nseq >= 1; keys, new_keys, means
+ *   16-byte aligned; key_seq_stride % 8 == 0.
+ * workspace: >= 256 bytes (the error word).
+ */
+MISA_API misa_status misa_append_keys(uint16_t* keys, int64_t nseq, int64_t key_seq_stride, int64_t L_cap,
+                             const int32_t* len, const uint16_t* new_keys, int n_new, int B, float* means,
+                             int64_t means_seq_stride, void* workspace, size_t workspace_bytes,
+                             misa_stream_t stream);
 
 /*
  * misa_route_heads -- block-aggregated head router (MISA).

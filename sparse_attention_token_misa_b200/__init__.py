@@ -6,12 +6,12 @@ device tensors (`_native`), and the four indexers as preallocated call
 sequences (`indexer`).
 """
 from . import _native
-from ._native import (MisaError, alloc_workspace, block_stats, error_query, error_reset,  # noqa: F401
+from ._native import (MisaError, alloc_workspace, append_keys, block_stats, error_query, error_reset,  # noqa: F401
                       hier_rerank, hisa_block_filter, index_score, lib, route_heads, topk, workspace_bytes)
 from .indexer import DenseIndexer, HisaIndexer, MisaDaggerIndexer, MisaIndexer  # noqa: F401
 
 __all__ = [
-    "MisaError", "alloc_workspace", "block_stats", "error_query", "error_reset", "hier_rerank",
+    "MisaError", "alloc_workspace", "append_keys", "block_stats", "error_query", "error_reset", "hier_rerank",
     "hisa_block_filter", "index_score", "lib", "route_heads", "topk", "workspace_bytes",
     "DenseIndexer", "HisaIndexer", "MisaDaggerIndexer", "MisaIndexer",
 ]

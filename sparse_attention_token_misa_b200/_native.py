@@ -20,6 +20,7 @@ OP_INDEX_SCORE = 2
 OP_TOPK = 3
 OP_HIER_RERANK = 4
 OP_HISA_BLOCK_FILTER = 5
+OP_APPEND_KEYS = 6
 
 DEVERR_TIMEOUT = 1
 DEVERR_BAD_SEQ = 2
@@ -42,6 +43,8 @@ SIGNATURES = {
     "misa_error_reset": (c_int, [c_vp, c_vp]),
     "misa_error_query": (c_int, [c_vp, c_vp, ctypes.POINTER(ctypes.c_uint32)]),
     "misa_block_stats": (c_int, [c_vp, c_i64, c_i64, c_i64, c_int, c_vp, c_vp]),
+    "misa_append_keys": (c_int, [c_vp, c_i64, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_vp, c_i64, c_vp, c_size,
+                                 c_vp]),
     "misa_route_heads": (c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_i64, c_int,
                                  c_int, c_int, c_vp, c_vp, c_vp, c_size, c_vp]),
     "misa_route_heads_noalloc": (c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_i64, c_int,
@@ -150,6 +153,28 @@ def block_stats(keys: torch.Tensor, B: int, out: torch.Tensor | None = None, str
         out = torch.empty((nseq, M, HEAD_DIM), dtype=torch.float32, device=keys.device)
     _call("misa_block_stats", _p(keys), nseq, L, _key_stride(keys) if nseq > 1 else 0, B, _p(out), _stream(stream))
     return out
+
+
+def append_keys(keys: torch.Tensor, lens: torch.Tensor, new_keys: torch.Tensor, B: int, means: torch.Tensor,
+                workspace: torch.Tensor | None = None, stream=None) -> None:
+    """misa_append_keys: new_keys [nseq, n_new, 128] bf16 go to rows
+    [lens[b], lens[b] + n_new) of keys [nseq, L_cap, 128]; means [nseq, M_cap,
+    128] fp32 of the touched blocks are recomputed.  lens is not advanced."""
+    _req(keys, torch.bfloat16, "keys", contiguous=False)
+    _req(new_keys, torch.bfloat16, "new_keys")
+    _req(lens, torch.int32, "lens")
+    _req(means, torch.float32, "means", contiguous=False)
+    if keys.stride(2) != 1 or keys.stride(1) != HEAD_DIM:
+        raise ValueError("keys rows must be contiguous 128-element rows")
+    if means.stride(2) != 1 or means.stride(1) != HEAD_DIM:
+        raise ValueError("means rows must be contiguous 128-element rows")
+    nseq, L_cap, _ = keys.shape
+    n_new = new_keys.shape[1]
+    if new_keys.shape[0] != nseq or lens.numel() != nseq or means.shape[0] != nseq:
+        raise ValueError("keys, lens, new_keys and means must agree on nseq")
+    ws = workspace if workspace is not None else alloc_workspace(256, keys.device)
+    _call("misa_append_keys", _p(keys), nseq, int(keys.stride(0)) if nseq > 1 else 0, L_cap, _p(lens),
+          _p(new_keys), n_new, B, _p(means), int(means.stride(0)), _p(ws), ws.numel(), _stream(stream))
 
 
 def route_heads(q, w, means, seq_of, prefix_len, L: int, B: int, q_block: int, h: int,

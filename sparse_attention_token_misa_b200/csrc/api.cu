@@ -113,6 +113,7 @@ size_t misa_workspace_bytes(int op, int T, int H, int64_t L, int B, int k, int k
       return kErrBytes + misa::router_scratch_bytes(T, H, L, B, 1);
     case MISA_OP_INDEX_SCORE:
     case MISA_OP_TOPK:
+    case MISA_OP_APPEND_KEYS:
       return kErrBytes;
     case MISA_OP_HIER_RERANK:
       return kErrBytes + static_cast<size_t>(T) * round_up4(kp) * sizeof(float);
@@ -150,6 +151,25 @@ misa_status misa_block_stats(const uint16_t* keys, int64_t nseq, int64_t L, int6
     return MISA_ERR_INVALID_ARG;
   if (nseq > 1 && key_seq_stride < L * MISA_HEAD_DIM) return MISA_ERR_INVALID_ARG;
   return cuda_status(misa::launch_block_stats(keys, nseq, L, key_seq_stride, B, means,
+                                              reinterpret_cast<cudaStream_t>(stream)));
+}
+
+misa_status misa_append_keys(uint16_t* keys, int64_t nseq, int64_t key_seq_stride, int64_t L_cap, const int32_t* len,
+                             const uint16_t* new_keys, int n_new, int B, float* means, int64_t means_seq_stride,
+                             void* workspace, size_t workspace_bytes, misa_stream_t stream) {
+  if (!keys || !len || !new_keys || !means || nseq < 1 || L_cap < 1 || n_new < 1 || B < 1)
+    return MISA_ERR_INVALID_ARG;
+  if (B > 4096) return MISA_ERR_UNSUPPORTED;
+  if (!aligned16(keys) || !aligned16(new_keys) || !aligned16(means) || key_seq_stride < 0 || key_seq_stride % 8 != 0)
+    return MISA_ERR_INVALID_ARG;
+  if (nseq > 1 && key_seq_stride < L_cap * MISA_HEAD_DIM) return MISA_ERR_INVALID_ARG;
+  const int64_t M_cap = ceil_div(L_cap, B);
+  if (means_seq_stride % MISA_HEAD_DIM != 0 || (nseq > 1 && means_seq_stride < M_cap * MISA_HEAD_DIM))
+    return MISA_ERR_INVALID_ARG;
+  misa_status st = check_ws(workspace, workspace_bytes, kErrBytes);
+  if (st != MISA_OK) return st;
+  return cuda_status(misa::launch_append_keys(keys, nseq, key_seq_stride, L_cap, len, new_keys, n_new, B, means,
+                                              means_seq_stride, err_word(workspace),
                                               reinterpret_cast<cudaStream_t>(stream)));
 }
 

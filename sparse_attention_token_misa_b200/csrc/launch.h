@@ -56,6 +56,9 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 
 cudaError_t launch_block_stats(const uint16_t* keys, int64_t nseq, int64_t L, int64_t key_seq_stride, int B,
                                float* means, cudaStream_t stream);
+cudaError_t launch_append_keys(uint16_t* keys, int64_t nseq, int64_t key_seq_stride, int64_t L_cap,
+                               const int32_t* len, const uint16_t* new_keys, int n_new, int B, float* means,
+                               int64_t means_seq_stride, uint32_t* err, cudaStream_t stream);
 
 int router_chunks(int M);
 

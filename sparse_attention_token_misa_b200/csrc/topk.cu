@@ -901,8 +901,8 @@ constexpr int kBThreads = 512;
 constexpr int kBWarps = kBThreads / 32;
 constexpr int kBSample = 4096;
 constexpr int kBBins = 4096;
-constexpr int kBWarpCap = 256;                  // band entries kept per warp
-constexpr int kBCandCap = kBWarpCap * kBWarps;  // 4096
+constexpr int kBWarpCap = 384;                  // band entries kept per warp
+constexpr int kBCandCap = kBWarpCap * kBWarps;  // 6144
 constexpr int kBMaxN = 131072;                  // longest row (bitmaps in shared memory)
 constexpr int kBWords = kBMaxN / 32 + kBWarps * 4;  // + segment rounding
 #ifndef MISA_BAND_UNROLL
@@ -912,9 +912,11 @@ constexpr int kBUnroll = MISA_BAND_UNROLL;  // steps whose loads are in flight t
 
 struct BSmem {
   uint32_t hist[kBBins];
-  float sval[kBSample];
-  float cval[kBCandCap];    // band entries, kBWarpCap per warp, and their positions
-  int32_t cpos[kBCandCap];
+  union {
+    float sval[kBSample];     // the sample (until the thresholds are known)
+    float cval[kBCandCap];    // then the band entries, kBWarpCap per warp,
+  };
+  int32_t cpos[kBCandCap];    // and their positions
   uint32_t gt[kBWords];     // bitmap: selected, above tau
   uint32_t eq[kBWords];     // bitmap: equal to tau
   uint32_t wa[kBWarps], wc[kBWarps];  // per warp: entries above hi, entries gathered

@@ -34,7 +34,7 @@ def declared_functions():
 def test_library_loads_and_exports_every_declared_symbol():
     l = pkg.lib()
     names = declared_functions()
-    assert len(names) == 12, names
+    assert len(names) == 13, names
     for n in names:
         assert hasattr(l, n), n
         assert n in nat.SIGNATURES, n
@@ -55,6 +55,7 @@ def test_workspace_formula():
     assert ws(nat.OP_ROUTE_HEADS, 3, 5, 100, 7) == 256 + 256 + 4 * 3
     assert ws(nat.OP_INDEX_SCORE, 5, 5, 5, 5) == 256
     assert ws(nat.OP_TOPK, 5, 5, 5, 5) == 256
+    assert ws(nat.OP_APPEND_KEYS, 5, 5, 5, 5) == 256
     assert ws(nat.OP_HIER_RERANK, 64, 32, 65536, 128, 2048, 8192) == 256 + 64 * 8192 * 4
     assert ws(nat.OP_HIER_RERANK, 2, 32, 100, 1, 3, 5) == 256 + 2 * 8 * 4
     assert ws(nat.OP_HISA_BLOCK_FILTER, 16, 64, 131072, 128, 64) == 256 + 16 * 1024 * 4
@@ -172,3 +173,25 @@ def test_error_query_rejects_null():
     bits = ctypes.c_uint32(0)
     assert pkg.lib().misa_error_query(None, None, ctypes.byref(bits)) == INVALID
     assert pkg.lib().misa_error_reset(None, None) == INVALID
+
+
+def append(keys=P, nseq=2, key_seq_stride=1024 * 128, L_cap=1024, lens=P2, new_keys=P2 + 4096, n_new=1, B=128,
+           means=P2 + 8192, means_seq_stride=8 * 128, ws=P2 + 16384, ws_bytes=256):
+    return pkg.lib().misa_append_keys(keys, nseq, key_seq_stride, L_cap, lens, new_keys, n_new, B, means,
+                                      means_seq_stride, ws, ws_bytes, None)
+
+
+def test_append_keys_validation():
+    # every case is rejected on the host; nothing is launched
+    assert append(keys=None) == INVALID
+    assert append(lens=None) == INVALID
+    assert append(n_new=0) == INVALID
+    assert append(B=0) == INVALID
+    assert append(B=5000) == UNSUPPORTED
+    assert append(keys=MIS) == INVALID
+    assert append(new_keys=MIS) == INVALID
+    assert append(key_seq_stride=1023 * 128) == INVALID      # shorter than L_cap rows
+    assert append(means_seq_stride=7 * 128) == INVALID       # fewer than ceil(L_cap / B) blocks
+    assert append(means_seq_stride=8 * 128 + 4) == INVALID   # not whole 128-float rows
+    assert append(ws=None) == WORKSPACE
+    assert append(ws_bytes=255) == WORKSPACE

@@ -192,3 +192,43 @@ def test_hisa_decode_sampled(B, m):
     sample = [0, 7, 15]
     o = to_ora(wl, seqs=sample)
     _check_hisa(wl, hx, sample, _sub(o, sample, sample), B=B, m=m)
+
+
+def test_prefill_128k_dagger_sampled_blocks():
+    """MISA-dagger on the causal 128K prefill (coarse top-8192 of the routed
+    scores per query, all-head rerank of the candidates, top-2048): the first
+    and the last routing block against the oracle."""
+    wl = make_workload("prefill_L131072")
+    kp = 8192
+    g = to_gpu(wl)
+    means = misa.block_stats(g["keys"], wl.B)
+    dg = misa.MisaDaggerIndexer(wl.T, wl.H, wl.h, wl.L, wl.B, kp, wl.k, wl.q_block)
+    dg.run(g["q"], g["w"], g["keys"], means, g["seq_of"], g["prefix_len"], want_scores=True)
+    torch.cuda.synchronize()
+    G = wl.T // wl.q_block
+    blocks = [0, G - 1]
+    ts = [t for b in blocks for t in range(b * wl.q_block, (b + 1) * wl.q_block)]
+    o_sub = _sub(to_ora(wl), ts, None)
+    idx_g = np_i(dg.idx[ts])
+    cand_g = np_i(dg.coarse.idx[ts])
+    cs_g = dg.cand_scores[ts].cpu().numpy()
+    check_bit_exact_topk(idx_g, cs_g, wl.k, ids=cand_g, what="dagger idx vs CPU sort")
+    check_bit_exact_topk(cand_g, dg.coarse.scores[ts].cpu().numpy(), kp, what="dagger coarse vs CPU sort")
+    r = oracle.misa_dagger_indexer(o_sub["q"], o_sub["w"], o_sub["keys"], o_sub["seq_of"], o_sub["prefix_len"],
+                                   wl.B, wl.q_block, wl.h, kp, wl.k)
+    heads_g = np_i(dg.coarse.heads[blocks])
+    divergent = 0
+    for gi in range(len(blocks)):
+        check_selection(heads_g[gi], r["importance"][gi], wl.h, what=f"dagger heads block {blocks[gi]}")
+        rows = range(gi * wl.q_block, (gi + 1) * wl.q_block)
+        if not np.array_equal(heads_g[gi], r["heads"][gi]):
+            divergent += len(rows)
+            continue
+        for i in rows:
+            check_selection(cand_g[i], r["coarse_scores"][i], kp, what=f"dagger coarse t{ts[i]}")
+            if not np.array_equal(cand_g[i], r["cand"][i]):
+                divergent += 1
+                continue
+            check_scores(cs_g[i:i + 1].astype(np.float64), r["cand_scores"][i:i + 1], wl.k)
+            check_selection(idx_g[i], r["cand_scores"][i], wl.k, what=f"dagger t{ts[i]}", ids=r["cand"][i])
+    assert divergent <= MAX_DIVERGENT_FRAC * len(ts), divergent
