@@ -43,7 +43,10 @@ namespace {
 constexpr int kTileM = 128;                      // keys per tile (MMA M)
 constexpr int kATileBytes = kTileM * kD * 2;     // 32 KB
 constexpr int kProdThreads = 128;
-constexpr int kGatherLag = 2;
+#ifndef MISA_GATHER_LAG
+#define MISA_GATHER_LAG 2
+#endif
+constexpr int kGatherLag = MISA_GATHER_LAG;  // tiles of gathered rows in flight per producer thread
 #ifndef MISA_SHARED_EPI_WARPS
 #define MISA_SHARED_EPI_WARPS 4
 #endif
@@ -275,14 +278,29 @@ score_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreParams p) {
       }
     } else {
       // gather mode: all 128 producer threads stage the query rows, then
-      // gather the candidate key rows with 16-byte cp.async
+      // gather the candidate key rows with 16-byte cp.async.  Thread pt copies
+      // chunk pt % 16 of rows pt / 16 + 8 i (i < 16) of every tile; the
+      // candidate ids of the next tile are loaded one tile ahead, so a tile's
+      // copies are issued without waiting for its ids.
       int64_t it = 0;
       int groups = 0;
       int cur_g = -1;
       bool ok = true;
       int64_t seq_row0 = 0;
-      int32_t t_gather = 0;
       int64_t pending_from = 0;  // first iteration not yet signalled
+      constexpr int kRowsPerThread = kTileM * 16 / kProdThreads;  // 16
+      int32_t next_ids[kRowsPerThread];
+      auto load_ids = [&](int64_t item2, int32_t (&dst)[kRowsPerThread]) {
+        const int g2 = static_cast<int>(item2 / tpg);
+        const int j2 = static_cast<int>(item2 - static_cast<int64_t>(g2) * tpg);
+        const int32_t* crow = p.cand + static_cast<int64_t>(g2) * p.n_cand;
+#pragma unroll
+        for (int i = 0; i < kRowsPerThread; ++i) {
+          const int64_t pos = static_cast<int64_t>(j2) * kTileM + (pt >> 4) + 8 * i;
+          dst[i] = pos < p.n_cand ? __ldg(crow + pos) : -1;
+        }
+      };
+      if (i0 < i1) load_ids(i0, next_ids);
       for (int64_t item = i0; item < i1 && ok; ++item) {
         const int g = static_cast<int>(item / tpg);
         const int j = static_cast<int>(item - static_cast<int64_t>(g) * tpg);
@@ -297,7 +315,6 @@ score_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreParams p) {
           mbar_arrive(qfull);
           ++groups;
           cur_g = g;
-          t_gather = g;
           int64_t seq = p.seq_of[g];
           if (seq < 0 || seq >= p.nkeyseq) {
             if (pt == 0) record_error(p.err, MISA_DEVERR_BAD_SEQ);
@@ -305,16 +322,20 @@ score_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreParams p) {
           }
           seq_row0 = seq * (p.key_seq_stride / kD);
         }
+        int32_t ids[kRowsPerThread];
+#pragma unroll
+        for (int i = 0; i < kRowsPerThread; ++i) ids[i] = next_ids[i];
+        if (item + 1 < i1) load_ids(item + 1, next_ids);
+        (void)j;
         const int s = static_cast<int>(it % S);
         const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
         if (!mbar_wait(&empty[s], ph ^ 1u, p.err, abort)) { ok = false; break; }
         uint8_t* dst = sA + s * kATileBytes;
-        const int32_t* crow = p.cand + static_cast<int64_t>(t_gather) * p.n_cand;
-        for (int x = pt; x < kTileM * 16; x += kProdThreads) {
-          const int r = x >> 4, ch = x & 15;
-          const int64_t pos = static_cast<int64_t>(j) * kTileM + r;
-          int64_t id = -1;
-          if (pos < p.n_cand) id = crow[pos];
+        const int ch = pt & 15;
+#pragma unroll
+        for (int i = 0; i < kRowsPerThread; ++i) {
+          const int r = (pt >> 4) + 8 * i;
+          const int64_t id = ids[i];
           const bool valid = (id >= 0) && (id < p.L);
           const uint16_t* src = p.keys + (seq_row0 + (valid ? id : 0)) * kD + ch * 8;
           cp_async_16(dst + sw128_tile_offset(kTileM, r, ch), src, valid);
