@@ -475,6 +475,13 @@ def _hisa(misa, dev, stream, flush, steps, timed):
     dx = misa.DenseIndexer(wl.T, wl.H, wl.L, wl.k, device=dev)
     ms = timed(lambda evs: dx.run(q, w, keys, so, pl))
     out["hisa_decode_L131072_dense64"] = {"ms_per_step": ms, "pairs_per_s": int(wl.prefix_len.sum()) / (ms * 1e-3)}
+    # causal prefill: every query keeps the block its prefix cuts
+    wp = make_workload("prefill_L131072")
+    q, w, keys, so, pl = (x.to(dev) for x in (wp.q, wp.w, wp.keys, wp.seq_of, wp.prefix_len))
+    means = misa.block_stats(keys, 128)
+    hx = misa.HisaIndexer(wp.T, wp.H, wp.L, 128, 64, wp.k, device=dev)
+    ms = timed(lambda evs: hx.run(q, w, keys, means, so, pl))
+    out["prefill_L131072_hisa_B128_m64"] = {"ms_per_step": ms, "pairs_per_s": int(wp.prefix_len.sum()) / (ms * 1e-3)}
     return out
 
 

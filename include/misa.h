@@ -304,7 +304,10 @@ MISA_API misa_status misa_hier_rerank(const uint16_t* q, const float* w, const u
  *   mean-pooled block representatives only and the top-m blocks are kept, cost
  *   O(L/B); Stage 2 then looks at the at most m*B tokens inside them.]
  * block score bs[t][j] = sum over all H heads of w[t,h] * ReLU(q[t,h] . means_j)
- * for visible blocks (min((j+1)*B, L) <= prefix_len[t]), -inf otherwise.
+ * for wholly visible blocks (min((j+1)*B, L) <= prefix_len[t]); +inf for the
+ * block the prefix cuts (j*B < prefix_len[t] < min((j+1)*B, L): a causal
+ * query's own block, whose mean would include future keys, is always kept and
+ * masked token by token below); -inf otherwise.
  * blocks[t][0..m): chosen block ids ascending, -1 padded.
  * cand[t][i*B + r] = blocks[t][i]*B + r, or -1 if that block slot is empty or the
  * id is >= min(prefix_len[t], L).  block_scores: [T][M] fp32 out, may be NULL.

@@ -303,9 +303,18 @@ def hisa_block_filter(q, w, means, seq_of, prefix_len, L, B, m):
     representatives and the m best blocks are kept; Stage 2 then looks at the
     at most m*B tokens of those blocks.  HISA keeps every indexer head.
 
+    A block the prefix cuts (some of its tokens visible, some not: a causal
+    query's own, partly filled block) has a mean that includes future keys, so it
+    is not scored; it is always kept instead (score +inf) and its tokens past the
+    prefix are masked like any other -- the other m - 1 blocks are the best
+    wholly visible ones.  (The pages do not say how Stage 1 treats a partly
+    visible block; keeping the query's local block is the plainest causal
+    reading.)
+
     Returns blocks [T, m] (ascending, -1 padded), cand [T, m*B] (token ids of the
     chosen blocks in ascending order, -1 where a slot is past the prefix or past
-    the cache) and block scores [T, M] (-inf where not visible).
+    the cache) and block scores [T, M] (-inf where not visible, +inf for a block
+    the prefix cuts).
     """
     T, H, _ = q.shape
     M = (L + B - 1) // B
@@ -313,10 +322,14 @@ def hisa_block_filter(q, w, means, seq_of, prefix_len, L, B, m):
     blocks = np.full((T, m), -1, dtype=np.int64)
     cand = np.full((T, m * B), -1, dtype=np.int64)
     for t in range(T):
-        vis = visible_blocks(int(prefix_len[t]), L, B)
+        plen = int(prefix_len[t])
+        vis = visible_blocks(plen, L, B)
         if vis.size:
             A = head_block_affinity(q[t], w[t], means[seq_of[t]][vis])
             bs[t, vis] = A.sum(axis=0)
+        jp = plen // B  # the block holding token plen, if the prefix cuts it
+        if 0 <= jp < M and jp * B < plen < min((jp + 1) * B, L):
+            bs[t, jp] = np.inf
         chosen = topk_ascending(bs[t], m)
         blocks[t] = chosen
         limit = min(int(prefix_len[t]), L)

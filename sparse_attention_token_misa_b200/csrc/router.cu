@@ -45,7 +45,7 @@ block_score_kernel(const uint16_t* __restrict__ q, const float* __restrict__ w, 
     if (tid == 0) record_error(err, MISA_DEVERR_BAD_SEQ);
     seq = 0;
   }
-  // Visibility: a block is seen iff it lies wholly inside the query's prefix.
+  // Visibility: a block is scored iff it lies wholly inside the query's prefix.
   const int64_t plen = prefix_len[t];
 
   // Stage q[t] (bf16 -> fp32), w[t] and the chunk's block means (zeros past
@@ -147,7 +147,12 @@ block_score_kernel(const uint16_t* __restrict__ q, const float* __restrict__ w, 
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
       const int j = chunk * kChunk + jq * 4 + u;
-      if (lane == 0 && j < M) bscore[static_cast<int64_t>(t) * bs_stride + j] = vis[u] ? s : -__int_as_float(0x7f800000);
+      // a block the prefix cuts (a causal query's own block) is always kept:
+      // +inf; other blocks that are not wholly visible: -inf
+      const int64_t jend = (static_cast<int64_t>(j) + 1) * B < L ? (static_cast<int64_t>(j) + 1) * B : L;
+      const bool cut = static_cast<int64_t>(j) * B < plen && plen < jend;
+      const float inf = __int_as_float(0x7f800000);
+      if (lane == 0 && j < M) bscore[static_cast<int64_t>(t) * bs_stride + j] = vis[u] ? s : (cut ? inf : -inf);
   }
 }
 

@@ -39,6 +39,10 @@ def check_scores(S_gpu: np.ndarray, S_ora: np.ndarray, k: int, what: str = "scor
         mg = S_gpu[t] == -np.inf
         bad = np.nonzero(mo != mg)[0]
         assert bad.size == 0, f"{what} row {t}: mask differs at {bad[:8]} (ora {S_ora[t, bad[:4]]}, gpu {S_gpu[t, bad[:4]]})"
+        # +inf marks a forced choice (HISA: the block a causal prefix cuts): exact
+        po = S_ora[t] == np.inf
+        assert np.array_equal(po, S_gpu[t] == np.inf), f"{what} row {t}: +inf entries differ"
+        mo = mo | po
         if mo.all():
             continue
         tau = kth_threshold(S_ora[t], k)

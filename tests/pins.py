@@ -95,6 +95,25 @@ def check_hand_hisa_partial_block(orc):
     assert _one(r4["idx"]) == p["hisa_m2_top4"], r4["idx"]
 
 
+def check_hand_hisa_causal_cut_block(orc):
+    """prefix 6 with B = 4: block 0 is wholly visible, block 1 is cut (tokens 4, 5
+    visible, 6, 7 in the future).  The cut block is always kept and only its
+    visible tokens are candidates; with m = 2 the candidates are tokens 0..5."""
+    g, q, w, keys = hand_case()
+    dense = np.asarray(g["dense_scores"], dtype=np.float64)
+    r1 = orc.hisa_indexer(q, w, keys, np.array([0]), np.array([6]), 4, 1, 3)
+    assert _one(r1["blocks"]) == [1], r1["blocks"]
+    assert _one(r1["cand"]) == [4, 5, -1, -1], r1["cand"]
+    assert r1["block_scores"][0, 1] == np.inf, r1["block_scores"]
+    assert _one(r1["idx"]) == [4, 5, -1], r1["idx"]          # two visible candidates for k = 3
+    r2 = orc.hisa_indexer(q, w, keys, np.array([0]), np.array([6]), 4, 2, 3)
+    assert _one(r2["blocks"]) == [0, 1], r2["blocks"]
+    assert _one(r2["cand"]) == [0, 1, 2, 3, 4, 5, -1, -1], r2["cand"]
+    # top-3 of the dense scores over tokens 0..5 (score desc, lower id first)
+    order = sorted(range(6), key=lambda s: (-dense[s], s))[:3]
+    assert _one(r2["idx"]) == sorted(order), (r2["idx"], order)
+
+
 def check_hand_causal_router(orc):
     """prefix 6 with B = 4: only block 0 is complete; the two heads tie at 0.25
     and the lower head id wins."""
@@ -249,6 +268,21 @@ def check_invariant_hisa_covering_is_dense(orc):
             assert np.array_equal(r["idx"], idx_d), (seed, B)
 
 
+def check_invariant_hisa_causal_covering_is_dense(orc):
+    """Causal prefixes that end inside a block: with every block kept (m*B >= L)
+    HISA must still see exactly the dense indexer's tokens, the cut block's
+    visible tokens included."""
+    for seed in range(4):
+        q, w, keys, seq_of, _ = _tiny_problem(seed + 20)
+        L = keys.shape[1]
+        plen = np.array([5, 22, 36])       # mid-block prefixes for B = 4 and 5
+        idx_d, _ = orc.dense_indexer(q, w, keys, seq_of, plen, 9)
+        for B in (4, 5):
+            m = (L + B - 1) // B
+            r = orc.hisa_indexer(q, w, keys, seq_of, plen, B, m, 9)
+            assert np.array_equal(r["idx"], idx_d), (seed, B)
+
+
 def check_invariant_dagger_full_candidates_is_dense(orc):
     for seed in range(4):
         q, w, keys, seq_of, plen = _tiny_problem(seed + 20)
@@ -266,9 +300,10 @@ def check_iou(orc):
 
 ALL_CHECKS = [
     check_hand_dense, check_hand_block_means, check_hand_router, check_hand_misa,
-    check_hand_dagger, check_hand_hisa, check_hand_hisa_partial_block,
+    check_hand_dagger, check_hand_hisa, check_hand_hisa_partial_block, check_hand_hisa_causal_cut_block,
     check_hand_causal_router, check_hand_causal_scores, check_hand_candidate_scores, check_block_means_closed_form,
     check_visible_blocks, check_router_query_block_sum, check_topk_brute_force,
     check_invariant_all_heads_is_dense, check_invariant_hisa_covering_is_dense,
+    check_invariant_hisa_causal_covering_is_dense,
     check_invariant_dagger_full_candidates_is_dense, check_iou,
 ]

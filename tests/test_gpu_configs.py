@@ -232,3 +232,24 @@ def test_prefill_128k_dagger_sampled_blocks():
             check_scores(cs_g[i:i + 1].astype(np.float64), r["cand_scores"][i:i + 1], wl.k)
             check_selection(idx_g[i], r["cand_scores"][i], wl.k, what=f"dagger t{ts[i]}", ids=r["cand"][i])
     assert divergent <= MAX_DIVERGENT_FRAC * len(ts), divergent
+
+
+def test_prefill_128k_hisa_sampled():
+    """HISA on the causal 128K prefill (B = 128, m = 64): every query keeps the
+    block its prefix cuts; sampled queries against the oracle."""
+    wl = make_workload("prefill_L131072")
+    B, m = 128, 64
+    g = to_gpu(wl)
+    means = misa.block_stats(g["keys"], B)
+    hx = misa.HisaIndexer(wl.T, wl.H, wl.L, B, m, wl.k)
+    hx.run(g["q"], g["w"], g["keys"], means, g["seq_of"], g["prefix_len"])
+    torch.cuda.synchronize()
+    ts = [0, 1, 127, 1000, 2047, 4094, 4095]
+    o_sub = _sub(to_ora(wl), ts, None)
+    _check_hisa(wl, hx, ts, o_sub, B=B, m=m)
+    # the cut block is among the chosen ones wherever the prefix ends inside a block
+    blocks_g = np_i(hx.blocks[ts])
+    for i, t in enumerate(ts):
+        p = int(wl.prefix_len[t])
+        if p % B:
+            assert p // B in blocks_g[i], (t, p)

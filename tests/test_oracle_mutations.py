@@ -48,6 +48,8 @@ MUTANTS = {
     "hisa_block_sum_over_blocks": ("bs[t, vis] = A.sum(axis=0)", "bs[t, vis] = A.sum(axis=0) * 0 + A.max(axis=0)"),
     "hisa_cand_wrong_block": ("ids = np.arange(j * B, j * B + B)", "ids = np.arange(j * B + 1, j * B + B + 1)"),
     "hisa_partial_not_masked": ("ids[ids >= limit] = -1", "ids[ids > limit] = -1"),
+    "hisa_cut_block_not_kept": ("            bs[t, jp] = np.inf", "            pass"),
+    "hisa_cut_block_scored_low": ("            bs[t, jp] = np.inf", "            bs[t, jp] = -1.0"),
     "transposed_means": ("dots = q_t @ means.T", "dots = (means @ q_t.T).T[:, ::-1]"),
     "iou_intersection_as_union": ("return len(sa & sb) / len(sa | sb)", "return len(sa & sb) / max(len(sa), len(sb))"),
 }
