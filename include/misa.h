@@ -311,7 +311,7 @@ MISA_API misa_status misa_hier_rerank(const uint16_t* q, const float* w, const u
  * blocks[t][0..m): chosen block ids ascending, -1 padded.
  * cand[t][i*B + r] = blocks[t][i]*B + r, or -1 if that block slot is empty or the
  * id is >= min(prefix_len[t], L).  block_scores: [T][M] fp32 out, may be NULL.
- * means / nseq / seq_of as for misa_route_heads (means_seq_stride % 4 == 0 suffices).
+ * means / nseq / seq_of as for misa_route_heads (means_seq_stride % 128 == 0).
  * Limits: 1 <= H <= 128, 1 <= m <= MISA_MAX_TOPK, 1 <= B.
  * workspace: >= misa_workspace_bytes(MISA_OP_HISA_BLOCK_FILTER, T, H, L, B, m, 0).
  */

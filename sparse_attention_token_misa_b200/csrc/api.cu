@@ -297,6 +297,7 @@ misa_status hisa_block_filter(const uint16_t* q, const float* w, const float* me
   misa_status st = check_block_args(q, w, means, nseq, means_seq_stride, seq_of, prefix_len, T, H, L, B);
   if (st != MISA_OK) return st;
   if (!blocks || !cand || m < 1) return MISA_ERR_INVALID_ARG;
+  if (means_seq_stride % MISA_HEAD_DIM != 0) return MISA_ERR_INVALID_ARG;  // rows of 128 means for the TMA map
   if (m > MISA_MAX_TOPK || T > MISA_MAX_TOPK_ROWS) return MISA_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(m) * B >= (static_cast<int64_t>(1) << 31)) return MISA_ERR_UNSUPPORTED;
   st = check_ws(workspace, workspace_bytes, misa_workspace_bytes(MISA_OP_HISA_BLOCK_FILTER, T, H, L, B, m, 0));
@@ -305,8 +306,8 @@ misa_status hisa_block_filter(const uint16_t* q, const float* w, const float* me
   const int64_t M = ceil_div(L, B);
   const int64_t M_pad = round_up4(M);
   float* bs = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kErrBytes);
-  cudaError_t e = misa::launch_hisa_block_scores(q, w, means, means_seq_stride, seq_of, prefix_len, T, H, L, B,
-                                                 static_cast<int>(nseq), bs, M_pad, err_word(workspace), s);
+  cudaError_t e = misa::launch_hisa_block_scores_tc(q, w, means, means_seq_stride, static_cast<int>(nseq), seq_of,
+                                                    prefix_len, T, H, L, B, bs, M_pad, err_word(workspace), s);
   if (e != cudaSuccess) return MISA_ERR_CUDA;
   e = misa::launch_topk(bs, T, M, M_pad, nullptr, nullptr, 0, m, blocks, s);
   if (e != cudaSuccess) return MISA_ERR_CUDA;

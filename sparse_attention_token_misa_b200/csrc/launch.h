@@ -76,10 +76,10 @@ cudaError_t launch_route_heads_tc(const uint16_t* q, const float* w, const float
 size_t router_scratch_bytes(int T, int H, int64_t L, int B, int q_block);
 size_t router_counters_offset(int T, int H, int64_t L, int B);
 
-cudaError_t launch_hisa_block_scores(const uint16_t* q, const float* w, const float* means, int64_t means_seq_stride,
-                                     const int32_t* seq_of, const int32_t* prefix_len, int T, int H, int64_t L, int B,
-                                     int nseq_means, float* bscore, int64_t bs_stride, uint32_t* err,
-                                     cudaStream_t stream);
+cudaError_t launch_hisa_block_scores_tc(const uint16_t* q, const float* w, const float* means,
+                                        int64_t means_seq_stride, int nseq, const int32_t* seq_of,
+                                        const int32_t* prefix_len, int T, int H, int64_t L, int B, float* bscore,
+                                        int64_t bs_stride, uint32_t* err, cudaStream_t stream);
 
 cudaError_t launch_hisa_expand(const int32_t* blocks, const int32_t* prefix_len, int T, int m, int B, int64_t L,
                                int32_t* cand, cudaStream_t stream);

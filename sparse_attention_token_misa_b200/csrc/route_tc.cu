@@ -67,7 +67,9 @@ constexpr int kROffRed = (kROffTmem + 4 + 15) / 16 * 16;       // [128] row cont
 constexpr int kROffImp = kROffRed + kRM * 4;                     // [MISA_MAX_HEADS] decision importances
 constexpr int kROffImp2 = kROffImp + MISA_MAX_HEADS * 4;         // [MISA_MAX_HEADS] cluster sums
 constexpr int kROffFlag = kROffImp2 + MISA_MAX_HEADS * 4;        // flag, abort, 4 warp counts
-constexpr int kRSmemBytes = kROffFlag + 32 + 1024;
+constexpr int kTPitch = kRM + 1;                                  // HISA: [kRN][kTPitch] row contributions
+constexpr int kROffT = (kROffFlag + 32 + 15) / 16 * 16;
+constexpr int kRSmemBytes = kROffT + kRN * kTPitch * 4 + 1024;
 
 struct RouteParams {
   const uint16_t* q;
@@ -87,6 +89,8 @@ struct RouteParams {
   unsigned* counters;        // [G] items finished per decision (zero on entry)
   int32_t* heads;            // [G][h]
   float* importance;         // [G][H] or NULL
+  float* bscore;             // HISA block scores [T][bs_stride]
+  int64_t bs_stride;
   uint32_t* err;
 };
 
@@ -136,7 +140,10 @@ __device__ void select_top_h(const float* imp, int H, int h, int g, int32_t* hea
   if (sel && pos < h) heads[static_cast<int64_t>(g) * h + pos] = tid;
 }
 
-template <bool kCluster>
+// kHisa: the same MMAs give the HISA block scores instead: per (query, block)
+// the sum over heads of w * ReLU(q . mean), written out per block tile (no
+// reduction across work items).
+template <bool kCluster, bool kHisa>
 __global__ void __launch_bounds__(kRThreads, 1)
 route_tc_kernel(const __grid_constant__ CUtensorMap means_map, const __grid_constant__ CUtensorMap q_map,
                 const RouteParams p) {
@@ -347,6 +354,43 @@ route_tc_kernel(const __grid_constant__ CUtensorMap means_map, const __grid_cons
       }
       const int a = static_cast<int>(it & 1);
       const uint32_t aph = static_cast<uint32_t>((it >> 1) & 1);
+      if constexpr (kHisa) {
+        // rows (ql, hh) of the tile through shared memory, then thread
+        // (ql, jj) adds its query's heads in ascending order
+        float* tb = reinterpret_cast<float*>(smem + kROffT);
+        if (!skip && mbar_wait(&tfull[a], aph, p.err, abort)) {
+          tc_fence_after();
+          uint32_t v[kRN];
+#pragma unroll
+          for (int u = 0; u < kRN / 16; ++u) tmem_ld16(t_lane + static_cast<uint32_t>(a * kRN + 16 * u), v + 16 * u);
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(&tempty[a]);
+#pragma unroll
+          for (int jj = 0; jj < kRN; ++jj) tb[jj * kTPitch + r] = wrow * fmaxf(__uint_as_float(v[jj]), 0.f);
+        } else {
+          skip = true;
+        }
+        named_bar_sync(1, kREpiThreads);
+        if (!skip && tid < p.qpm * kRN) {
+          const int ql = tid / kRN, jj = tid - ql * kRN;
+          const int t = pg * p.qpm + ql;
+          const int64_t j = static_cast<int64_t>(bt) * kRN + jj;
+          if (t < p.T && j < p.M) {
+            float sum = 0.f;
+            for (int hh = 0; hh < p.H; ++hh) sum += tb[jj * kTPitch + ql * p.H + hh];
+            // wholly visible: the score; cut by the prefix (the query's own
+            // block): +inf, always kept; later: -inf
+            const int64_t plen = p.prefix_len[t];
+            const int64_t end = (j + 1) * p.B < p.L ? (j + 1) * p.B : p.L;
+            const float inf = __int_as_float(0x7f800000);
+            p.bscore[static_cast<int64_t>(t) * p.bs_stride + j] =
+                end <= plen ? sum : ((j * p.B < plen && plen < end) ? inf : -inf);
+          }
+        }
+        named_bar_sync(1, kREpiThreads);  // tb is reused by the next item
+        continue;
+      }
       float contrib = 0.f;
       if (!skip && mbar_wait(&tfull[a], aph, p.err, abort)) {
         tc_fence_after();
@@ -462,7 +506,7 @@ cudaError_t launch_route_heads_tc(const uint16_t* q, const float* w, const float
                                   int B, int q_block, int h, int qpm, int32_t* heads, float* importance,
                                   float* partial, unsigned* counters, bool clear_counters, uint32_t* err,
                                   cudaStream_t stream) {
-  RouteParams p;
+  RouteParams p = {};
   p.q = q;
   p.w = w;
   p.means_seq_rows = means_seq_stride / kD;
@@ -503,20 +547,64 @@ cudaError_t launch_route_heads_tc(const uint16_t* q, const float* w, const float
   const bool cluster = items_per_dec <= 8 * kRMaxCluster && static_cast<int64_t>(G) * D <= sms;
   cudaError_t e = cudaSuccess;
   if (cluster) {
-    e = ensure_dynamic_smem(reinterpret_cast<const void*>(route_tc_kernel<true>), kRSmemBytes);
+    e = ensure_dynamic_smem(reinterpret_cast<const void*>(route_tc_kernel<true, false>), kRSmemBytes);
     if (e != cudaSuccess) return e;
-    return launch_pdl(route_tc_kernel<true>, dim3(static_cast<unsigned>(G * D)), dim3(kRThreads), kRSmemBytes, stream,
+    return launch_pdl(route_tc_kernel<true, false>, dim3(static_cast<unsigned>(G * D)), dim3(kRThreads), kRSmemBytes, stream,
                       D, map, qmap, p);
   }
   if (clear_counters) {
     e = cudaMemsetAsync(counters, 0, static_cast<size_t>(G) * sizeof(unsigned), stream);
     if (e != cudaSuccess) return e;
   }
-  e = ensure_dynamic_smem(reinterpret_cast<const void*>(route_tc_kernel<false>), kRSmemBytes);
+  e = ensure_dynamic_smem(reinterpret_cast<const void*>(route_tc_kernel<false, false>), kRSmemBytes);
   if (e != cudaSuccess) return e;
   const int64_t grid = p.n_items < sms ? p.n_items : sms;
-  return launch_pdl(route_tc_kernel<false>, dim3(static_cast<unsigned>(grid)), dim3(kRThreads), kRSmemBytes, stream, 0,
+  return launch_pdl(route_tc_kernel<false, false>, dim3(static_cast<unsigned>(grid)), dim3(kRThreads), kRSmemBytes, stream, 0,
                     map, qmap, p);
+}
+
+cudaError_t launch_hisa_block_scores_tc(const uint16_t* q, const float* w, const float* means,
+                                        int64_t means_seq_stride, int nseq, const int32_t* seq_of,
+                                        const int32_t* prefix_len, int T, int H, int64_t L, int B, float* bscore,
+                                        int64_t bs_stride, uint32_t* err, cudaStream_t stream) {
+  if (H > kRM) return cudaErrorInvalidValue;
+  const bool shared = nseq == 1 || means_seq_stride == 0;
+  int qpm = 1;
+  while (shared && qpm * 2 * H <= kRM) qpm *= 2;
+  RouteParams p = {};
+  p.q = q;
+  p.w = w;
+  p.means_seq_rows = means_seq_stride / kD;
+  p.nseq = nseq;
+  p.seq_of = seq_of;
+  p.prefix_len = prefix_len;
+  p.T = T;
+  p.H = H;
+  p.L = L;
+  p.B = B;
+  p.M = static_cast<int>((L + B - 1) / B);
+  p.q_block = qpm;  // (no routing decisions in this mode)
+  p.h = 1;
+  p.qpm = qpm;
+  p.n_pg = (T + qpm - 1) / qpm;
+  p.n_bt = (p.M + kRN - 1) / kRN;
+  p.n_items = static_cast<int64_t>(p.n_pg) * p.n_bt;
+  p.bscore = bscore;
+  p.bs_stride = bs_stride;
+  p.err = err;
+  CUtensorMap map;
+  const uint64_t rows = static_cast<uint64_t>(nseq - 1) * static_cast<uint64_t>(p.means_seq_rows) + p.M;
+  if (!encode_2d_map(&map, false, means, kD, rows, kD * 4, kD, kRN, false)) return cudaErrorInvalidValue;
+  CUtensorMap qmap;
+  if (!encode_2d_map(&qmap, true, q, kD, static_cast<uint64_t>(T) * H, kD * 2, 64, kRM, true))
+    return cudaErrorInvalidValue;
+  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(route_tc_kernel<false, true>), kRSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int sms = device_sm_count();
+  if (sms <= 0) return cudaErrorInvalidDevice;
+  const int64_t grid = p.n_items < sms ? p.n_items : sms;
+  return launch_pdl(route_tc_kernel<false, true>, dim3(static_cast<unsigned>(grid)), dim3(kRThreads), kRSmemBytes,
+                    stream, 0, map, qmap, p);
 }
 
 }  // namespace misa

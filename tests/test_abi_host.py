@@ -167,6 +167,8 @@ def test_hier_rerank_and_hisa_reject():
     assert hf(P, P, P, 1, 0, P, P, 2, 64, 1000, 128, 20000, P2, P2, None, P2, 1 << 20, None) == UNSUPPORTED
     assert hf(P, P, P, 1, 0, P, P, 2, 64, 1000, 128, 4, None, P2, None, P2, 1 << 20, None) == INVALID
     assert hf(P, P, P, 1, 0, P, P, 2, 64, 1000, 128, 4, P2, P2, None, P2, 256, None) == WORKSPACE
+    # sequence stride of the means: whole 128-float rows (TMA rows)
+    assert hf(P, P, P, 2, 8 * 128 + 4, P, P, 2, 64, 1000, 128, 4, P2, P2, None, P2, 1 << 20, None) == INVALID
 
 
 def test_error_query_rejects_null():
