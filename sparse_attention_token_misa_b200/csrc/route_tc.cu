@@ -355,8 +355,8 @@ route_tc_kernel(const __grid_constant__ CUtensorMap means_map, const __grid_cons
       const int a = static_cast<int>(it & 1);
       const uint32_t aph = static_cast<uint32_t>((it >> 1) & 1);
       if constexpr (kHisa) {
-        // rows (ql, hh) of the tile through shared memory, then thread
-        // (ql, jj) adds its query's heads in ascending order
+        // rows (ql, hh) of the tile through shared memory, then each (query
+        // ql, block jj) pair adds its query's heads in ascending order
         float* tb = reinterpret_cast<float*>(smem + kROffT);
         if (!skip && mbar_wait(&tfull[a], aph, p.err, abort)) {
           tc_fence_after();
@@ -372,8 +372,8 @@ route_tc_kernel(const __grid_constant__ CUtensorMap means_map, const __grid_cons
           skip = true;
         }
         named_bar_sync(1, kREpiThreads);
-        if (!skip && tid < p.qpm * kRN) {
-          const int ql = tid / kRN, jj = tid - ql * kRN;
+        for (int x = tid; !skip && x < p.qpm * kRN; x += kREpiThreads) {
+          const int ql = x / kRN, jj = x - ql * kRN;
           const int t = pg * p.qpm + ql;
           const int64_t j = static_cast<int64_t>(bt) * kRN + jj;
           if (t < p.T && j < p.M) {

@@ -266,6 +266,27 @@ def test_hisa_block_filter(T, L, B, m):
         assert np.array_equal(cand_g[t], exp), t
 
 
+@pytest.mark.parametrize("T,L,H,B,m", [(9, 3000, 32, 128, 6), (6, 1500, 16, 64, 5), (5, 2000, 64, 100, 4)])
+def test_hisa_block_filter_shared_cache_causal(T, L, H, B, m):
+    """One cache shared by every query (several queries per MMA row group),
+    causal prefixes that end inside a block (the cut block is kept, +inf)."""
+    wl = make_prefill("hfp", 500 + L, T=T, L=L, H=H, h=H, B=B, k=16, q_block=1, n_regions=0, region_len=1,
+                      first_pos=L // 3)
+    g, o = to_gpu(wl), to_ora(wl)
+    means = oracle.block_means(o["keys"][0], B)[None]
+    blocks_o, cand_o, bs_o = oracle.hisa_block_filter(o["q"], o["w"], means, o["seq_of"], o["prefix_len"], L, B, m)
+    blocks, cand, bs = misa.hisa_block_filter(g["q"], g["w"], dev(torch.from_numpy(means).float()), g["seq_of"],
+                                              g["prefix_len"], L, B, m, want_scores=True)
+    torch.cuda.synchronize()
+    check_scores(np_f(bs), bs_o, m, what="block scores")
+    blocks_g = np_i(blocks)
+    for t in range(T):
+        check_selection(blocks_g[t], bs_o[t], m, what=f"blocks t{t}")
+        p = int(wl.prefix_len[t])
+        if p % B and p < L:
+            assert p // B in blocks_g[t], (t, p)
+
+
 # ------------------------------------------------------------------ MISA-dagger rerank
 def test_hier_rerank():
     T, L, H, kp, k = 5, 4000, 32, 700, 150
