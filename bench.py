@@ -199,7 +199,7 @@ def run_cuda(args):
     T, H, h, L, B, k = wl.T, wl.H, wl.h, wl.L, wl.B, wl.k
     pairs = int(wl.prefix_len.sum())
 
-    means = misa.block_stats(keys, B)
+    means = misa.block_stats(keys, B, split=True)
     ix = misa.MisaIndexer(T, H, h, L, B, k, q_block=1, device=dev)
     dense = misa.DenseIndexer(T, H, L, k, device=dev)
     flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
@@ -268,7 +268,8 @@ def run_cuda(args):
                                                 dense.g_select.replay()), args.steps, flush, stream,
                                    marks=["score", "topk"])
     dense_one_ms, _ = _time_steps(lambda evs: dense.g_step.replay(), args.steps, flush, stream)
-    stats_ms, _ = _time_steps(lambda evs: misa.block_stats(keys, B, out=means), args.steps, flush, stream)
+    stats_ms, _ = _time_steps(lambda evs: misa.block_stats(keys, B, out=means[0], out_hi=means[1], out_lo=means[2]),
+                              args.steps, flush, stream)
     dense_ms /= args.steps
     dense_one_ms /= args.steps
     stats_ms /= args.steps
@@ -357,7 +358,7 @@ def run_cuda(args):
                    "dense64_ms": dense_one_ms, "dense64_score_ms": dparts["score"] / args.steps,
                    "dense64_topk_ms": dparts["topk"] / args.steps, "dense64_over_misa8": dense_one_ms / ms_step,
                    "block_stats_ms": stats_ms,
-                   "block_stats_GBps": (T * L * 128 * 2 + T * (L // B) * 128 * 4) / (stats_ms * 1e-3) / 1e9,
+                   "block_stats_GBps": (T * L * 128 * 2 + T * (L // B) * 128 * 8) / (stats_ms * 1e-3) / 1e9,
                    "wall_s_timed_region": wall},
     }
     summ = clk.summary()
@@ -399,7 +400,7 @@ def _prefill(misa, dev, stream, flush, steps):
     out = {}
     wl = make_workload("prefill_L131072")
     q, w, keys, so, pl = (x.to(dev) for x in (wl.q, wl.w, wl.keys, wl.seq_of, wl.prefix_len))
-    means = misa.block_stats(keys, wl.B)
+    means = misa.block_stats(keys, wl.B, split=True)
     ix = misa.MisaIndexer(wl.T, wl.H, wl.h, wl.L, wl.B, wl.k, wl.q_block, device=dev)
     pairs = int(wl.prefix_len.sum())
 
@@ -444,7 +445,7 @@ def _dagger_prefill(misa, dev, stream, flush, steps, timed):
     out = {}
     wl = make_workload("prefill_L131072")
     q, w, keys, so, pl = (x.to(dev) for x in (wl.q, wl.w, wl.keys, wl.seq_of, wl.prefix_len))
-    means = misa.block_stats(keys, wl.B)
+    means = misa.block_stats(keys, wl.B, split=True)
     dg = misa.MisaDaggerIndexer(wl.T, wl.H, wl.h, wl.L, wl.B, 8192, wl.k, wl.q_block, device=dev)
     ms = timed(lambda evs: dg.run(q, w, keys, means, so, pl))
     out["prefill_L131072_dagger_kp8192"] = {"ms_per_step": ms, "pairs_per_s": int(wl.prefix_len.sum()) / (ms * 1e-3)}
@@ -455,7 +456,7 @@ def _dagger(misa, dev, stream, flush, steps, timed):
     out = {}
     wl = make_workload("glm5_dagger_decode_L65536")
     q, w, keys, so, pl = (x.to(dev) for x in (wl.q, wl.w, wl.keys, wl.seq_of, wl.prefix_len))
-    means = misa.block_stats(keys, wl.B)
+    means = misa.block_stats(keys, wl.B, split=True)
     dg = misa.MisaDaggerIndexer(wl.T, wl.H, wl.h, wl.L, wl.B, wl.kp, wl.k, device=dev)
     ms = timed(lambda evs: dg.run(q, w, keys, means, so, pl))
     out["glm5_dagger_decode_L65536"] = {"ms_per_step": ms, "pairs_per_s": int(wl.prefix_len.sum()) / (ms * 1e-3)}
@@ -467,7 +468,7 @@ def _hisa(misa, dev, stream, flush, steps, timed):
     wl = make_workload("hisa_decode_L131072")
     q, w, keys, so, pl = (x.to(dev) for x in (wl.q, wl.w, wl.keys, wl.seq_of, wl.prefix_len))
     for B, m in ((128, 64), (64, 128)):
-        means = misa.block_stats(keys, B)
+        means = misa.block_stats(keys, B, split=True)
         hx = misa.HisaIndexer(wl.T, wl.H, wl.L, B, m, wl.k, device=dev)
         ms = timed(lambda evs: hx.run(q, w, keys, means, so, pl))
         out[f"hisa_decode_L131072_B{B}_m{m}"] = {"ms_per_step": ms,
@@ -478,7 +479,7 @@ def _hisa(misa, dev, stream, flush, steps, timed):
     # causal prefill: every query keeps the block its prefix cuts
     wp = make_workload("prefill_L131072")
     q, w, keys, so, pl = (x.to(dev) for x in (wp.q, wp.w, wp.keys, wp.seq_of, wp.prefix_len))
-    means = misa.block_stats(keys, 128)
+    means = misa.block_stats(keys, 128, split=True)
     hx = misa.HisaIndexer(wp.T, wp.H, wp.L, 128, 64, wp.k, device=dev)
     ms = timed(lambda evs: hx.run(q, w, keys, means, so, pl))
     out["prefill_L131072_hisa_B128_m64"] = {"ms_per_step": ms, "pairs_per_s": int(wp.prefix_len.sum()) / (ms * 1e-3)}

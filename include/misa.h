@@ -138,11 +138,17 @@ MISA_API misa_status misa_error_query(const void* workspace, misa_stream_t strea
  *   means[b * M * 128 + j * 128 + c] = mean over s in block j of keys[b][s][c]
  * as fp32 (fp32 accumulation of the bf16 inputs), M = ceil(L / B); the last,
  * partial block averages the L - (M-1)*B keys it holds.
- * Limits: 1 <= B <= 4096, L >= 1, nseq >= 1.  keys 16-byte aligned,
- * key_seq_stride % 8 == 0.
+ * means_hi, means_lo: both NULL, or both [nseq][M][128] bf16 at the same
+ * element offsets as means, receiving the split of each mean m into
+ * hi = bf16(m) and lo = bf16(m - hi) (round to nearest even), the two operands
+ * the tensor-core router multiplies (about 16 significant bits together).
+ * Passing them to misa_route_heads / hisa_block_filter saves the per-call split.
+ * Limits: 1 <= B <= 4096, L >= 1, nseq >= 1.  keys, means, means_hi, means_lo
+ * 16-byte aligned, key_seq_stride % 8 == 0.
  */
 MISA_API misa_status misa_block_stats(const uint16_t* keys, int64_t nseq, int64_t L, int64_t key_seq_stride,
-                             int B, float* means, misa_stream_t stream);
+                             int B, float* means, uint16_t* means_hi, uint16_t* means_lo,
+                             misa_stream_t stream);
 
 /*
  * misa_append_keys -- append indexer keys to nseq caches and keep their block
@@ -162,16 +168,19 @@ MISA_API misa_status misa_block_stats(const uint16_t* keys, int64_t nseq, int64_
  *   touch is rewritten as the mean of rows [j*B, min((j+1)*B, len[b] + n_new)),
  *   bit for bit what misa_block_stats computes on the longer cache; other
  *   blocks are untouched.
+ * means_hi, means_lo: both NULL, or both bf16 at the same element offsets as
+ *   means (stride means_seq_stride), in/out: the touched blocks' split is
+ *   rewritten as misa_block_stats writes it.
  * A sequence with len[b] < 0 or len[b] + n_new > L_cap is skipped and sets
  * MISA_DEVERR_BAD_LEN in the workspace error word.
- * Limits: 1 <= B <= 4096, 1 <= n_new, nseq >= 1; keys, new_keys, means
- *   16-byte aligned; key_seq_stride % 8 == 0.
+ * Limits: 1 <= B <= 4096, 1 <= n_new, nseq >= 1; keys, new_keys, means,
+ *   means_hi, means_lo 16-byte aligned; key_seq_stride % 8 == 0.
  * workspace: >= 256 bytes (the error word).
  */
 MISA_API misa_status misa_append_keys(uint16_t* keys, int64_t nseq, int64_t key_seq_stride, int64_t L_cap,
                              const int32_t* len, const uint16_t* new_keys, int n_new, int B, float* means,
-                             int64_t means_seq_stride, void* workspace, size_t workspace_bytes,
-                             misa_stream_t stream);
+                             uint16_t* means_hi, uint16_t* means_lo, int64_t means_seq_stride,
+                             void* workspace, size_t workspace_bytes, misa_stream_t stream);
 
 /*
  * misa_route_heads -- block-aggregated head router (MISA).
@@ -188,13 +197,16 @@ MISA_API misa_status misa_append_keys(uint16_t* keys, int64_t nseq, int64_t key_
  *   means: nseq sequences of [M][128] fp32 at sequence stride means_seq_stride
  *          elements (as written by misa_block_stats: M * 128); 16-byte aligned,
  *          means_seq_stride % 128 == 0; seq_of values must lie in [0, nseq).
+ *   means_hi, means_lo: both NULL, or both the bf16 split misa_block_stats
+ *          writes, laid out like means.  When given they are read instead of
+ *          means (which may then be NULL) and the results are bit-identical.
  *   heads: [ceil(T/q_block)][h] int32 out.  importance: [ceil(T/q_block)][H]
  *          fp32 out, may be NULL.
  * Limits: 1 <= H <= 128, 1 <= h <= H, 1 <= q_block, T >= 1.
  * workspace: >= misa_workspace_bytes(MISA_OP_ROUTE_HEADS, T, H, L, B, 0, 0).
  */
 MISA_API misa_status misa_route_heads(const uint16_t* q, const float* w, const float* means,
-                             int64_t nseq, int64_t means_seq_stride, const int32_t* seq_of,
+                             const uint16_t* means_hi, const uint16_t* means_lo, int64_t nseq, int64_t means_seq_stride, const int32_t* seq_of,
                              const int32_t* prefix_len, int T, int H, int64_t L, int B,
                              int q_block, int h, int32_t* heads, float* importance,
                              void* workspace, size_t workspace_bytes, misa_stream_t stream);
@@ -205,8 +217,9 @@ MISA_API misa_status misa_route_heads(const uint16_t* q, const float* w, const f
  * For callers that cannot allocate device memory at the point where they route:
  * an inference engine that reserved all device memory up front and gives its
  * plug-ins no allocator, or a serving loop that must not call cudaMalloc /
- * cudaFree because they can synchronise the whole device.  Inputs, outputs and
- * results are exactly those of misa_route_heads (same kernels); only the
+ * cudaFree because they can synchronise the whole device.  Inputs (fp32 means
+ * only, no bf16 split), outputs and results are exactly those of
+ * misa_route_heads (same kernels); only the
  * router's per-chunk partial importances move from the workspace into a fixed
  * array of MISA_ROUTE_NOALLOC_SCRATCH_BYTES bytes compiled into the library,
  * which every device that loads the library holds until the process exits.
@@ -311,12 +324,13 @@ MISA_API misa_status misa_hier_rerank(const uint16_t* q, const float* w, const u
  * blocks[t][0..m): chosen block ids ascending, -1 padded.
  * cand[t][i*B + r] = blocks[t][i]*B + r, or -1 if that block slot is empty or the
  * id is >= min(prefix_len[t], L).  block_scores: [T][M] fp32 out, may be NULL.
- * means / nseq / seq_of as for misa_route_heads (means_seq_stride % 128 == 0).
+ * means / means_hi / means_lo / nseq / seq_of as for misa_route_heads
+ * (means_seq_stride % 128 == 0).
  * Limits: 1 <= H <= 128, 1 <= m <= MISA_MAX_TOPK, 1 <= B.
  * workspace: >= misa_workspace_bytes(MISA_OP_HISA_BLOCK_FILTER, T, H, L, B, m, 0).
  */
 MISA_API misa_status hisa_block_filter(const uint16_t* q, const float* w, const float* means,
-                              int64_t nseq, int64_t means_seq_stride, const int32_t* seq_of,
+                              const uint16_t* means_hi, const uint16_t* means_lo, int64_t nseq, int64_t means_seq_stride, const int32_t* seq_of,
                               const int32_t* prefix_len, int T, int H, int64_t L, int B, int m,
                               int32_t* blocks, int32_t* cand, float* block_scores,
                               void* workspace, size_t workspace_bytes, misa_stream_t stream);

@@ -42,11 +42,11 @@ SIGNATURES = {
     "misa_workspace_bytes": (c_size, [c_int, c_int, c_int, c_i64, c_int, c_int, c_int]),
     "misa_error_reset": (c_int, [c_vp, c_vp]),
     "misa_error_query": (c_int, [c_vp, c_vp, ctypes.POINTER(ctypes.c_uint32)]),
-    "misa_block_stats": (c_int, [c_vp, c_i64, c_i64, c_i64, c_int, c_vp, c_vp]),
-    "misa_append_keys": (c_int, [c_vp, c_i64, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_vp, c_i64, c_vp, c_size,
-                                 c_vp]),
-    "misa_route_heads": (c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_i64, c_int,
-                                 c_int, c_int, c_vp, c_vp, c_vp, c_size, c_vp]),
+    "misa_block_stats": (c_int, [c_vp, c_i64, c_i64, c_i64, c_int, c_vp, c_vp, c_vp, c_vp]),
+    "misa_append_keys": (c_int, [c_vp, c_i64, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_vp, c_vp, c_vp, c_i64,
+                                 c_vp, c_size, c_vp]),
+    "misa_route_heads": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_i64,
+                                 c_int, c_int, c_int, c_vp, c_vp, c_vp, c_size, c_vp]),
     "misa_route_heads_noalloc": (c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_i64, c_int,
                                          c_int, c_int, c_vp, c_vp, c_vp]),
     "misa_index_score": (c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_i64, c_vp, c_int,
@@ -54,8 +54,8 @@ SIGNATURES = {
     "misa_topk": (c_int, [c_vp, c_int, c_i64, c_i64, c_vp, c_vp, c_i64, c_int, c_vp, c_vp, c_size, c_vp]),
     "misa_hier_rerank": (c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_i64, c_vp, c_int,
                                  c_int, c_vp, c_vp, c_vp, c_size, c_vp]),
-    "hisa_block_filter": (c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_i64, c_int, c_int,
-                                  c_vp, c_vp, c_vp, c_vp, c_size, c_vp]),
+    "hisa_block_filter": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_i64,
+                                  c_int, c_int, c_vp, c_vp, c_vp, c_vp, c_size, c_vp]),
 }
 
 
@@ -142,8 +142,22 @@ def _key_stride(keys: torch.Tensor) -> int:
     return 0 if keys.shape[0] == 1 else int(keys.stride(0))
 
 
-def block_stats(keys: torch.Tensor, B: int, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """misa_block_stats: keys [nseq, L, 128] bf16 -> means [nseq, M, 128] fp32."""
+def _split_pair(hi, lo, like: torch.Tensor | None = None):
+    """Check the bf16 hi / lo split of the block means (both or neither)."""
+    if (hi is None) != (lo is None):
+        raise ValueError("means_hi and means_lo go together")
+    if hi is None:
+        return
+    _req(hi, torch.bfloat16, "means_hi"); _req(lo, torch.bfloat16, "means_lo")
+    for t in (hi, lo):
+        if like is not None and (t.shape != like.shape or t.stride() != like.stride()):
+            raise ValueError("the split must be laid out like the fp32 means")
+
+
+def block_stats(keys: torch.Tensor, B: int, out: torch.Tensor | None = None, stream=None, split: bool = False,
+                out_hi: torch.Tensor | None = None, out_lo: torch.Tensor | None = None):
+    """misa_block_stats: keys [nseq, L, 128] bf16 -> means [nseq, M, 128] fp32,
+    or (means, means_hi, means_lo) with the bf16 split when split=True."""
     _req(keys, torch.bfloat16, "keys", contiguous=False)
     if keys.stride(2) != 1 or keys.stride(1) != HEAD_DIM:
         raise ValueError("keys rows must be contiguous 128-element rows")
@@ -151,15 +165,21 @@ def block_stats(keys: torch.Tensor, B: int, out: torch.Tensor | None = None, str
     M = (L + B - 1) // B
     if out is None:
         out = torch.empty((nseq, M, HEAD_DIM), dtype=torch.float32, device=keys.device)
-    _call("misa_block_stats", _p(keys), nseq, L, _key_stride(keys) if nseq > 1 else 0, B, _p(out), _stream(stream))
-    return out
+    if split and out_hi is None:
+        out_hi = torch.empty((nseq, M, HEAD_DIM), dtype=torch.bfloat16, device=keys.device)
+        out_lo = torch.empty_like(out_hi)
+    _split_pair(out_hi, out_lo, out)
+    _call("misa_block_stats", _p(keys), nseq, L, _key_stride(keys) if nseq > 1 else 0, B, _p(out), _p(out_hi),
+          _p(out_lo), _stream(stream))
+    return (out, out_hi, out_lo) if out_hi is not None else out
 
 
 def append_keys(keys: torch.Tensor, lens: torch.Tensor, new_keys: torch.Tensor, B: int, means: torch.Tensor,
-                workspace: torch.Tensor | None = None, stream=None) -> None:
+                workspace: torch.Tensor | None = None, stream=None, means_hi=None, means_lo=None) -> None:
     """misa_append_keys: new_keys [nseq, n_new, 128] bf16 go to rows
     [lens[b], lens[b] + n_new) of keys [nseq, L_cap, 128]; means [nseq, M_cap,
-    128] fp32 of the touched blocks are recomputed.  lens is not advanced."""
+    128] fp32 (and its bf16 split, if given) of the touched blocks are
+    recomputed.  lens is not advanced."""
     _req(keys, torch.bfloat16, "keys", contiguous=False)
     _req(new_keys, torch.bfloat16, "new_keys")
     _req(lens, torch.int32, "lens")
@@ -172,15 +192,31 @@ def append_keys(keys: torch.Tensor, lens: torch.Tensor, new_keys: torch.Tensor, 
     n_new = new_keys.shape[1]
     if new_keys.shape[0] != nseq or lens.numel() != nseq or means.shape[0] != nseq:
         raise ValueError("keys, lens, new_keys and means must agree on nseq")
+    _split_pair(means_hi, means_lo, means)
     ws = workspace if workspace is not None else alloc_workspace(256, keys.device)
     _call("misa_append_keys", _p(keys), nseq, int(keys.stride(0)) if nseq > 1 else 0, L_cap, _p(lens),
-          _p(new_keys), n_new, B, _p(means), int(means.stride(0)), _p(ws), ws.numel(), _stream(stream))
+          _p(new_keys), n_new, B, _p(means), _p(means_hi), _p(means_lo), int(means.stride(0)), _p(ws), ws.numel(),
+          _stream(stream))
+
+
+def _means_layout(means, means_hi, means_lo):
+    """(nseq, sequence stride) of the block means given as fp32 and/or split."""
+    if means is not None:
+        _req(means, torch.float32, "means")
+    _split_pair(means_hi, means_lo, means)
+    ref = means if means is not None else means_hi
+    if ref is None:
+        raise ValueError("the block means are needed, as fp32 or as the bf16 split")
+    return ref.shape[0], int(ref.stride(0))
 
 
 def route_heads(q, w, means, seq_of, prefix_len, L: int, B: int, q_block: int, h: int,
-                heads=None, importance=None, workspace=None, want_importance: bool = True, stream=None):
-    """misa_route_heads -> (heads [G, h] int32, importance [G, H] fp32 or None)."""
-    _req(q, torch.bfloat16, "q"); _req(w, torch.float32, "w"); _req(means, torch.float32, "means")
+                heads=None, importance=None, workspace=None, want_importance: bool = True, stream=None,
+                means_hi=None, means_lo=None):
+    """misa_route_heads -> (heads [G, h] int32, importance [G, H] fp32 or None).
+    means may be None when the bf16 split (means_hi, means_lo) is given."""
+    _req(q, torch.bfloat16, "q"); _req(w, torch.float32, "w")
+    nseq, mstride = _means_layout(means, means_hi, means_lo)
     _req(seq_of, torch.int32, "seq_of"); _req(prefix_len, torch.int32, "prefix_len")
     T, H, _ = q.shape
     G = (T + q_block - 1) // q_block
@@ -192,7 +228,7 @@ def route_heads(q, w, means, seq_of, prefix_len, L: int, B: int, q_block: int, h
     need = workspace_bytes(OP_ROUTE_HEADS, T, H, L, B)
     if workspace is None:
         workspace = alloc_workspace(need, dev)
-    _call("misa_route_heads", _p(q), _p(w), _p(means), means.shape[0], int(means.stride(0)), _p(seq_of),
+    _call("misa_route_heads", _p(q), _p(w), _p(means), _p(means_hi), _p(means_lo), nseq, mstride, _p(seq_of),
           _p(prefix_len), T, H, L, B, q_block, h, _p(heads), _p(importance), _p(workspace),
           workspace.numel(), _stream(stream))
     return heads, importance
@@ -278,8 +314,11 @@ def hier_rerank(q, w, keys, seq_of, prefix_len, cand, k: int, idx=None, cand_sco
 
 
 def hisa_block_filter(q, w, means, seq_of, prefix_len, L: int, B: int, m: int, blocks=None, cand=None,
-                      block_scores=None, want_scores=False, workspace=None, stream=None):
-    """hisa_block_filter -> (blocks [T, m], cand [T, m*B], block_scores [T, M] or None)."""
+                      block_scores=None, want_scores=False, workspace=None, stream=None, means_hi=None,
+                      means_lo=None):
+    """hisa_block_filter -> (blocks [T, m], cand [T, m*B], block_scores [T, M] or None).
+    means may be None when the bf16 split (means_hi, means_lo) is given."""
+    nseq, mstride = _means_layout(means, means_hi, means_lo)
     T, H, _ = q.shape
     M = (L + B - 1) // B
     dev = q.device
@@ -291,7 +330,7 @@ def hisa_block_filter(q, w, means, seq_of, prefix_len, L: int, B: int, m: int, b
         block_scores = torch.empty((T, M), dtype=torch.float32, device=dev)
     if workspace is None:
         workspace = alloc_workspace(workspace_bytes(OP_HISA_BLOCK_FILTER, T, H, L, B, m), dev)
-    _call("hisa_block_filter", _p(q), _p(w), _p(means), means.shape[0], int(means.stride(0)), _p(seq_of),
+    _call("hisa_block_filter", _p(q), _p(w), _p(means), _p(means_hi), _p(means_lo), nseq, mstride, _p(seq_of),
           _p(prefix_len), T, H, L, B, m, _p(blocks), _p(cand), _p(block_scores), _p(workspace), workspace.numel(),
           _stream(stream))
     return blocks, cand, block_scores

@@ -71,13 +71,20 @@ misa_status check_topk_args(const float* scores, int T, int64_t n, int64_t row_s
   return MISA_OK;
 }
 
-misa_status check_block_args(const uint16_t* q, const float* w, const float* means, int64_t nseq,
-                             int64_t means_seq_stride, const int32_t* seq_of, const int32_t* prefix_len, int T,
-                             int H, int64_t L, int B) {
-  if (!q || !w || !means || !seq_of || !prefix_len) return MISA_ERR_INVALID_ARG;
+// The bf16 split of the block means: both pointers or neither, 16-byte aligned.
+bool split_ok(const uint16_t* hi, const uint16_t* lo) {
+  if (!hi && !lo) return true;
+  return hi && lo && aligned16(hi) && aligned16(lo);
+}
+
+misa_status check_block_args(const uint16_t* q, const float* w, const float* means, const uint16_t* means_hi,
+                             const uint16_t* means_lo, int64_t nseq, int64_t means_seq_stride, const int32_t* seq_of,
+                             const int32_t* prefix_len, int T, int H, int64_t L, int B) {
+  if (!q || !w || !seq_of || !prefix_len || !split_ok(means_hi, means_lo)) return MISA_ERR_INVALID_ARG;
+  if (!means && !means_hi) return MISA_ERR_INVALID_ARG;
   if (T < 1 || H < 1 || L < 1 || B < 1 || nseq < 1) return MISA_ERR_INVALID_ARG;
   if (H > MISA_MAX_HEADS) return MISA_ERR_UNSUPPORTED;
-  if (!aligned16(q) || !aligned16(means) || means_seq_stride < 0 || means_seq_stride % 4 != 0)
+  if (!aligned16(q) || (means && !aligned16(means)) || means_seq_stride < 0 || means_seq_stride % 4 != 0)
     return MISA_ERR_INVALID_ARG;
   const int64_t M = ceil_div(L, B);
   if (nseq > 1 && means_seq_stride < M * MISA_HEAD_DIM) return MISA_ERR_INVALID_ARG;
@@ -144,20 +151,22 @@ misa_status misa_error_query(const void* workspace, misa_stream_t stream, uint32
 }
 
 misa_status misa_block_stats(const uint16_t* keys, int64_t nseq, int64_t L, int64_t key_seq_stride, int B,
-                             float* means, misa_stream_t stream) {
-  if (!keys || !means || nseq < 1 || L < 1 || B < 1) return MISA_ERR_INVALID_ARG;
+                             float* means, uint16_t* means_hi, uint16_t* means_lo, misa_stream_t stream) {
+  if (!keys || !means || nseq < 1 || L < 1 || B < 1 || !split_ok(means_hi, means_lo)) return MISA_ERR_INVALID_ARG;
   if (B > 4096) return MISA_ERR_UNSUPPORTED;
   if (!aligned16(keys) || !aligned16(means) || key_seq_stride < 0 || key_seq_stride % 8 != 0)
     return MISA_ERR_INVALID_ARG;
   if (nseq > 1 && key_seq_stride < L * MISA_HEAD_DIM) return MISA_ERR_INVALID_ARG;
-  return cuda_status(misa::launch_block_stats(keys, nseq, L, key_seq_stride, B, means,
+  return cuda_status(misa::launch_block_stats(keys, nseq, L, key_seq_stride, B, means, means_hi, means_lo,
                                               reinterpret_cast<cudaStream_t>(stream)));
 }
 
 misa_status misa_append_keys(uint16_t* keys, int64_t nseq, int64_t key_seq_stride, int64_t L_cap, const int32_t* len,
-                             const uint16_t* new_keys, int n_new, int B, float* means, int64_t means_seq_stride,
-                             void* workspace, size_t workspace_bytes, misa_stream_t stream) {
-  if (!keys || !len || !new_keys || !means || nseq < 1 || L_cap < 1 || n_new < 1 || B < 1)
+                             const uint16_t* new_keys, int n_new, int B, float* means, uint16_t* means_hi,
+                             uint16_t* means_lo, int64_t means_seq_stride, void* workspace, size_t workspace_bytes,
+                             misa_stream_t stream) {
+  if (!keys || !len || !new_keys || !means || nseq < 1 || L_cap < 1 || n_new < 1 || B < 1 ||
+      !split_ok(means_hi, means_lo))
     return MISA_ERR_INVALID_ARG;
   if (B > 4096) return MISA_ERR_UNSUPPORTED;
   if (!aligned16(keys) || !aligned16(new_keys) || !aligned16(means) || key_seq_stride < 0 || key_seq_stride % 8 != 0)
@@ -169,15 +178,16 @@ misa_status misa_append_keys(uint16_t* keys, int64_t nseq, int64_t key_seq_strid
   misa_status st = check_ws(workspace, workspace_bytes, kErrBytes);
   if (st != MISA_OK) return st;
   return cuda_status(misa::launch_append_keys(keys, nseq, key_seq_stride, L_cap, len, new_keys, n_new, B, means,
-                                              means_seq_stride, err_word(workspace),
+                                              means_hi, means_lo, means_seq_stride, err_word(workspace),
                                               reinterpret_cast<cudaStream_t>(stream)));
 }
 
-misa_status misa_route_heads(const uint16_t* q, const float* w, const float* means, int64_t nseq,
-                             int64_t means_seq_stride, const int32_t* seq_of, const int32_t* prefix_len, int T, int H,
+misa_status misa_route_heads(const uint16_t* q, const float* w, const float* means, const uint16_t* means_hi,
+                             const uint16_t* means_lo, int64_t nseq, int64_t means_seq_stride, const int32_t* seq_of, const int32_t* prefix_len, int T, int H,
                              int64_t L, int B, int q_block, int h, int32_t* heads, float* importance, void* workspace,
                              size_t workspace_bytes, misa_stream_t stream) {
-  misa_status st = check_block_args(q, w, means, nseq, means_seq_stride, seq_of, prefix_len, T, H, L, B);
+  misa_status st =
+      check_block_args(q, w, means, means_hi, means_lo, nseq, means_seq_stride, seq_of, prefix_len, T, H, L, B);
   if (st != MISA_OK) return st;
   if (!heads || q_block < 1 || h < 1 || h > H) return MISA_ERR_INVALID_ARG;
   if (means_seq_stride % MISA_HEAD_DIM != 0) return MISA_ERR_INVALID_ARG;  // rows of 128 means for the TMA map
@@ -187,7 +197,8 @@ misa_status misa_route_heads(const uint16_t* q, const float* w, const float* mea
   float* partial = reinterpret_cast<float*>(scratch);
   unsigned* counters = reinterpret_cast<unsigned*>(scratch + misa::router_counters_offset(T, H, L, B));
   const int qpm = misa::route_tc_queries_per_group(H, q_block, nseq == 1 || means_seq_stride == 0);
-  return cuda_status(misa::launch_route_heads_tc(q, w, means, means_seq_stride, static_cast<int>(nseq), seq_of,
+  return cuda_status(misa::launch_route_heads_tc(q, w, means, means_hi, means_lo, means_seq_stride,
+                                                 static_cast<int>(nseq), seq_of,
                                                  prefix_len, T, H, L, B, q_block, h, qpm, heads, importance, partial,
                                                  counters, false, err_word(workspace),
                                                  reinterpret_cast<cudaStream_t>(stream)));
@@ -290,11 +301,12 @@ misa_status misa_hier_rerank(const uint16_t* q, const float* w, const uint16_t* 
   return MISA_OK;
 }
 
-misa_status hisa_block_filter(const uint16_t* q, const float* w, const float* means, int64_t nseq,
-                              int64_t means_seq_stride, const int32_t* seq_of, const int32_t* prefix_len, int T, int H,
+misa_status hisa_block_filter(const uint16_t* q, const float* w, const float* means, const uint16_t* means_hi,
+                              const uint16_t* means_lo, int64_t nseq, int64_t means_seq_stride, const int32_t* seq_of, const int32_t* prefix_len, int T, int H,
                               int64_t L, int B, int m, int32_t* blocks, int32_t* cand, float* block_scores,
                               void* workspace, size_t workspace_bytes, misa_stream_t stream) {
-  misa_status st = check_block_args(q, w, means, nseq, means_seq_stride, seq_of, prefix_len, T, H, L, B);
+  misa_status st =
+      check_block_args(q, w, means, means_hi, means_lo, nseq, means_seq_stride, seq_of, prefix_len, T, H, L, B);
   if (st != MISA_OK) return st;
   if (!blocks || !cand || m < 1) return MISA_ERR_INVALID_ARG;
   if (means_seq_stride % MISA_HEAD_DIM != 0) return MISA_ERR_INVALID_ARG;  // rows of 128 means for the TMA map
@@ -306,7 +318,8 @@ misa_status hisa_block_filter(const uint16_t* q, const float* w, const float* me
   const int64_t M = ceil_div(L, B);
   const int64_t M_pad = round_up4(M);
   float* bs = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kErrBytes);
-  cudaError_t e = misa::launch_hisa_block_scores_tc(q, w, means, means_seq_stride, static_cast<int>(nseq), seq_of,
+  cudaError_t e = misa::launch_hisa_block_scores_tc(q, w, means, means_hi, means_lo, means_seq_stride,
+                                                    static_cast<int>(nseq), seq_of,
                                                     prefix_len, T, H, L, B, bs, M_pad, err_word(workspace), s);
   if (e != cudaSuccess) return MISA_ERR_CUDA;
   e = misa::launch_topk(bs, T, M, M_pad, nullptr, nullptr, 0, m, blocks, s);

@@ -36,10 +36,13 @@ __device__ __forceinline__ void acc_bf16x8(float (&acc)[8], const uint4 v) {
   }
 }
 
-// Mean of rows [s0, s1) of one block into out[0..128); chunk_at(s) is the
-// lane's 16-byte chunk of row s.  Every lane of the warp calls.
+// Mean of rows [s0, s1) of one block into out[0..128) and, when hi is not
+// NULL, its split into two bf16 rows: hi = bf16(mean), lo = bf16(mean - hi)
+// (the tensor-core router's operands); chunk_at(s) is the lane's 16-byte chunk
+// of row s.  Every lane of the warp calls.
 template <class ChunkAt>
-__device__ __forceinline__ void block_mean_warp(int64_t s0, int64_t s1, ChunkAt chunk_at, float* out) {
+__device__ __forceinline__ void block_mean_warp(int64_t s0, int64_t s1, ChunkAt chunk_at, float* out, uint16_t* hi,
+                                                uint16_t* lo) {
   const int lane = threadIdx.x & 31;
   const int half = lane >> 4;   // which row of the pair
   const int chunk = lane & 15;  // 16-byte chunk of the row (8 bf16)
@@ -59,15 +62,33 @@ __device__ __forceinline__ void block_mean_warp(int64_t s0, int64_t s1, ChunkAt 
   for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], 16);
   if (half == 0) {
     const float inv = 1.0f / static_cast<float>(s1 - s0);
+    float m[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = acc[i] * inv;
     float4* o = reinterpret_cast<float4*>(out + chunk * 8);
-    o[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
-    o[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
+    o[0] = make_float4(m[0], m[1], m[2], m[3]);
+    o[1] = make_float4(m[4], m[5], m[6], m[7]);
+    if (hi) {
+      uint32_t hw[4], lw[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const __nv_bfloat16 h0 = __float2bfloat16_rn(m[2 * c]);
+        const __nv_bfloat16 h1 = __float2bfloat16_rn(m[2 * c + 1]);
+        const __nv_bfloat16 l0 = __float2bfloat16_rn(m[2 * c] - __bfloat162float(h0));
+        const __nv_bfloat16 l1 = __float2bfloat16_rn(m[2 * c + 1] - __bfloat162float(h1));
+        hw[c] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
+        lw[c] = static_cast<uint32_t>(__bfloat16_as_ushort(l0)) | (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
+      }
+      *reinterpret_cast<uint4*>(hi + chunk * 8) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      *reinterpret_cast<uint4*>(lo + chunk * 8) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    }
   }
 }
 
 __global__ void __launch_bounds__(kWarpsPerCta * 32)
 block_stats_kernel(const uint16_t* __restrict__ keys, int64_t nseq, int64_t L, int64_t key_seq_stride, int B,
-                   int64_t M, float* __restrict__ means) {
+                   int64_t M, float* __restrict__ means, uint16_t* __restrict__ means_hi,
+                   uint16_t* __restrict__ means_lo) {
   const int lane = threadIdx.x & 31;
   const int64_t gw = static_cast<int64_t>(blockIdx.x) * kWarpsPerCta + (threadIdx.x >> 5);
   if (gw >= nseq * M) return;
@@ -76,8 +97,9 @@ block_stats_kernel(const uint16_t* __restrict__ keys, int64_t nseq, int64_t L, i
   const int64_t s0 = j * B;
   const int64_t s1 = (s0 + B < L) ? s0 + B : L;
   const uint16_t* base = keys + b * key_seq_stride + static_cast<int64_t>(lane & 15) * 8;
+  const int64_t row = (b * M + j) * kD;
   block_mean_warp(s0, s1, [&](int64_t s) { return __ldg(reinterpret_cast<const uint4*>(base + s * kD)); },
-                  means + (b * M + j) * kD);
+                  means + row, means_hi ? means_hi + row : nullptr, means_lo ? means_lo + row : nullptr);
 }
 
 // One warp per (sequence, touched block): copies the new rows of its block
@@ -87,8 +109,8 @@ block_stats_kernel(const uint16_t* __restrict__ keys, int64_t nseq, int64_t L, i
 __global__ void __launch_bounds__(kWarpsPerCta * 32)
 append_keys_kernel(uint16_t* __restrict__ keys, int64_t nseq, int64_t key_seq_stride, int64_t L_cap,
                    const int32_t* __restrict__ len, const uint16_t* __restrict__ new_keys, int n_new, int B,
-                   int64_t blocks_per_seq, float* __restrict__ means, int64_t means_seq_stride,
-                   uint32_t* __restrict__ err) {
+                   int64_t blocks_per_seq, float* __restrict__ means, uint16_t* __restrict__ means_hi,
+                   uint16_t* __restrict__ means_lo, int64_t means_seq_stride, uint32_t* __restrict__ err) {
   const int lane = threadIdx.x & 31;
   const int64_t gw = static_cast<int64_t>(blockIdx.x) * kWarpsPerCta + (threadIdx.x >> 5);
   if (gw >= nseq * blocks_per_seq) return;
@@ -117,32 +139,35 @@ append_keys_kernel(uint16_t* __restrict__ keys, int64_t nseq, int64_t key_seq_st
         return s < l0 ? __ldg(reinterpret_cast<const uint4*>(cache + s * kD + cofs))
                       : __ldg(reinterpret_cast<const uint4*>(fresh + (s - l0) * kD + cofs));
       },
-      means + b * means_seq_stride + j * kD);
+      means + b * means_seq_stride + j * kD, means_hi ? means_hi + b * means_seq_stride + j * kD : nullptr,
+      means_lo ? means_lo + b * means_seq_stride + j * kD : nullptr);
 }
 
 }  // namespace
 
 cudaError_t launch_block_stats(const uint16_t* keys, int64_t nseq, int64_t L, int64_t key_seq_stride, int B,
-                               float* means, cudaStream_t stream) {
+                               float* means, uint16_t* means_hi, uint16_t* means_lo, cudaStream_t stream) {
   const int64_t M = (L + B - 1) / B;
   const int64_t warps = nseq * M;
   const int64_t ctas = (warps + kWarpsPerCta - 1) / kWarpsPerCta;
   if (ctas > 0x7fffffff) return cudaErrorInvalidValue;
   block_stats_kernel<<<static_cast<unsigned>(ctas), kWarpsPerCta * 32, 0, stream>>>(keys, nseq, L, key_seq_stride,
-                                                                                   B, M, means);
+                                                                                   B, M, means, means_hi, means_lo);
   return cudaGetLastError();
 }
 
 cudaError_t launch_append_keys(uint16_t* keys, int64_t nseq, int64_t key_seq_stride, int64_t L_cap,
                                const int32_t* len, const uint16_t* new_keys, int n_new, int B, float* means,
-                               int64_t means_seq_stride, uint32_t* err, cudaStream_t stream) {
+                               uint16_t* means_hi, uint16_t* means_lo, int64_t means_seq_stride, uint32_t* err,
+                               cudaStream_t stream) {
   // [l0, l0 + n_new) touches at most ceil(n_new / B) + 1 blocks
   const int64_t blocks_per_seq = (n_new + B - 1) / B + 1;
   const int64_t warps = nseq * blocks_per_seq;
   const int64_t ctas = (warps + kWarpsPerCta - 1) / kWarpsPerCta;
   if (ctas > 0x7fffffff) return cudaErrorInvalidValue;
   append_keys_kernel<<<static_cast<unsigned>(ctas), kWarpsPerCta * 32, 0, stream>>>(
-      keys, nseq, key_seq_stride, L_cap, len, new_keys, n_new, B, blocks_per_seq, means, means_seq_stride, err);
+      keys, nseq, key_seq_stride, L_cap, len, new_keys, n_new, B, blocks_per_seq, means, means_hi, means_lo,
+      means_seq_stride, err);
   return cudaGetLastError();
 }
 

@@ -55,17 +55,19 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 }
 
 cudaError_t launch_block_stats(const uint16_t* keys, int64_t nseq, int64_t L, int64_t key_seq_stride, int B,
-                               float* means, cudaStream_t stream);
+                               float* means, uint16_t* means_hi, uint16_t* means_lo, cudaStream_t stream);
 cudaError_t launch_append_keys(uint16_t* keys, int64_t nseq, int64_t key_seq_stride, int64_t L_cap,
                                const int32_t* len, const uint16_t* new_keys, int n_new, int B, float* means,
-                               int64_t means_seq_stride, uint32_t* err, cudaStream_t stream);
+                               uint16_t* means_hi, uint16_t* means_lo, int64_t means_seq_stride, uint32_t* err,
+                               cudaStream_t stream);
 
 int router_chunks(int M);
 
 // Tensor-core router (route_tc.cu).  qpm = queries per MMA row group (>1 only
 // when the queries share one sequence's block means).
 int route_tc_queries_per_group(int H, int q_block, bool shared_sequence);
-cudaError_t launch_route_heads_tc(const uint16_t* q, const float* w, const float* means, int64_t means_seq_stride,
+cudaError_t launch_route_heads_tc(const uint16_t* q, const float* w, const float* means, const uint16_t* means_hi,
+                                  const uint16_t* means_lo, int64_t means_seq_stride,
                                   int nseq, const int32_t* seq_of, const int32_t* prefix_len, int T, int H, int64_t L,
                                   int B, int q_block, int h, int qpm, int32_t* heads, float* importance,
                                   float* partial, unsigned* counters, bool clear_counters, uint32_t* err,
@@ -77,8 +79,9 @@ size_t router_scratch_bytes(int T, int H, int64_t L, int B, int q_block);
 size_t router_counters_offset(int T, int H, int64_t L, int B);
 
 cudaError_t launch_hisa_block_scores_tc(const uint16_t* q, const float* w, const float* means,
-                                        int64_t means_seq_stride, int nseq, const int32_t* seq_of,
-                                        const int32_t* prefix_len, int T, int H, int64_t L, int B, float* bscore,
+                                        const uint16_t* means_hi, const uint16_t* means_lo, int64_t means_seq_stride,
+                                        int nseq, const int32_t* seq_of, const int32_t* prefix_len, int T, int H,
+                                        int64_t L, int B, float* bscore,
                                         int64_t bs_stride, uint32_t* err, cudaStream_t stream);
 
 cudaError_t launch_hisa_expand(const int32_t* blocks, const int32_t* prefix_len, int T, int m, int B, int64_t L,

@@ -13,7 +13,9 @@
 // tile, K = 128.  The fp32 block means of a tile arrive by one TMA copy; the
 // producers split them into bf16 hi = bf16(m) and lo = bf16(m - hi) (together
 // about 16 significant bits) and D = q . hi + q . lo accumulates in fp32 in
-// TMEM.  The epilogue thread of row (t, h) sums ReLU(D) over the tile's
+// TMEM.  When the caller already holds the split (written with the block
+// means) the two bf16 tiles arrive by TMA in the MMA's swizzled layout and no
+// conversion runs.  The epilogue thread of row (t, h) sums ReLU(D) over the tile's
 // visible blocks and multiplies by w[t][h] (no cross-thread reduction); the
 // rows of one head are added in shared memory.  Two ways to combine the work
 // items (row group, block tile) of one decision:
@@ -30,7 +32,8 @@
 //
 // Roles (416 threads): warps 0-3 epilogue (TMEM lane quarter = warp), warp 4
 // TMEM allocation + MMA issue, warp 5 lane 0 TMA of the query rows (once per
-// row group) and of the fp32 mean tiles, warps 6-12 the hi/lo conversion.
+// row group) and of the mean tiles, warps 6-12 the hi/lo conversion (idle
+// when the split comes from memory).
 // Waits are bounded and share a CTA-wide abort flag.
 #include <cooperative_groups.h>
 
@@ -75,6 +78,7 @@ struct RouteParams {
   const uint16_t* q;
   const float* w;
   int64_t means_seq_rows;    // rows of 128 means between sequences in the TMA map
+  bool presplit;             // mean tiles given as bf16 hi / lo (else fp32, split here)
   int nseq;
   const int32_t* seq_of;
   const int32_t* prefix_len;
@@ -145,14 +149,15 @@ __device__ void select_top_h(const float* imp, int H, int h, int g, int32_t* hea
 // reduction across work items).
 template <bool kCluster, bool kHisa>
 __global__ void __launch_bounds__(kRThreads, 1)
-route_tc_kernel(const __grid_constant__ CUtensorMap means_map, const __grid_constant__ CUtensorMap q_map,
+route_tc_kernel(const __grid_constant__ CUtensorMap means_map, const __grid_constant__ CUtensorMap hi_map,
+                const __grid_constant__ CUtensorMap lo_map, const __grid_constant__ CUtensorMap q_map,
                 const RouteParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem + kROffA;
   uint8_t* sS = smem + kROffS;  // stage s: [fp32 means | hi | lo]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kROffBar);
-  uint64_t* ffull = bars;                    // [S] fp32 tile landed (TMA)
+  uint64_t* ffull = bars;                    // [S] mean tile(s) landed (TMA)
   uint64_t* bfull = bars + kRStages;         // [S] hi/lo tile written
   uint64_t* empty = bars + 2 * kRStages;     // [S] MMAs of the stage done
   uint64_t* tfull = bars + 3 * kRStages;     // [2]
@@ -190,7 +195,12 @@ route_tc_kernel(const __grid_constant__ CUtensorMap means_map, const __grid_cons
     tmem_relinquish();
   }
   if (tid == kRTmaWarp * 32) {
-    tma_prefetch_desc(&means_map);
+    if (p.presplit) {
+      tma_prefetch_desc(&hi_map);
+      tma_prefetch_desc(&lo_map);
+    } else {
+      tma_prefetch_desc(&means_map);
+    }
     tma_prefetch_desc(&q_map);
   }
   tc_fence_before();
@@ -222,7 +232,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap means_map, const __grid_cons
   }
 
   if (warp == kRTmaWarp) {
-    // ------------------------------------------------------------ query rows and fp32 mean tiles by TMA
+    // ------------------------------------------------------------ query rows and mean tiles by TMA
     if (lane == 0) {
       int64_t it = 0;
       int cur_pg = -1, ng = 0;
@@ -245,9 +255,19 @@ route_tc_kernel(const __grid_constant__ CUtensorMap means_map, const __grid_cons
         const int s = static_cast<int>(it % kRStages);
         const uint32_t ph = static_cast<uint32_t>((it / kRStages) & 1);
         if (!mbar_wait(&empty[s], ph ^ 1u, p.err, abort)) break;
-        mbar_arrive_expect_tx(&ffull[s], kRFTileBytes);
         const int y = static_cast<int>(group_seq(p, pg) * p.means_seq_rows + static_cast<int64_t>(bt) * kRN);
-        tma_load_2d(sS + s * kRStageBytes, &means_map, &ffull[s], 0, y);
+        if (p.presplit) {
+          // hi and lo straight into the MMA operand slots, two 64-column halves each
+          uint8_t* hi_t = sS + s * kRStageBytes + kRFTileBytes;
+          mbar_arrive_expect_tx(&ffull[s], 2 * kRBTileBytes);
+          tma_load_2d(hi_t, &hi_map, &ffull[s], 0, y);
+          tma_load_2d(hi_t + kRN * 128, &hi_map, &ffull[s], 64, y);
+          tma_load_2d(hi_t + kRBTileBytes, &lo_map, &ffull[s], 0, y);
+          tma_load_2d(hi_t + kRBTileBytes + kRN * 128, &lo_map, &ffull[s], 64, y);
+        } else {
+          mbar_arrive_expect_tx(&ffull[s], kRFTileBytes);
+          tma_load_2d(sS + s * kRStageBytes, &means_map, &ffull[s], 0, y);
+        }
       }
       // no TMA write may still be in flight when the CTA exits
       const int64_t first = it > kRStages ? it - kRStages : 0;
@@ -259,7 +279,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap means_map, const __grid_cons
     // ------------------------------------------------------------ hi/lo conversion
     const int ct = tid - (kRTmaWarp + 1) * 32;
     int64_t it = 0;
-    for (int64_t item = i0; item < i1; ++item, ++it) {
+    for (int64_t item = i0; !p.presplit && item < i1; ++item, ++it) {
       const int s = static_cast<int>(it % kRStages);
       const uint32_t ph = static_cast<uint32_t>((it / kRStages) & 1);
       if (!mbar_wait(&ffull[s], ph, p.err, abort)) break;
@@ -294,6 +314,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap means_map, const __grid_cons
       int64_t it = 0;
       int cur_pg = -1, ng = 0;
       const uint32_t a_addr = smem_u32(sA);
+      uint64_t* bready = p.presplit ? ffull : bfull;  // hi/lo tiles of a stage in place
       for (int64_t item = i0; item < i1; ++item, ++it) {
         const int pg = static_cast<int>(item / nbt);
         if (pg != cur_pg) {
@@ -306,7 +327,7 @@ route_tc_kernel(const __grid_constant__ CUtensorMap means_map, const __grid_cons
         if (!mbar_wait(&tempty[a], aph ^ 1u, p.err, abort)) break;
         const int s = static_cast<int>(it % kRStages);
         const uint32_t ph = static_cast<uint32_t>((it / kRStages) & 1);
-        if (!mbar_wait(&bfull[s], ph, p.err, abort)) break;
+        if (!mbar_wait(&bready[s], ph, p.err, abort)) break;
         tc_fence_after();
         const uint32_t hi_addr = smem_u32(sS + s * kRStageBytes + kRFTileBytes);
         const uint32_t lo_addr = hi_addr + kRBTileBytes;
@@ -501,7 +522,26 @@ int route_tc_queries_per_group(int H, int q_block, bool shared_sequence) {
   return qpm;
 }
 
-cudaError_t launch_route_heads_tc(const uint16_t* q, const float* w, const float* means, int64_t means_seq_stride,
+namespace {
+
+// Tensor maps of the block means: fp32 rows of 128 (one TMA box per tile),
+// or, when the split is given, the bf16 hi and lo rows in 128-byte swizzled
+// halves (the MMA's B layout).  The maps a launch does not use stay zero.
+bool encode_mean_maps(const float* means, const uint16_t* hi, const uint16_t* lo, uint64_t rows, CUtensorMap* fmap,
+                      CUtensorMap* hmap, CUtensorMap* lmap) {
+  *fmap = CUtensorMap{};
+  *hmap = CUtensorMap{};
+  *lmap = CUtensorMap{};
+  if (hi && lo)
+    return encode_2d_map(hmap, true, hi, kD, rows, kD * 2, 64, kRN, true) &&
+           encode_2d_map(lmap, true, lo, kD, rows, kD * 2, 64, kRN, true);
+  return encode_2d_map(fmap, false, means, kD, rows, kD * 4, kD, kRN, false);
+}
+
+}  // namespace
+
+cudaError_t launch_route_heads_tc(const uint16_t* q, const float* w, const float* means, const uint16_t* means_hi,
+                                  const uint16_t* means_lo, int64_t means_seq_stride,
                                   int nseq, const int32_t* seq_of, const int32_t* prefix_len, int T, int H, int64_t L,
                                   int B, int q_block, int h, int qpm, int32_t* heads, float* importance,
                                   float* partial, unsigned* counters, bool clear_counters, uint32_t* err,
@@ -529,10 +569,11 @@ cudaError_t launch_route_heads_tc(const uint16_t* q, const float* w, const float
   p.heads = heads;
   p.importance = importance;
   p.err = err;
-  // fp32 means as rows of 128: sequence b's block j is row b * means_seq_rows + j
-  CUtensorMap map;
+  p.presplit = means_hi && means_lo;
+  // means as rows of 128: sequence b's block j is row b * means_seq_rows + j
+  CUtensorMap map, hmap, lmap;
   const uint64_t rows = static_cast<uint64_t>(nseq - 1) * static_cast<uint64_t>(p.means_seq_rows) + p.M;
-  if (!encode_2d_map(&map, false, means, kD, rows, kD * 4, kD, kRN, false)) return cudaErrorInvalidValue;
+  if (!encode_mean_maps(means, means_hi, means_lo, rows, &map, &hmap, &lmap)) return cudaErrorInvalidValue;
   // query rows, bf16, 128-byte swizzled K-major like the keys
   CUtensorMap qmap;
   if (!encode_2d_map(&qmap, true, q, kD, static_cast<uint64_t>(T) * H, kD * 2, 64, kRM, true))
@@ -550,7 +591,7 @@ cudaError_t launch_route_heads_tc(const uint16_t* q, const float* w, const float
     e = ensure_dynamic_smem(reinterpret_cast<const void*>(route_tc_kernel<true, false>), kRSmemBytes);
     if (e != cudaSuccess) return e;
     return launch_pdl(route_tc_kernel<true, false>, dim3(static_cast<unsigned>(G * D)), dim3(kRThreads), kRSmemBytes, stream,
-                      D, map, qmap, p);
+                      D, map, hmap, lmap, qmap, p);
   }
   if (clear_counters) {
     e = cudaMemsetAsync(counters, 0, static_cast<size_t>(G) * sizeof(unsigned), stream);
@@ -560,11 +601,11 @@ cudaError_t launch_route_heads_tc(const uint16_t* q, const float* w, const float
   if (e != cudaSuccess) return e;
   const int64_t grid = p.n_items < sms ? p.n_items : sms;
   return launch_pdl(route_tc_kernel<false, false>, dim3(static_cast<unsigned>(grid)), dim3(kRThreads), kRSmemBytes, stream, 0,
-                    map, qmap, p);
+                    map, hmap, lmap, qmap, p);
 }
 
 cudaError_t launch_hisa_block_scores_tc(const uint16_t* q, const float* w, const float* means,
-                                        int64_t means_seq_stride, int nseq, const int32_t* seq_of,
+                                        const uint16_t* means_hi, const uint16_t* means_lo, int64_t means_seq_stride, int nseq, const int32_t* seq_of,
                                         const int32_t* prefix_len, int T, int H, int64_t L, int B, float* bscore,
                                         int64_t bs_stride, uint32_t* err, cudaStream_t stream) {
   if (H > kRM) return cudaErrorInvalidValue;
@@ -592,9 +633,10 @@ cudaError_t launch_hisa_block_scores_tc(const uint16_t* q, const float* w, const
   p.bscore = bscore;
   p.bs_stride = bs_stride;
   p.err = err;
-  CUtensorMap map;
+  p.presplit = means_hi && means_lo;
+  CUtensorMap map, hmap, lmap;
   const uint64_t rows = static_cast<uint64_t>(nseq - 1) * static_cast<uint64_t>(p.means_seq_rows) + p.M;
-  if (!encode_2d_map(&map, false, means, kD, rows, kD * 4, kD, kRN, false)) return cudaErrorInvalidValue;
+  if (!encode_mean_maps(means, means_hi, means_lo, rows, &map, &hmap, &lmap)) return cudaErrorInvalidValue;
   CUtensorMap qmap;
   if (!encode_2d_map(&qmap, true, q, kD, static_cast<uint64_t>(T) * H, kD * 2, 64, kRM, true))
     return cudaErrorInvalidValue;
@@ -604,7 +646,7 @@ cudaError_t launch_hisa_block_scores_tc(const uint16_t* q, const float* w, const
   if (sms <= 0) return cudaErrorInvalidDevice;
   const int64_t grid = p.n_items < sms ? p.n_items : sms;
   return launch_pdl(route_tc_kernel<false, true>, dim3(static_cast<unsigned>(grid)), dim3(kRThreads), kRSmemBytes,
-                    stream, 0, map, qmap, p);
+                    stream, 0, map, hmap, lmap, qmap, p);
 }
 
 }  // namespace misa

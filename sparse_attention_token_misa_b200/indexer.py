@@ -3,7 +3,9 @@
 Each class owns its device buffers (outputs and workspaces) for one batch shape
 and issues the C-ABI calls on the current CUDA stream in `run`, so a step
 allocates nothing and can be captured in a CUDA graph.  All arithmetic runs in
-the library's kernels.
+the library's kernels.  `means` is what `block_stats` returns: the fp32 block
+means, or the tuple (means, means_hi, means_lo) with their bf16 split, which
+the router and the block filter then read directly.
 
 * MisaIndexer   -- router (h of H heads per query block), routed token scoring,
                    top-k.  MISA page (gist.science), "Methodology: MISA".
@@ -22,6 +24,13 @@ from . import _native as nat
 
 def _pad4(n: int) -> int:
     return (n + 3) // 4 * 4
+
+
+def _means_args(means) -> dict:
+    if isinstance(means, tuple):
+        m, hi, lo = means
+        return dict(means=m, means_hi=hi, means_lo=lo)
+    return dict(means=means)
 
 
 def capture_graph(fn) -> torch.cuda.CUDAGraph:
@@ -60,8 +69,9 @@ class MisaIndexer:
         self.ws = nat.alloc_workspace(256, device)
 
     def route(self, q, w, means, seq_of, prefix_len, stream=None):
-        nat.route_heads(q, w, means, seq_of, prefix_len, self.L, self.B, self.q_block, self.h,
-                        heads=self.heads, importance=self.importance, workspace=self.ws_route, stream=stream)
+        nat.route_heads(q, w, seq_of=seq_of, prefix_len=prefix_len, L=self.L, B=self.B, q_block=self.q_block,
+                        h=self.h, heads=self.heads, importance=self.importance, workspace=self.ws_route,
+                        stream=stream, **_means_args(means))
 
     def score(self, q, w, keys, seq_of, prefix_len, stream=None):
         nat.index_score(q, w, keys, seq_of, prefix_len, heads=self.heads, h=self.h, q_block=self.q_block,
@@ -145,8 +155,9 @@ class HisaIndexer:
         self.ws = nat.alloc_workspace(256, device)
 
     def run(self, q, w, keys, means, seq_of, prefix_len, stream=None) -> torch.Tensor:
-        nat.hisa_block_filter(q, w, means, seq_of, prefix_len, self.L, self.B, self.m, blocks=self.blocks,
-                              cand=self.cand, workspace=self.ws_filter, stream=stream)
+        nat.hisa_block_filter(q, w, seq_of=seq_of, prefix_len=prefix_len, L=self.L, B=self.B, m=self.m,
+                              blocks=self.blocks, cand=self.cand, workspace=self.ws_filter, stream=stream,
+                              **_means_args(means))
         nat.index_score(q, w, keys, seq_of, prefix_len, cand=self.cand, scores=self.scores_buf, workspace=self.ws,
                         stream=stream)
         nat.topk(self.scores_buf, self.k, n=self.m * self.B, id_map=self.cand, idx=self.idx, workspace=self.ws,

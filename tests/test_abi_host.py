@@ -119,10 +119,10 @@ def test_index_score_rejects(kw, status):
     assert score(**kw) == status
 
 
-def route(q=P, w=P, means=P, nseq=1, mstride=0, seq_of=P, plen=P, T=4, H=64, L=1024, B=128, q_block=1, h=8,
-          heads=P2, imp=None, ws=P2, ws_bytes=1 << 20):
-    return pkg.lib().misa_route_heads(q, w, means, nseq, mstride, seq_of, plen, T, H, L, B, q_block, h, heads, imp, ws,
-                                      ws_bytes, None)
+def route(q=P, w=P, means=P, hi=None, lo=None, nseq=1, mstride=0, seq_of=P, plen=P, T=4, H=64, L=1024, B=128,
+          q_block=1, h=8, heads=P2, imp=None, ws=P2, ws_bytes=1 << 20):
+    return pkg.lib().misa_route_heads(q, w, means, hi, lo, nseq, mstride, seq_of, plen, T, H, L, B, q_block, h, heads,
+                                      imp, ws, ws_bytes, None)
 
 
 @pytest.mark.parametrize("kw,status", [
@@ -138,6 +138,10 @@ def route(q=P, w=P, means=P, nseq=1, mstride=0, seq_of=P, plen=P, T=4, H=64, L=1
     (dict(heads=None), INVALID),
     (dict(ws_bytes=256), WORKSPACE),
     (dict(ws=None), WORKSPACE),
+    (dict(means=None), INVALID),                     # neither fp32 means nor the split
+    (dict(hi=P), INVALID),                           # hi without lo
+    (dict(lo=P), INVALID),
+    (dict(means=None, hi=P, lo=MIS), INVALID),       # misaligned split
 ])
 def test_route_rejects(kw, status):
     assert route(**kw) == status
@@ -145,14 +149,18 @@ def test_route_rejects(kw, status):
 
 def test_block_stats_rejects():
     f = pkg.lib().misa_block_stats
-    assert f(P, 1, 100, 0, 0, P2, None) == INVALID
-    assert f(P, 1, 100, 0, 5000, P2, None) == UNSUPPORTED
-    assert f(MIS, 1, 100, 0, 4, P2, None) == INVALID
-    assert f(P, 1, 100, 0, 4, MIS, None) == INVALID
-    assert f(P, 2, 100, 4, 4, P2, None) == INVALID        # stride % 8
-    assert f(P, 2, 100, 128, 4, P2, None) == INVALID      # overlapping sequences
-    assert f(None, 1, 100, 0, 4, P2, None) == INVALID
-    assert f(P, 0, 100, 0, 4, P2, None) == INVALID
+    assert f(P, 1, 100, 0, 0, P2, None, None, None) == INVALID
+    assert f(P, 1, 100, 0, 5000, P2, None, None, None) == UNSUPPORTED
+    assert f(MIS, 1, 100, 0, 4, P2, None, None, None) == INVALID
+    assert f(P, 1, 100, 0, 4, MIS, None, None, None) == INVALID
+    assert f(P, 2, 100, 4, 4, P2, None, None, None) == INVALID        # stride % 8
+    assert f(P, 2, 100, 128, 4, P2, None, None, None) == INVALID      # overlapping sequences
+    assert f(None, 1, 100, 0, 4, P2, None, None, None) == INVALID
+    assert f(P, 0, 100, 0, 4, P2, None, None, None) == INVALID
+    # the bf16 split: both outputs or neither, 16-byte aligned
+    assert f(P, 1, 100, 0, 4, P2, P, None, None) == INVALID
+    assert f(P, 1, 100, 0, 4, P2, None, P, None) == INVALID
+    assert f(P, 1, 100, 0, 4, P2, P, MIS, None) == INVALID
 
 
 def test_hier_rerank_and_hisa_reject():
@@ -163,12 +171,16 @@ def test_hier_rerank_and_hisa_reject():
     assert r(P, P, P, 1, 0, P, P, 2, 32, 100, None, 4, 2, None, P2, P2, 1 << 20, None) == INVALID
     assert r(P, P, P, 1, 0, P, P, 2, 32, 100, P, 4, 2, None, P2, P2, 64, None) == WORKSPACE
     hf = l.hisa_block_filter
-    assert hf(P, P, P, 1, 0, P, P, 2, 64, 1000, 128, 0, P2, P2, None, P2, 1 << 20, None) == INVALID
-    assert hf(P, P, P, 1, 0, P, P, 2, 64, 1000, 128, 20000, P2, P2, None, P2, 1 << 20, None) == UNSUPPORTED
-    assert hf(P, P, P, 1, 0, P, P, 2, 64, 1000, 128, 4, None, P2, None, P2, 1 << 20, None) == INVALID
-    assert hf(P, P, P, 1, 0, P, P, 2, 64, 1000, 128, 4, P2, P2, None, P2, 256, None) == WORKSPACE
+    N = None
+    assert hf(P, P, P, N, N, 1, 0, P, P, 2, 64, 1000, 128, 0, P2, P2, N, P2, 1 << 20, N) == INVALID
+    assert hf(P, P, P, N, N, 1, 0, P, P, 2, 64, 1000, 128, 20000, P2, P2, N, P2, 1 << 20, N) == UNSUPPORTED
+    assert hf(P, P, P, N, N, 1, 0, P, P, 2, 64, 1000, 128, 4, N, P2, N, P2, 1 << 20, N) == INVALID
+    assert hf(P, P, P, N, N, 1, 0, P, P, 2, 64, 1000, 128, 4, P2, P2, N, P2, 256, N) == WORKSPACE
     # sequence stride of the means: whole 128-float rows (TMA rows)
-    assert hf(P, P, P, 2, 8 * 128 + 4, P, P, 2, 64, 1000, 128, 4, P2, P2, None, P2, 1 << 20, None) == INVALID
+    assert hf(P, P, P, N, N, 2, 8 * 128 + 4, P, P, 2, 64, 1000, 128, 4, P2, P2, N, P2, 1 << 20, N) == INVALID
+    # the bf16 split: both or neither; with it the fp32 means may be absent
+    assert hf(P, P, N, P, N, 1, 0, P, P, 2, 64, 1000, 128, 4, P2, P2, N, P2, 1 << 20, N) == INVALID
+    assert hf(P, P, N, N, N, 1, 0, P, P, 2, 64, 1000, 128, 4, P2, P2, N, P2, 1 << 20, N) == INVALID
 
 
 def test_error_query_rejects_null():
@@ -178,8 +190,8 @@ def test_error_query_rejects_null():
 
 
 def append(keys=P, nseq=2, key_seq_stride=1024 * 128, L_cap=1024, lens=P2, new_keys=P2 + 4096, n_new=1, B=128,
-           means=P2 + 8192, means_seq_stride=8 * 128, ws=P2 + 16384, ws_bytes=256):
-    return pkg.lib().misa_append_keys(keys, nseq, key_seq_stride, L_cap, lens, new_keys, n_new, B, means,
+           means=P2 + 8192, hi=None, lo=None, means_seq_stride=8 * 128, ws=P2 + 16384, ws_bytes=256):
+    return pkg.lib().misa_append_keys(keys, nseq, key_seq_stride, L_cap, lens, new_keys, n_new, B, means, hi, lo,
                                       means_seq_stride, ws, ws_bytes, None)
 
 
@@ -197,3 +209,5 @@ def test_append_keys_validation():
     assert append(means_seq_stride=8 * 128 + 4) == INVALID   # not whole 128-float rows
     assert append(ws=None) == WORKSPACE
     assert append(ws_bytes=255) == WORKSPACE
+    assert append(hi=P) == INVALID                           # split: both or neither
+    assert append(hi=P, lo=MIS) == INVALID
