@@ -393,6 +393,8 @@ def other_workloads(misa, dev, stream, flush, steps, only=None):
         out.update(_dagger_prefill(misa, dev, stream, flush, steps, timed))
     if only in (None, "hisa"):
         out.update(_hisa(misa, dev, stream, flush, steps, timed))
+    if only in (None, "attn"):
+        out.update(_sparse_attention(misa, dev, stream, flush, steps, timed))
     return out
 
 
@@ -486,6 +488,60 @@ def _hisa(misa, dev, stream, flush, steps, timed):
     return out
 
 
+def _latent_cache(dev, seed: int, nseq: int, L: int) -> torch.Tensor:
+    """Seeded synthetic latent KV rows [nseq, L, 576] bf16 ~ N(0, 1), drawn on the
+    device (timing only; the parity tests draw theirs on the host)."""
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+    kv = torch.empty((nseq, L, 576), dtype=torch.bfloat16, device=dev)
+    for b in range(nseq):
+        kv[b] = torch.randn((L, 576), generator=g, device=dev).to(torch.bfloat16)
+    return kv
+
+
+def _sparse_attention(misa, dev, stream, flush, steps, timed):
+    """Sparse attention (128 heads over one 576-entry latent row per token, values
+    = its first 512 entries) over the k = 2048 tokens the indexer selected, and
+    the indexer's share of indexer + attention, at 32K and 128K."""
+    out = {}
+    scale = 192 ** -0.5
+    cases = (("dsv32_decode_L32768", "misa8", lambda wl, B: misa.MisaIndexer(wl.T, wl.H, wl.h, wl.L, B, wl.k,
+                                                                               device=dev)),
+             ("hisa_decode_L131072", "hisa_B128_m64", lambda wl, B: misa.HisaIndexer(wl.T, wl.H, wl.L, B, 64, wl.k,
+                                                                                       device=dev)))
+    for name, tag, make_ix in cases:
+        wl = make_workload(name)
+        q, w, keys, so, pl = (x.to(dev) for x in (wl.q, wl.w, wl.keys, wl.seq_of, wl.prefix_len))
+        means = misa.block_stats(keys, wl.B, split=True)
+        ix = make_ix(wl, wl.B)
+        dx = misa.DenseIndexer(wl.T, wl.H, wl.L, wl.k, device=dev)
+        kv = _latent_cache(dev, 11, wl.nseq, wl.L)
+        g = torch.Generator(device=dev)
+        g.manual_seed(12)
+        qa = torch.randn((wl.T, 128, 576), generator=g, device=dev).to(torch.bfloat16)
+        o = torch.empty((wl.T, 128, 512), dtype=torch.bfloat16, device=dev)
+        ws = misa.alloc_workspace(misa.workspace_bytes(misa._native.OP_SPARSE_MLA, wl.T, 128, 0, 0, wl.k), dev)
+        idx = ix.run(q, w, keys, means, so, pl)
+        attn = lambda evs: misa.sparse_mla(qa, kv, so, idx, scale, out=o, workspace=ws)
+        ms_attn = timed(attn)
+        ms_ix = timed(lambda evs: ix.run(q, w, keys, means, so, pl))
+        ms_dense = timed(lambda evs: dx.run(q, w, keys, so, pl))
+        ms_both = timed(lambda evs: (ix.run(q, w, keys, means, so, pl), attn(evs)))
+        if misa.error_query(ws) != 0:
+            raise RuntimeError("sparse attention recorded a device error")
+        gathered = wl.T * wl.k * 576 * 2
+        flops = 2.0 * wl.T * 128 * wl.k * (576 + 512)
+        out[f"{name}_sparse_mla_k2048"] = {
+            "attention_ms": ms_attn, "attention_GBps_unique_rows": gathered / (ms_attn * 1e-3) / 1e9,
+            "attention_TFLOPs": flops / (ms_attn * 1e-3) / 1e12,
+            f"{tag}_indexer_ms": ms_ix, f"{tag}_plus_attention_ms": ms_both,
+            f"{tag}_share_of_indexer_plus_attention": ms_ix / (ms_ix + ms_attn),
+            "dense64_indexer_ms": ms_dense, "dense64_share_of_indexer_plus_attention": ms_dense / (ms_dense + ms_attn)}
+        del kv, keys
+        torch.cuda.empty_cache()
+    return out
+
+
 def _blas_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -553,7 +609,7 @@ def main():
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     ap.add_argument("--quick", action="store_true", help="skip the other four workloads")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
-    ap.add_argument("--only", choices=["prefill", "dagger", "hisa"], default=None,
+    ap.add_argument("--only", choices=["prefill", "dagger", "hisa", "attn"], default=None,
                     help="time one of the other workloads alone (for profiler captures); prints its own JSON")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -79,6 +79,8 @@ extern "C" {
 #define MISA_MAX_TOPK 16384    /* k (and k') limit of misa_topk */
 #define MISA_MAX_TOPK_ROWS 65535 /* rows (T) limit of the calls that run a top-k */
 #define MISA_ABI_VERSION 1
+#define MISA_MLA_DQK 576       /* misa_sparse_mla: latent KV row (512 latent + 64 rotary) */
+#define MISA_MLA_DV 512        /* misa_sparse_mla: value part (the first 512 entries of a row) */
 
 /* Same object as cudaStream_t (a CUDA runtime stream handle); NULL is the
  * legacy default stream. */
@@ -98,6 +100,7 @@ typedef enum misa_status {
 #define MISA_DEVERR_BAD_SEQ 2u    /* seq_of[t] outside [0, nseq) */
 #define MISA_DEVERR_BAD_HEAD 4u   /* a head id outside [0, H) */
 #define MISA_DEVERR_BAD_LEN 8u    /* misa_append_keys: len[b] < 0 or len[b] + n_new > L_cap */
+#define MISA_DEVERR_BAD_INDEX 16u /* misa_sparse_mla: an index outside [-1, L) (treated as empty) */
 
 /* Static description of a status code (never NULL). */
 MISA_API const char* misa_status_string(int status);
@@ -112,12 +115,14 @@ MISA_API int misa_abi_version(void);
 #define MISA_OP_HIER_RERANK 4
 #define MISA_OP_HISA_BLOCK_FILTER 5
 #define MISA_OP_APPEND_KEYS 6
+#define MISA_OP_SPARSE_MLA 7
 
 /* Bytes of device workspace the operation needs for these sizes (>= 256: the
  * first 256 bytes hold the device error word).  Arguments an operation does not
  * use are ignored:
  *   ROUTE_HEADS: T, H, L, B;  INDEX_SCORE: none;  TOPK: none;
- *   HIER_RERANK: T, kp;  HISA_BLOCK_FILTER: T, L, B;  APPEND_KEYS: none.
+ *   HIER_RERANK: T, kp;  HISA_BLOCK_FILTER: T, L, B;  APPEND_KEYS: none;
+ *   SPARSE_MLA: T, H (= Hq), k.
  * Returns 0 for an unknown op or negative sizes. */
 MISA_API size_t misa_workspace_bytes(int op, int T, int H, int64_t L, int B, int k, int kp);
 
@@ -334,6 +339,40 @@ MISA_API misa_status hisa_block_filter(const uint16_t* q, const float* w, const 
                               const int32_t* prefix_len, int T, int H, int64_t L, int B, int m,
                               int32_t* blocks, int32_t* cand, float* block_scores,
                               void* workspace, size_t workspace_bytes, misa_stream_t stream);
+
+/*
+ * misa_sparse_mla -- attention of every query head over its query's k selected
+ * tokens (the operator the indexer feeds).
+ *   [HISA page (zhichai.net), section 二 (DSA 的工作原理): after the indexer
+ *   picks k tokens per query, attention is computed over those tokens only;
+ *   section 四 (Drop-in Replacement): that operator (Sparse MLA) takes the k
+ *   token indices over the unchanged KV cache.  The pages print no formula;
+ *   this is textbook softmax attention in the multi-query latent form a
+ *   DeepSeek-V3.2-shaped model decodes with.]
+ * kv: nseq caches of L latent rows of MISA_MLA_DQK bf16 (row stride 576,
+ *   sequence stride kv_seq_stride elements, 0 allowed when nseq == 1), shared by
+ *   all query heads: keys are whole rows, values their first MISA_MLA_DV entries.
+ * q: [T][Hq][576] bf16 (the queries with the key up-projection absorbed).
+ * idx: [T] rows of k int32 slots (row stride idx_stride >= k): token ids in
+ *   [0, L) of cache seq_of[t]; -1 = empty slot (the indexer's padding).  Other
+ *   values set MISA_DEVERR_BAD_INDEX and are treated as empty.  Each listed slot
+ *   takes part once.
+ *   out[t][h] = sum_i p_i v_i / sum_i p_i over the listed slots i, with
+ *   p_i = exp(scale * q[t][h] . k_i - max); bf16 [T][Hq][512].  A query with no
+ *   valid slot gets zeros.
+ * lse: [T][Hq] fp32 natural-log sum_i exp(scale * q . k_i) (-inf when empty),
+ *   may be NULL.
+ * Precision: scores fp32 (bf16 inputs), weights rounded to bf16 for the value
+ *   product, fp32 accumulation, bf16 output.
+ * Limits: 1 <= Hq <= 128, 1 <= k <= MISA_MAX_TOPK, T >= 1; q, kv, out 16-byte
+ *   aligned; kv_seq_stride % 8 == 0 and >= L * 576 when nseq > 1.
+ * workspace: >= misa_workspace_bytes(MISA_OP_SPARSE_MLA, T, Hq, 0, 0, k, 0)
+ *   (per-chunk partial results: T * ceil(k / 256) * Hq * 514 * 4 bytes + 256).
+ */
+MISA_API misa_status misa_sparse_mla(const uint16_t* q, const uint16_t* kv, int64_t nseq, int64_t kv_seq_stride,
+                             int64_t L, const int32_t* seq_of, int T, int Hq, const int32_t* idx, int k,
+                             int64_t idx_stride, float scale, uint16_t* out, float* lse, void* workspace,
+                             size_t workspace_bytes, misa_stream_t stream);
 
 #ifdef __cplusplus
 }  /* extern "C" */

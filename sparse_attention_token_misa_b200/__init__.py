@@ -1,4 +1,5 @@
-"""B200-native (sm_100a) MISA / MISA-dagger / HISA token indexer.
+"""B200-native (sm_100a) MISA / MISA-dagger / HISA token indexer, and the
+sparse attention over the tokens it selects.
 
 The compute path is libmisa.so (C ABI in include/misa.h, CUDA kernels under
 csrc/); this package is its Python binding: the same entry points taking torch
@@ -7,11 +8,12 @@ sequences (`indexer`).
 """
 from . import _native
 from ._native import (MisaError, alloc_workspace, append_keys, block_stats, error_query, error_reset,  # noqa: F401
-                      hier_rerank, hisa_block_filter, index_score, lib, route_heads, topk, workspace_bytes)
+                      hier_rerank, hisa_block_filter, index_score, lib, route_heads, sparse_mla, topk,
+                      workspace_bytes)
 from .indexer import DenseIndexer, HisaIndexer, MisaDaggerIndexer, MisaIndexer  # noqa: F401
 
 __all__ = [
     "MisaError", "alloc_workspace", "append_keys", "block_stats", "error_query", "error_reset", "hier_rerank",
-    "hisa_block_filter", "index_score", "lib", "route_heads", "topk", "workspace_bytes",
+    "hisa_block_filter", "index_score", "lib", "route_heads", "sparse_mla", "topk", "workspace_bytes",
     "DenseIndexer", "HisaIndexer", "MisaDaggerIndexer", "MisaIndexer",
 ]

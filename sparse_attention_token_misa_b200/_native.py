@@ -21,10 +21,16 @@ OP_TOPK = 3
 OP_HIER_RERANK = 4
 OP_HISA_BLOCK_FILTER = 5
 OP_APPEND_KEYS = 6
+OP_SPARSE_MLA = 7
 
 DEVERR_TIMEOUT = 1
 DEVERR_BAD_SEQ = 2
 DEVERR_BAD_HEAD = 4
+DEVERR_BAD_LEN = 8
+DEVERR_BAD_INDEX = 16
+
+MLA_DQK = 576   # latent KV row: 512 latent + 64 rotary
+MLA_DV = 512    # value part: the first 512 entries of a row
 
 HEAD_DIM = 128
 
@@ -54,6 +60,8 @@ SIGNATURES = {
     "misa_topk": (c_int, [c_vp, c_int, c_i64, c_i64, c_vp, c_vp, c_i64, c_int, c_vp, c_vp, c_size, c_vp]),
     "misa_hier_rerank": (c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_i64, c_vp, c_int,
                                  c_int, c_vp, c_vp, c_vp, c_size, c_vp]),
+    "misa_sparse_mla": (c_int, [c_vp, c_vp, c_i64, c_i64, c_i64, c_vp, c_int, c_int, c_vp, c_int, c_i64,
+                                ctypes.c_float, c_vp, c_vp, c_vp, c_size, c_vp]),
     "hisa_block_filter": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_i64,
                                   c_int, c_int, c_vp, c_vp, c_vp, c_vp, c_size, c_vp]),
 }
@@ -334,3 +342,30 @@ def hisa_block_filter(q, w, means, seq_of, prefix_len, L: int, B: int, m: int, b
           _p(prefix_len), T, H, L, B, m, _p(blocks), _p(cand), _p(block_scores), _p(workspace), workspace.numel(),
           _stream(stream))
     return blocks, cand, block_scores
+
+
+def sparse_mla(q, kv, seq_of, idx, scale: float, out=None, lse=None, want_lse: bool = False, workspace=None,
+               stream=None):
+    """misa_sparse_mla -> (out [T, Hq, 512] bf16, lse [T, Hq] fp32 or None).
+
+    q [T, Hq, 576] bf16; kv [nseq, L, 576] bf16 latent rows (keys = whole row,
+    values = the first 512 entries); idx [T, k] int32 token ids, -1 = empty."""
+    _req(q, torch.bfloat16, "q"); _req(kv, torch.bfloat16, "kv", contiguous=False)
+    _req(seq_of, torch.int32, "seq_of"); _req(idx, torch.int32, "idx", contiguous=False)
+    if kv.stride(2) != 1 or kv.stride(1) != MLA_DQK:
+        raise ValueError("kv rows must be contiguous 576-element rows")
+    if idx.stride(1) != 1:
+        raise ValueError("idx rows must be contiguous")
+    T, Hq, _ = q.shape
+    nseq, L, _ = kv.shape
+    k = idx.shape[1]
+    if out is None:
+        out = torch.empty((T, Hq, MLA_DV), dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty((T, Hq), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(workspace_bytes(OP_SPARSE_MLA, T, Hq, 0, 0, k), q.device)
+    _call("misa_sparse_mla", _p(q), _p(kv), nseq, int(kv.stride(0)) if nseq > 1 else 0, L, _p(seq_of), T, Hq,
+          _p(idx), k, int(idx.stride(0)), float(scale), _p(out), _p(lse), _p(workspace), workspace.numel(),
+          _stream(stream))
+    return out, lse

@@ -111,7 +111,6 @@ const char* misa_status_string(int status) {
 int misa_abi_version(void) { return MISA_ABI_VERSION; }
 
 size_t misa_workspace_bytes(int op, int T, int H, int64_t L, int B, int k, int kp) {
-  (void)k;
   if (T < 0 || H < 0 || L < 0 || B < 0 || kp < 0) return 0;
   switch (op) {
     case MISA_OP_ROUTE_HEADS:
@@ -124,6 +123,9 @@ size_t misa_workspace_bytes(int op, int T, int H, int64_t L, int B, int k, int k
       return kErrBytes;
     case MISA_OP_HIER_RERANK:
       return kErrBytes + static_cast<size_t>(T) * round_up4(kp) * sizeof(float);
+    case MISA_OP_SPARSE_MLA:
+      if (k < 1) return 0;
+      return kErrBytes + static_cast<size_t>(T) * misa::sparse_mla_chunks(k) * H * (MISA_MLA_DV + 2) * sizeof(float);
     case MISA_OP_HISA_BLOCK_FILTER: {
       if (B < 1) return 0;
       const int64_t M = ceil_div(L, B);
@@ -333,6 +335,31 @@ misa_status hisa_block_filter(const uint16_t* q, const float* w, const float* me
     if (e != cudaSuccess) return MISA_ERR_CUDA;
   }
   return MISA_OK;
+}
+
+misa_status misa_sparse_mla(const uint16_t* q, const uint16_t* kv, int64_t nseq, int64_t kv_seq_stride, int64_t L,
+                            const int32_t* seq_of, int T, int Hq, const int32_t* idx, int k, int64_t idx_stride,
+                            float scale, uint16_t* out, float* lse, void* workspace, size_t workspace_bytes,
+                            misa_stream_t stream) {
+  if (!q || !kv || !seq_of || !idx || !out) return MISA_ERR_INVALID_ARG;
+  if (T < 1 || Hq < 1 || k < 1 || L < 1 || nseq < 1 || idx_stride < k) return MISA_ERR_INVALID_ARG;
+  if (Hq > 128 || k > MISA_MAX_TOPK) return MISA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(kv) || !aligned16(out) || kv_seq_stride < 0 || kv_seq_stride % 8 != 0)
+    return MISA_ERR_INVALID_ARG;
+  if (nseq > 1 && kv_seq_stride < L * MISA_MLA_DQK) return MISA_ERR_INVALID_ARG;
+  // query rows and grid sizes are 32-bit
+  if (static_cast<int64_t>(T) * Hq >= (static_cast<int64_t>(1) << 31) ||
+      static_cast<int64_t>(T) * misa::sparse_mla_chunks(k) >= (static_cast<int64_t>(1) << 31) ||
+      L >= (static_cast<int64_t>(1) << 31))
+    return MISA_ERR_UNSUPPORTED;
+  misa_status st = check_ws(workspace, workspace_bytes, misa_workspace_bytes(MISA_OP_SPARSE_MLA, T, Hq, 0, 0, k, 0));
+  if (st != MISA_OK) return st;
+  const int nch = misa::sparse_mla_chunks(k);
+  float* part_o = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kErrBytes);
+  float* part_ml = part_o + static_cast<size_t>(T) * nch * Hq * MISA_MLA_DV;
+  return cuda_status(misa::launch_sparse_mla(q, kv, nseq, kv_seq_stride, L, seq_of, T, Hq, idx, k, idx_stride, scale,
+                                             out, lse, part_o, part_ml, err_word(workspace),
+                                             reinterpret_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

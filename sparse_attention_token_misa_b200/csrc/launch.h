@@ -84,6 +84,15 @@ cudaError_t launch_hisa_block_scores_tc(const uint16_t* q, const float* w, const
                                         int64_t L, int B, float* bscore,
                                         int64_t bs_stride, uint32_t* err, cudaStream_t stream);
 
+// Sparse attention over selected tokens (sparse_mla.cu): chunks of 256 index
+// slots per query, partial results in part_o [T][nch][Hq][512] and part_ml
+// [T][nch][Hq][2], merged by a second kernel into out / lse.
+int sparse_mla_chunks(int k);
+cudaError_t launch_sparse_mla(const uint16_t* q, const uint16_t* kv, int64_t nseq, int64_t kv_seq_stride, int64_t L,
+                              const int32_t* seq_of, int T, int Hq, const int32_t* idx, int k, int64_t idx_stride,
+                              float scale, uint16_t* out, float* lse, float* part_o, float* part_ml, uint32_t* err,
+                              cudaStream_t stream);
+
 cudaError_t launch_hisa_expand(const int32_t* blocks, const int32_t* prefix_len, int T, int m, int B, int64_t L,
                                int32_t* cand, cudaStream_t stream);
 

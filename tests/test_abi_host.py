@@ -34,7 +34,7 @@ def declared_functions():
 def test_library_loads_and_exports_every_declared_symbol():
     l = pkg.lib()
     names = declared_functions()
-    assert len(names) == 13, names
+    assert len(names) == 14, names
     for n in names:
         assert hasattr(l, n), n
         assert n in nat.SIGNATURES, n
@@ -60,6 +60,10 @@ def test_workspace_formula():
     assert ws(nat.OP_HIER_RERANK, 2, 32, 100, 1, 3, 5) == 256 + 2 * 8 * 4
     assert ws(nat.OP_HISA_BLOCK_FILTER, 16, 64, 131072, 128, 64) == 256 + 16 * 1024 * 4
     assert ws(nat.OP_HISA_BLOCK_FILTER, 1, 2, 8, 3, 2) == 256 + 1 * 4 * 4
+    # sparse attention: 256 + T * ceil(k / 256) * Hq * (512 + 2) * 4
+    assert ws(nat.OP_SPARSE_MLA, 32, 128, 0, 0, 2048) == 256 + 32 * 8 * 128 * 514 * 4
+    assert ws(nat.OP_SPARSE_MLA, 3, 16, 0, 0, 257) == 256 + 3 * 2 * 16 * 514 * 4
+    assert ws(nat.OP_SPARSE_MLA, 3, 16, 0, 0, 0) == 0
     assert ws(99, 1, 1, 1, 1) == 0
     assert ws(nat.OP_ROUTE_HEADS, -1, 1, 1, 1) == 0
 
@@ -211,3 +215,32 @@ def test_append_keys_validation():
     assert append(ws_bytes=255) == WORKSPACE
     assert append(hi=P) == INVALID                           # split: both or neither
     assert append(hi=P, lo=MIS) == INVALID
+
+
+def mla(q=P, kv=P, nseq=1, stride=0, L=1000, seq_of=P, T=2, Hq=128, idx=P2, k=300, idx_stride=300, scale=0.1,
+        out=P2 + 4096, lse=None, ws=P2 + 8192, ws_bytes=1 << 22):
+    return pkg.lib().misa_sparse_mla(q, kv, nseq, stride, L, seq_of, T, Hq, idx, k, idx_stride, scale, out, lse, ws,
+                                     ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), INVALID),
+    (dict(kv=None), INVALID),
+    (dict(idx=None), INVALID),
+    (dict(out=None), INVALID),
+    (dict(T=0), INVALID),
+    (dict(Hq=0), INVALID),
+    (dict(Hq=129), UNSUPPORTED),
+    (dict(k=0), INVALID),
+    (dict(k=16385, idx_stride=16385), UNSUPPORTED),
+    (dict(idx_stride=299), INVALID),              # rows shorter than k
+    (dict(q=MIS), INVALID),
+    (dict(kv=MIS), INVALID),
+    (dict(out=MIS), INVALID),
+    (dict(nseq=2, stride=4), INVALID),            # stride % 8
+    (dict(nseq=2, stride=576 * 999), INVALID),    # sequences would overlap
+    (dict(ws=None), WORKSPACE),
+    (dict(ws_bytes=256), WORKSPACE),
+])
+def test_sparse_mla_rejects(kw, status):
+    assert mla(**kw) == status
