@@ -60,7 +60,8 @@ static_assert(kS3 * kVStageBytes <= kStageRegion, "value stages must fit the QK 
 constexpr int kOffP = kOffStage + kStageRegion;
 constexpr int kPBytes = kHM * kSlots * 2;      // 64 KB
 constexpr int kOffIds = kOffP + kPBytes;
-constexpr int kOffBar = kOffIds + kSlots * 4;
+constexpr int kOffMask = kOffIds + kSlots * 4;   // [kSlots / 32] valid-slot bits
+constexpr int kOffBar = kOffMask + (kSlots / 32) * 4;
 constexpr int kNumBars = 2 * kS1 + 2 * kS3 + 4;
 constexpr int kOffTmem = kOffBar + kNumBars * 8;
 constexpr int kOffFlag = kOffTmem + 16;
@@ -109,6 +110,7 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap q_map, const MlaParams p) 
   uint8_t* sStage = smem + kOffStage;
   uint8_t* sP = smem + kOffP;
   int32_t* sIds = reinterpret_cast<int32_t*>(smem + kOffIds);
+  uint32_t* sMask = reinterpret_cast<uint32_t*>(smem + kOffMask);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
   uint64_t* full1 = bars;                    // [kS1] query block (TMA) + key rows (cp.async) landed
   uint64_t* empty1 = bars + kS1;             // [kS1] QK MMAs of the stage done
@@ -166,6 +168,11 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap q_map, const MlaParams p) 
     sIds[j] = id;
   }
   __syncthreads();
+  if (warp < kSlots / 32) {
+    const unsigned bits = __ballot_sync(0xffffffffu, sIds[warp * 32 + lane] >= 0);
+    if (lane == 0) sMask[warp] = bits;
+  }
+  __syncthreads();
 
   if (warp >= kProdWarp0) {
     // ------------------------------------------------------------ producers
@@ -202,8 +209,8 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap q_map, const MlaParams p) 
           cp_async_16(kdst + r * 128 + ((ch ^ (r & 7)) << 4), src, valid);
         }
         cp_async_commit();
-        if (kb - pending >= 1) {
-          cp_async_wait_group<1>();
+        if (kb - pending >= kS1 - 1) {
+          cp_async_wait_group<kS1 - 1>();
           fence_proxy_async_smem();
           mbar_arrive(&full1[pending % kS1]);
           ++pending;
@@ -234,8 +241,8 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap q_map, const MlaParams p) 
           cp_async_16(vdst + (ch >> 3) * kVAtomBytes + r * 128 + (((ch & 7) ^ (r & 7)) << 4), src, valid);
         }
         cp_async_commit();
-        if (vb - pending >= 1) {
-          cp_async_wait_group<1>();
+        if (vb - pending >= kS3 - 1) {
+          cp_async_wait_group<kS3 - 1>();
           fence_proxy_async_smem();
           mbar_arrive(&full3[pending % kS3]);
           ++pending;
@@ -303,7 +310,8 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap q_map, const MlaParams p) 
     const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
     const bool live = r < p.Hq;
     const float kNegInf = -__int_as_float(0x7f800000);
-    bool ok = mbar_wait(sfull, 0, p.err, abort);
+    // warp-uniform outcome of the wait: the TMEM loads below are warp-wide
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(sfull, 0, p.err, abort));
     float mx = kNegInf, l = 0.f;
     if (ok) {
       tc_fence_after();
@@ -311,20 +319,21 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap q_map, const MlaParams p) 
       for (int c0 = 0; c0 < kSlots; c0 += 16) {
         tmem_ld16(t_lane + c0, v);
         tmem_wait_ld();
+        const uint32_t bits = sMask[c0 >> 5] >> (c0 & 31);
 #pragma unroll
         for (int j = 0; j < 16; ++j)
-          if (sIds[c0 + j] >= 0) mx = fmaxf(mx, __uint_as_float(v[j]) * p.scale_log2);
+          if ((bits >> j) & 1u) mx = fmaxf(mx, __uint_as_float(v[j]) * p.scale_log2);
       }
       const bool any = mx != kNegInf;
       for (int c0 = 0; c0 < kSlots; c0 += 16) {
         tmem_ld16(t_lane + c0, v);
         tmem_wait_ld();
+        const uint32_t bits = any ? sMask[c0 >> 5] >> (c0 & 31) : 0u;
         uint32_t w[8];
 #pragma unroll
         for (int j = 0; j < 16; j += 2) {
-          const float a = (any && sIds[c0 + j] >= 0) ? exp2f(__uint_as_float(v[j]) * p.scale_log2 - mx) : 0.f;
-          const float b =
-              (any && sIds[c0 + j + 1] >= 0) ? exp2f(__uint_as_float(v[j + 1]) * p.scale_log2 - mx) : 0.f;
+          const float a = ((bits >> j) & 1u) ? exp2f(__uint_as_float(v[j]) * p.scale_log2 - mx) : 0.f;
+          const float b = ((bits >> (j + 1)) & 1u) ? exp2f(__uint_as_float(v[j + 1]) * p.scale_log2 - mx) : 0.f;
           const __nv_bfloat16 ha = __float2bfloat16_rn(a), hb = __float2bfloat16_rn(b);
           l += __bfloat162float(ha) + __bfloat162float(hb);
           w[j >> 1] = static_cast<uint32_t>(__bfloat16_as_ushort(ha)) |
@@ -348,20 +357,35 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap q_map, const MlaParams p) 
       p.part_ml[prow * 2] = mx;
       p.part_ml[prow * 2 + 1] = l;
     }
-    if (ok && mbar_wait(ofull, 0, p.err, abort)) {
-      tc_fence_after();
-      float* orow = p.part_o + prow * kDv;
-      uint32_t v[16];
-      for (int c0 = 0; c0 < kDv; c0 += 16) {
-        tmem_ld16(t_lane + c0, v);
-        tmem_wait_ld();
-        if (live) {
+    // O by quarters of 128 columns through the (now idle) stage region, so that
+    // each row leaves as one coalesced 512-byte store: thread r writes its row
+    // quarter at pitch 132 floats (4 store wavefronts per warp, the minimum),
+    // then warp w copies rows w, w + 4, ...
+    const bool ok_o = __all_sync(0xffffffffu, ok && mbar_wait(ofull, 0, p.err, abort));
+    if (ok_o) tc_fence_after();
+    constexpr int kPitch = 132;
+    float* stg = reinterpret_cast<float*>(sStage);
+    for (int q4 = 0; q4 < kDv / 128; ++q4) {
+      if (ok_o) {
+        uint32_t v[16];
+        for (int u = 0; u < 8; ++u) {
+          tmem_ld16(t_lane + q4 * 128 + u * 16, v);
+          tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 16; j += 4)
-            *reinterpret_cast<float4*>(orow + c0 + j) = make_float4(
+            *reinterpret_cast<float4*>(stg + r * kPitch + u * 16 + j) = make_float4(
                 __uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
         }
       }
+      named_bar_sync(1, kEpiThreads);
+      if (ok_o) {
+        for (int rr = warp; rr < p.Hq; rr += kEpiThreads / 32) {
+          const float4 x = *reinterpret_cast<const float4*>(stg + rr * kPitch + lane * 4);
+          const int64_t orow = (static_cast<int64_t>(t) * p.nch + c) * p.Hq + rr;
+          *reinterpret_cast<float4*>(p.part_o + orow * kDv + q4 * 128 + lane * 4) = x;
+        }
+      }
+      named_bar_sync(1, kEpiThreads);
     }
   }
 
