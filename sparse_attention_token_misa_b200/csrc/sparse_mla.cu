@@ -17,10 +17,11 @@
 //     blocks of 64; the query block arrives by TMA, the 256 gathered key rows by
 //     16-byte cp.async in the 128-byte-swizzled K-major layout; S in TMEM
 //     columns [0, 256).
-//  2. Exact softmax over the chunk: the epilogue thread of head h reads its S
-//     row twice from TMEM (max, then exp2), rounds p to bf16, adds the rounded
-//     values into l and writes p as the A operand of the next MMA (K-major,
-//     swizzled) to shared memory.
+//  2. Exact softmax over the chunk: two epilogue threads per head h (one per
+//     half of the slots) read their part of the S row twice from TMEM (max,
+//     exchanged through shared memory, then exp2), round p to bf16, add the
+//     rounded values into l and write p as the A operand of the next MMA
+//     (K-major, swizzled) to shared memory.
 //  3. O = P V: M = 128 heads, N = 512 value columns (two MMAs of 256), K = 256
 //     slots in blocks of 32.  V is staged MN-major (each token's 512 values are
 //     one row of eight 64-column swizzle atoms), so the gathered rows need no
@@ -31,9 +32,10 @@
 //     kernel merges the chunks of each query (flash-decoding style) and writes
 //     bf16 out and, optionally, the log-sum-exp.
 //
-// Roles (288 threads): warps 0-3 epilogue (TMEM lane quarter = warp), warp 4
-// TMEM allocation + MMA issue, warps 5-8 producers (thread 0 of them also
-// issues the query TMA).  Waits are bounded and share a CTA-wide abort flag.
+// Roles (416 threads): warps 0-7 epilogue (warp w: TMEM lane quarter w % 4,
+// slot / column half w / 4), warp 8 TMEM allocation + MMA issue, warps 9-12
+// producers (thread 0 of them also issues the query TMA).  Waits are bounded
+// and share a CTA-wide abort flag.
 #include "launch.h"
 #include "misa_device.cuh"
 
@@ -65,12 +67,15 @@ constexpr int kOffBar = kOffMask + (kSlots / 32) * 4;
 constexpr int kNumBars = 2 * kS1 + 2 * kS3 + 4;
 constexpr int kOffTmem = kOffBar + kNumBars * 8;
 constexpr int kOffFlag = kOffTmem + 16;
-constexpr int kSmemBytes = kOffFlag + 16 + 1024;
-constexpr int kThreads = 288;
-constexpr int kEpiThreads = 128;
-constexpr int kMmaWarp = 4;
-constexpr int kProdWarp0 = 5;
+constexpr int kOffRed = kOffFlag + 16;           // [2][kHM] per-half row maxima / sums
+constexpr int kSmemBytes = kOffRed + 2 * kHM * 4 + 1024;
+constexpr int kThreads = 416;
+constexpr int kEpiThreads = 256;
+constexpr int kMmaWarp = 8;
+constexpr int kProdWarp0 = 9;
 constexpr int kProdThreads = 128;
+constexpr int kPitch = 132;                      // O staging row pitch (floats)
+static_assert(2 * kHM * kPitch * 4 <= kStageRegion, "O staging must fit the stage region");
 constexpr uint32_t kIdescS = idesc_bf16_f32(kHM, kSlots);
 // P V: B (the values) is MN-major
 constexpr uint32_t kIdescO = idesc_bf16_f32(kHM, 256) | (1u << 16);
@@ -305,18 +310,21 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap q_map, const MlaParams p) 
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ epilogue (thread = head row)
-    const int r = warp * 32 + lane;
-    const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
+    // ------------------------------------------------------------ epilogue (two threads per head row)
+    const int quarter = warp & 3, half = warp >> 2;
+    const int r = quarter * 32 + lane;  // head row
+    const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16);
     const bool live = r < p.Hq;
     const float kNegInf = -__int_as_float(0x7f800000);
+    float* sRed = reinterpret_cast<float*>(smem + kOffRed);
     // warp-uniform outcome of the wait: the TMEM loads below are warp-wide
     const bool ok = __all_sync(0xffffffffu, mbar_wait(sfull, 0, p.err, abort));
+    const int cbeg = half * (kSlots / 2), cend = cbeg + kSlots / 2;
     float mx = kNegInf, l = 0.f;
+    uint32_t v[16];
     if (ok) {
       tc_fence_after();
-      uint32_t v[16];
-      for (int c0 = 0; c0 < kSlots; c0 += 16) {
+      for (int c0 = cbeg; c0 < cend; c0 += 16) {
         tmem_ld16(t_lane + c0, v);
         tmem_wait_ld();
         const uint32_t bits = sMask[c0 >> 5] >> (c0 & 31);
@@ -324,8 +332,13 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap q_map, const MlaParams p) 
         for (int j = 0; j < 16; ++j)
           if ((bits >> j) & 1u) mx = fmaxf(mx, __uint_as_float(v[j]) * p.scale_log2);
       }
+    }
+    sRed[half * kHM + r] = mx;
+    named_bar_sync(1, kEpiThreads);
+    mx = fmaxf(sRed[r], sRed[kHM + r]);
+    if (ok) {
       const bool any = mx != kNegInf;
-      for (int c0 = 0; c0 < kSlots; c0 += 16) {
+      for (int c0 = cbeg; c0 < cend; c0 += 16) {
         tmem_ld16(t_lane + c0, v);
         tmem_wait_ld();
         const uint32_t bits = any ? sMask[c0 >> 5] >> (c0 & 31) : 0u;
@@ -350,24 +363,26 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap q_map, const MlaParams p) 
     }
     fence_proxy_async_smem();
     tc_fence_before();
+    named_bar_sync(1, kEpiThreads);  // P complete, S read, every maximum read
+    if (ok && warp == 0 && lane == 0) mbar_arrive(pfull);
+    sRed[half * kHM + r] = l;
     named_bar_sync(1, kEpiThreads);
-    if (ok && r == 0) mbar_arrive(pfull);
-    const int64_t prow = (static_cast<int64_t>(t) * p.nch + c) * p.Hq + r;
-    if (live) {
+    if (half == 0 && live) {
+      const int64_t prow = (static_cast<int64_t>(t) * p.nch + c) * p.Hq + r;
       p.part_ml[prow * 2] = mx;
-      p.part_ml[prow * 2 + 1] = l;
+      p.part_ml[prow * 2 + 1] = sRed[r] + sRed[kHM + r];
     }
-    // O by quarters of 128 columns through the (now idle) stage region, so that
-    // each row leaves as one coalesced 512-byte store: thread r writes its row
-    // quarter at pitch 132 floats (4 store wavefronts per warp, the minimum),
-    // then warp w copies rows w, w + 4, ...
+    // O by quarters of 128 columns (half h: quarters 2h, 2h + 1) through the
+    // (now idle) stage region, so that each row leaves as one coalesced
+    // 512-byte store: thread r writes its row quarter at pitch 132 floats (4
+    // store wavefronts per warp, the minimum), then the half's warp q copies
+    // rows q, q + 4, ...
     const bool ok_o = __all_sync(0xffffffffu, ok && mbar_wait(ofull, 0, p.err, abort));
     if (ok_o) tc_fence_after();
-    constexpr int kPitch = 132;
-    float* stg = reinterpret_cast<float*>(sStage);
-    for (int q4 = 0; q4 < kDv / 128; ++q4) {
+    float* stg = reinterpret_cast<float*>(sStage) + half * (kHM * kPitch);
+    for (int qq = 0; qq < 2; ++qq) {
+      const int q4 = half * 2 + qq;
       if (ok_o) {
-        uint32_t v[16];
         for (int u = 0; u < 8; ++u) {
           tmem_ld16(t_lane + q4 * 128 + u * 16, v);
           tmem_wait_ld();
@@ -377,15 +392,15 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap q_map, const MlaParams p) 
                 __uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
         }
       }
-      named_bar_sync(1, kEpiThreads);
+      named_bar_sync(2 + half, kEpiThreads / 2);
       if (ok_o) {
-        for (int rr = warp; rr < p.Hq; rr += kEpiThreads / 32) {
+        for (int rr = quarter; rr < p.Hq; rr += 4) {
           const float4 x = *reinterpret_cast<const float4*>(stg + rr * kPitch + lane * 4);
           const int64_t orow = (static_cast<int64_t>(t) * p.nch + c) * p.Hq + rr;
           *reinterpret_cast<float4*>(p.part_o + orow * kDv + q4 * 128 + lane * 4) = x;
         }
       }
-      named_bar_sync(1, kEpiThreads);
+      named_bar_sync(2 + half, kEpiThreads / 2);
     }
   }
 
@@ -396,32 +411,67 @@ sparse_mla_kernel(const __grid_constant__ CUtensorMap q_map, const MlaParams p) 
 }
 
 // out[t, h] = sum_c 2^(m_c - m) O_c / sum_c 2^(m_c - m) l_c, m = max_c m_c; one
-// CTA of 128 threads per (t, h), 4 value columns per thread.
+// CTA of 128 threads per (t, h), 4 value columns per thread.  The chunk
+// statistics are read by one thread each, the weights and the denominator are
+// formed in chunk order (deterministic), and the chunk rows are then loaded
+// four at a time.
+constexpr int kMaxChunks = (MISA_MAX_TOPK + kSlots - 1) / kSlots;  // 64
 __global__ void __launch_bounds__(128)
 sparse_mla_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml, int T, int Hq,
                           int nch, uint16_t* __restrict__ out, float* __restrict__ lse) {
+  __shared__ float s_m[kMaxChunks], s_w[kMaxChunks];
+  __shared__ float s_den;
   pdl_wait_inputs();
   pdl_allow_next();
   const int th = static_cast<int>(blockIdx.x);
   const int t = th / Hq, h = th - t * Hq;
+  const int tid = threadIdx.x;
   const float kNegInf = -__int_as_float(0x7f800000);
+  const int64_t row0 = static_cast<int64_t>(t) * nch * Hq + h;  // chunk c: row0 + c * Hq
+  float lc = 0.f;
+  if (tid < nch) {
+    s_m[tid] = part_ml[(row0 + static_cast<int64_t>(tid) * Hq) * 2];
+    lc = part_ml[(row0 + static_cast<int64_t>(tid) * Hq) * 2 + 1];
+  }
+  __syncthreads();
   float m = kNegInf;
-  for (int c = 0; c < nch; ++c) m = fmaxf(m, part_ml[((static_cast<int64_t>(t) * nch + c) * Hq + h) * 2]);
+  for (int c = 0; c < nch; ++c) m = fmaxf(m, s_m[c]);
+  if (tid < nch) s_w[tid] = (m == kNegInf || s_m[tid] == kNegInf) ? 0.f : exp2f(s_m[tid] - m);
+  __syncthreads();
+  if (tid < nch) s_m[tid] = s_w[tid] * lc;  // weighted sums, reusing s_m
+  __syncthreads();
+  if (tid == 0) {
+    float den = 0.f;
+    for (int c = 0; c < nch; ++c) den += s_m[c];
+    s_den = den;
+  }
+  __syncthreads();
+  const float den = s_den;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  float den = 0.f;
-  if (m != kNegInf) {
-    for (int c = 0; c < nch; ++c) {
-      const int64_t row = (static_cast<int64_t>(t) * nch + c) * Hq + h;
-      const float mc = part_ml[row * 2];
-      if (mc == kNegInf) continue;
-      const float wc = exp2f(mc - m);
-      den += wc * part_ml[row * 2 + 1];
-      const float4 o = __ldcs(reinterpret_cast<const float4*>(part_o + row * kDv) + threadIdx.x);
-      acc.x += wc * o.x;
-      acc.y += wc * o.y;
-      acc.z += wc * o.z;
-      acc.w += wc * o.w;
+  const float4* base = reinterpret_cast<const float4*>(part_o + row0 * kDv) + tid;
+  const int64_t cstride = static_cast<int64_t>(Hq) * kDv / 4;  // float4s between chunks
+  int c = 0;
+  for (; c + 4 <= nch; c += 4) {
+    float4 o[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) o[u] = s_w[c + u] != 0.f ? __ldcs(base + (c + u) * cstride) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float wc = s_w[c + u];
+      acc.x += wc * o[u].x;
+      acc.y += wc * o[u].y;
+      acc.z += wc * o[u].z;
+      acc.w += wc * o[u].w;
     }
+  }
+  for (; c < nch; ++c) {
+    const float wc = s_w[c];
+    if (wc == 0.f) continue;
+    const float4 o = __ldcs(base + c * cstride);
+    acc.x += wc * o.x;
+    acc.y += wc * o.y;
+    acc.z += wc * o.z;
+    acc.w += wc * o.w;
   }
   const float inv = den > 0.f ? 1.0f / den : 0.f;
   const __nv_bfloat16 a = __float2bfloat16_rn(acc.x * inv), b = __float2bfloat16_rn(acc.y * inv);
@@ -429,9 +479,8 @@ sparse_mla_combine_kernel(const float* __restrict__ part_o, const float* __restr
   uint2 packed;
   packed.x = static_cast<uint32_t>(__bfloat16_as_ushort(a)) | (static_cast<uint32_t>(__bfloat16_as_ushort(b)) << 16);
   packed.y = static_cast<uint32_t>(__bfloat16_as_ushort(c2)) | (static_cast<uint32_t>(__bfloat16_as_ushort(d)) << 16);
-  *reinterpret_cast<uint2*>(out + (static_cast<int64_t>(t) * Hq + h) * kDv + threadIdx.x * 4) = packed;
-  if (lse && threadIdx.x == 0)
-    lse[static_cast<int64_t>(t) * Hq + h] = den > 0.f ? (m + log2f(den)) * 0.69314718055994531f : kNegInf;
+  *reinterpret_cast<uint2*>(out + (static_cast<int64_t>(t) * Hq + h) * kDv + tid * 4) = packed;
+  if (lse && tid == 0) lse[static_cast<int64_t>(t) * Hq + h] = den > 0.f ? (m + log2f(den)) * 0.69314718055994531f : kNegInf;
 }
 
 }  // namespace
