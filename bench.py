@@ -530,10 +530,15 @@ def _sparse_attention(misa, dev, stream, flush, steps, timed):
         if misa.error_query(ws) != 0:
             raise RuntimeError("sparse attention recorded a device error")
         gathered = wl.T * wl.k * 576 * 2
+        moved = gathered + wl.T * 128 * (576 + 512) * 2          # + q rows and the bf16 output
         flops = 2.0 * wl.T * 128 * wl.k * (576 + 512)
+        hbm, tc, kind = _peaks()
         out[f"{name}_sparse_mla_k2048"] = {
             "attention_ms": ms_attn, "attention_GBps_unique_rows": gathered / (ms_attn * 1e-3) / 1e9,
             "attention_TFLOPs": flops / (ms_attn * 1e-3) / 1e12,
+            "attention_roofline": {"bound": "hbm", "achieved": moved / (ms_attn * 1e-3) / 1e9, "peak": hbm,
+                                   "unit": "GB/s", "frac": moved / (ms_attn * 1e-3) / 1e9 / hbm,
+                                   "tensor_frac": flops / (ms_attn * 1e-3) / 1e12 / tc, "peaks": kind},
             f"{tag}_indexer_ms": ms_ix, f"{tag}_plus_attention_ms": ms_both,
             f"{tag}_share_of_indexer_plus_attention": ms_ix / (ms_ix + ms_attn),
             "dense64_indexer_ms": ms_dense, "dense64_share_of_indexer_plus_attention": ms_dense / (ms_dense + ms_attn)}
