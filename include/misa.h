@@ -341,6 +341,40 @@ MISA_API misa_status hisa_block_filter(const uint16_t* q, const float* w, const 
                               void* workspace, size_t workspace_bytes, misa_stream_t stream);
 
 /*
+ * misa_shard_prefix -- prefix lengths of one key shard (context parallelism).
+ *   [MISA page (gist.science), "Methodology: MISA": the head importance sums
+ *   over visible blocks and the scores are per token, so a key shard can be
+ *   indexed on its own.  The pages do not shard; this is the library's
+ *   key-sharded form.]
+ * A rank holds keys [s0, s0 + L_shard) of every sequence; its key at local
+ * position s is visible to query t iff s < out[t] = clamp(prefix_len[t] - s0,
+ * 0, L_shard).  Pass out as the prefix_len of misa_route_heads /
+ * misa_index_score / misa_topk (row_valid) over the shard (s0 a multiple of B,
+ * so the shard's blocks are the global blocks).
+ * prefix_len, out: [T] int32, device.  T >= 1, s0 >= 0, L_shard >= 1.
+ */
+MISA_API misa_status misa_shard_prefix(const int32_t* prefix_len, int T, int64_t s0, int64_t L_shard, int32_t* out,
+                             misa_stream_t stream);
+
+/*
+ * misa_gather_candidates -- (score, global token id) pairs of a shard's local
+ * top-k, for the exchange that merges the shards.
+ *   out_scores[t][i] = scores[t * row_stride + idx[t][i]] and
+ *   out_ids[t][i] = idx[t][i] + id_offset when 0 <= idx[t][i] < n; otherwise
+ *   (-inf, -1), which misa_topk never selects.  The top-k of the union of the
+ *   shards' candidate lists (misa_topk with id_map = the gathered ids, shards
+ *   in ascending s0 order) is the top-k of the whole row, ties included: the
+ *   lists are ascending, so the lower position is the lower token id.
+ * scores: [T] rows of n fp32 (row stride row_stride); idx: [T][k] int32 local
+ * positions; out_scores [T][k] fp32, out_ids [T][k] int32; all device.
+ * Limits: T >= 1, 1 <= k, n >= 1, row_stride >= n, 0 <= id_offset and
+ *   id_offset + n < 2^31.
+ */
+MISA_API misa_status misa_gather_candidates(const float* scores, int T, int64_t n, int64_t row_stride,
+                             const int32_t* idx, int k, int64_t id_offset, float* out_scores,
+                             int32_t* out_ids, misa_stream_t stream);
+
+/*
  * misa_sparse_mla -- attention of every query head over its query's k selected
  * tokens (the operator the indexer feeds).
  *   [HISA page (zhichai.net), section 二 (DSA 的工作原理): after the indexer

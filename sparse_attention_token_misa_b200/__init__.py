@@ -8,12 +8,14 @@ sequences (`indexer`).
 """
 from . import _native
 from ._native import (MisaError, alloc_workspace, append_keys, block_stats, error_query, error_reset,  # noqa: F401
-                      hier_rerank, hisa_block_filter, index_score, lib, route_heads, sparse_mla, topk,
-                      workspace_bytes)
+                      gather_candidates, hier_rerank, hisa_block_filter, index_score, lib, route_heads,
+                      shard_prefix, sparse_mla, topk, workspace_bytes)
 from .indexer import DenseIndexer, HisaIndexer, MisaDaggerIndexer, MisaIndexer  # noqa: F401
+from .sharded import ShardedMisaIndexer, TorchShardComm, shard_bounds  # noqa: F401
 
 __all__ = [
-    "MisaError", "alloc_workspace", "append_keys", "block_stats", "error_query", "error_reset", "hier_rerank",
+    "MisaError", "alloc_workspace", "append_keys", "block_stats", "error_query", "error_reset",
+    "gather_candidates", "hier_rerank", "shard_prefix", "ShardedMisaIndexer", "TorchShardComm", "shard_bounds",
     "hisa_block_filter", "index_score", "lib", "route_heads", "sparse_mla", "topk", "workspace_bytes",
     "DenseIndexer", "HisaIndexer", "MisaDaggerIndexer", "MisaIndexer",
 ]

@@ -60,6 +60,8 @@ SIGNATURES = {
     "misa_topk": (c_int, [c_vp, c_int, c_i64, c_i64, c_vp, c_vp, c_i64, c_int, c_vp, c_vp, c_size, c_vp]),
     "misa_hier_rerank": (c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_i64, c_vp, c_int,
                                  c_int, c_vp, c_vp, c_vp, c_size, c_vp]),
+    "misa_shard_prefix": (c_int, [c_vp, c_int, c_i64, c_i64, c_vp, c_vp]),
+    "misa_gather_candidates": (c_int, [c_vp, c_int, c_i64, c_i64, c_vp, c_int, c_i64, c_vp, c_vp, c_vp]),
     "misa_sparse_mla": (c_int, [c_vp, c_vp, c_i64, c_i64, c_i64, c_vp, c_int, c_int, c_vp, c_int, c_i64,
                                 ctypes.c_float, c_vp, c_vp, c_vp, c_size, c_vp]),
     "hisa_block_filter": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_i64,
@@ -369,3 +371,27 @@ def sparse_mla(q, kv, seq_of, idx, scale: float, out=None, lse=None, want_lse: b
           _p(idx), k, int(idx.stride(0)), float(scale), _p(out), _p(lse), _p(workspace), workspace.numel(),
           _stream(stream))
     return out, lse
+
+
+def shard_prefix(prefix_len, s0: int, L_shard: int, out=None, stream=None) -> torch.Tensor:
+    """misa_shard_prefix -> [T] int32 prefix lengths local to keys [s0, s0 + L_shard)."""
+    _req(prefix_len, torch.int32, "prefix_len")
+    T = prefix_len.numel()
+    if out is None:
+        out = torch.empty_like(prefix_len)
+    _call("misa_shard_prefix", _p(prefix_len), T, int(s0), int(L_shard), _p(out), _stream(stream))
+    return out
+
+
+def gather_candidates(scores, idx, n: int, id_offset: int, out_scores=None, out_ids=None, stream=None):
+    """misa_gather_candidates -> (scores [T, k] fp32, global ids [T, k] int32) of local picks."""
+    _req(scores, torch.float32, "scores", contiguous=False)
+    _req(idx, torch.int32, "idx")
+    T, k = idx.shape
+    if out_scores is None:
+        out_scores = torch.empty((T, k), dtype=torch.float32, device=idx.device)
+    if out_ids is None:
+        out_ids = torch.empty((T, k), dtype=torch.int32, device=idx.device)
+    _call("misa_gather_candidates", _p(scores), T, int(n), int(scores.stride(0)), _p(idx), k, int(id_offset),
+          _p(out_scores), _p(out_ids), _stream(stream))
+    return out_scores, out_ids

@@ -362,4 +362,21 @@ misa_status misa_sparse_mla(const uint16_t* q, const uint16_t* kv, int64_t nseq,
                                              reinterpret_cast<cudaStream_t>(stream)));
 }
 
+misa_status misa_shard_prefix(const int32_t* prefix_len, int T, int64_t s0, int64_t L_shard, int32_t* out,
+                              misa_stream_t stream) {
+  if (!prefix_len || !out || T < 1 || s0 < 0 || L_shard < 1) return MISA_ERR_INVALID_ARG;
+  if (L_shard >= (static_cast<int64_t>(1) << 31)) return MISA_ERR_UNSUPPORTED;
+  return cuda_status(misa::launch_shard_prefix(prefix_len, T, s0, L_shard, out, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+misa_status misa_gather_candidates(const float* scores, int T, int64_t n, int64_t row_stride, const int32_t* idx,
+                                   int k, int64_t id_offset, float* out_scores, int32_t* out_ids,
+                                   misa_stream_t stream) {
+  if (!scores || !idx || !out_scores || !out_ids || T < 1 || k < 1 || n < 1 || row_stride < n || id_offset < 0)
+    return MISA_ERR_INVALID_ARG;
+  if (id_offset + n >= (static_cast<int64_t>(1) << 31)) return MISA_ERR_UNSUPPORTED;
+  return cuda_status(misa::launch_gather_candidates(scores, T, n, row_stride, idx, k, id_offset, out_scores, out_ids,
+                                                    reinterpret_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

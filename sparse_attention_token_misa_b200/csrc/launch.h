@@ -84,6 +84,13 @@ cudaError_t launch_hisa_block_scores_tc(const uint16_t* q, const float* w, const
                                         int64_t L, int B, float* bscore,
                                         int64_t bs_stride, uint32_t* err, cudaStream_t stream);
 
+// Key-sharded indexer helpers (shard.cu).
+cudaError_t launch_shard_prefix(const int32_t* prefix_len, int T, int64_t s0, int64_t L_shard, int32_t* out,
+                                cudaStream_t stream);
+cudaError_t launch_gather_candidates(const float* scores, int T, int64_t n, int64_t row_stride, const int32_t* idx,
+                                     int k, int64_t id_offset, float* out_scores, int32_t* out_ids,
+                                     cudaStream_t stream);
+
 // Sparse attention over selected tokens (sparse_mla.cu): chunks of 256 index
 // slots per query, partial results in part_o [T][nch][Hq][512] and part_ml
 // [T][nch][Hq][2], merged by a second kernel into out / lse.

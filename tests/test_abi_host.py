@@ -34,7 +34,7 @@ def declared_functions():
 def test_library_loads_and_exports_every_declared_symbol():
     l = pkg.lib()
     names = declared_functions()
-    assert len(names) == 14, names
+    assert len(names) == 16, names
     for n in names:
         assert hasattr(l, n), n
         assert n in nat.SIGNATURES, n
@@ -244,3 +244,18 @@ def mla(q=P, kv=P, nseq=1, stride=0, L=1000, seq_of=P, T=2, Hq=128, idx=P2, k=30
 ])
 def test_sparse_mla_rejects(kw, status):
     assert mla(**kw) == status
+
+
+def test_shard_helpers_reject():
+    l = pkg.lib()
+    assert l.misa_shard_prefix(None, 4, 0, 100, P2, None) == INVALID
+    assert l.misa_shard_prefix(P, 0, 0, 100, P2, None) == INVALID
+    assert l.misa_shard_prefix(P, 4, -1, 100, P2, None) == INVALID
+    assert l.misa_shard_prefix(P, 4, 0, 0, P2, None) == INVALID
+    assert l.misa_shard_prefix(P, 4, 0, 1 << 31, P2, None) == UNSUPPORTED
+    g = l.misa_gather_candidates
+    assert g(None, 2, 100, 100, P, 8, 0, P2, P2, None) == INVALID
+    assert g(P, 2, 100, 99, P, 8, 0, P2, P2, None) == INVALID      # rows shorter than n
+    assert g(P, 2, 100, 100, P, 0, 0, P2, P2, None) == INVALID
+    assert g(P, 2, 100, 100, P, 8, -5, P2, P2, None) == INVALID
+    assert g(P, 2, 100, 100, P, 8, (1 << 31) - 50, P2, P2, None) == UNSUPPORTED
