@@ -79,8 +79,8 @@ class ShardedMisaIndexer:
                  q_block: int = 1, device="cuda"):
         if s0 % B != 0 or not (0 <= s0 < s1 <= L):
             raise ValueError("a shard starts on a block boundary and is non-empty")
-        if H % 4 != 0:
-            raise ValueError("H must be a multiple of 4 (importance rows are top-k rows)")
+        if H % 4 != 0 or k % 4 != 0:
+            raise ValueError("H and k must be multiples of 4 (importance and candidate rows are top-k rows)")
         self.T, self.H, self.h, self.L, self.B, self.k, self.q_block = T, H, h, L, B, k, q_block
         self.s0, self.s1, self.Ls, self.world = s0, s1, s1 - s0, world
         G = (T + q_block - 1) // q_block
@@ -94,9 +94,8 @@ class ShardedMisaIndexer:
         self.local_idx = torch.empty((T, k), dtype=torch.int32, device=device)
         self.cand_scores = torch.empty((T, k), dtype=torch.float32, device=device)
         self.cand_ids = torch.empty((T, k), dtype=torch.int32, device=device)
-        wk = (world * k + 3) // 4 * 4
-        self.all_scores = torch.empty((T, wk), dtype=torch.float32, device=device)
-        self.all_ids = torch.empty((T, wk), dtype=torch.int32, device=device)
+        self.all_scores = torch.empty((T, world * k), dtype=torch.float32, device=device)
+        self.all_ids = torch.empty((T, world * k), dtype=torch.int32, device=device)
         self.idx = torch.empty((T, k), dtype=torch.int32, device=device)
         self.ws_route = nat.alloc_workspace(nat.workspace_bytes(nat.OP_ROUTE_HEADS, T, H, self.Ls, B), device)
         self.ws = nat.alloc_workspace(256, device)
@@ -127,9 +126,11 @@ class ShardedMisaIndexer:
     # -- phase 4 (after the all-gather): top-k over the W*k candidates of each row
     def merge(self, gathered_scores, gathered_ids, stream=None):
         W = gathered_scores.shape[0]
+        if W != self.world:
+            raise ValueError("one candidate list per rank")
         n = W * self.k
-        candidate_rows(gathered_scores, out=self.all_scores[:, :n])
-        candidate_rows(gathered_ids, out=self.all_ids[:, :n])
+        candidate_rows(gathered_scores, out=self.all_scores)
+        candidate_rows(gathered_ids, out=self.all_ids)
         nat.topk(self.all_scores, self.k, n=n, id_map=self.all_ids, idx=self.idx, workspace=self.ws, stream=stream)
         return self.idx
 
