@@ -17,6 +17,11 @@
  *     section 三, Stage 1 and Stage 2.]
  *   - the dense DSA indexer (all H heads score every token) is the same calls
  *     with heads == NULL.  [MISA page, "Problem statement".]
+ * Around the indexer: block statistics kept current as keys are appended
+ * (misa_append_keys); the sparse attention that consumes the k indices
+ * (misa_sparse_mla) [HISA page, sections 二 and 四]; and two small steps of
+ * the key-sharded (context-parallel) indexer (misa_shard_prefix,
+ * misa_gather_candidates).
  *
  * Indexer score (the pages print no formula; this is the library's definition):
  *     S[t, s] = sum over active heads h (ascending id) of w[t, h] * ReLU(q[t, h] . k[s])
@@ -29,13 +34,15 @@
  *        q        [T][H][128]            bf16
  *        w        [T][H]                 fp32
  *        keys     row s of sequence b at keys + b * key_seq_stride + s * 128 (bf16)
- *        means    block j of sequence b at means + b * means_seq_stride + j * 128 (fp32)
+ *        means    block j of sequence b at means + b * means_seq_stride + j * 128 (fp32);
+ *                 its optional bf16 split means_hi / means_lo at the same offsets
  *        seq_of   [T] int32   which sequence (key cache) query t reads
  *        prefix_len [T] int32 query t may see keys 0 <= s < prefix_len[t]
  *  - Every pointer argument is a DEVICE pointer owned by the caller (except
  *    where a comment says "host").  The library allocates no device memory,
  *    keeps no pointer after a call returns and holds no global state apart from
- *    constant tables and the cached address of the driver's tensor-map encoder.
+ *    constant tables, the cached address of the driver's tensor-map encoder and
+ *    the fixed scratch array of misa_route_heads_noalloc.
  *  - Every compute call is asynchronous on `stream` and never synchronises.
  *    Only misa_error_query() synchronises (on the given stream).
  *  - Arguments are checked on the host before anything is launched; a bad
@@ -43,7 +50,7 @@
  *    well-formed request outside what the kernels implement, or
  *    MISA_ERR_WORKSPACE for a workspace smaller than misa_workspace_bytes()).
  *    Such a call has no effect.  A CUDA launch error returns MISA_ERR_CUDA.
- *  - Device-side checks: an out-of-range seq_of[t] or head id, and a pipeline
+ *  - Device-side checks: an out-of-range seq_of[t], head id or token index, and a pipeline
  *    wait that gives up (a bounded wait of about two seconds), are recorded as
  *    bits in the error word at the start of the workspace (MISA_DEVERR_*); the
  *    kernel then skips the affected work and returns.  Read the word with
@@ -54,7 +61,8 @@
  *    entries are valid the row is padded with -1.
  *  - Visibility: key s is visible to query t iff 0 <= s < min(prefix_len[t], L).
  *    A routing decision (and a HISA block score) sees block j iff the whole
- *    block lies inside the prefix: min((j + 1) * B, L) <= prefix_len.
+ *    block lies inside the prefix: min((j + 1) * B, L) <= prefix_len; HISA also
+ *    keeps the one block a prefix cuts (see hisa_block_filter).
  */
 #ifndef MISA_H
 #define MISA_H
