@@ -23,10 +23,12 @@
 //    clusters): each CTA adds its items' contributions in registers, then CTA
 //    0 of the cluster sums the D per-CTA importances in rank order through
 //    distributed shared memory and selects;
-//  * persistent CTAs over all items (large batches): each item stores its H
-//    partial importances; when a CTA finishes its items of a decision it adds
-//    their count to the decision's counter (one atomic per run of items); the
-//    CTA that completes the count sums the decision's partials in item order.
+//  * persistent CTAs over all items (large batches): each epilogue thread adds
+//    its row's contributions over a run (the CTA's consecutive items of one
+//    decision) in a register; at the end of the run the rows of each head are
+//    added once and the run's H partial importances stored; the run's item
+//    count goes to the decision's counter (one atomic per run); the CTA that
+//    completes the count sums the decision's run partials in CTA order.
 // Both orders are fixed, so the result is deterministic.  The top-h are taken
 // by rank (value desc, ties to the lower head id), ids ascending.
 //
@@ -361,6 +363,8 @@ route_tc_kernel(const __grid_constant__ CUtensorMap means_map, const __grid_cons
     float wrow = 0.f;
     int nvis = 0, g = 0;
     int64_t run_items = 0;  // items of decision g done by this CTA since the last counter update
+    int64_t run_first = i0;  // first item of the current run (this CTA's consecutive items of one decision)
+    float racc = 0.f;        // this row's contributions over the run, in item order
     bool skip = false;
     for (int64_t item = i0; item < i1; ++item, ++it) {
       const int pg = static_cast<int>(item / nbt);
@@ -435,23 +439,27 @@ route_tc_kernel(const __grid_constant__ CUtensorMap means_map, const __grid_cons
       } else {
         skip = true;
       }
-      // this item's partial importance of each head: the rows of one head added
-      red[r] = contrib;
+      racc += contrib;
+      ++run_items;
+      // a run ends with this CTA's last item of decision g: only then are the
+      // rows of one head added (shared memory) and the run's partial stored
+      const bool run_ends = (item + 1 == i1) || (static_cast<int>((((item + 1) / nbt) * p.qpm) / p.q_block) != g);
+      if (!run_ends) continue;
+      red[r] = racc;
+      racc = 0.f;
       named_bar_sync(1, kREpiThreads);
-      if (tid < p.H && !skip) {
-        float sum = 0.f;
-        for (int k2 = 0; k2 < p.qpm; ++k2) sum += red[k2 * p.H + tid];
-        if constexpr (kCluster) acc += sum;
-        else p.partial[item * p.H + tid] = sum;
-      }
+      float hsum = 0.f;
+      if (tid < p.H)
+        for (int k2 = 0; k2 < p.qpm; ++k2) hsum += red[k2 * p.H + tid];
       if constexpr (kCluster) {
-        named_bar_sync(1, kREpiThreads);  // red is reused by the next item
+        if (tid < p.H && !skip) acc += hsum;
+        run_items = 0;
+        run_first = item + 1;
+        named_bar_sync(1, kREpiThreads);  // red is reused by the next run
         continue;
       }
-      ++run_items;
-      // last item of decision g in this CTA's range: count them in
-      const bool run_ends = (item + 1 == i1) || (static_cast<int>((((item + 1) / nbt) * p.qpm) / p.q_block) != g);
-      if (run_ends) {
+      if (tid < p.H && !skip) p.partial[run_first * p.H + tid] = hsum;
+      {
         const int first_pg = g * pgs_per_dec;
         const int last_pg = (first_pg + pgs_per_dec < p.n_pg ? first_pg + pgs_per_dec : p.n_pg) - 1;
         const int64_t first_item = static_cast<int64_t>(first_pg) * nbt;
@@ -469,17 +477,24 @@ route_tc_kernel(const __grid_constant__ CUtensorMap means_map, const __grid_cons
         if (flag[0]) {
           __threadfence();
           if (tid < p.H) {
-            float sum = 0.f;
-            for (int64_t x = first_item; x < end_item; ++x) sum += __ldcg(&p.partial[x * p.H + tid]);
+            // the decision's runs in CTA order: one starts at its first item,
+            // the others where the item range of a CTA begins inside it (the
+            // grid never exceeds the item count, so those starts are distinct)
+            float sum = __ldcg(&p.partial[first_item * p.H + tid]);
+            for (int c2 = 1; c2 < static_cast<int>(gridDim.x); ++c2) {
+              const int64_t st = p.n_items * c2 / gridDim.x;
+              if (st > first_item && st < end_item) sum += __ldcg(&p.partial[st * p.H + tid]);
+            }
             imp[tid] = sum;
           }
           named_bar_sync(1, kREpiThreads);
           select_top_h(imp, p.H, p.h, g, p.heads, p.importance, wcnt);
           if (tid == 0) p.counters[g] = 0u;  // ready for the next call
         }
-        run_items = 0;
       }
-      named_bar_sync(1, kREpiThreads);  // red / imp / flag are reused by the next item
+      run_items = 0;
+      run_first = item + 1;
+      named_bar_sync(1, kREpiThreads);  // red / imp / flag are reused by the next run
     }
     if constexpr (kCluster) {
       if (tid < p.H) imp[tid] = acc;
