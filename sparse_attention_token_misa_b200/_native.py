@@ -126,6 +126,23 @@ def _req(t: torch.Tensor, dtype, name: str, contiguous: bool = True):
     return t
 
 
+def _shape(t, name: str, *dims):
+    """Raise unless t has exactly these sizes (None: any).  The library sees
+    only pointers, so a tensor smaller than the call implies must be caught
+    here, before any launch."""
+    if t is None:
+        return
+    if t.dim() != len(dims) or any(d is not None and t.shape[i] != d for i, d in enumerate(dims)):
+        raise ValueError(f"{name}: expected shape {tuple('*' if d is None else d for d in dims)}, "
+                         f"got {tuple(t.shape)}")
+
+
+def _rows(t, name: str, T: int, min_cols: int):
+    """A [T, >= min_cols] matrix with contiguous rows."""
+    if t.dim() != 2 or t.shape[0] != T or t.shape[1] < min_cols or t.stride(1) != 1:
+        raise ValueError(f"{name}: expected [{T}, >= {min_cols}] with contiguous rows, got {tuple(t.shape)}")
+
+
 def workspace_bytes(op: int, T: int, H: int, L: int, B: int, k: int = 0, kp: int = 0) -> int:
     return int(lib().misa_workspace_bytes(op, T, H, L, B, k, kp))
 
@@ -169,10 +186,13 @@ def block_stats(keys: torch.Tensor, B: int, out: torch.Tensor | None = None, str
     """misa_block_stats: keys [nseq, L, 128] bf16 -> means [nseq, M, 128] fp32,
     or (means, means_hi, means_lo) with the bf16 split when split=True."""
     _req(keys, torch.bfloat16, "keys", contiguous=False)
+    _shape(keys, "keys", None, None, HEAD_DIM)
     if keys.stride(2) != 1 or keys.stride(1) != HEAD_DIM:
         raise ValueError("keys rows must be contiguous 128-element rows")
     nseq, L, _ = keys.shape
     M = (L + B - 1) // B
+    _shape(out, "out", nseq, M, HEAD_DIM)
+    _shape(out_hi, "out_hi", nseq, M, HEAD_DIM)
     if out is None:
         out = torch.empty((nseq, M, HEAD_DIM), dtype=torch.float32, device=keys.device)
     if split and out_hi is None:
@@ -198,7 +218,10 @@ def append_keys(keys: torch.Tensor, lens: torch.Tensor, new_keys: torch.Tensor, 
         raise ValueError("keys rows must be contiguous 128-element rows")
     if means.stride(2) != 1 or means.stride(1) != HEAD_DIM:
         raise ValueError("means rows must be contiguous 128-element rows")
+    _shape(keys, "keys", None, None, HEAD_DIM)
     nseq, L_cap, _ = keys.shape
+    _shape(new_keys, "new_keys", nseq, None, HEAD_DIM)
+    _shape(means, "means", nseq, (L_cap + B - 1) // B, HEAD_DIM)
     n_new = new_keys.shape[1]
     if new_keys.shape[0] != nseq or lens.numel() != nseq or means.shape[0] != nseq:
         raise ValueError("keys, lens, new_keys and means must agree on nseq")
@@ -228,8 +251,16 @@ def route_heads(q, w, means, seq_of, prefix_len, L: int, B: int, q_block: int, h
     _req(q, torch.bfloat16, "q"); _req(w, torch.float32, "w")
     nseq, mstride = _means_layout(means, means_hi, means_lo)
     _req(seq_of, torch.int32, "seq_of"); _req(prefix_len, torch.int32, "prefix_len")
+    _shape(q, "q", None, None, HEAD_DIM)
     T, H, _ = q.shape
     G = (T + q_block - 1) // q_block
+    _shape(w, "w", T, H); _shape(seq_of, "seq_of", T); _shape(prefix_len, "prefix_len", T)
+    M = (L + B - 1) // B
+    for name_, m_ in (("means", means), ("means_hi", means_hi)):
+        _shape(m_, name_, nseq, None, HEAD_DIM)
+        if m_ is not None and m_.shape[1] < M:
+            raise ValueError(f"{name_}: fewer than {M} blocks")
+    _shape(heads, "heads", G, h); _shape(importance, "importance", G, H)
     dev = q.device
     if heads is None:
         heads = torch.empty((G, h), dtype=torch.int32, device=dev)
@@ -249,8 +280,14 @@ def route_heads_noalloc(q, w, means, seq_of, prefix_len, L: int, B: int, q_block
     """misa_route_heads_noalloc (no workspace; library-owned fixed scratch)."""
     _req(q, torch.bfloat16, "q"); _req(w, torch.float32, "w"); _req(means, torch.float32, "means")
     _req(seq_of, torch.int32, "seq_of"); _req(prefix_len, torch.int32, "prefix_len")
+    _shape(q, "q", None, None, HEAD_DIM)
     T, H, _ = q.shape
     G = (T + q_block - 1) // q_block
+    _shape(w, "w", T, H); _shape(seq_of, "seq_of", T); _shape(prefix_len, "prefix_len", T)
+    _shape(means, "means", None, None, HEAD_DIM)
+    if means.shape[1] < (L + B - 1) // B:
+        raise ValueError("means: fewer blocks than ceil(L / B)")
+    _shape(heads, "heads", G, h); _shape(importance, "importance", G, H)
     if heads is None:
         heads = torch.empty((G, h), dtype=torch.int32, device=q.device)
     if importance is None and want_importance:
@@ -265,16 +302,22 @@ def index_score(q, w, keys, seq_of, prefix_len, heads=None, h: int | None = None
     """misa_index_score -> scores [T, L] (or [T, n_cand]) fp32."""
     _req(q, torch.bfloat16, "q"); _req(w, torch.float32, "w"); _req(keys, torch.bfloat16, "keys")
     _req(seq_of, torch.int32, "seq_of"); _req(prefix_len, torch.int32, "prefix_len")
+    _shape(q, "q", None, None, HEAD_DIM); _shape(keys, "keys", None, None, HEAD_DIM)
     T, H, _ = q.shape
     L = keys.shape[1]
+    _shape(w, "w", T, H); _shape(seq_of, "seq_of", T); _shape(prefix_len, "prefix_len", T)
     if heads is not None:
         _req(heads, torch.int32, "heads")
         h = heads.shape[1] if h is None else h
+        _shape(heads, "heads", (T + q_block - 1) // q_block, h)
     n_cand = 0
     if cand is not None:
         _req(cand, torch.int32, "cand")
+        _shape(cand, "cand", T, None)
         n_cand = cand.shape[1]
     ncol = n_cand if cand is not None else L
+    if scores is not None:
+        _rows(scores, "scores", T, ncol)
     if scores is None:
         scores = torch.empty((T, ncol), dtype=torch.float32, device=q.device)
     if workspace is None:
@@ -291,6 +334,10 @@ def topk(scores, k: int, n: int | None = None, row_valid=None, id_map=None, idx=
     _req(scores, torch.float32, "scores", contiguous=False)
     T = scores.shape[0]
     n = scores.shape[1] if n is None else n
+    _rows(scores, "scores", T, n)
+    _shape(idx, "idx", T, k)
+    if row_valid is not None:
+        _req(row_valid, torch.int32, "row_valid"); _shape(row_valid, "row_valid", T)
     if idx is None:
         idx = torch.empty((T, k), dtype=torch.int32, device=scores.device)
     if workspace is None:
@@ -298,7 +345,9 @@ def topk(scores, k: int, n: int | None = None, row_valid=None, id_map=None, idx=
     idm_stride = 0
     if id_map is not None:
         _req(id_map, torch.int32, "id_map", contiguous=False)
-        idm_stride = int(id_map.stride(0))
+        if id_map.dim() != 2 or id_map.shape[1] < n or id_map.stride(1) != 1 or id_map.shape[0] not in (1, T):
+            raise ValueError(f"id_map: expected [{T} or 1, >= {n}] with contiguous rows, got {tuple(id_map.shape)}")
+        idm_stride = int(id_map.stride(0)) if id_map.shape[0] == T else 0
     _call("misa_topk", _p(scores), T, n, int(scores.stride(0)), _p(row_valid), _p(id_map), idm_stride, k, _p(idx),
           _p(workspace), workspace.numel(), _stream(stream))
     return idx
@@ -307,10 +356,14 @@ def topk(scores, k: int, n: int | None = None, row_valid=None, id_map=None, idx=
 def hier_rerank(q, w, keys, seq_of, prefix_len, cand, k: int, idx=None, cand_scores=None, want_scores=False,
                 workspace=None, stream=None):
     """misa_hier_rerank -> (idx [T, k], cand_scores [T, kp] or None)."""
+    _req(q, torch.bfloat16, "q"); _req(w, torch.float32, "w"); _req(keys, torch.bfloat16, "keys")
+    _shape(q, "q", None, None, HEAD_DIM); _shape(keys, "keys", None, None, HEAD_DIM)
     T, H, _ = q.shape
     L = keys.shape[1]
-    kp = cand.shape[1]
     _req(cand, torch.int32, "cand")
+    _shape(w, "w", T, H); _shape(cand, "cand", T, None); _shape(seq_of, "seq_of", T)
+    kp = cand.shape[1]
+    _shape(idx, "idx", T, k); _shape(cand_scores, "cand_scores", T, kp)
     if idx is None:
         idx = torch.empty((T, k), dtype=torch.int32, device=q.device)
     if cand_scores is None and want_scores:
@@ -329,8 +382,16 @@ def hisa_block_filter(q, w, means, seq_of, prefix_len, L: int, B: int, m: int, b
     """hisa_block_filter -> (blocks [T, m], cand [T, m*B], block_scores [T, M] or None).
     means may be None when the bf16 split (means_hi, means_lo) is given."""
     nseq, mstride = _means_layout(means, means_hi, means_lo)
+    _req(q, torch.bfloat16, "q"); _req(w, torch.float32, "w")
+    _shape(q, "q", None, None, HEAD_DIM)
     T, H, _ = q.shape
     M = (L + B - 1) // B
+    _shape(w, "w", T, H); _shape(seq_of, "seq_of", T); _shape(prefix_len, "prefix_len", T)
+    for name_, m_ in (("means", means), ("means_hi", means_hi)):
+        _shape(m_, name_, nseq, None, HEAD_DIM)
+        if m_ is not None and m_.shape[1] < M:
+            raise ValueError(f"{name_}: fewer than {M} blocks")
+    _shape(blocks, "blocks", T, m); _shape(cand, "cand", T, m * B); _shape(block_scores, "block_scores", T, M)
     dev = q.device
     if blocks is None:
         blocks = torch.empty((T, m), dtype=torch.int32, device=dev)
@@ -358,9 +419,12 @@ def sparse_mla(q, kv, seq_of, idx, scale: float, out=None, lse=None, want_lse: b
         raise ValueError("kv rows must be contiguous 576-element rows")
     if idx.stride(1) != 1:
         raise ValueError("idx rows must be contiguous")
+    _shape(q, "q", None, None, MLA_DQK); _shape(kv, "kv", None, None, MLA_DQK)
     T, Hq, _ = q.shape
     nseq, L, _ = kv.shape
+    _shape(idx, "idx", T, None); _shape(seq_of, "seq_of", T)
     k = idx.shape[1]
+    _shape(out, "out", T, Hq, MLA_DV); _shape(lse, "lse", T, Hq)
     if out is None:
         out = torch.empty((T, Hq, MLA_DV), dtype=torch.bfloat16, device=q.device)
     if lse is None and want_lse:
@@ -388,6 +452,8 @@ def gather_candidates(scores, idx, n: int, id_offset: int, out_scores=None, out_
     _req(scores, torch.float32, "scores", contiguous=False)
     _req(idx, torch.int32, "idx")
     T, k = idx.shape
+    _rows(scores, "scores", T, n)
+    _shape(out_scores, "out_scores", T, k); _shape(out_ids, "out_ids", T, k)
     if out_scores is None:
         out_scores = torch.empty((T, k), dtype=torch.float32, device=idx.device)
     if out_ids is None:
