@@ -156,6 +156,30 @@ def reduce_max(x: float, dist, device) -> float:
     return float(t.item())
 
 
+def selection_agreement(a, b):
+    """(mean IoU, mean recovery |a & b| / |b|) over the rows of two [T, k]
+    index arrays (-1: empty slot); informational, computed on the host."""
+    a = np.asarray(a.cpu() if hasattr(a, "cpu") else a)
+    b = np.asarray(b.cpu() if hasattr(b, "cpu") else b)
+    ious, recs = [], []
+    for ra, rb in zip(a, b):
+        sa, sb = set(ra[ra >= 0].tolist()), set(rb[rb >= 0].tolist())
+        inter, uni = len(sa & sb), len(sa | sb)
+        ious.append(inter / uni if uni else 1.0)
+        recs.append(inter / len(sb) if sb else 1.0)
+    return float(np.mean(ious)), float(np.mean(recs))
+
+
+def planted_recall(idx, planted):
+    """Fraction of the planted key positions that the indices select."""
+    idx = np.asarray(idx.cpu() if hasattr(idx, "cpu") else idx)
+    planted = np.asarray(planted)
+    if planted.size == 0:
+        return None
+    hits = sum(len(set(planted[t].tolist()) & set(idx[t].tolist())) for t in range(planted.shape[0]))
+    return hits / planted.size
+
+
 def _time_steps(step, steps, flush, stream, marks=None, after=None):
     """Per-step CUDA-event timing with an untimed L2 flush before every step.
     marks: optional list of names; step(ev) records intermediate events.
@@ -313,6 +337,11 @@ def run_cuda(args):
         raise RuntimeError("e2e indices differ from the device-timed step")
     h2d = stage_h.numel()   # q, w, seq_of, prefix_len, each padded to 256 bytes
     d2h = idx_h.numel() * 4
+    # selection agreement with the dense indexer on the same batch (for information)
+    sel_iou, sel_rec = selection_agreement(ix.idx, dense.idx)
+    selection = {"misa8_iou_vs_dense64": sel_iou, "misa8_recovery_of_dense64": sel_rec,
+                 "misa8_planted_recall": planted_recall(ix.idx, wl.planted),
+                 "dense64_planted_recall": planted_recall(dense.idx, wl.planted)}
 
     if dist:
         dist.barrier()
@@ -362,6 +391,7 @@ def run_cuda(args):
                 "how": "q/w/seq_of/prefix_len packed in one pinned host buffer -> device in one copy, MisaIndexer "
                        "step on device views of it, idx -> pinned host; one CUDA graph replay per step",
                 "eager_ms_per_step": e2e_eager_ms},
+        "selection": selection,
         "detail": {"route_ms": parts["route"] / args.steps, "score_ms": score_ms, "topk_ms": parts["topk"] / args.steps,
                    "misa8_ms": ms_step, "misa8_split_ms": split_ms / args.steps,
                    "dense64_ms": dense_one_ms, "dense64_score_ms": dparts["score"] / args.steps,
@@ -470,7 +500,14 @@ def _dagger(misa, dev, stream, flush, steps, timed):
     means = misa.block_stats(keys, wl.B, split=True)
     dg = misa.MisaDaggerIndexer(wl.T, wl.H, wl.h, wl.L, wl.B, wl.kp, wl.k, device=dev)
     ms = timed(lambda evs: dg.run(q, w, keys, means, so, pl))
-    out["glm5_dagger_decode_L65536"] = {"ms_per_step": ms, "pairs_per_s": int(wl.prefix_len.sum()) / (ms * 1e-3)}
+    dx = misa.DenseIndexer(wl.T, wl.H, wl.L, wl.k, device=dev)
+    dx.run(q, w, keys, so, pl)
+    torch.cuda.synchronize()
+    iou, rec = selection_agreement(dg.idx, dx.idx)
+    out["glm5_dagger_decode_L65536"] = {"ms_per_step": ms, "pairs_per_s": int(wl.prefix_len.sum()) / (ms * 1e-3),
+                                        "iou_vs_dense32": iou, "recovery_of_dense32": rec,
+                                        "planted_recall": planted_recall(dg.idx, wl.planted),
+                                        "dense32_planted_recall": planted_recall(dx.idx, wl.planted)}
     return out
 
 
@@ -478,15 +515,20 @@ def _hisa(misa, dev, stream, flush, steps, timed):
     out = {}
     wl = make_workload("hisa_decode_L131072")
     q, w, keys, so, pl = (x.to(dev) for x in (wl.q, wl.w, wl.keys, wl.seq_of, wl.prefix_len))
+    dx = misa.DenseIndexer(wl.T, wl.H, wl.L, wl.k, device=dev)
+    dense_idx = dx.run(q, w, keys, so, pl).clone()
     for B, m in ((128, 64), (64, 128)):
         means = misa.block_stats(keys, B, split=True)
         hx = misa.HisaIndexer(wl.T, wl.H, wl.L, B, m, wl.k, device=dev)
         ms = timed(lambda evs: hx.run(q, w, keys, means, so, pl))
+        iou, rec = selection_agreement(hx.idx, dense_idx)
         out[f"hisa_decode_L131072_B{B}_m{m}"] = {"ms_per_step": ms,
-                                                 "pairs_per_s": int(wl.prefix_len.sum()) / (ms * 1e-3)}
-    dx = misa.DenseIndexer(wl.T, wl.H, wl.L, wl.k, device=dev)
+                                                 "pairs_per_s": int(wl.prefix_len.sum()) / (ms * 1e-3),
+                                                 "iou_vs_dense64": iou, "recovery_of_dense64": rec,
+                                                 "needle_recall": planted_recall(hx.idx, wl.planted)}
     ms = timed(lambda evs: dx.run(q, w, keys, so, pl))
-    out["hisa_decode_L131072_dense64"] = {"ms_per_step": ms, "pairs_per_s": int(wl.prefix_len.sum()) / (ms * 1e-3)}
+    out["hisa_decode_L131072_dense64"] = {"ms_per_step": ms, "pairs_per_s": int(wl.prefix_len.sum()) / (ms * 1e-3),
+                                          "needle_recall": planted_recall(dense_idx, wl.planted)}
     # causal prefill: every query keeps the block its prefix cuts
     wp = make_workload("prefill_L131072")
     q, w, keys, so, pl = (x.to(dev) for x in (wp.q, wp.w, wp.keys, wp.seq_of, wp.prefix_len))

@@ -55,3 +55,16 @@ def test_ranks_get_distinct_batches_of_one_shape():
     assert not torch.equal(b.keys, c.keys)
     assert a.T == 32 and a.L == 32768 and a.H == 64 and a.h == 8 and a.k == 2048
     assert bench.reduce_max(1.5, None, torch.device("cpu")) == 1.5
+
+
+def test_selection_agreement_and_planted_recall():
+    import numpy as np
+
+    import bench
+    a = np.array([[1, 2, 3, -1], [5, 6, 7, 8]])
+    b = np.array([[2, 3, 4, -1], [5, 6, 7, 8]])
+    iou, rec = bench.selection_agreement(a, b)
+    assert abs(iou - (0.5 + 1.0) / 2) < 1e-12          # {2,3} of {1,2,3,4}; identical rows
+    assert abs(rec - (2 / 3 + 1.0) / 2) < 1e-12        # 2 of b's 3 valid ids; all 4
+    assert bench.planted_recall(a, np.array([[3, 9], [8, 5]])) == 3 / 4
+    assert bench.planted_recall(a, np.zeros((2, 0), dtype=np.int64)) is None
