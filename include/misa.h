@@ -349,6 +349,17 @@ MISA_API misa_status hisa_block_filter(const uint16_t* q, const float* w, const 
                               void* workspace, size_t workspace_bytes, misa_stream_t stream);
 
 /*
+ * misa_selftest_wait_timeout -- failure-detection self-test (no counterpart in
+ * the pages).  Launches one CTA that waits, through the bounded wait every
+ * pipeline of the library uses, on an mbarrier that nothing completes.  After
+ * the wait's limit (about two seconds) the kernel records MISA_DEVERR_TIMEOUT
+ * in the workspace error word, writes 0 to the word after it (1 would mean the
+ * wait wrongly succeeded) and returns; the context stays usable.  Read the
+ * outcome with misa_error_query.  workspace: >= 256 bytes, device.
+ */
+MISA_API misa_status misa_selftest_wait_timeout(void* workspace, size_t workspace_bytes, misa_stream_t stream);
+
+/*
  * misa_shard_prefix -- prefix lengths of one key shard (context parallelism).
  *   [MISA page (gist.science), "Methodology: MISA": the head importance sums
  *   over visible blocks and the scores are per token, so a key shard can be

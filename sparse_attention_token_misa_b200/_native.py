@@ -60,6 +60,7 @@ SIGNATURES = {
     "misa_topk": (c_int, [c_vp, c_int, c_i64, c_i64, c_vp, c_vp, c_i64, c_int, c_vp, c_vp, c_size, c_vp]),
     "misa_hier_rerank": (c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_i64, c_vp, c_int,
                                  c_int, c_vp, c_vp, c_vp, c_size, c_vp]),
+    "misa_selftest_wait_timeout": (c_int, [c_vp, c_size, c_vp]),
     "misa_shard_prefix": (c_int, [c_vp, c_int, c_i64, c_i64, c_vp, c_vp]),
     "misa_gather_candidates": (c_int, [c_vp, c_int, c_i64, c_i64, c_vp, c_int, c_i64, c_vp, c_vp, c_vp]),
     "misa_sparse_mla": (c_int, [c_vp, c_vp, c_i64, c_i64, c_i64, c_vp, c_int, c_int, c_vp, c_int, c_i64,
@@ -461,3 +462,9 @@ def gather_candidates(scores, idx, n: int, id_offset: int, out_scores=None, out_
     _call("misa_gather_candidates", _p(scores), T, int(n), int(scores.stride(0)), _p(idx), k, int(id_offset),
           _p(out_scores), _p(out_ids), _stream(stream))
     return out_scores, out_ids
+
+
+def selftest_wait_timeout(workspace: torch.Tensor, stream=None) -> None:
+    """misa_selftest_wait_timeout: a bounded wait on a barrier nothing completes
+    (about two seconds); read the outcome with error_query."""
+    _call("misa_selftest_wait_timeout", _p(workspace), workspace.numel(), _stream(stream))

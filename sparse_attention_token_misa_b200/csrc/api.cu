@@ -379,4 +379,11 @@ misa_status misa_gather_candidates(const float* scores, int T, int64_t n, int64_
                                                     reinterpret_cast<cudaStream_t>(stream)));
 }
 
+misa_status misa_selftest_wait_timeout(void* workspace, size_t workspace_bytes, misa_stream_t stream) {
+  misa_status st = check_ws(workspace, workspace_bytes, kErrBytes);
+  if (st != MISA_OK) return st;
+  uint32_t* err = err_word(workspace);
+  return cuda_status(misa::launch_wait_timeout_selftest(err, err + 1, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

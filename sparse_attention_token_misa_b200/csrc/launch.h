@@ -84,6 +84,9 @@ cudaError_t launch_hisa_block_scores_tc(const uint16_t* q, const float* w, const
                                         int64_t L, int B, float* bscore,
                                         int64_t bs_stride, uint32_t* err, cudaStream_t stream);
 
+// Bounded-wait self-test (selftest.cu): result[0] = 1 if the wait returned true.
+cudaError_t launch_wait_timeout_selftest(uint32_t* err, uint32_t* result, cudaStream_t stream);
+
 // Key-sharded indexer helpers (shard.cu).
 cudaError_t launch_shard_prefix(const int32_t* prefix_len, int T, int64_t s0, int64_t L_shard, int32_t* out,
                                 cudaStream_t stream);

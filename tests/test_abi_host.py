@@ -34,7 +34,7 @@ def declared_functions():
 def test_library_loads_and_exports_every_declared_symbol():
     l = pkg.lib()
     names = declared_functions()
-    assert len(names) == 16, names
+    assert len(names) == 17, names
     for n in names:
         assert hasattr(l, n), n
         assert n in nat.SIGNATURES, n
@@ -259,3 +259,9 @@ def test_shard_helpers_reject():
     assert g(P, 2, 100, 100, P, 0, 0, P2, P2, None) == INVALID
     assert g(P, 2, 100, 100, P, 8, -5, P2, P2, None) == INVALID
     assert g(P, 2, 100, 100, P, 8, (1 << 31) - 50, P2, P2, None) == UNSUPPORTED
+
+
+def test_selftest_needs_a_workspace():
+    l = pkg.lib()
+    assert l.misa_selftest_wait_timeout(None, 256, None) == WORKSPACE
+    assert l.misa_selftest_wait_timeout(P, 255, None) == WORKSPACE
