@@ -115,3 +115,72 @@ def test_shard_comm_gloo():
         # row t: rank 0's k candidates, then rank 1's
         assert rows_s[t] == [float(t * k + i) for i in range(k)] + [float(100 + t * k + i) for i in range(k)]
         assert rows_i[t] == [t * k + i for i in range(k)] + [1000 + t * k + i for i in range(k)]
+
+
+def test_sharded_run_orchestration(monkeypatch):
+    """ShardedMisaIndexer.run on the CPU with the library calls stubbed: the
+    means tuple reaches the router as (means, hi, lo), the importances are
+    all-reduced before the heads are picked, both candidate arrays are gathered
+    and the merge reads the gathered rows."""
+    import sparse_attention_token_misa_b200.sharded as sh
+
+    log = []
+
+    class Nat:
+        OP_ROUTE_HEADS = 1
+
+        def workspace_bytes(self, *a):
+            return 256
+
+        def alloc_workspace(self, n, device=None):
+            return torch.zeros(max(n, 256), dtype=torch.uint8)
+
+        def shard_prefix(self, prefix_len, s0, Ls, out=None, stream=None):
+            log.append(("shard_prefix", s0, Ls))
+            out.copy_((prefix_len - s0).clamp(0, Ls))
+
+        def route_heads(self, q, w, means, seq_of, prefix_len, L, B, q_block, h, heads=None, importance=None,
+                        workspace=None, stream=None, means_hi=None, means_lo=None):
+            log.append(("route", means is not None, means_hi is not None, means_lo is not None, L))
+            importance.fill_(1.0)
+
+        def topk(self, scores, k, n=None, row_valid=None, id_map=None, idx=None, workspace=None, stream=None):
+            log.append(("topk", k, n, id_map is not None, float(scores[0, 0])))
+            idx.copy_(torch.arange(k, dtype=torch.int32).expand_as(idx))
+
+        def index_score(self, *a, **kw):
+            log.append(("score",))
+
+        def gather_candidates(self, scores, idx, n, s0, out_scores=None, out_ids=None, stream=None):
+            log.append(("gather", s0))
+            out_scores.fill_(float(s0))
+            out_ids.copy_(idx + s0)
+
+    class Comm:
+        world = 2
+
+        def all_reduce_sum_(self, t):
+            log.append(("all_reduce", tuple(t.shape)))
+            t.mul_(2)                               # two ranks' equal partials
+            return t
+
+        def all_gather(self, t):
+            log.append(("all_gather", tuple(t.shape)))
+            return torch.stack([t, t + 1])
+
+    monkeypatch.setattr(sh, "nat", Nat())
+    T, H, h, L, B, k = 3, 8, 4, 1000, 128, 8
+    ix = sh.ShardedMisaIndexer(T, H, h, L, B, k, 512, 1000, world=2, device="cpu")
+    q, w = torch.zeros(T, H, 128), torch.zeros(T, H)
+    keys, means = torch.zeros(1, 488, 128), (torch.zeros(1, 4, 128), torch.zeros(1, 4, 128), torch.zeros(1, 4, 128))
+    so, pl = torch.zeros(T, dtype=torch.int32), torch.full((T,), 1000, dtype=torch.int32)
+    idx = ix.run(q, w, keys, means, so, pl, Comm())
+    names = [e[0] for e in log]
+    assert names == ["shard_prefix", "route", "all_reduce", "topk", "score", "topk", "gather", "all_gather",
+                     "all_gather", "topk"]
+    assert log[0] == ("shard_prefix", 512, 488)
+    assert log[1] == ("route", True, True, True, 488)          # the split means reached the router
+    assert log[3][1:3] == (h, H) and log[3][4] == 2.0          # heads picked from the all-reduced sum
+    assert log[-1][1:4] == (k, 2 * k, True)                    # merge over W * k candidates with the id map
+    assert float(ix.all_scores[0, 0]) == 512.0 and float(ix.all_scores[0, k]) == 513.0   # rank 0's, then rank 1's
+    assert idx.shape == (T, k)
