@@ -53,6 +53,53 @@ def _peaks():
     return 6650.0, 1590.0, "fallback"
 
 
+def bench_config(wl, ws_n: int) -> dict:
+    """The `config` object both arms print (identical keys and values)."""
+    return {"workload": WORKLOAD, "queries": wl.T, "L": wl.L, "H": wl.H, "h": wl.h, "B": wl.B, "k": wl.k, "d": 128,
+            "parallelism": f"dp{ws_n} (independent batches)",
+            "l2": "flushed before every timed step (256 MiB write, untimed); K is 268 MB > L2"}
+
+
+def decode_step_bytes(T: int, L: int, H: int, h: int, B: int, k: int) -> int:
+    """Algorithmic HBM bytes of one MISA decode step (router + routed scoring +
+    top-k), each byte the method must move once: the keys, the bf16 hi/lo block
+    means and all heads' query rows the router reads, the head weights, the
+    fp32 score rows written by the scoring and read back by the top-k, the
+    indices written (the routed heads and rows re-read from L2 are not
+    counted)."""
+    M = (L + B - 1) // B
+    return (T * L * 256 + T * M * 128 * 2 * 2 + T * H * 256 + T * H * 4 + 2 * T * L * 4 + T * k * 4)
+
+
+def dagger_step_bytes(T: int, L: int, H: int, B: int, kp: int, k: int) -> int:
+    """MISA-dagger decode step: the routed coarse pass (as decode_step_bytes with
+    k' outputs), the k' candidate ids read back, the gathered candidate key rows,
+    the k' rerank scores written and read, the final indices."""
+    return (decode_step_bytes(T, L, H, 8, B, kp) + T * kp * 4 + T * kp * 256 + 2 * T * kp * 4 + T * k * 4)
+
+
+def hisa_step_bytes(T: int, L: int, H: int, B: int, m: int, k: int) -> int:
+    """HISA decode step: bf16 hi/lo block means and the query rows (block
+    filter), block scores written and read, the candidate list written and read
+    twice (scoring, top-k id map), the candidate key rows, their scores written
+    and read, the indices."""
+    M = (L + B - 1) // B
+    n = m * B
+    return (T * M * 128 * 2 * 2 + T * H * 256 + T * H * 4 + 2 * T * M * 4 + 3 * T * n * 4 + T * n * 256
+            + 2 * T * n * 4 + T * k * 4)
+
+
+def router_flops(wl) -> float:
+    """Tensor-core flops of the router: for every query and every block visible
+    to its routing decision, H dot products of 128 against the block mean's bf16
+    hi and lo halves (2 flops per multiply-add)."""
+    pl = wl.prefix_len.numpy().astype(np.int64)
+    first = pl[(np.arange(wl.T) // wl.q_block) * wl.q_block]
+    M = (wl.L + wl.B - 1) // wl.B
+    vis = np.where(first >= wl.L, M, first // wl.B)
+    return float(vis.sum()) * wl.H * 128 * 2 * 2
+
+
 def _source_hash(paths) -> str:
     h = hashlib.sha256()
     for rel in paths:
@@ -356,6 +403,7 @@ def run_cuda(args):
     score_bytes = T * L * 128 * 2 + T * h * (128 * 2 + 4 + 4) + T * L * 4
     achieved = score_bytes / (score_ms * 1e-3) / 1e9
     traffic = _traffic_for("score_kernel", WORKLOAD)
+    step_bytes = decode_step_bytes(T, L, H, h, B, k)
     value = pairs * ws_n / (ms_step * 1e-3)
     line = {
         "metric": METRIC,
@@ -370,9 +418,7 @@ def run_cuda(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded; shapes of the DeepSeek-V3.2 indexer decode)",
-        "config": {"workload": WORKLOAD, "queries": T, "L": L, "H": H, "h": h, "B": B, "k": k, "d": 128,
-                   "parallelism": f"dp{ws_n} (independent batches)",
-                   "l2": "flushed before every timed step (256 MiB write, untimed); K is 268 MB > L2"},
+        "config": bench_config(wl, ws_n),
         "queries_per_s": T * ws_n / (ms_step * 1e-3),
         # the work actually done: q.k products over the routed heads (MISA-8),
         # and over all heads for the dense indexer on the same batch
@@ -386,6 +432,11 @@ def run_cuda(args):
                      "peak": hbm_gbs, "peak_kind": f"{peak_kind} hbm copy GB/s", "unit": "GB/s",
                      "frac": achieved / hbm_gbs, "traffic": traffic,
                      "algorithmic_bytes_per_launch": score_bytes, "launch_ms": score_ms},
+        "step_roofline": {"bound": "hbm", "what": "whole step (router + scoring + top-k), one graph replay",
+                          "algorithmic_bytes_per_step": step_bytes,
+                          "achieved": step_bytes / (ms_step * 1e-3) / 1e9, "peak": hbm_gbs, "unit": "GB/s",
+                          "frac": step_bytes / (ms_step * 1e-3) / 1e9 / hbm_gbs,
+                          "frac_of_8TBps": step_bytes / (ms_step * 1e-3) / 8e12},
         "e2e": {"value": pairs * ws_n / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                 "how": "q/w/seq_of/prefix_len packed in one pinned host buffer -> device in one copy, MisaIndexer "
@@ -408,6 +459,8 @@ def run_cuda(args):
         del flush_buf
     if ws_n == 1:
         line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_budget)
+        if not args.quick and args.cpu_budget > 0:
+            line["cpu_baseline"]["other_workloads"] = cpu_baselines()
     print(json.dumps(line), flush=True)
 
 
@@ -469,14 +522,56 @@ def _prefill(misa, dev, stream, flush, steps):
         parts["topk"] += inner[2].elapsed_time(inner[3])
 
     ms, _ = _time_steps(lambda evs: g.replay(), steps, flush, stream, after=after)
+    g_step = capture_graph(lambda: ix.run(q, w, keys, means, so, pl))
+    for _ in range(2):
+        g_step.replay()
+    torch.cuda.synchronize()
+    step_ms, _ = _time_steps(lambda evs: g_step.replay(), steps, flush, stream)
+    step_ms /= steps
     score_ms = parts["score"] / steps
+    route_ms = parts["route"] / steps
+    topk_ms = parts["topk"] / steps
     flops = 2.0 * 128 * wl.h * pairs
-    _, tc, kind = _peaks()
-    out["prefill_L131072"] = {"ms_per_step": ms / steps, "pairs_per_s": pairs / (ms / steps * 1e-3),
-                              "route_ms": parts["route"] / steps, "score_ms": score_ms,
-                              "topk_ms": parts["topk"] / steps,
-                              "score_tflops": flops / (score_ms * 1e-3) / 1e12,
-                              "score_frac_of_bf16_peak": flops / (score_ms * 1e-3) / 1e12 / tc}
+    rflops = router_flops(wl)
+    topk_bytes = pairs * 4 + wl.T * wl.k * 4      # the visible scores read once, the indices written
+    hbm, tc, kind = _peaks()
+    misa_idx = ix.idx.clone()
+    del ix, g, g_step
+    torch.cuda.empty_cache()
+
+    # the dense 64-head indexer on the same prefill chunk (every head scores every visible pair)
+    dx = misa.DenseIndexer(wl.T, wl.H, wl.L, wl.k, device=dev)
+    dx.capture(q, w, keys, so, pl)
+    for _ in range(2):
+        dx.g_step.replay()
+    torch.cuda.synchronize()
+    d_ms, dparts = _time_steps(lambda evs: (dx.g_score.replay(), evs[0].record(stream), dx.g_select.replay()),
+                               steps, flush, stream, marks=["score", "topk"])
+    d_one, _ = _time_steps(lambda evs: dx.g_step.replay(), steps, flush, stream)
+    d_one /= steps
+    d_score = dparts["score"] / steps
+    dflops = 2.0 * 128 * wl.H * pairs
+    iou, rec = selection_agreement(misa_idx, dx.idx)
+    del dx
+    torch.cuda.empty_cache()
+    out["prefill_L131072"] = {
+        "ms_per_step": step_ms, "pairs_per_s": pairs / (step_ms * 1e-3),
+        "split_ms": ms / steps, "route_ms": route_ms, "score_ms": score_ms, "topk_ms": topk_ms,
+        "score_tflops": flops / (score_ms * 1e-3) / 1e12,
+        "score_frac_of_bf16_peak": flops / (score_ms * 1e-3) / 1e12 / tc,
+        "route_tflops": rflops / (route_ms * 1e-3) / 1e12,
+        "route_frac_of_bf16_peak": rflops / (route_ms * 1e-3) / 1e12 / tc,
+        "topk_GBps": topk_bytes / (topk_ms * 1e-3) / 1e9,
+        "topk_frac_of_hbm": topk_bytes / (topk_ms * 1e-3) / 1e9 / hbm,
+        "step_frac_of_bf16_peak": (flops + rflops) / (step_ms * 1e-3) / 1e12 / tc,
+        "algorithmic": {"score_flops": flops, "route_flops": rflops, "topk_bytes": topk_bytes,
+                        "peaks": f"{kind}: {hbm} GB/s, {tc} TFLOP/s bf16 (burst)"},
+        "dense64_ms": d_one, "dense64_score_ms": d_score, "dense64_topk_ms": dparts["topk"] / steps,
+        "dense64_score_tflops": dflops / (d_score * 1e-3) / 1e12,
+        "dense64_score_frac_of_bf16_peak": dflops / (d_score * 1e-3) / 1e12 / tc,
+        "dense64_over_misa8": d_one / step_ms,
+        "dense64_score_over_misa8_score": d_score / score_ms,
+        "misa8_iou_vs_dense64": iou, "misa8_recovery_of_dense64": rec}
     return out
 
 
@@ -504,7 +599,12 @@ def _dagger(misa, dev, stream, flush, steps, timed):
     dx.run(q, w, keys, so, pl)
     torch.cuda.synchronize()
     iou, rec = selection_agreement(dg.idx, dx.idx)
+    hbm, _, _ = _peaks()
+    nb = dagger_step_bytes(wl.T, wl.L, wl.H, wl.B, wl.kp, wl.k)
     out["glm5_dagger_decode_L65536"] = {"ms_per_step": ms, "pairs_per_s": int(wl.prefix_len.sum()) / (ms * 1e-3),
+                                        "roofline": {"bound": "hbm", "algorithmic_bytes_per_step": nb,
+                                                     "achieved": nb / (ms * 1e-3) / 1e9, "peak": hbm,
+                                                     "unit": "GB/s", "frac": nb / (ms * 1e-3) / 1e9 / hbm},
                                         "iou_vs_dense32": iou, "recovery_of_dense32": rec,
                                         "planted_recall": planted_recall(dg.idx, wl.planted),
                                         "dense32_planted_recall": planted_recall(dx.idx, wl.planted)}
@@ -522,8 +622,14 @@ def _hisa(misa, dev, stream, flush, steps, timed):
         hx = misa.HisaIndexer(wl.T, wl.H, wl.L, B, m, wl.k, device=dev)
         ms = timed(lambda evs: hx.run(q, w, keys, means, so, pl))
         iou, rec = selection_agreement(hx.idx, dense_idx)
+        hbm, _, _ = _peaks()
+        nb = hisa_step_bytes(wl.T, wl.L, wl.H, B, m, wl.k)
         out[f"hisa_decode_L131072_B{B}_m{m}"] = {"ms_per_step": ms,
                                                  "pairs_per_s": int(wl.prefix_len.sum()) / (ms * 1e-3),
+                                                 "roofline": {"bound": "hbm (latency-dominated)",
+                                                              "algorithmic_bytes_per_step": nb,
+                                                              "achieved": nb / (ms * 1e-3) / 1e9, "peak": hbm,
+                                                              "unit": "GB/s", "frac": nb / (ms * 1e-3) / 1e9 / hbm},
                                                  "iou_vs_dense64": iou, "recovery_of_dense64": rec,
                                                  "needle_recall": planted_recall(hx.idx, wl.planted)}
     ms = timed(lambda evs: dx.run(q, w, keys, so, pl))
@@ -629,7 +735,100 @@ def cpu_baseline(wl, budget_s: float = 15.0, max_queries: int | None = None):
             break
     return {"value": pairs / t_used, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
             "sample": f"{done} queries (cycling over the {wl.T} of {wl.name}; full route+score+top-k each), "
-                      f"{t_used:.1f} s"}
+                      f"{t_used:.1f} s", **_host()}
+
+
+def _cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def _host():
+    return {"cores_used": _blas_threads(), "host_cpus": os.cpu_count(), "cpu_model": _cpu_model(),
+            "note": "numpy fp64; matrix products use the BLAS threads, the rest runs on one core"}
+
+
+def cpu_baselines(budget_s: float = 20.0):
+    """The fp64 oracle on the other workloads, each step of the path timed on
+    the host (the block means, which the GPU path keeps as cache state, are
+    computed before the clock starts): the tiny decode, the GLM-5-shaped
+    MISA-dagger decode and the HISA decode in full, the 128K prefill on a
+    seeded subsample of 8 of its 64 query blocks (the first and the last among
+    them), labelled as such.  Value = indexed pairs / oracle seconds."""
+    import oracle
+
+    out = {}
+
+    def per_query(wl, run_one, label):
+        t_used, pairs, done = 0.0, 0, 0
+        for t in range(wl.T):
+            b = int(wl.seq_of[t])
+            keys = wl.keys[b:b + 1].to(torch.float64).numpy()
+            means = np.stack([oracle.block_means(keys[0], wl.B)])
+            a = dict(q=wl.q[t:t + 1].to(torch.float64).numpy(), w=wl.w[t:t + 1].numpy().astype(np.float64),
+                     keys=keys, seq_of=np.zeros(1, np.int64),
+                     prefix_len=wl.prefix_len[t:t + 1].numpy().astype(np.int64), means=means)
+            t0 = time.perf_counter()
+            run_one(a)
+            t_used += time.perf_counter() - t0
+            pairs += int(wl.prefix_len[t])
+            done += 1
+            if t_used > budget_s:
+                break
+        full = done == wl.T
+        out[wl.name] = {"value": pairs / t_used, "unit": UNIT, "queries": done, "seconds": t_used,
+                        "sample": ("full batch" if full else f"first {done} of {wl.T} queries") + f"; {label}"}
+
+    wl = make_workload("tiny_decode_L4096")
+    k64 = wl.keys.to(torch.float64).numpy()
+    means = np.stack([oracle.block_means(k64[0], wl.B)])
+    t0 = time.perf_counter()
+    oracle.misa_indexer(wl.q.to(torch.float64).numpy(), wl.w.numpy().astype(np.float64), k64,
+                        wl.seq_of.numpy().astype(np.int64), wl.prefix_len.numpy().astype(np.int64), wl.B, 1, wl.h,
+                        wl.k, means=means)
+    dt = time.perf_counter() - t0
+    out[wl.name] = {"value": int(wl.prefix_len.sum()) / dt, "unit": UNIT, "queries": wl.T, "seconds": dt,
+                    "sample": "full batch; MISA route + score + top-k"}
+
+    wl = make_workload("glm5_dagger_decode_L65536")
+    per_query(wl, lambda a: oracle.misa_dagger_indexer(a["q"], a["w"], a["keys"], a["seq_of"], a["prefix_len"],
+                                                       wl.B, 1, wl.h, wl.kp, wl.k, means=a["means"]),
+              "MISA-dagger route + coarse score + top-k' + rerank + top-k")
+    wl = make_workload("hisa_decode_L131072")
+    per_query(wl, lambda a: oracle.hisa_indexer(a["q"], a["w"], a["keys"], a["seq_of"], a["prefix_len"],
+                                                wl.B, wl.m, wl.k, means=a["means"]),
+              "HISA block filter + candidate scoring + top-k (B=128, m=64)")
+
+    wl = make_workload("prefill_L131072")
+    k64 = wl.keys.to(torch.float64).numpy()
+    means = np.stack([oracle.block_means(k64[0], wl.B)])
+    n_blk = wl.T // wl.q_block
+    rng = np.random.default_rng(33)
+    chosen = sorted({0, n_blk - 1} | set(rng.choice(np.arange(1, n_blk - 1), size=6, replace=False).tolist()))
+    t_used, pairs, done = 0.0, 0, []
+    for gblk in chosen:
+        sl = slice(gblk * wl.q_block, (gblk + 1) * wl.q_block)
+        q = wl.q[sl].to(torch.float64).numpy()
+        wv = wl.w[sl].numpy().astype(np.float64)
+        pl = wl.prefix_len[sl].numpy().astype(np.int64)
+        t0 = time.perf_counter()
+        oracle.misa_indexer(q, wv, k64, np.zeros(q.shape[0], np.int64), pl, wl.B, wl.q_block, wl.h, wl.k,
+                            means=means)
+        t_used += time.perf_counter() - t0
+        pairs += int(pl.sum())
+        done.append(gblk)
+        if t_used > budget_s:
+            break
+    out[wl.name] = {"value": pairs / t_used, "unit": UNIT, "queries": len(done) * wl.q_block, "seconds": t_used,
+                    "sample": f"subsample: query blocks {done} of {n_blk} (64 queries each, seed 33; first and "
+                              f"last always included); MISA route + score + top-k; not extrapolated"}
+    return out
 
 
 def run_reference(args):
@@ -649,9 +848,10 @@ def run_reference(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws_n, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": wall / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "queries": wl.T, "L": wl.L, "H": wl.H, "h": wl.h, "B": wl.B, "k": wl.k},
+        "config": bench_config(wl, ws_n),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
-                         "sample": "1 query of the batch per step (route + score + top-k in fp64 numpy)"},
+                         "sample": "1 query of the batch per step (route + score + top-k in fp64 numpy)",
+                         **_host()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)

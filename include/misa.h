@@ -216,7 +216,9 @@ MISA_API misa_status misa_append_keys(uint16_t* keys, int64_t nseq, int64_t key_
  *   heads: [ceil(T/q_block)][h] int32 out.  importance: [ceil(T/q_block)][H]
  *          fp32 out, may be NULL.
  * Limits: 1 <= H <= 128, 1 <= h <= H, 1 <= q_block, T >= 1.
- * workspace: >= misa_workspace_bytes(MISA_OP_ROUTE_HEADS, T, H, L, B, 0, 0).
+ * workspace: >= misa_workspace_bytes(MISA_OP_ROUTE_HEADS, T, H, L, B, 0, 0);
+ *   its contents on entry do not matter (the call clears the scratch it relies
+ *   on with an asynchronous memset on `stream`), apart from the error word.
  */
 MISA_API misa_status misa_route_heads(const uint16_t* q, const float* w, const float* means,
                              const uint16_t* means_hi, const uint16_t* means_lo, int64_t nseq, int64_t means_seq_stride, const int32_t* seq_of,
@@ -248,7 +250,11 @@ MISA_API misa_status misa_route_heads(const uint16_t* q, const float* w, const f
  *    overlap on the GPU (unordered streams) race on it and give wrong results:
  *    order them on one stream or with events.
  *  - There is no device error word: an out-of-range seq_of is clamped to 0
- *    without being reported.
+ *    without being reported, and a pipeline wait that gives up (about two
+ *    seconds, which only a stalled GPU reaches) stops the kernel with the
+ *    affected heads left unwritten, also unreported.
+ *  - The cached address is only valid in the CUDA context it was looked up
+ *    in: do not call this function again after cudaDeviceReset.
  *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
  */
 #define MISA_ROUTE_NOALLOC_SCRATCH_BYTES (2u << 20)

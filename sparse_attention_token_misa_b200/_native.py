@@ -33,6 +33,7 @@ MLA_DQK = 576   # latent KV row: 512 latent + 64 rotary
 MLA_DV = 512    # value part: the first 512 entries of a row
 
 HEAD_DIM = 128
+ROUTE_NOALLOC_SCRATCH_BYTES = 2 << 20  # MISA_ROUTE_NOALLOC_SCRATCH_BYTES
 
 _lib = None
 

@@ -195,6 +195,9 @@ misa_status misa_route_heads(const uint16_t* q, const float* w, const float* mea
   if (means_seq_stride % MISA_HEAD_DIM != 0) return MISA_ERR_INVALID_ARG;  // rows of 128 means for the TMA map
   st = check_ws(workspace, workspace_bytes, misa_workspace_bytes(MISA_OP_ROUTE_HEADS, T, H, L, B, 0, 0));
   if (st != MISA_OK) return st;
+  // The per-decision counters of the persistent path are cleared on the stream
+  // before the kernel (one small memset), so the workspace needs no
+  // initialisation and a call after a wait that gave up starts clean.
   uint8_t* scratch = static_cast<uint8_t*>(workspace) + kErrBytes;
   float* partial = reinterpret_cast<float*>(scratch);
   unsigned* counters = reinterpret_cast<unsigned*>(scratch + misa::router_counters_offset(T, H, L, B));
@@ -202,7 +205,7 @@ misa_status misa_route_heads(const uint16_t* q, const float* w, const float* mea
   return cuda_status(misa::launch_route_heads_tc(q, w, means, means_hi, means_lo, means_seq_stride,
                                                  static_cast<int>(nseq), seq_of,
                                                  prefix_len, T, H, L, B, q_block, h, qpm, heads, importance, partial,
-                                                 counters, false, err_word(workspace),
+                                                 counters, true, err_word(workspace),
                                                  reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -237,6 +237,36 @@ def test_route_heads(T, L, H, h, B, q_block):
     check_bit_exact_topk(heads_g, imp.cpu().numpy(), h, what="heads vs CPU sort of GPU importance")
 
 
+def test_route_heads_workspace_contents_do_not_matter():
+    """The router's workspace may hold anything on entry (a buffer reused from
+    another call, or never initialised): fill it with 0xFF bytes (error word
+    cleared) and route a prefill-shaped batch that takes the persistent path,
+    whose per-decision counters live in the workspace; twice in a row, and
+    equal to the result on a zeroed workspace."""
+    T, L, H, h, B, q_block = 256, 20000, 64, 8, 128, 64
+    wl = make_prefill("rtff", 777, T=T, L=L, H=H, h=h, B=B, k=16, q_block=q_block, n_regions=1, region_len=1024)
+    g, o = to_gpu(wl), to_ora(wl)
+    means = np.stack([oracle.block_means(o["keys"][b], B) for b in range(o["keys"].shape[0])])
+    m_d = dev(torch.from_numpy(means).float())
+    nbytes = misa.workspace_bytes(1, T, H, L, B)
+    ws0 = misa.alloc_workspace(nbytes)
+    ref_heads, ref_imp = misa.route_heads(g["q"], g["w"], m_d, g["seq_of"], g["prefix_len"], L, B, q_block, h,
+                                          workspace=ws0)
+    ws = misa.alloc_workspace(nbytes)
+    ws.fill_(0xFF)
+    misa.error_reset(ws)
+    for _ in range(2):
+        heads, imp = misa.route_heads(g["q"], g["w"], m_d, g["seq_of"], g["prefix_len"], L, B, q_block, h,
+                                      workspace=ws)
+        torch.cuda.synchronize()
+        assert_no_device_error(ws)
+        assert torch.equal(heads, ref_heads)
+        assert torch.equal(imp, ref_imp)
+    heads_ora, imp_ora = oracle.route_heads(o["q"], o["w"], means, o["seq_of"], o["prefix_len"], L, B, q_block, h)
+    for gi in range(heads_ora.shape[0]):
+        check_selection(np_i(heads)[gi], imp_ora[gi], h, what=f"heads g{gi}")
+
+
 # ------------------------------------------------------------------ HISA block filter
 @pytest.mark.parametrize("T,L,B,m", [(4, 5000, 128, 8), (3, 1000, 64, 40), (2, 777, 100, 3), (2, 300, 128, 9)])
 def test_hisa_block_filter(T, L, B, m):
