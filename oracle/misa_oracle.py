@@ -52,6 +52,8 @@ import numpy as np
 
 __all__ = [
     "block_means",
+    "num_windows",
+    "window_stats",
     "visible_blocks",
     "head_block_affinity",
     "route_heads",
@@ -92,15 +94,54 @@ def block_means(keys: np.ndarray, B: int) -> np.ndarray:
     return out
 
 
-def visible_blocks(prefix_len: int, L: int, B: int) -> np.ndarray:
-    """Ids of the blocks a routing decision may look at.
+def num_windows(L: int, B: int, S: int) -> int:
+    """Number of B-token windows that start every S tokens (1 <= S <= B).
+
+    HISA-zh, 七 (局限与未来方向, 潜在改进) names overlapping blocks as a way to
+    soften block-boundary effects; the pages give no layout.  Reading: window j
+    covers tokens [j*S, min(j*S + B, L)); windows are added while the previous
+    one does not reach the end of the cache, so every token is covered and no
+    window lies inside another one's extent: M = 1 + ceil(max(L - B, 0) / S).
+    With S = B this is the plain M = ceil(L / B) blocks.
+    """
+    return 1 + (max(L - B, 0) + S - 1) // S
+
+
+def window_stats(keys: np.ndarray, B: int, S: int | None = None, pool: str = "mean") -> np.ndarray:
+    """Block statistics over windows of B tokens starting every S tokens.
+
+    pool = "mean": the arithmetic mean of the window's keys (MISA-gist,
+    Methodology; HISA-zh, Stage 1: mean pooling).  pool = "max": the
+    coordinate-wise maximum of the window's keys (HISA-zh, 七, 潜在改进: max
+    pooling in place of mean pooling; the plainest reading of max pooling a
+    set of vectors).  S = None means S = B (non-overlapping blocks).  A window
+    cut by the end of the cache pools the tokens it holds.
+
+    keys: [L, d].  Returns [num_windows(L, B, S), d] float64.
+    """
+    L, d = keys.shape
+    S = B if S is None else S
+    M = num_windows(L, B, S)
+    out = np.zeros((M, d), dtype=np.float64)
+    for j in range(M):
+        lo = j * S
+        hi = min(lo + B, L)
+        win = keys[lo:hi]
+        out[j] = win.max(axis=0) if pool == "max" else win.sum(axis=0) / float(hi - lo)
+    return out
+
+
+def visible_blocks(prefix_len: int, L: int, B: int, S: int | None = None) -> np.ndarray:
+    """Ids of the blocks (windows) a routing decision may look at.
 
     Block j is visible iff every token it holds is inside the prefix, i.e.
     min((j + 1) * B, L) <= prefix_len.  At decode prefix_len == L, so every block
-    (the partial last one included) is visible.
+    (the partial last one included) is visible.  With windows every S tokens
+    the same rule holds for window j = [j*S, min(j*S + B, L)).
     """
-    M = (L + B - 1) // B
-    ends = np.minimum((np.arange(M) + 1) * B, L)
+    S = B if S is None else S
+    M = num_windows(L, B, S)
+    ends = np.minimum(np.arange(M) * S + B, L)
     return np.nonzero(ends <= prefix_len)[0]
 
 
@@ -129,7 +170,7 @@ def _top_ids(values: np.ndarray, count: int) -> np.ndarray:
     return np.sort(np.asarray(order[:count], dtype=np.int64))
 
 
-def route_heads(q, w, means, seq_of, prefix_len, L, B, q_block, h):
+def route_heads(q, w, means, seq_of, prefix_len, L, B, q_block, h, S=None):
     """Per-query-block head routing (MISA router).
 
     MISA-gist, Methodology: the router aggregates the per-head block affinities
@@ -139,7 +180,8 @@ def route_heads(q, w, means, seq_of, prefix_len, L, B, q_block, h):
     q: [T, H, d]; w: [T, H]; means: [nseq, M, d]; seq_of, prefix_len: [T].
     Queries [g*q_block, min((g+1)*q_block, T)) share one decision g; block
     visibility follows the first query of the block.  importance[g, h] is the sum
-    over the block's queries and the visible blocks of A[h, j].
+    over the block's queries and the visible blocks of A[h, j].  S: the window
+    stride of the statistics (None: S = B, plain blocks).
     Returns heads [G, min(h, H)] (ascending ids) and importance [G, H].
     """
     T, H, _ = q.shape
@@ -150,7 +192,7 @@ def route_heads(q, w, means, seq_of, prefix_len, L, B, q_block, h):
     for g in range(G):
         t0 = g * q_block
         t1 = min(t0 + q_block, T)
-        vis = visible_blocks(int(prefix_len[t0]), L, B)
+        vis = visible_blocks(int(prefix_len[t0]), L, B, S)
         for t in range(t0, t1):
             A = head_block_affinity(q[t], w[t], means[seq_of[t]][vis])
             importance[g] += A.sum(axis=1)
@@ -261,18 +303,22 @@ def dense_indexer(q, w, keys, seq_of, prefix_len, k):
     return topk_rows(S, k), S
 
 
-def misa_indexer(q, w, keys, seq_of, prefix_len, B, q_block, h, k, means=None):
+def misa_indexer(q, w, keys, seq_of, prefix_len, B, q_block, h, k, means=None, S=None, pool="mean"):
     """MISA: route h of H heads per query block, score with them, top-k.
 
     MISA-gist, Methodology (router, then sparse token scoring of the whole prefix
-    by the h active heads, then top-k on the reduced scores).
+    by the h active heads, then top-k on the reduced scores).  S / pool select
+    the block statistic (window_stats); the defaults are the mean-pooled blocks.
     Returns dict with heads, importance, scores, idx.
     """
     T, H, _ = q.shape
     L = keys.shape[1]
     if means is None:
-        means = np.stack([block_means(keys[b], B) for b in range(keys.shape[0])])
-    heads, imp = route_heads(q, w, means, seq_of, prefix_len, L, B, q_block, h)
+        if S is None and pool == "mean":
+            means = np.stack([block_means(keys[b], B) for b in range(keys.shape[0])])
+        else:
+            means = np.stack([window_stats(keys[b], B, S, pool) for b in range(keys.shape[0])])
+    heads, imp = route_heads(q, w, means, seq_of, prefix_len, L, B, q_block, h, S)
     per_query = np.stack([heads[t // q_block] for t in range(T)])
     S = index_scores(q, w, keys, seq_of, prefix_len, per_query)
     return {"heads": heads, "importance": imp, "scores": S, "idx": topk_rows(S, k)}
@@ -296,7 +342,7 @@ def misa_dagger_indexer(q, w, keys, seq_of, prefix_len, B, q_block, h, kp, k, me
             "cand_scores": S_fine, "idx": idx}
 
 
-def hisa_block_filter(q, w, means, seq_of, prefix_len, L, B, m):
+def hisa_block_filter(q, w, means, seq_of, prefix_len, L, B, m, S=None):
     """HISA Stage 1: score block representatives with all heads, keep top-m.
 
     HISA-zh, Stage 1: the query is scored only against the mean-pooled block
@@ -311,47 +357,61 @@ def hisa_block_filter(q, w, means, seq_of, prefix_len, L, B, m):
     visible block; keeping the query's local block is the plainest causal
     reading.)
 
+    Overlapping windows (S < B, window j = [j*S, min(j*S + B, L)); HISA-zh, 七,
+    潜在改进): the same rules apply per window; every window the prefix cuts is
+    kept; a token that an earlier chosen window already lists is listed once
+    only (its later slot is -1), so the candidate ids stay distinct and
+    ascending.  The chosen windows ascend, so token x of the i-th one is
+    already listed iff x < (start of the (i-1)-th) + B.
+
     Returns blocks [T, m] (ascending, -1 padded), cand [T, m*B] (token ids of the
     chosen blocks in ascending order, -1 where a slot is past the prefix or past
     the cache) and block scores [T, M] (-inf where not visible, +inf for a block
     the prefix cuts).
     """
     T, H, _ = q.shape
-    M = (L + B - 1) // B
+    S = B if S is None else S
+    M = num_windows(L, B, S)
     bs = np.full((T, M), -np.inf, dtype=np.float64)
     blocks = np.full((T, m), -1, dtype=np.int64)
     cand = np.full((T, m * B), -1, dtype=np.int64)
     for t in range(T):
         plen = int(prefix_len[t])
-        vis = visible_blocks(plen, L, B)
+        vis = visible_blocks(plen, L, B, S)
         if vis.size:
             A = head_block_affinity(q[t], w[t], means[seq_of[t]][vis])
             bs[t, vis] = A.sum(axis=0)
-        jp = plen // B  # the block holding token plen, if the prefix cuts it
-        if 0 <= jp < M and jp * B < plen < min((jp + 1) * B, L):
-            bs[t, jp] = np.inf
+        for jp in range(M):  # the blocks holding token plen, if the prefix cuts them
+            if jp * S < plen < min(jp * S + B, L):
+                bs[t, jp] = np.inf
         chosen = topk_ascending(bs[t], m)
         blocks[t] = chosen
         limit = min(int(prefix_len[t]), L)
+        prev_end = -1
         for i, j in enumerate(chosen):
             if j < 0:
                 continue
-            ids = np.arange(j * B, j * B + B)
-            ids[ids >= limit] = -1
+            ids = np.arange(j * S, j * S + B)
+            ids[(ids >= limit) | (ids < prev_end)] = -1
             cand[t, i * B:(i + 1) * B] = ids
+            prev_end = j * S + B
     return blocks, cand, bs
 
 
-def hisa_indexer(q, w, keys, seq_of, prefix_len, B, m, k, means=None):
+def hisa_indexer(q, w, keys, seq_of, prefix_len, B, m, k, means=None, S=None, pool="mean"):
     """HISA: block coarse filter, then all-head token scoring inside, top-k.
 
-    HISA-zh, Stage 1 + Stage 2; cost per query O(L/B + m*B).
+    HISA-zh, Stage 1 + Stage 2; cost per query O(L/B + m*B).  S / pool select
+    the block statistic (window_stats: overlapping windows, max pooling).
     """
     T, H, _ = q.shape
     L = keys.shape[1]
     if means is None:
-        means = np.stack([block_means(keys[b], B) for b in range(keys.shape[0])])
-    blocks, cand, bs = hisa_block_filter(q, w, means, seq_of, prefix_len, L, B, m)
+        if S is None and pool == "mean":
+            means = np.stack([block_means(keys[b], B) for b in range(keys.shape[0])])
+        else:
+            means = np.stack([window_stats(keys[b], B, S, pool) for b in range(keys.shape[0])])
+    blocks, cand, bs = hisa_block_filter(q, w, means, seq_of, prefix_len, L, B, m, S)
     all_heads = np.tile(np.arange(H), (T, 1))
     S = candidate_scores(q, w, keys, seq_of, prefix_len, all_heads, cand)
     idx = topk_rows(S, k, id_map=cand)

@@ -10,7 +10,11 @@ Kinds of pin used here:
 * brute force on tiny inputs (top-k by its rank definition, evaluated pairwise);
 * invariants that follow from the definitions (all heads routed == dense
   indexer; HISA with m*B >= L == dense; hierarchical rerank with k' >= L ==
-  dense).
+  dense; HISA over overlapping windows, all kept, == dense; a max-pooled
+  block score bounds its tokens' scores for nonnegative q and w);
+* the same hand case with max pooling and overlapping windows
+  (tests/golden/hand_case_window_stats.json), and a hand-counted table of
+  window counts, visible and cut windows.
 """
 from __future__ import annotations
 
@@ -20,6 +24,7 @@ import os
 import numpy as np
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "hand_case_2head_8token.json")
+GOLDEN_WIN = os.path.join(os.path.dirname(__file__), "golden", "hand_case_window_stats.json")
 
 
 def hand_case():
@@ -292,6 +297,176 @@ def check_invariant_dagger_full_candidates_is_dense(orc):
         assert np.array_equal(r["idx"], idx_d), seed
 
 
+# ---------------------------------------------------------------- max pooling and overlapping windows
+def _win_golden():
+    with open(GOLDEN_WIN, encoding="utf-8") as f:
+        return json.load(f)
+
+
+def check_hand_max_pool(orc):
+    """HISA-zh, 七 (潜在改进): max pooling instead of mean pooling."""
+    _, q, w, keys = hand_case()
+    g = _win_golden()["max_B4"]
+    st = orc.window_stats(keys[0], 4, None, "max")
+    assert np.array_equal(st, np.asarray(g["block_max"])), st
+    heads, imp = orc.route_heads(q, w, st[None], np.array([0]), np.array([8]), 8, 4, 1, 1)
+    assert np.array_equal(imp[0], np.asarray(g["router_importance"])), imp
+    assert _one(heads) == g["router_heads_h1"]
+    blocks, cand, bs = orc.hisa_block_filter(q, w, st[None], np.array([0]), np.array([8]), 8, 4, 1)
+    assert np.array_equal(bs[0], np.asarray(g["hisa_block_scores"])), bs
+    assert _one(blocks) == g["hisa_m1_blocks"] and _one(cand) == g["hisa_m1_cand"]
+    r = orc.hisa_indexer(q, w, keys, np.array([0]), np.array([8]), 4, 1, 3, pool="max")
+    assert _one(r["idx"]) == g["hisa_m1_top3"], r["idx"]
+
+
+def check_hand_overlap(orc):
+    """HISA-zh, 七 (潜在改进): overlapping blocks; windows of B = 4 every S = 2."""
+    _, q, w, keys = hand_case()
+    g = _win_golden()["overlap_B4_S2"]
+    assert orc.num_windows(8, 4, 2) == g["num_windows"]
+    st = orc.window_stats(keys[0], 4, 2, "mean")
+    assert np.array_equal(st, np.asarray(g["window_means"])), st
+    heads, imp = orc.route_heads(q, w, st[None], np.array([0]), np.array([8]), 8, 4, 1, 1, 2)
+    assert np.array_equal(imp[0], np.asarray(g["router_importance"])), imp
+    assert _one(heads) == g["router_heads_h1"]
+    for m in (1, 2):
+        blocks, cand, bs = orc.hisa_block_filter(q, w, st[None], np.array([0]), np.array([8]), 8, 4, m, 2)
+        assert np.array_equal(bs[0], np.asarray(g["hisa_block_scores"])), bs
+        assert _one(blocks) == g[f"hisa_m{m}_blocks"], blocks
+        assert _one(cand) == g[f"hisa_m{m}_cand"], cand
+    assert _one(orc.hisa_indexer(q, w, keys, np.array([0]), np.array([8]), 4, 1, 3, S=2)["idx"]) == g["hisa_m1_top3"]
+    assert _one(orc.hisa_indexer(q, w, keys, np.array([0]), np.array([8]), 4, 2, 3, S=2)["idx"]) == g["hisa_m2_top3"]
+    assert _one(orc.hisa_indexer(q, w, keys, np.array([0]), np.array([8]), 4, 2, 4, S=2)["idx"]) == g["hisa_m2_top4"]
+
+
+def check_hand_overlap_causal(orc):
+    _, q, w, keys = hand_case()
+    g = _win_golden()["overlap_B4_S2_causal_prefix6"]
+    assert orc.visible_blocks(6, 8, 4, 2).tolist() == g["visible_windows"]
+    st = orc.window_stats(keys[0], 4, 2, "mean")[None]
+    blocks, cand, bs = orc.hisa_block_filter(q, w, st, np.array([0]), np.array([6]), 8, 4, 2, 2)
+    exp_bs = [float(x) for x in g["hisa_block_scores"]]
+    assert bs[0].tolist() == exp_bs, bs
+    assert _one(blocks) == g["hisa_m2_blocks"] and _one(cand) == g["hisa_m2_cand"], (blocks, cand)
+    r = orc.hisa_indexer(q, w, keys, np.array([0]), np.array([6]), 4, 2, 3, S=2)
+    assert _one(r["idx"]) == g["hisa_m2_top3"]
+    _, imp = orc.route_heads(q, w, st, np.array([0]), np.array([6]), 8, 4, 1, 1, 2)
+    assert np.array_equal(imp[0], np.asarray(g["router_importance"])), imp
+
+
+def check_window_counts(orc):
+    """Hand-counted windows: [L, B, S, M, start, end of the last window]."""
+    for L, B, S, M, s0, s1 in _win_golden()["window_counts"]["cases"]:
+        assert orc.num_windows(L, B, S) == M, (L, B, S)
+        keys = np.arange(L, dtype=np.float64)[:, None] * np.ones((1, 2))
+        st = orc.window_stats(keys, B, S, "max")
+        assert st.shape == (M, 2)
+        assert st[-1, 0] == s1 - 1                       # the last window ends at token s1 - 1
+        mean_last = orc.window_stats(keys, B, S, "mean")[-1, 0]
+        assert mean_last == (s0 + s1 - 1) / 2.0          # ... and starts at s0
+    for L in range(1, 40):                                # S = B: the plain blocks
+        assert orc.num_windows(L, 4, 4) == (L + 3) // 4
+
+
+def check_window_closed_forms(orc):
+    rng = np.random.default_rng(17)
+    d = 6
+    v = np.abs(rng.standard_normal(d))          # nonnegative ramp direction
+    c = rng.standard_normal(d)
+    for L, B, S in ((13, 4, 2), (20, 5, 3), (9, 9, 1), (7, 3, 3)):
+        ramp = np.arange(L, dtype=np.float64)[:, None] * v[None]
+        const = np.tile(c, (L, 1))
+        mx, mn = orc.window_stats(ramp, B, S, "max"), orc.window_stats(ramp, B, S, "mean")
+        for j in range(mx.shape[0]):
+            s0, s1 = j * S, min(j * S + B, L)
+            assert np.allclose(mx[j], (s1 - 1) * v, rtol=1e-15, atol=0)          # max of a ramp: its last token
+            assert np.allclose(mn[j], 0.5 * (s0 + s1 - 1) * v, rtol=1e-14, atol=0)  # mean: its midpoint
+        assert np.allclose(orc.window_stats(const, B, S, "max"), c[None], rtol=0, atol=0)
+        assert np.allclose(orc.window_stats(const, B, S, "mean"), c[None], rtol=1e-15, atol=1e-15)
+
+
+def check_window_stats_brute_force(orc):
+    """Each window statistic against a scan that tests every token for
+    membership (j*S <= s < j*S + B, s < L) and pools with scalar loops."""
+    rng = np.random.default_rng(19)
+    for trial in range(12):
+        L = int(rng.integers(1, 30)); B = int(rng.integers(1, 9)); S = int(rng.integers(1, B + 1))
+        keys = rng.standard_normal((L, 3))
+        for pool in ("mean", "max"):
+            st = orc.window_stats(keys, B, S, pool)
+            for j in range(st.shape[0]):
+                members = [s for s in range(L) if j * S <= s < j * S + B]
+                assert members, (trial, j)
+                for c in range(3):
+                    vals = [keys[s, c] for s in members]
+                    ref = max(vals) if pool == "max" else sum(vals) / len(vals)
+                    assert abs(st[j, c] - ref) <= 1e-14 * max(1.0, abs(ref)), (trial, pool, j, c)
+            # every token lies in some window
+            covered = {s for j in range(st.shape[0]) for s in range(L) if j * S <= s < j * S + B}
+            assert covered == set(range(L)), (trial, L, B, S)
+
+
+def check_max_pool_bounds_token_scores(orc):
+    """With nonnegative q and w, a max-pooled block score bounds the dense score
+    of every token of the block from above (q . max_j >= q . k_s, ReLU and the
+    weighted sum are monotone); a mean does not."""
+    rng = np.random.default_rng(23)
+    for seed in range(3):
+        T, H, d, L, B, S = 2, 4, 5, 23, 4, 3
+        q = np.abs(rng.standard_normal((T, H, d)))
+        w = np.abs(rng.standard_normal((T, H)))
+        keys = rng.standard_normal((1, L, d))
+        st = orc.window_stats(keys[0], B, S, "max")[None]
+        _, _, bs = orc.hisa_block_filter(q, w, st, np.zeros(T, np.int64), np.full(T, L), L, B, 1, S)
+        _, Sd = orc.dense_indexer(q, w, keys, np.zeros(T, np.int64), np.full(T, L), 1)
+        for t in range(T):
+            for j in range(bs.shape[1]):
+                toks = np.arange(j * S, min(j * S + B, L))
+                assert np.all(bs[t, j] >= Sd[t, toks] - 1e-12), (seed, t, j)
+
+
+def check_invariant_hisa_overlap_covering_is_dense(orc):
+    """Overlapping windows with every window kept: each visible token is listed
+    once (distinct, ascending candidate ids) and HISA equals the dense indexer,
+    at decode and for causal prefixes that end inside windows."""
+    for seed in range(3):
+        q, w, keys, seq_of, plen = _tiny_problem(seed + 30)
+        L = keys.shape[1]
+        for B, S in ((6, 2), (5, 3), (8, 5)):
+            m = orc.num_windows(L, B, S)
+            for pl in (plen, np.array([7, 20, 33])):
+                idx_d, _ = orc.dense_indexer(q, w, keys, seq_of, pl, 9)
+                r = orc.hisa_indexer(q, w, keys, seq_of, pl, B, m, 9, S=S)
+                assert np.array_equal(r["idx"], idx_d), (seed, B, S)
+                for t in range(q.shape[0]):
+                    ids = r["cand"][t][r["cand"][t] >= 0]
+                    assert np.all(np.diff(ids) > 0), (seed, B, S, t)
+                    assert ids.tolist() == list(range(min(int(pl[t]), L))), (seed, B, S, t)
+
+
+def check_window_visibility_and_cuts(orc):
+    """Hand-derived: for L = 8, B = 4, S = 2 (windows [0,4), [2,6), [4,8)) and
+    L = 11, B = 4, S = 3 (windows [0,4), [3,7), [6,10), [9,11)), which windows a
+    prefix sees whole (finite score) and which it cuts (kept, +inf)."""
+    table = [  # L, B, S, prefix, visible, cut
+        (8, 4, 2, 3, [], [0, 1]), (8, 4, 2, 4, [0], [1]), (8, 4, 2, 5, [0], [1, 2]), (8, 4, 2, 6, [0, 1], [2]),
+        (8, 4, 2, 7, [0, 1], [2]), (8, 4, 2, 8, [0, 1, 2], []),
+        (11, 4, 3, 5, [0], [1]), (11, 4, 3, 7, [0, 1], [2]), (11, 4, 3, 10, [0, 1, 2], [3]),
+        (11, 4, 3, 11, [0, 1, 2, 3], []),
+    ]
+    rng = np.random.default_rng(29)
+    for L, B, S, pl, vis, cut in table:
+        assert orc.visible_blocks(pl, L, B, S).tolist() == vis, (L, B, S, pl)
+        q = np.abs(rng.standard_normal((1, 2, 3)))
+        w = np.abs(rng.standard_normal((1, 2)))
+        keys = rng.standard_normal((1, L, 3))
+        st = orc.window_stats(keys[0], B, S, "mean")[None]
+        _, _, bs = orc.hisa_block_filter(q, w, st, np.array([0]), np.array([pl]), L, B, 1, S)
+        got_vis = [j for j in range(bs.shape[1]) if np.isfinite(bs[0, j])]
+        got_cut = [j for j in range(bs.shape[1]) if bs[0, j] == np.inf]
+        assert got_vis == vis and got_cut == cut, (L, B, S, pl, bs)
+
+
 def check_iou(orc):
     assert orc.iou([1, 2, 3, -1], [2, 3, 4, -1]) == 0.5
     assert orc.iou([5, 6], [6, 5]) == 1.0
@@ -306,4 +481,7 @@ ALL_CHECKS = [
     check_invariant_all_heads_is_dense, check_invariant_hisa_covering_is_dense,
     check_invariant_hisa_causal_covering_is_dense,
     check_invariant_dagger_full_candidates_is_dense, check_iou,
+    check_hand_max_pool, check_hand_overlap, check_hand_overlap_causal, check_window_counts,
+    check_window_closed_forms, check_window_stats_brute_force, check_max_pool_bounds_token_scores,
+    check_invariant_hisa_overlap_covering_is_dense, check_window_visibility_and_cuts,
 ]
