@@ -124,13 +124,14 @@ MISA_API int misa_abi_version(void);
 #define MISA_OP_HISA_BLOCK_FILTER 5
 #define MISA_OP_APPEND_KEYS 6
 #define MISA_OP_SPARSE_MLA 7
+#define MISA_OP_INDEX_DECODE 8
 
 /* Bytes of device workspace the operation needs for these sizes (>= 256: the
  * first 256 bytes hold the device error word).  Arguments an operation does not
  * use are ignored:
  *   ROUTE_HEADS: T, H, L, B;  INDEX_SCORE: none;  TOPK: none;
  *   HIER_RERANK: T, kp;  HISA_BLOCK_FILTER: T, L, B;  APPEND_KEYS: none;
- *   SPARSE_MLA: T, H (= Hq), k.
+ *   SPARSE_MLA: T, H (= Hq), k;  INDEX_DECODE: T, L.
  * Returns 0 for an unknown op or negative sizes. */
 MISA_API size_t misa_workspace_bytes(int op, int T, int H, int64_t L, int B, int k, int kp);
 
@@ -162,6 +163,56 @@ MISA_API misa_status misa_error_query(const void* workspace, misa_stream_t strea
 MISA_API misa_status misa_block_stats(const uint16_t* keys, int64_t nseq, int64_t L, int64_t key_seq_stride,
                              int B, float* means, uint16_t* means_hi, uint16_t* means_lo,
                              misa_stream_t stream);
+
+/*
+ * Block statistics over overlapping windows, and max pooling.
+ *   [HISA page (zhichai.net), section 七 (局限与未来方向), 潜在改进: overlapping
+ *   blocks to soften block-boundary effects, and max pooling in place of mean
+ *   pooling, as ways around the information a block mean loses.  The pages give
+ *   no layout; the library's reading:]
+ * Window j of a cache of L keys covers keys [j*S, min(j*S + B, L)), for a window
+ * length B and a stride 1 <= S <= B; there are
+ *     M = misa_num_windows(L, B, S) = 1 + ceil(max(L - B, 0) / S)
+ * windows, so every key is covered and no window lies inside another one's
+ * extent.  S = B gives the plain blocks (M = ceil(L / B)) of the calls above.
+ * The statistic of a window is the mean of its keys (MISA_POOL_MEAN) or their
+ * coordinate-wise maximum (MISA_POOL_MAX; keys must be finite).  The _ex calls
+ * below take (B, S, pool); the plain calls are the same with S = B and
+ * MISA_POOL_MEAN.  Visibility generalises to windows: a routing decision (and a
+ * HISA window score) sees window j iff min(j*S + B, L) <= prefix_len; HISA keeps
+ * every window the prefix cuts (j*S < prefix_len < min(j*S + B, L)).
+ * Workspace sizes: misa_workspace_bytes with S passed as B is enough for the
+ * windows of stride S (ceil(L / S) >= M).
+ */
+#define MISA_POOL_MEAN 0
+#define MISA_POOL_MAX 1
+
+/* M = 1 + ceil(max(L - B, 0) / S) (host; 0 for L < 1, B < 1, S < 1 or S > B). */
+MISA_API int64_t misa_num_windows(int64_t L, int B, int S);
+
+/*
+ * misa_block_stats_ex -- misa_block_stats over windows of B keys every S keys,
+ * mean or max pooled.  means (and means_hi / means_lo) are [nseq][M][128] with
+ * M = misa_num_windows(L, B, S); the bf16 split of a max is (max, 0) exactly.
+ * Limits as misa_block_stats, and 1 <= S <= B, pool in {MISA_POOL_MEAN,
+ * MISA_POOL_MAX}.
+ */
+MISA_API misa_status misa_block_stats_ex(const uint16_t* keys, int64_t nseq, int64_t L, int64_t key_seq_stride,
+                                         int B, int S, int pool, float* means, uint16_t* means_hi,
+                                         uint16_t* means_lo, misa_stream_t stream);
+
+/*
+ * misa_append_keys_ex -- misa_append_keys for windowed / max-pooled
+ * statistics: every window the new rows [len[b], len[b] + n_new) touch (those
+ * reaching past len[b], up to the last window of the longer cache) is
+ * recomputed over the longer cache, bit for bit what misa_block_stats_ex
+ * computes on it.  means_seq_stride >= misa_num_windows(L_cap, B, S) * 128.
+ */
+MISA_API misa_status misa_append_keys_ex(uint16_t* keys, int64_t nseq, int64_t key_seq_stride, int64_t L_cap,
+                                         const int32_t* len, const uint16_t* new_keys, int n_new, int B, int S,
+                                         int pool, float* means, uint16_t* means_hi, uint16_t* means_lo,
+                                         int64_t means_seq_stride, void* workspace, size_t workspace_bytes,
+                                         misa_stream_t stream);
 
 /*
  * misa_append_keys -- append indexer keys to nseq caches and keep their block
@@ -225,6 +276,21 @@ MISA_API misa_status misa_route_heads(const uint16_t* q, const float* w, const f
                              const int32_t* prefix_len, int T, int H, int64_t L, int B,
                              int q_block, int h, int32_t* heads, float* importance,
                              void* workspace, size_t workspace_bytes, misa_stream_t stream);
+
+/*
+ * misa_route_heads_ex -- misa_route_heads over window statistics of stride S
+ * (means [nseq][M][128], M = misa_num_windows(L, B, S), as misa_block_stats_ex
+ * writes them, mean or max pooled: the router reads whatever statistic it is
+ * given).  Window j is visible iff min(j*S + B, L) <= prefix_len[g*q_block].
+ * 1 <= S <= B.  workspace: >= misa_workspace_bytes(MISA_OP_ROUTE_HEADS, T, H,
+ * L, S, 0, 0).
+ */
+MISA_API misa_status misa_route_heads_ex(const uint16_t* q, const float* w, const float* means,
+                                         const uint16_t* means_hi, const uint16_t* means_lo, int64_t nseq,
+                                         int64_t means_seq_stride, const int32_t* seq_of, const int32_t* prefix_len,
+                                         int T, int H, int64_t L, int B, int S, int q_block, int h, int32_t* heads,
+                                         float* importance, void* workspace, size_t workspace_bytes,
+                                         misa_stream_t stream);
 
 /*
  * misa_route_heads_noalloc -- misa_route_heads without a caller workspace.
@@ -293,6 +359,42 @@ MISA_API misa_status misa_index_score(const uint16_t* q, const float* w, const u
                              void* workspace, size_t workspace_bytes, misa_stream_t stream);
 
 /*
+ * misa_index_decode -- one whole MISA decode step in a single launch: the
+ * router, the routed token scoring and the per-query top-k.
+ *   [MISA page (gist.science), "Methodology: MISA": the router reads the
+ *   mean-pooled block statistics and keeps h of the H heads per query; only
+ *   those heads score every prefix token; the top-k tokens are kept.]
+ * Computes exactly what misa_route_heads (q_block = 1, bf16 split means),
+ * misa_index_score (with those heads) and misa_topk (row_valid = prefix_len)
+ * compute one after the other, with one query per routing decision:
+ *   heads [T][h] out (ascending ids), importance [T][H] out (may be NULL),
+ *   scores [T] rows of L fp32 out (row stride scores_row_stride; -inf past the
+ *     prefix; the top-k reads them back from L2, so they are also an output),
+ *   idx [T][k] out (ascending positions, -1 padded).
+ * The importances are summed in another order than misa_route_heads sums them
+ * (a per-block reduction on the tensor-core accumulator), so they can differ
+ * in the last bits and a head choice can differ where two importances are that
+ * close; given the heads, the scores equal misa_index_score's bit for bit and
+ * idx is the exact top-k of the scores written.
+ * means_hi / means_lo: the bf16 split misa_block_stats writes (block size B,
+ * nmeanseq sequences of ceil(L/B) rows at stride means_seq_stride, a multiple
+ * of 128).  Keys as misa_index_score.
+ * Limits: 1 <= H <= 64, 1 <= h <= 16, h <= H, 1 <= L <= 65536, 1 <= k <=
+ *   MISA_MAX_TOPK; other shapes return MISA_ERR_UNSUPPORTED (use the separate
+ *   calls).  q, keys, means_hi, means_lo, scores 16-byte aligned,
+ *   scores_row_stride >= L and a multiple of 4.
+ * workspace: >= misa_workspace_bytes(MISA_OP_INDEX_DECODE, T, H, L, B, k, 0):
+ *   error word, per-query counters (cleared by the call on `stream`) and
+ *   per-query score histograms; its contents on entry do not matter.
+ */
+MISA_API misa_status misa_index_decode(const uint16_t* q, const float* w, const uint16_t* keys, int64_t nkeyseq,
+                                       int64_t key_seq_stride, const uint16_t* means_hi, const uint16_t* means_lo,
+                                       int64_t nmeanseq, int64_t means_seq_stride, const int32_t* seq_of,
+                                       const int32_t* prefix_len, int T, int H, int64_t L, int B, int h, int k,
+                                       int32_t* heads, float* importance, float* scores, int64_t scores_row_stride,
+                                       int32_t* idx, void* workspace, size_t workspace_bytes, misa_stream_t stream);
+
+/*
  * misa_topk -- per-row top-k of fp32 scores (fused radix select).
  *   [MISA forum thread, "DeepSeek稀疏注意力（DSA）的突破": the indexer keeps the
  *   most relevant token subset; HISA page, section 二: top-k tokens per query;
@@ -353,6 +455,25 @@ MISA_API misa_status hisa_block_filter(const uint16_t* q, const float* w, const 
                               const int32_t* prefix_len, int T, int H, int64_t L, int B, int m,
                               int32_t* blocks, int32_t* cand, float* block_scores,
                               void* workspace, size_t workspace_bytes, misa_stream_t stream);
+
+/*
+ * hisa_block_filter_ex -- hisa_block_filter over window statistics of stride S
+ * (overlapping windows when S < B; mean or max pooled, as misa_block_stats_ex
+ * writes them).  bs[t][j] over the M = misa_num_windows(L, B, S) windows, with
+ * the visibility and cut rules above.  blocks[t][0..m): chosen window ids
+ * ascending, -1 padded.  cand[t][i*B + r] = blocks[t][i]*S + r, or -1 if the
+ * slot is empty, the id is >= min(prefix_len[t], L), or an earlier chosen
+ * window already lists it (id < blocks[t][i-1]*S + B): each token appears at
+ * most once and the listed ids ascend.  block_scores: [T][M] fp32 out, may be
+ * NULL.  1 <= S <= B.
+ * workspace: >= misa_workspace_bytes(MISA_OP_HISA_BLOCK_FILTER, T, H, L, S, m, 0).
+ */
+MISA_API misa_status hisa_block_filter_ex(const uint16_t* q, const float* w, const float* means,
+                                          const uint16_t* means_hi, const uint16_t* means_lo, int64_t nseq,
+                                          int64_t means_seq_stride, const int32_t* seq_of,
+                                          const int32_t* prefix_len, int T, int H, int64_t L, int B, int S, int m,
+                                          int32_t* blocks, int32_t* cand, float* block_scores, void* workspace,
+                                          size_t workspace_bytes, misa_stream_t stream);
 
 /*
  * misa_selftest_wait_timeout -- failure-detection self-test (no counterpart in

@@ -22,6 +22,7 @@ OP_HIER_RERANK = 4
 OP_HISA_BLOCK_FILTER = 5
 OP_APPEND_KEYS = 6
 OP_SPARSE_MLA = 7
+OP_INDEX_DECODE = 8
 
 DEVERR_TIMEOUT = 1
 DEVERR_BAD_SEQ = 2
@@ -33,6 +34,7 @@ MLA_DQK = 576   # latent KV row: 512 latent + 64 rotary
 MLA_DV = 512    # value part: the first 512 entries of a row
 
 HEAD_DIM = 128
+POOL = {"mean": 0, "max": 1}   # MISA_POOL_MEAN, MISA_POOL_MAX
 ROUTE_NOALLOC_SCRATCH_BYTES = 2 << 20  # MISA_ROUTE_NOALLOC_SCRATCH_BYTES
 
 _lib = None
@@ -50,6 +52,14 @@ SIGNATURES = {
     "misa_error_reset": (c_int, [c_vp, c_vp]),
     "misa_error_query": (c_int, [c_vp, c_vp, ctypes.POINTER(ctypes.c_uint32)]),
     "misa_block_stats": (c_int, [c_vp, c_i64, c_i64, c_i64, c_int, c_vp, c_vp, c_vp, c_vp]),
+    "misa_num_windows": (c_i64, [c_i64, c_int, c_int]),
+    "misa_block_stats_ex": (c_int, [c_vp, c_i64, c_i64, c_i64, c_int, c_int, c_int, c_vp, c_vp, c_vp, c_vp]),
+    "misa_append_keys_ex": (c_int, [c_vp, c_i64, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_int, c_int, c_vp, c_vp,
+                                    c_vp, c_i64, c_vp, c_size, c_vp]),
+    "misa_route_heads_ex": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_i64,
+                                    c_int, c_int, c_int, c_int, c_vp, c_vp, c_vp, c_size, c_vp]),
+    "hisa_block_filter_ex": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_i64,
+                                     c_int, c_int, c_int, c_vp, c_vp, c_vp, c_vp, c_size, c_vp]),
     "misa_append_keys": (c_int, [c_vp, c_i64, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_vp, c_vp, c_vp, c_i64,
                                  c_vp, c_size, c_vp]),
     "misa_route_heads": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_i64,
@@ -59,6 +69,9 @@ SIGNATURES = {
     "misa_index_score": (c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_i64, c_vp, c_int,
                                  c_int, c_vp, c_int, c_vp, c_i64, c_vp, c_size, c_vp]),
     "misa_topk": (c_int, [c_vp, c_int, c_i64, c_i64, c_vp, c_vp, c_i64, c_int, c_vp, c_vp, c_size, c_vp]),
+    "misa_index_decode": (c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_int,
+                                  c_int, c_i64, c_int, c_int, c_int, c_vp, c_vp, c_vp, c_i64, c_vp, c_vp, c_size,
+                                  c_vp]),
     "misa_hier_rerank": (c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_i64, c_vp, c_int,
                                  c_int, c_vp, c_vp, c_vp, c_size, c_vp]),
     "misa_selftest_wait_timeout": (c_int, [c_vp, c_size, c_vp]),
@@ -183,16 +196,35 @@ def _split_pair(hi, lo, like: torch.Tensor | None = None):
             raise ValueError("the split must be laid out like the fp32 means")
 
 
+def num_windows(L: int, B: int, stride: int | None = None) -> int:
+    """misa_num_windows: windows of B keys every `stride` keys (None: B) over L keys."""
+    S = B if stride is None else stride
+    M = int(lib().misa_num_windows(L, B, S))
+    if M < 1:
+        raise ValueError(f"bad window geometry L={L} B={B} S={S}")
+    return M
+
+
+def _pool(pool: str) -> int:
+    if pool not in POOL:
+        raise ValueError(f"pool must be one of {tuple(POOL)}")
+    return POOL[pool]
+
+
 def block_stats(keys: torch.Tensor, B: int, out: torch.Tensor | None = None, stream=None, split: bool = False,
-                out_hi: torch.Tensor | None = None, out_lo: torch.Tensor | None = None):
-    """misa_block_stats: keys [nseq, L, 128] bf16 -> means [nseq, M, 128] fp32,
-    or (means, means_hi, means_lo) with the bf16 split when split=True."""
+                out_hi: torch.Tensor | None = None, out_lo: torch.Tensor | None = None,
+                stride: int | None = None, pool: str = "mean"):
+    """misa_block_stats_ex: keys [nseq, L, 128] bf16 -> block statistics
+    [nseq, M, 128] fp32 over windows of B keys every `stride` keys (None: B,
+    plain blocks), mean or max pooled; or (stats, hi, lo) with the bf16 split
+    when split=True."""
     _req(keys, torch.bfloat16, "keys", contiguous=False)
     _shape(keys, "keys", None, None, HEAD_DIM)
     if keys.stride(2) != 1 or keys.stride(1) != HEAD_DIM:
         raise ValueError("keys rows must be contiguous 128-element rows")
     nseq, L, _ = keys.shape
-    M = (L + B - 1) // B
+    S = B if stride is None else stride
+    M = num_windows(L, B, S)
     _shape(out, "out", nseq, M, HEAD_DIM)
     _shape(out_hi, "out_hi", nseq, M, HEAD_DIM)
     if out is None:
@@ -201,17 +233,18 @@ def block_stats(keys: torch.Tensor, B: int, out: torch.Tensor | None = None, str
         out_hi = torch.empty((nseq, M, HEAD_DIM), dtype=torch.bfloat16, device=keys.device)
         out_lo = torch.empty_like(out_hi)
     _split_pair(out_hi, out_lo, out)
-    _call("misa_block_stats", _p(keys), nseq, L, _key_stride(keys) if nseq > 1 else 0, B, _p(out), _p(out_hi),
-          _p(out_lo), _stream(stream))
+    _call("misa_block_stats_ex", _p(keys), nseq, L, _key_stride(keys) if nseq > 1 else 0, B, S, _pool(pool), _p(out),
+          _p(out_hi), _p(out_lo), _stream(stream))
     return (out, out_hi, out_lo) if out_hi is not None else out
 
 
 def append_keys(keys: torch.Tensor, lens: torch.Tensor, new_keys: torch.Tensor, B: int, means: torch.Tensor,
-                workspace: torch.Tensor | None = None, stream=None, means_hi=None, means_lo=None) -> None:
-    """misa_append_keys: new_keys [nseq, n_new, 128] bf16 go to rows
-    [lens[b], lens[b] + n_new) of keys [nseq, L_cap, 128]; means [nseq, M_cap,
-    128] fp32 (and its bf16 split, if given) of the touched blocks are
-    recomputed.  lens is not advanced."""
+                workspace: torch.Tensor | None = None, stream=None, means_hi=None, means_lo=None,
+                stride: int | None = None, pool: str = "mean") -> None:
+    """misa_append_keys_ex: new_keys [nseq, n_new, 128] bf16 go to rows
+    [lens[b], lens[b] + n_new) of keys [nseq, L_cap, 128]; the statistics
+    [nseq, M_cap, 128] fp32 (and their bf16 split, if given) of the touched
+    windows are recomputed.  lens is not advanced."""
     _req(keys, torch.bfloat16, "keys", contiguous=False)
     _req(new_keys, torch.bfloat16, "new_keys")
     _req(lens, torch.int32, "lens")
@@ -223,15 +256,16 @@ def append_keys(keys: torch.Tensor, lens: torch.Tensor, new_keys: torch.Tensor, 
     _shape(keys, "keys", None, None, HEAD_DIM)
     nseq, L_cap, _ = keys.shape
     _shape(new_keys, "new_keys", nseq, None, HEAD_DIM)
-    _shape(means, "means", nseq, (L_cap + B - 1) // B, HEAD_DIM)
+    S = B if stride is None else stride
+    _shape(means, "means", nseq, num_windows(L_cap, B, S), HEAD_DIM)
     n_new = new_keys.shape[1]
     if new_keys.shape[0] != nseq or lens.numel() != nseq or means.shape[0] != nseq:
         raise ValueError("keys, lens, new_keys and means must agree on nseq")
     _split_pair(means_hi, means_lo, means)
     ws = workspace if workspace is not None else alloc_workspace(256, keys.device)
-    _call("misa_append_keys", _p(keys), nseq, int(keys.stride(0)) if nseq > 1 else 0, L_cap, _p(lens),
-          _p(new_keys), n_new, B, _p(means), _p(means_hi), _p(means_lo), int(means.stride(0)), _p(ws), ws.numel(),
-          _stream(stream))
+    _call("misa_append_keys_ex", _p(keys), nseq, int(keys.stride(0)) if nseq > 1 else 0, L_cap, _p(lens),
+          _p(new_keys), n_new, B, S, _pool(pool), _p(means), _p(means_hi), _p(means_lo), int(means.stride(0)),
+          _p(ws), ws.numel(), _stream(stream))
 
 
 def _means_layout(means, means_hi, means_lo):
@@ -247,9 +281,10 @@ def _means_layout(means, means_hi, means_lo):
 
 def route_heads(q, w, means, seq_of, prefix_len, L: int, B: int, q_block: int, h: int,
                 heads=None, importance=None, workspace=None, want_importance: bool = True, stream=None,
-                means_hi=None, means_lo=None):
-    """misa_route_heads -> (heads [G, h] int32, importance [G, H] fp32 or None).
-    means may be None when the bf16 split (means_hi, means_lo) is given."""
+                means_hi=None, means_lo=None, stride: int | None = None):
+    """misa_route_heads_ex -> (heads [G, h] int32, importance [G, H] fp32 or None).
+    means may be None when the bf16 split (means_hi, means_lo) is given;
+    stride: the window stride of the statistics (None: B, plain blocks)."""
     _req(q, torch.bfloat16, "q"); _req(w, torch.float32, "w")
     nseq, mstride = _means_layout(means, means_hi, means_lo)
     _req(seq_of, torch.int32, "seq_of"); _req(prefix_len, torch.int32, "prefix_len")
@@ -257,7 +292,8 @@ def route_heads(q, w, means, seq_of, prefix_len, L: int, B: int, q_block: int, h
     T, H, _ = q.shape
     G = (T + q_block - 1) // q_block
     _shape(w, "w", T, H); _shape(seq_of, "seq_of", T); _shape(prefix_len, "prefix_len", T)
-    M = (L + B - 1) // B
+    S = B if stride is None else stride
+    M = num_windows(L, B, S)
     for name_, m_ in (("means", means), ("means_hi", means_hi)):
         _shape(m_, name_, nseq, None, HEAD_DIM)
         if m_ is not None and m_.shape[1] < M:
@@ -268,11 +304,11 @@ def route_heads(q, w, means, seq_of, prefix_len, L: int, B: int, q_block: int, h
         heads = torch.empty((G, h), dtype=torch.int32, device=dev)
     if importance is None and want_importance:
         importance = torch.empty((G, H), dtype=torch.float32, device=dev)
-    need = workspace_bytes(OP_ROUTE_HEADS, T, H, L, B)
+    need = workspace_bytes(OP_ROUTE_HEADS, T, H, L, S)
     if workspace is None:
         workspace = alloc_workspace(need, dev)
-    _call("misa_route_heads", _p(q), _p(w), _p(means), _p(means_hi), _p(means_lo), nseq, mstride, _p(seq_of),
-          _p(prefix_len), T, H, L, B, q_block, h, _p(heads), _p(importance), _p(workspace),
+    _call("misa_route_heads_ex", _p(q), _p(w), _p(means), _p(means_hi), _p(means_lo), nseq, mstride, _p(seq_of),
+          _p(prefix_len), T, H, L, B, S, q_block, h, _p(heads), _p(importance), _p(workspace),
           workspace.numel(), _stream(stream))
     return heads, importance
 
@@ -330,6 +366,44 @@ def index_score(q, w, keys, seq_of, prefix_len, heads=None, h: int | None = None
     return scores
 
 
+def index_decode(q, w, keys, means_hi, means_lo, seq_of, prefix_len, B: int, h: int, k: int, heads=None,
+                 importance=None, scores=None, idx=None, workspace=None, want_importance: bool = True, stream=None):
+    """misa_index_decode: router + routed scoring + top-k in one launch ->
+    (heads [T, h], importance [T, H] or None, scores [T, >= L], idx [T, k])."""
+    _req(q, torch.bfloat16, "q"); _req(w, torch.float32, "w"); _req(keys, torch.bfloat16, "keys")
+    _req(seq_of, torch.int32, "seq_of"); _req(prefix_len, torch.int32, "prefix_len")
+    _shape(q, "q", None, None, HEAD_DIM); _shape(keys, "keys", None, None, HEAD_DIM)
+    T, H, _ = q.shape
+    L = keys.shape[1]
+    M = (L + B - 1) // B
+    _shape(w, "w", T, H); _shape(seq_of, "seq_of", T); _shape(prefix_len, "prefix_len", T)
+    _split_pair(means_hi, means_lo)
+    if means_hi is None:
+        raise ValueError("misa_index_decode reads the bf16 split of the block means")
+    _shape(means_hi, "means_hi", None, None, HEAD_DIM)
+    if means_hi.shape[1] < M or means_lo.shape != means_hi.shape:
+        raise ValueError(f"means_hi / means_lo: expected [nseq, >= {M}, 128]")
+    _shape(heads, "heads", T, h); _shape(importance, "importance", T, H); _shape(idx, "idx", T, k)
+    dev = q.device
+    if heads is None:
+        heads = torch.empty((T, h), dtype=torch.int32, device=dev)
+    if importance is None and want_importance:
+        importance = torch.empty((T, H), dtype=torch.float32, device=dev)
+    if scores is None:
+        scores = torch.empty((T, (L + 3) // 4 * 4), dtype=torch.float32, device=dev)
+    _rows(scores, "scores", T, L)
+    if idx is None:
+        idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    need = workspace_bytes(OP_INDEX_DECODE, T, H, L, B, k)
+    if workspace is None:
+        workspace = alloc_workspace(need, dev)
+    _call("misa_index_decode", _p(q), _p(w), _p(keys), keys.shape[0], _key_stride(keys), _p(means_hi),
+          _p(means_lo), means_hi.shape[0], int(means_hi.stride(0)) if means_hi.shape[0] > 1 else 0, _p(seq_of),
+          _p(prefix_len), T, H, L, B, h, k, _p(heads), _p(importance), _p(scores), int(scores.stride(0)), _p(idx),
+          _p(workspace), workspace.numel(), _stream(stream))
+    return heads, importance, scores, idx
+
+
 def topk(scores, k: int, n: int | None = None, row_valid=None, id_map=None, idx=None, workspace=None,
          stream=None) -> torch.Tensor:
     """misa_topk -> idx [T, k] int32 (ascending positions / ids, -1 padded)."""
@@ -380,14 +454,16 @@ def hier_rerank(q, w, keys, seq_of, prefix_len, cand, k: int, idx=None, cand_sco
 
 def hisa_block_filter(q, w, means, seq_of, prefix_len, L: int, B: int, m: int, blocks=None, cand=None,
                       block_scores=None, want_scores=False, workspace=None, stream=None, means_hi=None,
-                      means_lo=None):
-    """hisa_block_filter -> (blocks [T, m], cand [T, m*B], block_scores [T, M] or None).
-    means may be None when the bf16 split (means_hi, means_lo) is given."""
+                      means_lo=None, stride: int | None = None):
+    """hisa_block_filter_ex -> (blocks [T, m], cand [T, m*B], block_scores [T, M] or None).
+    means may be None when the bf16 split (means_hi, means_lo) is given;
+    stride: the window stride of the statistics (None: B, plain blocks)."""
     nseq, mstride = _means_layout(means, means_hi, means_lo)
     _req(q, torch.bfloat16, "q"); _req(w, torch.float32, "w")
     _shape(q, "q", None, None, HEAD_DIM)
     T, H, _ = q.shape
-    M = (L + B - 1) // B
+    S = B if stride is None else stride
+    M = num_windows(L, B, S)
     _shape(w, "w", T, H); _shape(seq_of, "seq_of", T); _shape(prefix_len, "prefix_len", T)
     for name_, m_ in (("means", means), ("means_hi", means_hi)):
         _shape(m_, name_, nseq, None, HEAD_DIM)
@@ -402,10 +478,10 @@ def hisa_block_filter(q, w, means, seq_of, prefix_len, L: int, B: int, m: int, b
     if block_scores is None and want_scores:
         block_scores = torch.empty((T, M), dtype=torch.float32, device=dev)
     if workspace is None:
-        workspace = alloc_workspace(workspace_bytes(OP_HISA_BLOCK_FILTER, T, H, L, B, m), dev)
-    _call("hisa_block_filter", _p(q), _p(w), _p(means), _p(means_hi), _p(means_lo), nseq, mstride, _p(seq_of),
-          _p(prefix_len), T, H, L, B, m, _p(blocks), _p(cand), _p(block_scores), _p(workspace), workspace.numel(),
-          _stream(stream))
+        workspace = alloc_workspace(workspace_bytes(OP_HISA_BLOCK_FILTER, T, H, L, S, m), dev)
+    _call("hisa_block_filter_ex", _p(q), _p(w), _p(means), _p(means_hi), _p(means_lo), nseq, mstride, _p(seq_of),
+          _p(prefix_len), T, H, L, B, S, m, _p(blocks), _p(cand), _p(block_scores), _p(workspace),
+          workspace.numel(), _stream(stream))
     return blocks, cand, block_scores
 
 

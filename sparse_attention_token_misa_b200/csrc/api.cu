@@ -79,14 +79,14 @@ bool split_ok(const uint16_t* hi, const uint16_t* lo) {
 
 misa_status check_block_args(const uint16_t* q, const float* w, const float* means, const uint16_t* means_hi,
                              const uint16_t* means_lo, int64_t nseq, int64_t means_seq_stride, const int32_t* seq_of,
-                             const int32_t* prefix_len, int T, int H, int64_t L, int B) {
+                             const int32_t* prefix_len, int T, int H, int64_t L, int B, int S) {
   if (!q || !w || !seq_of || !prefix_len || !split_ok(means_hi, means_lo)) return MISA_ERR_INVALID_ARG;
   if (!means && !means_hi) return MISA_ERR_INVALID_ARG;
-  if (T < 1 || H < 1 || L < 1 || B < 1 || nseq < 1) return MISA_ERR_INVALID_ARG;
+  if (T < 1 || H < 1 || L < 1 || B < 1 || nseq < 1 || S < 1 || S > B) return MISA_ERR_INVALID_ARG;
   if (H > MISA_MAX_HEADS) return MISA_ERR_UNSUPPORTED;
   if (!aligned16(q) || (means && !aligned16(means)) || means_seq_stride < 0 || means_seq_stride % 4 != 0)
     return MISA_ERR_INVALID_ARG;
-  const int64_t M = ceil_div(L, B);
+  const int64_t M = misa::num_windows(L, B, S);
   if (nseq > 1 && means_seq_stride < M * MISA_HEAD_DIM) return MISA_ERR_INVALID_ARG;
   if (M >= (static_cast<int64_t>(1) << 24) || nseq >= (static_cast<int64_t>(1) << 31)) return MISA_ERR_UNSUPPORTED;
   return MISA_OK;
@@ -131,6 +131,12 @@ size_t misa_workspace_bytes(int op, int T, int H, int64_t L, int B, int k, int k
       const int64_t M = ceil_div(L, B);
       return kErrBytes + static_cast<size_t>(T) * round_up4(M) * sizeof(float);
     }
+    case MISA_OP_INDEX_DECODE: {
+      if (T < 1 || L < 1) return 0;
+      const size_t counters = (static_cast<size_t>(T) * 4 + 255) / 256 * 256;
+      const int64_t R = misa::decode_fused_hist_slots(T, L, misa::kDecodeFusedMaxGrid);
+      return kErrBytes + counters + static_cast<size_t>(T) * R * misa::decode_fused_hist_bins() * 4;
+    }
     default:
       return 0;
   }
@@ -152,61 +158,92 @@ misa_status misa_error_query(const void* workspace, misa_stream_t stream, uint32
   return v == 0 ? MISA_OK : MISA_ERR_DEVICE;
 }
 
-misa_status misa_block_stats(const uint16_t* keys, int64_t nseq, int64_t L, int64_t key_seq_stride, int B,
-                             float* means, uint16_t* means_hi, uint16_t* means_lo, misa_stream_t stream) {
+int64_t misa_num_windows(int64_t L, int B, int S) {
+  if (L < 1 || B < 1 || S < 1 || S > B) return 0;
+  return misa::num_windows(L, B, S);
+}
+
+misa_status misa_block_stats_ex(const uint16_t* keys, int64_t nseq, int64_t L, int64_t key_seq_stride, int B, int S,
+                                int pool, float* means, uint16_t* means_hi, uint16_t* means_lo,
+                                misa_stream_t stream) {
   if (!keys || !means || nseq < 1 || L < 1 || B < 1 || !split_ok(means_hi, means_lo)) return MISA_ERR_INVALID_ARG;
+  if (S < 1 || S > B || (pool != MISA_POOL_MEAN && pool != MISA_POOL_MAX)) return MISA_ERR_INVALID_ARG;
   if (B > 4096) return MISA_ERR_UNSUPPORTED;
   if (!aligned16(keys) || !aligned16(means) || key_seq_stride < 0 || key_seq_stride % 8 != 0)
     return MISA_ERR_INVALID_ARG;
   if (nseq > 1 && key_seq_stride < L * MISA_HEAD_DIM) return MISA_ERR_INVALID_ARG;
-  return cuda_status(misa::launch_block_stats(keys, nseq, L, key_seq_stride, B, means, means_hi, means_lo,
-                                              reinterpret_cast<cudaStream_t>(stream)));
+  return cuda_status(misa::launch_block_stats(keys, nseq, L, key_seq_stride, B, S, pool == MISA_POOL_MAX, means,
+                                              means_hi, means_lo, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+misa_status misa_block_stats(const uint16_t* keys, int64_t nseq, int64_t L, int64_t key_seq_stride, int B,
+                             float* means, uint16_t* means_hi, uint16_t* means_lo, misa_stream_t stream) {
+  return misa_block_stats_ex(keys, nseq, L, key_seq_stride, B, B, MISA_POOL_MEAN, means, means_hi, means_lo, stream);
+}
+
+misa_status misa_append_keys_ex(uint16_t* keys, int64_t nseq, int64_t key_seq_stride, int64_t L_cap,
+                                const int32_t* len, const uint16_t* new_keys, int n_new, int B, int S, int pool,
+                                float* means, uint16_t* means_hi, uint16_t* means_lo, int64_t means_seq_stride,
+                                void* workspace, size_t workspace_bytes, misa_stream_t stream) {
+  if (!keys || !len || !new_keys || !means || nseq < 1 || L_cap < 1 || n_new < 1 || B < 1 ||
+      !split_ok(means_hi, means_lo))
+    return MISA_ERR_INVALID_ARG;
+  if (S < 1 || S > B || (pool != MISA_POOL_MEAN && pool != MISA_POOL_MAX)) return MISA_ERR_INVALID_ARG;
+  if (B > 4096) return MISA_ERR_UNSUPPORTED;
+  if (!aligned16(keys) || !aligned16(new_keys) || !aligned16(means) || key_seq_stride < 0 || key_seq_stride % 8 != 0)
+    return MISA_ERR_INVALID_ARG;
+  if (nseq > 1 && key_seq_stride < L_cap * MISA_HEAD_DIM) return MISA_ERR_INVALID_ARG;
+  const int64_t M_cap = misa::num_windows(L_cap, B, S);
+  if (means_seq_stride % MISA_HEAD_DIM != 0 || (nseq > 1 && means_seq_stride < M_cap * MISA_HEAD_DIM))
+    return MISA_ERR_INVALID_ARG;
+  misa_status st = check_ws(workspace, workspace_bytes, kErrBytes);
+  if (st != MISA_OK) return st;
+  return cuda_status(misa::launch_append_keys(keys, nseq, key_seq_stride, L_cap, len, new_keys, n_new, B, S,
+                                              pool == MISA_POOL_MAX, means, means_hi, means_lo, means_seq_stride,
+                                              err_word(workspace), reinterpret_cast<cudaStream_t>(stream)));
 }
 
 misa_status misa_append_keys(uint16_t* keys, int64_t nseq, int64_t key_seq_stride, int64_t L_cap, const int32_t* len,
                              const uint16_t* new_keys, int n_new, int B, float* means, uint16_t* means_hi,
                              uint16_t* means_lo, int64_t means_seq_stride, void* workspace, size_t workspace_bytes,
                              misa_stream_t stream) {
-  if (!keys || !len || !new_keys || !means || nseq < 1 || L_cap < 1 || n_new < 1 || B < 1 ||
-      !split_ok(means_hi, means_lo))
-    return MISA_ERR_INVALID_ARG;
-  if (B > 4096) return MISA_ERR_UNSUPPORTED;
-  if (!aligned16(keys) || !aligned16(new_keys) || !aligned16(means) || key_seq_stride < 0 || key_seq_stride % 8 != 0)
-    return MISA_ERR_INVALID_ARG;
-  if (nseq > 1 && key_seq_stride < L_cap * MISA_HEAD_DIM) return MISA_ERR_INVALID_ARG;
-  const int64_t M_cap = ceil_div(L_cap, B);
-  if (means_seq_stride % MISA_HEAD_DIM != 0 || (nseq > 1 && means_seq_stride < M_cap * MISA_HEAD_DIM))
-    return MISA_ERR_INVALID_ARG;
-  misa_status st = check_ws(workspace, workspace_bytes, kErrBytes);
-  if (st != MISA_OK) return st;
-  return cuda_status(misa::launch_append_keys(keys, nseq, key_seq_stride, L_cap, len, new_keys, n_new, B, means,
-                                              means_hi, means_lo, means_seq_stride, err_word(workspace),
-                                              reinterpret_cast<cudaStream_t>(stream)));
+  return misa_append_keys_ex(keys, nseq, key_seq_stride, L_cap, len, new_keys, n_new, B, B, MISA_POOL_MEAN, means,
+                             means_hi, means_lo, means_seq_stride, workspace, workspace_bytes, stream);
 }
 
-misa_status misa_route_heads(const uint16_t* q, const float* w, const float* means, const uint16_t* means_hi,
-                             const uint16_t* means_lo, int64_t nseq, int64_t means_seq_stride, const int32_t* seq_of, const int32_t* prefix_len, int T, int H,
-                             int64_t L, int B, int q_block, int h, int32_t* heads, float* importance, void* workspace,
-                             size_t workspace_bytes, misa_stream_t stream) {
+misa_status misa_route_heads_ex(const uint16_t* q, const float* w, const float* means, const uint16_t* means_hi,
+                                const uint16_t* means_lo, int64_t nseq, int64_t means_seq_stride,
+                                const int32_t* seq_of, const int32_t* prefix_len, int T, int H, int64_t L, int B,
+                                int S, int q_block, int h, int32_t* heads, float* importance, void* workspace,
+                                size_t workspace_bytes, misa_stream_t stream) {
   misa_status st =
-      check_block_args(q, w, means, means_hi, means_lo, nseq, means_seq_stride, seq_of, prefix_len, T, H, L, B);
+      check_block_args(q, w, means, means_hi, means_lo, nseq, means_seq_stride, seq_of, prefix_len, T, H, L, B, S);
   if (st != MISA_OK) return st;
   if (!heads || q_block < 1 || h < 1 || h > H) return MISA_ERR_INVALID_ARG;
   if (means_seq_stride % MISA_HEAD_DIM != 0) return MISA_ERR_INVALID_ARG;  // rows of 128 means for the TMA map
-  st = check_ws(workspace, workspace_bytes, misa_workspace_bytes(MISA_OP_ROUTE_HEADS, T, H, L, B, 0, 0));
+  const int64_t M = misa::num_windows(L, B, S);
+  st = check_ws(workspace, workspace_bytes, kErrBytes + misa::router_scratch_bytes_m(T, H, M, 1));
   if (st != MISA_OK) return st;
   // The per-decision counters of the persistent path are cleared on the stream
   // before the kernel (one small memset), so the workspace needs no
   // initialisation and a call after a wait that gave up starts clean.
   uint8_t* scratch = static_cast<uint8_t*>(workspace) + kErrBytes;
   float* partial = reinterpret_cast<float*>(scratch);
-  unsigned* counters = reinterpret_cast<unsigned*>(scratch + misa::router_counters_offset(T, H, L, B));
+  unsigned* counters = reinterpret_cast<unsigned*>(scratch + misa::router_counters_offset_m(T, H, M));
   const int qpm = misa::route_tc_queries_per_group(H, q_block, nseq == 1 || means_seq_stride == 0);
   return cuda_status(misa::launch_route_heads_tc(q, w, means, means_hi, means_lo, means_seq_stride,
-                                                 static_cast<int>(nseq), seq_of,
-                                                 prefix_len, T, H, L, B, q_block, h, qpm, heads, importance, partial,
-                                                 counters, true, err_word(workspace),
-                                                 reinterpret_cast<cudaStream_t>(stream)));
+                                                 static_cast<int>(nseq), seq_of, prefix_len, T, H, L, B, S, q_block, h,
+                                                 qpm, heads, importance, partial, counters, true,
+                                                 err_word(workspace), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+misa_status misa_route_heads(const uint16_t* q, const float* w, const float* means, const uint16_t* means_hi,
+                             const uint16_t* means_lo, int64_t nseq, int64_t means_seq_stride, const int32_t* seq_of,
+                             const int32_t* prefix_len, int T, int H, int64_t L, int B, int q_block, int h,
+                             int32_t* heads, float* importance, void* workspace, size_t workspace_bytes,
+                             misa_stream_t stream) {
+  return misa_route_heads_ex(q, w, means, means_hi, means_lo, nseq, means_seq_stride, seq_of, prefix_len, T, H, L, B,
+                             B, q_block, h, heads, importance, workspace, workspace_bytes, stream);
 }
 
 misa_status misa_index_score(const uint16_t* q, const float* w, const uint16_t* keys, int64_t nkeyseq,
@@ -260,6 +297,63 @@ misa_status misa_topk(const float* scores, int T, int64_t n, int64_t row_stride,
                                        reinterpret_cast<cudaStream_t>(stream)));
 }
 
+misa_status misa_index_decode(const uint16_t* q, const float* w, const uint16_t* keys, int64_t nkeyseq,
+                              int64_t key_seq_stride, const uint16_t* means_hi, const uint16_t* means_lo,
+                              int64_t nmeanseq, int64_t means_seq_stride, const int32_t* seq_of,
+                              const int32_t* prefix_len, int T, int H, int64_t L, int B, int h, int k, int32_t* heads,
+                              float* importance, float* scores, int64_t scores_row_stride, int32_t* idx,
+                              void* workspace, size_t workspace_bytes, misa_stream_t stream) {
+  if (!q || !w || !keys || !means_hi || !means_lo || !seq_of || !prefix_len || !heads || !scores || !idx)
+    return MISA_ERR_INVALID_ARG;
+  if (T < 1 || H < 1 || L < 1 || B < 1 || h < 1 || h > H || k < 1 || nkeyseq < 1 || nmeanseq < 1)
+    return MISA_ERR_INVALID_ARG;
+  if (!misa::decode_fused_supported(T, H, h, L, k) || T > MISA_MAX_TOPK_ROWS) return MISA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(keys) || !aligned16(means_hi) || !aligned16(means_lo) || !aligned16(scores))
+    return MISA_ERR_INVALID_ARG;
+  if (key_seq_stride < 0 || key_seq_stride % MISA_HEAD_DIM != 0 || (nkeyseq > 1 && key_seq_stride < L * MISA_HEAD_DIM))
+    return MISA_ERR_INVALID_ARG;
+  const int64_t M = ceil_div(L, B);
+  if (means_seq_stride < 0 || means_seq_stride % MISA_HEAD_DIM != 0 ||
+      (nmeanseq > 1 && means_seq_stride < M * MISA_HEAD_DIM))
+    return MISA_ERR_INVALID_ARG;
+  if (scores_row_stride < L || scores_row_stride % 4 != 0) return MISA_ERR_INVALID_ARG;
+  const int64_t krows = (nkeyseq - 1) * (key_seq_stride / MISA_HEAD_DIM) + L;
+  const int64_t mrows = (nmeanseq - 1) * (means_seq_stride / MISA_HEAD_DIM) + M;
+  if (krows + 128 >= (static_cast<int64_t>(1) << 31) || mrows + 128 >= (static_cast<int64_t>(1) << 31) ||
+      static_cast<int64_t>(T) * H >= (static_cast<int64_t>(1) << 31))
+    return MISA_ERR_UNSUPPORTED;   // TMA coordinates are int32
+  misa_status st = check_ws(workspace, workspace_bytes, misa_workspace_bytes(MISA_OP_INDEX_DECODE, T, H, L, B, k, 0));
+  if (st != MISA_OK) return st;
+  uint8_t* base = static_cast<uint8_t*>(workspace) + kErrBytes;
+  misa::DecodeArgs a;
+  a.q = q;
+  a.w = w;
+  a.keys = keys;
+  a.nkeyseq = nkeyseq;
+  a.key_seq_stride = key_seq_stride;
+  a.means_hi = means_hi;
+  a.means_lo = means_lo;
+  a.nmeanseq = nmeanseq;
+  a.means_seq_stride = means_seq_stride;
+  a.seq_of = seq_of;
+  a.prefix_len = prefix_len;
+  a.T = T;
+  a.H = H;
+  a.h = h;
+  a.k = k;
+  a.B = B;
+  a.L = L;
+  a.heads = heads;
+  a.importance = importance;
+  a.scores = scores;
+  a.row_stride = scores_row_stride;
+  a.idx = idx;
+  a.counters = reinterpret_cast<unsigned*>(base);
+  a.hist = reinterpret_cast<uint32_t*>(base + (static_cast<size_t>(T) * 4 + 255) / 256 * 256);
+  a.err = err_word(workspace);
+  return cuda_status(misa::launch_decode_fused(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 misa_status misa_hier_rerank(const uint16_t* q, const float* w, const uint16_t* keys, int64_t nkeyseq,
                              int64_t key_seq_stride, const int32_t* seq_of, const int32_t* prefix_len, int T, int H,
                              int64_t L, const int32_t* cand, int kp, int k, float* cand_scores, int32_t* idx,
@@ -306,30 +400,31 @@ misa_status misa_hier_rerank(const uint16_t* q, const float* w, const uint16_t* 
   return MISA_OK;
 }
 
-misa_status hisa_block_filter(const uint16_t* q, const float* w, const float* means, const uint16_t* means_hi,
-                              const uint16_t* means_lo, int64_t nseq, int64_t means_seq_stride, const int32_t* seq_of, const int32_t* prefix_len, int T, int H,
-                              int64_t L, int B, int m, int32_t* blocks, int32_t* cand, float* block_scores,
-                              void* workspace, size_t workspace_bytes, misa_stream_t stream) {
+misa_status hisa_block_filter_ex(const uint16_t* q, const float* w, const float* means, const uint16_t* means_hi,
+                                 const uint16_t* means_lo, int64_t nseq, int64_t means_seq_stride,
+                                 const int32_t* seq_of, const int32_t* prefix_len, int T, int H, int64_t L, int B,
+                                 int S, int m, int32_t* blocks, int32_t* cand, float* block_scores, void* workspace,
+                                 size_t workspace_bytes, misa_stream_t stream) {
   misa_status st =
-      check_block_args(q, w, means, means_hi, means_lo, nseq, means_seq_stride, seq_of, prefix_len, T, H, L, B);
+      check_block_args(q, w, means, means_hi, means_lo, nseq, means_seq_stride, seq_of, prefix_len, T, H, L, B, S);
   if (st != MISA_OK) return st;
   if (!blocks || !cand || m < 1) return MISA_ERR_INVALID_ARG;
   if (means_seq_stride % MISA_HEAD_DIM != 0) return MISA_ERR_INVALID_ARG;  // rows of 128 means for the TMA map
   if (m > MISA_MAX_TOPK || T > MISA_MAX_TOPK_ROWS) return MISA_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(m) * B >= (static_cast<int64_t>(1) << 31)) return MISA_ERR_UNSUPPORTED;
-  st = check_ws(workspace, workspace_bytes, misa_workspace_bytes(MISA_OP_HISA_BLOCK_FILTER, T, H, L, B, m, 0));
+  const int64_t M = misa::num_windows(L, B, S);
+  const int64_t M_pad = round_up4(M);
+  st = check_ws(workspace, workspace_bytes, kErrBytes + static_cast<size_t>(T) * M_pad * sizeof(float));
   if (st != MISA_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int64_t M = ceil_div(L, B);
-  const int64_t M_pad = round_up4(M);
   float* bs = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kErrBytes);
   cudaError_t e = misa::launch_hisa_block_scores_tc(q, w, means, means_hi, means_lo, means_seq_stride,
-                                                    static_cast<int>(nseq), seq_of,
-                                                    prefix_len, T, H, L, B, bs, M_pad, err_word(workspace), s);
+                                                    static_cast<int>(nseq), seq_of, prefix_len, T, H, L, B, S, bs,
+                                                    M_pad, err_word(workspace), s);
   if (e != cudaSuccess) return MISA_ERR_CUDA;
   e = misa::launch_topk(bs, T, M, M_pad, nullptr, nullptr, 0, m, blocks, s);
   if (e != cudaSuccess) return MISA_ERR_CUDA;
-  e = misa::launch_hisa_expand(blocks, prefix_len, T, m, B, L, cand, s);
+  e = misa::launch_hisa_expand(blocks, prefix_len, T, m, B, S, L, cand, s);
   if (e != cudaSuccess) return MISA_ERR_CUDA;
   if (block_scores) {
     e = cudaMemcpy2DAsync(block_scores, static_cast<size_t>(M) * sizeof(float), bs,
@@ -338,6 +433,15 @@ misa_status hisa_block_filter(const uint16_t* q, const float* w, const float* me
     if (e != cudaSuccess) return MISA_ERR_CUDA;
   }
   return MISA_OK;
+}
+
+misa_status hisa_block_filter(const uint16_t* q, const float* w, const float* means, const uint16_t* means_hi,
+                              const uint16_t* means_lo, int64_t nseq, int64_t means_seq_stride, const int32_t* seq_of,
+                              const int32_t* prefix_len, int T, int H, int64_t L, int B, int m, int32_t* blocks,
+                              int32_t* cand, float* block_scores, void* workspace, size_t workspace_bytes,
+                              misa_stream_t stream) {
+  return hisa_block_filter_ex(q, w, means, means_hi, means_lo, nseq, means_seq_stride, seq_of, prefix_len, T, H, L, B,
+                              B, m, blocks, cand, block_scores, workspace, workspace_bytes, stream);
 }
 
 misa_status misa_sparse_mla(const uint16_t* q, const uint16_t* kv, int64_t nseq, int64_t kv_seq_stride, int64_t L,

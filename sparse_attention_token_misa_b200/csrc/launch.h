@@ -54,34 +54,42 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return cudaGetLastError();
 }
 
-cudaError_t launch_block_stats(const uint16_t* keys, int64_t nseq, int64_t L, int64_t key_seq_stride, int B,
-                               float* means, uint16_t* means_hi, uint16_t* means_lo, cudaStream_t stream);
-cudaError_t launch_append_keys(uint16_t* keys, int64_t nseq, int64_t key_seq_stride, int64_t L_cap,
-                               const int32_t* len, const uint16_t* new_keys, int n_new, int B, float* means,
-                               uint16_t* means_hi, uint16_t* means_lo, int64_t means_seq_stride, uint32_t* err,
+// Windows of B keys every S keys over a cache of L keys: 1 + ceil(max(L - B, 0) / S).
+int64_t num_windows(int64_t L, int64_t B, int64_t S);
+cudaError_t launch_block_stats(const uint16_t* keys, int64_t nseq, int64_t L, int64_t key_seq_stride, int B, int S,
+                               bool pool_max, float* means, uint16_t* means_hi, uint16_t* means_lo,
                                cudaStream_t stream);
+cudaError_t launch_append_keys(uint16_t* keys, int64_t nseq, int64_t key_seq_stride, int64_t L_cap,
+                               const int32_t* len, const uint16_t* new_keys, int n_new, int B, int S, bool pool_max,
+                               float* means, uint16_t* means_hi, uint16_t* means_lo, int64_t means_seq_stride,
+                               uint32_t* err, cudaStream_t stream);
 
 int router_chunks(int M);
 
 // Tensor-core router (route_tc.cu).  qpm = queries per MMA row group (>1 only
 // when the queries share one sequence's block means).
 int route_tc_queries_per_group(int H, int q_block, bool shared_sequence);
+// S: the window stride of the block statistics (S = B: plain blocks).
 cudaError_t launch_route_heads_tc(const uint16_t* q, const float* w, const float* means, const uint16_t* means_hi,
                                   const uint16_t* means_lo, int64_t means_seq_stride,
                                   int nseq, const int32_t* seq_of, const int32_t* prefix_len, int T, int H, int64_t L,
-                                  int B, int q_block, int h, int qpm, int32_t* heads, float* importance,
+                                  int B, int S, int q_block, int h, int qpm, int32_t* heads, float* importance,
                                   float* partial, unsigned* counters, bool clear_counters, uint32_t* err,
                                   cudaStream_t stream);
 
-// Bytes of router scratch: partial importances (at most [T][ceil(M/32)][H]
-// fp32) followed, at a 256-byte boundary, by one counter per routing decision.
+// Bytes of router scratch for M block statistics: partial importances (at most
+// [T][ceil(M/32)][H] fp32) followed, at a 256-byte boundary, by one counter
+// per routing decision.
+size_t router_scratch_bytes_m(int T, int H, int64_t M, int q_block);
+size_t router_counters_offset_m(int T, int H, int64_t M);
+// The same for M = ceil(L / B) plain blocks.
 size_t router_scratch_bytes(int T, int H, int64_t L, int B, int q_block);
 size_t router_counters_offset(int T, int H, int64_t L, int B);
 
 cudaError_t launch_hisa_block_scores_tc(const uint16_t* q, const float* w, const float* means,
                                         const uint16_t* means_hi, const uint16_t* means_lo, int64_t means_seq_stride,
                                         int nseq, const int32_t* seq_of, const int32_t* prefix_len, int T, int H,
-                                        int64_t L, int B, float* bscore,
+                                        int64_t L, int B, int S, float* bscore,
                                         int64_t bs_stride, uint32_t* err, cudaStream_t stream);
 
 // Bounded-wait self-test (selftest.cu): result[0] = 1 if the wait returned true.
@@ -103,8 +111,8 @@ cudaError_t launch_sparse_mla(const uint16_t* q, const uint16_t* kv, int64_t nse
                               float scale, uint16_t* out, float* lse, float* part_o, float* part_ml, uint32_t* err,
                               cudaStream_t stream);
 
-cudaError_t launch_hisa_expand(const int32_t* blocks, const int32_t* prefix_len, int T, int m, int B, int64_t L,
-                               int32_t* cand, cudaStream_t stream);
+cudaError_t launch_hisa_expand(const int32_t* blocks, const int32_t* prefix_len, int T, int m, int B, int S,
+                               int64_t L, int32_t* cand, cudaStream_t stream);
 
 // Rows per TMA box of the key map (a 128-key tile is loaded as 128 / kTmaBoxRows
 // boxes per 64-element K half; the host encodes the map with this box height).
@@ -139,6 +147,37 @@ struct ScoreArgs {
 int score_mode_hp(int h_eff, bool shared_groups);
 
 cudaError_t launch_index_score(const CUtensorMap* tmap, const ScoreArgs& a, cudaStream_t stream);
+
+// The fused decode step (decode_fused.cu): router + routed scoring + top-k in
+// one persistent kernel.
+constexpr int kDecodeFusedMaxGrid = 256;   // CTAs at most (one per SM)
+struct DecodeArgs {
+  const uint16_t* q;
+  const float* w;
+  const uint16_t* keys;
+  int64_t nkeyseq, key_seq_stride;
+  const uint16_t* means_hi;
+  const uint16_t* means_lo;
+  int64_t nmeanseq, means_seq_stride;
+  const int32_t* seq_of;
+  const int32_t* prefix_len;
+  int T, H, h, k, B;
+  int64_t L;
+  int32_t* heads;
+  float* importance;
+  float* scores;
+  int64_t row_stride;
+  int32_t* idx;
+  unsigned* counters;   // [T] workspace
+  uint32_t* hist;       // [T][slots][2048] workspace
+  uint32_t* err;
+};
+bool decode_fused_supported(int T, int H, int h, int64_t L, int k);
+// first-digit bins of the per-segment score histograms
+int decode_fused_hist_bins();
+// histogram slots per query for grids of at most sms_bound CTAs
+int64_t decode_fused_hist_slots(int T, int64_t L, int sms_bound);
+cudaError_t launch_decode_fused(const DecodeArgs& a, cudaStream_t stream);
 
 size_t topk_smem_bytes();
 

@@ -79,7 +79,7 @@ misa_status misa_route_heads_noalloc(const uint16_t* q, const float* w, const fl
   // (there is no error word).
   const int qpm = misa::route_tc_queries_per_group(H, q_block, nseq == 1 || means_seq_stride == 0);
   cudaError_t e = misa::launch_route_heads_tc(q, w, means, nullptr, nullptr, means_seq_stride, static_cast<int>(nseq), seq_of,
-                                              prefix_len, T, H, L, B, q_block, h, qpm, heads, importance, partial,
+                                              prefix_len, T, H, L, B, B, q_block, h, qpm, heads, importance, partial,
                                               counters, true, nullptr, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MISA_OK : MISA_ERR_CUDA;
 }

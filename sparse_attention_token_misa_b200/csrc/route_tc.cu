@@ -1,5 +1,10 @@
 // Head router on the 5th-generation tensor cores.
 //
+// The block statistics may be windows of B keys every S keys (S < B:
+// overlapping windows, HISA explainer (zhichai.net), section 七, 潜在改进);
+// window j = [j*S, min(j*S + B, L)) and the visibility rule below hold for any
+// S <= B.
+//
 // "MISA: Mixture of Indexer Sparse Attention for Long-Context LLM Inference"
 // (gist.science), Methodology: per-head affinities against block-aggregated
 // keys are aggregated into an importance per head for the current query (block)
@@ -86,7 +91,7 @@ struct RouteParams {
   const int32_t* prefix_len;
   int T, H;
   int64_t L;
-  int B, M, q_block, h;
+  int B, S, M, q_block, h;  // window length, stride (S = B: plain blocks), windows per sequence
   int qpm;        // queries per row group (share one sequence and one decision)
   int n_pg;       // row groups
   int n_bt;       // block tiles
@@ -109,12 +114,16 @@ __device__ __forceinline__ int group_seq(const RouteParams& p, int pg) {
   return seq;
 }
 
-// number of blocks visible to decision g (whole blocks inside the prefix of its first query)
+// number of windows visible to decision g (whole windows inside the prefix of
+// its first query): window j = [j*S, min(j*S + B, L)) is visible iff
+// min(j*S + B, L) <= prefix, so for a prefix shorter than L the visible
+// windows are j <= (prefix - B) / S (S = B: prefix / B whole blocks)
 __device__ __forceinline__ int visible_blocks(const RouteParams& p, int g) {
   const int64_t pl = p.prefix_len[static_cast<int64_t>(g) * p.q_block];
   if (pl >= p.L) return p.M;
-  if (pl <= 0) return 0;
-  return static_cast<int>(pl / p.B);
+  if (pl < p.B) return 0;
+  const int64_t n = (pl - p.B) / p.S + 1;
+  return static_cast<int>(n < p.M ? n : p.M);
 }
 
 // Top-h of imp[0, H) (value desc, ties to the lower id; NaN ranks as -inf),
@@ -407,10 +416,11 @@ route_tc_kernel(const __grid_constant__ CUtensorMap means_map, const __grid_cons
             // wholly visible: the score; cut by the prefix (the query's own
             // block): +inf, always kept; later: -inf
             const int64_t plen = p.prefix_len[t];
-            const int64_t end = (j + 1) * p.B < p.L ? (j + 1) * p.B : p.L;
+            const int64_t start = j * p.S;
+            const int64_t end = start + p.B < p.L ? start + p.B : p.L;
             const float inf = __int_as_float(0x7f800000);
             p.bscore[static_cast<int64_t>(t) * p.bs_stride + j] =
-                end <= plen ? sum : ((j * p.B < plen && plen < end) ? inf : -inf);
+                end <= plen ? sum : ((start < plen && plen < end) ? inf : -inf);
           }
         }
         named_bar_sync(1, kREpiThreads);  // tb is reused by the next item
@@ -558,7 +568,7 @@ bool encode_mean_maps(const float* means, const uint16_t* hi, const uint16_t* lo
 cudaError_t launch_route_heads_tc(const uint16_t* q, const float* w, const float* means, const uint16_t* means_hi,
                                   const uint16_t* means_lo, int64_t means_seq_stride,
                                   int nseq, const int32_t* seq_of, const int32_t* prefix_len, int T, int H, int64_t L,
-                                  int B, int q_block, int h, int qpm, int32_t* heads, float* importance,
+                                  int B, int S, int q_block, int h, int qpm, int32_t* heads, float* importance,
                                   float* partial, unsigned* counters, bool clear_counters, uint32_t* err,
                                   cudaStream_t stream) {
   RouteParams p = {};
@@ -572,7 +582,8 @@ cudaError_t launch_route_heads_tc(const uint16_t* q, const float* w, const float
   p.H = H;
   p.L = L;
   p.B = B;
-  p.M = static_cast<int>((L + B - 1) / B);
+  p.S = S;
+  p.M = static_cast<int>(num_windows(L, B, S));
   p.q_block = q_block;
   p.h = h;
   p.qpm = qpm;
@@ -621,8 +632,8 @@ cudaError_t launch_route_heads_tc(const uint16_t* q, const float* w, const float
 
 cudaError_t launch_hisa_block_scores_tc(const uint16_t* q, const float* w, const float* means,
                                         const uint16_t* means_hi, const uint16_t* means_lo, int64_t means_seq_stride, int nseq, const int32_t* seq_of,
-                                        const int32_t* prefix_len, int T, int H, int64_t L, int B, float* bscore,
-                                        int64_t bs_stride, uint32_t* err, cudaStream_t stream) {
+                                        const int32_t* prefix_len, int T, int H, int64_t L, int B, int S,
+                                        float* bscore, int64_t bs_stride, uint32_t* err, cudaStream_t stream) {
   if (H > kRM) return cudaErrorInvalidValue;
   const bool shared = nseq == 1 || means_seq_stride == 0;
   int qpm = 1;
@@ -638,7 +649,8 @@ cudaError_t launch_hisa_block_scores_tc(const uint16_t* q, const float* w, const
   p.H = H;
   p.L = L;
   p.B = B;
-  p.M = static_cast<int>((L + B - 1) / B);
+  p.S = S;
+  p.M = static_cast<int>(num_windows(L, B, S));
   p.q_block = qpm;  // (no routing decisions in this mode)
   p.h = 1;
   p.qpm = qpm;

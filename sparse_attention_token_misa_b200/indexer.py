@@ -55,23 +55,34 @@ def capture_graph(fn) -> torch.cuda.CUDAGraph:
 
 
 class MisaIndexer:
-    """Router + routed token scoring + top-k for one batch shape."""
+    """Router + routed token scoring + top-k for one batch shape.
 
-    def __init__(self, T: int, H: int, h: int, L: int, B: int, k: int, q_block: int = 1, device="cuda"):
+    fused=True runs the step as the single kernel of misa_index_decode (decode:
+    one routing decision per query; needs the bf16 split of the block means);
+    route / score / select stay available as the three separate calls."""
+
+    def __init__(self, T: int, H: int, h: int, L: int, B: int, k: int, q_block: int = 1, device="cuda",
+                 stride: int | None = None, fused: bool = False):
         self.T, self.H, self.h, self.L, self.B, self.k, self.q_block = T, H, h, L, B, k, q_block
+        self.fused = fused
+        if fused and (q_block != 1 or (stride is not None and stride != B)):
+            raise ValueError("the fused decode step routes per query over plain blocks")
+        self.stride = B if stride is None else stride   # window stride of the block statistics
         G = (T + q_block - 1) // q_block
         self.heads = torch.empty((G, h), dtype=torch.int32, device=device)
         self.importance = torch.empty((G, H), dtype=torch.float32, device=device)
         self.scores_buf = torch.empty((T, _pad4(L)), dtype=torch.float32, device=device)
         self.scores = self.scores_buf[:, :L]
         self.idx = torch.empty((T, k), dtype=torch.int32, device=device)
-        self.ws_route = nat.alloc_workspace(nat.workspace_bytes(nat.OP_ROUTE_HEADS, T, H, L, B), device)
+        self.ws_route = nat.alloc_workspace(nat.workspace_bytes(nat.OP_ROUTE_HEADS, T, H, L, self.stride), device)
         self.ws = nat.alloc_workspace(256, device)
+        if fused:
+            self.ws_decode = nat.alloc_workspace(nat.workspace_bytes(nat.OP_INDEX_DECODE, T, H, L, B, k), device)
 
     def route(self, q, w, means, seq_of, prefix_len, stream=None):
         nat.route_heads(q, w, seq_of=seq_of, prefix_len=prefix_len, L=self.L, B=self.B, q_block=self.q_block,
                         h=self.h, heads=self.heads, importance=self.importance, workspace=self.ws_route,
-                        stream=stream, **_means_args(means))
+                        stream=stream, stride=self.stride, **_means_args(means))
 
     def score(self, q, w, keys, seq_of, prefix_len, stream=None):
         nat.index_score(q, w, keys, seq_of, prefix_len, heads=self.heads, h=self.h, q_block=self.q_block,
@@ -82,6 +93,12 @@ class MisaIndexer:
                  stream=stream)
 
     def run(self, q, w, keys, means, seq_of, prefix_len, stream=None) -> torch.Tensor:
+        if self.fused:
+            _, hi, lo = means
+            nat.index_decode(q, w, keys, hi, lo, seq_of, prefix_len, self.B, self.h, self.k, heads=self.heads,
+                             importance=self.importance, scores=self.scores_buf, idx=self.idx,
+                             workspace=self.ws_decode, stream=stream)
+            return self.idx
         self.route(q, w, means, seq_of, prefix_len, stream)
         self.score(q, w, keys, seq_of, prefix_len, stream)
         self.select(prefix_len, stream)
@@ -144,20 +161,26 @@ class MisaDaggerIndexer:
 
 
 class HisaIndexer:
-    def __init__(self, T: int, H: int, L: int, B: int, m: int, k: int, device="cuda"):
+    """`stride` < B: the block statistics are overlapping windows of B keys every
+    `stride` keys (as block_stats(..., stride=) writes them); candidates that
+    two chosen windows share are listed once."""
+
+    def __init__(self, T: int, H: int, L: int, B: int, m: int, k: int, device="cuda", stride: int | None = None):
         self.T, self.H, self.L, self.B, self.m, self.k = T, H, L, B, m, k
+        self.stride = B if stride is None else stride
         self.blocks = torch.empty((T, m), dtype=torch.int32, device=device)
         self.cand = torch.empty((T, m * B), dtype=torch.int32, device=device)
         self.scores_buf = torch.empty((T, _pad4(m * B)), dtype=torch.float32, device=device)
         self.scores = self.scores_buf[:, : m * B]
         self.idx = torch.empty((T, k), dtype=torch.int32, device=device)
-        self.ws_filter = nat.alloc_workspace(nat.workspace_bytes(nat.OP_HISA_BLOCK_FILTER, T, H, L, B, m), device)
+        self.ws_filter = nat.alloc_workspace(nat.workspace_bytes(nat.OP_HISA_BLOCK_FILTER, T, H, L, self.stride, m),
+                                             device)
         self.ws = nat.alloc_workspace(256, device)
 
     def run(self, q, w, keys, means, seq_of, prefix_len, stream=None) -> torch.Tensor:
         nat.hisa_block_filter(q, w, seq_of=seq_of, prefix_len=prefix_len, L=self.L, B=self.B, m=self.m,
                               blocks=self.blocks, cand=self.cand, workspace=self.ws_filter, stream=stream,
-                              **_means_args(means))
+                              stride=self.stride, **_means_args(means))
         nat.index_score(q, w, keys, seq_of, prefix_len, cand=self.cand, scores=self.scores_buf, workspace=self.ws,
                         stream=stream)
         nat.topk(self.scores_buf, self.k, n=self.m * self.B, id_map=self.cand, idx=self.idx, workspace=self.ws,

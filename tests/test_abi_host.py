@@ -34,7 +34,7 @@ def declared_functions():
 def test_library_loads_and_exports_every_declared_symbol():
     l = pkg.lib()
     names = declared_functions()
-    assert len(names) == 17, names
+    assert len(names) == 23, names
     for n in names:
         assert hasattr(l, n), n
         assert n in nat.SIGNATURES, n
@@ -265,3 +265,34 @@ def test_selftest_needs_a_workspace():
     l = pkg.lib()
     assert l.misa_selftest_wait_timeout(None, 256, None) == WORKSPACE
     assert l.misa_selftest_wait_timeout(P, 255, None) == WORKSPACE
+
+
+def test_window_entry_points_reject_and_count():
+    l = pkg.lib()
+    # window counts: 1 + ceil(max(L - B, 0) / S); 0 for a bad geometry
+    assert l.misa_num_windows(10, 4, 2) == 4 and l.misa_num_windows(11, 4, 2) == 5
+    assert l.misa_num_windows(3, 4, 2) == 1 and l.misa_num_windows(32768, 128, 128) == 256
+    assert l.misa_num_windows(100, 4, 5) == 0 and l.misa_num_windows(100, 4, 0) == 0
+    assert l.misa_num_windows(0, 4, 2) == 0
+    f = l.misa_block_stats_ex
+    assert f(P, 1, 100, 0, 8, 9, 0, P2, None, None, None) == INVALID     # S > B
+    assert f(P, 1, 100, 0, 8, 0, 0, P2, None, None, None) == INVALID     # S < 1
+    assert f(P, 1, 100, 0, 8, 4, 2, P2, None, None, None) == INVALID     # unknown pool
+    assert f(P, 1, 100, 0, 5000, 4, 0, P2, None, None, None) == UNSUPPORTED
+    a = l.misa_append_keys_ex
+    assert a(P, 1, 0, 1024, P2, P2, 1, 128, 200, 0, P2, None, None, 8 * 128, P2, 256, None) == INVALID
+    assert a(P, 1, 0, 1024, P2, P2, 1, 128, 64, 3, P2, None, None, 16 * 128, P2, 256, None) == INVALID
+    # the statistics stride must hold every window of the cache (1024 keys, B 128, S 64: 15 windows)
+    assert a(P, 2, 1024 * 128, 1024, P2, P2, 1, 128, 64, 0, P2, None, None, 14 * 128, P2, 256, None) == INVALID
+    r = l.misa_route_heads_ex
+    N = None
+    assert r(P, P, P, N, N, 1, 0, P, P, 2, 64, 1000, 128, 129, 1, 8, P2, N, P2, 1 << 20, N) == INVALID
+    assert r(P, P, P, N, N, 1, 0, P, P, 2, 64, 1000, 128, 0, 1, 8, P2, N, P2, 1 << 20, N) == INVALID
+    # workspace sized for plain blocks is too small for windows every 32 keys
+    need_blocks = nat.workspace_bytes(nat.OP_ROUTE_HEADS, 2, 64, 10000, 128)   # 79 blocks: 3 chunks of 32
+    assert need_blocks < nat.workspace_bytes(nat.OP_ROUTE_HEADS, 2, 64, 10000, 32)  # 310 windows: 10 chunks
+    assert r(P, P, P, N, N, 1, 0, P, P, 2, 64, 10000, 128, 32, 1, 8, P2, N, P2, need_blocks, N) == WORKSPACE
+    hf = l.hisa_block_filter_ex
+    assert hf(P, P, P, N, N, 1, 0, P, P, 2, 64, 1000, 128, 256, 4, P2, P2, N, P2, 1 << 20, N) == INVALID
+    need = nat.workspace_bytes(nat.OP_HISA_BLOCK_FILTER, 2, 64, 1000, 128, 4)
+    assert hf(P, P, P, N, N, 1, 0, P, P, 2, 64, 1000, 128, 32, 4, P2, P2, N, P2, need, N) == WORKSPACE

@@ -62,7 +62,7 @@ def _scratch_bytes(wl) -> int:
 def _persistent_cases():
     # causal prefill chunks over one shared cache: many work items per decision
     c = make_prefill("na_c", 43, T=256, L=32768, H=64, h=8, B=128, k=16, q_block=64, n_regions=2, region_len=1024)
-    d = make_prefill("na_d", 44, T=200, L=20000, H=32, h=6, B=64, k=16, q_block=32, n_regions=1, region_len=512)
+    d = make_prefill("na_d", 44, T=200, L=40000, H=32, h=6, B=64, k=16, q_block=32, n_regions=1, region_len=512)
     return c, d
 
 
