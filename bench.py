@@ -485,6 +485,8 @@ def other_workloads(misa, dev, stream, flush, steps, only=None):
         out.update(_dagger_prefill(misa, dev, stream, flush, steps, timed))
     if only in (None, "hisa"):
         out.update(_hisa(misa, dev, stream, flush, steps, timed))
+    if only in (None, "quality"):
+        out["selection_quality_local_inputs"] = _selection_quality(misa, dev)
     if only in (None, "attn"):
         out.update(_sparse_attention(misa, dev, stream, flush, steps, timed))
     return out
@@ -632,6 +634,22 @@ def _hisa(misa, dev, stream, flush, steps, timed):
                                                               "unit": "GB/s", "frac": nb / (ms * 1e-3) / 1e9 / hbm},
                                                  "iou_vs_dense64": iou, "recovery_of_dense64": rec,
                                                  "needle_recall": planted_recall(hx.idx, wl.planted)}
+    # the block statistics the HISA page names as improvements (section 七): max
+    # pooling, and half-overlapping windows (stride 64)
+    for tag, B, S, m, pool in (("max", 128, 128, 64, "max"), ("overlap_S64", 128, 64, 64, "mean")):
+        means = misa.block_stats(keys, B, split=True, stride=S, pool=pool)
+        hx = misa.HisaIndexer(wl.T, wl.H, wl.L, B, m, wl.k, device=dev, stride=S)
+        ms = timed(lambda evs: hx.run(q, w, keys, means, so, pl))
+        iou, rec = selection_agreement(hx.idx, dense_idx)
+        hbm, _, _ = _peaks()
+        M = misa.num_windows(wl.L, B, S)
+        nb = hisa_step_bytes(wl.T, wl.L, wl.H, B, m, wl.k) + wl.T * (M - (wl.L + B - 1) // B) * 128 * 4
+        out[f"hisa_decode_L131072_B{B}_m{m}_{tag}"] = {
+            "ms_per_step": ms, "pairs_per_s": int(wl.prefix_len.sum()) / (ms * 1e-3), "windows": M,
+            "roofline": {"bound": "hbm (latency-dominated)", "algorithmic_bytes_per_step": nb,
+                         "achieved": nb / (ms * 1e-3) / 1e9, "peak": hbm, "unit": "GB/s",
+                         "frac": nb / (ms * 1e-3) / 1e9 / hbm},
+            "iou_vs_dense64": iou, "recovery_of_dense64": rec, "needle_recall": planted_recall(hx.idx, wl.planted)}
     ms = timed(lambda evs: dx.run(q, w, keys, so, pl))
     out["hisa_decode_L131072_dense64"] = {"ms_per_step": ms, "pairs_per_s": int(wl.prefix_len.sum()) / (ms * 1e-3),
                                           "needle_recall": planted_recall(dense_idx, wl.planted)}
@@ -642,6 +660,43 @@ def _hisa(misa, dev, stream, flush, steps, timed):
     hx = misa.HisaIndexer(wp.T, wp.H, wp.L, 128, 64, wp.k, device=dev)
     ms = timed(lambda evs: hx.run(q, w, keys, means, so, pl))
     out["prefill_L131072_hisa_B128_m64"] = {"ms_per_step": ms, "pairs_per_s": int(wp.prefix_len.sum()) / (ms * 1e-3)}
+    return out
+
+
+def _selection_quality(misa, dev):
+    """Selection agreement with the dense 64-head indexer on inputs with
+    locality (keys in contiguous regions around their own centroids, needles
+    aligned with the positively weighted heads' query rows): the HISA decode
+    shape (16 x 131072 keys, k = 2048) through MISA-8, MISA-dagger (k' = 8192)
+    and HISA with mean-pooled blocks, max-pooled blocks and half-overlapping
+    windows.  Information only: the pages' figures come from real text."""
+    from workloads import make_local_decode
+    wl = make_local_decode("local_decode_L131072", 6, T=16, L=131072, H=64, h=8, B=128, k=2048, n_planted=8,
+                           planted_range=(0.4, 0.6))
+    q, w, keys, so, pl = (x.to(dev) for x in (wl.q, wl.w, wl.keys, wl.seq_of, wl.prefix_len))
+    dx = misa.DenseIndexer(wl.T, wl.H, wl.L, wl.k, device=dev)
+    dense_idx = dx.run(q, w, keys, so, pl).clone()
+    out = {"inputs": "16 caches of 131072 keys in regions of 256-4096 tokens around their own centroid "
+                     "(k = c + 0.3 eps), 8 needles per query aligned with sum_h max(w_h, 0) q_h, in [0.4 L, 0.6 L)",
+           "dense64_needle_recall": planted_recall(dense_idx, wl.planted)}
+    means = misa.block_stats(keys, wl.B, split=True)
+    ix = misa.MisaIndexer(wl.T, wl.H, wl.h, wl.L, wl.B, wl.k, device=dev)
+    ix.run(q, w, keys, means, so, pl)
+    dg = misa.MisaDaggerIndexer(wl.T, wl.H, wl.h, wl.L, wl.B, 8192, wl.k, device=dev)
+    dg.run(q, w, keys, means, so, pl)
+    runs = {"misa8": ix.idx, "misa_dagger_kp8192": dg.idx}
+    for tag, S, pool in (("hisa_B128_m64_mean", 128, "mean"), ("hisa_B128_m64_max", 128, "max"),
+                         ("hisa_B128_m64_overlap_S64", 64, "mean")):
+        st = misa.block_stats(keys, 128, split=True, stride=S, pool=pool)
+        hx = misa.HisaIndexer(wl.T, wl.H, wl.L, 128, 64, wl.k, device=dev, stride=S)
+        runs[tag] = hx.run(q, w, keys, st, so, pl).clone()
+    torch.cuda.synchronize()
+    for tag, idx in runs.items():
+        iou, rec = selection_agreement(idx, dense_idx)
+        out[tag] = {"iou_vs_dense64": iou, "recovery_of_dense64": rec,
+                    "needle_recall": planted_recall(idx, wl.planted)}
+    del keys
+    torch.cuda.empty_cache()
     return out
 
 
@@ -865,7 +920,7 @@ def main():
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     ap.add_argument("--quick", action="store_true", help="skip the other four workloads")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
-    ap.add_argument("--only", choices=["prefill", "dagger", "hisa", "attn"], default=None,
+    ap.add_argument("--only", choices=["prefill", "dagger", "hisa", "attn", "quality"], default=None,
                     help="time one of the other workloads alone (for profiler captures); prints its own JSON")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -118,6 +118,22 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* map, uint64_t
       : "memory");
 }
 
+// Bulk copy of `bytes` (a multiple of 16; both addresses 16-byte aligned) from
+// global to shared memory, completion counted in bytes on `bar`.
+__device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+// Ask L2 for the 2-D box of a tensor map at (x, y) (no shared memory, no
+// completion to wait for).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const void* map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(x), "r"(y)
+               : "memory");
+}
+
 // L2 policy for data read once (the key stream): evict first, so that it does
 // not push out data that is read again soon (e.g. the fp32 score rows).
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {

@@ -149,6 +149,51 @@ def make_prefill(name: str, seed: int, T: int, L: int, H: int, h: int, B: int, k
         H=H, h=h, B=B, k=k, q_block=q_block, shared_cache=True)
 
 
+def make_local_decode(name: str, seed: int, T: int, L: int, H: int, h: int, B: int, k: int, n_planted: int,
+                      region_len=(256, 4096), sigma: float = 0.3, planted_range=(0.0, 1.0)) -> Workload:
+    """Decode batch whose keys have locality, with needles the dense score favours.
+
+    Used only for the selection-quality figures (IoU, recall); the timed
+    workloads are the ones below.  Each cache is cut into consecutive regions
+    of uniform random length in region_len; region r draws a centroid
+    c_r ~ N(0, 1) / sqrt(d) and its keys are c_r + sigma * eps (eps ~ N(0, 1) /
+    sqrt(d)), so neighbouring keys resemble each other the way text does and a
+    block statistic says something about its tokens.  Needle keys for query t
+    point along the query rows of its positively weighted heads,
+    normalize(sum_h max(w[t, h], 0) * q[t, h]) + N(0, 0.1^2 / d), at distinct
+    uniform positions in planted_range.  Draw order: per cache region lengths,
+    centroids and noise; then q, w, needle positions and noise.
+    """
+    rng = np.random.default_rng(seed)
+    keys = np.empty((T, L, D), dtype=np.float32)
+    for b in range(T):
+        s = 0
+        while s < L:
+            n = int(rng.integers(region_len[0], region_len[1] + 1))
+            n = min(n, L - s)
+            c = rng.standard_normal(D, dtype=np.float32) / np.float32(np.sqrt(D))
+            eps = rng.standard_normal((n, D), dtype=np.float32) / np.float32(np.sqrt(D))
+            keys[b, s:s + n] = c + np.float32(sigma) * eps
+            s += n
+    q = _bf16(rng.standard_normal((T, H, D), dtype=np.float32))
+    w = torch.from_numpy(rng.standard_normal((T, H), dtype=np.float32) / np.float32(8.0))
+    q32 = q.to(torch.float32).numpy()
+    w32 = w.numpy()
+    lo = int(planted_range[0] * L)
+    hi = max(int(planted_range[1] * L), lo + n_planted)
+    planted = np.zeros((T, n_planted), dtype=np.int64)
+    for t in range(T):
+        planted[t] = rng.choice(np.arange(lo, hi), size=n_planted, replace=False)
+        u = (np.maximum(w32[t], 0.0)[:, None] * q32[t]).sum(axis=0)
+        u = u / max(float(np.linalg.norm(u)), 1e-12)
+        for p_ in planted[t]:
+            keys[t, p_] = u + rng.standard_normal(D, dtype=np.float32) * np.float32(0.1 / np.sqrt(D))
+    return Workload(
+        name=name, mode="misa", q=q, w=w, keys=_bf16(keys),
+        seq_of=torch.arange(T, dtype=torch.int32), prefix_len=torch.full((T,), L, dtype=torch.int32),
+        H=H, h=h, B=B, k=k, q_block=1, planted=planted)
+
+
 # The five workloads, by what they are.  Names say the shape.
 CONFIG_NAMES = (
     "tiny_decode_L4096",
