@@ -82,7 +82,7 @@ constexpr int kFRouterTmaWarp = 10;
 constexpr int kFBins = 1024;                    // first digit: the top 10 key bits
 constexpr int kFBinShift = 22;
 constexpr int kFLoBin = 2;                      // bins below hold only NaN and -inf (key <= 0x007FFFFF)
-constexpr int kFCandCap = 4096;                 // threshold-bin entries resolved in shared memory
+constexpr int kFCandCap = 9216;                 // threshold-bin entries resolved in shared memory
 constexpr int kFMaxL = 65536;                   // longest row (position bitmaps)
 constexpr int kFMaxNR = 64;                     // router columns (H <= 64)
 constexpr int kFMaxGroups = 1024;               // queries one CTA may work on
@@ -112,8 +112,8 @@ constexpr int kFScrBits = 0;                                      // [kFMaxL / 3
 constexpr int kFScrTBits = kFScrBits + kFMaxL / 8;                // [kFMaxL / 32] u32
 constexpr int kFScrRHist = kFScrTBits + kFMaxL / 8;               // [2048] u32
 constexpr int kFScrCand = kFScrRHist + 2048 * 4;                  // [kFCandCap] (key, position) u32 pairs
-constexpr int kFScrStage = kFScrCand + kFCandCap * 8;             // [2][8192] f32 row chunks
-static_assert(kFScrStage + 2 * 8192 * 4 <= kFStages * kFTileBytes, "selection scratch fits the ring");
+constexpr int kFScrStage = kFScrCand + kFCandCap * 8;             // [2][4096] f32 row chunks
+static_assert(kFScrStage + 2 * 4096 * 4 <= kFStages * kFTileBytes, "selection scratch fits the ring");
 static_assert(kFSmemBytes <= 232448, "shared memory per CTA");
 static_assert(4 * 12 <= 64, "append mask bits per batch");
 
@@ -277,7 +277,7 @@ struct RowStage {
   uint32_t* err;
   volatile uint32_t* abort;
 };
-constexpr int kFChunk = 8192;   // 32 KB
+constexpr int kFChunk = 4096;   // 16 KB
 
 // tid 0 starts the copy of chunk ch (entries [ch kFChunk, min(n, ...))) into
 // buffer ch & 1; the byte count is rounded up to 16 (rows are padded to a
@@ -293,20 +293,26 @@ __device__ __forceinline__ void f_stage_issue(RowStage& st, const float* row, in
 }
 
 // One pass over the first n entries of a score row by the 128 epilogue
-// threads, from the shared-memory chunks.  Element e4 of a chunk is its
-// positions 4 e4 .. 4 e4 + 3, so a warp covers 128 consecutive positions per
-// step, four 32-bit bitmap words: f(pos, key) returns a code per position (bit
-// 0: set in `bits`, bit 1: set in `tbits`, bit 2: append (key, pos) to the
-// candidate list `cand`, counted in *cnt, at most kFCandCap kept); the words
-// are formed by shuffles and stored by one lane each (OR-ed into what they
-// already hold); the appends of a step take one shared-memory atomic per warp.
-// g(ok, pos, key) is called for every position for side work.
+// threads, from the shared-memory chunks.  Warp w takes the 32-position words
+// w, w + 4, ... of each chunk, kFWordsPerStep of them per step for
+// instruction-level parallelism, one entry per lane: f(pos, key) returns a code
+// (bit 0: set in `bits`, bit 1: set in `tbits`, bit 2: append (key, pos) to the
+// warp's candidate region); a ballot per code bit gives the bitmap word
+// directly and the append slots (no atomics, no scans).  cand: per-warp regions
+// of kFWarpCand (key, pos) pairs; ccount: per-warp counts (kept in a register,
+// may exceed kFWarpCand: the excess is not stored).  g(ok, pos, key) is called
+// for every position for side work.
+constexpr int kFWarpCand = kFCandCap / 4;
+constexpr int kFWordsPerStep = 4;
 template <class F, class Gf>
 __device__ __forceinline__ void f_row_pass(RowStage& st, const float* row, int n, uint32_t* bits, uint32_t* tbits,
-                                           uint32_t* cand, uint32_t* cnt, F f, Gf gside) {
-  const int tid = threadIdx.x, lane = tid & 31;
+                                           uint32_t* cand, uint32_t* ccount, F f, Gf gside) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t lt = (1u << lane) - 1u;
   if (n <= 0) return;
   const int nch = (n + kFChunk - 1) / kFChunk;
+  uint32_t cw = cand != nullptr ? ccount[warp] : 0u;
+  uint32_t* wcand = cand != nullptr ? cand + 2 * warp * kFWarpCand : nullptr;
   f_stage_issue(st, row, n, 0);
   if (nch > 1) f_stage_issue(st, row, n, 1);
   for (int ch = 0; ch < nch; ++ch) {
@@ -315,68 +321,110 @@ __device__ __forceinline__ void f_row_pass(RowStage& st, const float* row, int n
       // a copy that never lands: the row is left unselected (error recorded)
     }
     ++st.fills[bi];
-    const float4* src = reinterpret_cast<const float4*>(st.buf[bi]);
+    const float* src = st.buf[bi];
     const int first = ch * kFChunk;
     const int cn = min(kFChunk, n - first);
-    const int n4 = (cn + 3) >> 2;
-    for (int e0 = 0; e0 < n4; e0 += kFEpiThreads) {   // (warp-uniform trip count)
-      const int e4 = e0 + tid;
-      const float4 v = src[min(e4, n4 - 1)];
-      const float vv[4] = {v.x, v.y, v.z, v.w};
-      uint32_t nib = 0, tnib = 0, cbits = 0;
+    const int nwc = (cn + 31) >> 5;
+    for (int w0 = warp; w0 < nwc; w0 += 4 * kFWordsPerStep) {   // (warp-uniform)
+      float x[kFWordsPerStep];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int lpos = 4 * e4 + c;
-        const bool ok = e4 < n4 && lpos < cn;
-        const int pos = first + lpos;
-        const uint32_t key = ok ? f_sel_key(vv[c]) : 0u;
+      for (int u = 0; u < kFWordsPerStep; ++u) {
+        const int lp = (w0 + 4 * u) * 32 + lane;
+        x[u] = lp < cn ? src[lp] : -__int_as_float(0x7f800000);
+      }
+#pragma unroll
+      for (int u = 0; u < kFWordsPerStep; ++u) {
+        const int word = w0 + 4 * u;
+        if (word >= nwc) break;   // (warp-uniform)
+        const int lp = word * 32 + lane;
+        const bool ok = lp < cn;
+        const int pos = first + lp;
+        const uint32_t key = ok ? f_sel_key(x[u]) : 0u;
         const uint32_t code = ok ? f(pos, key) : 0u;
-        nib |= (code & 1u) << c;
-        tnib |= ((code >> 1) & 1u) << c;
-        cbits |= ((code >> 2) & 1u) << c;
+        const uint32_t m0 = __ballot_sync(0xffffffffu, code & 1u);
+        const uint32_t m1 = __ballot_sync(0xffffffffu, code & 2u);
+        const uint32_t m2 = __ballot_sync(0xffffffffu, code & 4u);
+        if (lane == 0) {
+          const int gw = (first >> 5) + word;
+          if (m0) bits[gw] |= m0;
+          if (m1) tbits[gw] |= m1;
+        }
+        if (m2) {
+          const uint32_t slot = cw + __popc(m2 & lt);
+          if ((code & 4u) && slot < static_cast<uint32_t>(kFWarpCand)) {
+            wcand[2 * slot] = key;
+            wcand[2 * slot + 1] = static_cast<uint32_t>(pos);
+          }
+          cw += __popc(m2);
+        }
         gside(ok, pos, key);
       }
-      // eight lanes hold one word's 32 positions, a nibble each
-      uint32_t x = nib << (4 * (lane & 7)), y = tnib << (4 * (lane & 7));
+    }
+    named_bar_sync(1, kFEpiThreads);   // the buffer is read: it may be refilled
+    if (ch + 2 < nch) f_stage_issue(st, row, n, ch + 2);
+  }
+  if (cand != nullptr && lane == 0) ccount[warp] = cw;
+}
+
+// The float whose order-preserving key is k (inverse of float_key).
+__device__ __forceinline__ float f_key_to_float(uint32_t k) {
+  const uint32_t u = (k & 0x80000000u) ? (k ^ 0x80000000u) : ~k;
+  return __uint_as_float(u);
+}
+
+// The common first pass of the selection: entries x >= hiv (none when `top`)
+// into `bits`, entries lov <= x < hiv into the per-warp candidate regions (as
+// (key, position)).  Two comparisons and two ballots per entry; NaN compares
+// false and is never taken.
+__device__ __forceinline__ void f_row_pass_values(RowStage& st, const float* row, int n, uint32_t* bits,
+                                                  uint32_t* cand, uint32_t* ccount, float lov, float hiv,
+                                                  bool top) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t lt = (1u << lane) - 1u;
+  if (n <= 0) return;
+  const int nch = (n + kFChunk - 1) / kFChunk;
+  uint32_t cw = ccount[warp];
+  uint32_t* wcand = cand + 2 * warp * kFWarpCand;
+  f_stage_issue(st, row, n, 0);
+  if (nch > 1) f_stage_issue(st, row, n, 1);
+  for (int ch = 0; ch < nch; ++ch) {
+    const int bi = ch & 1;
+    mbar_wait(st.bar[bi], st.fills[bi] & 1u, st.err, st.abort);   // (a copy that never lands: error recorded)
+    ++st.fills[bi];
+    const float* src = st.buf[bi];
+    const int first = ch * kFChunk;
+    const int cn = min(kFChunk, n - first);
+    const int nwc = (cn + 31) >> 5;
+    for (int w0 = warp; w0 < nwc; w0 += 4 * kFWordsPerStep) {   // (warp-uniform)
+      float x[kFWordsPerStep];
 #pragma unroll
-      for (int o = 1; o < 8; o <<= 1) {
-        x |= __shfl_xor_sync(0xffffffffu, x, o);
-        y |= __shfl_xor_sync(0xffffffffu, y, o);
+      for (int u = 0; u < kFWordsPerStep; ++u) {
+        const int lp = (w0 + 4 * u) * 32 + lane;
+        x[u] = lp < cn ? src[lp] : __int_as_float(0x7fc00000);   // NaN: neither above nor in
       }
-      if ((lane & 7) == 0 && e4 < n4) {
-        const int word = (first + 4 * (e4 - (lane & 7))) >> 5;   // the group's first position / 32
-        if (x) bits[word] |= x;
-        if (y) tbits[word] |= y;
-      }
-      if (cand != nullptr) {
-        const uint32_t mine = __popc(cbits);
-        const unsigned any = __ballot_sync(0xffffffffu, mine != 0u);
-        if (any) {
-          uint32_t inc = mine;
 #pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y2 = __shfl_up_sync(0xffffffffu, inc, o);
-            if (lane >= o) inc += y2;
+      for (int u = 0; u < kFWordsPerStep; ++u) {
+        const int word = w0 + 4 * u;
+        if (word >= nwc) break;   // (warp-uniform)
+        const bool above = !top && x[u] >= hiv;
+        const bool in = x[u] >= lov && !above;
+        const uint32_t ma = __ballot_sync(0xffffffffu, above);
+        const uint32_t mi = __ballot_sync(0xffffffffu, in);
+        if (lane == 0 && ma) bits[(first >> 5) + word] |= ma;
+        if (mi) {
+          const uint32_t slot = cw + __popc(mi & lt);
+          if (in && slot < static_cast<uint32_t>(kFWarpCand)) {
+            wcand[2 * slot] = f_sel_key(x[u]);
+            wcand[2 * slot + 1] = static_cast<uint32_t>(first + word * 32 + lane);
           }
-          uint32_t base = 0;
-          if (lane == 31) base = atomicAdd(cnt, inc);
-          base = __shfl_sync(0xffffffffu, base, 31) + inc - mine;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            if ((cbits >> c) & 1u) {
-              if (base < kFCandCap) {
-                cand[2 * base] = f_sel_key(vv[c]);
-                cand[2 * base + 1] = static_cast<uint32_t>(first + 4 * e4 + c);
-              }
-              ++base;
-            }
-          }
+          cw += __popc(mi);
         }
       }
     }
     named_bar_sync(1, kFEpiThreads);   // the buffer is read: it may be refilled
     if (ch + 2 < nch) f_stage_issue(st, row, n, ch + 2);
   }
+  if (lane == 0) ccount[warp] = cw;
 }
 
 // Top-k of one finished score row, by the 128 scoring-epilogue threads.  hist:
@@ -402,25 +450,37 @@ __device__ void f_select_row(const FusedParams& p, int g, const uint32_t* hist, 
   auto no_side = [](bool, int, uint32_t) {};
   if (nvalid <= k) {
     // every selectable entry
-    f_row_pass(st, row, n, bits, tbits, nullptr, nullptr, [](int, uint32_t key) { return key > kNegInfKey ? 1u : 0u; },
-               no_side);
+    // every selectable entry: x >= -FLT_MAX (not NaN, not -inf)
+    if (tid < 4) ws[8 + tid] = 0u;
+    named_bar_sync(1, kFEpiThreads);
+    f_row_pass_values(st, row, n, bits, cand, ws + 8, __int_as_float(0x7f800000), -__int_as_float(0x7f7fffff),
+                      false);
   } else {
     uint32_t above = 0;
     const int bstar = f_find_bin(hist, kFBins, kFLoBin, k, ws, &above);
     const uint32_t need = k - above;       // entries to take from bin bstar, >= 1
     const uint32_t ub = static_cast<uint32_t>(bstar);
-    // one pass: entries above the bin into the bitmap, entries in it into the list
-    if (tid == 0) ws[6] = 0u;
+    // one pass: entries above the bin into the bitmap, entries in it into the
+    // per-warp candidate regions (counts in ws[8 .. 12))
+    uint32_t* ccount = ws + 8;
+    if (tid < 4) ccount[tid] = 0u;
     named_bar_sync(1, kFEpiThreads);
-    f_row_pass(st, row, n, bits, tbits, cand, ws + 6,
-               [ub](int, uint32_t key) {
-                 const uint32_t b = key >> kFBinShift;
-                 return b > ub ? 1u : ((b == ub && key > kNegInfKey) ? 4u : 0u);
-               },
-               no_side);
+    // the bin's edges as values (the key order is the value order, -0 == +0):
+    // an entry is above the bin iff x >= hiv, in it iff lov <= x < hiv
+    const float lov = f_key_to_float(ub << kFBinShift);
+    const bool top = ub + 1u >= static_cast<uint32_t>(kFBins);
+    const float hiv = top ? __int_as_float(0x7fc00000) : f_key_to_float((ub + 1u) << kFBinShift);
+    f_row_pass_values(st, row, n, bits, cand, ccount, lov, hiv, top);
     named_bar_sync(1, kFEpiThreads);
-    const uint32_t nc = ws[6];
-    const bool in_list = nc <= kFCandCap;
+    uint32_t wc[4];
+    bool in_list = true;
+#pragma unroll
+    for (int w2 = 0; w2 < 4; ++w2) {
+      wc[w2] = ccount[w2];
+      in_list = in_list && wc[w2] <= static_cast<uint32_t>(kFWarpCand);
+    }
+    // candidate i (< kFCandCap) is stored iff its slot in its warp's region is used
+    auto cand_ok = [&](int i) { return static_cast<uint32_t>(i % kFWarpCand) < wc[i / kFWarpCand]; };
     // exact threshold inside the bin: two more 11-bit digits
     uint32_t need2 = need, pre = ub << kFBinShift, pre_mask = 0xFFFFFFFFu << kFBinShift;
     for (int round = 0; round < 2; ++round) {
@@ -429,7 +489,8 @@ __device__ void f_select_row(const FusedParams& p, int g, const uint32_t* hist, 
       for (int b = tid; b < nb; b += kFEpiThreads) rhist[b] = 0u;
       named_bar_sync(1, kFEpiThreads);
       if (in_list) {
-        for (uint32_t i = tid; i < nc; i += kFEpiThreads) {
+        for (int i = tid; i < kFCandCap; i += kFEpiThreads) {
+          if (!cand_ok(i)) continue;
           const uint32_t key = cand[2 * i];
           if ((key & pre_mask) == pre) atomicAdd(&rhist[(key >> shift) & (nb - 1)], 1u);
         }
@@ -452,7 +513,8 @@ __device__ void f_select_row(const FusedParams& p, int g, const uint32_t* hist, 
     const uint32_t need_eq = need2; // entries equal to tau to take, lowest positions first
     // the bin's entries above tau into the bitmap, its ties into the tie bitmap
     if (in_list) {
-      for (uint32_t i = tid; i < nc; i += kFEpiThreads) {
+      for (int i = tid; i < kFCandCap; i += kFEpiThreads) {
+        if (!cand_ok(i)) continue;
         const uint32_t key = cand[2 * i], pos = cand[2 * i + 1];
         if (key > tau) atomicOr(&bits[pos >> 5], 1u << (pos & 31));
         else if (key == tau) atomicOr(&tbits[pos >> 5], 1u << (pos & 31));
