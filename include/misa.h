@@ -359,8 +359,9 @@ MISA_API misa_status misa_index_score(const uint16_t* q, const float* w, const u
                              void* workspace, size_t workspace_bytes, misa_stream_t stream);
 
 /*
- * misa_index_decode -- one whole MISA decode step in a single launch: the
- * router, the routed token scoring and the per-query top-k.
+ * misa_index_decode -- one whole MISA decode step in one call: the router and
+ * the routed token scoring in one persistent kernel, the per-query top-k in a
+ * second kernel that starts while the first one's last CTAs finish.
  *   [MISA page (gist.science), "Methodology: MISA": the router reads the
  *   mean-pooled block statistics and keeps h of the H heads per query; only
  *   those heads score every prefix token; the top-k tokens are kept.]
@@ -375,17 +376,17 @@ MISA_API misa_status misa_index_score(const uint16_t* q, const float* w, const u
  * (a per-block reduction on the tensor-core accumulator), so they can differ
  * in the last bits and a head choice can differ where two importances are that
  * close; given the heads, the scores equal misa_index_score's bit for bit and
- * idx is the exact top-k of the scores written.
+ * idx is misa_topk's of the scores written.
  * means_hi / means_lo: the bf16 split misa_block_stats writes (block size B,
  * nmeanseq sequences of ceil(L/B) rows at stride means_seq_stride, a multiple
  * of 128).  Keys as misa_index_score.
  * Limits: 1 <= H <= 64, 1 <= h <= 16, h <= H, 1 <= L <= 65536, 1 <= k <=
- *   MISA_MAX_TOPK; other shapes return MISA_ERR_UNSUPPORTED (use the separate
- *   calls).  q, keys, means_hi, means_lo, scores 16-byte aligned,
- *   scores_row_stride >= L and a multiple of 4.
- * workspace: >= misa_workspace_bytes(MISA_OP_INDEX_DECODE, T, H, L, B, k, 0):
- *   error word, per-query counters (cleared by the call on `stream`) and
- *   per-query score histograms; its contents on entry do not matter.
+ *   MISA_MAX_TOPK, T <= MISA_MAX_TOPK_ROWS; other shapes return
+ *   MISA_ERR_UNSUPPORTED (use the separate calls).  q, keys, means_hi,
+ *   means_lo, scores 16-byte aligned, scores_row_stride >= L and a multiple
+ *   of 4.
+ * workspace: >= misa_workspace_bytes(MISA_OP_INDEX_DECODE, T, H, L, B, k, 0)
+ *   (the error word).
  */
 MISA_API misa_status misa_index_decode(const uint16_t* q, const float* w, const uint16_t* keys, int64_t nkeyseq,
                                        int64_t key_seq_stride, const uint16_t* means_hi, const uint16_t* means_lo,

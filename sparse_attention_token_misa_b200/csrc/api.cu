@@ -118,6 +118,7 @@ size_t misa_workspace_bytes(int op, int T, int H, int64_t L, int B, int k, int k
       if (B < 1) return 0;
       return kErrBytes + misa::router_scratch_bytes(T, H, L, B, 1);
     case MISA_OP_INDEX_SCORE:
+    case MISA_OP_INDEX_DECODE:
     case MISA_OP_TOPK:
     case MISA_OP_APPEND_KEYS:
       return kErrBytes;
@@ -130,12 +131,6 @@ size_t misa_workspace_bytes(int op, int T, int H, int64_t L, int B, int k, int k
       if (B < 1) return 0;
       const int64_t M = ceil_div(L, B);
       return kErrBytes + static_cast<size_t>(T) * round_up4(M) * sizeof(float);
-    }
-    case MISA_OP_INDEX_DECODE: {
-      if (T < 1 || L < 1) return 0;
-      const size_t counters = (static_cast<size_t>(T) * 4 + 255) / 256 * 256;
-      const int64_t R = misa::decode_fused_hist_slots(T, L, misa::kDecodeFusedMaxGrid);
-      return kErrBytes + counters + static_cast<size_t>(T) * R * misa::decode_fused_hist_bins() * 4;
     }
     default:
       return 0;
@@ -307,7 +302,7 @@ misa_status misa_index_decode(const uint16_t* q, const float* w, const uint16_t*
     return MISA_ERR_INVALID_ARG;
   if (T < 1 || H < 1 || L < 1 || B < 1 || h < 1 || h > H || k < 1 || nkeyseq < 1 || nmeanseq < 1)
     return MISA_ERR_INVALID_ARG;
-  if (!misa::decode_fused_supported(T, H, h, L, k) || T > MISA_MAX_TOPK_ROWS) return MISA_ERR_UNSUPPORTED;
+  if (!misa::decode_fused_supported(H, h, L) || k > MISA_MAX_TOPK || T > MISA_MAX_TOPK_ROWS) return MISA_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(keys) || !aligned16(means_hi) || !aligned16(means_lo) || !aligned16(scores))
     return MISA_ERR_INVALID_ARG;
   if (key_seq_stride < 0 || key_seq_stride % MISA_HEAD_DIM != 0 || (nkeyseq > 1 && key_seq_stride < L * MISA_HEAD_DIM))
@@ -324,7 +319,6 @@ misa_status misa_index_decode(const uint16_t* q, const float* w, const uint16_t*
     return MISA_ERR_UNSUPPORTED;   // TMA coordinates are int32
   misa_status st = check_ws(workspace, workspace_bytes, misa_workspace_bytes(MISA_OP_INDEX_DECODE, T, H, L, B, k, 0));
   if (st != MISA_OK) return st;
-  uint8_t* base = static_cast<uint8_t*>(workspace) + kErrBytes;
   misa::DecodeArgs a;
   a.q = q;
   a.w = w;
@@ -340,18 +334,19 @@ misa_status misa_index_decode(const uint16_t* q, const float* w, const uint16_t*
   a.T = T;
   a.H = H;
   a.h = h;
-  a.k = k;
   a.B = B;
   a.L = L;
   a.heads = heads;
   a.importance = importance;
   a.scores = scores;
   a.row_stride = scores_row_stride;
-  a.idx = idx;
-  a.counters = reinterpret_cast<unsigned*>(base);
-  a.hist = reinterpret_cast<uint32_t*>(base + (static_cast<size_t>(T) * 4 + 255) / 256 * 256);
   a.err = err_word(workspace);
-  return cuda_status(misa::launch_decode_fused(a, reinterpret_cast<cudaStream_t>(stream)));
+  const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  misa_status rs = cuda_status(misa::launch_decode_fused(a, cs));
+  if (rs != MISA_OK) return rs;
+  // the top-k starts while the last CTAs of the scoring kernel finish and
+  // waits for their rows (programmatic dependent launch)
+  return cuda_status(misa::launch_topk(scores, T, L, scores_row_stride, prefix_len, nullptr, 0, k, idx, cs));
 }
 
 misa_status misa_hier_rerank(const uint16_t* q, const float* w, const uint16_t* keys, int64_t nkeyseq,

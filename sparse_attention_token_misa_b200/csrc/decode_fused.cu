@@ -1,5 +1,4 @@
-// The whole MISA decode step in one kernel: router, routed token scoring and
-// per-query top-k.
+// Router and routed token scoring of a MISA decode step in one kernel.
 //
 // "MISA: Mixture of Indexer Sparse Attention for Long-Context LLM Inference"
 // (gist.science), Methodology: a router scores the heads against mean-pooled
@@ -7,15 +6,14 @@
 // those heads score every prefix token; the top-k tokens are kept.  The
 // library's definitions (misa.h): A[t,h,j] = w[t,h] * ReLU(q[t,h] . mean_j),
 // importance = sum over visible blocks, top-h by rank (ties to the lower head),
-// S[t,s] = sum over the routed heads of w * ReLU(q . k_s), top-k with ties to
-// the lower position, ascending output.
+// S[t,s] = sum over the routed heads of w * ReLU(q . k_s).  The top-k of the
+// score rows is the top-k kernel's, launched right behind this one (topk.cu).
 //
 // Why one kernel: at decode the step is one pass over the keys (HBM-bound),
-// and the router and the top-k are short chains of dependent steps that leave
-// HBM idle when they run as kernels of their own.  Here every CTA streams its
-// key tiles from the start, routes the queries it works on from a buffer of
-// its own while those tiles land, and selects the top-k of the rows it
-// completes at the end, from L2.
+// and the router is a short chain of dependent steps that leaves HBM idle when
+// it runs as a kernel of its own.  Here every CTA starts its key stream as
+// soon as its first router tiles are on their way, and routes the queries it
+// works on from a buffer of its own while the key tiles land.
 //
 // Work: one persistent CTA per SM over the items (query g, key tile j) in
 // contiguous ranges, exactly as the scoring kernel splits them.  Per query the
@@ -36,28 +34,15 @@
 //    the query rows already in shared memory into the B operand; the key tiles
 //    stream through a four-stage ring; the scoring epilogue is the scoring
 //    kernel's (ReLU, head weights, heads summed in ascending order), so the
-//    scores equal misa_index_score's bit for bit given the same heads.  Each
-//    score is also counted in a per-CTA histogram of its order-preserving
-//    key's top 10 bits.
-//  * selection: at the end of its run of a query's tiles the CTA stores its
-//    histogram in the workspace and adds its tile count to the query's
-//    counter; the CTA that completes the count owns the row's top-k, which it
-//    runs once all its own tiles are scored, with the (then idle) key ring as
-//    scratch: it sums the row's histograms, finds the bin of the k-th largest
-//    score, reads the row once from L2 (entries above that bin into a position
-//    bitmap, entries in it into a candidate list), resolves the exact
-//    threshold inside the bin by two more 11-bit radix digits over the
-//    candidates, takes the ties lowest position first through a tie bitmap,
-//    and writes the positions in ascending order.  When the bin holds more
-//    entries than the list, the digits are counted from the row instead.  The
-//    result is exact for any input.
+//    scores equal misa_index_score's bit for bit given the same heads.  The
+//    score rows stay in L2 for the top-k kernel.
 //
-// Roles (352 threads): warps 0-3 scoring epilogue and selection (TMEM lane
-// quarter = warp), warps 4-7 router epilogue (lane quarter = warp - 4), warp 8
-// TMEM allocation + single-thread MMA issue, warp 9 one thread for the key
-// tiles, warp 10 one thread for the query rows and router tiles.  Every wait is
-// bounded; a wait that gives up records MISA_DEVERR_TIMEOUT, raises a CTA-wide
-// abort flag and the roles stop; TMEM is freed before exit.
+// Roles (352 threads): warps 0-3 scoring epilogue (TMEM lane quarter = warp),
+// warps 4-7 router epilogue (lane quarter = warp - 4), warp 8 TMEM allocation
+// + single-thread MMA issue, warp 9 one thread for the key tiles, warp 10 one
+// thread for the query rows and router tiles.  Every wait is bounded; a wait
+// that gives up records MISA_DEVERR_TIMEOUT, raises a CTA-wide abort flag and
+// the roles stop; TMEM is freed before exit.
 #include <algorithm>
 #include <cstring>
 
@@ -79,50 +64,35 @@ constexpr int kFRouteWarp0 = 4;                 // router epilogue (warps 4-7)
 constexpr int kFMmaWarp = 8;
 constexpr int kFKeyWarp = 9;
 constexpr int kFRouterTmaWarp = 10;
-constexpr int kFBins = 1024;                    // first digit: the top 10 key bits
-constexpr int kFBinShift = 22;
-constexpr int kFLoBin = 2;                      // bins below hold only NaN and -inf (key <= 0x007FFFFF)
-constexpr int kFCandCap = 9216;                 // threshold-bin entries resolved in shared memory
-constexpr int kFMaxL = 65536;                   // longest row (position bitmaps)
+constexpr int kFMaxL = 65536;                   // longest row
 constexpr int kFMaxNR = 64;                     // router columns (H <= 64)
-constexpr int kFMaxGroups = 1024;               // queries one CTA may work on
 constexpr int kFTmemCols = 256;                 // 2 router accumulators (<= 64 each) + 2 x 16 scoring
 
 // shared memory map (offsets from a 1024-byte aligned base)
-constexpr int kFOffRing = 0;                                      // [4] key tiles; selection scratch at the end
+constexpr int kFOffRing = 0;                                      // [4] key tiles
 constexpr int kFOffRBuf = kFOffRing + kFStages * kFTileBytes;     // [2] router tiles
 constexpr int kFOffQall = kFOffRBuf + kFRSlots * kFTileBytes;     // [NR rows x 128] router B operand
 constexpr int kFOffSQ = kFOffQall + kFMaxNR * kD * 2;             // 2 x [16 rows x 128] scoring B operand
 constexpr int kFSQBytes = kFHP * kD * 2;                          // 4 KB
-constexpr int kFOffHist = kFOffSQ + 2 * kFSQBytes;                // [kFBins] u32 per-CTA histogram
-constexpr int kFOffRed = kFOffHist + kFBins * 4;                  // [4][64] f32 router warp partial sums
+constexpr int kFOffRed = kFOffSQ + 2 * kFSQBytes;                 // [4][64] f32 router warp partial sums
 constexpr int kFOffImp = kFOffRed + 4 * kFMaxNR * 4;              // [64] f32 head sums
 constexpr int kFOffHeads = kFOffImp + kFMaxNR * 4;                // [16] i32 routed heads (router epilogue)
 constexpr int kFOffW = kFOffHeads + kFHP * 4;                     // [2][16] f32 routed weights
 constexpr int kFOffMisc = kFOffW + 2 * kFHP * 4;                  // [64] u32 scratch words
-constexpr int kFOffFin = kFOffMisc + 64 * 4;                      // [kFMaxGroups / 32] u32 rows to select
-constexpr int kFOffBar = kFOffFin + kFMaxGroups / 8;
+constexpr int kFOffBar = kFOffMisc + 64 * 4;
 // full[4] empty[4] rbfull[2] rbempty[2] qa_full qa_empty, then pairs rfull
 // rempty tfull tempty qfull qempty wempty, then done
-constexpr int kFNumBars = 2 * kFStages + 2 * kFRSlots + 2 + 2 * 7 + 1 + 2;   // + 2 row-chunk barriers
+constexpr int kFNumBars = 2 * kFStages + 2 * kFRSlots + 2 + 2 * 7 + 1;
 constexpr int kFOffTmem = kFOffBar + kFNumBars * 8;
 constexpr int kFSmemBytes = kFOffTmem + 16 + 1024;                // + alignment slack
-// selection scratch inside the key ring (used once the CTA's tiles are scored)
-constexpr int kFScrBits = 0;                                      // [kFMaxL / 32] u32
-constexpr int kFScrTBits = kFScrBits + kFMaxL / 8;                // [kFMaxL / 32] u32
-constexpr int kFScrRHist = kFScrTBits + kFMaxL / 8;               // [2048] u32
-constexpr int kFScrCand = kFScrRHist + 2048 * 4;                  // [kFCandCap] (key, position) u32 pairs
-constexpr int kFScrStage = kFScrCand + kFCandCap * 8;             // [2][4096] f32 row chunks
-static_assert(kFScrStage + 2 * 4096 * 4 <= kFStages * kFTileBytes, "selection scratch fits the ring");
 static_assert(kFSmemBytes <= 232448, "shared memory per CTA");
-static_assert(4 * 12 <= 64, "append mask bits per batch");
 
 struct FusedParams {
   const uint16_t* q;
   const float* w;
   const int32_t* seq_of;
   const int32_t* prefix_len;
-  int T, H, h, k;
+  int T, H, h;
   int64_t L;
   int B, M, n_rt;           // block size, blocks per sequence, router tiles (128 blocks) per query
   int64_t key_seq_rows;     // key rows between sequences in the key map
@@ -130,22 +100,14 @@ struct FusedParams {
   int64_t nkeyseq, nmeanseq;
   int tpg;                  // key tiles per query
   int64_t n_items;
-  int R;                    // histogram slots per query
   int32_t* heads;           // [T][h] out
   float* importance;        // [T][H] out or NULL
-  float* scores;            // [T][row_stride] out (also the selection's input)
+  float* scores;            // [T][row_stride] out
   int64_t row_stride;
-  int32_t* idx;             // [T][k] out
-  unsigned* counters;       // [T] tiles done per query (zero on entry)
-  uint32_t* hist;           // [T][R][kFBins] per-segment histograms
   uint32_t* err;
 };
 
 __device__ __forceinline__ int64_t f_item_begin(int64_t n_items, int c, int G) { return n_items * c / G; }
-// the CTA whose item range holds item i (ranges [n c / G, n (c+1) / G))
-__device__ __forceinline__ int f_cta_of(int64_t i, int64_t n_items, int G) {
-  return static_cast<int>(((i + 1) * G - 1) / n_items);
-}
 
 __device__ __forceinline__ int f_seq_checked(const FusedParams& p, int g, int64_t nseq) {
   int64_t s = p.seq_of[g];
@@ -169,11 +131,6 @@ __device__ __forceinline__ int f_visible_blocks(const FusedParams& p, int g) {
   if (pl >= p.L) return p.M;
   if (pl <= 0) return 0;
   return static_cast<int>(pl / p.B);
-}
-
-__device__ __forceinline__ uint32_t f_sel_key(float v) {
-  const bool ok = v == v && v > -__int_as_float(0x7f800000);
-  return ok ? float_key(v) : 0u;
 }
 
 // Sum over the lanes of a warp of NR per-lane values (one per head), leaving
@@ -211,362 +168,6 @@ constexpr int f_lane_heads() {
   return NR >= 32 ? NR / 32 : 1;
 }
 
-// Exclusive prefix sum over the 128 epilogue threads (uses 4 words at ws).
-__device__ __forceinline__ uint32_t f_block_excl_scan(uint32_t x, uint32_t* ws, uint32_t* total) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  uint32_t inc = x;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
-    if (lane >= o) inc += y;
-  }
-  if (lane == 31) ws[warp] = inc;
-  named_bar_sync(1, kFEpiThreads);
-  uint32_t before = 0, all = 0;
-#pragma unroll
-  for (int w2 = 0; w2 < 4; ++w2) {
-    const uint32_t t = ws[w2];
-    if (w2 < warp) before += t;
-    all += t;
-  }
-  named_bar_sync(1, kFEpiThreads);
-  *total = all;
-  return before + inc - x;
-}
-
-// The bin holding the need-th largest entry of hist[lo_bin, nb): returns the
-// bin and sets *above = entries in higher bins.  128 threads; nb % 128 == 0.
-__device__ __forceinline__ int f_find_bin(const uint32_t* hist, int nb, int lo_bin, uint32_t need, uint32_t* ws,
-                                          uint32_t* above) {
-  const int tid = threadIdx.x;
-  const int per = nb / kFEpiThreads;
-  // thread tid owns bins [nb - (tid + 1) per, nb - tid per): thread 0 the highest
-  const int b_hi = nb - tid * per;
-  uint32_t local = 0;
-  for (int b = b_hi - per; b < b_hi; ++b)
-    if (b >= lo_bin) local += hist[b];
-  uint32_t tot;
-  const uint32_t before = f_block_excl_scan(local, ws, &tot);  // entries in higher bins
-  if (before < need && need <= before + local) {
-    uint32_t acc = before;
-    for (int b = b_hi - 1; b >= b_hi - per; --b) {
-      const uint32_t c = b >= lo_bin ? hist[b] : 0u;
-      if (acc + c >= need) {
-        ws[4] = static_cast<uint32_t>(b);
-        ws[5] = acc;
-        break;
-      }
-      acc += c;
-    }
-  }
-  named_bar_sync(1, kFEpiThreads);
-  const int bin = static_cast<int>(ws[4]);
-  *above = ws[5];
-  named_bar_sync(1, kFEpiThreads);
-  return bin;
-}
-
-// Row chunks staged in shared memory for the selection passes: the row is
-// read by bulk copies (kFChunk entries each, two buffers, completion on an
-// mbarrier per buffer), so the loads are asynchronous and many bytes are in
-// flight whatever the compiler does with registers.
-struct RowStage {
-  float* buf[2];
-  uint64_t* bar[2];
-  uint32_t fills[2];   // completed fills per buffer (same in every thread)
-  uint32_t* err;
-  volatile uint32_t* abort;
-};
-constexpr int kFChunk = 4096;   // 16 KB
-
-// tid 0 starts the copy of chunk ch (entries [ch kFChunk, min(n, ...))) into
-// buffer ch & 1; the byte count is rounded up to 16 (rows are padded to a
-// multiple of 4 entries).
-__device__ __forceinline__ void f_stage_issue(RowStage& st, const float* row, int n, int ch) {
-  if (threadIdx.x != 0) return;
-  const int first = ch * kFChunk;
-  const int cnt = min(kFChunk, n - first);
-  const uint32_t bytes = static_cast<uint32_t>((cnt + 3) / 4 * 16);
-  uint64_t* b = st.bar[ch & 1];
-  mbar_arrive_expect_tx(b, bytes);
-  bulk_copy_g2s(st.buf[ch & 1], row + first, bytes, b);
-}
-
-// One pass over the first n entries of a score row by the 128 epilogue
-// threads, from the shared-memory chunks.  Warp w takes the 32-position words
-// w, w + 4, ... of each chunk, kFWordsPerStep of them per step for
-// instruction-level parallelism, one entry per lane: f(pos, key) returns a code
-// (bit 0: set in `bits`, bit 1: set in `tbits`, bit 2: append (key, pos) to the
-// warp's candidate region); a ballot per code bit gives the bitmap word
-// directly and the append slots (no atomics, no scans).  cand: per-warp regions
-// of kFWarpCand (key, pos) pairs; ccount: per-warp counts (kept in a register,
-// may exceed kFWarpCand: the excess is not stored).  g(ok, pos, key) is called
-// for every position for side work.
-constexpr int kFWarpCand = kFCandCap / 4;
-constexpr int kFWordsPerStep = 4;
-template <class F, class Gf>
-__device__ __forceinline__ void f_row_pass(RowStage& st, const float* row, int n, uint32_t* bits, uint32_t* tbits,
-                                           uint32_t* cand, uint32_t* ccount, F f, Gf gside) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const uint32_t lt = (1u << lane) - 1u;
-  if (n <= 0) return;
-  const int nch = (n + kFChunk - 1) / kFChunk;
-  uint32_t cw = cand != nullptr ? ccount[warp] : 0u;
-  uint32_t* wcand = cand != nullptr ? cand + 2 * warp * kFWarpCand : nullptr;
-  f_stage_issue(st, row, n, 0);
-  if (nch > 1) f_stage_issue(st, row, n, 1);
-  for (int ch = 0; ch < nch; ++ch) {
-    const int bi = ch & 1;
-    if (!mbar_wait(st.bar[bi], st.fills[bi] & 1u, st.err, st.abort)) {
-      // a copy that never lands: the row is left unselected (error recorded)
-    }
-    ++st.fills[bi];
-    const float* src = st.buf[bi];
-    const int first = ch * kFChunk;
-    const int cn = min(kFChunk, n - first);
-    const int nwc = (cn + 31) >> 5;
-    for (int w0 = warp; w0 < nwc; w0 += 4 * kFWordsPerStep) {   // (warp-uniform)
-      float x[kFWordsPerStep];
-#pragma unroll
-      for (int u = 0; u < kFWordsPerStep; ++u) {
-        const int lp = (w0 + 4 * u) * 32 + lane;
-        x[u] = lp < cn ? src[lp] : -__int_as_float(0x7f800000);
-      }
-#pragma unroll
-      for (int u = 0; u < kFWordsPerStep; ++u) {
-        const int word = w0 + 4 * u;
-        if (word >= nwc) break;   // (warp-uniform)
-        const int lp = word * 32 + lane;
-        const bool ok = lp < cn;
-        const int pos = first + lp;
-        const uint32_t key = ok ? f_sel_key(x[u]) : 0u;
-        const uint32_t code = ok ? f(pos, key) : 0u;
-        const uint32_t m0 = __ballot_sync(0xffffffffu, code & 1u);
-        const uint32_t m1 = __ballot_sync(0xffffffffu, code & 2u);
-        const uint32_t m2 = __ballot_sync(0xffffffffu, code & 4u);
-        if (lane == 0) {
-          const int gw = (first >> 5) + word;
-          if (m0) bits[gw] |= m0;
-          if (m1) tbits[gw] |= m1;
-        }
-        if (m2) {
-          const uint32_t slot = cw + __popc(m2 & lt);
-          if ((code & 4u) && slot < static_cast<uint32_t>(kFWarpCand)) {
-            wcand[2 * slot] = key;
-            wcand[2 * slot + 1] = static_cast<uint32_t>(pos);
-          }
-          cw += __popc(m2);
-        }
-        gside(ok, pos, key);
-      }
-    }
-    named_bar_sync(1, kFEpiThreads);   // the buffer is read: it may be refilled
-    if (ch + 2 < nch) f_stage_issue(st, row, n, ch + 2);
-  }
-  if (cand != nullptr && lane == 0) ccount[warp] = cw;
-}
-
-// The float whose order-preserving key is k (inverse of float_key).
-__device__ __forceinline__ float f_key_to_float(uint32_t k) {
-  const uint32_t u = (k & 0x80000000u) ? (k ^ 0x80000000u) : ~k;
-  return __uint_as_float(u);
-}
-
-// The common first pass of the selection: entries x >= hiv (none when `top`)
-// into `bits`, entries lov <= x < hiv into the per-warp candidate regions (as
-// (key, position)).  Two comparisons and two ballots per entry; NaN compares
-// false and is never taken.
-__device__ __forceinline__ void f_row_pass_values(RowStage& st, const float* row, int n, uint32_t* bits,
-                                                  uint32_t* cand, uint32_t* ccount, float lov, float hiv,
-                                                  bool top) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const uint32_t lt = (1u << lane) - 1u;
-  if (n <= 0) return;
-  const int nch = (n + kFChunk - 1) / kFChunk;
-  uint32_t cw = ccount[warp];
-  uint32_t* wcand = cand + 2 * warp * kFWarpCand;
-  f_stage_issue(st, row, n, 0);
-  if (nch > 1) f_stage_issue(st, row, n, 1);
-  for (int ch = 0; ch < nch; ++ch) {
-    const int bi = ch & 1;
-    mbar_wait(st.bar[bi], st.fills[bi] & 1u, st.err, st.abort);   // (a copy that never lands: error recorded)
-    ++st.fills[bi];
-    const float* src = st.buf[bi];
-    const int first = ch * kFChunk;
-    const int cn = min(kFChunk, n - first);
-    const int nwc = (cn + 31) >> 5;
-    for (int w0 = warp; w0 < nwc; w0 += 4 * kFWordsPerStep) {   // (warp-uniform)
-      float x[kFWordsPerStep];
-#pragma unroll
-      for (int u = 0; u < kFWordsPerStep; ++u) {
-        const int lp = (w0 + 4 * u) * 32 + lane;
-        x[u] = lp < cn ? src[lp] : __int_as_float(0x7fc00000);   // NaN: neither above nor in
-      }
-#pragma unroll
-      for (int u = 0; u < kFWordsPerStep; ++u) {
-        const int word = w0 + 4 * u;
-        if (word >= nwc) break;   // (warp-uniform)
-        const bool above = !top && x[u] >= hiv;
-        const bool in = x[u] >= lov && !above;
-        const uint32_t ma = __ballot_sync(0xffffffffu, above);
-        const uint32_t mi = __ballot_sync(0xffffffffu, in);
-        if (lane == 0 && ma) bits[(first >> 5) + word] |= ma;
-        if (mi) {
-          const uint32_t slot = cw + __popc(mi & lt);
-          if (in && slot < static_cast<uint32_t>(kFWarpCand)) {
-            wcand[2 * slot] = f_sel_key(x[u]);
-            wcand[2 * slot + 1] = static_cast<uint32_t>(first + word * 32 + lane);
-          }
-          cw += __popc(mi);
-        }
-      }
-    }
-    named_bar_sync(1, kFEpiThreads);   // the buffer is read: it may be refilled
-    if (ch + 2 < nch) f_stage_issue(st, row, n, ch + 2);
-  }
-  if (lane == 0) ccount[warp] = cw;
-}
-
-// Top-k of one finished score row, by the 128 scoring-epilogue threads.  hist:
-// the row's summed first-digit histogram (shared, kFBins bins); rhist (2048
-// bins), bits, tbits, cand, ws: shared scratch.
-__device__ void f_select_row(const FusedParams& p, int g, const uint32_t* hist, uint32_t* rhist, uint32_t* bits,
-                             uint32_t* tbits, uint32_t* cand, uint32_t* ws, RowStage& st) {
-  const int tid = threadIdx.x;
-  const int n = f_valid_len(p, g);
-  const float* row = p.scores + static_cast<int64_t>(g) * p.row_stride;
-  const uint32_t k = static_cast<uint32_t>(p.k);
-  const int nwords = (n + 31) >> 5;
-  for (int i = tid; i < nwords; i += kFEpiThreads) {
-    bits[i] = 0u;
-    tbits[i] = 0u;
-  }
-  // selectable entries: keys above -inf's key, i.e. bins >= kFLoBin (the bins
-  // below hold only NaN and -inf)
-  uint32_t vcount = 0;
-  for (int b = kFLoBin + tid; b < kFBins; b += kFEpiThreads) vcount += hist[b];
-  uint32_t nvalid;
-  (void)f_block_excl_scan(vcount, ws, &nvalid);   // (its barriers also order the zeroing above)
-  auto no_side = [](bool, int, uint32_t) {};
-  if (nvalid <= k) {
-    // every selectable entry
-    // every selectable entry: x >= -FLT_MAX (not NaN, not -inf)
-    if (tid < 4) ws[8 + tid] = 0u;
-    named_bar_sync(1, kFEpiThreads);
-    f_row_pass_values(st, row, n, bits, cand, ws + 8, __int_as_float(0x7f800000), -__int_as_float(0x7f7fffff),
-                      false);
-  } else {
-    uint32_t above = 0;
-    const int bstar = f_find_bin(hist, kFBins, kFLoBin, k, ws, &above);
-    const uint32_t need = k - above;       // entries to take from bin bstar, >= 1
-    const uint32_t ub = static_cast<uint32_t>(bstar);
-    // one pass: entries above the bin into the bitmap, entries in it into the
-    // per-warp candidate regions (counts in ws[8 .. 12))
-    uint32_t* ccount = ws + 8;
-    if (tid < 4) ccount[tid] = 0u;
-    named_bar_sync(1, kFEpiThreads);
-    // the bin's edges as values (the key order is the value order, -0 == +0):
-    // an entry is above the bin iff x >= hiv, in it iff lov <= x < hiv
-    const float lov = f_key_to_float(ub << kFBinShift);
-    const bool top = ub + 1u >= static_cast<uint32_t>(kFBins);
-    const float hiv = top ? __int_as_float(0x7fc00000) : f_key_to_float((ub + 1u) << kFBinShift);
-    f_row_pass_values(st, row, n, bits, cand, ccount, lov, hiv, top);
-    named_bar_sync(1, kFEpiThreads);
-    uint32_t wc[4];
-    bool in_list = true;
-#pragma unroll
-    for (int w2 = 0; w2 < 4; ++w2) {
-      wc[w2] = ccount[w2];
-      in_list = in_list && wc[w2] <= static_cast<uint32_t>(kFWarpCand);
-    }
-    // candidate i (< kFCandCap) is stored iff its slot in its warp's region is used
-    auto cand_ok = [&](int i) { return static_cast<uint32_t>(i % kFWarpCand) < wc[i / kFWarpCand]; };
-    // exact threshold inside the bin: two more 11-bit digits
-    uint32_t need2 = need, pre = ub << kFBinShift, pre_mask = 0xFFFFFFFFu << kFBinShift;
-    for (int round = 0; round < 2; ++round) {
-      const int shift = round == 0 ? 11 : 0;
-      constexpr int nb = 2048;
-      for (int b = tid; b < nb; b += kFEpiThreads) rhist[b] = 0u;
-      named_bar_sync(1, kFEpiThreads);
-      if (in_list) {
-        for (int i = tid; i < kFCandCap; i += kFEpiThreads) {
-          if (!cand_ok(i)) continue;
-          const uint32_t key = cand[2 * i];
-          if ((key & pre_mask) == pre) atomicAdd(&rhist[(key >> shift) & (nb - 1)], 1u);
-        }
-      } else {
-        // more entries in the bin than the list holds: count them from the row
-        f_row_pass(st, row, n, bits, tbits, nullptr, nullptr, [](int, uint32_t) { return 0u; },
-                   [rhist, pre, pre_mask, shift](bool ok, int, uint32_t key) {
-                     if (ok && (key & pre_mask) == pre && key > kNegInfKey)
-                       atomicAdd(&rhist[(key >> shift) & (nb - 1)], 1u);
-                   });
-      }
-      named_bar_sync(1, kFEpiThreads);
-      uint32_t ab;
-      const int d = f_find_bin(rhist, nb, 0, need2, ws, &ab);
-      need2 -= ab;
-      pre |= static_cast<uint32_t>(d) << shift;
-      pre_mask |= static_cast<uint32_t>(nb - 1) << shift;
-    }
-    const uint32_t tau = pre;       // the exact key of the k-th largest entry
-    const uint32_t need_eq = need2; // entries equal to tau to take, lowest positions first
-    // the bin's entries above tau into the bitmap, its ties into the tie bitmap
-    if (in_list) {
-      for (int i = tid; i < kFCandCap; i += kFEpiThreads) {
-        if (!cand_ok(i)) continue;
-        const uint32_t key = cand[2 * i], pos = cand[2 * i + 1];
-        if (key > tau) atomicOr(&bits[pos >> 5], 1u << (pos & 31));
-        else if (key == tau) atomicOr(&tbits[pos >> 5], 1u << (pos & 31));
-      }
-    } else {
-      f_row_pass(st, row, n, bits, tbits, nullptr, nullptr,
-                 [ub, tau](int, uint32_t key) {
-                   return ((key >> kFBinShift) == ub && key > tau ? 1u : 0u) | (key == tau ? 2u : 0u);
-                 },
-                 no_side);
-    }
-    named_bar_sync(1, kFEpiThreads);
-    // the first need_eq ties in position order: contiguous word ranges per
-    // thread, counted, scanned, then taken
-    const int wchunk = (nwords + kFEpiThreads - 1) / kFEpiThreads;
-    const int w0 = tid * wchunk, w1 = min(nwords, w0 + wchunk);
-    uint32_t cnt = 0;
-    for (int i = w0; i < w1; ++i) cnt += __popc(tbits[i]);
-    uint32_t tot;
-    uint32_t r = f_block_excl_scan(cnt, ws, &tot);
-    for (int i = w0; i < w1 && r < need_eq; ++i) {
-      uint32_t word = tbits[i], take = 0u;
-      while (word && r < need_eq) {
-        const uint32_t low = word & (~word + 1u);
-        take |= low;
-        word ^= low;
-        ++r;
-      }
-      if (take) bits[i] |= take;   // this thread owns words [w0, w1)
-    }
-  }
-  named_bar_sync(1, kFEpiThreads);
-  // positions out in ascending order
-  int32_t* out = p.idx + static_cast<int64_t>(g) * p.k;
-  const int wchunk = (nwords + kFEpiThreads - 1) / kFEpiThreads;
-  const int w0 = tid * wchunk, w1 = min(nwords, w0 + wchunk);
-  uint32_t cnt = 0;
-  for (int i = w0; i < w1; ++i) cnt += __popc(bits[i]);
-  uint32_t total;
-  uint32_t o = f_block_excl_scan(cnt, ws, &total);
-  for (int i = w0; i < w1; ++i) {
-    uint32_t word = bits[i];
-    while (word && o < k) {
-      const int b = __ffs(word) - 1;
-      out[o++] = i * 32 + b;
-      word &= word - 1;
-    }
-  }
-  for (uint32_t i = min(total, k) + tid; i < k; i += kFEpiThreads) out[i] = -1;
-  named_bar_sync(1, kFEpiThreads);
-}
-
 template <int NR>
 __global__ void __launch_bounds__(kFThreads, 1)
 decode_fused_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap hmap,
@@ -578,13 +179,11 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
   uint8_t* rbuf = smem + kFOffRBuf;
   uint8_t* qall = smem + kFOffQall;
   uint8_t* sq = smem + kFOffSQ;
-  uint32_t* hist = reinterpret_cast<uint32_t*>(smem + kFOffHist);
   float* red = reinterpret_cast<float*>(smem + kFOffRed);
   float* imp = reinterpret_cast<float*>(smem + kFOffImp);
   int32_t* heads_r = reinterpret_cast<int32_t*>(smem + kFOffHeads);
   float* w_s = reinterpret_cast<float*>(smem + kFOffW);
-  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + kFOffMisc);   // [0,8) router, [8,64) scoring epilogue
-  uint32_t* fin = reinterpret_cast<uint32_t*>(smem + kFOffFin);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + kFOffMisc);   // [0,8) router, [63] key-stream start flag
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kFOffBar);
   uint64_t* full = bars;                        // [4] key tile landed
   uint64_t* empty = full + kFStages;            // [4] MMAs reading the key tile done
@@ -600,8 +199,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
   uint64_t* qempty = qfull + 2;                 // [2] MMAs of the query using the staged rows done
   uint64_t* wempty = qempty + 2;                // [2] scoring epilogue took the weights
   uint64_t* done = wempty + 2;
-  uint64_t* sbar = done + 1;                    // [2] row chunk landed (selection)
-  static_assert(2 * kFStages + 2 * kFRSlots + 2 + 2 * 7 + 1 + 2 == kFNumBars, "barrier layout");
+  static_assert(2 * kFStages + 2 * kFRSlots + 2 + 2 * 7 + 1 == kFNumBars, "barrier layout");
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kFOffTmem);
   volatile uint32_t* abort = reinterpret_cast<volatile uint32_t*>(smem + kFOffTmem + 4);
 
@@ -630,12 +228,9 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
       mbar_init(&wempty[a], kFEpiThreads);
     }
     mbar_init(done, 1);
-    mbar_init(&sbar[0], 1);
-    mbar_init(&sbar[1], 1);
     *abort = 0u;
     fence_mbar_init();
   }
-  for (int i = tid; i < kFMaxGroups / 32; i += kFThreads) fin[i] = 0u;
   if (tid == 0) misc[63] = 0u;   // router producer -> key producer: the first router loads are issued
   if (warp == kFMmaWarp) {
     tmem_alloc(tmem_slot, kFTmemCols);
@@ -935,7 +530,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
       named_bar_sync(2, kFEpiThreads);   // heads_r / imp / red are reused by the next query
     }
   } else {
-    // ------------------------------------------------------------ scoring epilogue (warps 0-3) and selection
+    // ------------------------------------------------------------ scoring epilogue (warps 0-3)
     const uint32_t t_lane = tmem_base + (static_cast<uint32_t>(warp * 32) << 16);
     int64_t acc = 0;
     bool skip = false;
@@ -948,15 +543,12 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
 #pragma unroll
       for (int i = 0; i < kFHP; ++i) wv[i] = w_s[qb * kFHP + i];
       mbar_arrive(&wempty[qb]);
-      for (int b = tid; b < kFBins; b += kFEpiThreads) hist[b] = 0u;
       const int plen = f_valid_len(p, g);
       float* rowp = p.scores + static_cast<int64_t>(g) * p.row_stride;
-      named_bar_sync(1, kFEpiThreads);
-      const int64_t a = run_begin(gl), b = run_end(gl);
-      for (int64_t item = a; item < b; ++item, ++acc) {
+      for (int64_t item = run_begin(gl); item < run_end(gl); ++item, ++acc) {
         const int ta = static_cast<int>(acc & 1);
         const bool ok = !skip && mbar_wait(&tfull[ta], static_cast<uint32_t>((acc >> 1) & 1), p.err, abort);
-        if (!__all_sync(0xffffffffu, ok)) {   // warp-uniform, for the warp-wide steps below
+        if (!__all_sync(0xffffffffu, ok)) {   // warp-uniform, for the warp-wide TMEM load
           skip = true;
           continue;
         }
@@ -972,79 +564,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
         const int j = static_cast<int>(item - static_cast<int64_t>(g) * tpg);
         const int pos2 = j * kFTileM + r;
         if (pos2 < p.L) rowp[pos2] = pos2 < plen ? sacc : -__int_as_float(0x7f800000);   // stays in L2
-        // the score's histogram bin; lanes that share a bin add once
-        const bool counted = pos2 < plen;
-        const uint32_t bin = counted ? (f_sel_key(sacc) >> kFBinShift) : 0xFFFFFFFFu;
-        const unsigned same = __match_any_sync(0xffffffffu, bin);
-        if (counted && (__ffs(same) - 1) == lane) atomicAdd(&hist[bin], static_cast<uint32_t>(__popc(same)));
       }
-      // the run of this query ends: store the histogram, count the tiles
-      named_bar_sync(1, kFEpiThreads);
-      const int seg = f_cta_of(a, p.n_items, G) - f_cta_of(static_cast<int64_t>(g) * tpg, p.n_items, G);
-      if (seg >= 0 && seg < p.R) {   // (always: the host sizes R for the grid)
-        uint32_t* slot = p.hist + (static_cast<int64_t>(g) * p.R + seg) * kFBins;
-        for (int b2 = tid; b2 < kFBins / 4; b2 += kFEpiThreads)
-          reinterpret_cast<uint4*>(slot)[b2] = reinterpret_cast<const uint4*>(hist)[b2];
-      } else if (tid == 0) {
-        record_error(p.err, MISA_DEVERR_BAD_INDEX);
-        *abort = 1u;
-      }
-      __threadfence();
-      named_bar_sync(1, kFEpiThreads);
-      if (tid == 0) {
-        const unsigned n_run = static_cast<unsigned>(b - a);
-        if (!skip && !*abort && atomicAdd(&p.counters[g], n_run) + n_run == static_cast<unsigned>(tpg) &&
-            gl < kFMaxGroups)
-          fin[gl >> 5] |= 1u << (gl & 31);
-      }
-    }
-    // ---- the rows this CTA completed: top-k, with the idle key ring as scratch
-    named_bar_sync(1, kFEpiThreads);
-    uint32_t* bits = reinterpret_cast<uint32_t*>(ring + kFScrBits);
-    uint32_t* tbits = reinterpret_cast<uint32_t*>(ring + kFScrTBits);
-    uint32_t* rhist = reinterpret_cast<uint32_t*>(ring + kFScrRHist);
-    uint32_t* cand = reinterpret_cast<uint32_t*>(ring + kFScrCand);
-    RowStage st;
-    st.buf[0] = reinterpret_cast<float*>(ring + kFScrStage);
-    st.buf[1] = st.buf[0] + kFChunk;
-    st.bar[0] = &sbar[0];
-    st.bar[1] = &sbar[1];
-    st.fills[0] = st.fills[1] = 0u;
-    st.err = p.err;
-    st.abort = abort;
-    fence_proxy_async_smem();   // the ring's earlier contents were written and read through the async proxy
-    for (int gl = 0; gl < ng && gl < kFMaxGroups; ++gl) {
-      if (!(fin[gl >> 5] & (1u << (gl & 31)))) continue;   // (uniform: shared flag)
-      const int g = g0 + gl;
-      __threadfence();
-      const int nseg = min(p.R, f_cta_of(static_cast<int64_t>(g + 1) * tpg - 1, p.n_items, G) -
-                                    f_cta_of(static_cast<int64_t>(g) * tpg, p.n_items, G) + 1);
-      const uint32_t* base = p.hist + static_cast<int64_t>(g) * p.R * kFBins;
-      // sum the row's histograms: each thread 8 bins (two uint4) of every segment, loads batched
-      uint4 s0 = make_uint4(0u, 0u, 0u, 0u), s1 = s0;
-      for (int sg0 = 0; sg0 < nseg; sg0 += 8) {
-        uint4 t0[8], t1[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          if (sg0 + u < nseg) {
-            const uint4* src = reinterpret_cast<const uint4*>(base + static_cast<int64_t>(sg0 + u) * kFBins);
-            t0[u] = __ldcg(src + 2 * tid);
-            t1[u] = __ldcg(src + 2 * tid + 1);
-          } else {
-            t0[u] = make_uint4(0u, 0u, 0u, 0u);
-            t1[u] = t0[u];
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          s0.x += t0[u].x; s0.y += t0[u].y; s0.z += t0[u].z; s0.w += t0[u].w;
-          s1.x += t1[u].x; s1.y += t1[u].y; s1.z += t1[u].z; s1.w += t1[u].w;
-        }
-      }
-      reinterpret_cast<uint4*>(hist)[2 * tid] = s0;
-      reinterpret_cast<uint4*>(hist)[2 * tid + 1] = s1;
-      named_bar_sync(1, kFEpiThreads);
-      f_select_row(p, g, hist, rhist, bits, tbits, cand, misc + 8, st);
     }
   }
 
@@ -1056,24 +576,8 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
 
 }  // namespace
 
-int64_t decode_fused_hist_slots(int T, int64_t L, int sms_bound) {
-  const int64_t tpg = (L + kFTileM - 1) / kFTileM;
-  const int64_t n = static_cast<int64_t>(T) * tpg;
-  int64_t per = n / sms_bound;
-  if (per < 1) per = 1;
-  int64_t R = (tpg + per - 1) / per + 1;
-  return R < tpg ? R : tpg;
-}
-
-int decode_fused_hist_bins() { return kFBins; }
-
-bool decode_fused_supported(int T, int H, int h, int64_t L, int k) {
-  if (H < 1 || H > kFMaxNR || h < 1 || h > kFHP || h > H || L < 1 || L > kFMaxL || k < 1 || k > MISA_MAX_TOPK)
-    return false;
-  // queries one CTA works on (the grid is at most one CTA per SM, at least one)
-  const int64_t tpg = (L + kFTileM - 1) / kFTileM;
-  const int64_t per_cta = static_cast<int64_t>(T) * tpg;   // with a grid of one
-  return (per_cta + tpg - 1) / tpg + 1 <= kFMaxGroups || T <= kFMaxGroups;
+bool decode_fused_supported(int H, int h, int64_t L) {
+  return H >= 1 && H <= kFMaxNR && h >= 1 && h <= kFHP && h <= H && L >= 1 && L <= kFMaxL;
 }
 
 cudaError_t launch_decode_fused(const DecodeArgs& a, cudaStream_t stream) {
@@ -1087,7 +591,6 @@ cudaError_t launch_decode_fused(const DecodeArgs& a, cudaStream_t stream) {
   p.T = a.T;
   p.H = a.H;
   p.h = a.h;
-  p.k = a.k;
   p.L = a.L;
   p.B = a.B;
   p.M = static_cast<int>((a.L + a.B - 1) / a.B);
@@ -1102,15 +605,8 @@ cudaError_t launch_decode_fused(const DecodeArgs& a, cudaStream_t stream) {
   p.importance = a.importance;
   p.scores = a.scores;
   p.row_stride = a.row_stride;
-  p.idx = a.idx;
-  p.counters = a.counters;
-  p.hist = a.hist;
   p.err = a.err;
   const int64_t grid = std::min<int64_t>(p.n_items, sms);
-  if (grid > kDecodeFusedMaxGrid) return cudaErrorInvalidValue;
-  // queries per CTA within the deferred-selection flags
-  if ((p.n_items + grid - 1) / grid / p.tpg + 2 > kFMaxGroups) return cudaErrorInvalidValue;
-  p.R = static_cast<int>(decode_fused_hist_slots(a.T, a.L, kDecodeFusedMaxGrid));
 
   // tensor maps: keys (128-row tiles as 64-row boxes, 128-byte swizzle), the
   // bf16 hi / lo block means (same layout), the query rows (box of H rows)
@@ -1123,8 +619,6 @@ cudaError_t launch_decode_fused(const DecodeArgs& a, cudaStream_t stream) {
       !encode_2d_map(&qmap, true, a.q, kD, static_cast<uint64_t>(a.T) * a.H, kD * 2, 64,
                      static_cast<uint32_t>(a.H), true))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaMemsetAsync(a.counters, 0, static_cast<size_t>(a.T) * sizeof(unsigned), stream);
-  if (e != cudaSuccess) return e;
   auto go = [&](auto kern) -> cudaError_t {
     cudaError_t e2 = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), kFSmemBytes);
     if (e2 != cudaSuccess) return e2;

@@ -148,9 +148,8 @@ int score_mode_hp(int h_eff, bool shared_groups);
 
 cudaError_t launch_index_score(const CUtensorMap* tmap, const ScoreArgs& a, cudaStream_t stream);
 
-// The fused decode step (decode_fused.cu): router + routed scoring + top-k in
-// one persistent kernel.
-constexpr int kDecodeFusedMaxGrid = 256;   // CTAs at most (one per SM)
+// Router + routed scoring of a decode step in one persistent kernel
+// (decode_fused.cu); the top-k of its score rows is launch_topk's.
 struct DecodeArgs {
   const uint16_t* q;
   const float* w;
@@ -161,22 +160,15 @@ struct DecodeArgs {
   int64_t nmeanseq, means_seq_stride;
   const int32_t* seq_of;
   const int32_t* prefix_len;
-  int T, H, h, k, B;
+  int T, H, h, B;
   int64_t L;
   int32_t* heads;
   float* importance;
   float* scores;
   int64_t row_stride;
-  int32_t* idx;
-  unsigned* counters;   // [T] workspace
-  uint32_t* hist;       // [T][slots][2048] workspace
   uint32_t* err;
 };
-bool decode_fused_supported(int T, int H, int h, int64_t L, int k);
-// first-digit bins of the per-segment score histograms
-int decode_fused_hist_bins();
-// histogram slots per query for grids of at most sms_bound CTAs
-int64_t decode_fused_hist_slots(int T, int64_t L, int sms_bound);
+bool decode_fused_supported(int H, int h, int64_t L);
 cudaError_t launch_decode_fused(const DecodeArgs& a, cudaStream_t stream);
 
 size_t topk_smem_bytes();

@@ -1,4 +1,4 @@
-// Per-row top-k of fp32 scores by radix select, one thread-block cluster per row.
+// Per-row top-k of fp32 scores.
 //
 // MISA forum thread (zingnex.cn), "DeepSeek稀疏注意力（DSA）的突破": the indexer
 // keeps the most relevant token subset for the main attention.  HISA explainer
@@ -9,25 +9,21 @@
 // (and NaN) never selected; the selected positions come out in ascending order,
 // -1 padded when the row holds fewer than k selectable entries.
 //
-// Rows of up to 65536 entries (topk_range_kernel): a cluster of up to 8 CTAs
-// per row, the row's entries held in registers, a value-range histogram whose
-// threshold bin is gathered across the cluster; described above the kernel.
-//
-// Longer rows (topk_cluster_kernel) are split into CL = 8 contiguous slices,
-// one per CTA of a cluster.  Scores become order-preserving uint32 keys
-// (re-read from global memory when a slice does not fit in shared memory).
-// The k-th largest key tau is found digit by digit (12 + 10 + 10 bits): every
-// CTA histograms the digit over its slice (keys whose higher digits match the
-// prefix found so far), the CL histograms are summed through distributed
-// shared memory (each CTA owns 1/CL of the bins), every CTA pulls the summed
-// histogram and finds the bin holding the k-th key.  A final pass writes the
-// selected positions: each warp owns a contiguous chunk of its slice, warp
-// ballots, a scan over the warps and the per-CTA counts exchanged across the
-// cluster give every selected entry its output slot, so the output is in
-// position order without a sort.
-//
-// In both kernels keys equal to tau are taken lowest position first, exactly
-// as many as needed.
+// Four kernels, by row count and length (launch_topk):
+//  * many rows (at least two per SM), up to 131072 entries: topk_band_kernel,
+//    one CTA per row, a sampled band around the k-th entry;
+//  * few rows of up to 8192 entries: topk_row_kernel, one CTA per row, the
+//    row in registers, a value-range histogram;
+//  * few rows of 8193 .. 131072 entries: topk_rowc_kernel, the same over a
+//    cluster of up to 8 CTAs per row;
+//  * few longer rows: topk_cluster_kernel, a cluster of 8 CTAs per row, the
+//    k-th largest key digit by digit (12 + 10 + 10 bits): every CTA
+//    histograms the digit over its slice, the histograms are summed through
+//    distributed shared memory (each CTA owns 1/8 of the bins), every CTA
+//    finds the bin holding the k-th key; ballots, a scan over the warps and
+//    the per-CTA counts give every selected entry its slot.
+// Each kernel's comment describes it.  In every kernel keys equal to the k-th
+// largest are taken lowest position first, exactly as many as needed.
 #include <cooperative_groups.h>
 
 #include "launch.h"
@@ -347,535 +343,9 @@ topk_cluster_kernel(const float* __restrict__ scores, int64_t n, int64_t row_str
   }
 }
 
-// ---------------------------------------------------------------------------
-// Rows of up to 8 x 512 x 16 entries: a cluster of CL <= 8 CTAs of 512
-// threads per row, each thread holding V contiguous entries of the row in
-// registers (V = 8 or 16 by row length).  Instead of bit digits (whose top
-// bits put most scores of a row into a few exponent bins) the histogram splits
-// the value range of a fixed sample of the row (the same 512 entries in every
-// CTA, so every CTA derives the same bins) into 1024 equal ranges; the map is
-// monotone, values outside the sample's range go to the end bins.  The path
-// is a short chain of dependent steps, each a cluster barrier followed by
-// small rounds of distributed shared memory reads (they are slow; bytes are
-// kept few):
-//   (1) every CTA sums the CL histograms' 32 super-bin totals, finds the
-//       super-bin holding the k-th entry, then sums its 32 bins (a second
-//       read round) and finds the threshold bin;
-//   (2) every CTA reads the counts above the threshold bin and the threshold
-//       bin's entries (few) of every slice, finds the exact threshold among
-//       them by counting, and so knows how many entries above and equal to it
-//       each slice holds: the output slots follow from a scan.
-// A threshold bin with more entries than one read round takes is gathered in
-// a second round (radix select over the gathered entries when they are many);
-// one too full to gather (massive ties, a sample range spoilt by outliers)
-// falls back to a cluster-wide bit-digit radix select inside it.
-constexpr int kXThreads = 512;
-constexpr int kXWarps = kXThreads / 32;
-constexpr int kXBins = 2048;          // histogram array (fallback digits use all of it)
-constexpr int kXFastBins = 1024;      // value-range bins: 2 per thread
-constexpr int kXSup = kXBins / 32;
-constexpr int kXFastCand = kXThreads / kMaxCluster;  // threshold-bin entries per slice read in one round
-constexpr int kXCandCap = 512;        // threshold-bin entries kept per CTA
-constexpr int kXMergeCap = 2048;      // and over the cluster
-#ifndef MISA_TOPK_RANGE_CLUSTER
-#define MISA_TOPK_RANGE_CLUSTER 8
-#endif
-constexpr int kXRangeCluster = MISA_TOPK_RANGE_CLUSTER;  // CTAs per row at most
-
-struct XSmem {
-  uint32_t hist[kXBins];     // this CTA's histogram (read by the cluster)
-  uint32_t sup[kXSup];       // fallback: its super-bin totals (read by the cluster)
-  uint32_t meta[4];          // valid entries, entries above the threshold bin, threshold-bin entries (read by the cluster)
-  uint32_t cnt2[2];          // fallback: entries above / equal to tau (read by the cluster)
-  uint32_t gsup[kXSup];      // super-bin totals summed over the cluster
-  uint32_t gbin[32];
-  uint32_t bc[8];
-  float fbc;
-  uint32_t rv[kMaxCluster], ra[kMaxCluster], rc[kMaxCluster];
-  uint32_t at[kMaxCluster], et[kMaxCluster];
-  float wmin[kXWarps], wmax[kXWarps];
-  uint64_t wscan[kXWarps];
-  union {
-    struct {
-      float cval[kXCandCap];     // this CTA's threshold-bin entries (read by the cluster)
-      float fval[kXThreads];     // first kXFastCand entries of every slice, [rank][i]
-      float mval[kXMergeCap];    // the cluster's threshold-bin entries, by rank
-      uint8_t mrank[kXMergeCap];
-    } c;
-    struct {
-      uint32_t h[kXBins];        // fallback digit histogram, second buffer (read by the cluster)
-      uint32_t s[kXSup];
-    } r;
-  } u;
-};
-
-__device__ __forceinline__ void cluster_arrive_relaxed() {
-  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
-
-// One warp: among tot[0, cnt) (cnt <= 128) the index i with
-// above(i) < need <= above(i) + tot[i], above(i) = sum of tot[i+1 .. cnt);
-// out[0] = i, out[1] = above(i).
-__device__ __forceinline__ void warp_suffix_find(const uint32_t* tot, int cnt, uint32_t need, uint32_t* out) {
-  const int lane = threadIdx.x & 31;
-  const int per = (cnt + 31) / 32;
-  const int b0 = lane * per;
-  uint32_t local = 0;
-  for (int i = 0; i < per; ++i)
-    if (b0 + i < cnt) local += tot[b0 + i];
-  uint32_t inc = local;  // sum over lanes >= this one
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t y = __shfl_down_sync(0xffffffffu, inc, o);
-    if (lane + o < 32) inc += y;
-  }
-  const uint32_t after = inc - local;
-  if (after < need && need <= inc) {
-    uint32_t acc = after;
-    for (int i = per - 1; i >= 0; --i) {
-      if (b0 + i >= cnt) continue;
-      const uint32_t c = tot[b0 + i];
-      if (acc + c >= need) {
-        out[0] = static_cast<uint32_t>(b0 + i);
-        out[1] = acc;
-        break;
-      }
-      acc += c;
-    }
-  }
-}
-
-// Super-bin totals of a histogram of nbins (a multiple of 128, <= 2048): each
-// thread adds 4 bins, 8 lanes make one super-bin of 32.
-__device__ __forceinline__ void make_supers(const uint32_t* h, uint32_t* sup, int nbins) {
-  const int base = threadIdx.x * 4;
-  if (base < nbins) {  // whole warps
-    const uint4 x = *reinterpret_cast<const uint4*>(h + base);
-    uint32_t s = x.x + x.y + x.z + x.w;
-    s += __shfl_xor_sync(0xffffffffu, s, 1);
-    s += __shfl_xor_sync(0xffffffffu, s, 2);
-    s += __shfl_xor_sync(0xffffffffu, s, 4);
-    if ((threadIdx.x & 7) == 0) sup[base / 32] = s;
-  }
-}
-
-// The bin holding the need-th largest entry of the histogram summed over nsrc
-// sources (hist_of(r), sup_of(r): source r's bins and super-bin totals, all
-// complete); *above = entries in higher bins.  Every thread of the CTA calls.
-template <class HistOf, class SupOf>
-__device__ int two_level_find(XSmem& sm, int nsrc, HistOf hist_of, SupOf sup_of, int nsup, uint32_t need,
-                              uint32_t* above) {
-  const int tid = threadIdx.x;
-  for (int i = tid; i < nsup; i += kXThreads) sm.gsup[i] = 0;
-  if (tid < 32) sm.gbin[tid] = 0;
-  __syncthreads();
-  for (int i = tid; i < nsup * nsrc; i += kXThreads) {
-    const int s = i % nsup, r = i / nsup;
-    atomicAdd(&sm.gsup[s], sup_of(r)[s]);
-  }
-  __syncthreads();
-  if (tid < 32) warp_suffix_find(sm.gsup, nsup, need, sm.bc);
-  __syncthreads();
-  // (the index is in range by construction; the clamps only keep a wrong
-  // count from addressing outside the arrays)
-  const int S = sm.bc[0] < static_cast<uint32_t>(nsup) ? static_cast<int>(sm.bc[0]) : nsup - 1;
-  const uint32_t above_s = sm.bc[1];
-  for (int i = tid; i < 32 * nsrc; i += kXThreads) {
-    const int j = i & 31, r = i >> 5;
-    atomicAdd(&sm.gbin[j], hist_of(r)[S * 32 + j]);
-  }
-  __syncthreads();
-  if (tid < 32) warp_suffix_find(sm.gbin, 32, need - above_s, sm.bc + 2);
-  __syncthreads();
-  *above = above_s + sm.bc[3];
-  return S * 32 + static_cast<int>(sm.bc[2] & 31u);
-}
-
-// Bit digits of a key for the radix rounds: 11, 11, 10 bits from the top.
-__device__ __forceinline__ int digit_shift(int round) { return round == 0 ? 21 : (round == 1 ? 10 : 0); }
-__device__ __forceinline__ int digit_bins(int round) { return round == 2 ? 1024 : 2048; }
-
 __device__ __forceinline__ float key_to_float(uint32_t kk) {
   const uint32_t u = (kk & 0x80000000u) ? (kk ^ 0x80000000u) : ~kk;
   return __uint_as_float(u);
-}
-
-template <int V>
-__global__ void __launch_bounds__(kXThreads, 2)
-topk_range_kernel(const float* __restrict__ scores, int64_t n, int64_t row_stride, const int32_t* __restrict__ row_valid,
-                  const int32_t* __restrict__ id_map, int64_t id_map_stride, int k, int32_t* __restrict__ idx) {
-  extern __shared__ __align__(16) uint8_t smem_raw[];
-  XSmem& sm = *reinterpret_cast<XSmem*>(smem_raw);
-  cg::cluster_group cl = cg::this_cluster();
-  const int CL = static_cast<int>(cl.num_blocks());
-  const int rank = static_cast<int>(cl.block_rank());
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t t = blockIdx.y;
-  constexpr int kSlice = kXThreads * V;
-  const float kNegInf = -__int_as_float(0x7f800000);
-  const float kPosInf = __int_as_float(0x7f800000);
-  const uint32_t ku = static_cast<uint32_t>(k);
-
-  for (int i = tid; i < kXFastBins; i += kXThreads) sm.hist[i] = 0;
-  if (tid < 4) sm.meta[tid] = 0;
-  pdl_wait_inputs();
-  pdl_allow_next();
-
-  const float* row = scores + t * row_stride;
-  const int32_t* idrow = id_map ? id_map + t * id_map_stride : nullptr;
-  int32_t* out = idx + t * k;
-  int64_t nt64 = n;
-  if (row_valid) {
-    const int64_t rv = row_valid[t];
-    nt64 = rv < 0 ? 0 : (rv < n ? rv : n);
-  }
-  const int nt = static_cast<int>(nt64);
-  const int s0 = rank * kSlice < nt ? rank * kSlice : nt;
-  const int s1 = s0 + kSlice < nt ? s0 + kSlice : nt;
-  const int p0 = s0 + tid * V;  // this thread's entries: positions [p0, p0 + V) of the row
-
-  // ---------------- load (the slice start and p0 are multiples of 4 entries)
-  float v[V];
-#pragma unroll
-  for (int j = 0; j < V; j += 4) {
-    const int p = p0 + j;
-    if (p + 3 < s1) {
-      const float4 f = __ldg(reinterpret_cast<const float4*>(row + p));
-      v[j] = f.x;
-      v[j + 1] = f.y;
-      v[j + 2] = f.z;
-      v[j + 3] = f.w;
-    } else {
-#pragma unroll
-      for (int c = 0; c < 4; ++c) v[j + c] = p + c < s1 ? __ldg(row + p + c) : kNegInf;
-    }
-  }
-  float smp = nt > 0 ? __ldg(row + static_cast<int64_t>(tid) * nt / kXThreads) : kNegInf;
-  smp = valid_or_neg_inf(smp);
-  float mx = smp, mn = smp > kNegInf ? smp : kPosInf;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-  }
-  if (lane == 0) {
-    sm.wmax[warp] = mx;
-    sm.wmin[warp] = mn;
-  }
-  __syncthreads();
-  mx = sm.wmax[0];
-  mn = sm.wmin[0];
-#pragma unroll
-  for (int i = 1; i < kXWarps; ++i) {
-    mx = fmaxf(mx, sm.wmax[i]);
-    mn = fminf(mn, sm.wmin[i]);
-  }
-  const float range = mx - mn;
-  const float scale = (range > 0.f && range < kPosInf) ? static_cast<float>(kXFastBins) / range : 0.f;
-  // monotone in x; a NaN intermediate (no valid sample, infinite entries) maps to bin 0
-  auto bin_of = [&](float x) -> int {
-    const float y = __fmul_rn(__fsub_rn(x, mn), scale);
-    return y > 0.f ? (y >= static_cast<float>(kXFastBins - 1) ? kXFastBins - 1 : static_cast<int>(y)) : 0;
-  };
-
-  // ---------------- value-range histogram of the slice
-  uint32_t nval = 0;
-#pragma unroll
-  for (int j = 0; j < V; ++j) {
-    v[j] = valid_or_neg_inf(v[j]);
-    if (v[j] > kNegInf) {
-      atomicAdd(&sm.hist[bin_of(v[j])], 1u);
-      ++nval;
-    }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) nval += __shfl_xor_sync(0xffffffffu, nval, o);
-  if (lane == 0 && nval) atomicAdd(&sm.meta[0], nval);
-  __syncthreads();
-  make_supers(sm.hist, sm.sup, kXFastBins);
-  __syncthreads();
-  cl.sync();  // (1) every CTA's histogram, super-bin totals and valid count are complete
-
-  // ---------------- the threshold bin, from the CL histograms in two read
-  // rounds of 32 x CL words each: super-bin totals, then the 32 bins of the
-  // super-bin holding the k-th entry.  Thread (s, r) = (tid / 8, tid % 8)
-  // reads item s of source (r + rank) mod CL (the CTAs start on different
-  // SMs); 8 lanes add their sources.
-  const int fs = tid >> 3, fr = tid & 7;
-  const int fsrc = fr + rank < CL ? fr + rank : fr + rank - CL;
-  if (tid >= 32 * kMaxCluster && tid < 32 * kMaxCluster + CL)
-    sm.rv[tid - 32 * kMaxCluster] = cl.map_shared_rank(&sm.meta[0], tid - 32 * kMaxCluster)[0];
-  if (tid < 32 * kMaxCluster) {
-    uint32_t x = fr < CL ? cl.map_shared_rank(&sm.sup[0], fsrc)[fs] : 0u;
-    x += __shfl_xor_sync(0xffffffffu, x, 1);
-    x += __shfl_xor_sync(0xffffffffu, x, 2);
-    x += __shfl_xor_sync(0xffffffffu, x, 4);
-    if (fr == 0) sm.gsup[fs] = x;
-  }
-  __syncthreads();
-  if (warp == 0) {
-    uint32_t x = sm.gsup[lane];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-    if (lane == 0) sm.bc[3] = x;  // valid entries of the row
-    if (x > ku) warp_suffix_find(sm.gsup, 32, ku, sm.bc);
-  }
-  __syncthreads();
-  const uint32_t total = sm.bc[3];
-
-  float tau = kNegInf;  // selected: entries above tau, and the first need_eq entries equal to it
-  uint32_t need_eq = 0;
-  if (total <= ku) {
-    if (tid < CL) {
-      sm.at[tid] = sm.rv[tid];
-      sm.et[tid] = 0;
-    }
-  } else {
-    const int S = static_cast<int>(sm.bc[0] & 31u);
-    const uint32_t above_s = sm.bc[1];
-    if (tid < 32 * kMaxCluster) {
-      uint32_t x = fr < CL ? cl.map_shared_rank(&sm.hist[0], fsrc)[S * 32 + fs] : 0u;
-      x += __shfl_xor_sync(0xffffffffu, x, 1);
-      x += __shfl_xor_sync(0xffffffffu, x, 2);
-      x += __shfl_xor_sync(0xffffffffu, x, 4);
-      if (fr == 0) sm.gbin[fs] = x;
-    }
-    __syncthreads();
-    if (warp == 0) warp_suffix_find(sm.gbin, 32, ku - above_s, sm.bc + 4);
-    __syncthreads();
-    const int bstar = S * 32 + static_cast<int>(sm.bc[4] & 31u);
-    const uint32_t above_b = above_s + sm.bc[5];
-    const uint32_t need = ku - above_b;
-    // entries above the threshold bin, and the threshold bin's entries
-    uint32_t a = 0;
-#pragma unroll
-    for (int j = 0; j < V; ++j) {
-      if (v[j] > kNegInf) {
-        const int b = bin_of(v[j]);
-        a += b > bstar ? 1u : 0u;
-        if (b == bstar) {
-          const uint32_t slot = atomicAdd(&sm.meta[2], 1u);
-          if (slot < static_cast<uint32_t>(kXCandCap)) sm.u.c.cval[slot] = v[j];
-        }
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-    if (lane == 0 && a) atomicAdd(&sm.meta[1], a);
-    __syncthreads();
-    cl.sync();  // (2) every CTA's counts and threshold-bin entries are complete
-    {
-      // one read round: slice r's counts and its first kXFastCand entries
-      // (thread group j of CTA c reads slice (j + c) mod CL: the CTAs start on
-      // different slices)
-      const int j = tid / kXFastCand, i = tid - j * kXFastCand;
-      if (j < CL) {
-        const int r = j + rank < CL ? j + rank : j + rank - CL;
-        const uint32_t* m = cl.map_shared_rank(&sm.meta[0], r);
-        const float x = cl.map_shared_rank(&sm.u.c.cval[0], r)[i];
-        if (i == 0) {
-          sm.ra[r] = m[1];
-          sm.rc[r] = m[2];
-        }
-        sm.u.c.fval[r * kXFastCand + i] = x;
-      }
-    }
-    __syncthreads();
-    uint32_t ctot = 0, cmax = 0;
-#pragma unroll
-    for (int r = 0; r < kMaxCluster; ++r) {
-      const uint32_t c = r < CL ? sm.rc[r] : 0u;
-      ctot += c;
-      cmax = c > cmax ? c : cmax;
-    }
-    const bool overflow = cmax > static_cast<uint32_t>(kXCandCap) || ctot > static_cast<uint32_t>(kXMergeCap);
-    if (cmax <= static_cast<uint32_t>(kXFastCand)) {
-      // compact the entries read in the round above
-      const int r = tid / kXFastCand, i = tid - r * kXFastCand;
-      if (r < CL && static_cast<uint32_t>(i) < sm.rc[r]) {
-        uint32_t off = 0;
-        for (int r2 = 0; r2 < r; ++r2) off += sm.rc[r2];
-        sm.u.c.mval[off + i] = sm.u.c.fval[tid];
-        sm.u.c.mrank[off + i] = static_cast<uint8_t>(r);
-      }
-      __syncthreads();
-    } else if (!overflow) {
-      // a second read round for the rest of the threshold bin
-      for (int i = tid; i < static_cast<int>(ctot); i += kXThreads) {
-        int r = 0;
-        uint32_t off = 0;
-        while (off + sm.rc[r] <= static_cast<uint32_t>(i)) off += sm.rc[r++];
-        sm.u.c.mval[i] = cl.map_shared_rank(&sm.u.c.cval[0], r)[i - off];
-        sm.u.c.mrank[i] = static_cast<uint8_t>(r);
-      }
-      __syncthreads();
-    }
-    if (!overflow) {
-      if (ctot <= static_cast<uint32_t>(kXThreads)) {
-        // exact rank by counting
-        if (tid < static_cast<int>(ctot)) {
-          const float x = sm.u.c.mval[tid];
-          uint32_t g = 0, ge = 0;
-#pragma unroll 4
-          for (int j = 0; j < static_cast<int>(ctot); ++j) {
-            const float y = sm.u.c.mval[j];
-            g += y > x ? 1u : 0u;
-            ge += y >= x ? 1u : 0u;
-          }
-          if (g < need && need <= ge) {
-            sm.fbc = x;
-            sm.bc[2] = need - g;
-          }
-        }
-        __syncthreads();
-        tau = sm.fbc;
-        need_eq = sm.bc[2];
-      } else {
-        // bit-digit radix select over the gathered entries (local; the
-        // histogram arrays are no longer read by the cluster after (2))
-        uint32_t prefix = 0, nd = need;
-        for (int round = 0; round < 3; ++round) {
-          const int sh = digit_shift(round), nb = digit_bins(round);
-          for (int i = tid; i < nb; i += kXThreads) sm.hist[i] = 0;
-          __syncthreads();
-          for (int i = tid; i < static_cast<int>(ctot); i += kXThreads) {
-            const uint32_t kk = float_key(sm.u.c.mval[i]);
-            if (round == 0 || (kk >> digit_shift(round - 1)) == prefix) atomicAdd(&sm.hist[(kk >> sh) & (nb - 1)], 1u);
-          }
-          __syncthreads();
-          make_supers(sm.hist, sm.sup, nb);
-          __syncthreads();
-          uint32_t ab;
-          const int b = two_level_find(
-              sm, 1, [&](int) { return &sm.hist[0]; }, [&](int) { return &sm.sup[0]; }, nb / 32, nd, &ab);
-          nd -= ab;
-          prefix = round == 0 ? static_cast<uint32_t>(b) : ((prefix << (round == 1 ? 11 : 10)) | static_cast<uint32_t>(b));
-        }
-        tau = key_to_float(prefix);
-        need_eq = nd;
-      }
-      // entries above / equal to tau in every slice
-      if (tid < CL) {
-        sm.at[tid] = sm.ra[tid];
-        sm.et[tid] = 0;
-      }
-      __syncthreads();
-      for (int i = tid; i < static_cast<int>(ctot); i += kXThreads) {
-        const float x = sm.u.c.mval[i];
-        if (x > tau) atomicAdd(&sm.at[sm.u.c.mrank[i]], 1u);
-        else if (x == tau) atomicAdd(&sm.et[sm.u.c.mrank[i]], 1u);
-      }
-    } else {
-      // ---------------- fallback: cluster-wide radix select inside bin bstar.
-      // Digit histograms alternate between two buffers, so a CTA never
-      // overwrites one that another CTA may still be reading.
-      uint32_t prefix = 0, nd = need;
-      for (int round = 0; round < 3; ++round) {
-        uint32_t* H = (round & 1) ? sm.u.r.h : sm.hist;
-        uint32_t* S = (round & 1) ? sm.u.r.s : sm.sup;
-        const int sh = digit_shift(round), nb = digit_bins(round);
-        for (int i = tid; i < nb; i += kXThreads) H[i] = 0;
-        __syncthreads();
-#pragma unroll
-        for (int j = 0; j < V; ++j) {
-          if (v[j] > kNegInf && bin_of(v[j]) == bstar) {
-            const uint32_t kk = float_key(v[j]);
-            if (round == 0 || (kk >> digit_shift(round - 1)) == prefix) atomicAdd(&H[(kk >> sh) & (nb - 1)], 1u);
-          }
-        }
-        __syncthreads();
-        make_supers(H, S, nb);
-        __syncthreads();
-        cl.sync();
-        uint32_t ab;
-        const int b = two_level_find(
-            sm, CL, [&](int r) { return cl.map_shared_rank(H, r); }, [&](int r) { return cl.map_shared_rank(S, r); },
-            nb / 32, nd, &ab);
-        nd -= ab;
-        prefix = round == 0 ? static_cast<uint32_t>(b) : ((prefix << (round == 1 ? 11 : 10)) | static_cast<uint32_t>(b));
-      }
-      tau = key_to_float(prefix);
-      need_eq = nd;
-      uint32_t ac = 0, ec = 0;
-#pragma unroll
-      for (int j = 0; j < V; ++j) {
-        ac += v[j] > tau ? 1u : 0u;
-        ec += (v[j] > kNegInf && v[j] == tau) ? 1u : 0u;
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        ac += __shfl_xor_sync(0xffffffffu, ac, o);
-        ec += __shfl_xor_sync(0xffffffffu, ec, o);
-      }
-      if (tid < 2) sm.cnt2[tid] = 0;
-      __syncthreads();
-      if (lane == 0) {
-        atomicAdd(&sm.cnt2[0], ac);
-        atomicAdd(&sm.cnt2[1], ec);
-      }
-      __syncthreads();
-      cl.sync();
-      if (tid < CL) {
-        const uint32_t* c2 = cl.map_shared_rank(&sm.cnt2[0], tid);
-        sm.at[tid] = c2[0];
-        sm.et[tid] = c2[1];
-      }
-    }
-  }
-  __syncthreads();
-  // every value read from another CTA's shared memory has arrived: it may exit
-  // once all CTAs are here
-  cluster_arrive_relaxed();
-
-  // ---------------- output slots: entries above tau before this one, plus the
-  // equal entries before it (at most need_eq of them)
-  uint32_t a_before = 0, e_before = 0, a_all = 0, e_all = 0;
-#pragma unroll
-  for (int r = 0; r < kMaxCluster; ++r) {
-    const uint32_t ar = r < CL ? sm.at[r] : 0u, er = r < CL ? sm.et[r] : 0u;
-    a_before += r < rank ? ar : 0u;
-    e_before += r < rank ? er : 0u;
-    a_all += ar;
-    e_all += er;
-  }
-  uint32_t a_t = 0, e_t = 0;
-#pragma unroll
-  for (int j = 0; j < V; ++j) {
-    a_t += v[j] > tau ? 1u : 0u;
-    e_t += (v[j] > kNegInf && v[j] == tau) ? 1u : 0u;
-  }
-  uint64_t x = static_cast<uint64_t>(a_t) | (static_cast<uint64_t>(e_t) << 32);
-  uint64_t incl = x;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint64_t y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  if (lane == 31) sm.wscan[warp] = incl;
-  __syncthreads();
-  uint64_t wbase = 0;
-  for (int i = 0; i < warp; ++i) wbase += sm.wscan[i];
-  const uint64_t excl = wbase + incl - x;
-  uint32_t A = a_before + static_cast<uint32_t>(excl & 0xffffffffull);
-  uint32_t E = e_before + static_cast<uint32_t>(excl >> 32);
-#pragma unroll
-  for (int j = 0; j < V; ++j) {
-    const float y = v[j];
-    if (y > tau) {
-      const uint32_t slot = A + (E < need_eq ? E : need_eq);
-      if (slot < ku) out[slot] = idrow ? idrow[p0 + j] : p0 + j;
-      ++A;
-    } else if (y > kNegInf && y == tau) {
-      if (E < need_eq && A + E < ku) out[A + E] = idrow ? idrow[p0 + j] : p0 + j;
-      ++E;
-    }
-  }
-  if (rank == CL - 1) {
-    const uint32_t chosen = a_all + (e_all < need_eq ? e_all : need_eq);
-    for (uint32_t i = chosen + tid; i < ku; i += kXThreads) out[i] = -1;
-  }
-  cluster_wait();  // no CTA exits while another may still read its shared memory
 }
 
 // ---------------------------------------------------------------------------
@@ -1340,6 +810,750 @@ topk_band_kernel(const float* __restrict__ scores, int64_t n, int64_t row_stride
   for (uint32_t i = chosen + tid; i < ku; i += kBThreads) out[i] = -1;
 }
 
+// ---------------------------------------------------------------------------
+// Rows of up to 8192 entries, few rows (topk_row_kernel): one CTA of 1024
+// threads per row, no cluster.  Warp w holds positions [w 32V, (w+1) 32V) of
+// the row in registers (V = 4 or 8 per thread, loaded as coalesced float4:
+// in step i lane l holds positions w 32V + 128 i + 4 l + (0..3)), so the row
+// is read once and every later step is a pass over registers:
+//   (1) a value range from a sample (each thread's first entry: 1024 evenly
+//       spaced positions);
+//   (2) a histogram over 2048 equal-width bins of that range (entries outside
+//       it go to the end bins; the bin of a value is monotone in the value)
+//       gives the selectable count, the bin b* holding the k-th largest entry
+//       and the count above b*;
+//   (3) one pass marks the entries above b* and lists those in b* (few, as a
+//       rule) in shared memory; each listed entry's rank (value descending,
+//       position ascending) is counted against the others, and the need
+//       best-ranked ones are marked in their owner thread's mask;
+//   (4) every thread writes its marked positions into slots from a scan over
+//       the warp (per step) and over the warps, in position order.
+// Values are compared as floats: NaN fails every test (never selected), -0.0
+// equals +0.0.  General path, for a degenerate range or a long list: the
+// exact k-th largest key tau by three radix rounds (11, 11, 10 key bits) over
+// the list or over the registers, then the entries above tau and the lowest-
+// position entries equal to it.
+constexpr int kRThreads = 1024;
+constexpr int kRWarps = kRThreads / 32;
+constexpr int kRBins = 2048;
+constexpr int kRCandCap = 4096;   // entries of b* listed in shared memory
+constexpr int kRRankMax = 128;    // lists this short are ranked by counting
+
+struct alignas(16) RSmem {
+  uint32_t hist[kRBins];
+  float cv[kRCandCap];        // the listed entries of b* and their positions
+  int32_t cp[kRCandCap];
+  uint32_t extra[kRThreads];  // per thread: listed entries that are selected (bit j)
+  uint32_t red[3][kRWarps];   // scan scratch (halves 0 and 1 alternate), reductions
+  uint32_t bc[2];
+  uint32_t ccount;
+  float tau;
+  uint32_t take, eqtot;
+};
+
+// Exclusive scan of x over the CTA's 1024 threads, with red (32 words) as
+// scratch; *total = the sum.  Alternating two scratch arrays, two scans in a
+// row need no barrier between them.
+__device__ __forceinline__ uint32_t cta_excl_scan(uint32_t x, uint32_t* red, uint32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t inc = x;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  if (lane == 31) red[warp] = inc;
+  __syncthreads();
+  const uint32_t wv = red[lane];
+  uint32_t winc = wv;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, winc, o);
+    if (lane >= o) winc += y;
+  }
+  const uint32_t before = __shfl_sync(0xffffffffu, winc - wv, warp);
+  *total = __shfl_sync(0xffffffffu, winc, 31);
+  return before + inc - x;
+}
+
+// The bin of h[0, nb) (nb = 1024 or 2048) holding the need-th largest entry:
+// bc[0] = bin, bc[1] = entries in higher bins (set only when need <= the
+// total).  Returns the histogram's total.  All 1024 threads; ends with a
+// barrier.
+__device__ __forceinline__ uint32_t cta_find_bin(const uint32_t* h, int nb, uint32_t need, uint32_t* red,
+                                                 uint32_t* bc) {
+  const int per = nb / kRThreads;
+  const int b0 = threadIdx.x * per;
+  uint32_t local = 0;
+  for (int i = 0; i < per; ++i) local += h[b0 + i];
+  uint32_t total;
+  const uint32_t excl = cta_excl_scan(local, red, &total);
+  const uint32_t after = total - excl - local;   // entries in the bins of higher threads
+  if (after < need && need <= after + local) {
+    uint32_t acc = after;
+    for (int i = per - 1; i >= 0; --i) {
+      const uint32_t c = h[b0 + i];
+      if (acc + c >= need) {
+        bc[0] = static_cast<uint32_t>(b0 + i);
+        bc[1] = acc;
+        break;
+      }
+      acc += c;
+    }
+  }
+  __syncthreads();
+  return total;
+}
+
+__device__ __forceinline__ uint32_t row_find_bin(RSmem& sm, int nb, uint32_t need, int buf) {
+  return cta_find_bin(sm.hist, nb, need, sm.red[buf], sm.bc);
+}
+
+// Three radix rounds (11, 11, 10 key bits): the need-th largest key among the
+// keys add_round(prefix, pmask, shift, nbins) counts into hist.  Leaves tau,
+// take (entries equal to tau taken) and eqtot (entries equal to tau) in sm.
+template <class AddRound>
+__device__ __forceinline__ void row_radix(RSmem& sm, uint32_t need, AddRound add_round) {
+  const int tid = threadIdx.x;
+  uint32_t prefix = 0u, pmask = 0u, eqtot = 0u;
+#pragma unroll 1
+  for (int round = 0; round < 3; ++round) {
+    const int sh = round == 0 ? 21 : (round == 1 ? 10 : 0);
+    const int nb = round == 2 ? 1024 : 2048;
+    __syncthreads();   // the previous readers of hist / bc are done
+    for (int i = tid; i < nb; i += kRThreads) sm.hist[i] = 0u;
+    __syncthreads();
+    add_round(prefix, pmask, sh, nb);
+    __syncthreads();
+    row_find_bin(sm, nb, need, round & 1);
+    const uint32_t d = sm.bc[0];
+    need -= sm.bc[1];
+    prefix |= d << sh;
+    pmask |= static_cast<uint32_t>(nb - 1) << sh;
+    if (round == 2) eqtot = sm.hist[d];
+  }
+  __syncthreads();
+  if (tid == 0) {
+    sm.tau = key_to_float(prefix);
+    sm.take = need;
+    sm.eqtot = eqtot;
+  }
+  __syncthreads();
+}
+
+// For each warp: the exclusive prefix of its total over the lower warps, and
+// *all = the sum over the CTA.  x: this warp's total (same in every lane);
+// red: 32 words of scratch.
+__device__ __forceinline__ uint32_t cta_warp_base(uint32_t x, uint32_t* red, uint32_t* all) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane == 0) red[warp] = x;
+  __syncthreads();
+  const uint32_t wv = red[lane];
+  uint32_t winc = wv;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, winc, o);
+    if (lane >= o) winc += y;
+  }
+  *all = __shfl_sync(0xffffffffu, winc, 31);
+  return __shfl_sync(0xffffffffu, winc - wv, warp);
+}
+
+__device__ __forceinline__ uint32_t row_warp_base(RSmem& sm, uint32_t x, int buf, uint32_t* all) {
+  return cta_warp_base(x, sm.red[buf], all);
+}
+
+__device__ __forceinline__ uint32_t warp_sum(uint32_t x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+// Entries are held as in topk_row_kernel: bit j of a thread's mask is its
+// entry j, at position base + 128 (j / 4) + 4 lane + j % 4 of its warp's chunk.
+//
+// Of the entries marked in tk, the first `take` in position order over the
+// CTA (warps in order, then steps, lanes, entries).  All threads.
+template <int V>
+__device__ __forceinline__ uint32_t cta_keep_first(uint32_t tk, uint32_t take, uint32_t* red) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t lt = (1u << lane) - 1u;
+  uint32_t all;
+  uint32_t run = cta_warp_base(warp_sum(__popc(tk)), red, &all);
+  uint32_t keep = 0u;
+#pragma unroll
+  for (int i = 0; i < V / 4; ++i) {
+    uint32_t before = 0u, tot = 0u;
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+      const uint32_t b = __ballot_sync(0xffffffffu, (tk >> (4 * i + cc)) & 1u);
+      before += __popc(b & lt);
+      tot += __popc(b);
+    }
+    uint32_t r = run + before;
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc)
+      if ((tk >> (4 * i + cc)) & 1u) {
+        if (r < take) keep |= 1u << (4 * i + cc);
+        ++r;
+      }
+    run += tot;
+  }
+  return keep;
+}
+
+// Writes the entries marked in selm to out[base + slot] (through idrow when
+// given), slots in position order over the CTA; per step i (4 entries per
+// lane) the lane counts are packed in 8-bit fields (a warp's step total is
+// <= 128).  Slots at or past ku are not written.  Returns the CTA's count.
+// All threads.
+template <int V, class PosOf>
+__device__ __forceinline__ uint32_t cta_write_selected(uint32_t selm, uint32_t base, PosOf pos_of,
+                                                       const int32_t* __restrict__ idrow, int32_t* __restrict__ out,
+                                                       uint32_t ku, uint32_t* red) {
+  static_assert(V <= 32, "eight steps at most");
+  const int lane = threadIdx.x & 31;
+  uint32_t plo = 0u, phi = 0u;
+#pragma unroll
+  for (int i = 0; i < V / 4; ++i) {
+    const uint32_t cnt = static_cast<uint32_t>(__popc((selm >> (4 * i)) & 0xFu));
+    if (i < 4) plo |= cnt << (8 * i);
+    else phi |= cnt << (8 * (i - 4));
+  }
+  uint32_t ilo = plo, ihi = phi;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, ilo, o);
+    const uint32_t z = __shfl_up_sync(0xffffffffu, ihi, o);
+    if (lane >= o) {
+      ilo += y;
+      ihi += z;
+    }
+  }
+  const uint32_t tlo = __shfl_sync(0xffffffffu, ilo, 31), thi = __shfl_sync(0xffffffffu, ihi, 31);
+  const uint32_t elo = ilo - plo, ehi = ihi - phi;
+  const uint32_t wtot = (tlo & 0xFFu) + ((tlo >> 8) & 0xFFu) + ((tlo >> 16) & 0xFFu) + (tlo >> 24) + (thi & 0xFFu) +
+                        ((thi >> 8) & 0xFFu) + ((thi >> 16) & 0xFFu) + (thi >> 24);
+  uint32_t chosen;
+  uint32_t run = base + cta_warp_base(wtot, red, &chosen);
+#pragma unroll
+  for (int i = 0; i < V / 4; ++i) {
+    const uint32_t sh = 8 * (i & 3);
+    const uint32_t tot_i = ((i < 4 ? tlo : thi) >> sh) & 0xFFu;
+    const uint32_t ex_i = ((i < 4 ? elo : ehi) >> sh) & 0xFFu;
+    uint32_t nib = (selm >> (4 * i)) & 0xFu;
+    uint32_t o = run + ex_i;
+    while (nib) {
+      const int cc = __ffs(nib) - 1;
+      nib &= nib - 1u;
+      const int p = pos_of(4 * i + cc);
+      if (o < ku) out[o] = idrow ? idrow[p] : p;
+      ++o;
+    }
+    run += tot_i;
+  }
+  return chosen;
+}
+
+template <int V>
+__global__ void __launch_bounds__(kRThreads, 1)
+topk_row_kernel(const float* __restrict__ scores, int64_t n, int64_t row_stride, const int32_t* __restrict__ row_valid,
+                const int32_t* __restrict__ id_map, int64_t id_map_stride, int k, int32_t* __restrict__ idx) {
+  __shared__ RSmem sm;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t t = blockIdx.x;
+  const uint32_t ku = static_cast<uint32_t>(k);
+  const float kNegInf = -__int_as_float(0x7f800000);
+  const float kPosInf = __int_as_float(0x7f800000);
+  for (int i = tid; i < kRBins; i += kRThreads) sm.hist[i] = 0u;
+  sm.extra[tid] = 0u;
+  if (tid == 0) sm.ccount = 0u;
+  pdl_wait_inputs();
+  pdl_allow_next();
+
+  const float* row = scores + t * row_stride;
+  const int32_t* idrow = id_map ? id_map + t * id_map_stride : nullptr;
+  int32_t* out = idx + t * k;
+  int64_t nt64 = n;
+  if (row_valid) {
+    const int64_t rv = row_valid[t];
+    nt64 = rv < 0 ? 0 : (rv < n ? rv : n);
+  }
+  const int nt = static_cast<int>(nt64);
+  const int wbase = warp * 32 * V;
+  auto pos_of = [&](int j) { return wbase + 128 * (j >> 2) + 4 * lane + (j & 3); };
+
+  // ---- the row in registers
+  float v[V];
+#pragma unroll
+  for (int i = 0; i < V / 4; ++i) {
+    const int p = wbase + 128 * i + 4 * lane;
+    if (p + 3 < nt) {
+      const float4 x = __ldg(reinterpret_cast<const float4*>(row + p));
+      v[4 * i] = x.x;
+      v[4 * i + 1] = x.y;
+      v[4 * i + 2] = x.z;
+      v[4 * i + 3] = x.w;
+    } else {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) v[4 * i + c] = p + c < nt ? __ldg(row + p + c) : kNegInf;
+    }
+  }
+  // ---- (1) the sample's range (finite selectable values)
+  const bool sok = v[0] > kNegInf && v[0] < kPosInf;
+  float mn = sok ? v[0] : kPosInf, mx = sok ? v[0] : kNegInf;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  if (lane == 0) {
+    sm.red[1][warp] = __float_as_uint(mn);
+    sm.red[2][warp] = __float_as_uint(mx);
+  }
+  __syncthreads();
+  mn = __uint_as_float(sm.red[1][lane]);
+  mx = __uint_as_float(sm.red[2][lane]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  const float span = mx - mn;
+  const float scale = static_cast<float>(kRBins) / span;
+  // (a finite positive scale keeps the bin arithmetic finite and monotone)
+  const float off = -mn * scale;
+  const bool ranged = mx > mn && span > 0.f && isfinite(span) && isfinite(scale) && isfinite(off);
+  // bin of a selectable value: round(clamp(x * scale + off, 0, 2047)) through
+  // the float adder (2^23 + r holds r in its low mantissa bits); monotone in x
+  auto bin_of = [&](float x) {
+    const float y = fminf(fmaxf(fmaf(x, scale, off), 0.f), static_cast<float>(kRBins - 1)) + 8388608.f;
+    return __float_as_uint(y) & static_cast<uint32_t>(kRBins - 1);
+  };
+
+  uint32_t selm = 0u;     // bit j: entry j is selected
+  bool general = true;    // tau / take / eqtot still to be found and applied
+  bool all_sel = false;   // at most k selectable entries: all of them
+  uint32_t need = ku;
+  uint32_t inb = 0u;      // general path, radix over registers: bit j takes part
+  bool over_list = false; // general path: radix over the list
+  uint32_t c = 0u;
+  if (ranged) {
+    // ---- (2) histogram of the range
+#pragma unroll
+    for (int j = 0; j < V; ++j)
+      if (v[j] > kNegInf) atomicAdd(&sm.hist[bin_of(v[j])], 1u);
+    __syncthreads();
+    const uint32_t nsel = row_find_bin(sm, kRBins, ku, 0);
+    if (nsel <= ku) {
+      all_sel = true;
+    } else {
+      const uint32_t bstar = sm.bc[0];
+      need = ku - sm.bc[1];
+      c = sm.hist[bstar];
+      const bool listed = c <= static_cast<uint32_t>(kRCandCap);
+      // ---- (3) mark the entries above b*, list those in it
+#pragma unroll
+      for (int j = 0; j < V; ++j) {
+        if (!(v[j] > kNegInf)) continue;
+        const uint32_t b = bin_of(v[j]);
+        if (b > bstar) selm |= 1u << j;
+        if (b == bstar) {
+          if (listed) {
+            const uint32_t s = atomicAdd(&sm.ccount, 1u);
+            if (s < static_cast<uint32_t>(kRCandCap)) {
+              sm.cv[s] = v[j];
+              sm.cp[s] = pos_of(j);
+            }
+          } else {
+            inb |= 1u << j;
+          }
+        }
+      }
+      __syncthreads();
+      if (listed && c <= static_cast<uint32_t>(kRRankMax)) {
+        // rank by counting: (value descending, position ascending); the need
+        // best are selected, marked in their owner's mask
+        if (static_cast<uint32_t>(tid) < c) {
+          const float x = sm.cv[tid];
+          const int32_t px = sm.cp[tid];
+          uint32_t rank = 0;
+          for (uint32_t i = 0; i < c; ++i) {
+            const float y = sm.cv[i];
+            rank += (y > x || (y == x && sm.cp[i] < px)) ? 1u : 0u;
+          }
+          if (rank < need) {
+            const int w = px / (32 * V), rem = px - w * 32 * V;
+            const int owner = w * 32 + ((rem >> 2) & 31);
+            atomicOr(&sm.extra[owner], 1u << (4 * (rem >> 7) + (rem & 3)));
+          }
+        }
+        __syncthreads();
+        selm |= sm.extra[tid];
+        general = false;
+      } else {
+        over_list = listed;
+      }
+    }
+  } else {
+    uint32_t nl = 0;
+#pragma unroll
+    for (int j = 0; j < V; ++j)
+      if (v[j] > kNegInf) {
+        inb |= 1u << j;
+        ++nl;
+      }
+    uint32_t nsel;
+    row_warp_base(sm, warp_sum(nl), 0, &nsel);
+    all_sel = nsel <= ku;
+  }
+
+  if (all_sel) {
+#pragma unroll
+    for (int j = 0; j < V; ++j)
+      if (v[j] > kNegInf) selm |= 1u << j;
+  } else if (general) {
+    // ---- general path: tau by radix rounds over the list or the registers
+    if (over_list) {
+      row_radix(sm, need, [&](uint32_t prefix, uint32_t pmask, int sh, int nb) {
+        for (uint32_t i = tid; i < c; i += kRThreads) {
+          const uint32_t kk = float_key(sm.cv[i]);
+          if ((kk & pmask) == prefix) atomicAdd(&sm.hist[(kk >> sh) & static_cast<uint32_t>(nb - 1)], 1u);
+        }
+      });
+    } else {
+      row_radix(sm, need, [&](uint32_t prefix, uint32_t pmask, int sh, int nb) {
+#pragma unroll
+        for (int j = 0; j < V; ++j) {
+          const uint32_t kk = float_key(v[j]);
+          if (((inb >> j) & 1u) && (kk & pmask) == prefix)
+            atomicAdd(&sm.hist[(kk >> sh) & static_cast<uint32_t>(nb - 1)], 1u);
+        }
+      });
+    }
+    const float tau = sm.tau;
+    const uint32_t take = sm.take, eqtot = sm.eqtot;
+    // entries above tau, and of those equal to it the lowest positions
+    uint32_t tk = 0u;
+#pragma unroll
+    for (int j = 0; j < V; ++j)
+      if (v[j] == tau) tk |= 1u << j;
+    if (eqtot > take) tk = cta_keep_first<V>(tk, take, sm.red[0]);   // (CTA-uniform)
+    selm = tk;
+#pragma unroll
+    for (int j = 0; j < V; ++j)
+      if (v[j] > tau) selm |= 1u << j;
+  }
+
+  // ---- (4) slots in position order
+  const uint32_t chosen = cta_write_selected<V>(selm, 0u, pos_of, idrow, out, ku, sm.red[1]);
+  for (uint32_t i = chosen + tid; i < ku; i += kRThreads) out[i] = -1;
+}
+
+// ---------------------------------------------------------------------------
+// Rows of 8193 .. 131072 entries, few rows (topk_rowc_kernel): the algorithm
+// of topk_row_kernel over a cluster of CL CTAs per row (1024 threads, V = 8 or
+// 16 entries each; CTA r holds positions [r 1024V, (r+1) 1024V)), so that each
+// pass over the row's registers is CL times shorter.  Every CTA takes the same
+// sample (1024 evenly spaced positions of the whole row), so all agree on the
+// value range without an exchange.  Two cluster barriers on the common path:
+// after the histograms (each CTA sums the CL histograms through distributed
+// shared memory and finds b* itself) and after the lists of b*'s entries
+// (each CTA gathers the cluster's list, ranks every entry and marks its own;
+// the slots before CTA r follow from every CTA's count above b* and its
+// selected listed entries).  General path: three radix rounds whose
+// histograms are summed the same way, then every CTA's counts above and equal
+// to tau.  No CTA exits while another may still read its shared memory.
+constexpr int kCMaxCL = 8;
+
+struct alignas(16) CSmem {
+  uint32_t hist[2][kRBins];   // own histograms (read by the cluster): [0] range, radix round 1; [1] rounds 0, 2
+  uint32_t ghist[kRBins];     // the cluster's sum
+  float cv[kRRankMax];        // own entries of b* (read by the cluster)
+  int32_t cp[kRRankMax];
+  float uv[kRRankMax];        // the cluster's entries of b*, in CTA order
+  int32_t up[kRRankMax];
+  uint32_t ur[kRRankMax];     // ... and the CTA holding each
+  uint32_t extra[kRThreads];  // per thread: listed entries that are selected (bit j)
+  uint32_t red[3][kRWarps];
+  uint32_t bc[2];
+  uint32_t meta[4];           // own counts (read by the cluster): selectable, above tau, equal to tau, listed
+  uint32_t gsrc[kCMaxCL];     // per CTA: entries above b*
+  uint32_t csrc[kCMaxCL];     // per CTA: listed entries selected
+};
+
+template <int V>
+__global__ void __launch_bounds__(kRThreads, 1)
+topk_rowc_kernel(const float* __restrict__ scores, int64_t n, int64_t row_stride, const int32_t* __restrict__ row_valid,
+                 const int32_t* __restrict__ id_map, int64_t id_map_stride, int k, int32_t* __restrict__ idx) {
+  __shared__ CSmem sm;
+  cg::cluster_group cl = cg::this_cluster();
+  const int CL = static_cast<int>(cl.num_blocks());
+  const int rank = static_cast<int>(cl.block_rank());
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t t = blockIdx.y;
+  const uint32_t ku = static_cast<uint32_t>(k);
+  const float kNegInf = -__int_as_float(0x7f800000);
+  const float kPosInf = __int_as_float(0x7f800000);
+  for (int i = tid; i < kRBins; i += kRThreads) sm.hist[0][i] = 0u;
+  sm.extra[tid] = 0u;
+  if (tid < 4) sm.meta[tid] = 0u;
+  if (tid < kCMaxCL) {
+    sm.gsrc[tid] = 0u;
+    sm.csrc[tid] = 0u;
+  }
+  pdl_wait_inputs();
+  pdl_allow_next();
+
+  const float* row = scores + t * row_stride;
+  const int32_t* idrow = id_map ? id_map + t * id_map_stride : nullptr;
+  int32_t* out = idx + t * k;
+  int64_t nt64 = n;
+  if (row_valid) {
+    const int64_t rv = row_valid[t];
+    nt64 = rv < 0 ? 0 : (rv < n ? rv : n);
+  }
+  const int nt = static_cast<int>(nt64);
+  const int wbase = rank * kRThreads * V + warp * 32 * V;
+  auto pos_of = [&](int j) { return wbase + 128 * (j >> 2) + 4 * lane + (j & 3); };
+
+  float v[V];
+#pragma unroll
+  for (int i = 0; i < V / 4; ++i) {
+    const int p = wbase + 128 * i + 4 * lane;
+    if (p + 3 < nt) {
+      const float4 x = __ldg(reinterpret_cast<const float4*>(row + p));
+      v[4 * i] = x.x;
+      v[4 * i + 1] = x.y;
+      v[4 * i + 2] = x.z;
+      v[4 * i + 3] = x.w;
+    } else {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) v[4 * i + c] = p + c < nt ? __ldg(row + p + c) : kNegInf;
+    }
+  }
+  // ---- (1) the range of a sample of the whole row (the same in every CTA)
+  const float smp = nt > 0 ? __ldg(row + static_cast<int64_t>(tid) * nt / kRThreads) : kNegInf;
+  const bool sok = smp > kNegInf && smp < kPosInf;
+  float mn = sok ? smp : kPosInf, mx = sok ? smp : kNegInf;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  if (lane == 0) {
+    sm.red[1][warp] = __float_as_uint(mn);
+    sm.red[2][warp] = __float_as_uint(mx);
+  }
+  __syncthreads();
+  mn = __uint_as_float(sm.red[1][lane]);
+  mx = __uint_as_float(sm.red[2][lane]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  const float span = mx - mn;
+  const float scale = static_cast<float>(kRBins) / span;
+  const float off = -mn * scale;
+  const bool ranged = mx > mn && span > 0.f && isfinite(span) && isfinite(scale) && isfinite(off);
+  auto bin_of = [&](float x) {
+    const float y = fminf(fmaxf(fmaf(x, scale, off), 0.f), static_cast<float>(kRBins - 1)) + 8388608.f;
+    return __float_as_uint(y) & static_cast<uint32_t>(kRBins - 1);
+  };
+
+  // ---- (2) own histogram (or, with no range, the selectable entries)
+  uint32_t inb = 0u, nl = 0u;
+#pragma unroll
+  for (int j = 0; j < V; ++j) {
+    if (!(v[j] > kNegInf)) continue;
+    ++nl;
+    if (ranged) atomicAdd(&sm.hist[0][bin_of(v[j])], 1u);
+    else inb |= 1u << j;
+  }
+  nl = warp_sum(nl);
+  if (lane == 0 && nl) atomicAdd(&sm.meta[0], nl);
+  cl.sync();   // every CTA's histogram and selectable count are complete
+
+  const uint32_t src_sel = lane < CL ? cl.map_shared_rank(&sm.meta[0], lane)[0] : 0u;
+  const uint32_t nsel = warp_sum(src_sel);
+  uint32_t selm = 0u;       // bit j: entry j is selected
+  uint32_t base = 0u;       // slots before this CTA's entries
+  uint32_t need = ku;
+  bool general = false;
+  if (nsel <= ku) {
+#pragma unroll
+    for (int j = 0; j < V; ++j)
+      if (v[j] > kNegInf) selm |= 1u << j;
+    base = warp_sum(lane < rank ? src_sel : 0u);
+  } else if (ranged) {
+    // the cluster's histogram: this thread's two bins of every CTA
+    uint2 hs[kCMaxCL];
+#pragma unroll
+    for (int r = 0; r < kCMaxCL; ++r)
+      hs[r] = r < CL ? reinterpret_cast<const uint2*>(cl.map_shared_rank(&sm.hist[0][0], r))[tid] : make_uint2(0u, 0u);
+    uint2 g = make_uint2(0u, 0u);
+#pragma unroll
+    for (int r = 0; r < kCMaxCL; ++r) {
+      g.x += hs[r].x;
+      g.y += hs[r].y;
+    }
+    reinterpret_cast<uint2*>(sm.ghist)[tid] = g;
+    __syncthreads();
+    cta_find_bin(sm.ghist, kRBins, ku, sm.red[0], sm.bc);
+    const uint32_t bstar = sm.bc[0];
+    need = ku - sm.bc[1];
+    const uint32_t c = sm.ghist[bstar];
+    // entries above b* held by each CTA
+#pragma unroll
+    for (int r = 0; r < kCMaxCL; ++r) {
+      if (r >= CL) break;
+      uint32_t a = (2u * tid > bstar ? hs[r].x : 0u) + (2u * tid + 1u > bstar ? hs[r].y : 0u);
+      a = warp_sum(a);
+      if (lane == 0 && a) atomicAdd(&sm.gsrc[r], a);
+    }
+    if (c <= static_cast<uint32_t>(kRRankMax)) {
+      // ---- (3) mark own entries above b*, list own entries in it
+#pragma unroll
+      for (int j = 0; j < V; ++j) {
+        if (!(v[j] > kNegInf)) continue;
+        const uint32_t b = bin_of(v[j]);
+        if (b > bstar) selm |= 1u << j;
+        if (b == bstar) {
+          const uint32_t s2 = atomicAdd(&sm.meta[3], 1u);
+          if (s2 < static_cast<uint32_t>(kRRankMax)) {
+            sm.cv[s2] = v[j];
+            sm.cp[s2] = pos_of(j);
+          }
+        }
+      }
+      cl.sync();   // every CTA's list is complete
+      // the cluster's list in CTA order (warp r copies CTA r's)
+      if (warp < CL) {
+        const uint32_t cnt_l = lane < CL ? cl.map_shared_rank(&sm.meta[3], lane)[0] : 0u;
+        uint32_t inc = cnt_l;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+          if (lane >= o) inc += y;
+        }
+        const uint32_t off_r = __shfl_sync(0xffffffffu, inc - cnt_l, warp);
+        const uint32_t cnt_r = __shfl_sync(0xffffffffu, cnt_l, warp);
+        const float* rcv = cl.map_shared_rank(&sm.cv[0], warp);
+        const int32_t* rcp = cl.map_shared_rank(&sm.cp[0], warp);
+        for (uint32_t i = lane; i < cnt_r && off_r + i < static_cast<uint32_t>(kRRankMax); i += 32) {
+          sm.uv[off_r + i] = rcv[i];
+          sm.up[off_r + i] = rcp[i];
+          sm.ur[off_r + i] = static_cast<uint32_t>(warp);
+        }
+      }
+      __syncthreads();
+      // rank by counting over the cluster's list; the need best are selected
+      if (static_cast<uint32_t>(tid) < c) {
+        const float x = sm.uv[tid];
+        const int32_t px = sm.up[tid];
+        uint32_t rk = 0;
+        for (uint32_t i = 0; i < c; ++i) {
+          const float y = sm.uv[i];
+          rk += (y > x || (y == x && sm.up[i] < px)) ? 1u : 0u;
+        }
+        if (rk < need) {
+          const uint32_t owner_cta = sm.ur[tid];
+          atomicAdd(&sm.csrc[owner_cta], 1u);
+          if (owner_cta == static_cast<uint32_t>(rank)) {
+            const int loc = px - rank * kRThreads * V;
+            const int w = loc / (32 * V), rem = loc - w * 32 * V;
+            atomicOr(&sm.extra[w * 32 + ((rem >> 2) & 31)], 1u << (4 * (rem >> 7) + (rem & 3)));
+          }
+        }
+      }
+      __syncthreads();
+      selm |= sm.extra[tid];
+      for (int r = 0; r < rank; ++r) base += sm.gsrc[r] + sm.csrc[r];
+    } else {
+      general = true;
+#pragma unroll
+      for (int j = 0; j < V; ++j)
+        if (v[j] > kNegInf && bin_of(v[j]) == bstar) inb |= 1u << j;
+    }
+  } else {
+    general = true;   // inb: every selectable entry
+  }
+
+  if (general) {
+    // ---- general path: radix rounds over the cluster's marked entries
+    uint32_t prefix = 0u, pmask = 0u, eqtot = 0u;
+#pragma unroll 1
+    for (int round = 0; round < 3; ++round) {
+      const int sh = round == 0 ? 21 : (round == 1 ? 10 : 0);
+      const int nb = round == 2 ? 1024 : 2048;
+      uint32_t* hb = sm.hist[round == 1 ? 0 : 1];
+      __syncthreads();
+      for (int i = tid; i < nb; i += kRThreads) hb[i] = 0u;
+      __syncthreads();
+#pragma unroll
+      for (int j = 0; j < V; ++j) {
+        const uint32_t kk = float_key(v[j]);
+        if (((inb >> j) & 1u) && (kk & pmask) == prefix) atomicAdd(&hb[(kk >> sh) & static_cast<uint32_t>(nb - 1)], 1u);
+      }
+      cl.sync();   // every CTA's round histogram is complete (and the previous one of this buffer read)
+      for (int i = tid; i < nb; i += kRThreads) {
+        uint32_t g = 0u;
+        for (int r = 0; r < CL; ++r) g += cl.map_shared_rank(hb, r)[i];
+        sm.ghist[i] = g;
+      }
+      __syncthreads();
+      cta_find_bin(sm.ghist, nb, need, sm.red[round & 1], sm.bc);
+      const uint32_t d = sm.bc[0];
+      need -= sm.bc[1];
+      prefix |= d << sh;
+      pmask |= static_cast<uint32_t>(nb - 1) << sh;
+      if (round == 2) eqtot = sm.ghist[d];
+    }
+    const float tau = key_to_float(prefix);
+    const uint32_t take = need;
+    (void)eqtot;
+    uint32_t gt_l = 0u, tk = 0u;
+#pragma unroll
+    for (int j = 0; j < V; ++j) {
+      if (v[j] > tau) selm |= 1u << j;
+      if (v[j] == tau) tk |= 1u << j;
+    }
+    gt_l = warp_sum(__popc(selm));
+    const uint32_t eq_l = warp_sum(__popc(tk));
+    if (lane == 0) {
+      if (gt_l) atomicAdd(&sm.meta[1], gt_l);
+      if (eq_l) atomicAdd(&sm.meta[2], eq_l);
+    }
+    cl.sync();   // every CTA's counts above and equal to tau are complete
+    const uint32_t gt_r = lane < CL ? cl.map_shared_rank(&sm.meta[1], lane)[0] : 0u;
+    const uint32_t eq_r = lane < CL ? cl.map_shared_rank(&sm.meta[2], lane)[0] : 0u;
+    uint32_t einc = eq_r;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, einc, o);
+      if (lane >= o) einc += y;
+    }
+    const uint32_t ebefore = einc - eq_r;   // ties held by lower CTAs
+    const uint32_t taken_r = ebefore >= take ? 0u : (take - ebefore < eq_r ? take - ebefore : eq_r);
+    base = warp_sum(lane < rank ? gt_r + taken_r : 0u);
+    const uint32_t my_take = __shfl_sync(0xffffffffu, taken_r, rank);
+    const uint32_t my_eq = __shfl_sync(0xffffffffu, eq_r, rank);
+    if (my_eq > my_take) tk = cta_keep_first<V>(tk, my_take, sm.red[0]);   // (CTA-uniform)
+    selm |= tk;
+  }
+
+  // no shared memory of another CTA is read past this point
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  // ---- (4) slots: this CTA's after the lower CTAs'
+  const uint32_t mine = cta_write_selected<V>(selm, base, pos_of, idrow, out, ku, sm.red[1]);
+  if (rank == CL - 1) {
+    const uint32_t chosen = base + mine;   // the last CTA's slots end the row's
+    for (uint32_t i = chosen + tid; i < ku; i += kRThreads) out[i] = -1;
+  }
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 int pick_cluster(int64_t n) {
   int cl = 1;
   while (cl < kMaxCluster && static_cast<int64_t>(cl) * kSliceCap < n) cl <<= 1;
@@ -1363,20 +1577,29 @@ cudaError_t launch_topk(const float* scores, int T, int64_t n, int64_t row_strid
     return launch_pdl(topk_band_kernel, dim3(T), dim3(kBThreads), smem, stream, 0, scores, n, row_stride, row_valid,
                       id_map, id_map_stride, k, idx);
   }
-  if (n <= static_cast<int64_t>(kXRangeCluster) * kXThreads * 16) {
-    // smallest V with ceil(n / (512 V)) <= kXRangeCluster CTAs per row
-    const int V = n <= static_cast<int64_t>(kXRangeCluster) * kXThreads * 8 ? 8 : 16;
-    const int64_t slice = static_cast<int64_t>(kXThreads) * V;
-    const int CL = static_cast<int>((n + slice - 1) / slice);
-    const size_t smem = sizeof(XSmem);
+  if (n > static_cast<int64_t>(kRThreads) * 8 && n <= static_cast<int64_t>(kRThreads) * 16 * kCMaxCL) {
+    // a cluster per row, the row in registers: 8 entries per thread, or 16
+    // when 8 would need more CTAs than there are SMs (or more than 8 per row)
+    const int64_t cl8 = (n + kRThreads * 8 - 1) / (kRThreads * 8);
+    const bool v8 = cl8 <= kCMaxCL && (sms <= 0 || static_cast<int64_t>(T) * cl8 <= sms);
+    const int V = v8 ? 8 : 16;
+    const int CL = static_cast<int>((n + static_cast<int64_t>(kRThreads) * V - 1) / (static_cast<int64_t>(kRThreads) * V));
     auto go = [&](auto kern) -> cudaError_t {
-      cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
-      if (e != cudaSuccess) return e;
-      return launch_pdl(kern, dim3(CL, T, 1), dim3(kXThreads), smem, stream, CL, scores, n, row_stride, row_valid,
+      return launch_pdl(kern, dim3(CL, T, 1), dim3(kRThreads), 0, stream, CL, scores, n, row_stride, row_valid,
                         id_map, id_map_stride, k, idx);
     };
-    if (V == 8) return go(topk_range_kernel<8>);
-    return go(topk_range_kernel<16>);
+    if (V == 8) return go(topk_rowc_kernel<8>);
+    return go(topk_rowc_kernel<16>);
+  }
+  if (n <= static_cast<int64_t>(kRThreads) * 8) {
+    // one CTA per row, the row in registers: V entries per thread
+    const int V = n <= kRThreads * 4 ? 4 : 8;
+    auto go = [&](auto kern) -> cudaError_t {
+      return launch_pdl(kern, dim3(T), dim3(kRThreads), 0, stream, 0, scores, n, row_stride, row_valid, id_map,
+                        id_map_stride, k, idx);
+    };
+    if (V == 4) return go(topk_row_kernel<4>);
+    return go(topk_row_kernel<8>);
   }
   const int CL = pick_cluster(n);
   int64_t slice = (n + CL - 1) / CL;

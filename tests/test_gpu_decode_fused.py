@@ -1,4 +1,4 @@
-"""misa_index_decode (router + routed scoring + top-k in one kernel) on the GPU.
+"""misa_index_decode (router + routed scoring in one kernel, the top-k behind it) on the GPU.
 
 The fused step must compute what misa_route_heads, misa_index_score and
 misa_topk compute one after the other (MISA page, gist.science, "Methodology:
@@ -7,8 +7,9 @@ bit-exactly against a CPU sort of the kernel's own importances; scores equal,
 bit for bit, those of misa_index_score run with the kernel's heads, and within
 the score tolerance of the oracle on those heads; indices bit-exactly the
 top-k of the kernel's own scores (CPU sort, ties to the lower position) and
-within the tolerance band of the oracle's.  Rows with massive exact ties drive
-the selection's two tie paths (candidate list, and position-ordered row pass).
+within the tolerance band of the oracle's.  Rows with massive exact ties check
+that the top-k, started while the scoring kernel still runs, reads the whole
+rows the scoring kernel wrote.
 """
 import numpy as np
 import pytest
@@ -88,9 +89,8 @@ def test_fused_decode_parity(T, L, H, h, B, k, shared, ragged):
 @pytest.mark.parametrize("distinct", [16, 4, 1])
 def test_fused_decode_massive_ties(distinct):
     """Keys repeat `distinct` rows over the cache, so every score value occurs
-    L / distinct times: the k-th value's bin holds 2048 (candidate list), 8192
-    (row pass) or all 32768 (every score equal) entries; the top-k must still
-    be the lowest positions among the ties."""
+    L / distinct times (2048, 8192, or all 32768 entries equal); the top-k must
+    still be the lowest positions among the ties."""
     T, L, H, h, B, k = 3, 32768, 64, 8, 128, 2048
     wl = make_decode("ft", 77 + distinct, T=T, L=L, H=H, h=h, B=B, k=k, n_planted=0)
     base = wl.keys[:, :distinct].clone()

@@ -37,29 +37,33 @@ def test_block_stats(nseq, L, B):
 
 # ------------------------------------------------------------------ top-k on its own
 @pytest.mark.parametrize("T,n,k,ties,neg_inf,zeros", [
-    (4, 4096, 256, 0.0, 0.0, 0.0),
-    (3, 32768, 2048, 0.0, 0.0, 0.0),
-    (2, 131072, 2048, 0.0, 0.0, 0.0),
+    (4, 4096, 256, 0.0, 0.0, 0.0),        # one CTA per row, 4 entries per thread
+    (3, 32768, 2048, 0.0, 0.0, 0.0),      # cluster of 4 CTAs per row, 8 entries per thread
+    (2, 131072, 2048, 0.0, 0.0, 0.0),     # cluster of 8, 16 entries per thread
     (5, 10001, 300, 0.3, 0.1, 0.1),       # ties, masked, +-0, ragged length
     (3, 50000, 100, 0.9, 0.0, 0.0),       # threshold bin far above candidate capacity
     (2, 70000, 9000, 0.0, 0.0, 0.0),      # k above the fast path's list capacity
     (2, 9000, 16384, 0.0, 0.2, 0.0),      # fewer valid entries than k (padding)
     (3, 7, 3, 0.5, 0.3, 0.3),             # tiny row
     (2, 20000, 1, 0.5, 0.0, 0.5),
-    (2, 300000, 2048, 0.0, 0.0, 0.0),     # slices too long for shared memory (keys re-read from global)
-    (3, 16385, 100, 0.2, 0.1, 0.1),       # 8-CTA cluster, last slice nearly empty
-    (4, 4097, 50, 0.3, 0.0, 0.2),         # 2-CTA cluster
+    (2, 300000, 2048, 0.0, 0.0, 0.0),     # digit-radix cluster kernel (keys re-read from global)
+    (3, 16385, 100, 0.2, 0.1, 0.1),       # cluster of 3, the last CTA holds one entry
+    (4, 4097, 50, 0.3, 0.0, 0.2),         # 8 entries per thread, one valid in the last group
     (65, 1024, 64, 0.1, 0.0, 0.0),        # many short rows
-    (3, 30000, 100, 0.9, 0.0, 0.0),       # threshold bin beyond the gather capacity: cluster radix inside it
-    (2, 12000, 700, 0.35, 0.0, 0.0),      # heavy ties: threshold bin gathered (> 512 entries, radix over them)
-    (2, 5000, 100, 0.0, 0.0, 1.0),        # every entry +-0: one value range, select by position
-    (2, 3000, 10, 0.0, 0.0, 1.0),         # same, one CTA
-    (2, 40960, 2048, 0.0, 0.0, 0.0),
-    (2, 32768, 2048, 0.1, 0.0, 0.0),      # largest row of 8 entries per thread
-    (2, 32769, 2048, 0.0, 0.0, 0.0),      # smallest row of 16 per thread
-    (2, 65536, 2048, 0.0, 0.1, 0.0),      # largest row held in registers
-    (2, 131072, 5000, 0.2, 0.0, 0.0),     # digit-radix cluster kernel, keys in shared memory
-    (2, 65537, 2048, 0.0, 0.0, 0.0),      # smallest row of the digit-radix cluster kernel
+    (3, 30000, 100, 0.9, 0.0, 0.0),       # the k-th entry's value-range bin holds most of the row
+    (2, 12000, 700, 0.35, 0.0, 0.0),      # heavy ties at the threshold
+    (2, 5000, 100, 0.0, 0.0, 1.0),        # every entry +-0: no value range, select by position
+    (2, 3000, 10, 0.0, 0.0, 1.0),         # same, 4 entries per thread
+    (2, 40960, 2048, 0.0, 0.0, 0.0),      # cluster of 5
+    (2, 32768, 2048, 0.1, 0.0, 0.0),      # cluster of 4, ties
+    (2, 32769, 2048, 0.0, 0.0, 0.0),      # cluster of 5, the last CTA holds one entry
+    (2, 65536, 2048, 0.0, 0.1, 0.0),      # cluster of 8, 8 entries per thread
+    (2, 131072, 5000, 0.2, 0.0, 0.0),     # cluster of 8, 16 entries per thread, ties
+    (2, 65537, 2048, 0.0, 0.0, 0.0),      # 16 entries per thread, cluster of 5
+    (3, 40000, 100, 0.0, 0.0, 1.0),       # cluster, every entry +-0: no value range
+    (2, 45000, 700, 0.35, 0.0, 0.0),      # cluster per row, heavy ties at the threshold
+    (2, 60000, 300, 0.3, 0.1, 0.1),       # cluster per row, ties, masked, +-0
+    (2, 200000, 700, 0.35, 0.1, 0.0),     # digit-radix cluster kernel, heavy ties
 ])
 def test_topk_exact(T, n, k, ties, neg_inf, zeros):
     _check_topk(random_scores(1000 + n + k, T, n, tie_frac=ties, neg_inf_frac=neg_inf, zero_frac=zeros), n, k)
@@ -104,6 +108,32 @@ def test_topk_unusual_rows():
     s[3, :] = torch.linspace(-1.0, 1.0, n)
     for k in (1, 50, 2048, 15000):
         _check_topk(s, n, k)
+
+
+def test_topk_register_rows():
+    """Rows for the register-resident kernels' range and tie paths (one CTA
+    per row up to 8192 entries, a cluster above): NaN entries (never
+    selected), values a few ulps apart, a range too wide for fp32, one of
+    denormals, values repeating every 16 positions (every lane of a warp in the
+    same bin), and exactly 100 selectable entries."""
+    rng = np.random.default_rng(11)
+    for n in (1000, 4096, 8193, 32768, 65536):
+        rows = []
+        r = rng.standard_normal(n).astype(np.float32)
+        r[rng.random(n) < 0.1] = np.nan
+        rows.append(r)
+        rows.append((np.float32(1.0) + rng.integers(0, 64, n).astype(np.float32) * np.float32(2.0**-23)))
+        r = rng.standard_normal(n).astype(np.float32)
+        r[0], r[n // 2] = np.float32(-3e38), np.float32(3e38)
+        rows.append(r)
+        rows.append((rng.random(n) * 1e-40).astype(np.float32))
+        rows.append(np.tile(rng.standard_normal(16).astype(np.float32), n // 16 + 1)[:n])
+        r = rng.standard_normal(n).astype(np.float32)
+        r[rng.permutation(n)[: n - 100]] = -np.inf
+        rows.append(r)
+        s = torch.from_numpy(np.stack(rows))
+        for k in (1, 100, min(2048, n)):
+            _check_topk(s, n, k)
 
 
 def _check_topk(s, n, k):
