@@ -57,7 +57,8 @@ def bench_config(wl, ws_n: int) -> dict:
     """The `config` object both arms print (identical keys and values)."""
     return {"workload": WORKLOAD, "queries": wl.T, "L": wl.L, "H": wl.H, "h": wl.h, "B": wl.B, "k": wl.k, "d": 128,
             "parallelism": f"dp{ws_n} (independent batches)",
-            "l2": "flushed before every timed step (256 MiB write, untimed); K is 268 MB > L2"}
+            "l2": "not flushed between steps: the keys (T x L x 256 B = 268 MB) exceed L2 (126 MB); "
+                  "detail.*_l2_flushed_ms repeat the timings with a 256 MiB write before every step"}
 
 
 def decode_step_bytes(T: int, L: int, H: int, h: int, B: int, k: int) -> int:
@@ -69,6 +70,14 @@ def decode_step_bytes(T: int, L: int, H: int, h: int, B: int, k: int) -> int:
     counted)."""
     M = (L + B - 1) // B
     return (T * L * 256 + T * M * 128 * 2 * 2 + T * H * 256 + T * H * 4 + 2 * T * L * 4 + T * k * 4)
+
+
+def fused_kernel_bytes(T: int, L: int, H: int, h: int, B: int) -> int:
+    """Algorithmic HBM bytes of the router + scoring kernel of the decode step:
+    the keys, the bf16 hi/lo block means, all heads' query rows and weights,
+    the fp32 score rows written, the heads and importances written."""
+    M = (L + B - 1) // B
+    return T * L * 256 + T * M * 128 * 2 * 2 + T * H * 256 + T * H * 4 + T * L * 4 + T * h * 4 + T * H * 4
 
 
 def dagger_step_bytes(T: int, L: int, H: int, B: int, kp: int, k: int) -> int:
@@ -271,6 +280,7 @@ def run_cuda(args):
     pairs = int(wl.prefix_len.sum())
 
     means = misa.block_stats(keys, B, split=True)
+    ixf = misa.MisaIndexer(T, H, h, L, B, k, q_block=1, device=dev, fused=True)
     ix = misa.MisaIndexer(T, H, h, L, B, k, q_block=1, device=dev)
     dense = misa.DenseIndexer(T, H, L, k, device=dev)
     flush_buf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
@@ -278,10 +288,13 @@ def run_cuda(args):
     def flush():
         flush_buf.fill_(1.0)
 
-    # warm-up (eager), then the step as one CUDA graph with timing events
-    # recorded inside it between the stages
+    def no_flush():
+        pass
+
+    # warm-up (eager), then every variant as one CUDA graph
     from sparse_attention_token_misa_b200.indexer import capture_graph
     for _ in range(args.warmup):
+        ixf.run(q, w, keys, means, seq_of, plen)
         ix.run(q, w, keys, means, seq_of, plen)
         dense.run(q, w, keys, seq_of, plen)
     torch.cuda.synchronize()
@@ -296,19 +309,24 @@ def run_cuda(args):
         ix.select(plen)
         inner[3].record()
 
-    # the timed step: one graph of route, score, top-k with nothing between
-    # the kernels (so each one's prologue overlaps the previous one's tail);
-    # the per-kernel split comes from a second graph with timing events
-    # recorded between the stages
+    # the timed step: misa_index_decode (router + scoring kernel, the top-k
+    # behind it), one graph; beside it the same without the top-k (the fused
+    # kernel alone, for its roofline) and the three separate calls (route,
+    # score, top-k), whose per-kernel split comes from a graph with timing
+    # events recorded between the stages
+    g_step = capture_graph(lambda: ixf.run(q, w, keys, means, seq_of, plen))
+    g_rs = capture_graph(lambda: ixf.route_score(q, w, keys, means, seq_of, plen))
     ix.capture(q, w, keys, means, seq_of, plen)
     g_split = capture_graph(misa_graph_body)
     dense.capture(q, w, keys, seq_of, plen)
     for _ in range(args.warmup):
+        g_step.replay()
+        g_rs.replay()
         ix.g_step.replay()
         g_split.replay()
     torch.cuda.synchronize()
-    misa.error_reset(ix.ws)
-    misa.error_reset(ix.ws_route)
+    for ws_ in (ixf.ws_decode, ix.ws, ix.ws_route):
+        misa.error_reset(ws_)
 
     parts = {"route": 0.0, "score": 0.0, "topk": 0.0}
 
@@ -322,25 +340,31 @@ def run_cuda(args):
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         t0 = time.perf_counter()
-        tot_ms, _ = _time_steps(lambda evs: ix.g_step.replay(), args.steps, flush, stream)
+        tot_ms, _ = _time_steps(lambda evs: g_step.replay(), args.steps, no_flush, stream)
         wall = time.perf_counter() - t0
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
-    split_ms, _ = _time_steps(lambda evs: g_split.replay(), args.steps, flush, stream, after=after_split)
-    dev_err = misa.error_query(ix.ws) | misa.error_query(ix.ws_route)
+    ms_step = reduce_max(tot_ms / args.steps, dist, dev)
+    rs_ms = _time_steps(lambda evs: g_rs.replay(), args.steps, no_flush, stream)[0] / args.steps
+    flushed_ms = _time_steps(lambda evs: g_step.replay(), args.steps, flush, stream)[0] / args.steps
+    three_ms = _time_steps(lambda evs: ix.g_step.replay(), args.steps, no_flush, stream)[0] / args.steps
+    three_flushed_ms = _time_steps(lambda evs: ix.g_step.replay(), args.steps, flush, stream)[0] / args.steps
+    split_ms, _ = _time_steps(lambda evs: g_split.replay(), args.steps, no_flush, stream, after=after_split)
+    dev_err = misa.error_query(ixf.ws_decode) | misa.error_query(ix.ws) | misa.error_query(ix.ws_route)
     if dev_err:
         raise RuntimeError(f"device error word {dev_err:#x}")
-    ms_step = reduce_max(tot_ms / args.steps, dist, dev)
+    if not torch.equal(ixf.idx, ix.idx) and torch.equal(ixf.heads, ix.heads):
+        raise RuntimeError("fused and three-call indices differ on equal heads")
 
     # the dense 64-head indexer and the block statistics on the same batch
     # (same protocol)
     dense_ms, dparts = _time_steps(lambda evs: (dense.g_score.replay(), evs[0].record(stream),
-                                                dense.g_select.replay()), args.steps, flush, stream,
+                                                dense.g_select.replay()), args.steps, no_flush, stream,
                                    marks=["score", "topk"])
-    dense_one_ms, _ = _time_steps(lambda evs: dense.g_step.replay(), args.steps, flush, stream)
+    dense_one_ms, _ = _time_steps(lambda evs: dense.g_step.replay(), args.steps, no_flush, stream)
     stats_ms, _ = _time_steps(lambda evs: misa.block_stats(keys, B, out=means[0], out_hi=means[1], out_lo=means[2]),
-                              args.steps, flush, stream)
+                              args.steps, no_flush, stream)
     dense_ms /= args.steps
     dense_one_ms /= args.steps
     stats_ms /= args.steps
@@ -365,7 +389,7 @@ def run_cuda(args):
         _view(stage_h, i).copy_(t_)
     q_d, w_d, so_d, pl_d = (_view(stage_d, i) for i in range(4))
     idx_h = torch.empty((T, k), dtype=torch.int32).pin_memory()
-    ix_e = misa.MisaIndexer(T, H, h, L, B, k, q_block=1, device=dev)
+    ix_e = misa.MisaIndexer(T, H, h, L, B, k, q_block=1, device=dev, fused=True)
 
     def e2e_eager():
         stage_d.copy_(stage_h, non_blocking=True)
@@ -376,18 +400,18 @@ def run_cuda(args):
     for _ in range(3):
         g_e2e.replay()
     torch.cuda.synchronize()
-    e2e_ms, _ = _time_steps(lambda evs: g_e2e.replay(), args.steps, flush, stream)
+    e2e_ms, _ = _time_steps(lambda evs: g_e2e.replay(), args.steps, no_flush, stream)
     e2e_ms = reduce_max(e2e_ms / args.steps, dist, dev)
-    e2e_eager_ms, _ = _time_steps(lambda evs: e2e_eager(), args.steps, flush, stream)
+    e2e_eager_ms, _ = _time_steps(lambda evs: e2e_eager(), args.steps, no_flush, stream)
     e2e_eager_ms /= args.steps
-    if not torch.equal(idx_h.cuda(dev), ix.idx):
+    if not torch.equal(idx_h.cuda(dev), ixf.idx):
         raise RuntimeError("e2e indices differ from the device-timed step")
     h2d = stage_h.numel()   # q, w, seq_of, prefix_len, each padded to 256 bytes
     d2h = idx_h.numel() * 4
     # selection agreement with the dense indexer on the same batch (for information)
-    sel_iou, sel_rec = selection_agreement(ix.idx, dense.idx)
+    sel_iou, sel_rec = selection_agreement(ixf.idx, dense.idx)
     selection = {"misa8_iou_vs_dense64": sel_iou, "misa8_recovery_of_dense64": sel_rec,
-                 "misa8_planted_recall": planted_recall(ix.idx, wl.planted),
+                 "misa8_planted_recall": planted_recall(ixf.idx, wl.planted),
                  "dense64_planted_recall": planted_recall(dense.idx, wl.planted)}
 
     if dist:
@@ -398,11 +422,13 @@ def run_cuda(args):
 
     hbm_gbs, tc_tflops, peak_kind = _peaks()
     score_ms = parts["score"] / args.steps
-    # algorithmic bytes of one scoring launch: K once, the routed query rows and
+    # algorithmic bytes of one launch of the router + scoring kernel
+    fk_bytes = fused_kernel_bytes(T, L, H, h, B)
+    achieved = fk_bytes / (rs_ms * 1e-3) / 1e9
+    traffic = _traffic_for("decode_fused_kernel", WORKLOAD)
+    # the three-call path's scoring kernel: K once, the routed query rows and
     # weights, the fp32 score rows written
     score_bytes = T * L * 128 * 2 + T * h * (128 * 2 + 4 + 4) + T * L * 4
-    achieved = score_bytes / (score_ms * 1e-3) / 1e9
-    traffic = _traffic_for("score_kernel", WORKLOAD)
     step_bytes = decode_step_bytes(T, L, H, h, B, k)
     value = pairs * ws_n / (ms_step * 1e-3)
     line = {
@@ -424,27 +450,33 @@ def run_cuda(args):
         # and over all heads for the dense indexer on the same batch
         "scored_head_pairs_per_s": pairs * h * ws_n / (ms_step * 1e-3),
         "dense64_scored_head_pairs_per_s": pairs * H * ws_n / (dense_one_ms * 1e-3),
-        "gpu_launches": 3 * args.steps,  # route, score, top-k kernels per step
-        "timing": "CUDA events on the launching stream around one graph replay per step (route, score, top-k "
-                  "with nothing between them); the per-kernel split from a second graph with timing events "
-                  "recorded between the stages (its total is detail.misa8_split_ms)",
-        "roofline": {"bound": "hbm", "kernel": "score_kernel (misa_index_score)", "achieved": achieved,
-                     "peak": hbm_gbs, "peak_kind": f"{peak_kind} hbm copy GB/s", "unit": "GB/s",
-                     "frac": achieved / hbm_gbs, "traffic": traffic,
-                     "algorithmic_bytes_per_launch": score_bytes, "launch_ms": score_ms},
-        "step_roofline": {"bound": "hbm", "what": "whole step (router + scoring + top-k), one graph replay",
+        "gpu_launches": 2 * args.steps,  # router + scoring kernel, top-k kernel per step
+        "timing": "CUDA events on the launching stream around one graph replay per step of misa_index_decode "
+                  "(router + scoring kernel, the top-k kernel behind it); the fused kernel alone from a graph of "
+                  "the same call without the top-k (detail.fused_kernel_ms); the three separate calls in "
+                  "detail.three_call_* (per-kernel split from a graph with timing events between the stages)",
+        "roofline": {"bound": "hbm", "kernel": "decode_fused_kernel (misa_index_decode without its top-k)",
+                     "achieved": achieved, "peak": hbm_gbs, "peak_kind": f"{peak_kind} hbm copy GB/s (burst)",
+                     "unit": "GB/s", "frac": achieved / hbm_gbs, "traffic": traffic,
+                     "algorithmic_bytes_per_launch": fk_bytes, "launch_ms": rs_ms},
+        "step_roofline": {"bound": "hbm", "what": "whole step (router + scoring kernel, top-k), one graph replay",
                           "algorithmic_bytes_per_step": step_bytes,
                           "achieved": step_bytes / (ms_step * 1e-3) / 1e9, "peak": hbm_gbs, "unit": "GB/s",
                           "frac": step_bytes / (ms_step * 1e-3) / 1e9 / hbm_gbs,
                           "frac_of_8TBps": step_bytes / (ms_step * 1e-3) / 8e12},
         "e2e": {"value": pairs * ws_n / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-                "how": "q/w/seq_of/prefix_len packed in one pinned host buffer -> device in one copy, MisaIndexer "
-                       "step on device views of it, idx -> pinned host; one CUDA graph replay per step",
+                "how": "q/w/seq_of/prefix_len packed in one pinned host buffer -> device in one copy, "
+                       "misa_index_decode on device views of it, idx -> pinned host; one CUDA graph replay per step",
                 "eager_ms_per_step": e2e_eager_ms},
         "selection": selection,
-        "detail": {"route_ms": parts["route"] / args.steps, "score_ms": score_ms, "topk_ms": parts["topk"] / args.steps,
-                   "misa8_ms": ms_step, "misa8_split_ms": split_ms / args.steps,
+        "detail": {"misa8_ms": ms_step, "misa8_l2_flushed_ms": flushed_ms, "fused_kernel_ms": rs_ms,
+                   "topk_tail_ms": ms_step - rs_ms,
+                   "three_call_ms": three_ms, "three_call_l2_flushed_ms": three_flushed_ms,
+                   "three_call_split_ms": split_ms / args.steps,
+                   "three_call_route_ms": parts["route"] / args.steps, "three_call_score_ms": score_ms,
+                   "three_call_topk_ms": parts["topk"] / args.steps,
+                   "three_call_score_GBps": score_bytes / (score_ms * 1e-3) / 1e9,
                    "dense64_ms": dense_one_ms, "dense64_score_ms": dparts["score"] / args.steps,
                    "dense64_topk_ms": dparts["topk"] / args.steps, "dense64_over_misa8": dense_one_ms / ms_step,
                    "block_stats_ms": stats_ms,

@@ -371,7 +371,8 @@ MISA_API misa_status misa_index_score(const uint16_t* q, const float* w, const u
  *   heads [T][h] out (ascending ids), importance [T][H] out (may be NULL),
  *   scores [T] rows of L fp32 out (row stride scores_row_stride; -inf past the
  *     prefix; the top-k reads them back from L2, so they are also an output),
- *   idx [T][k] out (ascending positions, -1 padded).
+ *   idx [T][k] out (ascending positions, -1 padded), or NULL: no top-k, the
+ *     call ends with the scores (k is still checked).
  * The importances are summed in another order than misa_route_heads sums them
  * (a per-block reduction on the tensor-core accumulator), so they can differ
  * in the last bits and a head choice can differ where two importances are that

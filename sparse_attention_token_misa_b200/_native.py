@@ -367,9 +367,11 @@ def index_score(q, w, keys, seq_of, prefix_len, heads=None, h: int | None = None
 
 
 def index_decode(q, w, keys, means_hi, means_lo, seq_of, prefix_len, B: int, h: int, k: int, heads=None,
-                 importance=None, scores=None, idx=None, workspace=None, want_importance: bool = True, stream=None):
-    """misa_index_decode: router + routed scoring + top-k in one launch ->
-    (heads [T, h], importance [T, H] or None, scores [T, >= L], idx [T, k])."""
+                 importance=None, scores=None, idx=None, workspace=None, want_importance: bool = True,
+                 select: bool = True, stream=None):
+    """misa_index_decode: router + routed scoring in one kernel, the top-k
+    behind it -> (heads [T, h], importance [T, H] or None, scores [T, >= L],
+    idx [T, k], or None with select=False: no top-k)."""
     _req(q, torch.bfloat16, "q"); _req(w, torch.float32, "w"); _req(keys, torch.bfloat16, "keys")
     _req(seq_of, torch.int32, "seq_of"); _req(prefix_len, torch.int32, "prefix_len")
     _shape(q, "q", None, None, HEAD_DIM); _shape(keys, "keys", None, None, HEAD_DIM)
@@ -392,7 +394,9 @@ def index_decode(q, w, keys, means_hi, means_lo, seq_of, prefix_len, B: int, h: 
     if scores is None:
         scores = torch.empty((T, (L + 3) // 4 * 4), dtype=torch.float32, device=dev)
     _rows(scores, "scores", T, L)
-    if idx is None:
+    if not select:
+        idx = None
+    elif idx is None:
         idx = torch.empty((T, k), dtype=torch.int32, device=dev)
     need = workspace_bytes(OP_INDEX_DECODE, T, H, L, B, k)
     if workspace is None:

@@ -298,7 +298,7 @@ misa_status misa_index_decode(const uint16_t* q, const float* w, const uint16_t*
                               const int32_t* prefix_len, int T, int H, int64_t L, int B, int h, int k, int32_t* heads,
                               float* importance, float* scores, int64_t scores_row_stride, int32_t* idx,
                               void* workspace, size_t workspace_bytes, misa_stream_t stream) {
-  if (!q || !w || !keys || !means_hi || !means_lo || !seq_of || !prefix_len || !heads || !scores || !idx)
+  if (!q || !w || !keys || !means_hi || !means_lo || !seq_of || !prefix_len || !heads || !scores)
     return MISA_ERR_INVALID_ARG;
   if (T < 1 || H < 1 || L < 1 || B < 1 || h < 1 || h > H || k < 1 || nkeyseq < 1 || nmeanseq < 1)
     return MISA_ERR_INVALID_ARG;
@@ -343,7 +343,7 @@ misa_status misa_index_decode(const uint16_t* q, const float* w, const uint16_t*
   a.err = err_word(workspace);
   const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   misa_status rs = cuda_status(misa::launch_decode_fused(a, cs));
-  if (rs != MISA_OK) return rs;
+  if (rs != MISA_OK || !idx) return rs;   // idx NULL: heads, importance and scores only
   // the top-k starts while the last CTAs of the scoring kernel finish and
   // waits for their rows (programmatic dependent launch)
   return cuda_status(misa::launch_topk(scores, T, L, scores_row_stride, prefix_len, nullptr, 0, k, idx, cs));

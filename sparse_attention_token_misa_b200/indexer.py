@@ -57,9 +57,10 @@ def capture_graph(fn) -> torch.cuda.CUDAGraph:
 class MisaIndexer:
     """Router + routed token scoring + top-k for one batch shape.
 
-    fused=True runs the step as the single kernel of misa_index_decode (decode:
-    one routing decision per query; needs the bf16 split of the block means);
-    route / score / select stay available as the three separate calls."""
+    fused=True runs the step through misa_index_decode (decode: one routing
+    decision per query; needs the bf16 split of the block means): router and
+    scoring in one kernel, the top-k behind it; route / score / select stay
+    available as the three separate calls."""
 
     def __init__(self, T: int, H: int, h: int, L: int, B: int, k: int, q_block: int = 1, device="cuda",
                  stride: int | None = None, fused: bool = False):
@@ -91,6 +92,13 @@ class MisaIndexer:
     def select(self, prefix_len, stream=None):
         nat.topk(self.scores_buf, self.k, n=self.L, row_valid=prefix_len, idx=self.idx, workspace=self.ws,
                  stream=stream)
+
+    def route_score(self, q, w, keys, means, seq_of, prefix_len, stream=None):
+        """The fused step without its top-k (heads, importance, scores)."""
+        _, hi, lo = means
+        nat.index_decode(q, w, keys, hi, lo, seq_of, prefix_len, self.B, self.h, self.k, heads=self.heads,
+                         importance=self.importance, scores=self.scores_buf, workspace=self.ws_decode,
+                         select=False, stream=stream)
 
     def run(self, q, w, keys, means, seq_of, prefix_len, stream=None) -> torch.Tensor:
         if self.fused:

@@ -149,3 +149,21 @@ def test_fused_decode_matches_three_calls_full_size():
     for i, t in enumerate(sample):
         check_selection(heads_g[i], imp_o[i], wl.h, what=f"heads t{t}")
         check_selection(np_i(idx[t]), S_o[i], wl.k, what=f"idx t{t}")
+
+
+def test_fused_decode_scores_only():
+    """idx = NULL: the call ends with heads, importances and scores (the same
+    as the full call's) and writes no indices."""
+    wl = make_decode("fs", 321, T=5, L=7000, H=64, h=8, B=128, k=300, n_planted=3)
+    g = to_gpu(wl)
+    means = misa.block_stats(g["keys"], wl.B, split=True)
+    ws = misa.alloc_workspace(misa.workspace_bytes(misa._native.OP_INDEX_DECODE, wl.T, wl.H, wl.L, wl.B, wl.k))
+    heads, imp, S, idx = misa.index_decode(g["q"], g["w"], g["keys"], means[1], means[2], g["seq_of"],
+                                           g["prefix_len"], wl.B, wl.h, wl.k, workspace=ws)
+    h2, imp2, S2, idx2 = misa.index_decode(g["q"], g["w"], g["keys"], means[1], means[2], g["seq_of"],
+                                           g["prefix_len"], wl.B, wl.h, wl.k, workspace=ws, select=False)
+    torch.cuda.synchronize()
+    assert_no_device_error(ws)
+    assert idx2 is None
+    assert torch.equal(heads, h2) and torch.equal(imp, imp2)
+    assert torch.equal(S[:, :wl.L], S2[:, :wl.L])
