@@ -56,6 +56,7 @@ namespace {
 constexpr int kFTileM = 128;                    // keys (or blocks) per tile
 constexpr int kFTileBytes = kFTileM * kD * 2;   // 32 KB
 constexpr int kFStages = 4;                     // key ring
+constexpr int kFPrefetch = kFStages + 2;        // key tiles asked into L2 this far ahead
 constexpr int kFRSlots = 2;                     // router buffer (hi / lo tiles)
 constexpr int kFHP = 16;                        // routed columns (h <= 16, zero padded)
 constexpr int kFThreads = 352;
@@ -270,6 +271,7 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
         while (*go == 0u && !*abort && globaltimer_ns() - t0 < kWaitLimitNs) {
         }
       }
+      const int64_t krows = (p.nkeyseq - 1) * p.key_seq_rows + p.L;   // rows of the key map
       int64_t it = 0;
       bool ok = true;
       for (int gl = 0; gl < ng && ok; ++gl) {
@@ -289,6 +291,15 @@ decode_fused_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_const
           for (int r0 = 0; r0 < kFTileM; r0 += kTmaBoxRows) {
             tma_load_2d_hint(dst + r0 * 128, &kmap, &full[s], 0, y + r0, kpol);
             tma_load_2d_hint(dst + kFTileBytes / 2 + r0 * 128, &kmap, &full[s], 64, y + r0, kpol);
+          }
+          // the tile two past the ring's reach is asked into L2 now, so that
+          // more of the stream is in flight than the ring holds
+          if (item + kFPrefetch < run_end(gl) && j + kFPrefetch < tpg) {
+            const int yp = y + kFPrefetch * kFTileM;
+            for (int r0 = 0; r0 < kFTileM && yp + r0 < krows; r0 += kTmaBoxRows) {
+              tma_prefetch_l2_2d(&kmap, 0, yp + r0);
+              tma_prefetch_l2_2d(&kmap, 64, yp + r0);
+            }
           }
         }
       }

@@ -149,8 +149,12 @@ class DenseIndexer:
 
 
 class MisaDaggerIndexer:
-    def __init__(self, T: int, H: int, h: int, L: int, B: int, kp: int, k: int, q_block: int = 1, device="cuda"):
-        self.coarse = MisaIndexer(T, H, h, L, B, kp, q_block, device)
+    """fused=True runs the coarse stage through misa_index_decode (decode, one
+    routing decision per query)."""
+
+    def __init__(self, T: int, H: int, h: int, L: int, B: int, kp: int, k: int, q_block: int = 1, device="cuda",
+                 fused: bool = False):
+        self.coarse = MisaIndexer(T, H, h, L, B, kp, q_block, device, fused=fused)
         self.T, self.H, self.L, self.kp, self.k = T, H, L, kp, k
         self.idx = torch.empty((T, k), dtype=torch.int32, device=device)
         self.cand_scores = torch.empty((T, kp), dtype=torch.float32, device=device)

@@ -169,11 +169,13 @@ def _check_hisa(wl, hx, ts, o_sub, B, m):
     assert divergent <= MAX_DIVERGENT_FRAC * len(ts), divergent
 
 
-def test_glm5_dagger_sampled():
+@pytest.mark.parametrize("fused", [False, True])
+def test_glm5_dagger_sampled(fused):
+    """fused: the coarse stage through misa_index_decode."""
     wl = make_workload("glm5_dagger_decode_L65536")
     g = to_gpu(wl)
-    means = misa.block_stats(g["keys"], wl.B)
-    dg = misa.MisaDaggerIndexer(wl.T, wl.H, wl.h, wl.L, wl.B, wl.kp, wl.k)
+    means = misa.block_stats(g["keys"], wl.B, split=True)
+    dg = misa.MisaDaggerIndexer(wl.T, wl.H, wl.h, wl.L, wl.B, wl.kp, wl.k, fused=fused)
     dg.run(g["q"], g["w"], g["keys"], means, g["seq_of"], g["prefix_len"], want_scores=True)
     torch.cuda.synchronize()
     sample = [0, 9, 22, 40, 63]
