@@ -376,9 +376,11 @@ constexpr int kBCandCap = kBWarpCap * kBWarps;  // 6144
 constexpr int kBMaxN = 131072;                  // longest row (bitmaps in shared memory)
 constexpr int kBWords = kBMaxN / 32 + kBWarps * 4;  // + segment rounding
 #ifndef MISA_BAND_UNROLL
-#define MISA_BAND_UNROLL 2
+#define MISA_BAND_UNROLL 4
 #endif
 constexpr int kBUnroll = MISA_BAND_UNROLL;  // steps whose loads are in flight together per warp
+
+constexpr int kBListCap = 256;  // band entries in one value-range bin ranked by counting
 
 struct BSmem {
   uint32_t hist[kBBins];
@@ -392,9 +394,12 @@ struct BSmem {
   uint32_t wa[kBWarps], wc[kBWarps];  // per warp: entries above hi, entries gathered
   uint32_t at[kBWarps], et[kBWarps];  // per warp: bits set in gt / eq
   uint32_t wtmp[kBWarps];
+  uint32_t wend[kBWarps];             // per warp: end of its candidates in the flat order
   float wmin[kBWarps], wmax[kBWarps];
   uint32_t bc[8];
   float fbc[2];
+  float lval[kBListCap];      // band entries in the bin of the k-th entry (range path)
+  uint32_t lcnt;
 };
 
 // Over hist[0, nbins) (nbins a multiple of 512, <= 4096): for each of the two
@@ -441,10 +446,10 @@ __device__ __forceinline__ void band_find(BSmem& sm, const uint32_t* hist, int n
 }
 
 // Exact radix select (12 + 10 + 10 key bits) of the need-th largest key among
-// n_keys keys produced by key_at(i) (0 = not a candidate); returns its key and
+// the keys visit(fn) hands to fn (0 = not a candidate); returns its key and
 // sets *gt to the number of larger keys.  All threads.
-template <class KeyAt>
-__device__ uint32_t band_radix(BSmem& sm, int n_keys, KeyAt key_at, uint32_t need, uint32_t* gt) {
+template <class Visit>
+__device__ uint32_t band_radix_visit(BSmem& sm, Visit visit, uint32_t need, uint32_t* gt) {
   const int tid = threadIdx.x;
   uint32_t prefix = 0, above = 0;
   for (int round = 0; round < 3; ++round) {
@@ -452,12 +457,11 @@ __device__ uint32_t band_radix(BSmem& sm, int n_keys, KeyAt key_at, uint32_t nee
     const int nb = round == 0 ? 4096 : 1024;
     for (int i = tid; i < nb; i += kBThreads) sm.hist[i] = 0;
     __syncthreads();
-    for (int i = tid; i < n_keys; i += kBThreads) {
-      const uint32_t kk = key_at(i);
-      if (kk == 0u) continue;
+    visit([&](uint32_t kk) {
+      if (kk == 0u) return;
       const bool match = round == 0 || (kk >> (round == 1 ? 20 : 10)) == prefix;
       if (match) atomicAdd(&sm.hist[(kk >> sh) & static_cast<uint32_t>(nb - 1)], 1u);
-    }
+    });
     __syncthreads();
     band_find(sm, sm.hist, nb, need, 0xffffffffu, sm.bc);
     const uint32_t b = sm.bc[0] & static_cast<uint32_t>(nb - 1);
@@ -469,6 +473,17 @@ __device__ uint32_t band_radix(BSmem& sm, int n_keys, KeyAt key_at, uint32_t nee
   }
   *gt = above;
   return prefix;
+}
+
+// The same over key_at(i), 0 <= i < n_keys.
+template <class KeyAt>
+__device__ uint32_t band_radix(BSmem& sm, int n_keys, KeyAt key_at, uint32_t need, uint32_t* gt) {
+  return band_radix_visit(
+      sm,
+      [&](auto fn) {
+        for (int i = threadIdx.x; i < n_keys; i += kBThreads) fn(key_at(i));
+      },
+      need, gt);
 }
 
 __global__ void __launch_bounds__(kBThreads, 2)
@@ -629,43 +644,65 @@ topk_band_kernel(const float* __restrict__ scores, int64_t n, int64_t row_stride
   const float hi_v = b_hi >= kBBins ? kPosInf : hv;
   const float lo_v = (r_lo >= static_cast<int64_t>(nsv) || !(lv <= hi_v)) ? kLowest : lv;
 
-  // ---------------- pass 1 (the only read of the row on the common path)
-  uint32_t a_w = 0, c_w = 0;  // (warp-uniform) entries above hi, band entries seen
+  // ---------------- pass 1 (the only read of the row on the common path):
+  // lane l of a warp holds positions 128 st + 4 l .. 4 l + 3 of step st (one
+  // 16-byte load); the 32 positions of bitmap word q of the step are held by
+  // lanes 8 q .. 8 q + 7, four bits each, OR-ed together over those lanes
+  if (lane == 0) sm.wc[warp] = 0u;
+  __syncwarp();
+  uint32_t a_l = 0;  // entries above hi seen by this lane
   float* wcval = sm.cval + warp * kBWarpCap;
   int32_t* wcpos = sm.cpos + warp * kBWarpCap;
   for (int s0 = warp; s0 < nsteps; s0 += kBWarps * kBUnroll) {
-    float xs[kBUnroll][4];
+    float4 xs[kBUnroll];
 #pragma unroll
-    for (int u = 0; u < kBUnroll; ++u) load_step(128 * (s0 + kBWarps * u), xs[u]);
+    for (int u = 0; u < kBUnroll; ++u) {
+      const int p = 128 * (s0 + kBWarps * u) + 4 * lane;
+      if (p + 3 < nt) {
+        xs[u] = __ldg(reinterpret_cast<const float4*>(row + p));
+      } else {
+        xs[u].x = p < nt ? __ldg(row + p) : kNegInf;
+        xs[u].y = p + 1 < nt ? __ldg(row + p + 1) : kNegInf;
+        xs[u].z = p + 2 < nt ? __ldg(row + p + 2) : kNegInf;
+        xs[u].w = kNegInf;
+      }
+    }
 #pragma unroll
     for (int u = 0; u < kBUnroll; ++u) {
       const int st = s0 + kBWarps * u;
       if (st >= nsteps) break;
-      const int base = 128 * st;
+      const float e[4] = {xs[u].x, xs[u].y, xs[u].z, xs[u].w};
+      uint32_t anib = 0u, bnib = 0u;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        const float x = xs[u][c];
-        const bool above = x > hi_v;                  // false for NaN
-        const bool band = !above && x >= lo_v;        // false for NaN and -inf
-        const uint32_t am = __ballot_sync(0xffffffffu, above);
-        const uint32_t bm = __ballot_sync(0xffffffffu, band);
-        if (lane == 0) sm.gt[(base >> 5) + c] = am;
-        a_w += __popc(am);
-        if (band) {
-          const uint32_t sl = c_w + __popc(bm & lt);
-          if (sl < static_cast<uint32_t>(kBWarpCap)) {
-            wcval[sl] = x;
-            wcpos[sl] = base + 32 * c + lane;
+        const bool above = e[c] > hi_v;            // false for NaN
+        const bool band = !above && e[c] >= lo_v;  // false for NaN and -inf
+        anib |= above ? 1u << c : 0u;
+        bnib |= band ? 1u << c : 0u;
+      }
+      uint32_t aw = anib << (4 * (lane & 7));
+      aw |= __shfl_xor_sync(0xffffffffu, aw, 1);
+      aw |= __shfl_xor_sync(0xffffffffu, aw, 2);
+      aw |= __shfl_xor_sync(0xffffffffu, aw, 4);
+      if ((lane & 7) == 0) sm.gt[4 * st + (lane >> 3)] = aw;
+      a_l += static_cast<uint32_t>(__popc(anib));
+      if (bnib) {
+        uint32_t sl = atomicAdd(&sm.wc[warp], static_cast<uint32_t>(__popc(bnib)));
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if ((bnib >> c) & 1u) {
+            if (sl < static_cast<uint32_t>(kBWarpCap)) {
+              wcval[sl] = e[c];
+              wcpos[sl] = 128 * st + 4 * lane + c;
+            }
+            ++sl;
           }
-        }
-        c_w += __popc(bm);
       }
     }
   }
-  if (lane == 0) {
-    sm.wa[warp] = a_w;
-    sm.wc[warp] = c_w;
-  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a_l += __shfl_xor_sync(0xffffffffu, a_l, o);
+  if (lane == 0) sm.wa[warp] = a_l;
   // the equal-to-tau bitmap starts empty
   const int nwords = nsteps * 4;
   for (int i = tid; i < nwords; i += kBThreads) sm.eq[i] = 0u;
@@ -684,22 +721,113 @@ topk_band_kernel(const float* __restrict__ scores, int64_t n, int64_t row_stride
   if (A < ku && ku <= A + C && !full) {
     // the k-th entry is in the band (so at least k entries are selectable):
     // exact tau among the gathered entries, which then join the bitmaps
-    uint32_t gt;
-    const uint32_t kk = band_radix(
-        sm, kBCandCap,
-        [&](int i) {
-          return (i % kBWarpCap) < static_cast<int>(sm.wc[i / kBWarpCap]) ? float_key(sm.cval[i]) : 0u;
-        },
-        ku - A, &gt);
-    tau = key_to_float(kk);
+    // the warps' filled candidate slots as one flat range: region ends in
+    // registers, a flat index mapped to (region, slot) by compares
+    if (tid < kBWarps) {
+      uint32_t e = 0;
+      for (int w2 = 0; w2 <= tid; ++w2) e += sm.wc[w2];
+      sm.wend[tid] = e;
+    }
+    __syncthreads();
+    auto each_cand = [&](auto fn) {
+      for (uint32_t f = tid; f < C; f += kBThreads) {
+        int slot = static_cast<int>(f);
+#pragma unroll
+        for (int w2 = 0; w2 < kBWarps - 1; ++w2) {
+          const uint32_t e = sm.wend[w2];
+          if (f >= e) slot = (w2 + 1) * kBWarpCap + static_cast<int>(f - e);
+        }
+        fn(slot);
+      }
+    };
+    // tau: a histogram of the band entries over their own value range (2048
+    // equal-width bins, monotone in the value), then the entries of the bin
+    // holding the k-th one ranked by counting; radix rounds over the band
+    // entries when the range is degenerate or that bin is crowded (ties)
+    uint32_t gt = 0;
+    bool resolved = false;
+    {
+      float cmn = kPosInf, cmx = kNegInf;
+      each_cand([&](int i) {
+        cmn = fminf(cmn, sm.cval[i]);
+        cmx = fmaxf(cmx, sm.cval[i]);
+      });
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        cmn = fminf(cmn, __shfl_xor_sync(0xffffffffu, cmn, o));
+        cmx = fmaxf(cmx, __shfl_xor_sync(0xffffffffu, cmx, o));
+      }
+      __syncthreads();   // wmin / wmax were read by every thread before
+      if (lane == 0) {
+        sm.wmin[warp] = cmn;
+        sm.wmax[warp] = cmx;
+      }
+      for (int i = tid; i < 2048; i += kBThreads) sm.hist[i] = 0u;
+      if (tid == 0) sm.lcnt = 0u;
+      __syncthreads();
+      cmn = sm.wmin[0];
+      cmx = sm.wmax[0];
+#pragma unroll
+      for (int i = 1; i < kBWarps; ++i) {
+        cmn = fminf(cmn, sm.wmin[i]);
+        cmx = fmaxf(cmx, sm.wmax[i]);
+      }
+      const float span = cmx - cmn;
+      const float cscale = 2048.f / span;
+      const float coff = -cmn * cscale;
+      if (cmx > cmn && span > 0.f && isfinite(span) && isfinite(cscale) && isfinite(coff)) {   // (CTA-uniform)
+        auto cbin = [&](float x) {
+          const float y = fminf(fmaxf(fmaf(x, cscale, coff), 0.f), 2047.f) + 8388608.f;
+          return __float_as_uint(y) & 2047u;
+        };
+        each_cand([&](int i) { atomicAdd(&sm.hist[cbin(sm.cval[i])], 1u); });
+        __syncthreads();
+        band_find(sm, sm.hist, 2048, ku - A, 0xffffffffu, sm.bc);
+        const uint32_t bstar = sm.bc[0] & 2047u;
+        const uint32_t above_b = sm.bc[1];
+        const uint32_t c = sm.hist[bstar];
+        if (c <= static_cast<uint32_t>(kBListCap)) {   // (CTA-uniform)
+          each_cand([&](int i) {
+            const float x = sm.cval[i];
+            if (cbin(x) == bstar) {
+              const uint32_t s2 = atomicAdd(&sm.lcnt, 1u);
+              if (s2 < static_cast<uint32_t>(kBListCap)) sm.lval[s2] = x;
+            }
+          });
+          __syncthreads();
+          const uint32_t need2 = ku - A - above_b;   // 1 <= need2 <= c
+          if (static_cast<uint32_t>(tid) < c) {
+            const float x = sm.lval[tid];
+            uint32_t g2 = 0, eb = 0;
+            for (uint32_t j = 0; j < c; ++j) {
+              const float y = sm.lval[j];
+              g2 += y > x ? 1u : 0u;
+              eb += (y == x && j < static_cast<uint32_t>(tid)) ? 1u : 0u;
+            }
+            if (g2 + eb == need2 - 1u) {
+              sm.fbc[0] = x;
+              sm.bc[4] = g2;
+            }
+          }
+          __syncthreads();
+          tau = sm.fbc[0];
+          gt = above_b + sm.bc[4];
+          resolved = true;
+        }
+      }
+    }
+    if (!resolved) {
+      const uint32_t kk = band_radix_visit(
+          sm, [&](auto fn) { each_cand([&](int i) { fn(float_key(sm.cval[i])); }); }, ku - A, &gt);
+      tau = key_to_float(kk);
+    }
     need_eq = ku - A - gt;
-    for (int i = tid; i < kBCandCap; i += kBThreads) {
-      if ((i % kBWarpCap) >= static_cast<int>(sm.wc[i / kBWarpCap])) continue;
+    each_cand([&](int i) {
       const float x = sm.cval[i];
       const int p = sm.cpos[i];
       if (x > tau) atomicOr(&sm.gt[p >> 5], 1u << (p & 31));
       else if (x == tau) atomicOr(&sm.eq[p >> 5], 1u << (p & 31));
-    }
+    });
   } else {
     // the sample misled, too many ties to gather, or fewer selectable entries
     // than k: count the selectable entries; exact tau by a radix select over
