@@ -359,6 +359,29 @@ MISA_API misa_status misa_index_score(const uint16_t* q, const float* w, const u
                              void* workspace, size_t workspace_bytes, misa_stream_t stream);
 
 /*
+ * misa_index_score_blocks -- the dense indexer (all H heads) over the tokens of
+ * chosen key blocks, read block by block.
+ *   [HISA page, section 三, Stage 2: inside the m chosen blocks the token-level
+ *   indexer scores every token; the candidates are the blocks' tokens.]
+ * blocks: [T][m] int32 block ids of B keys each (B = 64 or 128), -1 = empty
+ * slot (as hisa_block_filter writes them with stride B).  scores[t][i*B + r] =
+ * sum over h of w[t,h] * ReLU(q[t,h] . keys[blocks[t][i]*B + r]) when the
+ * block slot is filled and the token is inside the prefix (< min(prefix_len,
+ * L)), -inf otherwise -- bit for bit what misa_index_score computes on the
+ * candidate list cand[t][i*B + r] = blocks[t][i]*B + r (-1 past the prefix).
+ * Each block's keys are read as whole tiles (no per-row gather).  A block id
+ * at or past ceil(L / B) records MISA_DEVERR_BAD_INDEX and scores -inf.
+ * Limits: as misa_index_score (heads NULL), m*B < 2^31, scores_row_stride >=
+ * m*B.  workspace: >= 256 bytes (error word).
+ */
+MISA_API misa_status misa_index_score_blocks(const uint16_t* q, const float* w, const uint16_t* keys,
+                                             int64_t nkeyseq, int64_t key_seq_stride, const int32_t* seq_of,
+                                             const int32_t* prefix_len, int T, int H, int64_t L,
+                                             const int32_t* blocks, int m, int B, float* scores,
+                                             int64_t scores_row_stride, void* workspace, size_t workspace_bytes,
+                                             misa_stream_t stream);
+
+/*
  * misa_index_decode -- one whole MISA decode step in one call: the router and
  * the routed token scoring in one persistent kernel, the per-query top-k in a
  * second kernel that starts while the first one's last CTAs finish.

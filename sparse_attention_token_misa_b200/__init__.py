@@ -8,7 +8,7 @@ sequences (`indexer`).
 """
 from . import _native
 from ._native import (MisaError, alloc_workspace, append_keys, block_stats, error_query, error_reset,  # noqa: F401
-                      gather_candidates, hier_rerank, hisa_block_filter, index_decode, index_score, lib, num_windows,
+                      gather_candidates, hier_rerank, hisa_block_filter, index_decode, index_score, index_score_blocks, lib, num_windows,
                       route_heads,
                       shard_prefix, sparse_mla, topk, workspace_bytes)
 from .indexer import DenseIndexer, HisaIndexer, MisaDaggerIndexer, MisaIndexer  # noqa: F401
@@ -17,6 +17,6 @@ from .sharded import ShardedMisaIndexer, TorchShardComm, shard_bounds  # noqa: F
 __all__ = [
     "MisaError", "alloc_workspace", "append_keys", "block_stats", "error_query", "error_reset",
     "gather_candidates", "hier_rerank", "shard_prefix", "ShardedMisaIndexer", "TorchShardComm", "shard_bounds",
-    "hisa_block_filter", "index_decode", "index_score", "lib", "num_windows", "route_heads", "sparse_mla", "topk", "workspace_bytes",
+    "hisa_block_filter", "index_decode", "index_score", "index_score_blocks", "lib", "num_windows", "route_heads", "sparse_mla", "topk", "workspace_bytes",
     "DenseIndexer", "HisaIndexer", "MisaDaggerIndexer", "MisaIndexer",
 ]

@@ -69,6 +69,8 @@ SIGNATURES = {
     "misa_index_score": (c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_i64, c_vp, c_int,
                                  c_int, c_vp, c_int, c_vp, c_i64, c_vp, c_size, c_vp]),
     "misa_topk": (c_int, [c_vp, c_int, c_i64, c_i64, c_vp, c_vp, c_i64, c_int, c_vp, c_vp, c_size, c_vp]),
+    "misa_index_score_blocks": (c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_int, c_int, c_i64, c_vp,
+                                        c_int, c_int, c_vp, c_i64, c_vp, c_size, c_vp]),
     "misa_index_decode": (c_int, [c_vp, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_i64, c_i64, c_vp, c_vp, c_int,
                                   c_int, c_i64, c_int, c_int, c_int, c_vp, c_vp, c_vp, c_i64, c_vp, c_vp, c_size,
                                   c_vp]),
@@ -406,6 +408,31 @@ def index_decode(q, w, keys, means_hi, means_lo, seq_of, prefix_len, B: int, h: 
           _p(prefix_len), T, H, L, B, h, k, _p(heads), _p(importance), _p(scores), int(scores.stride(0)), _p(idx),
           _p(workspace), workspace.numel(), _stream(stream))
     return heads, importance, scores, idx
+
+
+def index_score_blocks(q, w, keys, seq_of, prefix_len, blocks, B: int, scores=None, workspace=None,
+                       stream=None) -> torch.Tensor:
+    """misa_index_score_blocks -> scores [T, m * B] fp32 (all heads over the
+    tokens of the chosen blocks, -inf for empty slots and past the prefix)."""
+    _req(q, torch.bfloat16, "q"); _req(w, torch.float32, "w"); _req(keys, torch.bfloat16, "keys")
+    _req(seq_of, torch.int32, "seq_of"); _req(prefix_len, torch.int32, "prefix_len")
+    _req(blocks, torch.int32, "blocks")
+    _shape(q, "q", None, None, HEAD_DIM); _shape(keys, "keys", None, None, HEAD_DIM)
+    T, H, _ = q.shape
+    L = keys.shape[1]
+    _shape(w, "w", T, H); _shape(seq_of, "seq_of", T); _shape(prefix_len, "prefix_len", T)
+    _shape(blocks, "blocks", T, None)
+    m = blocks.shape[1]
+    if scores is not None:
+        _rows(scores, "scores", T, m * B)
+    else:
+        scores = torch.empty((T, m * B), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = alloc_workspace(256, q.device)
+    _call("misa_index_score_blocks", _p(q), _p(w), _p(keys), keys.shape[0], _key_stride(keys), _p(seq_of),
+          _p(prefix_len), T, H, L, _p(blocks), m, B, _p(scores), int(scores.stride(0)), _p(workspace),
+          workspace.numel(), _stream(stream))
+    return scores
 
 
 def topk(scores, k: int, n: int | None = None, row_valid=None, id_map=None, idx=None, workspace=None,

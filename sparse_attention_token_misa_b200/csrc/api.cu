@@ -281,6 +281,48 @@ misa_status misa_index_score(const uint16_t* q, const float* w, const uint16_t* 
   return cuda_status(misa::launch_index_score(mp, a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+misa_status misa_index_score_blocks(const uint16_t* q, const float* w, const uint16_t* keys, int64_t nkeyseq,
+                                    int64_t key_seq_stride, const int32_t* seq_of, const int32_t* prefix_len, int T,
+                                    int H, int64_t L, const int32_t* blocks, int m, int B, float* scores,
+                                    int64_t scores_row_stride, void* workspace, size_t workspace_bytes,
+                                    misa_stream_t stream) {
+  if (!blocks || m < 1 || (B != 64 && B != 128)) return MISA_ERR_INVALID_ARG;
+  const int64_t n = static_cast<int64_t>(m) * B;
+  if (n >= (static_cast<int64_t>(1) << 31)) return MISA_ERR_UNSUPPORTED;
+  // (the block list stands in for a candidate list of m B entries)
+  misa_status st = check_score_args(q, w, keys, nkeyseq, key_seq_stride, seq_of, prefix_len, T, H, L, nullptr, H, 1,
+                                    blocks, static_cast<int>(n), scores, scores_row_stride);
+  if (st != MISA_OK) return st;
+  st = check_ws(workspace, workspace_bytes, kErrBytes);
+  if (st != MISA_OK) return st;
+  CUtensorMap map;
+  const int64_t rows = (nkeyseq - 1) * (key_seq_stride / MISA_HEAD_DIM) + L;
+  st = make_key_map(keys, rows, &map);
+  if (st != MISA_OK) return st;
+  misa::ScoreArgs a;
+  a.q = q;
+  a.w = w;
+  a.keys = keys;
+  a.nkeyseq = nkeyseq;
+  a.key_seq_stride = key_seq_stride;
+  a.seq_of = seq_of;
+  a.prefix_len = prefix_len;
+  a.T = T;
+  a.H = H;
+  a.L = L;
+  a.heads = nullptr;
+  a.h = H;
+  a.q_block = 1;
+  a.cand = nullptr;
+  a.n_cand = static_cast<int>(n);
+  a.blocks = blocks;
+  a.run = B;
+  a.scores = scores;
+  a.row_stride = scores_row_stride;
+  a.err = err_word(workspace);
+  return cuda_status(misa::launch_index_score(&map, a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 misa_status misa_topk(const float* scores, int T, int64_t n, int64_t row_stride, const int32_t* row_valid,
                       const int32_t* id_map, int64_t id_map_stride, int k, int32_t* idx, void* workspace,
                       size_t workspace_bytes, misa_stream_t stream) {

@@ -137,6 +137,8 @@ struct ScoreArgs {
   int q_block;
   const int32_t* cand;
   int n_cand;
+  const int32_t* blocks = nullptr;   // block mode (cand NULL): [T][n_cand / run] key blocks
+  int run = 0;
   float* scores;
   int64_t row_stride;
   uint32_t* err;

@@ -76,6 +76,9 @@ struct ScoreParams {
   int q_block;
   const int32_t* cand;      // NULL: contiguous keys
   int n_cand;
+  const int32_t* blocks;    // block mode: [T][n_cand / run] chosen key blocks (-1 = empty), or NULL
+  int run;                  // block mode: keys per block (64 or 128)
+  int64_t n_blocks_seq;     // block mode: blocks per sequence (ids at or above are invalid)
   float* scores;
   int64_t row_stride;
   int n_groups;
@@ -252,12 +255,40 @@ score_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreParams p) {
             const uint32_t ph = static_cast<uint32_t>((it / S) & 1);
             if (!mbar_wait(&empty[s], ph ^ 1u, p.err, abort)) break;
             uint8_t* dst = sA + s * kATileBytes;
-            mbar_arrive_expect_tx(&full[s], kATileBytes);
-            const int y = static_cast<int>(seq_row0 + static_cast<int64_t>(j) * kTileM);
+            if (p.blocks == nullptr) {
+              mbar_arrive_expect_tx(&full[s], kATileBytes);
+              const int y = static_cast<int>(seq_row0 + static_cast<int64_t>(j) * kTileM);
 #pragma unroll
-            for (int r0 = 0; r0 < kTileM; r0 += kTmaBoxRows) {
-              tma_load_2d_hint(dst + r0 * 128, &tmap, &full[s], 0, y + r0, policy);
-              tma_load_2d_hint(dst + kATileBytes / 2 + r0 * 128, &tmap, &full[s], 64, y + r0, policy);
+              for (int r0 = 0; r0 < kTileM; r0 += kTmaBoxRows) {
+                tma_load_2d_hint(dst + r0 * 128, &tmap, &full[s], 0, y + r0, policy);
+                tma_load_2d_hint(dst + kATileBytes / 2 + r0 * 128, &tmap, &full[s], 64, y + r0, policy);
+              }
+            } else {
+              // block mode: the 64-row box at candidate slot c holds keys
+              // blocks[c / run] * run + c % run ...; a box of an empty block slot
+              // (or past the list) is not loaded (its rows are masked)
+              int yb[kTileM / kTmaBoxRows];
+              uint32_t bytes = 0;
+#pragma unroll
+              for (int b2 = 0; b2 < kTileM / kTmaBoxRows; ++b2) {
+                const int slot = j * kTileM + b2 * kTmaBoxRows;
+                int64_t blk = -1;
+                if (slot < p.n_cand) blk = p.blocks[static_cast<int64_t>(g) * (p.n_cand / p.run) + slot / p.run];
+                if (blk >= p.n_blocks_seq) {
+                  record_error(p.err, MISA_DEVERR_BAD_INDEX);
+                  blk = -1;
+                }
+                yb[b2] = blk >= 0 ? static_cast<int>(seq_row0 + blk * p.run + slot % p.run) : -1;
+                if (yb[b2] >= 0) bytes += kATileBytes / (kTileM / kTmaBoxRows);
+              }
+              mbar_arrive_expect_tx(&full[s], bytes);
+#pragma unroll
+              for (int b2 = 0; b2 < kTileM / kTmaBoxRows; ++b2) {
+                if (yb[b2] < 0) continue;
+                const int r0 = b2 * kTmaBoxRows;
+                tma_load_2d_hint(dst + r0 * 128, &tmap, &full[s], 0, yb[b2], policy);
+                tma_load_2d_hint(dst + kATileBytes / 2 + r0 * 128, &tmap, &full[s], 64, yb[b2], policy);
+              }
             }
             ++it;
           }
@@ -453,6 +484,10 @@ score_kernel(const __grid_constant__ CUtensorMap tmap, const ScoreParams p) {
       if (kGather) {
         in_row = pos < p.n_cand;
         key_id = in_row ? p.cand[static_cast<int64_t>(g) * p.n_cand + pos] : -1;
+      } else if (p.blocks != nullptr) {
+        in_row = pos < p.n_cand;
+        const int64_t blk = in_row ? p.blocks[static_cast<int64_t>(g) * (p.n_cand / p.run) + pos / p.run] : -1;
+        key_id = (blk >= 0 && blk < p.n_blocks_seq) ? static_cast<int>(blk * p.run + pos % p.run) : -1;
       } else {
         in_row = pos < p.L;
         key_id = pos;
@@ -529,7 +564,7 @@ cudaError_t launch_index_score(const CUtensorMap* tmap, const ScoreArgs& a, cuda
 
   const int h_eff = a.heads ? a.h : a.H;
   const bool gather = a.cand != nullptr;
-  const bool shared_groups = !gather && a.key_seq_stride == 0;
+  const bool shared_groups = !gather && a.blocks == nullptr && a.key_seq_stride == 0;
   const int hp = score_mode_hp(h_eff, shared_groups);
   const int qpg = shared_groups ? 256 / hp : 1;
 
@@ -549,10 +584,13 @@ cudaError_t launch_index_score(const CUtensorMap* tmap, const ScoreArgs& a, cuda
   p.q_block = a.q_block;
   p.cand = a.cand;
   p.n_cand = a.n_cand;
+  p.blocks = a.blocks;
+  p.run = a.run;
+  p.n_blocks_seq = a.run > 0 ? (a.L + a.run - 1) / a.run : 0;
   p.scores = a.scores;
   p.row_stride = a.row_stride;
   p.err = a.err;
-  if (gather) {
+  if (gather || a.blocks) {
     p.n_groups = a.T;
     p.tiles_per_group = (a.n_cand + kTileM - 1) / kTileM;
   } else {

@@ -180,6 +180,7 @@ class HisaIndexer:
     def __init__(self, T: int, H: int, L: int, B: int, m: int, k: int, device="cuda", stride: int | None = None):
         self.T, self.H, self.L, self.B, self.m, self.k = T, H, L, B, m, k
         self.stride = B if stride is None else stride
+        self.by_blocks = self.stride == B and B in (64, 128)
         self.blocks = torch.empty((T, m), dtype=torch.int32, device=device)
         self.cand = torch.empty((T, m * B), dtype=torch.int32, device=device)
         self.scores_buf = torch.empty((T, _pad4(m * B)), dtype=torch.float32, device=device)
@@ -193,8 +194,13 @@ class HisaIndexer:
         nat.hisa_block_filter(q, w, seq_of=seq_of, prefix_len=prefix_len, L=self.L, B=self.B, m=self.m,
                               blocks=self.blocks, cand=self.cand, workspace=self.ws_filter, stream=stream,
                               stride=self.stride, **_means_args(means))
-        nat.index_score(q, w, keys, seq_of, prefix_len, cand=self.cand, scores=self.scores_buf, workspace=self.ws,
-                        stream=stream)
+        if self.by_blocks:
+            # plain blocks of 64 or 128 keys: score them block by block
+            nat.index_score_blocks(q, w, keys, seq_of, prefix_len, self.blocks, self.B, scores=self.scores_buf,
+                                   workspace=self.ws, stream=stream)
+        else:
+            nat.index_score(q, w, keys, seq_of, prefix_len, cand=self.cand, scores=self.scores_buf,
+                            workspace=self.ws, stream=stream)
         nat.topk(self.scores_buf, self.k, n=self.m * self.B, id_map=self.cand, idx=self.idx, workspace=self.ws,
                  stream=stream)
         return self.idx

@@ -34,7 +34,7 @@ def declared_functions():
 def test_library_loads_and_exports_every_declared_symbol():
     l = pkg.lib()
     names = declared_functions()
-    assert len(names) == 23, names
+    assert len(names) == 24, names
     for n in names:
         assert hasattr(l, n), n
         assert n in nat.SIGNATURES, n
@@ -296,3 +296,22 @@ def test_window_entry_points_reject_and_count():
     assert hf(P, P, P, N, N, 1, 0, P, P, 2, 64, 1000, 128, 256, 4, P2, P2, N, P2, 1 << 20, N) == INVALID
     need = nat.workspace_bytes(nat.OP_HISA_BLOCK_FILTER, 2, 64, 1000, 128, 4)
     assert hf(P, P, P, N, N, 1, 0, P, P, 2, 64, 1000, 128, 32, 4, P2, P2, N, P2, need, N) == WORKSPACE
+
+
+def test_index_score_blocks_rejects():
+    f = pkg.lib().misa_index_score_blocks
+    N = None
+    good = dict(q=P, w=P, keys=P, nseq=1, stride=0, seq_of=P, pl=P, T=2, H=64, L=1000, blocks=P2, m=4, B=128,
+                scores=P2, row_stride=512, ws=P2, ws_bytes=256)
+
+    def call(**kw):
+        a = dict(good, **kw)
+        return f(a["q"], a["w"], a["keys"], a["nseq"], a["stride"], a["seq_of"], a["pl"], a["T"], a["H"], a["L"],
+                 a["blocks"], a["m"], a["B"], a["scores"], a["row_stride"], a["ws"], a["ws_bytes"], N)
+
+    assert call(B=100) == INVALID            # blocks of 64 or 128 keys only
+    assert call(m=0) == INVALID
+    assert call(blocks=None) == INVALID
+    assert call(row_stride=511) == INVALID   # shorter than m * B
+    assert call(q=MIS) == INVALID
+    assert call(ws_bytes=64) == WORKSPACE
