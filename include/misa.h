@@ -17,7 +17,11 @@
  *     section 三, Stage 1 and Stage 2.]
  *   - the dense DSA indexer (all H heads score every token) is the same calls
  *     with heads == NULL.  [MISA page, "Problem statement".]
- * Around the indexer: block statistics kept current as keys are appended
+ * The decode step in one call: misa_index_decode (router and routed scoring in
+ * one kernel, the top-k behind it).  HISA's token stage straight from the
+ * chosen blocks: misa_index_score_blocks.
+ * Around the indexer: block statistics (mean or max pooling, plain blocks or
+ * overlapping windows: the *_ex calls) kept current as keys are appended
  * (misa_append_keys); the sparse attention that consumes the k indices
  * (misa_sparse_mla) [HISA page, sections 二 and 四]; and two small steps of
  * the key-sharded (context-parallel) indexer (misa_shard_prefix,

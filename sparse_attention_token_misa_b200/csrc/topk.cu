@@ -40,7 +40,6 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kBins1 = 4096;  // first digit: top 12 bits
 constexpr int kBins2 = 1024;  // second and third digits: 10 bits each
 constexpr int kMaxCluster = 8;
-constexpr int kSliceCap = 16384;  // keys kept in shared memory per CTA
 
 struct Smem {
   uint32_t hist[kBins1];   // local histogram, then the pulled cluster histogram
@@ -51,7 +50,7 @@ struct Smem {
   uint64_t warp_tot64[kWarps];
   uint64_t block_tot64;
 };
-constexpr size_t kKeysOff = (sizeof(Smem) + 15) / 16 * 16;
+constexpr size_t kClusterSmemBytes = (sizeof(Smem) + 15) / 16 * 16;   // topk_cluster_kernel's shared memory
 
 __device__ __forceinline__ bool selectable(float v) { return v == v && v > -__int_as_float(0x7f800000); }
 
@@ -164,14 +163,12 @@ __device__ __forceinline__ void cluster_hist_sum(cg::cluster_group& cl, Smem& sm
   __syncthreads();
 }
 
-template <bool kKeysInSmem>
 __global__ void __launch_bounds__(kThreads, 2)
 topk_cluster_kernel(const float* __restrict__ scores, int64_t n, int64_t row_stride, const int32_t* __restrict__ row_valid,
                     const int32_t* __restrict__ id_map, int64_t id_map_stride, int k, int32_t* __restrict__ idx,
                     int64_t slice_len) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
-  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + kKeysOff);
 
   pdl_wait_inputs();
   pdl_allow_next();
@@ -193,10 +190,9 @@ topk_cluster_kernel(const float* __restrict__ scores, int64_t n, int64_t row_str
   const int64_t s1 = s0 + slice_len < nt ? s0 + slice_len : nt;
   const int len = static_cast<int>(s1 - s0);
 
-  auto key_at = [&](int i) -> uint32_t {
-    if constexpr (kKeysInSmem) return keys[i];
-    else return sel_key(__ldg(row + s0 + i));
-  };
+  // (the slices of rows this long do not fit in shared memory: every pass
+  // reads its keys from global memory, where L2 keeps them)
+  auto key_at = [&](int i) -> uint32_t { return sel_key(__ldg(row + s0 + i)); };
 
   // ---------------- digit 1 (top 12 bits) while loading the slice
   for (int i = tid; i < kBins1; i += kThreads) sm.hist[i] = 0;
@@ -218,7 +214,6 @@ topk_cluster_kernel(const float* __restrict__ scores, int64_t n, int64_t row_str
         const int i = i0 + u * kThreads;
         if (i < nv) {
           const uint32_t kk[4] = {sel_key(f[u].x), sel_key(f[u].y), sel_key(f[u].z), sel_key(f[u].w)};
-          if constexpr (kKeysInSmem) *reinterpret_cast<uint4*>(&keys[4 * i]) = make_uint4(kk[0], kk[1], kk[2], kk[3]);
 #pragma unroll
           for (int e = 0; e < 4; ++e)
             if (kk[e]) atomicAdd(&sm.hist[kk[e] >> 20], 1u);
@@ -227,7 +222,6 @@ topk_cluster_kernel(const float* __restrict__ scores, int64_t n, int64_t row_str
     }
     for (int i = 4 * nv + tid; i < len; i += kThreads) {
       const uint32_t kk = sel_key(__ldg(row + s0 + i));
-      if constexpr (kKeysInSmem) keys[i] = kk;
       if (kk) atomicAdd(&sm.hist[kk >> 20], 1u);
     }
   }
@@ -497,7 +491,6 @@ topk_band_kernel(const float* __restrict__ scores, int64_t n, int64_t row_stride
   const float kPosInf = __int_as_float(0x7f800000);
   const float kLowest = -__int_as_float(0x7f7fffff);  // -FLT_MAX: v >= it iff v is selectable
   const uint32_t ku = static_cast<uint32_t>(k);
-  const uint32_t lt = (1u << lane) - 1u;
 
   pdl_wait_inputs();
   pdl_allow_next();
@@ -1682,15 +1675,9 @@ topk_rowc_kernel(const float* __restrict__ scores, int64_t n, int64_t row_stride
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-int pick_cluster(int64_t n) {
-  int cl = 1;
-  while (cl < kMaxCluster && static_cast<int64_t>(cl) * kSliceCap < n) cl <<= 1;
-  return cl;
-}
-
 }  // namespace
 
-size_t topk_smem_bytes() { return kKeysOff + static_cast<size_t>(kSliceCap) * 4; }
+size_t topk_smem_bytes() { return kClusterSmemBytes; }
 
 cudaError_t launch_topk(const float* scores, int T, int64_t n, int64_t row_stride, const int32_t* row_valid,
                         const int32_t* id_map, int64_t id_map_stride, int k, int32_t* idx, cudaStream_t stream) {
@@ -1729,21 +1716,15 @@ cudaError_t launch_topk(const float* scores, int T, int64_t n, int64_t row_strid
     if (V == 4) return go(topk_row_kernel<4>);
     return go(topk_row_kernel<8>);
   }
-  const int CL = pick_cluster(n);
+  // longer rows: a cluster of 8, slices starting on 16-byte boundaries
+  const int CL = kMaxCluster;
   int64_t slice = (n + CL - 1) / CL;
-  slice = (slice + 3) / 4 * 4;  // slices start on 16-byte boundaries
-  const bool in_smem = slice <= kSliceCap;
-  const size_t smem = in_smem ? kKeysOff + static_cast<size_t>(slice) * 4 : kKeysOff;
-  const void* fn = in_smem ? reinterpret_cast<const void*>(topk_cluster_kernel<true>)
-                           : reinterpret_cast<const void*>(topk_cluster_kernel<false>);
-  cudaError_t e = ensure_dynamic_smem(fn, static_cast<int>(topk_smem_bytes()));
+  slice = (slice + 3) / 4 * 4;
+  const size_t smem = topk_smem_bytes();
+  cudaError_t e = ensure_dynamic_smem(reinterpret_cast<const void*>(topk_cluster_kernel), static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-
-  if (in_smem)
-    return launch_pdl(topk_cluster_kernel<true>, dim3(CL, T, 1), dim3(kThreads), smem, stream, CL, scores, n,
-                      row_stride, row_valid, id_map, id_map_stride, k, idx, slice);
-  return launch_pdl(topk_cluster_kernel<false>, dim3(CL, T, 1), dim3(kThreads), smem, stream, CL, scores, n,
-                    row_stride, row_valid, id_map, id_map_stride, k, idx, slice);
+  return launch_pdl(topk_cluster_kernel, dim3(CL, T, 1), dim3(kThreads), smem, stream, CL, scores, n, row_stride,
+                    row_valid, id_map, id_map_stride, k, idx, slice);
 }
 
 }  // namespace misa
