@@ -194,8 +194,10 @@ class HisaIndexer:
         nat.hisa_block_filter(q, w, seq_of=seq_of, prefix_len=prefix_len, L=self.L, B=self.B, m=self.m,
                               blocks=self.blocks, cand=self.cand, workspace=self.ws_filter, stream=stream,
                               stride=self.stride, **_means_args(means))
-        if self.by_blocks:
-            # plain blocks of 64 or 128 keys: score them block by block
+        if self.by_blocks and keys.shape[0] > 1:
+            # plain blocks of 64 or 128 keys in per-query caches: score them
+            # block by block (a cache shared by every query, as in a causal
+            # prefill, is read faster by the candidate gather)
             nat.index_score_blocks(q, w, keys, seq_of, prefix_len, self.blocks, self.B, scores=self.scores_buf,
                                    workspace=self.ws, stream=stream)
         else:
