@@ -56,6 +56,7 @@ def test_workspace_formula():
     assert ws(nat.OP_INDEX_SCORE, 5, 5, 5, 5) == 256
     assert ws(nat.OP_TOPK, 5, 5, 5, 5) == 256
     assert ws(nat.OP_APPEND_KEYS, 5, 5, 5, 5) == 256
+    assert ws(nat.OP_INDEX_DECODE, 32, 64, 32768, 128, 2048) == 256   # the error word only
     assert ws(nat.OP_HIER_RERANK, 64, 32, 65536, 128, 2048, 8192) == 256 + 64 * 8192 * 4
     assert ws(nat.OP_HIER_RERANK, 2, 32, 100, 1, 3, 5) == 256 + 2 * 8 * 4
     assert ws(nat.OP_HISA_BLOCK_FILTER, 16, 64, 131072, 128, 64) == 256 + 16 * 1024 * 4
@@ -315,3 +316,32 @@ def test_index_score_blocks_rejects():
     assert call(row_stride=511) == INVALID   # shorter than m * B
     assert call(q=MIS) == INVALID
     assert call(ws_bytes=64) == WORKSPACE
+
+
+def test_index_decode_rejects():
+    """misa_index_decode: shapes outside the fused kernel's limits are
+    unsupported (the separate calls cover them); bad pointers, strides and a
+    short workspace are rejected before any launch."""
+    f = pkg.lib().misa_index_decode
+    N = None
+    good = dict(q=P, w=P, keys=P, nkeyseq=2, kstride=4096 * 128, hi=P2, lo=P2, nmeanseq=2, mstride=32 * 128,
+                seq_of=P, pl=P, T=2, H=64, L=4096, B=128, h=8, k=256, heads=P2, imp=N, scores=P2, sstride=4096,
+                idx=P2, ws=P2, ws_bytes=256)
+
+    def call(**kw):
+        a = dict(good, **kw)
+        return f(a["q"], a["w"], a["keys"], a["nkeyseq"], a["kstride"], a["hi"], a["lo"], a["nmeanseq"],
+                 a["mstride"], a["seq_of"], a["pl"], a["T"], a["H"], a["L"], a["B"], a["h"], a["k"], a["heads"],
+                 a["imp"], a["scores"], a["sstride"], a["idx"], a["ws"], a["ws_bytes"], N)
+
+    assert call(H=65) == UNSUPPORTED         # more than 64 router columns
+    assert call(h=17) == UNSUPPORTED         # more than 16 routed heads
+    assert call(L=65537, kstride=65537 * 128, sstride=65540) == UNSUPPORTED
+    assert call(k=16385) == UNSUPPORTED
+    assert call(h=0) == INVALID
+    assert call(heads=None) == INVALID
+    assert call(hi=None) == INVALID
+    assert call(q=MIS) == INVALID
+    assert call(sstride=4095) == INVALID     # shorter than L
+    assert call(kstride=4095 * 128) == INVALID
+    assert call(ws_bytes=255) == WORKSPACE
